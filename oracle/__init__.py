@@ -1,0 +1,278 @@
+"""Plain fp64 CPU oracle for the HadaNorm Hadamard-domain quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference legs of ``bench.py`` may import this module.  The
+product library (``hadamard_rotated_bit_token_b200``) never imports, links or
+runs anything here, and nothing here imports the product library.
+
+The arithmetic lives in ``hq_oracle.cpp`` (plain C++, fp64, dense block
+Hadamard products and triple loops); this file only builds that library with
+g++ and marshals numpy arrays through ctypes.
+
+Parity pins: see ``tests/test_oracle_pins.py`` (Hadamard orthogonality and the
+Sylvester recursion, the Eq. (1) identity with quantization off, hand-worked
+quantizer examples, brute force at K = 4 / 8, closed-form invariants, integer
+accumulation).  Every function here is pinned there; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hq_oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i8p = ctypes.POINTER(ctypes.c_int8)
+
+
+def build(force: bool = False) -> str:
+    """Compiles hq_oracle.cpp into liboracle.so next to it (g++, -O2)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < max(os.path.getmtime(_SRC),
+                                           os.path.getmtime(os.path.join(_HERE, "hq_oracle.h"))))
+    if force or stale:
+        tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-Wall",
+                               "-o", tmp, _SRC, "-lpthread"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            lib.hqo_hadamard_entry.argtypes = [ctypes.c_int64, ctypes.c_int64]
+            lib.hqo_hadamard_entry.restype = ctypes.c_int
+            lib.hqo_sylvester.argtypes = [ctypes.c_int64, _i8p]
+            lib.hqo_bf16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.hqo_bf16_to_f64.restype = ctypes.c_double
+            lib.hqo_f64_to_bf16.argtypes = [ctypes.c_double]
+            lib.hqo_f64_to_bf16.restype = ctypes.c_uint16
+            lib.hqo_rne.argtypes = [ctypes.c_double]
+            lib.hqo_rne.restype = ctypes.c_double
+            lib.hqo_col_absmax.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, _f64p]
+            lib.hqo_sigma.argtypes = [ctypes.c_int64, _f64p, _f64p, ctypes.c_double, _f64p]
+            lib.hqo_quantize_act.argtypes = [
+                ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                _u16p, ctypes.c_int64, _f64p, ctypes.c_double, _i64p, ctypes.c_int64,
+                _i8p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+            lib.hqo_prepare_weights.argtypes = [
+                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                _u16p, _u16p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+            lib.hqo_gemm_acc.argtypes = [_i8p, _i8p, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int64, _i64p, ctypes.c_int64, _i64p,
+                                         ctypes.c_int]
+            lib.hqo_epilogue.argtypes = [_i64p, ctypes.c_int64, ctypes.c_int64, _f64p, _f64p,
+                                         _f64p, _f64p, _f64p, _f64p, _u16p]
+            lib.hqo_exact_linear.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int64,
+                                             ctypes.c_int64, ctypes.c_int64, _i64p,
+                                             ctypes.c_int64, _f64p, ctypes.c_int]
+            for name in ("hqo_sylvester", "hqo_col_absmax", "hqo_sigma", "hqo_quantize_act",
+                         "hqo_prepare_weights", "hqo_gemm_acc", "hqo_epilogue",
+                         "hqo_exact_linear"):
+                getattr(lib, name).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a, ctype):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments")
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+# ---------------------------------------------------------------------------
+# scalar helpers
+# ---------------------------------------------------------------------------
+
+def hadamard_entry(j: int, k: int) -> int:
+    return _load().hqo_hadamard_entry(j, k)
+
+
+def sylvester(n: int) -> np.ndarray:
+    out = np.zeros((n, n), dtype=np.int8)
+    _check(_load().hqo_sylvester(n, _ptr(out, ctypes.c_int8)), "sylvester")
+    return out
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    bits = np.asarray(bits, dtype=np.uint16)
+    lib = _load()
+    return np.vectorize(lambda b: lib.hqo_bf16_to_f64(int(b)), otypes=[np.float64])(bits)
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    lib = _load()
+    return np.vectorize(lambda v: lib.hqo_f64_to_bf16(float(v)), otypes=[np.uint16])(x)
+
+
+def rne(x) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    lib = _load()
+    return np.vectorize(lambda v: lib.hqo_rne(float(v)), otypes=[np.float64])(x)
+
+
+# ---------------------------------------------------------------------------
+# layer steps
+# ---------------------------------------------------------------------------
+
+def col_absmax(M_bits: np.ndarray) -> np.ndarray:
+    M = _c(M_bits, np.uint16)
+    R, C = M.shape
+    out = np.zeros(C, dtype=np.float64)
+    _check(_load().hqo_col_absmax(_ptr(M, ctypes.c_uint16), R, C, _ptr(out, ctypes.c_double)),
+           "col_absmax")
+    return out
+
+
+def sigma(amax_x: np.ndarray, amax_w: np.ndarray, alpha: float) -> np.ndarray:
+    ax = _c(amax_x, np.float64)
+    aw = _c(amax_w, np.float64)
+    out = np.zeros_like(ax)
+    _check(_load().hqo_sigma(ax.size, _ptr(ax, ctypes.c_double), _ptr(aw, ctypes.c_double),
+                             float(alpha), _ptr(out, ctypes.c_double)), "sigma")
+    return out
+
+
+def quantize_act(X_bits, n, bits, gran=0, centering=1, sigma=None, static_scale=0.0,
+                 rows=None, want_tie=True, want_Z=False, nthreads=None):
+    """Returns dict(codes int8 [r,K], scale f64 [r], mean f64 [r], tie, Z)."""
+    X = _c(X_bits, np.uint16)
+    T, K = X.shape
+    sig = _c(sigma, np.float64)
+    r = None if rows is None else _c(rows, np.int64)
+    nr = T if r is None else r.size
+    codes = np.zeros((nr, K), dtype=np.int8)
+    scale = np.zeros(nr, dtype=np.float64)
+    mean = np.zeros(nr, dtype=np.float64)
+    tie = np.zeros((nr, K), dtype=np.float64) if want_tie else None
+    Z = np.zeros((nr, K), dtype=np.float64) if want_Z else None
+    rc = _load().hqo_quantize_act(
+        K, n, bits, gran, centering, _ptr(X, ctypes.c_uint16), T, _ptr(sig, ctypes.c_double),
+        float(static_scale), _ptr(r, ctypes.c_int64), nr, _ptr(codes, ctypes.c_int8),
+        _ptr(scale, ctypes.c_double), _ptr(mean, ctypes.c_double), _ptr(tie, ctypes.c_double),
+        _ptr(Z, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "quantize_act")
+    return {"codes": codes, "scale": scale, "mean": mean, "tie": tie, "Z": Z}
+
+
+def prepare_weights(W_bits, n, bits, bias_bits=None, sigma=None, want_tie=True,
+                    want_Wt=False, nthreads=None):
+    """Returns dict(codes int8 [N,K], scale [N], colsum [N], bias [N], tie, Wt)."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    b = _c(bias_bits, np.uint16)
+    sig = _c(sigma, np.float64)
+    codes = np.zeros((N, K), dtype=np.int8)
+    scale = np.zeros(N, dtype=np.float64)
+    colsum = np.zeros(N, dtype=np.float64)
+    bias = np.zeros(N, dtype=np.float64)
+    tie = np.zeros((N, K), dtype=np.float64) if want_tie else None
+    Wt = np.zeros((N, K), dtype=np.float64) if want_Wt else None
+    rc = _load().hqo_prepare_weights(
+        K, N, n, bits, _ptr(W, ctypes.c_uint16), _ptr(b, ctypes.c_uint16),
+        _ptr(sig, ctypes.c_double), _ptr(codes, ctypes.c_int8), _ptr(scale, ctypes.c_double),
+        _ptr(colsum, ctypes.c_double), _ptr(bias, ctypes.c_double), _ptr(tie, ctypes.c_double),
+        _ptr(Wt, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "prepare_weights")
+    return {"codes": codes, "scale": scale, "colsum": colsum, "bias": bias, "tie": tie, "Wt": Wt}
+
+
+def gemm_acc(A, B, rows=None, nthreads=None) -> np.ndarray:
+    A = _c(A, np.int8)
+    B = _c(B, np.int8)
+    M, K = A.shape
+    N, K2 = B.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    r = None if rows is None else _c(rows, np.int64)
+    nr = M if r is None else r.size
+    acc = np.zeros((nr, N), dtype=np.int64)
+    _check(_load().hqo_gemm_acc(_ptr(A, ctypes.c_int8), _ptr(B, ctypes.c_int8), M, N, K,
+                                _ptr(r, ctypes.c_int64), nr, _ptr(acc, ctypes.c_int64),
+                                nthreads or default_threads()), "gemm_acc")
+    return acc
+
+
+def epilogue(acc, sx, sw, colsum=None, bias=None, mean=None):
+    """Returns (y f64 [r,N], y_bf16 uint16 [r,N])."""
+    acc = _c(acc, np.int64)
+    nr, N = acc.shape
+    sx = _c(np.broadcast_to(np.asarray(sx, dtype=np.float64), (nr,)), np.float64)
+    sw = _c(sw, np.float64)
+    m = None if mean is None else _c(np.broadcast_to(np.asarray(mean, dtype=np.float64), (nr,)),
+                                     np.float64)
+    b = _c(bias, np.float64)
+    c = _c(colsum, np.float64)
+    y = np.zeros((nr, N), dtype=np.float64)
+    yb = np.zeros((nr, N), dtype=np.uint16)
+    _check(_load().hqo_epilogue(_ptr(acc, ctypes.c_int64), nr, N, _ptr(sx, ctypes.c_double),
+                                _ptr(m, ctypes.c_double), _ptr(sw, ctypes.c_double),
+                                _ptr(b, ctypes.c_double), _ptr(c, ctypes.c_double),
+                                _ptr(y, ctypes.c_double), _ptr(yb, ctypes.c_uint16)), "epilogue")
+    return y, yb
+
+
+def exact_linear(X_bits, W_bits, bias_bits=None, rows=None, nthreads=None) -> np.ndarray:
+    X = _c(X_bits, np.uint16)
+    W = _c(W_bits, np.uint16)
+    T, K = X.shape
+    N = W.shape[0]
+    b = _c(bias_bits, np.uint16)
+    r = None if rows is None else _c(rows, np.int64)
+    nr = T if r is None else r.size
+    y = np.zeros((nr, N), dtype=np.float64)
+    _check(_load().hqo_exact_linear(_ptr(X, ctypes.c_uint16), _ptr(W, ctypes.c_uint16),
+                                    _ptr(b, ctypes.c_uint16), T, K, N, _ptr(r, ctypes.c_int64),
+                                    nr, _ptr(y, ctypes.c_double), nthreads or default_threads()),
+           "exact_linear")
+    return y
+
+
+# ---------------------------------------------------------------------------
+# the whole layer, as the pages state it
+# ---------------------------------------------------------------------------
+
+def layer(X_bits, W_bits, bias_bits, n, a_bits, w_bits, gran=0, centering=1, alpha=0.5,
+          use_sigma=True, rows=None, static_scale=0.0, nthreads=None):
+    """Full oracle chain for the listed rows (all rows when rows is None):
+    sigma (Eq. 3, calibrated on this X) -> weight fold / quantize -> activation
+    transform / centering / quantize -> integer GEMM -> epilogue.
+    Returns a dict with every intermediate."""
+    sig = None
+    if use_sigma:
+        sig = sigma(col_absmax(X_bits), col_absmax(W_bits), alpha)
+    w = prepare_weights(W_bits, n, w_bits, bias_bits=bias_bits, sigma=sig, nthreads=nthreads)
+    a = quantize_act(X_bits, n, a_bits, gran=gran, centering=centering, sigma=sig,
+                     static_scale=static_scale, rows=rows, nthreads=nthreads)
+    acc = gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
+    y, yb = epilogue(acc, a["scale"], w["scale"], colsum=w["colsum"], bias=w["bias"],
+                     mean=a["mean"] if centering else None)
+    return {"sigma": sig, "w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb}

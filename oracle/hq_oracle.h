@@ -1,0 +1,109 @@
+/*
+ * hq_oracle.h -- plain fp64 CPU restatement of the HadaNorm Hadamard-domain
+ * quantized linear layer.  TEST INFRASTRUCTURE ONLY: the tests, the smoke
+ * check and the CPU-baseline leg of the benchmark may call it; the product
+ * library never does.  It shares no source with the CUDA path.
+ *
+ * Sources (page title, section / equation):
+ *   - "HadaNorm: Diffusion Transformer Quantization through Mean-Centered
+ *     Transformations" (pith.science review), "What carries the argument":
+ *     Eq. (1) XW+b = X~W~+b~ with X~ = X diag(sigma^-1) H - mu,
+ *     W~ = H^T diag(sigma) W, b~ = b + mu W~, and Eq. (3)
+ *     sigma_i = max|X_i|^alpha / max|W_i|^(1-alpha).
+ *   - "Hadamard-Domain Model Quantization for Learned Image Coding" (HaTQ),
+ *     Sec. III-A Eq. (3) (symmetric quantizer), Sec. III-C Eq. (7)-(8)
+ *     (normalized Hadamard), Sec. IV-B Eq. (13)-(14), (18) (double-Hadamard
+ *     product, accumulator scale), Supplement VII-A Eq. (34) (Sylvester).
+ *   - "Data-free 4-bit quantization for diffusion transformers",
+ *     "Hadamard rotation: the int4 improvement", step 7 (block-diagonal H).
+ *
+ * Conventions: bf16 values are passed as their 16-bit patterns (uint16_t).
+ * Matrices are row-major.  X is [T,K] (tokens x channels), W is [N,K]
+ * (output channels x input channels, so the math-convention weight of the
+ * pages is W^T).  Every function returns 0 on success, -1 on a bad argument.
+ */
+#ifndef HQ_ORACLE_H
+#define HQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Unnormalized Sylvester-order Hadamard entry (-1)^popcount(j & k). */
+int hqo_hadamard_entry(int64_t j, int64_t k);
+
+/* Builds the unnormalized Sylvester matrix of order n (a power of two) by the
+ * doubling recursion H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]] into
+ * out[n*n] (row-major, entries +-1). */
+int hqo_sylvester(int64_t n, int8_t* out);
+
+/* Exact bf16 -> double, and double -> bf16 with round-half-to-even. */
+double hqo_bf16_to_f64(uint16_t b);
+uint16_t hqo_f64_to_bf16(double x);
+
+/* Round half to even on doubles. */
+double hqo_rne(double x);
+
+/* out[c] = max_r |M[r,c]| for a bf16 matrix M[R,C]. */
+int hqo_col_absmax(const uint16_t* M, int64_t R, int64_t C, double* out);
+
+/* sigma_k = amax_x[k]^alpha / amax_w[k]^(1-alpha); sigma_k = 1 when either
+ * maximum is zero. */
+int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
+              double alpha, double* sigma);
+
+/* Activation side of the layer for the rows listed in `rows` (all T rows when
+ * rows == NULL, then nrows must equal T):
+ *   Z = X diag(sigma^-1) H            (dense block-diagonal H of order n)
+ *   m_t = mean_k Z[t,k]  (centering = 1) or 0 (centering = 0)
+ *   V = Z - m
+ *   per token  (gran 0): s_t = max_k |V[t,k]| / q
+ *   per tensor (gran 1): s   = max_{t,k} |V[t,k]| / q   over ALL T rows
+ *   static     (gran 2): s   = static_scale
+ *   code = clamp(rne(V / s), -q, q), q = 2^(bits-1) - 1; s = 0 gives code 0.
+ * Outputs per listed row i: codes[i*K+k], scale[i], mean[i]; optional
+ * tie[i*K+k] = | |V/s| - floor(|V/s|) - 1/2 | (distance of the scaled value
+ * from a rounding tie, in code units; 0.5 when s = 0) and Z[i*K+k]. */
+int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
+                     const uint16_t* X, int64_t T, const double* sigma,
+                     double static_scale, const int64_t* rows, int64_t nrows,
+                     int8_t* codes, double* scale, double* mean, double* tie,
+                     double* Z, int nthreads);
+
+/* Weight side:  W~[n,k] = sum_j H[j,k] sigma_j W[n,j]  (W~ = H^T diag(sigma) W
+ * in the pages' orientation), colsum[n] = sum_k W~[n,k],
+ * w_scale[n] = max_k |W~[n,k]| / q, w_codes = clamp(rne(W~ / w_scale), -q, q),
+ * bias_out[n] = b[n] (0 when bias == NULL).  sigma == NULL means sigma = 1.
+ * Optional outputs: tie[N*K] and Wt[N*K] (the unquantized W~). */
+int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
+                        const uint16_t* W, const uint16_t* bias,
+                        const double* sigma, int8_t* w_codes, double* w_scale,
+                        double* colsum, double* bias_out, double* tie,
+                        double* Wt, int nthreads);
+
+/* acc[i*N+c] = sum_k A[rows[i],k] * B[c,k] in 64-bit integers, for int8
+ * matrices A[M,K] and B[N,K] (rows == NULL: all M rows, nrows == M). */
+int hqo_gemm_acc(const int8_t* A, const int8_t* B, int64_t M, int64_t N,
+                 int64_t K, const int64_t* rows, int64_t nrows, int64_t* acc,
+                 int nthreads);
+
+/* y[i*N+c] = sx[i] * sw[c] * acc[i*N+c] + b[c] + m[i] * colsum[c]  (fp64), and
+ * y_bf16 its bf16 rounding (either output may be NULL).  sx and m are per
+ * listed row; m == NULL means m = 0; b == NULL means b = 0. */
+int hqo_epilogue(const int64_t* acc, int64_t nrows, int64_t N,
+                 const double* sx, const double* m, const double* sw,
+                 const double* b, const double* colsum, double* y,
+                 uint16_t* y_bf16);
+
+/* Unquantized reference y[i*N+c] = sum_k X[rows[i],k] W[c,k] + b[c] (fp64). */
+int hqo_exact_linear(const uint16_t* X, const uint16_t* W, const uint16_t* bias,
+                     int64_t T, int64_t K, int64_t N, const int64_t* rows,
+                     int64_t nrows, double* y, int nthreads);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_ORACLE_H */

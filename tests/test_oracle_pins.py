@@ -1,0 +1,343 @@
+"""Pins for the CPU oracle: each check compares the oracle with something other
+than itself (a second construction, a closed form, a hand-worked value, exact
+integer arithmetic, or the unquantized product).  CPU only."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+POW2 = [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024]
+
+
+def kron_sylvester(n):
+    """Sylvester matrix as a Kronecker power of [[1,1],[1,-1]] (independent of
+    both oracle constructions)."""
+    h = np.ones((1, 1), dtype=np.int64)
+    base = np.array([[1, 1], [1, -1]], dtype=np.int64)
+    while h.shape[0] < n:
+        h = np.kron(h, base)
+    return h
+
+
+# --------------------------------------------------------------------------
+# Hadamard matrix: HaTQ Eq. (32)-(34), blog step 7
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", POW2)
+def test_sylvester_recursion_matches_popcount_entries(n):
+    h_rec = oracle.sylvester(n).astype(np.int64)
+    h_pop = np.array([[oracle.hadamard_entry(j, k) for k in range(n)] for j in range(n)]) \
+        if n <= 64 else None
+    h_kron = kron_sylvester(n)
+    assert np.array_equal(h_rec, h_kron)
+    if h_pop is not None:
+        assert np.array_equal(h_pop, h_kron)
+    else:  # spot-check the popcount formula on a seeded sample for large orders
+        g = np.random.default_rng(n)
+        for j, k in g.integers(0, n, size=(2000, 2)):
+            assert oracle.hadamard_entry(int(j), int(k)) == h_kron[j, k]
+
+
+@pytest.mark.parametrize("n", POW2)
+def test_hadamard_orthogonality_exact(n):
+    h = oracle.sylvester(n).astype(np.int64)
+    assert np.array_equal(h @ h.T, n * np.eye(n, dtype=np.int64))
+    assert np.array_equal(h, h.T)  # symmetric, so H^T = H
+
+
+def test_h64_is_the_kronecker_power_printed_on_the_blog():
+    spec = json.load(open(os.path.join(GOLDEN, "hand_examples.json")))["h64_kronecker"]
+    f = np.array(spec["factor"], dtype=np.float64)
+    h = np.ones((1, 1))
+    for _ in range(spec["power"]):
+        h = np.kron(h, f)
+    h *= spec["scale"]
+    # the oracle's normalized block: Z for unit vectors e_j is row j of H_64
+    n = spec["n"]
+    X = synth.f32_to_bf16_bits(np.eye(n, dtype=np.float32))
+    r = oracle.quantize_act(X, n, 8, centering=0, want_Z=True)
+    assert np.allclose(r["Z"], h, rtol=0, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# scalar helpers
+# --------------------------------------------------------------------------
+
+def test_round_half_even():
+    xs = [0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 0.49999999999, 0.5000000001, 3.0, -7.5, 6.5, 2.4, -2.6]
+    want = [0.0, 2.0, 2.0, -0.0, -2.0, -2.0, 0.0, 1.0, 3.0, -8.0, 6.0, 2.0, -3.0]
+    got = oracle.rne(xs)
+    assert np.array_equal(got, np.array(want))
+
+
+def test_bf16_conversions():
+    # 1.0, 1 + 2^-8 (tie -> even 1.0), 1 + 3*2^-8 (tie -> even 1 + 2^-6 .. i.e. 0x3F82),
+    # -2.0, smallest normal, 65280 (max exact near 2^16), 1/3
+    vals = [1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.0, 2.0 ** -126, 65280.0, 1.0 / 3.0]
+    bits = [0x3F80, 0x3F80, 0x3F82, 0xC000, 0x0080, 0x477F, 0x3EAB]
+    assert list(oracle.f64_to_bf16(vals)) == bits
+    assert np.array_equal(oracle.bf16_to_f64(np.array(bits[:6], dtype=np.uint16)),
+                          np.array([1.0, 1.0, 1.0 + 2 ** -6, -2.0, 2.0 ** -126, 65280.0]))
+    # agreement with the float32 path of the generator on random data
+    g = np.random.default_rng(0)
+    x = g.standard_normal(5000) * 10.0 ** g.uniform(-3, 3, 5000)
+    assert np.array_equal(oracle.f64_to_bf16(x.astype(np.float32).astype(np.float64)),
+                          synth.f32_to_bf16_bits(x.astype(np.float32)))
+
+
+# --------------------------------------------------------------------------
+# hand-worked quantizer examples (golden)
+# --------------------------------------------------------------------------
+
+def test_hand_worked_examples():
+    spec = json.load(open(os.path.join(GOLDEN, "hand_examples.json")))
+    for ex in spec["examples"]:
+        X = synth.f32_to_bf16_bits(np.array([ex["x"]], dtype=np.float32))
+        r = oracle.quantize_act(X, ex["n"], ex["bits"], centering=ex["centering"], want_Z=True)
+        assert np.allclose(r["Z"][0], ex["Z"], atol=1e-15), ex["name"]
+        assert abs(r["mean"][0] - ex["mean"]) < 1e-15, ex["name"]
+        assert abs(r["scale"][0] - ex["scale"]) < 1e-15, ex["name"]
+        assert list(r["codes"][0]) == ex["codes"], ex["name"]
+
+
+# --------------------------------------------------------------------------
+# Eq. (1) identity with quantization off
+# --------------------------------------------------------------------------
+
+def _bf16(x):
+    return synth.bf16_bits_to_f32(x).astype(np.float64)
+
+
+@pytest.mark.parametrize("K,n,N,T", [(16, 4, 8, 5), (64, 16, 24, 9), (256, 64, 40, 7),
+                                     (1152, 128, 32, 4), (3072, 1024, 16, 3)])
+@pytest.mark.parametrize("centering", [0, 1])
+def test_eq1_identity_unquantized(K, n, N, T, centering):
+    g = np.random.default_rng(K + n + centering)
+    X = synth.f32_to_bf16_bits(g.standard_normal((T, K)) * 2 + g.standard_normal((T, 1)) * 3)
+    W = synth.f32_to_bf16_bits(g.standard_normal((N, K)) * 0.05)
+    b = synth.f32_to_bf16_bits(g.standard_normal(N) * 0.1)
+    sig = oracle.sigma(oracle.col_absmax(X), oracle.col_absmax(W), 0.5)
+    assert np.all(sig > 0) and not np.allclose(sig, 1.0)
+    a = oracle.quantize_act(X, n, 8, centering=centering, sigma=sig, want_Z=True)
+    w = oracle.prepare_weights(W, n, 8, bias_bits=b, sigma=sig, want_Wt=True)
+    V = a["Z"] - a["mean"][:, None]                       # X~ = X diag(s^-1) H - mu
+    y_tilde = V @ w["Wt"].T + w["bias"][None, :] + a["mean"][:, None] * w["colsum"][None, :]
+    y = _bf16(X) @ _bf16(W).T + _bf16(b)[None, :]          # XW + b
+    rel = np.linalg.norm(y_tilde - y) / np.linalg.norm(y)
+    assert rel <= 1e-10, rel
+    # the layer's own exact reference agrees with the numpy product
+    assert np.allclose(oracle.exact_linear(X, W, b), y, rtol=0, atol=1e-10 * np.abs(y).max())
+
+
+# --------------------------------------------------------------------------
+# closed-form invariants
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,n", [(64, 16), (1152, 128), (320, 64), (2048, 1024)])
+def test_invariants(K, n):
+    T, N = 6, 10
+    g = np.random.default_rng(K)
+    X = synth.f32_to_bf16_bits(g.standard_normal((T, K)) + 2.0)
+    W = synth.f32_to_bf16_bits(g.standard_normal((N, K)) * 0.02)
+    sig = oracle.sigma(oracle.col_absmax(X), oracle.col_absmax(W), 0.5)
+    a = oracle.quantize_act(X, n, 4, centering=1, sigma=sig, want_Z=True)
+    w = oracle.prepare_weights(W, n, 4, sigma=sig, want_Wt=True)
+    Y = _bf16(X) / sig[None, :]
+    Z = a["Z"]
+    B = K // n
+    rn = math.sqrt(n)
+    # HaTQ Eq. (23): the constant-basis coordinate is sqrt(n) times the block mean
+    for blk in range(B):
+        assert np.allclose(Z[:, blk * n], rn * Y[:, blk * n:(blk + 1) * n].mean(axis=1),
+                           rtol=1e-12, atol=1e-12)
+    # column sums of H~ vanish except the first: m_t = (sqrt(n)/K) sum_b Y[t, b n]
+    assert np.allclose(a["mean"], rn / K * Y[:, ::n].sum(axis=1), rtol=1e-12, atol=1e-12)
+    # same for the weight fold: c_n = sqrt(n) sum_b sigma_{bn} W[n, bn]
+    Wf = _bf16(W)
+    assert np.allclose(w["colsum"], rn * (Wf[:, ::n] * sig[None, ::n]).sum(axis=1),
+                       rtol=1e-11, atol=1e-12)
+    # centred activations sum to zero; the rotation preserves each block's norm
+    V = Z - a["mean"][:, None]
+    assert np.allclose(V.sum(axis=1), 0.0, atol=1e-10 * np.abs(Z).max())
+    for blk in range(B):
+        s = slice(blk * n, (blk + 1) * n)
+        assert np.allclose(np.linalg.norm(Z[:, s], axis=1), np.linalg.norm(Y[:, s], axis=1),
+                           rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# brute force at K = 8: exact integer decision of every code
+# --------------------------------------------------------------------------
+
+def _exact_codes_int(x_int, n, q, centering):
+    """Exact codes for integer inputs with sigma = 1, decided in integer
+    arithmetic.  Z_hat = x H~ is an integer vector and Z = Z_hat / sqrt(n);
+    the codes depend only on V / max|V|, so scale V by K*sqrt(n):
+    U = K*Z_hat - sum(Z_hat) (centred) or K*Z_hat (not centred).
+    code = rne(q * U / max|U|).  Returns (codes, is_exact_tie)."""
+    B = x_int.shape[1] // n
+    H = kron_sylvester(n)
+    zh = np.concatenate([x_int[:, b * n:(b + 1) * n] @ H for b in range(B)], axis=1)
+    K = x_int.shape[1]
+    U = K * zh - (zh.sum(axis=1, keepdims=True) if centering else 0)
+    D = np.abs(U).max(axis=1, keepdims=True)
+    num = q * U
+    den = np.where(D == 0, 1, D)
+    f = np.floor_divide(num, den)
+    r = num - f * den
+    two_r = 2 * r
+    up = two_r > den
+    tie = two_r == den
+    codes = f + up + (tie & (f % 2 != 0))
+    codes = np.where(D == 0, 0, codes)
+    return codes, tie & (D != 0), zh
+
+
+@pytest.mark.parametrize("n", [4, 8])
+@pytest.mark.parametrize("bits,centering", [(4, 1), (3, 1), (4, 0)])
+def test_bruteforce_k8(n, bits, centering):
+    vals = np.arange(-2, 3)
+    x_int = np.array(list(itertools.product(vals, repeat=8)), dtype=np.int64)  # 5^8 rows
+    X = synth.f32_to_bf16_bits(x_int.astype(np.float32))
+    q = 2 ** (bits - 1) - 1
+    r = oracle.quantize_act(X, n, bits, centering=centering, want_Z=True)
+    want, tie, zh = _exact_codes_int(x_int, n, q, centering)
+    # the dense transform equals an independent evaluation of HaTQ Eq. (8)
+    assert np.allclose(r["Z"], zh / math.sqrt(n), rtol=0, atol=1e-13)
+    codes = r["codes"].astype(np.int64)
+    off = codes != want
+    # away from exact ties the decision is unique
+    assert not np.any(off & ~tie)
+    # at exact ties (fp64 cannot see them when q/n makes the scale inexact) the
+    # oracle must still pick one of the two neighbours
+    assert np.all(np.abs(codes - want)[tie] <= 1)
+    assert np.all(np.abs(codes) <= q)
+    # exhaustive arg-min over the 2q+1 grid levels agrees with the code
+    levels = np.arange(-q, q + 1)
+    V = r["Z"] - r["mean"][:, None]
+    s = r["scale"][:, None]
+    safe = np.where(s == 0, 1.0, s)
+    dist = np.abs((V / safe)[..., None] - levels[None, None, :])
+    best = levels[np.argmin(dist + 1e-9 * (np.abs(levels) % 2)[None, None, :], axis=2)]
+    best = np.where(s == 0, 0, best)
+    assert np.array_equal(best[~tie], codes[~tie])
+
+
+def test_integer_accumulation_all_int4_vectors():
+    levels = np.arange(-7, 8, dtype=np.int8)
+    A = np.array(list(itertools.product(levels, repeat=4)), dtype=np.int8)  # 15^4 rows
+    g = np.random.default_rng(4)
+    B = g.integers(-8, 8, size=(6, 4)).astype(np.int8)
+    B[0] = 7
+    B[1] = -7
+    acc = oracle.gemm_acc(A, B)
+    assert np.array_equal(acc, A.astype(np.int64) @ B.astype(np.int64).T)
+
+
+def test_integer_accumulation_full_int8_range():
+    g = np.random.default_rng(5)
+    A = g.integers(-128, 128, size=(37, 300)).astype(np.int8)
+    B = g.integers(-128, 128, size=(19, 300)).astype(np.int8)
+    A[0] = -128
+    B[0] = -128
+    rows = np.array([0, 5, 36])
+    acc = oracle.gemm_acc(A, B, rows=rows)
+    assert np.array_equal(acc, (A.astype(np.int64) @ B.astype(np.int64).T)[rows])
+
+
+# --------------------------------------------------------------------------
+# lossless case: the quantized chain reproduces XW + b exactly
+# --------------------------------------------------------------------------
+
+def test_dyadic_lossless_chain_equals_exact_product():
+    """Build X and W whose rotated (and centred) values sit exactly on their
+    grids, so quantization loses nothing: then s_x s_w acc + b + m c must equal
+    XW + b (HadaNorm Eq. (1) with the HaTQ Eq. (18) accumulator scale).  A
+    dropped term, wrong sign or transposed operand breaks the equality."""
+    n, K, N, T = 4, 8, 5, 4
+    H = kron_sylvester(n) / 2.0                      # H~_4 / sqrt(4), exact
+    Hb = np.kron(np.eye(K // n), H)
+    g = np.random.default_rng(11)
+    X_rows, m_list = [], []
+    for t in range(T):
+        c = g.integers(-6, 7, size=K)
+        c[0] = 7
+        c[-1] = -(c[:-1].sum())                      # sum of V = 0
+        if abs(c[-1]) > 7:
+            c[1:-1] = 0
+            c[-1] = -7
+        s = 0.25
+        m = float(g.integers(-8, 9)) * 0.125
+        Z = s * c + m
+        X_rows.append(Z @ Hb.T)                      # X = Z H^T (H orthogonal)
+        m_list.append(m)
+    Xf = np.array(X_rows)
+    Wq = g.integers(-7, 8, size=(N, K))
+    Wq[:, 0] = 7
+    Wt = 0.125 * Wq
+    Wf = Wt @ Hb.T                                   # W~ = W H  =>  W = W~ H^T
+    bf = g.integers(-4, 5, size=N) * 0.0625
+    X = synth.f32_to_bf16_bits(Xf.astype(np.float32))
+    W = synth.f32_to_bf16_bits(Wf.astype(np.float32))
+    b = synth.f32_to_bf16_bits(bf.astype(np.float32))
+    assert np.array_equal(_bf16(X), Xf) and np.array_equal(_bf16(W), Wf)
+    out = oracle.layer(X, W, b, n, 4, 4, centering=1, use_sigma=False)
+    assert np.allclose(out["a"]["mean"], m_list, atol=0)
+    y_exact = oracle.exact_linear(X, W, b)
+    assert np.array_equal(out["y"], y_exact), np.abs(out["y"] - y_exact).max()
+    assert np.array_equal(out["y_bf16"], oracle.f64_to_bf16(y_exact))
+
+
+# --------------------------------------------------------------------------
+# granularities and row sampling
+# --------------------------------------------------------------------------
+
+def test_per_tensor_and_static_scales():
+    cfg = synth.CONFIGS[4].with_tokens(64)
+    X = synth.make_x(cfg)
+    tok = oracle.quantize_act(X, 64, 8, gran=0, centering=0)
+    ten = oracle.quantize_act(X, 64, 8, gran=1, centering=0)
+    assert np.allclose(ten["scale"], tok["scale"].max(), rtol=1e-15)
+    st = oracle.quantize_act(X, 64, 8, gran=2, centering=0, static_scale=ten["scale"][0])
+    assert np.array_equal(st["codes"], ten["codes"])
+    # sampled rows of a per-tensor quantization still use the whole-tensor scale
+    rows = np.array([3, 17, 63])
+    sub = oracle.quantize_act(X, 64, 8, gran=1, centering=0, rows=rows)
+    assert np.array_equal(sub["codes"], ten["codes"][rows])
+    assert np.all(sub["scale"] == ten["scale"][0])
+
+
+def test_row_subset_matches_full():
+    cfg = synth.CONFIGS[2].with_tokens(40)
+    X = synth.make_x(cfg)
+    full = oracle.quantize_act(X, 128, 4)
+    rows = np.array([0, 7, 39])
+    sub = oracle.quantize_act(X, 128, 4, rows=rows)
+    assert np.array_equal(sub["codes"], full["codes"][rows])
+    assert np.array_equal(sub["scale"], full["scale"][rows])
+    assert np.array_equal(sub["mean"], full["mean"][rows])
+
+
+def test_zero_row_gives_zero_codes_and_scale():
+    X = np.zeros((2, 64), dtype=np.uint16)
+    X[1] = synth.f32_to_bf16_bits(np.linspace(-1, 1, 64).astype(np.float32))
+    r = oracle.quantize_act(X, 64, 4)
+    assert r["scale"][0] == 0.0 and not r["codes"][0].any()
+    assert r["scale"][1] > 0.0
+
+
+def test_quantization_noise_is_within_grid_bound():
+    """|V - s * code| <= s / 2 for every element (HaTQ Eq. (3) with rne)."""
+    cfg = synth.CONFIGS[3].with_tokens(16)
+    X = synth.make_x(cfg)
+    r = oracle.quantize_act(X, 256, 3, want_Z=True)
+    V = r["Z"] - r["mean"][:, None]
+    err = np.abs(V - r["scale"][:, None] * r["codes"])
+    assert np.all(err <= r["scale"][:, None] / 2 * (1 + 1e-12))
