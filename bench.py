@@ -1,0 +1,446 @@
+"""Benchmark of the Hadamard-domain quantized linear layer on B200.
+
+One step = the layer's runtime hot path over one batch: hq_quantize_act
+(bf16 load, sigma^-1, block FWHT, centring, per-token int4 quantization)
+followed by hq_linear (tcgen05 int8 GEMM + fused epilogue) -- every step of
+the layer except the offline weight preparation, which is timed once and
+reported separately.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl hq|reference]
+
+Prints one JSON line (rank 0).  `value` is device-timed throughput of the
+whole job in TOPS (2*T*K*N integer ops of the layer per step, summed over
+ranks, divided by the max over ranks of the summed per-step CUDA-event times).
+L2 is flushed (memset of a buffer twice the L2 size) before every timed step,
+outside the timed events.  Ranks are independent data-parallel shards: each
+rank owns its own batch of tokens and a replica of the prepared weights; there
+is no collective on the data path (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "HadaNorm W4A4 linear TOPS & quantizer HBM GB/s (fraction of roofline), 1×B200"
+DEFAULT_CONFIG = 2          # the PixArt-Sigma-shaped qkv projection (the metric's workload)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0        # nominal dense int8 : bf16 tensor ratio (4.5 : 2.25 PFLOP/s)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the bounded oracle sample")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per step
+# ---------------------------------------------------------------------------
+
+def layer_ops(cfg) -> float:
+    return 2.0 * cfg.T * cfg.K * cfg.N
+
+
+def quantizer_bytes(cfg) -> float:
+    """Algorithmic bytes of hq_quantize_act: read X (2 B/elt), write int8 codes
+    (1 B/elt in the int8 container), write scale + mean (8 B/token); the
+    per-tensor dynamic mode reads X twice."""
+    passes = 2 if cfg.act_gran == 1 else 1
+    return cfg.T * cfg.K * (2.0 * passes + 1.0) + 8.0 * cfg.T
+
+
+def gemm_bytes(cfg) -> float:
+    """Algorithmic HBM bytes of hq_linear: A codes + B codes + bf16 Y + per-row
+    and per-column fp32 vectors."""
+    return cfg.T * cfg.K + cfg.N * cfg.K + 2.0 * cfg.T * cfg.N + 8.0 * cfg.T + 12.0 * cfg.N
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the timed region runs
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+def oracle_prepare(cfg, Xb, Wb, bb):
+    import oracle
+    sig = None
+    if cfg.use_sigma:
+        sig = oracle.sigma(oracle.col_absmax(Xb), oracle.col_absmax(Wb), cfg.alpha)
+    w = oracle.prepare_weights(Wb, cfg.had_order, cfg.w_bits, bias_bits=bb, sigma=sig,
+                               want_tie=False)
+    return sig, w
+
+
+def oracle_step(cfg, Xb, sig, w, rows, nthreads):
+    """The oracle's runtime path for the listed rows: transform / centre /
+    quantize, integer GEMM, epilogue (weight side prepared beforehand)."""
+    import oracle
+    a = oracle.quantize_act(Xb, cfg.had_order, cfg.a_bits, gran=cfg.act_gran,
+                            centering=cfg.centering, sigma=sig, rows=rows, want_tie=False,
+                            nthreads=nthreads)
+    acc = oracle.gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
+    oracle.epilogue(acc, a["scale"], w["scale"], colsum=w["colsum"], bias=w["bias"],
+                    mean=a["mean"] if cfg.centering else None)
+
+
+def size_oracle_sample(cfg, Xb, sig, w, nthreads, target_s):
+    """Number of rows whose oracle step takes about target_s seconds."""
+    probe = min(cfg.T, 16)
+    rows = synth.sample_rows(cfg.T, probe, tile=max(1, cfg.T // probe), seed=1)
+    t0 = time.perf_counter()
+    oracle_step(cfg, Xb, sig, w, rows, nthreads)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    per_row = dt / len(rows)
+    n = int(max(8, min(cfg.T, target_s / per_row)))
+    return n
+
+
+def cpu_baseline(cfg, Xb, Wb, bb, target_s):
+    nthreads = os.cpu_count() or 1
+    sig, w = oracle_prepare(cfg, Xb, Wb, bb)
+    n = size_oracle_sample(cfg, Xb, sig, w, nthreads, target_s)
+    rows = synth.sample_rows(cfg.T, n, tile=max(1, cfg.T // n), seed=2)
+    t0 = time.perf_counter()
+    oracle_step(cfg, Xb, sig, w, rows, nthreads)
+    dt = time.perf_counter() - t0
+    ops = 2.0 * len(rows) * cfg.K * cfg.N
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
+            "sample": f"{len(rows)} of {cfg.T} tokens (seeded, every tile), full K and N; "
+                      f"runtime path only (weights prepared beforehand); {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle as it stands, on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = synth.CONFIGS[args.config]
+    Xb, Wb, bb = synth.make_layer(cfg)
+    nthreads = os.cpu_count() or 1
+    sig, w = oracle_prepare(cfg, Xb, Wb, bb)
+    # size each step so that warmup + steps finish within about two minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = size_oracle_sample(cfg, Xb, sig, w, nthreads, budget)
+    rows = synth.sample_rows(cfg.T, n, tile=max(1, cfg.T // n), seed=3)
+    for _ in range(args.warmup):
+        oracle_step(cfg, Xb, sig, w, rows, nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(cfg, Xb, sig, w, rows, nthreads)
+    dt = (time.perf_counter() - t0) / args.steps
+    ops = 2.0 * len(rows) * cfg.K * cfg.N
+    value = ops / dt / 1e12
+    sample = f"{len(rows)} of {cfg.T} tokens per step (seeded, every tile), full K and N"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64+int64", "data": "synthetic",
+        "config": config_block(cfg, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, n_gpus):
+    gran = {0: "per_token", 1: "per_tensor_dynamic", 2: "per_tensor_static"}[cfg.act_gran]
+    return {"workload": cfg.workload(), "tokens_per_gpu": cfg.T, "K": cfg.K, "N": cfg.N,
+            "had_order": cfg.had_order, "bits": f"A{cfg.a_bits}W{cfg.w_bits}",
+            "act_granularity": gran, "centering": bool(cfg.centering), "sigma": cfg.use_sigma,
+            "l2": "flushed before every timed step (memset of 2x L2, outside the timed events)",
+            "parallelism": f"dp{n_gpus} (token shards, replicated weights, no collective)"}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_hq(args):
+    import torch
+    import torch.distributed as dist
+
+    import hadamard_rotated_bit_token_b200 as hq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    hq.load_library()
+    cfg = synth.CONFIGS[args.config]
+    # replicated weights (same seed on every rank), rank-local token batch
+    Wb, bb = synth.make_w(cfg)
+    Xb = synth.make_x(cfg, seed=cfg.index + 1000 * rank)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    X, W, b = to_dev(Xb), to_dev(Wb), to_dev(bb)
+    T, K, N = cfg.T, cfg.K, cfg.N
+    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering)
+    stream = torch.cuda.current_stream()
+
+    # offline: calibration + weight preparation (timed once, not part of the step)
+    absmax = torch.zeros(K, dtype=torch.float32, device=dev) if cfg.use_sigma else None
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    if absmax is not None:
+        hq.hq_calib_act_absmax(desc, X, absmax)
+    layer = hq.HadamardQuantLinear(desc, W, b, absmax, cfg.alpha)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prep_ms = p0.elapsed_time(p1)
+
+    bufs = layer.buffers(T)
+    Y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    sig_inv = layer.sigma_inv if layer.use_sigma else None
+    mean_in = bufs["a_mean"] if cfg.centering else None
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def quantize():
+        hq.hq_quantize_act(desc, X, sig_inv, bufs["a_codes"], bufs["a_scale"], bufs["a_mean"],
+                           layer.workspace)
+
+    def linear():
+        hq.hq_linear(desc, bufs["a_codes"], bufs["a_scale"], mean_in, layer.w_codes,
+                     layer.w_scale, layer.colsum, layer.bias_f32, Y)
+
+    launches_per_step = (2 if cfg.act_gran == 1 else 1) + 1
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        quantize()
+        linear()
+    torch.cuda.synchronize()
+    status = hq.hq_check_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error during warm-up: {hq.STATUS_NAMES.get(status)}")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        quantize()
+        ev[i][1].record(stream)
+        linear()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop()
+    status = hq.hq_check_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error in the timed region: {hq.STATUS_NAMES.get(status)}")
+
+    q_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    g_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    ops = layer_ops(cfg)
+    value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers (pinned), per step:
+    # H2D of X, quantize, GEMM, D2H of Y
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Yh = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
+        Xd = torch.empty_like(X)
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            hq.hq_quantize_act(desc, Xd, sig_inv, bufs["a_codes"], bufs["a_scale"],
+                               bufs["a_mean"], layer.workspace)
+            linear()
+            Yh.copy_(Y, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * ops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
+               "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()),
+               "ms_per_step": e2e_ms / args.steps}
+        status = hq.hq_check_device_error()
+        if status != 0:
+            raise RuntimeError(f"device error in the e2e region: {hq.STATUS_NAMES.get(status)}")
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    q_med = statistics.median(q_ms)
+    g_med = statistics.median(g_ms)
+    q_gbs = quantizer_bytes(cfg) / (q_med * 1e-3) / 1e9
+    g_tops = ops / (g_med * 1e-3) / 1e12
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    if g_med >= q_med:
+        roof = {"kernel": "hq_gemm_i8 (tcgen05 kind::i8 + epilogue)", "bound": "tensor",
+                "achieved": g_tops, "peak": int8_peak, "unit": "TFLOP/s",
+                "frac": g_tops / int8_peak, "traffic": None,
+                "peak_source": f"{peak_src}: 2 x bf16_tflops (burst), dense int8:bf16 = 4.5:2.25",
+                "algorithmic": f"2*T*K*N = {ops:.4g} int ops per launch"}
+    else:
+        roof = {"kernel": "hq_quantize_act (fused FWHT quantizer)", "bound": "hbm",
+                "achieved": q_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": q_gbs / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic": f"{quantizer_bytes(cfg):.4g} bytes per launch"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 (s8 x s8 -> s32; fp32 transform)", "data": "synthetic",
+        "config": config_block(cfg, world),
+        "roofline": roof,
+        "kernels": {
+            "quantizer": {"ms_median": q_med, "GB/s": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
+                          "bytes": quantizer_bytes(cfg)},
+            "gemm": {"ms_median": g_med, "TOPS": g_tops, "frac_int8": g_tops / int8_peak,
+                     "hbm_bytes": gemm_bytes(cfg)},
+            "weight_prep_ms": prep_ms,
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_info,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(cfg, Xb, Wb, bb, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_hq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

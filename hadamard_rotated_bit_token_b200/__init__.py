@@ -1,0 +1,262 @@
+"""Thin Python binding of libhq.so, the sm_100a Hadamard-domain quantized
+linear layer (HadaNorm identity X W + b = X~ W~ + b~; see include/hq.h).
+
+Every function marshals torch tensors (device memory, owned by the caller) and
+the current CUDA stream into the C ABI of the same name; all computation runs
+in the library's CUDA kernels.  There is no CPU fallback: if libhq.so is
+missing or the device is not sm_100, the calls raise.
+
+    hq_calib_act_absmax(desc, X, absmax)
+    hq_prepare_weights(desc, W, bias, act_absmax, alpha, w_codes, w_scale, colsum, sigma_inv, bias_f32)
+    hq_quantize_act(desc, X, sigma_inv, a_codes, a_scale, a_mean, workspace)
+    hq_linear(desc, a_codes, a_scale, a_mean, w_codes, w_scale, colsum, bias_f32, Y, acc_debug)
+    hq_check_device_error()
+
+`HadamardQuantLinear` bundles the caller-side buffers of one layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "HQError", "LayerDesc", "load_library", "library_path", "exported_symbols",
+    "HQ_PER_TOKEN", "HQ_PER_TENSOR_DYNAMIC", "HQ_PER_TENSOR_STATIC",
+    "HQ_CENTER_NONE", "HQ_CENTER_TOKEN_MEAN", "HQ_CODES_I8",
+    "HQ_FAULT_NONE", "HQ_FAULT_QUANT_WITHHOLD_LOAD", "STATUS_NAMES",
+    "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
+    "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
+    "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
+    "HadamardQuantLinear",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+HQ_PER_TOKEN, HQ_PER_TENSOR_DYNAMIC, HQ_PER_TENSOR_STATIC = 0, 1, 2
+HQ_CENTER_NONE, HQ_CENTER_TOKEN_MEAN = 0, 1
+HQ_CODES_I8 = 0
+HQ_FAULT_NONE, HQ_FAULT_QUANT_WITHHOLD_LOAD = 0, 1
+STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED",
+                3: "HQ_ERR_MISALIGNED", 4: "HQ_ERR_CUDA", 5: "HQ_ERR_TIMEOUT",
+                6: "HQ_ERR_DEVICE"}
+EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare_weights",
+            "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
+            "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault")
+
+
+class HQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class LayerDesc(ctypes.Structure):
+    """hq_layer_desc (host memory)."""
+    _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("had_order", ctypes.c_int32),
+                ("a_bits", ctypes.c_int32), ("w_bits", ctypes.c_int32),
+                ("act_gran", ctypes.c_int32), ("centering", ctypes.c_int32),
+                ("code_format", ctypes.c_int32)]
+
+    def __init__(self, K, N, had_order, a_bits=4, w_bits=4, act_gran=HQ_PER_TOKEN,
+                 centering=HQ_CENTER_TOKEN_MEAN, code_format=HQ_CODES_I8):
+        super().__init__(K, N, had_order, a_bits, w_bits, act_gran, centering, code_format)
+
+
+_lib = None
+_lock = threading.Lock()
+_vp = ctypes.c_void_p
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Loads libhq.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: run hadamard_rotated_bit_token_b200/build.py "
+                              "(or __graft_entry__.build()) first; there is no fallback path")
+        lib = ctypes.CDLL(_LIB_PATH)
+        desc_p = ctypes.POINTER(LayerDesc)
+        lib.hq_status_string.argtypes = [ctypes.c_int]
+        lib.hq_status_string.restype = ctypes.c_char_p
+        lib.hq_version.argtypes = []
+        lib.hq_version.restype = ctypes.c_int
+        lib.hq_calib_act_absmax.argtypes = [desc_p, _vp, ctypes.c_int64, _vp, _vp]
+        lib.hq_prepare_weights.argtypes = [desc_p, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp,
+                                           _vp, _vp, _vp]
+        lib.hq_quantize_act_workspace_bytes.argtypes = [desc_p, ctypes.c_int64]
+        lib.hq_quantize_act_workspace_bytes.restype = ctypes.c_size_t
+        lib.hq_quantize_act.argtypes = [desc_p, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
+                                        ctypes.c_size_t, _vp]
+        lib.hq_linear.argtypes = [desc_p, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _vp]
+        lib.hq_check_device_error.argtypes = [_vp]
+        lib.hq_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
+        lib.hq_debug_inject_fault.argtypes = [ctypes.c_int]
+        for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
+                     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def exported_symbols():
+    lib = load_library()
+    return {name: hasattr(lib, name) for name in EXPORTED}
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("tensor must live in CUDA device memory")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise HQError(status, where)
+
+
+# ---------------------------------------------------------------------------
+# C ABI, same names
+# ---------------------------------------------------------------------------
+
+def hq_version() -> int:
+    return load_library().hq_version()
+
+
+def hq_status_string(status: int) -> str:
+    return load_library().hq_status_string(status).decode()
+
+
+def hq_calib_act_absmax(desc: LayerDesc, X, absmax, T=None, stream=None):
+    T = X.shape[0] if T is None else T
+    _check(load_library().hq_calib_act_absmax(ctypes.byref(desc), _ptr(X), T, _ptr(absmax),
+                                              _stream(stream)), "hq_calib_act_absmax")
+
+
+def hq_prepare_weights(desc: LayerDesc, W, bias, act_absmax, alpha, w_codes, w_scale, colsum,
+                       sigma_inv, bias_f32, stream=None):
+    _check(load_library().hq_prepare_weights(
+        ctypes.byref(desc), _ptr(W), _ptr(bias), _ptr(act_absmax), float(alpha), _ptr(w_codes),
+        _ptr(w_scale), _ptr(colsum), _ptr(sigma_inv), _ptr(bias_f32), _stream(stream)),
+        "hq_prepare_weights")
+
+
+def hq_quantize_act_workspace_bytes(desc: LayerDesc, T: int) -> int:
+    return load_library().hq_quantize_act_workspace_bytes(ctypes.byref(desc), T)
+
+
+def hq_quantize_act(desc: LayerDesc, X, sigma_inv, a_codes, a_scale, a_mean=None, workspace=None,
+                    T=None, stream=None):
+    T = X.shape[0] if T is None else T
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().hq_quantize_act(
+        ctypes.byref(desc), _ptr(X), T, _ptr(sigma_inv), _ptr(a_codes), _ptr(a_scale),
+        _ptr(a_mean), _ptr(workspace), ws_bytes, _stream(stream)), "hq_quantize_act")
+
+
+def hq_linear(desc: LayerDesc, a_codes, a_scale, a_mean, w_codes, w_scale, colsum, bias_f32, Y,
+              acc_debug=None, T=None, stream=None):
+    T = a_codes.shape[0] if T is None else T
+    _check(load_library().hq_linear(
+        ctypes.byref(desc), T, _ptr(a_codes), _ptr(a_scale), _ptr(a_mean), _ptr(w_codes),
+        _ptr(w_scale), _ptr(colsum), _ptr(bias_f32), _ptr(Y), _ptr(acc_debug), _stream(stream)),
+        "hq_linear")
+
+
+def hq_check_device_error(stream=None) -> int:
+    """Synchronizes the stream and returns (and clears) the device error word."""
+    return load_library().hq_check_device_error(_stream(stream))
+
+
+def hq_debug_set_wait_limit(nanoseconds: int):
+    _check(load_library().hq_debug_set_wait_limit(int(nanoseconds)), "hq_debug_set_wait_limit")
+
+
+def hq_debug_inject_fault(kind: int):
+    _check(load_library().hq_debug_inject_fault(int(kind)), "hq_debug_inject_fault")
+
+
+# ---------------------------------------------------------------------------
+# one layer's caller-side buffers
+# ---------------------------------------------------------------------------
+
+class HadamardQuantLinear:
+    """Prepared weights and activation buffers of one Hadamard-domain layer.
+
+    Allocation is the caller's (PyTorch); the library only reads and writes the
+    tensors it is given.  `forward(X)` = hq_quantize_act + hq_linear."""
+
+    def __init__(self, desc: LayerDesc, W, bias=None, act_absmax=None, alpha=0.5, device=None):
+        import torch
+        self.desc = desc
+        dev = W.device if device is None else device
+        K, N = desc.K, desc.N
+        self.w_codes = torch.empty((N, K), dtype=torch.int8, device=dev)
+        self.w_scale = torch.empty(N, dtype=torch.float32, device=dev)
+        self.colsum = torch.empty(N, dtype=torch.float32, device=dev)
+        self.sigma_inv = torch.empty(K, dtype=torch.float32, device=dev)
+        self.bias_f32 = torch.empty(N, dtype=torch.float32, device=dev)
+        self.use_sigma = act_absmax is not None
+        hq_prepare_weights(desc, W, bias, act_absmax, alpha, self.w_codes, self.w_scale,
+                           self.colsum, self.sigma_inv, self.bias_f32)
+        ws = hq_quantize_act_workspace_bytes(desc, 0)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev) if ws else None
+        self._bufs = {}
+
+    def buffers(self, T: int):
+        import torch
+        b = self._bufs.get(T)
+        if b is None:
+            dev = self.w_codes.device
+            per_row = self.desc.act_gran == HQ_PER_TOKEN
+            b = {"a_codes": torch.empty((T, self.desc.K), dtype=torch.int8, device=dev),
+                 "a_scale": torch.empty(T if per_row else 1, dtype=torch.float32, device=dev),
+                 "a_mean": torch.empty(T, dtype=torch.float32, device=dev)}
+            self._bufs[T] = b
+        return b
+
+    def quantize(self, X):
+        b = self.buffers(X.shape[0])
+        hq_quantize_act(self.desc, X, self.sigma_inv if self.use_sigma else None, b["a_codes"],
+                        b["a_scale"], b["a_mean"], self.workspace)
+        return b
+
+    def forward(self, X, Y=None, acc_debug=None):
+        import torch
+        T = X.shape[0]
+        if Y is None:
+            Y = torch.empty((T, self.desc.N), dtype=torch.bfloat16, device=X.device)
+        b = self.quantize(X)
+        mean = b["a_mean"] if self.desc.centering == HQ_CENTER_TOKEN_MEAN else None
+        hq_linear(self.desc, b["a_codes"], b["a_scale"], mean, self.w_codes, self.w_scale,
+                  self.colsum, self.bias_f32, Y, acc_debug)
+        return Y
+
+    __call__ = forward

@@ -1,0 +1,437 @@
+// hq_api.cu -- host side of the C ABI declared in include/hq.h: argument
+// checks, launch configuration, tensor-map encoding, and the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/hq.h"
+#include "hq_kernels.h"
+
+namespace hq {
+
+// The device error word (one per device that loads the library).
+__device__ unsigned int g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kVersion = 10000;  // 1.0.0
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+  bool ready = false;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  unsigned int* err = nullptr;
+  bool quant_attr_set[8][4][2] = {};
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+unsigned long long g_wait_ns = 0;  // 0 -> default
+int g_fault = 0;
+
+unsigned long long wait_ns() { return g_wait_ns ? g_wait_ns : 2000000000ull; }
+
+hq_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return HQ_ERR_CUDA;
+    d.cc_major = prop.major;
+    d.cc_minor = prop.minor;
+    d.sm_count = prop.multiProcessorCount;
+    if (prop.major != 10) return HQ_ERR_DEVICE;  // sm_100a code only
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_error_word) != cudaSuccess) return HQ_ERR_CUDA;
+    d.err = static_cast<unsigned int*>(addr);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return HQ_ERR_DEVICE;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return HQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int ilog2_exact(int n) {
+  if (n <= 0 || (n & (n - 1)) != 0) return -1;
+  int l = 0;
+  while ((1 << l) < n) ++l;
+  return l;
+}
+
+// Shape rules shared by the quantizer entry points (K side only).
+hq_status check_k_side(const hq_layer_desc* d) {
+  const int logn = ilog2_exact(d->had_order);
+  if (d->K <= 0 || d->had_order <= 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (logn < 4 || logn > 10) return HQ_ERR_UNSUPPORTED;
+  if (d->K % d->had_order != 0 || d->K % 32 != 0 || d->K > 12288) return HQ_ERR_UNSUPPORTED;
+  if (d->code_format != HQ_CODES_I8) return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+
+hq_status check_desc(const hq_layer_desc* d) {
+  if (d == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  if (d->N <= 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (d->act_gran < HQ_PER_TOKEN || d->act_gran > HQ_PER_TENSOR_STATIC) return HQ_ERR_INVALID_ARGUMENT;
+  if (d->centering < HQ_CENTER_NONE || d->centering > HQ_CENTER_TOKEN_MEAN)
+    return HQ_ERR_INVALID_ARGUMENT;
+  hq_status s = check_k_side(d);
+  if (s != HQ_OK) return s;
+  if (d->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (d->a_bits != 3 && d->a_bits != 4 && d->a_bits != 8) return HQ_ERR_UNSUPPORTED;
+  if (d->w_bits != 4 && d->w_bits != 8) return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+
+hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+
+// Rows per tile R and threads per CTA for the row quantizer: every thread owns
+// a 32-channel slice of one row; prefer full warps and 256..384 threads.
+void quant_shape(int K, int* R_out, int* nt_out) {
+  const int S = K / 32;
+  const int maxT = quant_max_threads();
+  int bestR = 1, bestNT = ((S + 31) / 32) * 32;
+  double bestScore = -1.0;
+  for (int R = 1; R * S <= maxT; ++R) {
+    const int nt = ((R * S + 31) / 32) * 32;
+    if (nt > maxT) break;
+    const double util = double(R * S) / nt;
+    const double size_pref = nt >= 256 ? 1.0 : double(nt) / 256.0;
+    const double score = util * 4.0 + size_pref;
+    if (score > bestScore + 1e-9) {
+      bestScore = score;
+      bestR = R;
+      bestNT = nt;
+    }
+  }
+  *R_out = bestR;
+  *nt_out = bestNT;
+}
+
+struct QuantLaunch {
+  QuantParams p;
+  int threads;
+  size_t smem;
+  int grid;
+};
+
+QuantLaunch make_quant_launch(const DeviceState* dev, int K, int n, int64_t T) {
+  QuantLaunch L;
+  std::memset(&L.p, 0, sizeof(L.p));
+  int R, nt;
+  quant_shape(K, &R, &nt);
+  const int S = K / 32;
+  const int TT = n >= 32 ? n / 32 : 1;
+  const int E = S / TT;
+  const uint32_t raw = uint32_t(R) * uint32_t(K) * 2u;
+  const uint32_t tile_bytes = (raw + 1023u) & ~1023u;
+  int nstage = int((160u * 1024u) / tile_bytes);
+  if (nstage > 8) nstage = 8;
+  if (nstage < 2) nstage = 2;
+  L.p.T = T;
+  L.p.K = K;
+  L.p.S = S;
+  L.p.R = R;
+  L.p.nstage = nstage;
+  L.p.tile_bytes = tile_bytes;
+  L.p.inv_sqrt_n = float(1.0 / std::sqrt(double(n)));
+  L.p.sqrt_n = float(std::sqrt(double(n)));
+  L.p.err = dev->err;
+  L.p.wait_ns = wait_ns();
+  L.threads = nt;
+  // stages | barriers | pad to 16 | per-block partials | per-row stats | flags
+  L.smem = size_t(nstage) * tile_bytes + 8u * nstage + 16u + 16u * size_t(R) * E + 8u * R + 16u;
+  const int64_t ntiles = (T + R - 1) / R;
+  L.grid = int(ntiles < dev->sm_count ? ntiles : dev->sm_count);
+  return L;
+}
+
+hq_status run_quant(DeviceState* dev, const QuantLaunch& L, int logn, int mode, bool center,
+                    cudaStream_t st) {
+  const void* fn = quant_kernel_ptr(logn, mode, center);
+  if (fn == nullptr) return HQ_ERR_UNSUPPORTED;
+  if (L.p.T <= 0) return HQ_OK;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    bool& set = dev->quant_attr_set[logn - 4 < 0 ? 0 : logn - 4][mode][center ? 1 : 0];
+    if (!set) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+          cudaSuccess)
+        return HQ_ERR_CUDA;
+      set = true;
+    }
+  }
+  QuantParams p = L.p;
+  void* args[] = {&p};
+  return from_cuda(cudaLaunchKernel(fn, dim3(L.grid), dim3(L.threads), args, L.smem, st));
+}
+
+hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+  cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(K)};
+  cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
+int choose_bn(int64_t T, int N, int sms) {
+  static const int cands[] = {256, 192, 160, 128, 64};
+  const int64_t mt = (T + 127) / 128;
+  int best = 64;
+  double best_cost = 1e300;
+  for (int bn : cands) {
+    const int64_t nt = (N + bn - 1) / bn;
+    const int64_t tiles = mt * nt;
+    const int64_t waves = (tiles + sms - 1) / sms;
+    const double cost = double(waves) * double(bn + 32);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+}  // namespace
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" {
+
+const char* hq_status_string(hq_status s) {
+  switch (s) {
+    case HQ_OK: return "HQ_OK";
+    case HQ_ERR_INVALID_ARGUMENT: return "HQ_ERR_INVALID_ARGUMENT";
+    case HQ_ERR_UNSUPPORTED: return "HQ_ERR_UNSUPPORTED";
+    case HQ_ERR_MISALIGNED: return "HQ_ERR_MISALIGNED";
+    case HQ_ERR_CUDA: return "HQ_ERR_CUDA";
+    case HQ_ERR_TIMEOUT: return "HQ_ERR_TIMEOUT";
+    case HQ_ERR_DEVICE: return "HQ_ERR_DEVICE";
+    default: return "HQ_ERR_UNKNOWN";
+  }
+}
+
+int hq_version(void) { return kVersion; }
+
+hq_status hq_calib_act_absmax(const hq_layer_desc* desc, const uint16_t* X, int64_t T,
+                              float* absmax, hq_stream_t stream) {
+  if (desc == nullptr || T < 0 || desc->K <= 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->K % 8 != 0) return HQ_ERR_UNSUPPORTED;
+  if (T == 0) return HQ_OK;
+  if (X == nullptr || absmax == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(X) || !aligned4(absmax)) return HQ_ERR_MISALIGNED;
+  DeviceState* dev;
+  hq_status s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  return from_cuda(launch_col_absmax(X, T, desc->K, absmax, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const uint16_t* bias,
+                             const float* act_absmax, float alpha, int8_t* w_codes, float* w_scale,
+                             float* colsum, float* sigma_inv, float* bias_f32, hq_stream_t stream) {
+  hq_status s = check_desc(desc);
+  if (s != HQ_OK) return s;
+  if (W == nullptr || w_codes == nullptr || w_scale == nullptr || colsum == nullptr ||
+      sigma_inv == nullptr || bias_f32 == nullptr)
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(W) || !aligned16(w_codes) || !aligned16(sigma_inv) || !aligned4(w_scale) ||
+      !aligned4(colsum) || !aligned4(bias_f32) || (bias && !aligned4(bias)) ||
+      (act_absmax && !aligned4(act_absmax)))
+    return HQ_ERR_MISALIGNED;
+  DeviceState* dev;
+  s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int K = desc->K, N = desc->N;
+  // sigma^-1 (HadaNorm review Eq. (3)); sigma_inv first holds max_n |W[n,k]|
+  if (act_absmax) {
+    if (cudaMemsetAsync(sigma_inv, 0, sizeof(float) * size_t(K), st) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    s = from_cuda(launch_col_absmax(W, N, K, sigma_inv, st));
+    if (s != HQ_OK) return s;
+    s = from_cuda(launch_sigma_inv(act_absmax, sigma_inv, K, alpha, st));
+  } else {
+    s = from_cuda(launch_fill(sigma_inv, K, 1.0f, st));
+  }
+  if (s != HQ_OK) return s;
+  // W~ rows: multiply by sigma (= 1 / sigma_inv), rotate, quantize per row,
+  // and record each row's sum (colsum of W~ in the pages' orientation)
+  QuantLaunch L = make_quant_launch(dev, K, desc->had_order, N);
+  L.p.X = W;
+  L.p.mult = act_absmax ? sigma_inv : nullptr;
+  L.p.invert_mult = 1;
+  L.p.codes = w_codes;
+  L.p.scale = w_scale;
+  L.p.mean = nullptr;
+  L.p.rowsum = colsum;
+  L.p.q = (1 << (desc->w_bits - 1)) - 1;
+  s = run_quant(dev, L, ilog2_exact(desc->had_order), 0, false, st);
+  if (s != HQ_OK) return s;
+  if (bias) return from_cuda(launch_bf16_to_f32(bias, bias_f32, N, st));
+  return from_cuda(launch_fill(bias_f32, N, 0.0f, st));
+}
+
+size_t hq_quantize_act_workspace_bytes(const hq_layer_desc* desc, int64_t T) {
+  (void)T;
+  if (desc == nullptr) return 0;
+  return desc->act_gran == HQ_PER_TENSOR_DYNAMIC ? 16 : 0;
+}
+
+hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t T,
+                          const float* sigma_inv, int8_t* a_codes, float* a_scale, float* a_mean,
+                          void* workspace, size_t workspace_bytes, hq_stream_t stream) {
+  hq_status s = check_desc(desc);
+  if (s != HQ_OK) return s;
+  if (T < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (X == nullptr || a_codes == nullptr || a_scale == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  const bool dyn = desc->act_gran == HQ_PER_TENSOR_DYNAMIC;
+  if (dyn && (workspace == nullptr || workspace_bytes < 16)) return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(X) || !aligned16(a_codes) || !aligned4(a_scale) || (a_mean && !aligned4(a_mean)) ||
+      (sigma_inv && !aligned16(sigma_inv)) || (dyn && !aligned16(workspace)))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceState* dev;
+  s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  QuantLaunch L = make_quant_launch(dev, desc->K, desc->had_order, T);
+  L.p.X = X;
+  L.p.mult = sigma_inv;
+  L.p.invert_mult = 0;
+  L.p.codes = a_codes;
+  L.p.scale = a_scale;
+  L.p.mean = a_mean;
+  L.p.rowsum = nullptr;
+  L.p.q = (1 << (desc->a_bits - 1)) - 1;
+  L.p.fault_skip_load = g_fault == HQ_FAULT_QUANT_WITHHOLD_LOAD ? 1 : 0;
+  const int logn = ilog2_exact(desc->had_order);
+  const bool center = desc->centering == HQ_CENTER_TOKEN_MEAN;
+  if (desc->act_gran == HQ_PER_TOKEN) return run_quant(dev, L, logn, 0, center, st);
+  if (desc->act_gran == HQ_PER_TENSOR_STATIC) {
+    L.p.static_scale = a_scale;
+    L.p.scale = nullptr;
+    return run_quant(dev, L, logn, 3, center, st);
+  }
+  // dynamic per tensor: pass 1 finds max |V| over the tensor, pass 2 quantizes
+  L.p.tensor_max = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, 16, st) != cudaSuccess) return HQ_ERR_CUDA;
+  QuantLaunch L1 = L;
+  L1.p.codes = nullptr;
+  L1.p.mean = nullptr;
+  L1.p.fault_skip_load = 0;
+  s = run_quant(dev, L1, logn, 1, center, st);
+  if (s != HQ_OK) return s;
+  return run_quant(dev, L, logn, 2, center, st);
+}
+
+hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
+                    const float* a_scale, const float* a_mean, const int8_t* w_codes,
+                    const float* w_scale, const float* colsum, const float* bias_f32, uint16_t* Y,
+                    int32_t* acc_debug, hq_stream_t stream) {
+  if (desc == nullptr || T < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->K <= 0 || desc->N <= 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->act_gran < HQ_PER_TOKEN || desc->act_gran > HQ_PER_TENSOR_STATIC)
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (a_codes == nullptr || a_scale == nullptr || w_codes == nullptr || w_scale == nullptr ||
+      Y == nullptr)
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (a_mean != nullptr && colsum == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(Y) || !aligned16(w_scale) ||
+      (colsum && !aligned16(colsum)) || (bias_f32 && !aligned16(bias_f32)) || !aligned4(a_scale) ||
+      (a_mean && !aligned4(a_mean)) || (acc_debug && !aligned16(acc_debug)))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceState* dev;
+  hq_status s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  const int K = desc->K, N = desc->N;
+  const int bn = choose_bn(T, N, dev->sm_count);
+  CUtensorMap ta, tb;
+  s = encode_kmajor_i8(&ta, a_codes, T, K, 128);
+  if (s != HQ_OK) return s;
+  s = encode_kmajor_i8(&tb, w_codes, N, K, bn);
+  if (s != HQ_OK) return s;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.a_scale = a_scale;
+  p.a_scale_per_row = desc->act_gran == HQ_PER_TOKEN ? 1 : 0;
+  p.a_mean = a_mean;
+  p.w_scale = w_scale;
+  p.colsum = colsum;
+  p.bias = bias_f32;
+  p.Y = Y;
+  p.acc_debug = acc_debug;
+  p.T = T;
+  p.N = N;
+  p.K = K;
+  p.num_m_tiles = int((T + 127) / 128);
+  p.num_n_tiles = (N + bn - 1) / bn;
+  p.err = dev->err;
+  p.wait_ns = wait_ns();
+  const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
+  const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
+  return from_cuda(launch_gemm(bn, &ta, &tb, p, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hq_status hq_check_device_error(hq_stream_t stream) {
+  DeviceState* dev;
+  hq_status s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, dev->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return HQ_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpy(dev->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    return static_cast<hq_status>(word);
+  }
+  return HQ_OK;
+}
+
+hq_status hq_debug_set_wait_limit(uint64_t nanoseconds) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_wait_ns = nanoseconds;
+  return HQ_OK;
+}
+
+hq_status hq_debug_inject_fault(int kind) {
+  if (kind != HQ_FAULT_NONE && kind != HQ_FAULT_QUANT_WITHHOLD_LOAD) return HQ_ERR_INVALID_ARGUMENT;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_fault = kind;
+  return HQ_OK;
+}
+
+}  // extern "C"

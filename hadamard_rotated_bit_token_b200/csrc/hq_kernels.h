@@ -1,0 +1,69 @@
+// hq_kernels.h -- kernel parameter blocks and launch helpers shared between
+// the kernels (.cu) and the host-side C ABI (hq_api.cu).  Internal header.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace hq {
+
+struct QuantParams {
+  const uint16_t* X;          // [T,K] bf16 rows to transform
+  const float* mult;          // [K] channel multiplier (sigma^-1 or sigma), or null
+  int invert_mult;            // 1: use 1/mult[k] as the multiplier
+  int8_t* codes;              // [T,K] int8 codes
+  float* scale;               // [T] per-row scales, or [1] for per-tensor modes
+  float* mean;                // [T] per-row mean of the rotated row (real units), or null
+  float* rowsum;              // [T] per-row sum of the rotated row (real units), or null
+  unsigned int* tensor_max;   // per-tensor: bits of max |V_hat| (unnormalized)
+  const float* static_scale;  // per-tensor static scale (real units)
+  int64_t T;
+  int K;
+  int S;                      // 32-channel slices per row (K / 32)
+  int R;                      // rows per tile
+  int q;                      // 2^(bits-1) - 1
+  int nstage;                 // shared-memory stages
+  uint32_t tile_bytes;        // bytes per stage (R*K*2 rounded up to 1024)
+  float inv_sqrt_n;           // 1 / sqrt(n), fp32
+  float sqrt_n;               // sqrt(n), fp32
+  int fault_skip_load;        // test hook: withhold the first tile load
+  unsigned int* err;          // device error word
+  unsigned long long wait_ns; // bounded-wait limit
+};
+
+// Returns the kernel entry for log2(n) in [4,10], mode in [0,3].
+const void* quant_kernel_ptr(int logn, int mode, bool center);
+int quant_max_threads();
+
+struct GemmParams {
+  const float* a_scale;   // [T] or [1]
+  int a_scale_per_row;    // 1: a_scale[t]; 0: a_scale[0]
+  const float* a_mean;    // [T] or null
+  const float* w_scale;   // [N]
+  const float* colsum;    // [N] or null
+  const float* bias;      // [N] or null
+  uint16_t* Y;            // [T,N] bf16
+  int32_t* acc_debug;     // [T,N] or null
+  int64_t T;
+  int N;
+  int K;
+  int num_m_tiles;
+  int num_n_tiles;
+  unsigned int* err;          // device error word
+  unsigned long long wait_ns; // bounded-wait limit
+};
+
+// Launches the tcgen05 GEMM for N tile width bn (64, 128, 160, 192 or 256).
+// tmap_a / tmap_b point to host CUtensorMap objects (copied into the launch).
+cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const GemmParams& p,
+                        int grid, cudaStream_t st);
+size_t gemm_smem_bytes(int bn);
+int gemm_threads();
+
+cudaError_t launch_col_absmax(const uint16_t* M, int64_t rows, int K, float* out, cudaStream_t st);
+cudaError_t launch_sigma_inv(const float* act_absmax, float* sigma_inv, int K, float alpha,
+                             cudaStream_t st);
+cudaError_t launch_fill(float* p, int n, float v, cudaStream_t st);
+cudaError_t launch_bf16_to_f32(const uint16_t* in, float* out, int n, cudaStream_t st);
+
+}  // namespace hq

@@ -1,0 +1,189 @@
+/*
+ * hq.h -- C ABI of the B200 (sm_100a) Hadamard-domain quantized linear layer.
+ *
+ * The layer is the HadaNorm identity (HadaNorm review, "What carries the
+ * argument", Eq. (1)):
+ *
+ *     X W + b = X~ W~ + b~,   X~ = X diag(sigma^-1) H - mu,
+ *                             W~ = H^T diag(sigma) W,  b~ = b + mu W~,
+ *
+ * with sigma_i = max|X_i|^alpha / max|W_i|^(1-alpha) (same page, Eq. (3)),
+ * mu the per-token mean of the scaled and rotated activations, and H a
+ * block-diagonal Sylvester Hadamard matrix with blocks of order had_order
+ * ("Data-free 4-bit quantization for diffusion transformers", "Hadamard
+ * rotation", step 7; HaTQ supplement Eq. (34)).  X~ is quantized per token
+ * (or per tensor) and W~ per output channel with the symmetric quantizer of
+ * HaTQ Sec. III-A Eq. (3), round half to even, and the product runs as an
+ * int8 x int8 -> int32 tensor-core GEMM whose accumulator has scale
+ * s_x * s_w (HaTQ Sec. IV-B Eq. (18)).
+ *
+ * Memory conventions (all entry points):
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *     library never allocates, frees or retains device memory; it keeps one
+ *     4-byte device error word per device (see hq_check_device_error).
+ *   - Matrices are row-major.  X is [T,K] (tokens x input channels; NHWC
+ *     pixels for a 1x1 convolution), W is [N,K] (output x input channels, the
+ *     nn.Linear orientation, i.e. the transpose of the pages' W), Y is [T,N].
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Pointers to tensors read or written by the tensor-memory engine or by
+ *     16-byte vector accesses must be 16-byte aligned (HQ_ERR_MISALIGNED).
+ *   - All calls are asynchronous on `stream` (NULL = legacy default stream)
+ *     and never synchronize, except hq_check_device_error.
+ *   - Errors are returned, never raised: the library does not abort, exit or
+ *     trap.  Argument checks happen before any launch; a rejected call
+ *     launches nothing.
+ *
+ * Shapes supported:  had_order a power of two in [16, 1024]; K a multiple of
+ * had_order and of 32, K <= 12288; N a multiple of 16; T >= 0 (T = 0 is a
+ * no-op); a_bits in {3, 4, 8}, w_bits in {4, 8} (codes in an int8 container,
+ * one code per byte).
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Compatible with cudaStream_t (struct CUstream_st*). */
+typedef struct CUstream_st* hq_stream_t;
+
+typedef enum hq_status {
+  HQ_OK = 0,
+  HQ_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad enum */
+  HQ_ERR_UNSUPPORTED = 2,      /* shape / bit-width outside the list above */
+  HQ_ERR_MISALIGNED = 3,       /* a tensor pointer is not 16-byte aligned */
+  HQ_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+  HQ_ERR_TIMEOUT = 5,          /* a bounded device-side wait gave up */
+  HQ_ERR_DEVICE = 6            /* the device lacks sm_100a / tensor maps */
+} hq_status;
+
+enum { HQ_PER_TOKEN = 0, HQ_PER_TENSOR_DYNAMIC = 1, HQ_PER_TENSOR_STATIC = 2 };
+enum { HQ_CENTER_NONE = 0, HQ_CENTER_TOKEN_MEAN = 1 };
+enum { HQ_CODES_I8 = 0 };
+
+/* Layer description, host memory, passed by const pointer.
+ *   K, N        input / output channels.
+ *   had_order   Hadamard block order n (H = diag(H_n, ..., H_n), K/n blocks).
+ *   a_bits      activation code width: 4 (int4, [-7,7]), 3 (int3, [-3,3]) or
+ *               8 (int8, [-127,127]); q_a = 2^(a_bits-1) - 1.
+ *   w_bits      weight code width: 4 or 8; q_w = 2^(w_bits-1) - 1.
+ *   act_gran    HQ_PER_TOKEN: one dynamic scale per token.
+ *               HQ_PER_TENSOR_DYNAMIC: one scale from the whole tensor's
+ *               max |X~| (two passes over X).
+ *               HQ_PER_TENSOR_STATIC: one scale given by the caller.
+ *   centering   HQ_CENTER_TOKEN_MEAN: mu_t = mean over all K channels of the
+ *               scaled and rotated token (HadaNorm review Eq. (1)).
+ *               HQ_CENTER_NONE: mu = 0.
+ *   code_format HQ_CODES_I8 (one signed code per byte). */
+typedef struct hq_layer_desc {
+  int32_t K, N, had_order;
+  int32_t a_bits, w_bits;
+  int32_t act_gran;
+  int32_t centering;
+  int32_t code_format;
+} hq_layer_desc;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hq_status_string(hq_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int hq_version(void);
+
+/* hq_calib_act_absmax -- calibration reduction feeding sigma
+ * (HadaNorm review Eq. (3), the max|X_i| term).
+ *   X       bf16 [T,K] device, 16-byte aligned.
+ *   absmax  fp32 [K] device: on return absmax[k] = max(absmax[k], max_t |X[t,k]|),
+ *           so several batches can be accumulated; zero it before the first.
+ * Only desc->K is used (any K that is a multiple of 8).  T = 0 is a no-op. */
+hq_status hq_calib_act_absmax(const hq_layer_desc* desc, const uint16_t* X,
+                              int64_t T, float* absmax, hq_stream_t stream);
+
+/* hq_prepare_weights -- offline weight side of Eq. (1) (HadaNorm review):
+ *   sigma_k   = act_absmax[k]^alpha / max_n|W[n,k]|^(1-alpha)   (Eq. (3));
+ *               sigma_k = 1 when act_absmax == NULL or either max is zero
+ *   sigma_inv = 1 / sigma  (fp32 [K]; feeds hq_quantize_act)
+ *   W~[n,:]   = (W[n,:] * sigma) H    (W~ = H^T diag(sigma) W in the pages'
+ *               orientation), computed with a fast Walsh-Hadamard transform
+ *   colsum[n] = sum_k W~[n,k]          (the mu W~ term of b~)
+ *   w_scale[n]= max_k |W~[n,k]| / q_w,  w_codes = clamp(rne(W~ / w_scale), +-q_w)
+ *   bias_f32  = float(bias), or 0 when bias == NULL.
+ * Inputs:  W bf16 [N,K], bias bf16 [N] or NULL, act_absmax fp32 [K] or NULL.
+ * Outputs: w_codes int8 [N,K], w_scale fp32 [N], colsum fp32 [N],
+ *          sigma_inv fp32 [K], bias_f32 fp32 [N] (all device, caller-owned).
+ * sigma_inv is also used as scratch during the call.  alpha in [0, 1]. */
+hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W,
+                             const uint16_t* bias, const float* act_absmax,
+                             float alpha, int8_t* w_codes, float* w_scale,
+                             float* colsum, float* sigma_inv, float* bias_f32,
+                             hq_stream_t stream);
+
+/* Bytes of device workspace hq_quantize_act needs for this description
+ * (16 for HQ_PER_TENSOR_DYNAMIC, 0 otherwise). */
+size_t hq_quantize_act_workspace_bytes(const hq_layer_desc* desc, int64_t T);
+
+/* hq_quantize_act -- runtime activation side of Eq. (1), fused in one pass
+ * over X (two for HQ_PER_TENSOR_DYNAMIC):
+ *   Y = X diag(sigma^-1); Z = Y H (block fast Walsh-Hadamard transform);
+ *   m_t = mean_k Z[t,k] (HQ_CENTER_TOKEN_MEAN) else 0;  V = Z - m;
+ *   s = max|V| / q_a per token (or per tensor);  codes = clamp(rne(V/s), +-q_a).
+ * Inputs:  X bf16 [T,K]; sigma_inv fp32 [K] or NULL (sigma = 1).
+ * Outputs: a_codes int8 [T,K];
+ *          a_scale fp32 [T] (HQ_PER_TOKEN) or [1] (per tensor; for
+ *            HQ_PER_TENSOR_STATIC it is an INPUT holding s);
+ *          a_mean fp32 [T] or NULL (written with zeros when centering is off).
+ * workspace: device, >= hq_quantize_act_workspace_bytes(), 16-byte aligned,
+ *   contents need not be initialised (the call clears what it uses).
+ * A token whose max|V| is 0 gets scale 0 and all-zero codes. */
+hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X,
+                          int64_t T, const float* sigma_inv, int8_t* a_codes,
+                          float* a_scale, float* a_mean, void* workspace,
+                          size_t workspace_bytes, hq_stream_t stream);
+
+/* hq_linear -- integer GEMM and epilogue (HaTQ Eq. (18); HadaNorm Eq. (1)):
+ *   acc[t,n] = sum_k a_codes[t,k] * w_codes[n,k]            (int32, exact)
+ *   Y[t,n]   = bf16_rne( s_x[t] * w_scale[n] * acc[t,n]
+ *                        + bias_f32[n] + a_mean[t] * colsum[n] )
+ * on 5th-generation tensor cores (tcgen05 kind::i8, accumulator in TMEM).
+ * Inputs:  a_codes int8 [T,K], a_scale fp32 [T] or [1] (per tensor, selected
+ *          by desc->act_gran), a_mean fp32 [T] or NULL (then mu = 0),
+ *          w_codes int8 [N,K], w_scale fp32 [N], colsum fp32 [N] (may be NULL
+ *          when a_mean is NULL), bias_f32 fp32 [N] or NULL (b = 0).
+ * Outputs: Y bf16 [T,N]; acc_debug int32 [T,N] or NULL (raw accumulators, for
+ *          bit-exact checks; costs an extra 4 bytes per output).
+ * The codes may hold any int8 values (the GEMM is generic int8). */
+hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
+                    const float* a_scale, const float* a_mean,
+                    const int8_t* w_codes, const float* w_scale,
+                    const float* colsum, const float* bias_f32, uint16_t* Y,
+                    int32_t* acc_debug, hq_stream_t stream);
+
+/* hq_check_device_error -- synchronizes `stream`, then reads and clears the
+ * current device's error word, which kernels set instead of trapping when a
+ * bounded wait gives up (HQ_ERR_TIMEOUT).  Returns HQ_ERR_CUDA if the stream
+ * itself reports an error. */
+hq_status hq_check_device_error(hq_stream_t stream);
+
+/* Test hook: sets the time in nanoseconds after which every bounded device
+ * wait gives up (0 restores the default of 2 s).  Host state, applies to
+ * launches issued after the call. */
+hq_status hq_debug_set_wait_limit(uint64_t nanoseconds);
+
+/* Test hook for the bounded-wait error path, without faulting the GPU:
+ *   HQ_FAULT_NONE (0)                    normal operation;
+ *   HQ_FAULT_QUANT_WITHHOLD_LOAD (1)     each CTA of the next activation
+ *       quantize launches skips its first tile copy, so the barrier it waits
+ *       on never completes; the bounded wait expires, the kernel records
+ *       HQ_ERR_TIMEOUT, lets its other copies land and exits.
+ * Host state, applies to launches issued after the call. */
+enum { HQ_FAULT_NONE = 0, HQ_FAULT_QUANT_WITHHOLD_LOAD = 1 };
+hq_status hq_debug_inject_fault(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads,
+exports every entry point include/hq.h declares, and rejects bad arguments
+with the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hq():
+    from hadamard_rotated_bit_token_b200 import build as hq_build
+    hq_build.build()
+    import hadamard_rotated_bit_token_b200 as hq_mod
+    hq_mod.load_library()
+    return hq_mod
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "hq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(hq):
+    names = declared_functions()
+    assert "hq_quantize_act" in names and "hq_linear" in names and "hq_prepare_weights" in names
+    lib = hq.load_library()
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(hq.EXPORTED) >= set(names)
+
+
+def test_version_and_status_strings(hq):
+    assert hq.hq_version() == 10000
+    for code, name in hq.STATUS_NAMES.items():
+        assert hq.hq_status_string(code) == name
+    assert hq.hq_status_string(99) == "HQ_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def _call_quant(hq, desc, X=FAKE, T=4, codes=FAKE, scale=FAKE, ws=None, ws_bytes=0):
+    lib = hq.load_library()
+    d = None if desc is None else ctypes.byref(desc)
+    return lib.hq_quantize_act(d, X, T, None, codes, scale, None, ws, ws_bytes, None)
+
+
+def test_quantize_validation(hq):
+    D = hq.LayerDesc
+    assert _call_quant(hq, None) == 1
+    assert _call_quant(hq, D(1024, 16, 1024), X=None) == 1
+    assert _call_quant(hq, D(1024, 16, 1024), T=-1) == 1
+    assert _call_quant(hq, D(1024, 16, 1000)) == 2          # order not a power of two
+    assert _call_quant(hq, D(1024, 16, 2048)) == 2          # order above 1024
+    assert _call_quant(hq, D(1024, 16, 8)) == 2             # order below 16
+    assert _call_quant(hq, D(1000, 16, 8)) == 2
+    assert _call_quant(hq, D(96, 16, 64)) == 2              # K not a multiple of the order
+    assert _call_quant(hq, D(16384, 16, 1024)) == 2         # K above the limit
+    assert _call_quant(hq, D(1024, 15, 1024)) == 2          # N not a multiple of 16
+    assert _call_quant(hq, D(1024, 16, 1024, a_bits=5)) == 2
+    assert _call_quant(hq, D(1024, 16, 1024, w_bits=3)) == 2
+    assert _call_quant(hq, D(1024, 16, 1024, act_gran=7)) == 1
+    assert _call_quant(hq, D(1024, 16, 1024, centering=2)) == 1
+    assert _call_quant(hq, D(1024, 16, 1024, code_format=1)) == 2
+    assert _call_quant(hq, D(1024, 16, 1024), X=FAKE + 2) == 3   # misaligned
+    assert _call_quant(hq, D(1024, 16, 1024), codes=FAKE + 8) == 3
+    # per-tensor dynamic needs its workspace
+    assert _call_quant(hq, D(1024, 16, 1024, act_gran=1)) == 1
+    assert _call_quant(hq, D(1024, 16, 1024, act_gran=1), ws=FAKE + 4, ws_bytes=16) == 3
+    # T = 0 with valid arguments is a no-op that never touches the device
+    assert _call_quant(hq, D(1024, 16, 1024), T=0) == 0
+
+
+def test_workspace_bytes(hq):
+    lib = hq.load_library()
+    assert lib.hq_quantize_act_workspace_bytes(ctypes.byref(hq.LayerDesc(64, 16, 64)), 10) == 0
+    d = hq.LayerDesc(64, 16, 64, act_gran=hq.HQ_PER_TENSOR_DYNAMIC)
+    assert lib.hq_quantize_act_workspace_bytes(ctypes.byref(d), 10) == 16
+
+
+def test_linear_validation(hq):
+    lib = hq.load_library()
+    D = hq.LayerDesc
+
+    def call(desc, T=8, a=FAKE, sx=FAKE, m=None, w=FAKE, sw=FAKE, cs=None, b=None, y=FAKE, acc=None):
+        d = None if desc is None else ctypes.byref(desc)
+        return lib.hq_linear(d, T, a, sx, m, w, sw, cs, b, y, acc, None)
+
+    assert call(None) == 1
+    assert call(D(1024, 16, 1024), T=-3) == 1
+    assert call(D(1024, 16, 1024), a=None) == 1
+    assert call(D(1024, 16, 1024), m=FAKE) == 1            # mean without colsum
+    assert call(D(1000, 16, 8)) == 2                       # K not a multiple of 16
+    assert call(D(1024, 24, 1024)) == 2                    # N not a multiple of 16
+    assert call(D(1024, 16, 1024), y=FAKE + 2) == 3
+    assert call(D(1024, 16, 1024), sw=FAKE + 4) == 3
+    assert call(D(1024, 16, 1024), T=0) == 0
+
+
+def test_prepare_and_calib_validation(hq):
+    lib = hq.load_library()
+    D = hq.LayerDesc
+    d = D(1024, 16, 1024)
+    assert lib.hq_prepare_weights(ctypes.byref(d), None, None, None, 0.5, FAKE, FAKE, FAKE, FAKE,
+                                  FAKE, None) == 1
+    assert lib.hq_prepare_weights(ctypes.byref(d), FAKE, None, None, 1.5, FAKE, FAKE, FAKE, FAKE,
+                                  FAKE, None) == 1
+    assert lib.hq_prepare_weights(ctypes.byref(d), FAKE + 2, None, None, 0.5, FAKE, FAKE, FAKE,
+                                  FAKE, FAKE, None) == 3
+    assert lib.hq_calib_act_absmax(None, FAKE, 4, FAKE, None) == 1
+    assert lib.hq_calib_act_absmax(ctypes.byref(D(100, 16, 16)), FAKE, 4, FAKE, None) == 2
+    assert lib.hq_calib_act_absmax(ctypes.byref(d), FAKE, 0, FAKE, None) == 0
+    assert lib.hq_debug_inject_fault(9) == 1
+    assert lib.hq_debug_inject_fault(0) == 0
+    assert lib.hq_debug_set_wait_limit(0) == 0
+
+
+def test_binding_rejects_host_tensors(hq):
+    torch = pytest.importorskip("torch")
+    d = hq.LayerDesc(64, 16, 64)
+    with pytest.raises(ValueError):
+        hq.hq_quantize_act(d, torch.zeros((2, 64), dtype=torch.bfloat16), None,
+                           torch.zeros((2, 64), dtype=torch.int8), torch.zeros(2), None, None,
+                           stream=0)
+
+
+def test_library_has_no_cpu_fallback():
+    """The product package neither imports nor runs the oracle."""
+    pkg = os.path.join(ROOT, "hadamard_rotated_bit_token_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "hq_oracle" not in text and "liboracle" not in text, f

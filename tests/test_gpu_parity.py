@@ -1,0 +1,389 @@
+"""GPU parity: the sm_100a kernels (through the C ABI) against the CPU oracle,
+element by element on the same seeded inputs.  Needs a B200."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import (CODE_MATCH_MIN, SCALE_RTOL, TIE_TOL, Y_REL_FROB, bf16_bits, check_codes,
+                    check_rel, rel_frob, to_dev_u16)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def hq():
+    import hadamard_rotated_bit_token_b200 as hq_mod
+    from hadamard_rotated_bit_token_b200 import build as hq_build
+    hq_build.build()
+    hq_mod.load_library()
+    return hq_mod
+
+
+def _sigma_case(K, seed):
+    g = np.random.default_rng(seed)
+    return 10.0 ** g.uniform(-0.7, 0.7, size=K)
+
+
+def _gpu_quantize(hq, desc, X_bits, sigma_inv_f32=None, static_scale=None):
+    T, K = X_bits.shape
+    X = to_dev_u16(X_bits, torch)
+    codes = torch.full((T, K), 0x55, dtype=torch.int8, device="cuda")  # poison
+    per_row = desc.act_gran == hq.HQ_PER_TOKEN
+    scale = torch.full((T if per_row else 1,), float("nan"), dtype=torch.float32, device="cuda")
+    if static_scale is not None:
+        scale.fill_(static_scale)
+    mean = torch.full((T,), float("nan"), dtype=torch.float32, device="cuda")
+    si = None if sigma_inv_f32 is None else torch.from_numpy(sigma_inv_f32).cuda()
+    ws_bytes = hq.hq_quantize_act_workspace_bytes(desc, T)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda") if ws_bytes else None
+    hq.hq_quantize_act(desc, X, si, codes, scale, mean, ws)
+    assert hq.hq_check_device_error() == 0
+    return codes.cpu().numpy(), scale.cpu().numpy().astype(np.float64), mean.cpu().numpy()
+
+
+def _check_act(ref, codes, scale, mean, per_row=True, min_match=None, what="act"):
+    check_codes(codes, ref["codes"], ref["tie"], what + " codes", min_match=min_match)
+    if per_row:
+        check_rel(scale, ref["scale"], SCALE_RTOL, what + " scale")
+    else:
+        check_rel(scale[:1], ref["scale"][:1], SCALE_RTOL, what + " tensor scale")
+    if ref["Z"] is not None:
+        tol = 1e-6 * np.mean(np.abs(ref["Z"]), axis=1) + 1e-30
+        assert np.all(np.abs(mean - ref["mean"]) <= tol), what + " mean"
+
+
+# ---------------------------------------------------------------------------
+# activation quantizer, small shapes spanning several tiles and ragged tails
+# ---------------------------------------------------------------------------
+
+SMALL = []
+for i, (n, B) in enumerate([(16, 2), (16, 6), (32, 1), (32, 5), (64, 1), (64, 5), (128, 1),
+                            (128, 9), (256, 1), (256, 3), (512, 2), (1024, 1), (1024, 3)]):
+    for T in (1, 7, 129, 300):
+        bits = (4, 3, 8)[(i + T) % 3]
+        SMALL.append((n * B, n, T, bits, (i + T) % 2, (i % 3) != 0))
+
+
+@pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL)
+def test_quantize_small(hq, K, n, T, bits, center, use_sigma):
+    g = np.random.default_rng(K * 1000 + T)
+    x = g.standard_normal((T, K)).astype(np.float32)
+    x[:, g.choice(K, size=max(1, K // 64), replace=False)] *= 30.0
+    x += g.standard_normal((T, 1)).astype(np.float32) * 2.0
+    X = synth.f32_to_bf16_bits(x)
+    sigma = _sigma_case(K, T) if use_sigma else None
+    ref = oracle.quantize_act(X, n, bits, gran=0, centering=center, sigma=sigma, want_Z=True)
+    desc = hq.LayerDesc(K, 16, n, a_bits=bits, w_bits=4, act_gran=hq.HQ_PER_TOKEN,
+                        centering=center)
+    si = None if sigma is None else (1.0 / sigma).astype(np.float32)
+    codes, scale, mean = _gpu_quantize(hq, desc, X, si)
+    _check_act(ref, codes, scale, mean)
+    if not center:
+        assert np.all(mean == 0.0)
+
+
+@pytest.mark.parametrize("gran", [1, 2])
+@pytest.mark.parametrize("K,n,T,center", [(320, 64, 300, 0), (256, 256, 129, 1), (1024, 1024, 77, 0)])
+def test_quantize_per_tensor(hq, gran, K, n, T, center):
+    cfg = synth.CONFIGS[4]
+    g = np.random.default_rng(K + T)
+    x = (g.laplace(0, 1, size=(T, K)) * 10.0 ** g.uniform(-1, 1, size=K)).astype(np.float32)
+    X = synth.f32_to_bf16_bits(x)
+    dyn = oracle.quantize_act(X, n, 8, gran=1, centering=center, want_Z=True)
+    desc = hq.LayerDesc(K, 16, n, a_bits=8, w_bits=8, act_gran=gran, centering=center)
+    if gran == 1:
+        codes, scale, mean = _gpu_quantize(hq, desc, X)
+        _check_act(dyn, codes, scale, mean, per_row=False)
+    else:
+        s32 = float(np.float32(dyn["scale"][0] * 0.75))  # a scale that forces clamping
+        ref = oracle.quantize_act(X, n, 8, gran=2, centering=center, static_scale=s32, want_Z=True)
+        codes, scale, mean = _gpu_quantize(hq, desc, X, static_scale=s32)
+        check_codes(codes, ref["codes"], ref["tie"], "static codes")
+        assert np.abs(codes).max() == 127
+    del cfg
+
+
+def test_exact_ties_are_rounded_half_to_even(hq):
+    """Dyadic rows whose centred rotated values sit exactly on rounding ties;
+    both sides compute them exactly, so the codes must agree bit for bit."""
+    n, K, T, bits = 64, 128, 32, 3
+    H = np.ones((1, 1))
+    for _ in range(6):
+        H = np.kron(H, np.array([[1.0, 1.0], [1.0, -1.0]]))
+    Hn = np.kron(np.eye(K // n), H / 8.0)
+    g = np.random.default_rng(7)
+    rows = []
+    for t in range(T):
+        V = np.zeros(K)
+        pos = g.choice(K, size=6, replace=False)
+        vals = [3.0, g.choice([0.5, 1.5, 2.5]), g.choice([0.5, 1.5, 2.5])]
+        for j, v in enumerate(vals):
+            V[pos[2 * j]] = v
+            V[pos[2 * j + 1]] = -v
+        m = [0.0, 0.25, -0.5][t % 3]
+        rows.append((V + m) @ Hn.T)
+    xf = np.array(rows)
+    X = synth.f32_to_bf16_bits(xf.astype(np.float32))
+    assert np.array_equal(synth.bf16_bits_to_f32(X).astype(np.float64), xf)
+    ref = oracle.quantize_act(X, n, bits, gran=0, centering=1, want_Z=True)
+    assert np.sum(ref["tie"] == 0.0) >= 4 * T  # many exact ties
+    desc = hq.LayerDesc(K, 16, n, a_bits=bits, act_gran=hq.HQ_PER_TOKEN, centering=1)
+    codes, scale, mean = _gpu_quantize(hq, desc, X)
+    assert np.array_equal(codes, ref["codes"])
+    assert np.array_equal(scale, ref["scale"])
+
+
+# ---------------------------------------------------------------------------
+# weight preparation
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,n,w_bits,use_sigma",
+                         [(48, 64, 16, 4, True), (160, 256, 64, 8, True), (64, 1152, 128, 4, True),
+                          (32, 3072, 1024, 4, True), (320, 320, 64, 8, False),
+                          (1024, 1024, 1024, 4, True)])
+def test_prepare_weights(hq, N, K, n, w_bits, use_sigma):
+    g = np.random.default_rng(N + K)
+    Xb = synth.f32_to_bf16_bits(g.standard_normal((64, K)).astype(np.float32) *
+                                (1 + 20 * (g.random(K) < 0.02)).astype(np.float32))
+    Wb = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32) * 0.02)
+    bb = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32) * 0.01)
+    sig = oracle.sigma(oracle.col_absmax(Xb), oracle.col_absmax(Wb), 0.5) if use_sigma else None
+    ref = oracle.prepare_weights(Wb, n, w_bits, bias_bits=bb, sigma=sig, want_Wt=True)
+    desc = hq.LayerDesc(K, N, n, a_bits=4, w_bits=w_bits)
+    X = to_dev_u16(Xb, torch)
+    W = to_dev_u16(Wb, torch)
+    b = to_dev_u16(bb, torch)
+    absmax = None
+    if use_sigma:
+        absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
+        hq.hq_calib_act_absmax(desc, X, absmax)
+        assert np.array_equal(absmax.cpu().numpy().astype(np.float64), oracle.col_absmax(Xb))
+    w_codes = torch.full((N, K), 0x55, dtype=torch.int8, device="cuda")
+    w_scale = torch.empty(N, dtype=torch.float32, device="cuda")
+    colsum = torch.empty(N, dtype=torch.float32, device="cuda")
+    sigma_inv = torch.empty(K, dtype=torch.float32, device="cuda")
+    bias_f32 = torch.empty(N, dtype=torch.float32, device="cuda")
+    hq.hq_prepare_weights(desc, W, b, absmax, 0.5, w_codes, w_scale, colsum, sigma_inv, bias_f32)
+    assert hq.hq_check_device_error() == 0
+    if use_sigma:
+        check_rel(sigma_inv.cpu().numpy(), 1.0 / sig, SCALE_RTOL, "sigma_inv")
+    else:
+        assert np.all(sigma_inv.cpu().numpy() == 1.0)
+    check_codes(w_codes.cpu().numpy(), ref["codes"], ref["tie"], "w_codes")
+    check_rel(w_scale.cpu().numpy(), ref["scale"], SCALE_RTOL, "w_scale")
+    tol = 1e-6 * np.abs(ref["Wt"]).sum(axis=1)
+    assert np.all(np.abs(colsum.cpu().numpy() - ref["colsum"]) <= tol), "colsum"
+    assert np.array_equal(bias_f32.cpu().numpy().astype(np.float64), ref["bias"])
+
+
+# ---------------------------------------------------------------------------
+# integer GEMM: bit-exact accumulators, epilogue
+# ---------------------------------------------------------------------------
+
+GEMM_SHAPES = [(1, 16, 32), (127, 48, 160), (128, 192, 128), (129, 320, 320), (300, 512, 1152),
+               (256, 1024, 1024), (200, 3456, 256), (131, 160, 4608), (513, 64, 96)]
+
+
+@pytest.mark.parametrize("T,N,K", GEMM_SHAPES)
+def test_gemm_accumulators_bit_exact(hq, T, N, K):
+    g = np.random.default_rng(T * N + K)
+    A = g.integers(-128, 128, size=(T, K)).astype(np.int8)
+    B = g.integers(-128, 128, size=(N, K)).astype(np.int8)
+    A[0, :] = -128
+    B[0, :] = -128
+    acc_ref = oracle.gemm_acc(A, B)
+    sx = (g.random(T) * 0.1 + 1e-3)
+    sw = (g.random(N) * 0.01 + 1e-4)
+    cs = g.standard_normal(N)
+    bias = g.standard_normal(N) * 0.1
+    mean = g.standard_normal(T)
+    sx32, sw32, cs32, b32, m32 = (v.astype(np.float32) for v in (sx, sw, cs, bias, mean))
+    _, y_ref = oracle.epilogue(acc_ref, sx32.astype(np.float64), sw32.astype(np.float64),
+                               colsum=cs32.astype(np.float64), bias=b32.astype(np.float64),
+                               mean=m32.astype(np.float64))
+    desc = hq.LayerDesc(K, N, 16, act_gran=hq.HQ_PER_TOKEN)
+    d = {k: torch.from_numpy(v).cuda() for k, v in
+         dict(A=A, B=B, sx=sx32, sw=sw32, cs=cs32, b=b32, m=m32).items()}
+    Y = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    acc = torch.full((T, N), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    hq.hq_linear(desc, d["A"], d["sx"], d["m"], d["B"], d["sw"], d["cs"], d["b"], Y, acc)
+    assert hq.hq_check_device_error() == 0
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), acc_ref)
+    err = rel_frob(bf16_bits(Y), y_ref)
+    assert err <= 1e-5, err
+
+
+def test_gemm_worst_case_int4_accumulation(hq):
+    T, N, K = 256, 256, 4608
+    A = np.full((T, K), 7, dtype=np.int8)
+    A[1::2] = -7
+    B = np.full((N, K), 7, dtype=np.int8)
+    B[::3] = -7
+    acc_ref = oracle.gemm_acc(A, B)
+    desc = hq.LayerDesc(K, N, 256, act_gran=hq.HQ_PER_TENSOR_STATIC)
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    sw = torch.ones(N, dtype=torch.float32, device="cuda")
+    Y = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    hq.hq_linear(desc, torch.from_numpy(A).cuda(), one, None, torch.from_numpy(B).cuda(), sw, None,
+                 None, Y, acc)
+    assert hq.hq_check_device_error() == 0
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), acc_ref)
+
+
+# ---------------------------------------------------------------------------
+# whole layer
+# ---------------------------------------------------------------------------
+
+def _gpu_layer(hq, cfg, Xb, Wb, bb):
+    T, K = Xb.shape
+    N = Wb.shape[0]
+    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering)
+    X = to_dev_u16(Xb, torch)
+    W = to_dev_u16(Wb, torch)
+    b = to_dev_u16(bb, torch)
+    absmax = None
+    if cfg.use_sigma:
+        absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
+        hq.hq_calib_act_absmax(desc, X, absmax)
+    layer = hq.HadamardQuantLinear(desc, W, b, absmax, cfg.alpha)
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    Y = layer(X, acc_debug=acc)
+    assert hq.hq_check_device_error() == 0
+    bufs = layer.buffers(T)
+    return layer, bufs, Y, acc
+
+
+def _oracle_layer(cfg, Xb, Wb, bb, rows=None, cols=None):
+    sig = None
+    if cfg.use_sigma:
+        sig = oracle.sigma(oracle.col_absmax(Xb), oracle.col_absmax(Wb), cfg.alpha)
+    Wsel = Wb if cols is None else Wb[cols]
+    bsel = bb if cols is None else bb[cols]
+    w = oracle.prepare_weights(Wsel, cfg.had_order, cfg.w_bits, bias_bits=bsel, sigma=sig)
+    a = oracle.quantize_act(Xb, cfg.had_order, cfg.a_bits, gran=cfg.act_gran,
+                            centering=cfg.centering, sigma=sig, rows=rows, want_Z=True)
+    acc = oracle.gemm_acc(a["codes"], w["codes"])
+    y, yb = oracle.epilogue(acc, a["scale"], w["scale"], colsum=w["colsum"], bias=w["bias"],
+                            mean=a["mean"] if cfg.centering else None)
+    return {"w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb, "sigma": sig}
+
+
+@pytest.mark.parametrize("idx,T", [(1, 300), (2, 257), (3, 130), (4, 1000), (5, 129)])
+def test_layer_reduced_tokens(hq, idx, T):
+    cfg = synth.CONFIGS[idx].with_tokens(T)
+    Xb, Wb, bb = synth.make_layer(cfg)
+    if idx == 5:
+        Wb, bb = Wb[:768], bb[:768]          # keep the CPU oracle quick
+    layer, bufs, Y, acc = _gpu_layer(hq, cfg, Xb, Wb, bb)
+    ref = _oracle_layer(cfg, Xb, Wb, bb)
+    check_codes(bufs["a_codes"].cpu().numpy(), ref["a"]["codes"], ref["a"]["tie"], "a_codes")
+    check_codes(layer.w_codes.cpu().numpy(), ref["w"]["codes"], ref["w"]["tie"], "w_codes")
+    err = rel_frob(bf16_bits(Y), ref["y_bf16"])
+    assert err <= Y_REL_FROB, err
+    # accumulators are exact whenever both sides chose the same codes
+    same = (np.all(bufs["a_codes"].cpu().numpy() == ref["a"]["codes"]) and
+            np.all(layer.w_codes.cpu().numpy() == ref["w"]["codes"]))
+    if same:
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+
+
+def test_centering_off_variant_of_w4a3(hq):
+    cfg = synth.CONFIGS[3].with_tokens(200)
+    import dataclasses
+    cfg = dataclasses.replace(cfg, centering=0)
+    Xb, Wb, bb = synth.make_layer(cfg)
+    layer, bufs, Y, _ = _gpu_layer(hq, cfg, Xb, Wb, bb)
+    ref = _oracle_layer(cfg, Xb, Wb, bb)
+    check_codes(bufs["a_codes"].cpu().numpy(), ref["a"]["codes"], ref["a"]["tie"], "a_codes")
+    assert rel_frob(bf16_bits(Y), ref["y_bf16"]) <= Y_REL_FROB
+
+
+@pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
+def test_layer_full_size_sampled(hq, idx):
+    """Full configuration sizes in the benchmark's launch configuration; the
+    oracle checks a seeded sample of rows (every 128-row tile) and of output
+    channels (every 256-column tile)."""
+    cfg = synth.CONFIGS[idx]
+    Xb, Wb, bb = synth.make_layer(cfg)
+    layer, bufs, Y, acc = _gpu_layer(hq, cfg, Xb, Wb, bb)
+    rows = synth.sample_rows(cfg.T, 512, tile=128, seed=idx)
+    cols = synth.sample_rows(cfg.N, 384, tile=256, seed=100 + idx)
+    ref = _oracle_layer(cfg, Xb, Wb, bb, rows=rows, cols=cols)
+    a_codes = bufs["a_codes"].cpu().numpy()[rows]
+    w_codes = layer.w_codes.cpu().numpy()[cols]
+    check_codes(a_codes, ref["a"]["codes"], ref["a"]["tie"], "a_codes", min_match=CODE_MATCH_MIN)
+    check_codes(w_codes, ref["w"]["codes"], ref["w"]["tie"], "w_codes", min_match=CODE_MATCH_MIN)
+    per_row = cfg.act_gran == 0
+    sc = bufs["a_scale"].cpu().numpy().astype(np.float64)
+    check_rel(sc[rows] if per_row else sc[:1], ref["a"]["scale"] if per_row else ref["a"]["scale"][:1],
+              SCALE_RTOL, "a_scale")
+    Ys = bf16_bits(Y)[np.ix_(rows, cols)]
+    err = rel_frob(Ys, ref["y_bf16"])
+    assert err <= Y_REL_FROB, err
+    acc_s = acc.cpu().numpy()[np.ix_(rows, cols)].astype(np.int64)
+    # exact wherever both the row's and the column's codes agree
+    ra = np.all(a_codes == ref["a"]["codes"], axis=1)
+    ca = np.all(w_codes == ref["w"]["codes"], axis=1)
+    assert np.array_equal(acc_s[np.ix_(ra, ca)], ref["acc"][np.ix_(ra, ca)])
+
+
+def test_gemm_fed_oracle_codes_is_bit_exact(hq):
+    cfg = synth.CONFIGS[2].with_tokens(384)
+    Xb, Wb, bb = synth.make_layer(cfg)
+    ref = _oracle_layer(cfg, Xb, Wb[:512], bb[:512])
+    T, K = Xb.shape
+    N = 512
+    desc = hq.LayerDesc(K, N, cfg.had_order, act_gran=0, centering=1)
+    f32 = lambda v: torch.from_numpy(np.asarray(v, dtype=np.float32)).cuda()
+    Y = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    hq.hq_linear(desc, torch.from_numpy(ref["a"]["codes"]).cuda(), f32(ref["a"]["scale"]),
+                 f32(ref["a"]["mean"]), torch.from_numpy(ref["w"]["codes"]).cuda(),
+                 f32(ref["w"]["scale"]), f32(ref["w"]["colsum"]), f32(ref["w"]["bias"]), Y, acc)
+    assert hq.hq_check_device_error() == 0
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    assert rel_frob(bf16_bits(Y), ref["y_bf16"]) <= 1e-4
+
+
+# ---------------------------------------------------------------------------
+# edge cases and the error path
+# ---------------------------------------------------------------------------
+
+def test_empty_and_zero_rows(hq):
+    desc = hq.LayerDesc(128, 16, 128, a_bits=4)
+    X = torch.zeros((0, 128), dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty((0, 128), dtype=torch.int8, device="cuda")
+    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+    hq.hq_quantize_act(desc, X, None, codes, sc, None, T=0)
+    Xz = np.zeros((5, 128), dtype=np.uint16)
+    Xz[3] = synth.f32_to_bf16_bits(np.linspace(-1, 1, 128).astype(np.float32))
+    codes, scale, mean = _gpu_quantize(hq, desc, Xz)
+    assert np.all(codes[[0, 1, 2, 4]] == 0) and np.all(scale[[0, 1, 2, 4]] == 0)
+    ref = oracle.quantize_act(Xz, 128, 4)
+    assert np.array_equal(codes, ref["codes"])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(hq):
+    desc = hq.LayerDesc(1152, 16, 128, a_bits=4)
+    Xb = synth.make_x(synth.CONFIGS[2].with_tokens(64))
+    hq.hq_debug_set_wait_limit(2_000_000)  # 2 ms
+    hq.hq_debug_inject_fault(hq.HQ_FAULT_QUANT_WITHHOLD_LOAD)
+    try:
+        X = to_dev_u16(Xb, torch)
+        codes = torch.empty((64, 1152), dtype=torch.int8, device="cuda")
+        sc = torch.empty(64, dtype=torch.float32, device="cuda")
+        hq.hq_quantize_act(desc, X, None, codes, sc, None)
+        assert hq.hq_check_device_error() == 5  # HQ_ERR_TIMEOUT
+    finally:
+        hq.hq_debug_inject_fault(hq.HQ_FAULT_NONE)
+        hq.hq_debug_set_wait_limit(0)
+    # the context is still usable and the word was cleared
+    assert hq.hq_check_device_error() == 0
+    codes2, scale2, _ = _gpu_quantize(hq, desc, Xb)
+    ref = oracle.quantize_act(Xb, 128, 4)
+    check_codes(codes2, ref["codes"], ref["tie"], "after timeout")
