@@ -28,7 +28,7 @@ __all__ = [
     "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-    "HadamardQuantLinear",
+    "hq_quantize_act_noalloc", "HadamardQuantLinear",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +43,8 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED
                 6: "HQ_ERR_DEVICE"}
 EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare_weights",
             "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
-            "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault")
+            "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
+            "hq_quantize_act_noalloc")
 
 
 class HQError(RuntimeError):
@@ -97,11 +98,14 @@ def load_library():
                                         ctypes.c_size_t, _vp]
         lib.hq_linear.argtypes = [desc_p, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                   _vp, _vp]
+        lib.hq_quantize_act_noalloc.argtypes = [desc_p, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp,
+                                                _vp]
         lib.hq_check_device_error.argtypes = [_vp]
         lib.hq_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
         lib.hq_debug_inject_fault.argtypes = [ctypes.c_int]
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
-                     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault"):
+                     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
+                     "hq_quantize_act_noalloc"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -188,6 +192,19 @@ def hq_linear(desc: LayerDesc, a_codes, a_scale, a_mean, w_codes, w_scale, colsu
         ctypes.byref(desc), T, _ptr(a_codes), _ptr(a_scale), _ptr(a_mean), _ptr(w_codes),
         _ptr(w_scale), _ptr(colsum), _ptr(bias_f32), _ptr(Y), _ptr(acc_debug), _stream(stream)),
         "hq_linear")
+
+
+def hq_quantize_act_noalloc(desc: LayerDesc, X, sigma_inv, a_codes, a_scale, a_mean=None,
+                            T=None, stream=None):
+    """hq_quantize_act for callers that cannot allocate device memory: the
+    per-tensor scale's workspace is a fixed 256-byte device array inside the
+    library (see include/hq.h).  The first call on a device looks up that
+    array's address, so make it before any stream capture; calls that overlap
+    on the GPU share the array and race."""
+    T = X.shape[0] if T is None else T
+    _check(load_library().hq_quantize_act_noalloc(
+        ctypes.byref(desc), _ptr(X), T, _ptr(sigma_inv), _ptr(a_codes), _ptr(a_scale),
+        _ptr(a_mean), _stream(stream)), "hq_quantize_act_noalloc")
 
 
 def hq_check_device_error(stream=None) -> int:

@@ -312,6 +312,7 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   hq_status s = check_desc(desc);
   if (s != HQ_OK) return s;
   if (T < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
   if (X == nullptr || a_codes == nullptr || a_scale == nullptr) return HQ_ERR_INVALID_ARGUMENT;
   const bool dyn = desc->act_gran == HQ_PER_TENSOR_DYNAMIC;
   if (dyn && (workspace == nullptr || workspace_bytes < 16)) return HQ_ERR_INVALID_ARGUMENT;
@@ -362,6 +363,7 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   if (desc->act_gran < HQ_PER_TOKEN || desc->act_gran > HQ_PER_TENSOR_STATIC)
     return HQ_ERR_INVALID_ARGUMENT;
   if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
   if (a_codes == nullptr || a_scale == nullptr || w_codes == nullptr || w_scale == nullptr ||
       Y == nullptr)
     return HQ_ERR_INVALID_ARGUMENT;
@@ -435,3 +437,53 @@ hq_status hq_debug_inject_fault(int kind) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of hq_quantize_act.
+//
+// Some callers cannot allocate device memory at the point where they quantize:
+// a runtime whose device memory is fixed when the model is loaded (embedded or
+// safety-certified deployments), a host callback or plugin that has no
+// allocator handle, or code running where an allocation would synchronize or
+// is forbidden.  hq_quantize_act needs a small workspace for the per-tensor
+// dynamic scale; this variant takes it from a fixed array that the library
+// holds in device memory instead of from the caller.
+//
+// The array lives for as long as the library is loaded, on every device that
+// loads it (kNoAllocScratchBytes per device).  Its device address is looked up
+// once per device, on the first call made with that device current; make that
+// first call before any stream capture.  All calls share the one array and it
+// keeps the previous call's contents: the quantizer clears the bytes it uses
+// at the start of every call, and two calls whose kernels overlap on the GPU
+// (different streams without ordering between them) race on it.
+constexpr size_t kNoAllocScratchBytes = 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[hq::kMaxDevices] = {};
+}  // namespace
+
+extern "C" hq_status hq_quantize_act_noalloc(const hq_layer_desc* desc, const uint16_t* X,
+                                              int64_t T, const float* sigma_inv, int8_t* a_codes,
+                                              float* a_scale, float* a_mean, hq_stream_t stream) {
+  if (desc == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  const size_t need = hq_quantize_act_workspace_bytes(desc, T);
+  if (need > kNoAllocScratchBytes) return HQ_ERR_UNSUPPORTED;  // beyond the fixed array
+  void* ws = nullptr;
+  if (need > 0 && T > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
+    if (dev < 0 || dev >= hq::kMaxDevices) return HQ_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+        return HQ_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    ws = g_noalloc_ptr[dev];
+  }
+  return hq_quantize_act(desc, X, T, sigma_inv, a_codes, a_scale, a_mean, ws,
+                         ws ? kNoAllocScratchBytes : 0, stream);
+}

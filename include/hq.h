@@ -161,6 +161,26 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
                     const float* colsum, const float* bias_f32, uint16_t* Y,
                     int32_t* acc_debug, hq_stream_t stream);
 
+/* hq_quantize_act_noalloc -- hq_quantize_act without a caller workspace.
+ * (The paper has no counterpart: this is a deployment convenience.)
+ * For callers that cannot allocate device memory when they quantize -- a
+ * runtime whose device memory is fixed at load time, a plugin or host
+ * callback without an allocator, code where an allocation would be forbidden
+ * or would synchronize.  Same arguments and results as hq_quantize_act, but
+ * the per-tensor dynamic scale's workspace comes from a fixed device array of
+ * 256 bytes that the library holds on every device that loads it, until the
+ * process exits; the call itself allocates nothing.
+ *   - Returns HQ_ERR_UNSUPPORTED if the description needs more workspace than
+ *     the 256-byte array (hq_quantize_act_workspace_bytes > 256).
+ *   - The first call made with a given device current looks up the array's
+ *     device address; make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call clears the bytes it uses before using them.  Calls whose kernels
+ *     overlap on the GPU (unordered streams) race on the array. */
+hq_status hq_quantize_act_noalloc(const hq_layer_desc* desc, const uint16_t* X,
+                                  int64_t T, const float* sigma_inv, int8_t* a_codes,
+                                  float* a_scale, float* a_mean, hq_stream_t stream);
+
 /* hq_check_device_error -- synchronizes `stream`, then reads and clears the
  * current device's error word, which kernels set instead of trapping when a
  * bounded wait gives up (HQ_ERR_TIMEOUT).  Returns HQ_ERR_CUDA if the stream
