@@ -88,7 +88,7 @@ hq_status check_k_side(const hq_layer_desc* d) {
   const int logn = ilog2_exact(d->had_order);
   if (d->K <= 0 || d->had_order <= 0) return HQ_ERR_INVALID_ARGUMENT;
   if (logn < 4 || logn > 10) return HQ_ERR_UNSUPPORTED;
-  if (d->K % d->had_order != 0 || d->K % 32 != 0 || d->K > 12288) return HQ_ERR_UNSUPPORTED;
+  if (d->K % d->had_order != 0 || d->K % 64 != 0 || d->K > 9216) return HQ_ERR_UNSUPPORTED;
   if (d->code_format != HQ_CODES_I8) return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
@@ -109,16 +109,16 @@ hq_status check_desc(const hq_layer_desc* d) {
 
 hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
-// Rows per tile R and threads per CTA for the row quantizer: every thread owns
-// a 32-channel slice of one row; prefer full warps and 256..384 threads.
+// Rows per tile R and threads per CTA for the row quantizer: one producer
+// warp plus worker warps in which every thread owns a 32-channel slice of one
+// row; prefer full warps and 8-9 worker warps.
 void quant_shape(int K, int* R_out, int* nt_out) {
   const int S = K / 32;
-  const int maxT = quant_max_threads();
+  const int maxW = quant_max_threads() - 32;
   int bestR = 1, bestNT = ((S + 31) / 32) * 32;
   double bestScore = -1.0;
-  for (int R = 1; R * S <= maxT; ++R) {
+  for (int R = 1; R * S <= maxW && kQuantRowsPerThread * R <= 256; ++R) {  // a tile is one TMA box
     const int nt = ((R * S + 31) / 32) * 32;
-    if (nt > maxT) break;
     const double util = double(R * S) / nt;
     const double size_pref = nt >= 256 ? 1.0 : double(nt) / 256.0;
     const double score = util * 4.0 + size_pref;
@@ -129,32 +129,52 @@ void quant_shape(int K, int* R_out, int* nt_out) {
     }
   }
   *R_out = bestR;
-  *nt_out = bestNT;
+  *nt_out = bestNT + 32;  // + producer warp
 }
 
 struct QuantLaunch {
   QuantParams p;
+  CUtensorMap tmap;
   int threads;
   size_t smem;
   int grid;
+  int logn;
 };
 
-QuantLaunch make_quant_launch(const DeviceState* dev, int K, int n, int64_t T) {
-  QuantLaunch L;
+hq_status encode_rows_bf16(CUtensorMap* m, const void* base, int64_t rows, int K, int R) {
+  // [rows, K] bf16 viewed as {64 elements, K/64 line groups, rows}; one box is
+  // a whole tile of R rows, written to shared memory with 128-byte swizzle
+  cuuint64_t dims[3] = {64u, cuuint64_t(K / 64), cuuint64_t(rows)};
+  cuuint64_t strides[2] = {128u, cuuint64_t(K) * 2u};
+  cuuint32_t box[3] = {64u, cuuint32_t(K / 64), cuuint32_t(R)};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
+hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, const uint16_t* X,
+                            QuantLaunch* out) {
+  QuantLaunch& L = *out;
   std::memset(&L.p, 0, sizeof(L.p));
   int R, nt;
   quant_shape(K, &R, &nt);
-  const int S = K / 32;
-  const int TT = n >= 32 ? n / 32 : 1;
-  const int E = S / TT;
-  const uint32_t raw = uint32_t(R) * uint32_t(K) * 2u;
+  const int logn = ilog2_exact(n);
+  const bool xpose = logn >= 6;            // shared-memory transposes for n >= 64
+  const int per_sm = logn >= 8 ? 1 : 2;    // CTAs per SM (kernel launch bounds)
+  const int B = K / n;
+  const uint32_t raw = uint32_t(kQuantRowsPerThread * R) * uint32_t(K) * 2u;  // one tile
   const uint32_t tile_bytes = (raw + 1023u) & ~1023u;
-  int nstage = int((160u * 1024u) / tile_bytes);
-  if (nstage > 8) nstage = 8;
+  const uint32_t budget = per_sm == 1 ? 150u * 1024u : 100u * 1024u;
+  const size_t fixed = quant_smem_bytes(0, tile_bytes, R, K, B, (nt - 32) / 32, xpose);
+  int nstage = int((budget - uint32_t(fixed)) / tile_bytes);
+  if (nstage > 6) nstage = 6;
   if (nstage < 2) nstage = 2;
   L.p.T = T;
   L.p.K = K;
-  L.p.S = S;
+  L.p.S = K / 32;
   L.p.R = R;
   L.p.nstage = nstage;
   L.p.tile_bytes = tile_bytes;
@@ -163,15 +183,18 @@ QuantLaunch make_quant_launch(const DeviceState* dev, int K, int n, int64_t T) {
   L.p.err = dev->err;
   L.p.wait_ns = wait_ns();
   L.threads = nt;
-  // stages | barriers | pad to 16 | per-block partials | per-row stats | flags
-  L.smem = size_t(nstage) * tile_bytes + 8u * nstage + 16u + 16u * size_t(R) * E + 8u * R + 16u;
-  const int64_t ntiles = (T + R - 1) / R;
-  L.grid = int(ntiles < dev->sm_count ? ntiles : dev->sm_count);
-  return L;
+  L.logn = logn;
+  L.smem = quant_smem_bytes(nstage, tile_bytes, R, K, B, (nt - 32) / 32, xpose);
+  const int64_t tile_rows = kQuantRowsPerThread * R;
+  const int64_t ntiles = (T + tile_rows - 1) / tile_rows;
+  const int64_t slots = int64_t(dev->sm_count) * per_sm;
+  L.grid = int(ntiles < slots ? ntiles : slots);
+  if (T > 0) return encode_rows_bf16(&L.tmap, X, T, K, kQuantRowsPerThread * R);
+  return HQ_OK;
 }
 
-hq_status run_quant(DeviceState* dev, const QuantLaunch& L, int logn, int mode, bool center,
-                    cudaStream_t st) {
+hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, bool center, cudaStream_t st) {
+  const int logn = L.logn;
   const void* fn = quant_kernel_ptr(logn, mode, center);
   if (fn == nullptr) return HQ_ERR_UNSUPPORTED;
   if (L.p.T <= 0) return HQ_OK;
@@ -185,8 +208,7 @@ hq_status run_quant(DeviceState* dev, const QuantLaunch& L, int logn, int mode, 
       set = true;
     }
   }
-  QuantParams p = L.p;
-  void* args[] = {&p};
+  void* args[] = {&L.tmap, &L.p};
   return from_cuda(cudaLaunchKernel(fn, dim3(L.grid), dim3(L.threads), args, L.smem, st));
 }
 
@@ -201,8 +223,20 @@ hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K
   return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
 }
 
+hq_status encode_out_bf16(CUtensorMap* m, const void* base, int64_t rows, int N) {
+  cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(N) * 2u};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
 int choose_bn(int64_t T, int N, int sms) {
-  static const int cands[] = {256, 192, 160, 128, 64};
+  static const int cands[] = {256, 192, 128, 64};
   const int64_t mt = (T + 127) / 128;
   int best = 64;
   double best_cost = 1e300;
@@ -285,7 +319,9 @@ hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const
   if (s != HQ_OK) return s;
   // W~ rows: multiply by sigma (= 1 / sigma_inv), rotate, quantize per row,
   // and record each row's sum (colsum of W~ in the pages' orientation)
-  QuantLaunch L = make_quant_launch(dev, K, desc->had_order, N);
+  QuantLaunch L;
+  s = make_quant_launch(dev, K, desc->had_order, N, W, &L);
+  if (s != HQ_OK) return s;
   L.p.X = W;
   L.p.mult = act_absmax ? sigma_inv : nullptr;
   L.p.invert_mult = 1;
@@ -294,7 +330,7 @@ hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const
   L.p.mean = nullptr;
   L.p.rowsum = colsum;
   L.p.q = (1 << (desc->w_bits - 1)) - 1;
-  s = run_quant(dev, L, ilog2_exact(desc->had_order), 0, false, st);
+  s = run_quant(dev, L, 0, false, st);
   if (s != HQ_OK) return s;
   if (bias) return from_cuda(launch_bf16_to_f32(bias, bias_f32, N, st));
   return from_cuda(launch_fill(bias_f32, N, 0.0f, st));
@@ -324,7 +360,9 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   s = device_state(&dev);
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  QuantLaunch L = make_quant_launch(dev, desc->K, desc->had_order, T);
+  QuantLaunch L;
+  s = make_quant_launch(dev, desc->K, desc->had_order, T, X, &L);
+  if (s != HQ_OK) return s;
   L.p.X = X;
   L.p.mult = sigma_inv;
   L.p.invert_mult = 0;
@@ -334,13 +372,12 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   L.p.rowsum = nullptr;
   L.p.q = (1 << (desc->a_bits - 1)) - 1;
   L.p.fault_skip_load = g_fault == HQ_FAULT_QUANT_WITHHOLD_LOAD ? 1 : 0;
-  const int logn = ilog2_exact(desc->had_order);
   const bool center = desc->centering == HQ_CENTER_TOKEN_MEAN;
-  if (desc->act_gran == HQ_PER_TOKEN) return run_quant(dev, L, logn, 0, center, st);
+  if (desc->act_gran == HQ_PER_TOKEN) return run_quant(dev, L, 0, center, st);
   if (desc->act_gran == HQ_PER_TENSOR_STATIC) {
     L.p.static_scale = a_scale;
     L.p.scale = nullptr;
-    return run_quant(dev, L, logn, 3, center, st);
+    return run_quant(dev, L, 3, center, st);
   }
   // dynamic per tensor: pass 1 finds max |V| over the tensor, pass 2 quantizes
   L.p.tensor_max = static_cast<unsigned int*>(workspace);
@@ -349,9 +386,9 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   L1.p.codes = nullptr;
   L1.p.mean = nullptr;
   L1.p.fault_skip_load = 0;
-  s = run_quant(dev, L1, logn, 1, center, st);
+  s = run_quant(dev, L1, 1, center, st);
   if (s != HQ_OK) return s;
-  return run_quant(dev, L, logn, 2, center, st);
+  return run_quant(dev, L, 2, center, st);
 }
 
 hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
@@ -378,10 +415,12 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   if (s != HQ_OK) return s;
   const int K = desc->K, N = desc->N;
   const int bn = choose_bn(T, N, dev->sm_count);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   s = encode_kmajor_i8(&ta, a_codes, T, K, 128);
   if (s != HQ_OK) return s;
   s = encode_kmajor_i8(&tb, w_codes, N, K, bn);
+  if (s != HQ_OK) return s;
+  s = encode_out_bf16(&ty, Y, T, N);
   if (s != HQ_OK) return s;
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -402,7 +441,7 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.wait_ns = wait_ns();
   const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
   const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
-  return from_cuda(launch_gemm(bn, &ta, &tb, p, grid, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_gemm(bn, &ta, &tb, &ty, p, grid, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hq_status hq_check_device_error(hq_stream_t stream) {

@@ -12,8 +12,13 @@
 //   warp 1      allocates tensor memory; one thread issues tcgen05.mma
 //               (128 x BN x 32 per instruction) and commits each stage back
 //               to the producer and each finished accumulator to the epilogue;
-//   warps 2..5  read the accumulator from tensor memory (tcgen05.ld), apply
-//               the epilogue in fp32 and store bf16 rows.
+//   warps 2..9  the epilogue: two warps per 32-lane quarter of tensor memory,
+//               each taking half of the tile's columns.  Per tile a warp
+//               stages its columns' s_w, colsum and bias in shared memory;
+//               per 32-column chunk it reads the accumulator (tcgen05.ld),
+//               applies the epilogue in fp32, writes bf16 to a 64-byte
+//               swizzled shared buffer and lets a TMA tensor store write the
+//               32 x 32 box to Y (clipped at the tensor's edges).
 // Two accumulators in tensor memory let the epilogue of one tile overlap the
 // main loop of the next.  Every wait is bounded; a timeout records
 // HQ_ERR_TIMEOUT in the device error word and the CTA drains and exits.
@@ -29,15 +34,22 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 128;  // K bytes per stage: one 128-byte swizzle row
-constexpr int kGemmThreads = 192;
-constexpr int kStageBudget = 216 * 1024;
+constexpr int kEpiWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kSmemLimit = 227 * 1024;
 
 template <int BN>
 struct GemmCfg {
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_RAW = kStageBudget / STAGE_BYTES;
+  static constexpr int HC = BN / 2;  // columns per epilogue warp
+  // per epilogue warp: 2 KB output staging (1024-aligned) + params [3][HC]
+  static constexpr int EPI_STAGE_BYTES = 2048;
+  static constexpr int EPI_PARAM_BYTES = 3 * HC * 4;
+  static constexpr int EPI_BYTES = kEpiWarps * (EPI_STAGE_BYTES + EPI_PARAM_BYTES);
+  static constexpr int CTL_BYTES = 256;
+  static constexpr int STAGES_RAW = (kSmemLimit - 1024 - EPI_BYTES - CTL_BYTES - 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
@@ -45,9 +57,11 @@ struct GemmCfg {
   // 7-9 = 1, 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
   static constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) |
                                     (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
-  static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256 /*ctl*/;
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + EPI_BYTES + CTL_BYTES + 1024;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "two 32-column-aligned halves");
   static_assert(B_BYTES % 1024 == 0, "stage bases must stay 1024-byte aligned");
+  static_assert(STAGES >= 2, "shared memory budget");
+  static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
 };
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
@@ -64,19 +78,26 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 }  // namespace
 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + size_t(C::STAGES) * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + size_t(C::STAGES) * C::B_BYTES);
+  uint8_t* epi_stage = sB + size_t(C::STAGES) * C::B_BYTES;  // 1024-aligned, [8][2 KB]
+  float* epi_param = reinterpret_cast<float*>(epi_stage + kEpiWarps * C::EPI_STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_stage + C::EPI_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -95,13 +116,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -202,75 +224,89 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int ew = warp - 2;         // 0 .. 7
+    const int quarter = warp & 3;    // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int half = ew >> 2;        // columns [half*HC, half*HC + HC) of the tile
+    uint8_t* stg = epi_stage + ew * C::EPI_STAGE_BYTES;
+    float* prm = epi_param + ew * (3 * C::HC);
+    const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this thread's row
     int acc_iter = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++acc_iter) {
       const int acc = acc_iter & 1;
       const uint32_t acc_phase = (acc_iter >> 1) & 1;
-      const bool got = !(*abort_flag) && mbar_wait(&tfull[acc], acc_phase, wc);
-      if (!__all_sync(0xffffffffu, got)) {
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
       const int m_idx = tile % p.num_m_tiles;
       const int n_idx = tile / p.num_m_tiles;
-      const int64_t row = int64_t(m_idx) * BM + quarter * 32 + lane;
+      const int col_base = n_idx * BN + half * C::HC;
+      // this warp's columns: scale, colsum, bias (coalesced, before the wait)
+      for (int c = lane; c < C::HC; c += 32) {
+        const int gc = col_base + c;
+        const bool in = gc < p.N;
+        prm[c] = in ? p.w_scale[gc] : 0.0f;
+        prm[C::HC + c] = (in && p.a_mean) ? p.colsum[gc] : 0.0f;
+        prm[2 * C::HC + c] = (in && p.bias) ? p.bias[gc] : 0.0f;
+      }
+      const int row0 = m_idx * BM + quarter * 32;
+      const int64_t row = int64_t(row0) + lane;
       const bool row_ok = row < p.T;
       float sx = 0.0f, mt = 0.0f;
       if (row_ok) {
         sx = p.a_scale_per_row ? p.a_scale[row] : p.a_scale[0];
         mt = p.a_mean ? p.a_mean[row] : 0.0f;
       }
-      const uint32_t t_row = tmem_base + uint32_t(acc * BN) + (uint32_t(quarter * 32) << 16);
+      __syncwarp();
+      const bool got = !(*abort_flag) && mbar_wait(&tfull[acc], acc_phase, wc);
+      if (!__all_sync(0xffffffffu, got)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + uint32_t(acc * BN + half * C::HC) +
+                             (uint32_t(quarter * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < C::HC / 32; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
         tmem_wait_ld();
-        const int col0 = n_idx * BN + c * 32;
-        if (row_ok && col0 < p.N) {
-          uint32_t packed[16];
+        const int col0 = col_base + c * 32;
+        const float* pw = prm + c * 32;
+        uint32_t packed[16];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float4 sw = *reinterpret_cast<const float4*>(pw + 4 * g);
+          const float4 cs = *reinterpret_cast<const float4*>(pw + C::HC + 4 * g);
+          const float4 bb = *reinterpret_cast<const float4*>(pw + 2 * C::HC + 4 * g);
+          const float y0 = __fmaf_rn(__int2float_rn(int(r[4 * g + 0])), __fmul_rn(sx, sw.x),
+                                     __fmaf_rn(mt, cs.x, bb.x));
+          const float y1 = __fmaf_rn(__int2float_rn(int(r[4 * g + 1])), __fmul_rn(sx, sw.y),
+                                     __fmaf_rn(mt, cs.y, bb.y));
+          const float y2 = __fmaf_rn(__int2float_rn(int(r[4 * g + 2])), __fmul_rn(sx, sw.z),
+                                     __fmaf_rn(mt, cs.z, bb.z));
+          const float y3 = __fmaf_rn(__int2float_rn(int(r[4 * g + 3])), __fmul_rn(sx, sw.w),
+                                     __fmaf_rn(mt, cs.w, bb.w));
+          packed[2 * g] = pack_bf16x2(y0, y1);
+          packed[2 * g + 1] = pack_bf16x2(y2, y3);
+        }
+        // the previous chunk's TMA store must have finished reading the buffer
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ swz) << 4)) =
+              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && col0 < p.N && row0 < p.T) {
+          tma_store_2d(&tmY, stg, col0, row0);
+          bulk_commit_group();
+        }
+        if (p.acc_debug && row_ok) {
+          int32_t* arow = p.acc_debug + row * p.N;
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
-            const int col = col0 + 4 * g;
-            float4 sw = make_float4(0, 0, 0, 0), cs = make_float4(0, 0, 0, 0),
-                   bb = make_float4(0, 0, 0, 0);
-            if (col < p.N) {
-              sw = __ldg(reinterpret_cast<const float4*>(p.w_scale + col));
-              if (p.a_mean) cs = __ldg(reinterpret_cast<const float4*>(p.colsum + col));
-              if (p.bias) bb = __ldg(reinterpret_cast<const float4*>(p.bias + col));
-            }
-            const float sws[4] = {sw.x, sw.y, sw.z, sw.w};
-            const float css[4] = {cs.x, cs.y, cs.z, cs.w};
-            const float bbs[4] = {bb.x, bb.y, bb.z, bb.w};
-            float y[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float accf = __int2float_rn(int(r[4 * g + u]));
-              y[u] = __fmaf_rn(accf, __fmul_rn(sx, sws[u]), __fmaf_rn(mt, css[u], bbs[u]));
-            }
-            __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(y[2], y[3]);
-            packed[2 * g] = *reinterpret_cast<uint32_t*>(&lo);
-            packed[2 * g + 1] = *reinterpret_cast<uint32_t*>(&hi);
-          }
-          uint16_t* yrow = p.Y + row * p.N;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (col0 + 8 * g < p.N) {
-              *reinterpret_cast<uint4*>(yrow + col0 + 8 * g) =
-                  make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
-            }
-          }
-          if (p.acc_debug) {
-            int32_t* arow = p.acc_debug + row * p.N;
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              if (col0 + 4 * g < p.N) {
-                *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
-                    make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
-              }
+            if (col0 + 4 * g < p.N) {
+              *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
+                  make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
             }
           }
         }
@@ -279,6 +315,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -291,8 +329,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ------------------------------------------------------------------ launch
 template <int BN>
-static cudaError_t launch_bn(const void* tmap_a, const void* tmap_b, const GemmParams& p, int grid,
-                             cudaStream_t st) {
+static cudaError_t launch_bn(const void* tmap_a, const void* tmap_b, const void* tmap_y,
+                             const GemmParams& p, int grid, cudaStream_t st) {
   using C = GemmCfg<BN>;
   static bool configured = false;  // attribute is per function, device-agnostic
   if (!configured) {
@@ -302,18 +340,18 @@ static cudaError_t launch_bn(const void* tmap_a, const void* tmap_b, const GemmP
     configured = true;
   }
   gemm_i8_kernel<BN><<<grid, kGemmThreads, C::SMEM, st>>>(
-      *reinterpret_cast<const CUtensorMap*>(tmap_a), *reinterpret_cast<const CUtensorMap*>(tmap_b), p);
+      *reinterpret_cast<const CUtensorMap*>(tmap_a), *reinterpret_cast<const CUtensorMap*>(tmap_b),
+      *reinterpret_cast<const CUtensorMap*>(tmap_y), p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const GemmParams& p,
-                        int grid, cudaStream_t st) {
+cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const void* tmap_y,
+                        const GemmParams& p, int grid, cudaStream_t st) {
   switch (bn) {
-    case 64: return launch_bn<64>(tmap_a, tmap_b, p, grid, st);
-    case 128: return launch_bn<128>(tmap_a, tmap_b, p, grid, st);
-    case 160: return launch_bn<160>(tmap_a, tmap_b, p, grid, st);
-    case 192: return launch_bn<192>(tmap_a, tmap_b, p, grid, st);
-    case 256: return launch_bn<256>(tmap_a, tmap_b, p, grid, st);
+    case 64: return launch_bn<64>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 128: return launch_bn<128>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 192: return launch_bn<192>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 256: return launch_bn<256>(tmap_a, tmap_b, tmap_y, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -322,7 +360,6 @@ size_t gemm_smem_bytes(int bn) {
   switch (bn) {
     case 64: return GemmCfg<64>::SMEM;
     case 128: return GemmCfg<128>::SMEM;
-    case 160: return GemmCfg<160>::SMEM;
     case 192: return GemmCfg<192>::SMEM;
     case 256: return GemmCfg<256>::SMEM;
     default: return 0;

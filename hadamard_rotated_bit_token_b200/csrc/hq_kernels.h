@@ -20,10 +20,10 @@ struct QuantParams {
   int64_t T;
   int K;
   int S;                      // 32-channel slices per row (K / 32)
-  int R;                      // rows per tile
+  int R;                      // rows per thread pass (a tile holds kQuantRowsPerThread*R rows)
   int q;                      // 2^(bits-1) - 1
   int nstage;                 // shared-memory stages
-  uint32_t tile_bytes;        // bytes per stage (R*K*2 rounded up to 1024)
+  uint32_t tile_bytes;        // bytes per stage (tile rows * K * 2 rounded up to 1024)
   float inv_sqrt_n;           // 1 / sqrt(n), fp32
   float sqrt_n;               // sqrt(n), fp32
   int fault_skip_load;        // test hook: withhold the first tile load
@@ -31,9 +31,18 @@ struct QuantParams {
   unsigned long long wait_ns; // bounded-wait limit
 };
 
-// Returns the kernel entry for log2(n) in [4,10], mode in [0,3].
+// Returns the kernel entry for log2(n) in [4,10], mode in [0,3]; the kernel
+// takes (const CUtensorMap tmX, QuantParams p): tmX views the [T,K] bf16 rows
+// as a 3-D tensor {64, K/64, T} with box {64, K/64, R} and 128-byte swizzle.
 const void* quant_kernel_ptr(int logn, int mode, bool center);
 int quant_max_threads();
+// Dynamic shared memory of one quantizer CTA (includes 1 KB of alignment slack).
+// Rows of a tile each quantizer worker thread handles (one 32-channel slice of
+// each); a tile holds kQuantRowsPerThread * R rows.
+constexpr int kQuantRowsPerThread = 1;
+// R = rows covered by one pass of the worker threads.
+size_t quant_smem_bytes(int nstage, uint32_t tile_bytes, int R, int K, int B, int nworker_warps,
+                        bool xpose);
 
 struct GemmParams {
   const float* a_scale;   // [T] or [1]
@@ -53,10 +62,12 @@ struct GemmParams {
   unsigned long long wait_ns; // bounded-wait limit
 };
 
-// Launches the tcgen05 GEMM for N tile width bn (64, 128, 160, 192 or 256).
-// tmap_a / tmap_b point to host CUtensorMap objects (copied into the launch).
-cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const GemmParams& p,
-                        int grid, cudaStream_t st);
+// Launches the tcgen05 GEMM for N tile width bn (64, 128, 192 or 256).
+// tmap_a / tmap_b / tmap_y point to host CUtensorMap objects (copied into the
+// launch): A [T,K] and B [N,K] int8 with box {128, 128 | bn} and 128-byte
+// swizzle; Y [T,N] bf16 with box {32, 32} and 64-byte swizzle.
+cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const void* tmap_y,
+                        const GemmParams& p, int grid, cudaStream_t st);
 size_t gemm_smem_bytes(int bn);
 int gemm_threads();
 

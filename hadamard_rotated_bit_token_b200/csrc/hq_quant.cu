@@ -17,21 +17,30 @@
 //
 // Quantizer: HaTQ Sec. III-A Eq. (3), q = 2^(b-1) - 1, s = max|V| / q,
 // code = rne(V / s), computed as rne(V * (q / max|V|)) with one fused
-// multiply-add against 1.5 * 2^23, which rounds half to even.
+// multiply-add against 1.5 * 2^23, which rounds half to even and leaves the
+// code in the low byte of the result's bit pattern.
 //
-// Row mean: sum_k Z_hat[b,k] = n * Y[b,0] for each block b (the columns of
-// H~ sum to zero except the first), so mu_hat = (n / K) * sum_b Y[b, 0]; this
+// Row mean: sum_k Z_hat[b,k] = n * Y[b,0] for each block b (every column of
+// H~ but the first sums to zero), so mu_hat = (n / K) * sum_b Y[b,0]; this
 // identity (HaTQ Eq. (23) read column-wise) gives the exact mean of the
-// rotated row without a second reduction over Z.
+// rotated row from the first channel of each block, summed in a fixed order.
 //
-// Data path per CTA (persistent over row tiles of R rows):
-//   TMA bulk copy of the contiguous tile (R*K bf16) into a ring of shared
-//   memory stages -> each thread takes a 32-channel slice of one row ->
-//   bf16 -> fp32, times the channel multiplier -> butterflies on the 5
-//   in-register index bits -> butterflies on the remaining bits across the
-//   n/32 threads of the block (warp shuffles) -> per-block max / min ->
-//   barrier -> one warp per row reduces the blocks, computes mean and scale ->
-//   barrier -> codes, packed 4 per word, 32 bytes per thread, coalesced.
+// Work decomposition (persistent CTAs over tiles of R rows):
+//   warp 0 (one thread) streams tiles into a ring of shared-memory stages with
+//     a 3-D TMA tensor load (128-byte swizzle, so the row slices below are
+//     read without bank conflicts);
+//   worker warps: each thread owns a 32-channel slice of one row.  bf16 ->
+//     fp32, times the channel multiplier (kept in registers) -> butterflies on
+//     the 5 in-register index bits -> the remaining bits across the n/32
+//     threads of a block: warp shuffles for n <= 128; for n >= 256 an 8-lane
+//     shared-memory transpose swaps index bits 2-4 with 5-7 and shuffles take
+//     bits 8 and up -> row max / min by shared-memory atomics on ordered
+//     integers -> a per-row mbarrier (one arrival per thread of the row) ->
+//     codes packed 4 per word and stored.  No CTA-wide barrier in the loop:
+//     warps only wait for the other warps of their own rows.
+// Arithmetic on pairs of lanes uses Blackwell's packed fp32x2 instructions.
+#include <cuda.h>
+
 #include "hq_device.cuh"
 #include "hq_kernels.h"
 
@@ -39,13 +48,10 @@ namespace hq {
 
 namespace {
 
-constexpr int kMaxQuantThreads = 384;
+constexpr int kQuantThreads = 320;  // 1 producer warp + up to 9 worker warps
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
-
-struct __align__(16) RowPart {
-  float mx, mn, y0, pad;
-};
+constexpr int kStatBufs = 3;
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -61,277 +67,493 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
   return d;
 }
 
+// Order-preserving map of floats onto unsigned integers (for atomicMax/Min).
+__device__ __forceinline__ uint32_t ord_f32(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_f32(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+__device__ __forceinline__ uint32_t f2lo_bits(f2 x) { return __float_as_uint(x.x); }
+__device__ __forceinline__ uint32_t f2hi_bits(f2 x) { return __float_as_uint(x.y); }
+__device__ __forceinline__ f2 f2_from_bits(uint32_t lo, uint32_t hi) {
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+// Shared-memory layout of one CTA (offsets in bytes, from a 1024-byte aligned base).
+struct QuantSmem {
+  uint32_t stages, full, empty, rowbar, rowmax, rowmin, y0, mult, xbuf, flags, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ inline int padded_blocks(int B) { return (B + 3) & ~3; }
+
+// RT = rows per tile (2 per thread), K channels, B blocks per row.
+__host__ __device__ inline QuantSmem quant_smem_layout(int nstage, uint32_t tile_bytes, int RT, int K,
+                                                       int B, int nworker_warps, bool xpose) {
+  QuantSmem L;
+  uint32_t off = 0;
+  L.stages = off;
+  off += uint32_t(nstage) * tile_bytes;
+  L.full = off;
+  off += 8u * nstage;
+  L.empty = off;
+  off += 8u * nstage;
+  L.rowbar = off;
+  off += 8u * RT;
+  L.rowmax = off;
+  off += 4u * kStatBufs * RT;
+  L.rowmin = off;
+  off += 4u * kStatBufs * RT;
+  off = align_up(off, 16);
+  L.y0 = off;  // [kStatBufs][RT][padded B] first channel of every block
+  off += 4u * kStatBufs * RT * padded_blocks(B);
+  off = align_up(off, 16);
+  L.mult = off;  // channel multipliers, chunk-major [8][K/32] float4
+  off += 4u * K;
+  L.xbuf = off;
+  off += xpose ? 4096u * nworker_warps : 0u;
+  L.flags = off;
+  off += 16;
+  L.total = off;
+  return L;
+}
+
 }  // namespace
+
+size_t quant_smem_bytes(int nstage, uint32_t tile_bytes, int R, int K, int B, int nworker_warps,
+                        bool xpose) {
+  return quant_smem_layout(nstage, tile_bytes, kQuantRowsPerThread * R, K, B, nworker_warps, xpose)
+             .total + 1024;
+}
 
 // MODE 0: per-row dynamic scale (activations per token, or weights per row)
 // MODE 1: per-tensor pass 1: only the tensor-wide max |V| (into tensor_max)
 // MODE 2: per-tensor pass 2: scale from tensor_max
 // MODE 3: per-tensor static scale from static_scale[0] (real units)
+//
+// Each worker thread owns one 32-channel slice of RPT rows of a tile (rows r,
+// r + R, ...); the per-tile bookkeeping and multipliers are shared by them.
 template <int LOGN, int MODE, bool CENTER>
-__global__ void __launch_bounds__(kMaxQuantThreads, 1) quant_rows_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQuantThreads, (LOGN >= 8 ? 1 : 2))
+    quant_rows_kernel(const __grid_constant__ CUtensorMap tmX, const QuantParams p) {
   constexpr int N = 1 << LOGN;
-  constexpr int LREG = LOGN < 5 ? LOGN : 5;      // in-register butterfly bits
-  constexpr int TT = N >= 32 ? N / 32 : 1;        // threads per Hadamard block
-  constexpr int LOG_TT = LOGN > 5 ? LOGN - 5 : 0;
-  constexpr int BPT = N >= 32 ? 1 : 32 / N;       // blocks per thread slice
+  constexpr int LREG = LOGN < 5 ? LOGN : 5;        // index bits inside a thread's slice
+  constexpr int LOG_TT = LOGN > 5 ? LOGN - 5 : 0;  // index bits across threads
+  constexpr int TT = 1 << LOG_TT;                  // threads per Hadamard block
+  // Cross-thread bits: the lowest LX of them by a shared-memory transpose
+  // among G = 2^LX lanes (swapping them with in-register bits 5-LX..4), the
+  // rest by warp shuffles.
+  constexpr int LX = LOG_TT < 3 ? LOG_TT : 3;
+  constexpr int G = 1 << LX;                       // lanes per transpose group = groups per thread
+  constexpr int GS = 32 / G;                       // elements per group
+  constexpr int GP = GS / 2;                       // f32x2 pairs per group
+  constexpr int CH = GS / 4;                       // 16-byte chunks per group
+  constexpr bool XPOSE = LX > 0;
+  constexpr int NSHFL = LOG_TT - LX;
+  constexpr int BPT = N >= 32 ? 1 : 32 / N;        // blocks per thread slice (n < 32)
+  constexpr int RPT = kQuantRowsPerThread;         // rows per thread
   constexpr bool kClamp = (MODE >= 2);
+  constexpr bool kQuantize = (MODE != 1);
 
-  extern __shared__ __align__(1024) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
+  const int lane = tid & 31;
+  const int nworkers = int(blockDim.x) - 32;
   const int S = p.S;
-  const int R = p.R;
+  const int R = p.R;            // rows per half tile (threads cover R x S slices)
+  const int RT = RPT * R;       // rows per tile
   const int K = p.K;
-  const int E = S / TT;                            // block partials per row
-  const int active = R * S;
-  const bool is_worker = tid < active;
-  const int row_in_tile = is_worker ? tid / S : 0;
-  const int slice = is_worker ? tid - row_in_tile * S : 0;
-  const int team_idx = slice / TT;
-  const int member = slice - team_idx * TT;
-
-  // shared layout
-  const uint32_t tile_bytes = p.tile_bytes;
-  uint8_t* stages = smem;
-  size_t off = size_t(p.nstage) * tile_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
-  off = (off + 8u * p.nstage + 15u) & ~size_t(15);
-  RowPart* part = reinterpret_cast<RowPart*>(smem + off);      // 16-byte aligned
-  off += sizeof(RowPart) * size_t(R) * E;
-  float2* rowstat = reinterpret_cast<float2*>(smem + off);
-  off += sizeof(float2) * size_t(R);
-  int* flags = reinterpret_cast<int*>(smem + off);  // [0] abort, [1] cta max bits
-
+  const int B = K >> LOGN;
+  const int BP = padded_blocks(B);
+  const int lines_per_row = K >> 6;  // 128-byte lines of bf16
   const int64_t T = p.T;
-  const int64_t ntiles = (T + R - 1) / R;
+  const int64_t ntiles = (T + RT - 1) / RT;
+  const QuantSmem L = quant_smem_layout(p.nstage, p.tile_bytes, RT, K, B, nworkers >> 5, XPOSE);
+  uint8_t* stages = smem + L.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.full);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L.empty);
+  uint64_t* rowbar = reinterpret_cast<uint64_t*>(smem + L.rowbar);
+  uint32_t* rowmax = reinterpret_cast<uint32_t*>(smem + L.rowmax);
+  uint32_t* rowmin = reinterpret_cast<uint32_t*>(smem + L.rowmin);
+  float* y0buf = reinterpret_cast<float*>(smem + L.y0);
+  float4* msm = reinterpret_cast<float4*>(smem + L.mult);
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);  // [0] abort, [1] cta max
+  const WaitCtl wc{p.err, p.wait_ns};
+  const bool has_mult = p.mult != nullptr;
+  const bool need_sum = CENTER || p.rowsum != nullptr;
 
   if (tid == 0) {
-    for (int s = 0; s < p.nstage; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < p.nstage; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], uint32_t(nworkers));
+    }
+    for (int r = 0; r < RT; ++r) mbar_init(&rowbar[r], uint32_t(S));
     flags[0] = 0;
     flags[1] = 0;
     fence_mbarrier_init();
   }
+  for (int i = tid; i < kStatBufs * RT; i += blockDim.x) {
+    rowmax[i] = 0u;
+    rowmin[i] = 0xFFFFFFFFu;
+  }
+  for (int i = tid; i < kStatBufs * RT * BP; i += blockDim.x) y0buf[i] = 0.0f;
+  if (has_mult) {
+    // chunk-major copy: thread `slice` reads chunk c at msm[c * S + slice], so
+    // consecutive slices hit consecutive 16-byte words
+    for (int i = tid; i < 8 * S; i += blockDim.x) {
+      const int c = i / S, sl = i - c * S;
+      float4 m4 = *reinterpret_cast<const float4*>(p.mult + sl * 32 + 4 * c);
+      if (p.invert_mult) {
+        m4.x = 1.0f / m4.x;
+        m4.y = 1.0f / m4.y;
+        m4.z = 1.0f / m4.z;
+        m4.w = 1.0f / m4.w;
+      }
+      msm[i] = m4;
+    }
+  }
   __syncthreads();
 
-  auto issue = [&](int64_t tile, int s) {
-    const int64_t r0 = tile * R;
-    const int64_t rows = (T - r0) < R ? (T - r0) : R;
-    const uint32_t bytes = uint32_t(rows) * uint32_t(K) * 2u;
-    mbar_arrive_expect_tx(&full[s], bytes);
-    bulk_load(stages + size_t(s) * tile_bytes, p.X + r0 * K, bytes, &full[s]);
-  };
-
-  const WaitCtl wc{p.err, p.wait_ns};
-  const bool skip_first = (MODE == 0 || MODE == 2) && p.fault_skip_load;
-  if (tid == 0) {
-    int64_t t = blockIdx.x;
-    for (int s = 0; s < p.nstage && t < ntiles; ++s, t += gridDim.x) {
-      if (s == 0 && skip_first) continue;  // test hook: this stage never completes
-      issue(t, s);
-    }
-  }
-
-  // per-channel multipliers for this thread's 32 channels (fixed across tiles)
-  float mult[32];
-  const bool has_mult = p.mult != nullptr;
-  if (has_mult) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      float4 m4 = *reinterpret_cast<const float4*>(p.mult + slice * 32 + i);
-      if (p.invert_mult) {
-        mult[i] = 1.0f / m4.x;
-        mult[i + 1] = 1.0f / m4.y;
-        mult[i + 2] = 1.0f / m4.z;
-        mult[i + 3] = 1.0f / m4.w;
-      } else {
-        mult[i] = m4.x;
-        mult[i + 1] = m4.y;
-        mult[i + 2] = m4.z;
-        mult[i + 3] = m4.w;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      const uint32_t box_bytes = uint32_t(RT) * uint32_t(K) * 2u;
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool skipped = false;
+      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        if (flags[0] || !mbar_wait(&empty[s], ph ^ 1u, wc)) {
+          flags[0] = 1;
+          break;
+        }
+        if (issued == 0 && p.fault_skip_load && !skipped) {
+          skipped = true;  // test hook: this stage's barrier never completes
+        } else {
+          mbar_arrive_expect_tx(&full[s], box_bytes);
+          tma_load_3d(stages + size_t(s) * p.tile_bytes, &tmX, 0, 0, int32_t(tile * RT), &full[s]);
+        }
+        ++issued;
+        if (++s == p.nstage) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (flags[0]) {
+        // let copies still in flight land before the CTA exits
+        int s2 = s;
+        uint32_t ph2 = ph;
+        for (int i = 0; i < p.nstage && i < issued; ++i) {
+          if (--s2 < 0) {
+            s2 = p.nstage - 1;
+            ph2 ^= 1u;
+          }
+          if (!(skipped && i == issued - 1)) (void)mbar_wait(&full[s2], ph2, wc);
+        }
       }
     }
-  }
+  } else {
+    // -------------------------------------------------------------- workers
+    const int wid = tid - 32;
+    const bool active = wid < R * S;
+    const int row0 = active ? wid / S : 0;   // rows row0, row0 + R, ... of the tile
+    const int slice = active ? wid - row0 * S : 0;
+    const int member = slice & (TT - 1);
+    const int blk = slice >> LOG_TT;      // block of the row (n >= 32)
+    const int tl = lane & (G - 1);        // lane within the transpose group
+    const int sub = lane >> LX;           // transpose group within the warp
+    uint8_t* xb = smem + L.xbuf + (warp - 1) * 4096 + sub * (G * 128);
+    const int csw = sub & (CH - 1);       // chunk swizzle of this transpose group
 
-  // tensor-wide reciprocal scale for the per-tensor quantize passes
-  float r_tensor = 0.0f;
-  if (MODE == 2) {
-    const float a = __uint_as_float(*p.tensor_max);
-    r_tensor = a > 0.0f ? float(p.q) / a : 0.0f;
-    if (blockIdx.x == 0 && tid == 0 && p.scale) p.scale[0] = (a / float(p.q)) * p.inv_sqrt_n;
-  } else if (MODE == 3) {
-    const float s = p.static_scale[0];
-    r_tensor = s > 0.0f ? 1.0f / (s * p.sqrt_n) : 0.0f;
-  }
+    float r_tensor = 0.0f;
+    if (MODE == 2) {
+      const float a = __uint_as_float(*p.tensor_max);
+      r_tensor = a > 0.0f ? __fdiv_rn(float(p.q), a) : 0.0f;
+      if (blockIdx.x == 0 && wid == 0 && p.scale) p.scale[0] = (a / float(p.q)) * p.inv_sqrt_n;
+    } else if (MODE == 3) {
+      const float s = p.static_scale[0];
+      r_tensor = s > 0.0f ? __fdiv_rn(1.0f, s * p.sqrt_n) : 0.0f;
+    }
+    const float n_over_k = float(N) / float(K);
+    const float qf = float(p.q);
 
-  int it = 0;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int s = it % p.nstage;
-    const uint32_t parity = (it / p.nstage) & 1;
-    if (!mbar_wait(&full[s], parity, wc)) flags[0] = 1;
-
-    const int64_t row = tile * R + row_in_tile;
-    const bool valid = is_worker && row < T;
-
-    float v[32];
-    float y0 = 0.0f;
-    if (is_worker) {
-      const uint4* src = reinterpret_cast<const uint4*>(stages + size_t(s) * tile_bytes +
-                                                        (size_t(row_in_tile) * K + slice * 32) * 2);
+    // byte offsets of this thread's slices inside a stage (128-byte swizzle)
+    uint32_t chunk_off[RPT][4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 w = src[c];
-        v[8 * c + 0] = bf16lo(w.x);
-        v[8 * c + 1] = bf16hi(w.x);
-        v[8 * c + 2] = bf16lo(w.y);
-        v[8 * c + 3] = bf16hi(w.y);
-        v[8 * c + 4] = bf16lo(w.z);
-        v[8 * c + 5] = bf16hi(w.z);
-        v[8 * c + 6] = bf16lo(w.w);
-        v[8 * c + 7] = bf16hi(w.w);
+    for (int h = 0; h < RPT; ++h) {
+      const int line = (row0 + h * R) * lines_per_row + (slice >> 1);
+      const int c0 = (slice & 1) * 4;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) chunk_off[h][c] = uint32_t(line) * 128u + (uint32_t((c0 + c) ^ (line & 7)) << 4);
+    }
+
+    int s = 0;
+    uint32_t ph = 0;
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int sb = it % kStatBufs;
+      const bool got = mbar_wait(&full[s], ph, wc);
+      if (!__all_sync(0xffffffffu, got && !flags[0])) {  // warp-uniform exit
+        flags[0] = 1;
+        break;
       }
+      const uint8_t* st = stages + size_t(s) * p.tile_bytes;
+
+      f2 w[RPT][16];
+#pragma unroll
+      for (int h = 0; h < RPT; ++h) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (active) v = *reinterpret_cast<const uint4*>(st + chunk_off[h][c]);
+          w[h][4 * c + 0] = pk(bf16lo(v.x), bf16hi(v.x));
+          w[h][4 * c + 1] = pk(bf16lo(v.y), bf16hi(v.y));
+          w[h][4 * c + 2] = pk(bf16lo(v.z), bf16hi(v.z));
+          w[h][4 * c + 3] = pk(bf16lo(v.w), bf16hi(v.w));
+        }
+      }
+      mbar_arrive(&empty[s]);  // this thread is done with the stage
+      if (++s == p.nstage) {
+        s = 0;
+        ph ^= 1u;
+      }
+
       if (has_mult) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], mult[i]);
-      }
-      // first channel of each block, for the row mean / row sum
-      if (member == 0) {
+        for (int i = 0; i < 8; ++i) {
+          const float4 m4 = msm[i * S + slice];
+          const f2 ma = pk(m4.x, m4.y), mb = pk(m4.z, m4.w);
 #pragma unroll
-        for (int b = 0; b < BPT; ++b) y0 += v[b * (32 / BPT)];
-      }
-      // butterflies on the in-register index bits (natural Sylvester order)
-#pragma unroll
-      for (int h = 1; h < (1 << LREG); h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if ((i & h) == 0) {
-            const float a = v[i], b = v[i + h];
-            v[i] = __fadd_rn(a, b);
-            v[i + h] = __fsub_rn(a, b);
+          for (int h = 0; h < RPT; ++h) {
+            w[h][2 * i] = mul2(w[h][2 * i], ma);
+            w[h][2 * i + 1] = mul2(w[h][2 * i + 1], mb);
           }
         }
       }
-    } else {
+      // first channel of each block (Y[b,0]) for the row mean / row sum
+      if (need_sum && active && member == 0) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-    }
-    // butterflies across the n/32 threads of a block (element bit 5 + j is
-    // lane bit j); all lanes of the warp take part
+        for (int h = 0; h < RPT; ++h) {
+          float* yrow = y0buf + (sb * RT + row0 + h * R) * BP;
 #pragma unroll
-    for (int j = 0; j < LOG_TT; ++j) {
-      const float sgn = ((lane >> j) & 1) ? -1.0f : 1.0f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[i], 1 << j);
-        v[i] = __fmaf_rn(v[i], sgn, o);
+          for (int b = 0; b < BPT; ++b) yrow[blk * BPT + b] = w[h][(b * N) >> 1].x;
+        }
       }
-    }
-    // per-thread max / min, reduced over the block's threads
-    float mx = max3(v[0], v[1], v[2]);
-    float mn = min3(v[0], v[1], v[2]);
+      // index bit 0: the two halves of a pair
 #pragma unroll
-    for (int i = 3; i < 31; i += 2) {
-      mx = max3(mx, v[i], v[i + 1]);
-      mn = min3(mn, v[i], v[i + 1]);
-    }
-    mx = fmaxf(mx, v[31]);
-    mn = fminf(mn, v[31]);
+      for (int h = 0; h < RPT; ++h) {
 #pragma unroll
-    for (int j = 0; j < LOG_TT; ++j) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1 << j));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1 << j));
-    }
-    if (is_worker && member == 0) {
-      RowPart rp;
-      rp.mx = mx;
-      rp.mn = mn;
-      rp.y0 = y0;
-      rp.pad = 0.0f;
-      part[row_in_tile * E + team_idx] = rp;
-    }
-    __syncthreads();  // partials complete; the stage has been consumed
+        for (int i = 0; i < 16; ++i) {
+          const float a = w[h][i].x, b = w[h][i].y;
+          w[h][i] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
+        }
+      }
+      // index bits 1 .. LREG-1: between pairs
+#pragma unroll
+      for (int bit = 1; bit < LREG; ++bit) {
+        const int hh = 1 << (bit - 1);
+#pragma unroll
+        for (int h = 0; h < RPT; ++h) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if ((i & hh) == 0) {
+              const f2 x = w[h][i], y = w[h][i + hh];
+              w[h][i] = add2(x, y);
+              w[h][i + hh] = sub2(x, y);
+            }
+          }
+        }
+      }
+      if (XPOSE) {
+        // swap index bits 5..4+LX (lanes of a G-lane group) with bits
+        // 5-LX..4 (register groups of GS elements); slots XOR-swizzled by
+        // lane, chunks by group, so 16-byte accesses do not conflict
+#pragma unroll
+        for (int h = 0; h < RPT; ++h) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+              const f2 a = w[h][g * GP + 2 * c], b = w[h][g * GP + 2 * c + 1];
+              *reinterpret_cast<float4*>(xb + (tl * G + (g ^ tl)) * (GS * 4) + ((c ^ csw) << 4)) =
+                  make_float4(a.x, a.y, b.x, b.y);
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+              const float4 v = *reinterpret_cast<const float4*>(xb + (g * G + (tl ^ g)) * (GS * 4) +
+                                                                ((c ^ csw) << 4));
+              w[h][g * GP + 2 * c] = pk(v.x, v.y);
+              w[h][g * GP + 2 * c + 1] = pk(v.z, v.w);
+            }
+          }
+          __syncwarp();
+        }
+        // index bits 5..4+LX are now the register-group bits
+#pragma unroll
+        for (int k = 0; k < LX; ++k) {
+          const int hh = GP << k;
+#pragma unroll
+          for (int h = 0; h < RPT; ++h) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if ((i & hh) == 0) {
+                const f2 x = w[h][i], y = w[h][i + hh];
+                w[h][i] = add2(x, y);
+                w[h][i + hh] = sub2(x, y);
+              }
+            }
+          }
+        }
+      }
+      // remaining index bits (5+LX and up) across lanes
+#pragma unroll
+      for (int j = 0; j < NSHFL; ++j) {
+        const int mask = 1 << (LX + j);
+        const float sg = (lane & mask) ? -1.0f : 1.0f;
+        const f2 sg2 = pk(sg, sg);
+#pragma unroll
+        for (int h = 0; h < RPT; ++h) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const f2 o = pk(__shfl_xor_sync(0xffffffffu, w[h][i].x, mask),
+                            __shfl_xor_sync(0xffffffffu, w[h][i].y, mask));
+            w[h][i] = fma2(w[h][i], sg2, o);
+          }
+        }
+      }
 
-    if (flags[0]) break;
-    if (tid == 0) {
-      const int64_t nt = tile + int64_t(p.nstage) * gridDim.x;
-      if (nt < ntiles) issue(nt, s);
-    }
-
-    // one warp per row: reduce the block partials, derive mean and scale
-    for (int rr = warp; rr < R; rr += nwarps) {
-      float rmx = -INFINITY, rmn = INFINITY, rsum = 0.0f;
-      for (int e = lane; e < E; e += 32) {
-        const RowPart q = part[rr * E + e];
-        rmx = fmaxf(rmx, q.mx);
-        rmn = fminf(rmn, q.mn);
-        rsum += q.y0;
-      }
+      // row max / min, one row barrier per row (S arrivals)
+      bool ok = true;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        rmx = fmaxf(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
-        rmn = fminf(rmn, __shfl_xor_sync(0xffffffffu, rmn, o));
-        rsum += __shfl_xor_sync(0xffffffffu, rsum, o);
+      for (int h = 0; h < RPT; ++h) {
+        float mx = max3(w[h][0].x, w[h][0].y, w[h][1].x);
+        float mn = min3(w[h][0].x, w[h][0].y, w[h][1].x);
+        mx = fmaxf(mx, w[h][1].y);
+        mn = fminf(mn, w[h][1].y);
+#pragma unroll
+        for (int i = 2; i < 16; ++i) {
+          mx = max3(mx, w[h][i].x, w[h][i].y);
+          mn = min3(mn, w[h][i].x, w[h][i].y);
+        }
+        if (active) {
+          const int r = row0 + h * R;
+          atomicMax(&rowmax[sb * RT + r], ord_f32(mx));
+          atomicMin(&rowmin[sb * RT + r], ord_f32(mn));
+          mbar_arrive(&rowbar[r]);
+        }
       }
-      const int64_t grow = tile * R + rr;
-      if (lane == 0 && grow < T) {
-        const float m_hat = CENTER ? (float(N) / float(K)) * rsum : 0.0f;
+      if (active) {
+#pragma unroll
+        for (int h = 0; h < RPT; ++h) ok = ok && mbar_wait(&rowbar[row0 + h * R], uint32_t(it & 1), wc);
+      }
+      if (!__all_sync(0xffffffffu, ok)) {
+        flags[0] = 1;
+        break;
+      }
+      if (!active) continue;
+
+#pragma unroll
+      for (int h = 0; h < RPT; ++h) {
+        const int r = row0 + h * R;
+        float rsum = 0.0f;
+        if (need_sum) {
+          // sum of the row's first channels, in block order
+          const float4* y4 = reinterpret_cast<const float4*>(y0buf + (sb * RT + r) * BP);
+          for (int b4 = 0; b4 < (B + 3) / 4; ++b4) {
+            const float4 v = y4[b4];
+            rsum = __fadd_rn(rsum, v.x);
+            if (4 * b4 + 1 < B) rsum = __fadd_rn(rsum, v.y);
+            if (4 * b4 + 2 < B) rsum = __fadd_rn(rsum, v.z);
+            if (4 * b4 + 3 < B) rsum = __fadd_rn(rsum, v.w);
+          }
+        }
+        const float m_hat = CENTER ? n_over_k * rsum : 0.0f;
+        const float rmx = unord_f32(rowmax[sb * RT + r]);
+        const float rmn = unord_f32(rowmin[sb * RT + r]);
         const float a_hat = fmaxf(__fsub_rn(rmx, m_hat), __fsub_rn(m_hat, rmn));
         float r_rec;
         if (MODE == 0) {
-          r_rec = a_hat > 0.0f ? float(p.q) / a_hat : 0.0f;
-          p.scale[grow] = (a_hat / float(p.q)) * p.inv_sqrt_n;
-        } else if (MODE == 1) {
-          atomicMax(reinterpret_cast<unsigned*>(&flags[1]), __float_as_uint(a_hat));
-          r_rec = 0.0f;
+          r_rec = a_hat > 0.0f ? __fdiv_rn(qf, a_hat) : 0.0f;
         } else {
           r_rec = r_tensor;
         }
-        if (MODE != 1 && p.mean) p.mean[grow] = m_hat * p.inv_sqrt_n;
-        if (p.rowsum) p.rowsum[grow] = rsum * p.sqrt_n;  // sqrt(n) * sum_b Y[b,0]
-        rowstat[rr] = make_float2(m_hat, r_rec);
-      }
-    }
-    __syncthreads();
-
-    if (MODE != 1 && valid) {
-      const float2 st = rowstat[row_in_tile];
-      const float m_hat = st.x, rr = st.y;
-      uint32_t words[8];
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        uint32_t b[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float d = __fsub_rn(v[4 * w + u], m_hat);
-          const float t = __fmaf_rn(d, rr, kRoundMagic);
-          int c = int(__float_as_uint(t) - kRoundMagicBits);
-          if (kClamp) c = max(-p.q, min(p.q, c));
-          b[u] = uint32_t(c);
+        const int64_t row = tile * RT + r;
+        const bool valid = row < T;
+        if (slice == 0) {
+          // stats buffer of the previous tile is free again (see the row barrier)
+          rowmax[((it + 2) % kStatBufs) * RT + r] = 0u;
+          rowmin[((it + 2) % kStatBufs) * RT + r] = 0xFFFFFFFFu;
+          if (valid) {
+            if (MODE == 0) p.scale[row] = (a_hat / qf) * p.inv_sqrt_n;
+            if (MODE == 1) atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])),
+                                     __float_as_uint(a_hat));
+            if (kQuantize && p.mean) p.mean[row] = m_hat * p.inv_sqrt_n;
+            if (p.rowsum) p.rowsum[row] = rsum * p.sqrt_n;  // sqrt(n) * sum_b Y[b,0]
+          }
         }
-        words[w] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
-                               0x5410);
+        if (!kQuantize || !valid) continue;
+
+        const f2 mh2 = pk(m_hat, m_hat), rr2 = pk(r_rec, r_rec), mg2 = pk(kRoundMagic, kRoundMagic);
+        uint32_t words[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          uint32_t b[4];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const f2 t = fma2(sub2(w[h][2 * g + u], mh2), rr2, mg2);
+            b[2 * u] = __float_as_uint(t.x);
+            b[2 * u + 1] = __float_as_uint(t.y);
+          }
+          if (kClamp) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              int c = int(b[u] - kRoundMagicBits);
+              b[u] = uint32_t(max(-p.q, min(p.q, c)));
+            }
+          }
+          words[g] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                                 0x5410);
+        }
+        int8_t* crow = p.codes + row * K;
+        if (!XPOSE) {
+          uint4* dst = reinterpret_cast<uint4*>(crow + slice * 32);
+          dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+          dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+        } else {
+          // register group g: index bits 5..4+LX = g, bits 5-LX..4 = tl, bits
+          // 5+LX.. = member >> LX; GS consecutive codes per group
+          int8_t* base = crow + blk * N + GS * tl + (32 * G) * (member >> LX);
+          constexpr int WPG = GS / 4;  // words per group
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            if (WPG == 4) {
+              *reinterpret_cast<uint4*>(base + 32 * g) =
+                  make_uint4(words[4 * g], words[4 * g + 1], words[4 * g + 2], words[4 * g + 3]);
+            } else if (WPG == 2) {
+              *reinterpret_cast<uint2*>(base + 32 * g) = make_uint2(words[2 * g], words[2 * g + 1]);
+            } else {
+              *reinterpret_cast<uint32_t*>(base + 32 * g) = words[g];
+            }
+          }
+        }
       }
-      uint4* dst = reinterpret_cast<uint4*>(p.codes + row * K + slice * 32);
-      dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-      dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
     }
   }
 
-  if (flags[0]) {
-    // abort: let any bulk copies this CTA issued land before the CTA exits
-    if (tid == 0) {
-      int it2 = it;
-      for (int64_t t = int64_t(blockIdx.x) + int64_t(it) * gridDim.x; t < ntiles && it2 < it + p.nstage;
-           t += gridDim.x, ++it2) {
-        const int s = it2 % p.nstage;
-        if (!(it2 == 0 && skip_first)) (void)mbar_wait(&full[s], (it2 / p.nstage) & 1, wc);
-      }
-    }
-    __syncthreads();
-    return;
-  }
-  if (MODE == 1 && tid == 0) atomicMax(p.tensor_max, unsigned(flags[1]));
+  __syncthreads();
+  if (MODE == 1 && tid == 0 && !flags[0]) atomicMax(p.tensor_max, unsigned(flags[1]));
 }
 
 // ---------------------------------------------------------------- dispatch
@@ -359,7 +581,7 @@ const void* quant_kernel_ptr(int logn, int mode, bool center) {
   }
 }
 
-int quant_max_threads() { return kMaxQuantThreads; }
+int quant_max_threads() { return kQuantThreads; }
 
 // ------------------------------------------------- calibration reductions
 // out[k] = max(out[k], max_r |M[r,k]|) for a bf16 matrix M[rows, K]; out holds

@@ -34,7 +34,7 @@
  *     launches nothing.
  *
  * Shapes supported:  had_order a power of two in [16, 1024]; K a multiple of
- * had_order and of 32, K <= 12288; N a multiple of 16; T >= 0 (T = 0 is a
+ * had_order and of 64, K <= 9216; N a multiple of 16; T >= 0 (T = 0 is a
  * no-op); a_bits in {3, 4, 8}, w_bits in {4, 8} (codes in an int8 container,
  * one code per byte).
  */

@@ -60,7 +60,7 @@ def _check_act(ref, codes, scale, mean, per_row=True, min_match=None, what="act"
 # ---------------------------------------------------------------------------
 
 SMALL = []
-for i, (n, B) in enumerate([(16, 2), (16, 6), (32, 1), (32, 5), (64, 1), (64, 5), (128, 1),
+for i, (n, B) in enumerate([(16, 4), (16, 12), (32, 2), (32, 6), (64, 1), (64, 5), (128, 1),
                             (128, 9), (256, 1), (256, 3), (512, 2), (1024, 1), (1024, 3)]):
     for T in (1, 7, 129, 300):
         bits = (4, 3, 8)[(i + T) % 3]
