@@ -245,6 +245,7 @@ def config_block(cfg, n_gpus):
             "had_order": cfg.had_order, "bits": f"A{cfg.a_bits}W{cfg.w_bits}",
             "act_granularity": gran, "centering": bool(cfg.centering), "sigma": cfg.use_sigma,
             "l2": "flushed before every timed step (memset of 2x L2, outside the timed events)",
+            "timing": "CUDA events around CUDA-graph replays (one graph per kernel)",
             "parallelism": f"dp{n_gpus} (token shards, replicated weights, no collective)"}
 
 
@@ -315,6 +316,19 @@ def run_hq(args):
     if status != 0:
         raise RuntimeError(f"device error during warm-up: {hq.STATUS_NAMES.get(status)}")
 
+    # One CUDA graph per kernel: replays carry no host launch overhead, and an
+    # event between the two replays times each kernel separately.
+    g_quant, g_linear = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_quant):
+        quantize()
+    with torch.cuda.graph(g_linear):
+        linear()
+    for _ in range(args.warmup):
+        flush.zero_()
+        g_quant.replay()
+        g_linear.replay()
+    torch.cuda.synchronize()
+
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
@@ -325,9 +339,9 @@ def run_hq(args):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        quantize()
+        g_quant.replay()
         ev[i][1].record(stream)
-        linear()
+        g_linear.replay()
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -357,12 +371,21 @@ def run_hq(args):
         Yh = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
         Xd = torch.empty_like(X)
 
-        def e2e_step():
+        def e2e_body():
             Xd.copy_(Xh, non_blocking=True)
             hq.hq_quantize_act(desc, Xd, sig_inv, bufs["a_codes"], bufs["a_scale"],
                                bufs["a_mean"], layer.workspace)
             linear()
             Yh.copy_(Y, non_blocking=True)
+
+        e2e_body()
+        torch.cuda.synchronize()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e):
+            e2e_body()
+
+        def e2e_step():
+            g_e2e.replay()
 
         for _ in range(max(1, args.warmup)):
             e2e_step()

@@ -163,7 +163,7 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
   quant_shape(K, &R, &nt);
   const int logn = ilog2_exact(n);
   const bool xpose = logn >= 6;            // shared-memory transposes for n >= 64
-  const int per_sm = logn >= 8 ? 1 : 2;    // CTAs per SM (kernel launch bounds)
+  const int per_sm = 2;                    // CTAs per SM (kernel launch bounds)
   const int B = K / n;
   const uint32_t raw = uint32_t(kQuantRowsPerThread * R) * uint32_t(K) * 2u;  // one tile
   const uint32_t tile_bytes = (raw + 1023u) & ~1023u;
@@ -400,6 +400,8 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   if (desc->act_gran < HQ_PER_TOKEN || desc->act_gran > HQ_PER_TENSOR_STATIC)
     return HQ_ERR_INVALID_ARGUMENT;
   if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (desc->a_bits < 2 || desc->a_bits > 8 || desc->w_bits < 2 || desc->w_bits > 8)
+    return HQ_ERR_UNSUPPORTED;
   if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
   if (a_codes == nullptr || a_scale == nullptr || w_codes == nullptr || w_scale == nullptr ||
       Y == nullptr)
@@ -426,6 +428,11 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   std::memset(&p, 0, sizeof(p));
   p.a_scale = a_scale;
   p.a_scale_per_row = desc->act_gran == HQ_PER_TOKEN ? 1 : 0;
+  {
+    // |acc| <= 2^(a_bits-1) * 2^(w_bits-1) * K for codes within their declared widths
+    const double bound = std::ldexp(1.0, desc->a_bits - 1) * std::ldexp(1.0, desc->w_bits - 1) * K;
+    p.small_acc = bound < 4194304.0 ? 1 : 0;
+  }
   p.a_mean = a_mean;
   p.w_scale = w_scale;
   p.colsum = colsum;

@@ -37,6 +37,8 @@ constexpr int BK = 128;  // K bytes per stage: one 128-byte swizzle row
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemLimit = 227 * 1024;
+constexpr float kAccMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kAccMagicBits = 0x4B400000;
 
 template <int BN>
 struct GemmCfg {
@@ -275,16 +277,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const float4 sw = *reinterpret_cast<const float4*>(pw + 4 * g);
           const float4 cs = *reinterpret_cast<const float4*>(pw + C::HC + 4 * g);
           const float4 bb = *reinterpret_cast<const float4*>(pw + 2 * C::HC + 4 * g);
-          const float y0 = __fmaf_rn(__int2float_rn(int(r[4 * g + 0])), __fmul_rn(sx, sw.x),
-                                     __fmaf_rn(mt, cs.x, bb.x));
-          const float y1 = __fmaf_rn(__int2float_rn(int(r[4 * g + 1])), __fmul_rn(sx, sw.y),
-                                     __fmaf_rn(mt, cs.y, bb.y));
-          const float y2 = __fmaf_rn(__int2float_rn(int(r[4 * g + 2])), __fmul_rn(sx, sw.z),
-                                     __fmaf_rn(mt, cs.z, bb.z));
-          const float y3 = __fmaf_rn(__int2float_rn(int(r[4 * g + 3])), __fmul_rn(sx, sw.w),
-                                     __fmaf_rn(mt, cs.w, bb.w));
-          packed[2 * g] = pack_bf16x2(y0, y1);
-          packed[2 * g + 1] = pack_bf16x2(y2, y3);
+          f2 a01, a23;
+          if (p.small_acc) {
+            // |acc| < 2^22: acc + 1.5*2^23 is exact in fp32, so subtracting the
+            // magic constant recovers float(acc) without the conversion unit
+            const f2 mg = pk(kAccMagic, kAccMagic);
+            a01 = sub2(pk(__int_as_float(int(r[4 * g + 0]) + kAccMagicBits),
+                          __int_as_float(int(r[4 * g + 1]) + kAccMagicBits)), mg);
+            a23 = sub2(pk(__int_as_float(int(r[4 * g + 2]) + kAccMagicBits),
+                          __int_as_float(int(r[4 * g + 3]) + kAccMagicBits)), mg);
+          } else {
+            a01 = pk(__int2float_rn(int(r[4 * g + 0])), __int2float_rn(int(r[4 * g + 1])));
+            a23 = pk(__int2float_rn(int(r[4 * g + 2])), __int2float_rn(int(r[4 * g + 3])));
+          }
+          const f2 sx2 = pk(sx, sx), mt2 = pk(mt, mt);
+          // y = acc * (s_x * s_w) + (b + m * colsum)
+          const f2 y01 = fma2(a01, mul2(sx2, pk(sw.x, sw.y)), fma2(mt2, pk(cs.x, cs.y), pk(bb.x, bb.y)));
+          const f2 y23 = fma2(a23, mul2(sx2, pk(sw.z, sw.w)), fma2(mt2, pk(cs.z, cs.w), pk(bb.z, bb.w)));
+          packed[2 * g] = pack_bf16x2(y01.x, y01.y);
+          packed[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
         }
         // the previous chunk's TMA store must have finished reading the buffer
         if (lane == 0) bulk_wait_group_read<0>();

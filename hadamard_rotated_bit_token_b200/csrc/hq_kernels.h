@@ -47,6 +47,7 @@ size_t quant_smem_bytes(int nstage, uint32_t tile_bytes, int R, int K, int B, in
 struct GemmParams {
   const float* a_scale;   // [T] or [1]
   int a_scale_per_row;    // 1: a_scale[t]; 0: a_scale[0]
+  int small_acc;          // 1: every |acc| < 2^22 (from the declared code widths and K)
   const float* a_mean;    // [T] or null
   const float* w_scale;   // [N]
   const float* colsum;    // [N] or null

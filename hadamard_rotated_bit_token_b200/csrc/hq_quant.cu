@@ -137,7 +137,7 @@ size_t quant_smem_bytes(int nstage, uint32_t tile_bytes, int R, int K, int B, in
 // Each worker thread owns one 32-channel slice of RPT rows of a tile (rows r,
 // r + R, ...); the per-tile bookkeeping and multipliers are shared by them.
 template <int LOGN, int MODE, bool CENTER>
-__global__ void __launch_bounds__(kQuantThreads, (LOGN >= 8 ? 1 : 2))
+__global__ void __launch_bounds__(kQuantThreads, 2)
     quant_rows_kernel(const __grid_constant__ CUtensorMap tmX, const QuantParams p) {
   constexpr int N = 1 << LOGN;
   constexpr int LREG = LOGN < 5 ? LOGN : 5;        // index bits inside a thread's slice

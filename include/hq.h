@@ -154,7 +154,9 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X,
  *          when a_mean is NULL), bias_f32 fp32 [N] or NULL (b = 0).
  * Outputs: Y bf16 [T,N]; acc_debug int32 [T,N] or NULL (raw accumulators, for
  *          bit-exact checks; costs an extra 4 bytes per output).
- * The codes may hold any int8 values (the GEMM is generic int8). */
+ * Codes must lie within the declared widths: |a_codes| <= 2^(a_bits-1) and
+ * |w_codes| <= 2^(w_bits-1) (a_bits, w_bits in [2, 8]; 8 admits every int8
+ * value).  The epilogue converts accumulators exactly either way. */
 hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
                     const float* a_scale, const float* a_mean,
                     const int8_t* w_codes, const float* w_scale,

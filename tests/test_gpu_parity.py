@@ -204,7 +204,7 @@ def test_gemm_accumulators_bit_exact(hq, T, N, K):
     _, y_ref = oracle.epilogue(acc_ref, sx32.astype(np.float64), sw32.astype(np.float64),
                                colsum=cs32.astype(np.float64), bias=b32.astype(np.float64),
                                mean=m32.astype(np.float64))
-    desc = hq.LayerDesc(K, N, 16, act_gran=hq.HQ_PER_TOKEN)
+    desc = hq.LayerDesc(K, N, 16, a_bits=8, w_bits=8, act_gran=hq.HQ_PER_TOKEN)
     d = {k: torch.from_numpy(v).cuda() for k, v in
          dict(A=A, B=B, sx=sx32, sw=sw32, cs=cs32, b=b32, m=m32).items()}
     Y = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
