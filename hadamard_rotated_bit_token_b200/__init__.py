@@ -28,6 +28,7 @@ __all__ = [
     "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
+    "hq_debug_set_gemm_variant", "HQ_GEMM_AUTO", "HQ_GEMM_SINGLE_CTA", "HQ_GEMM_CTA_PAIR",
     "hq_quantize_act_noalloc", "HadamardQuantLinear",
 ]
 
@@ -38,13 +39,14 @@ HQ_PER_TOKEN, HQ_PER_TENSOR_DYNAMIC, HQ_PER_TENSOR_STATIC = 0, 1, 2
 HQ_CENTER_NONE, HQ_CENTER_TOKEN_MEAN = 0, 1
 HQ_CODES_I8 = 0
 HQ_FAULT_NONE, HQ_FAULT_QUANT_WITHHOLD_LOAD = 0, 1
+HQ_GEMM_AUTO, HQ_GEMM_SINGLE_CTA, HQ_GEMM_CTA_PAIR = 0, 1, 2
 STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED",
                 3: "HQ_ERR_MISALIGNED", 4: "HQ_ERR_CUDA", 5: "HQ_ERR_TIMEOUT",
                 6: "HQ_ERR_DEVICE"}
 EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare_weights",
             "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
             "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-            "hq_quantize_act_noalloc")
+            "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc")
 
 
 class HQError(RuntimeError):
@@ -103,9 +105,10 @@ def load_library():
         lib.hq_check_device_error.argtypes = [_vp]
         lib.hq_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
         lib.hq_debug_inject_fault.argtypes = [ctypes.c_int]
+        lib.hq_debug_set_gemm_variant.argtypes = [ctypes.c_int]
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
                      "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-                     "hq_quantize_act_noalloc"):
+                     "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -218,6 +221,11 @@ def hq_debug_set_wait_limit(nanoseconds: int):
 
 def hq_debug_inject_fault(kind: int):
     _check(load_library().hq_debug_inject_fault(int(kind)), "hq_debug_inject_fault")
+
+
+def hq_debug_set_gemm_variant(variant: int):
+    """Selects the GEMM kernel of later hq_linear calls (HQ_GEMM_*)."""
+    _check(load_library().hq_debug_set_gemm_variant(int(variant)), "hq_debug_set_gemm_variant")
 
 
 # ---------------------------------------------------------------------------

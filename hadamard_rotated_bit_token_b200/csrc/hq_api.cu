@@ -32,6 +32,7 @@ struct DeviceState {
   int cc_major = 0, cc_minor = 0;
   unsigned int* err = nullptr;
   bool quant_attr_set[8][4][2] = {};
+  int pair_clusters = -1;  // co-resident clusters of the CTA-pair GEMM (-1: not queried)
 };
 
 std::mutex g_mutex;
@@ -39,6 +40,7 @@ DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 unsigned long long g_wait_ns = 0;  // 0 -> default
 int g_fault = 0;
+int g_gemm_variant = 0;  // HQ_GEMM_AUTO
 
 unsigned long long wait_ns() { return g_wait_ns ? g_wait_ns : 2000000000ull; }
 
@@ -235,22 +237,45 @@ hq_status encode_out_bf16(CUtensorMap* m, const void* base, int64_t rows, int N)
   return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
 }
 
-int choose_bn(int64_t T, int N, int sms) {
+// GEMM kernel choice.  Both kernels are persistent with one CTA per SM, so a
+// launch takes about (tile rounds) x (time of one tile).  Measured on B200:
+// one 128 x n x 32 i8 MMA takes about 126 + n/16 cycles for n <= 256 --
+// nearly flat in n, so wide tiles win -- and the single-CTA main loop runs
+// about 15% behind that rate (operand loads).  The epilogue's traffic through
+// shared memory costs roughly 2000 cycles per 32-column chunk of each
+// epilogue warp (fitted to tile-width sweeps of several layer shapes).  The CTA pair halves the B bytes per
+// MMA but its 256 x 256 tiles carry twice the epilogue per CTA; it pays off
+// only for long main loops over wide N.
+struct GemmChoice {
+  bool pair;
+  int bn;  // single-CTA tile width
+};
+
+GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int variant) {
   static const int cands[] = {256, 192, 128, 64};
   const int64_t mt = (T + 127) / 128;
-  int best = 64;
+  const int64_t kb = (K + 127) / 128;
+  int best_bn = 64;
   double best_cost = 1e300;
   for (int bn : cands) {
-    const int64_t nt = (N + bn - 1) / bn;
-    const int64_t tiles = mt * nt;
-    const int64_t waves = (tiles + sms - 1) / sms;
-    const double cost = double(waves) * double(bn + 32);
+    const int64_t tiles = mt * ((N + bn - 1) / bn);
+    const int64_t rounds = (tiles + sms - 1) / sms;
+    const double tile = double(kb) * 4.0 * (126.0 + bn / 16.0) * 1.15 + 2000.0 * (bn / 64);
+    const double cost = double(rounds) * tile;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
-      best = bn;
+      best_bn = bn;
     }
   }
-  return best;
+  if (variant == HQ_GEMM_SINGLE_CTA || pair_clusters <= 0) return {false, best_bn};
+  if (variant == HQ_GEMM_CTA_PAIR) return {true, 256};
+  // automatic: the pair for long main loops (>= 20 K blocks) over N in whole
+  // 256-column tiles, when it needs no more tile rounds than the best single
+  const int64_t ptiles = ((T + 255) / 256) * ((N + 255) / 256);
+  const int64_t prounds = (ptiles + pair_clusters - 1) / pair_clusters;
+  const int64_t srounds = (mt * ((N + best_bn - 1) / best_bn) + sms - 1) / sms;
+  const bool pair = kb >= 20 && N % 256 == 0 && prounds <= srounds;
+  return {pair, best_bn};
 }
 
 }  // namespace
@@ -416,11 +441,26 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   hq_status s = device_state(&dev);
   if (s != HQ_OK) return s;
   const int K = desc->K, N = desc->N;
-  const int bn = choose_bn(T, N, dev->sm_count);
+  if (dev->pair_clusters < 0) {
+    int c = 0;
+    if (gemm_pair_max_clusters(&c) != cudaSuccess) {
+      (void)cudaGetLastError();
+      c = 0;
+    }
+    dev->pair_clusters = c;
+  }
+  int variant;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    variant = g_gemm_variant;
+  }
+  if (variant == HQ_GEMM_CTA_PAIR && dev->pair_clusters <= 0) return HQ_ERR_UNSUPPORTED;
+  const GemmChoice gc = choose_gemm(T, N, K, dev->sm_count, dev->pair_clusters, variant);
+  const int bn = gc.pair ? 256 : gc.bn;
   CUtensorMap ta, tb, ty;
   s = encode_kmajor_i8(&ta, a_codes, T, K, 128);
   if (s != HQ_OK) return s;
-  s = encode_kmajor_i8(&tb, w_codes, N, K, bn);
+  s = encode_kmajor_i8(&tb, w_codes, N, K, gc.pair ? 128 : bn);
   if (s != HQ_OK) return s;
   s = encode_out_bf16(&ty, Y, T, N);
   if (s != HQ_OK) return s;
@@ -442,13 +482,21 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.T = T;
   p.N = N;
   p.K = K;
-  p.num_m_tiles = int((T + 127) / 128);
-  p.num_n_tiles = (N + bn - 1) / bn;
   p.err = dev->err;
   p.wait_ns = wait_ns();
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (gc.pair) {
+    p.num_m_tiles = int((T + 255) / 256);
+    p.num_n_tiles = (N + 255) / 256;
+    const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
+    const int clusters = int(tiles < dev->pair_clusters ? tiles : dev->pair_clusters);
+    return from_cuda(launch_gemm_pair(&ta, &tb, &ty, p, clusters, st));
+  }
+  p.num_m_tiles = int((T + 127) / 128);
+  p.num_n_tiles = (N + bn - 1) / bn;
   const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
   const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
-  return from_cuda(launch_gemm(bn, &ta, &tb, &ty, p, grid, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_gemm(bn, &ta, &tb, &ty, p, grid, st));
 }
 
 hq_status hq_check_device_error(hq_stream_t stream) {
@@ -472,6 +520,14 @@ hq_status hq_check_device_error(hq_stream_t stream) {
 hq_status hq_debug_set_wait_limit(uint64_t nanoseconds) {
   std::lock_guard<std::mutex> lock(g_mutex);
   g_wait_ns = nanoseconds;
+  return HQ_OK;
+}
+
+hq_status hq_debug_set_gemm_variant(int variant) {
+  if (variant != HQ_GEMM_AUTO && variant != HQ_GEMM_SINGLE_CTA && variant != HQ_GEMM_CTA_PAIR)
+    return HQ_ERR_INVALID_ARGUMENT;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_gemm_variant = variant;
   return HQ_OK;
 }
 

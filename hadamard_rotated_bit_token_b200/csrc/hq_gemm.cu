@@ -6,22 +6,34 @@
 //                    + b[n] + mu_t * colsum[n] )      (b~ = b + mu W~, HadaNorm Eq. (1))
 //
 // A = activation codes [T,K] int8, B = weight codes [N,K] int8, both K-major.
-// Persistent CTAs (one per SM) walk output tiles of 128 x BN.  Roles:
+// Two kernels share one warp layout (320 threads, one CTA per SM):
 //   warp 0      one thread issues TMA tensor loads (128-byte swizzle) of the
-//               A and B K-slices into a ring of shared-memory stages;
-//   warp 1      allocates tensor memory; one thread issues tcgen05.mma
-//               (128 x BN x 32 per instruction) and commits each stage back
-//               to the producer and each finished accumulator to the epilogue;
+//               A and B K-slices into a ring of shared-memory stages, and per
+//               output tile bulk copies of the tile's columns of s_w, colsum
+//               and bias into a two-slot parameter ring;
+//   warp 1      allocates tensor memory; one thread issues tcgen05.mma and
+//               commits each stage back to the producer and each finished
+//               accumulator to the epilogue;
 //   warps 2..9  the epilogue: two warps per 32-lane quarter of tensor memory,
-//               each taking half of the tile's columns.  Per tile a warp
-//               stages its columns' s_w, colsum and bias in shared memory;
-//               per 32-column chunk it reads the accumulator (tcgen05.ld),
-//               applies the epilogue in fp32, writes bf16 to a 64-byte
-//               swizzled shared buffer and lets a TMA tensor store write the
-//               32 x 32 box to Y (clipped at the tensor's edges).
+//               each taking half of the tile's columns.  Per 32-column chunk a
+//               warp reads the accumulator (tcgen05.ld), applies the epilogue
+//               in fp32 (row scale and mean from registers, prefetched one
+//               tile ahead; column parameters from the ring), writes bf16 to
+//               a 64-byte swizzled shared buffer and lets a TMA tensor store
+//               write the 32 x 32 box to Y (clipped at the tensor's edges).
+//
+// gemm_i8_kernel<BN>: one CTA per 128 x BN output tile (BN 64..256).
+// gemm_i8_pair_kernel: a cluster of two CTAs per 256 x 256 output tile with
+//   the CTA-pair MMA (cta_group::2, M = 256): each CTA loads 128 rows of A and
+//   128 rows of B into its own shared memory, so one SM moves half the B
+//   bytes per MMA that the single-CTA kernel moves.  Both CTAs' copies
+//   complete on the even CTA's stage barrier, whose producer expects the
+//   bytes of both; the even CTA issues the MMAs and commits to both CTAs.
 // Two accumulators in tensor memory let the epilogue of one tile overlap the
 // main loop of the next.  Every wait is bounded; a timeout records
-// HQ_ERR_TIMEOUT in the device error word and the CTA drains and exits.
+// HQ_ERR_TIMEOUT in the device error word, and the CTA waits for every copy it
+// started (or, in the pair kernel, the even CTA for the pair's copies) before
+// it exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -37,34 +49,19 @@ constexpr int BK = 128;  // K bytes per stage: one 128-byte swizzle row
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kStageBox = 2048;           // one 32 x 32 bf16 output box
 constexpr float kAccMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr int kAccMagicBits = 0x4B400000;
 
-template <int BN>
-struct GemmCfg {
-  static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int HC = BN / 2;  // columns per epilogue warp
-  // per epilogue warp: 2 KB output staging (1024-aligned) + params [3][HC]
-  static constexpr int EPI_STAGE_BYTES = 2048;
-  static constexpr int EPI_PARAM_BYTES = 3 * HC * 4;
-  static constexpr int EPI_BYTES = kEpiWarps * (EPI_STAGE_BYTES + EPI_PARAM_BYTES);
-  static constexpr int CTL_BYTES = 256;
-  static constexpr int STAGES_RAW = (kSmemLimit - 1024 - EPI_BYTES - CTL_BYTES - 1024) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
-  // instruction descriptor: D s32 (bits 4-5 = 2), A and B signed int8 (bits
-  // 7-9 = 1, 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
-  static constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) |
-                                    (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
-  static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + EPI_BYTES + CTL_BYTES + 1024;
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "two 32-column-aligned halves");
-  static_assert(B_BYTES % 1024 == 0, "stage bases must stay 1024-byte aligned");
-  static_assert(STAGES >= 2, "shared memory budget");
-  static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
-};
+// instruction descriptor: D s32 (bits 4-5 = 2), A and B signed int8 (bits
+// 7-9 = 1, 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
+constexpr uint32_t i8_idesc(int m, int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+constexpr int tmem_cols_for(int cols) {
+  return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
+}
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA
 // with 128-byte swizzling: rows of 128 bytes, 8-row (1024-byte) swizzle atoms
@@ -85,7 +82,171 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ------------------------------------------------------- parameter ring
+// Slot a holds the columns [n0, n0 + W) of one output tile: s_w at [0, W),
+// colsum at [W, 2W), bias at [2W, 3W) (fp32).  An absent vector, and every
+// column past N, reads zero or a finite stale value: the ring is zeroed at
+// kernel start and absent vectors are never copied.
+template <int W>
+__device__ __forceinline__ void param_ring_zero(float* ring, int tid, int nthreads) {
+  for (int i = tid; i < 2 * 3 * W; i += nthreads) ring[i] = 0.0f;
+}
+
+// Producer side: copies the tile's columns [n0, min(n0 + W, N)) into `slot`,
+// completion counted on `bar`.
+template <int W>
+__device__ __forceinline__ void param_ring_load(const GemmParams& p, float* slot, int n0,
+                                                uint64_t* bar) {
+  const int cols = p.N - n0 < W ? p.N - n0 : W;
+  const uint32_t nb = uint32_t(cols) * 4u;  // N % 16 == 0: a multiple of 64 bytes
+  const bool cs = p.a_mean != nullptr && p.colsum != nullptr;
+  const bool bi = p.bias != nullptr;
+  mbar_arrive_expect_tx(bar, nb * (1u + (cs ? 1u : 0u) + (bi ? 1u : 0u)));
+  bulk_load(slot, p.w_scale + n0, nb, bar);
+  if (cs) bulk_load(slot + W, p.colsum + n0, nb, bar);
+  if (bi) bulk_load(slot + 2 * W, p.bias + n0, nb, bar);
+}
+
+// ------------------------------------------------------------- epilogue
+// Per-warp state of the epilogue for one output tile.
+struct EpiTile {
+  int row0;      // first output row of this warp's 32 rows
+  int col_base;  // first output column of this warp's columns
+  int64_t row;   // this thread's output row
+  bool row_ok;   // row < T
+  float sx, mt;  // this row's activation scale and mean
+};
+
+// This thread's row scale and mean (zero past T).
+__device__ __forceinline__ void load_row_params(const GemmParams& p, int64_t row, float& sx,
+                                                float& mt) {
+  sx = 0.0f;
+  mt = 0.0f;
+  if (row < p.T) {
+    sx = p.a_scale_per_row ? p.a_scale[row] : p.a_scale[0];
+    mt = p.a_mean ? p.a_mean[row] : 0.0f;
+  }
+}
+
+// One 32-column chunk c of the warp's columns: accumulators r (this thread's
+// row) -> fp32 epilogue -> bf16 -> swizzled staging buffer -> TMA store.
+// prm points at the warp's first column in a parameter slot of width W.
+// NBUF staging buffers of kStageBox bytes rotate; `nstore` counts the stores
+// this warp issued (warp-uniform).
+template <int W, int NBUF>
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, const CUtensorMap* tmY,
+                                          const uint32_t (&r)[32], int c, const EpiTile& e,
+                                          const float* prm, uint8_t* stg, int lane,
+                                          uint32_t& nstore) {
+  const int col0 = e.col_base + c * 32;
+  const float* pw = prm + c * 32;
+  uint32_t packed[16];
+  const f2 sx2 = pk(e.sx, e.sx), mt2 = pk(e.mt, e.mt);
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const float4 sw = *reinterpret_cast<const float4*>(pw + 4 * g);
+    const float4 cs = *reinterpret_cast<const float4*>(pw + W + 4 * g);
+    const float4 bb = *reinterpret_cast<const float4*>(pw + 2 * W + 4 * g);
+    f2 a01, a23;
+    if (p.small_acc) {
+      // |acc| < 2^22: acc + 1.5*2^23 is exact in fp32, so subtracting the
+      // magic constant recovers float(acc) without the conversion unit
+      const f2 mg = pk(kAccMagic, kAccMagic);
+      a01 = sub2(pk(__int_as_float(int(r[4 * g + 0]) + kAccMagicBits),
+                    __int_as_float(int(r[4 * g + 1]) + kAccMagicBits)), mg);
+      a23 = sub2(pk(__int_as_float(int(r[4 * g + 2]) + kAccMagicBits),
+                    __int_as_float(int(r[4 * g + 3]) + kAccMagicBits)), mg);
+    } else {
+      a01 = pk(__int2float_rn(int(r[4 * g + 0])), __int2float_rn(int(r[4 * g + 1])));
+      a23 = pk(__int2float_rn(int(r[4 * g + 2])), __int2float_rn(int(r[4 * g + 3])));
+    }
+    // y = acc * (s_x * s_w) + (b + m * colsum)
+    const f2 y01 = fma2(a01, mul2(sx2, pk(sw.x, sw.y)), fma2(mt2, pk(cs.x, cs.y), pk(bb.x, bb.y)));
+    const f2 y23 = fma2(a23, mul2(sx2, pk(sw.z, sw.w)), fma2(mt2, pk(cs.z, cs.w), pk(bb.z, bb.w)));
+    packed[2 * g] = pack_bf16x2(y01.x, y01.y);
+    packed[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
+  }
+  const bool do_store = col0 < p.N && e.row0 < p.T;  // warp-uniform
+  if (do_store) {
+    uint8_t* buf = stg + (nstore % NBUF) * kStageBox;
+    // the store that last used this buffer must have finished reading it
+    if (lane == 0) bulk_wait_group_read<NBUF - 1>();
+    __syncwarp();
+    const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this thread's row
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ swz) << 4)) =
+          make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmY, buf, col0, e.row0);
+      bulk_commit_group();
+    }
+    ++nstore;
+  }
+  if (p.acc_debug && e.row_ok) {
+    int32_t* arow = p.acc_debug + e.row * p.N;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (col0 + 4 * g < p.N) {
+        *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
+            make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+      }
+    }
+  }
+}
+
+// The warp's HC columns of one accumulator starting at tensor-memory address
+// t_addr (lane quarter already encoded): two chunks per tensor-memory wait.
+template <int HC, int W, int NBUF>
+__device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap* tmY,
+                                         uint32_t t_addr, const EpiTile& e, const float* prm,
+                                         uint8_t* stg, int lane, uint32_t& nstore) {
+  constexpr int NCH = HC / 32;
+#pragma unroll 1
+  for (int c = 0; c + 1 < NCH; c += 2) {
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(t_addr + uint32_t(c * 32), r0);
+    tmem_ld_32x32b_x32(t_addr + uint32_t(c * 32 + 32), r1);
+    tmem_wait_ld();
+    epi_chunk<W, NBUF>(p, tmY, r0, c, e, prm, stg, lane, nstore);
+    epi_chunk<W, NBUF>(p, tmY, r1, c + 1, e, prm, stg, lane, nstore);
+  }
+  if (NCH & 1) {
+    uint32_t r0[32];
+    tmem_ld_32x32b_x32(t_addr + uint32_t((NCH - 1) * 32), r0);
+    tmem_wait_ld();
+    epi_chunk<W, NBUF>(p, tmY, r0, NCH - 1, e, prm, stg, lane, nstore);
+  }
+}
+
 }  // namespace
+
+// ------------------------------------------------------- single-CTA kernel
+template <int BN>
+struct GemmCfg {
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int HC = BN / 2;  // columns per epilogue warp
+  static constexpr int NBUF = 1;     // output staging buffers per epilogue warp
+  static constexpr int EPI_STAGE_BYTES = NBUF * kStageBox;
+  static constexpr int RING_BYTES = 2 * 3 * BN * 4;
+  static constexpr int CTL_BYTES = 256;
+  static constexpr int FIXED = kEpiWarps * EPI_STAGE_BYTES + RING_BYTES + CTL_BYTES + 1024;
+  static constexpr int STAGES_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int TMEM_COLS = tmem_cols_for(2 * BN);
+  static constexpr uint32_t IDESC = i8_idesc(BM, BN);
+  static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + FIXED;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "two 32-column-aligned halves");
+  static_assert(B_BYTES % 1024 == 0, "stage bases must stay 1024-byte aligned");
+  static_assert(STAGES >= 2, "shared memory budget");
+  static_assert(16 * STAGES + 80 <= CTL_BYTES, "barrier block");
+  static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
+};
 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -97,13 +258,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + size_t(C::STAGES) * C::A_BYTES;
-  uint8_t* epi_stage = sB + size_t(C::STAGES) * C::B_BYTES;  // 1024-aligned, [8][2 KB]
-  float* epi_param = reinterpret_cast<float*>(epi_stage + kEpiWarps * C::EPI_STAGE_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi_stage + C::EPI_BYTES);
+  uint8_t* epi_stage = sB + size_t(C::STAGES) * C::B_BYTES;  // 1024-aligned
+  float* ring = reinterpret_cast<float*>(epi_stage + kEpiWarps * C::EPI_STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ring) + C::RING_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* tfull = empty + C::STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tfull = empty + C::STAGES;   // [2] accumulator complete
+  uint64_t* tempty = tfull + 2;          // [2] accumulator drained by the epilogue
+  uint64_t* pfull = tempty + 2;          // [2] parameter slot loaded
+  uint64_t* pempty = pfull + 2;          // [2] parameter slot read by the epilogue
+  uint64_t* drain = pempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -111,6 +274,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   const WaitCtl wc{p.err, p.wait_ns};
 
+  param_ring_zero<BN>(ring, threadIdx.x, kGemmThreads);
+  fence_proxy_async_smem();  // the zeros precede the ring's bulk copies
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -119,6 +284,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kEpiWarps);  // one arrival per epilogue warp
+      mbar_init(&pfull[a], 1);
+      mbar_init(&pempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -144,11 +311,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // ---------------------------------------------------------- producer
       int stage = 0;
       uint32_t phase = 0;
-      int issued = 0;
+      int issued = 0, tiles_issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m_idx = tile % p.num_m_tiles;
         const int n_idx = tile / p.num_m_tiles;
+        const int a = tiles_issued & 1;
+        if (*abort_flag || !mbar_wait(&pempty[a], ((tiles_issued >> 1) & 1) ^ 1u, wc)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        param_ring_load<BN>(p, ring + a * 3 * BN, n_idx * BN, &pfull[a]);
+        ++tiles_issued;
         for (int kb = 0; kb < KB; ++kb) {
           if (*abort_flag || !mbar_wait(&empty[stage], phase ^ 1u, wc)) {
             *abort_flag = 1;
@@ -166,7 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       if (!ok) {
-        // let the loads still in flight land before the CTA can exit
+        // let the copies still in flight land before the CTA can exit
         int s = stage;
         uint32_t ph = phase;
         for (int i = 0; i < C::STAGES && i < issued; ++i) {
@@ -176,6 +351,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           (void)mbar_wait(&full[s], ph, wc);
         }
+        for (int j = tiles_issued > 2 ? tiles_issued - 2 : 0; j < tiles_issued; ++j)
+          (void)mbar_wait(&pfull[j & 1], uint32_t(j >> 1) & 1u, wc);
       }
     }
   } else if (warp == 1) {
@@ -230,101 +407,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;    // TMEM lanes [32*quarter, 32*quarter + 32)
     const int half = ew >> 2;        // columns [half*HC, half*HC + HC) of the tile
     uint8_t* stg = epi_stage + ew * C::EPI_STAGE_BYTES;
-    float* prm = epi_param + ew * (3 * C::HC);
-    const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this thread's row
+    uint32_t nstore = 0;
     int acc_iter = 0;
+    float sx_next = 0.0f, mt_next = 0.0f;
+    if (int(blockIdx.x) < num_tiles)
+      load_row_params(p, int64_t(int(blockIdx.x) % p.num_m_tiles) * BM + quarter * 32 + lane,
+                      sx_next, mt_next);
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++acc_iter) {
       const int acc = acc_iter & 1;
       const uint32_t acc_phase = (acc_iter >> 1) & 1;
       const int m_idx = tile % p.num_m_tiles;
       const int n_idx = tile / p.num_m_tiles;
-      const int col_base = n_idx * BN + half * C::HC;
-      // this warp's columns: scale, colsum, bias (coalesced, before the wait)
-      for (int c = lane; c < C::HC; c += 32) {
-        const int gc = col_base + c;
-        const bool in = gc < p.N;
-        prm[c] = in ? p.w_scale[gc] : 0.0f;
-        prm[C::HC + c] = (in && p.a_mean) ? p.colsum[gc] : 0.0f;
-        prm[2 * C::HC + c] = (in && p.bias) ? p.bias[gc] : 0.0f;
-      }
-      const int row0 = m_idx * BM + quarter * 32;
-      const int64_t row = int64_t(row0) + lane;
-      const bool row_ok = row < p.T;
-      float sx = 0.0f, mt = 0.0f;
-      if (row_ok) {
-        sx = p.a_scale_per_row ? p.a_scale[row] : p.a_scale[0];
-        mt = p.a_mean ? p.a_mean[row] : 0.0f;
-      }
-      __syncwarp();
-      const bool got = !(*abort_flag) && mbar_wait(&tfull[acc], acc_phase, wc);
+      EpiTile e;
+      e.row0 = m_idx * BM + quarter * 32;
+      e.col_base = n_idx * BN + half * C::HC;
+      e.row = int64_t(e.row0) + lane;
+      e.row_ok = e.row < p.T;
+      e.sx = sx_next;
+      e.mt = mt_next;
+      const int next = tile + int(gridDim.x);
+      if (next < num_tiles)  // next tile's row parameters, in flight during this one
+        load_row_params(p, int64_t(next % p.num_m_tiles) * BM + quarter * 32 + lane, sx_next,
+                        mt_next);
+      const bool got = !(*abort_flag) && mbar_wait(&tfull[acc], acc_phase, wc) &&
+                       mbar_wait(&pfull[acc], acc_phase, wc);
       if (!__all_sync(0xffffffffu, got)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t t_row = tmem_base + uint32_t(acc * BN + half * C::HC) +
-                             (uint32_t(quarter * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < C::HC / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + uint32_t(c * 32), r);
-        tmem_wait_ld();
-        const int col0 = col_base + c * 32;
-        const float* pw = prm + c * 32;
-        uint32_t packed[16];
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const float4 sw = *reinterpret_cast<const float4*>(pw + 4 * g);
-          const float4 cs = *reinterpret_cast<const float4*>(pw + C::HC + 4 * g);
-          const float4 bb = *reinterpret_cast<const float4*>(pw + 2 * C::HC + 4 * g);
-          f2 a01, a23;
-          if (p.small_acc) {
-            // |acc| < 2^22: acc + 1.5*2^23 is exact in fp32, so subtracting the
-            // magic constant recovers float(acc) without the conversion unit
-            const f2 mg = pk(kAccMagic, kAccMagic);
-            a01 = sub2(pk(__int_as_float(int(r[4 * g + 0]) + kAccMagicBits),
-                          __int_as_float(int(r[4 * g + 1]) + kAccMagicBits)), mg);
-            a23 = sub2(pk(__int_as_float(int(r[4 * g + 2]) + kAccMagicBits),
-                          __int_as_float(int(r[4 * g + 3]) + kAccMagicBits)), mg);
-          } else {
-            a01 = pk(__int2float_rn(int(r[4 * g + 0])), __int2float_rn(int(r[4 * g + 1])));
-            a23 = pk(__int2float_rn(int(r[4 * g + 2])), __int2float_rn(int(r[4 * g + 3])));
-          }
-          const f2 sx2 = pk(sx, sx), mt2 = pk(mt, mt);
-          // y = acc * (s_x * s_w) + (b + m * colsum)
-          const f2 y01 = fma2(a01, mul2(sx2, pk(sw.x, sw.y)), fma2(mt2, pk(cs.x, cs.y), pk(bb.x, bb.y)));
-          const f2 y23 = fma2(a23, mul2(sx2, pk(sw.z, sw.w)), fma2(mt2, pk(cs.z, cs.w), pk(bb.z, bb.w)));
-          packed[2 * g] = pack_bf16x2(y01.x, y01.y);
-          packed[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
-        }
-        // the previous chunk's TMA store must have finished reading the buffer
-        if (lane == 0) bulk_wait_group_read<0>();
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ swz) << 4)) =
-              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && col0 < p.N && row0 < p.T) {
-          tma_store_2d(&tmY, stg, col0, row0);
-          bulk_commit_group();
-        }
-        if (p.acc_debug && row_ok) {
-          int32_t* arow = p.acc_debug + row * p.N;
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            if (col0 + 4 * g < p.N) {
-              *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
-                  make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
-            }
-          }
-        }
-      }
+      const uint32_t t_addr = tmem_base + uint32_t(acc * BN + half * C::HC) +
+                              (uint32_t(quarter * 32) << 16);
+      epi_tile<C::HC, BN, C::NBUF>(p, &tmY, t_addr, e, ring + acc * 3 * BN + half * C::HC, stg,
+                                   lane, nstore);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        mbar_arrive(&tempty[acc]);
+        mbar_arrive(&pempty[acc]);
+      }
     }
     if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
     __syncwarp();
@@ -335,6 +456,279 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------- CTA-pair kernel
+struct PairCfg {
+  static constexpr int BN = 256;          // output columns per pair tile (N of each MMA)
+  static constexpr int BM_PAIR = 2 * BM;  // output rows per pair tile (M of each MMA)
+  static constexpr int B_ROWS = BN / 2;   // rows of B each CTA holds
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = B_ROWS * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+  static constexpr int HC = BN / 2;  // columns per epilogue warp
+  static constexpr int NBUF = 2;     // output staging buffers per epilogue warp
+  static constexpr int EPI_STAGE_BYTES = NBUF * kStageBox;
+  static constexpr int RING_BYTES = 2 * 3 * BN * 4;
+  static constexpr int CTL_BYTES = 512;
+  static constexpr int FIXED = kEpiWarps * EPI_STAGE_BYTES + RING_BYTES + CTL_BYTES + 1024;
+  static constexpr int STAGES_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int TMEM_COLS = tmem_cols_for(2 * BN);
+  static constexpr uint32_t IDESC = i8_idesc(BM_PAIR, BN);
+  static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + FIXED;
+  static_assert(B_BYTES % 1024 == 0, "stage bases must stay 1024-byte aligned");
+  static_assert(STAGES >= 2, "shared memory budget");
+  static_assert(16 * STAGES + 96 <= CTL_BYTES, "barrier block");
+  static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
+};
+
+// Clusters of two CTAs; CTA rank r of a cluster owns rows [128 r, 128 r + 128)
+// of every 256-row pair tile (its A rows and its half of the accumulator) and
+// B rows [128 r, 128 r + 128) of the tile's 256 columns.  Barriers, all in
+// each CTA's own shared memory (those marked "rank 0" used only there):
+//   full[s]    (rank 0) stage s of both CTAs landed: rank 0's producer
+//              expects the bytes of both and both CTAs' copies count on it;
+//   empty[s]   the MMAs have read stage s (pair commit to both CTAs);
+//   tfull[a]   accumulator a is complete (pair commit to both CTAs);
+//   tempty[a]  (rank 0) the 16 epilogue warps of the pair have read
+//              accumulator a (remote arrivals);
+//   pfull[a], pempty[a]   this CTA's parameter slot a loaded / read;
+//   drain      every MMA issued has completed (pair commit to both CTAs).
+// At exit each producer posts the number of stages it loaded to rank 0,
+// whose producer then waits until every copy of either CTA has landed: it
+// supplies the missing arrival or cancels the missing bytes of a stage that
+// only one CTA loaded (after a bounded wait gave up).
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + size_t(C::STAGES) * C::A_BYTES;
+  uint8_t* epi_stage = sB + size_t(C::STAGES) * C::B_BYTES;  // 1024-aligned
+  float* ring = reinterpret_cast<float*>(epi_stage + kEpiWarps * C::EPI_STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ring) + C::RING_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* pfull = tempty + 2;
+  uint64_t* pempty = pfull + 2;
+  uint64_t* drain = pempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* issued_by = tmem_slot + 2;  // [2], rank 0: stages each CTA loaded
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const WaitCtl wc{p.err, p.wait_ns};
+
+  param_ring_zero<C::BN>(ring, threadIdx.x, kGemmThreads);
+  fence_proxy_async_smem();  // the zeros precede the ring's bulk copies
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kEpiWarps);
+      mbar_init(&pfull[a], 1);
+      mbar_init(&pempty[a], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    issued_by[0] = issued_by[1] = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised and tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.num_m_tiles * p.num_n_tiles;
+  const int cluster_id = int(blockIdx.x >> 1);
+  const int num_clusters = int(gridDim.x >> 1);
+  const int KB = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      const uint32_t full0 = mapa_shared(full, 0);  // rank 0's full[0]
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0, tiles_issued = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        const int m_idx = tile % p.num_m_tiles;
+        const int n_idx = tile / p.num_m_tiles;
+        const int a_row = m_idx * C::BM_PAIR + int(rank) * BM;
+        const int b_row = n_idx * C::BN + int(rank) * C::B_ROWS;
+        const int a = tiles_issued & 1;
+        if (*abort_flag || !mbar_wait(&pempty[a], ((tiles_issued >> 1) & 1) ^ 1u, wc)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        param_ring_load<C::BN>(p, ring + a * 3 * C::BN, n_idx * C::BN, &pfull[a]);
+        ++tiles_issued;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait<true>(&empty[stage], phase ^ 1u, wc)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          const uint32_t bar = full0 + uint32_t(stage) * 8u;
+          tma_load_2d_pair(sA + size_t(stage) * C::A_BYTES, &tmA, kb * BK, a_row, bar);
+          tma_load_2d_pair(sB + size_t(stage) * C::B_BYTES, &tmB, kb * BK, b_row, bar);
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        for (int j = tiles_issued > 2 ? tiles_issued - 2 : 0; j < tiles_issued; ++j)
+          (void)mbar_wait(&pfull[j & 1], uint32_t(j >> 1) & 1u, wc);
+      }
+      st_shared_cluster_u32(mapa_shared(&issued_by[rank], 0), uint32_t(issued));
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------ MMA issuer (rank 0)
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc_iter = 0;
+      bool ok = true;
+      const uint32_t a_base = smem_u32(sA);
+      const uint32_t b_base = smem_u32(sB);
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++acc_iter) {
+        const int acc = acc_iter & 1;
+        const uint32_t acc_phase = (acc_iter >> 1) & 1;
+        if (*abort_flag || !mbar_wait<true>(&tempty[acc], acc_phase ^ 1u, wc)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * C::BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (*abort_flag || !mbar_wait<true>(&full[stage], phase, wc)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(a_base + uint32_t(stage) * C::A_BYTES);
+          const uint64_t bdesc = sw128_kmajor_desc(b_base + uint32_t(stage) * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k) {
+            // advance 32 bytes along K inside the swizzle row (encoded >> 4)
+            mma_i8_pair(d_tmem, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), C::IDESC,
+                        (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[stage], 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc], 0x3);
+      }
+      // every issued MMA completes before either CTA releases its shared
+      // memory or tensor memory
+      mma_commit_pair(drain, 0x3);
+      (void)mbar_wait<true>(drain, 0, wc);
+    } else if (lane == 0) {
+      (void)mbar_wait<true>(drain, 0, wc);  // rank 1: the pair's last commit has landed
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int ew = warp - 2;         // 0 .. 7
+    const int quarter = warp & 3;    // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int half = ew >> 2;        // columns [half*HC, half*HC + HC) of the tile
+    uint8_t* stg = epi_stage + ew * C::EPI_STAGE_BYTES;
+    const uint32_t tempty0 = mapa_shared(tempty, 0);
+    const int row_off = int(rank) * BM + quarter * 32 + lane;
+    uint32_t nstore = 0;
+    int acc_iter = 0;
+    float sx_next = 0.0f, mt_next = 0.0f;
+    if (cluster_id < num_tiles)
+      load_row_params(p, int64_t(cluster_id % p.num_m_tiles) * C::BM_PAIR + row_off, sx_next,
+                      mt_next);
+    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++acc_iter) {
+      const int acc = acc_iter & 1;
+      const uint32_t acc_phase = (acc_iter >> 1) & 1;
+      const int m_idx = tile % p.num_m_tiles;
+      const int n_idx = tile / p.num_m_tiles;
+      EpiTile e;
+      e.row0 = m_idx * C::BM_PAIR + int(rank) * BM + quarter * 32;
+      e.col_base = n_idx * C::BN + half * C::HC;
+      e.row = int64_t(e.row0) + lane;
+      e.row_ok = e.row < p.T;
+      e.sx = sx_next;
+      e.mt = mt_next;
+      const int next = tile + num_clusters;
+      if (next < num_tiles)  // next tile's row parameters, in flight during this one
+        load_row_params(p, int64_t(next % p.num_m_tiles) * C::BM_PAIR + row_off, sx_next,
+                        mt_next);
+      const bool got = !(*abort_flag) && mbar_wait<true>(&tfull[acc], acc_phase, wc) &&
+                       mbar_wait(&pfull[acc], acc_phase, wc);
+      if (!__all_sync(0xffffffffu, got)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_addr = tmem_base + uint32_t(acc * C::BN + half * C::HC) +
+                              (uint32_t(quarter * 32) << 16);
+      epi_tile<C::HC, C::BN, C::NBUF>(p, &tmY, t_addr, e, ring + acc * 3 * C::BN + half * C::HC,
+                                      stg, lane, nstore);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_remote(tempty0 + uint32_t(acc) * 8u);
+        mbar_arrive(&pempty[acc]);
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both producers have posted their stage counts
+  if (rank == 0 && threadIdx.x == 0) {
+    // every stage copy of either CTA lands before either CTA can exit
+    const int L = int(issued_by[0]), P = int(issued_by[1]);
+    const int hi = L > P ? L : P;
+    for (int s = 0; s < C::STAGES && s < hi; ++s) {
+      const int i = s + ((hi - 1 - s) / C::STAGES) * C::STAGES;  // last copy into stage s
+      const bool by0 = i < L, by1 = i < P;
+      if (by0 && !by1) mbar_complete_tx(&full[s], C::STAGE_BYTES);
+      if (by1 && !by0) mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+      (void)mbar_wait<true>(&full[s], uint32_t(i / C::STAGES) & 1u, wc);
+    }
+  }
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -367,6 +761,43 @@ cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const vo
   }
 }
 
+static cudaError_t configure_pair() {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_pair_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(PairCfg::SMEM));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t gemm_pair_max_clusters(int* clusters) {
+  cudaError_t e = configure_pair();
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(sms & ~1));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = PairCfg::SMEM;
+  return cudaOccupancyMaxActiveClusters(clusters, gemm_i8_pair_kernel, &cfg);
+}
+
+cudaError_t launch_gemm_pair(const void* tmap_a, const void* tmap_b, const void* tmap_y,
+                             const GemmParams& p, int clusters, cudaStream_t st) {
+  cudaError_t e = configure_pair();
+  if (e != cudaSuccess) return e;
+  gemm_i8_pair_kernel<<<2 * clusters, kGemmThreads, PairCfg::SMEM, st>>>(
+      *reinterpret_cast<const CUtensorMap*>(tmap_a), *reinterpret_cast<const CUtensorMap*>(tmap_b),
+      *reinterpret_cast<const CUtensorMap*>(tmap_y), p);
+  return cudaGetLastError();
+}
+
 size_t gemm_smem_bytes(int bn) {
   switch (bn) {
     case 64: return GemmCfg<64>::SMEM;
@@ -376,6 +807,9 @@ size_t gemm_smem_bytes(int bn) {
     default: return 0;
   }
 }
+
+size_t gemm_pair_smem_bytes() { return PairCfg::SMEM; }
+int gemm_pair_stages() { return PairCfg::STAGES; }
 
 int gemm_threads() { return kGemmThreads; }
 

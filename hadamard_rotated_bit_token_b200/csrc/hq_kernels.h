@@ -72,6 +72,17 @@ cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const vo
 size_t gemm_smem_bytes(int bn);
 int gemm_threads();
 
+// The CTA-pair GEMM: clusters of two CTAs, each cluster computing 256 x 256
+// output tiles (GemmParams.num_m_tiles / num_n_tiles count pair tiles).
+// tmap_a / tmap_b: box {128, 128} like launch_gemm; tmap_y as above.
+// `clusters` must not exceed gemm_pair_max_clusters() (co-resident clusters
+// of the current device), since the kernel is persistent.
+cudaError_t launch_gemm_pair(const void* tmap_a, const void* tmap_b, const void* tmap_y,
+                             const GemmParams& p, int clusters, cudaStream_t st);
+cudaError_t gemm_pair_max_clusters(int* clusters);
+size_t gemm_pair_smem_bytes();
+int gemm_pair_stages();
+
 cudaError_t launch_col_absmax(const uint16_t* M, int64_t rows, int K, float* out, cudaStream_t st);
 cudaError_t launch_sigma_inv(const float* act_absmax, float* sigma_inv, int K, float alpha,
                              cudaStream_t st);

@@ -194,6 +194,20 @@ hq_status hq_check_device_error(hq_stream_t stream);
  * launches issued after the call. */
 hq_status hq_debug_set_wait_limit(uint64_t nanoseconds);
 
+/* Test hook: which GEMM kernel hq_linear launches.  Host state, applies to
+ * calls issued after it.
+ *   HQ_GEMM_AUTO (0)        chosen per shape (default);
+ *   HQ_GEMM_SINGLE_CTA (1)  one CTA per 128 x BN output tile (BN 64..256);
+ *   HQ_GEMM_CTA_PAIR (2)    clusters of two CTAs per 256 x 256 output tile
+ *                           (tcgen05 CTA-pair MMA); hq_linear returns
+ *                           HQ_ERR_UNSUPPORTED if the device cannot hold
+ *                           one such cluster.
+ * Results are identical either way: the integer accumulators are exact and
+ * the epilogue is the same code.  Returns HQ_ERR_INVALID_ARGUMENT for any
+ * other value. */
+enum { HQ_GEMM_AUTO = 0, HQ_GEMM_SINGLE_CTA = 1, HQ_GEMM_CTA_PAIR = 2 };
+hq_status hq_debug_set_gemm_variant(int variant);
+
 /* Test hook for the bounded-wait error path, without faulting the GPU:
  *   HQ_FAULT_NONE (0)                    normal operation;
  *   HQ_FAULT_QUANT_WITHHOLD_LOAD (1)     each CTA of the next activation

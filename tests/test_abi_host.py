@@ -118,6 +118,10 @@ def test_prepare_and_calib_validation(hq):
     assert lib.hq_debug_inject_fault(9) == 1
     assert lib.hq_debug_inject_fault(0) == 0
     assert lib.hq_debug_set_wait_limit(0) == 0
+    assert lib.hq_debug_set_gemm_variant(3) == 1
+    assert lib.hq_debug_set_gemm_variant(-1) == 1
+    for v in (hq.HQ_GEMM_CTA_PAIR, hq.HQ_GEMM_SINGLE_CTA, hq.HQ_GEMM_AUTO):
+        assert lib.hq_debug_set_gemm_variant(v) == 0
 
 
 def test_binding_rejects_host_tensors(hq):

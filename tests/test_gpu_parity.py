@@ -187,8 +187,17 @@ GEMM_SHAPES = [(1, 16, 32), (127, 48, 160), (128, 192, 128), (129, 320, 320), (3
                (256, 1024, 1024), (200, 3456, 256), (131, 160, 4608), (513, 64, 96)]
 
 
+@pytest.fixture(params=["single_cta", "cta_pair"])
+def gemm_variant(request, hq):
+    """Runs the test once per GEMM kernel; the automatic choice is restored after."""
+    v = {"single_cta": hq.HQ_GEMM_SINGLE_CTA, "cta_pair": hq.HQ_GEMM_CTA_PAIR}[request.param]
+    hq.hq_debug_set_gemm_variant(v)
+    yield v
+    hq.hq_debug_set_gemm_variant(hq.HQ_GEMM_AUTO)
+
+
 @pytest.mark.parametrize("T,N,K", GEMM_SHAPES)
-def test_gemm_accumulators_bit_exact(hq, T, N, K):
+def test_gemm_accumulators_bit_exact(hq, gemm_variant, T, N, K):
     g = np.random.default_rng(T * N + K)
     A = g.integers(-128, 128, size=(T, K)).astype(np.int8)
     B = g.integers(-128, 128, size=(N, K)).astype(np.int8)
@@ -216,7 +225,31 @@ def test_gemm_accumulators_bit_exact(hq, T, N, K):
     assert err <= 1e-5, err
 
 
-def test_gemm_worst_case_int4_accumulation(hq):
+def test_gemm_many_tiles_per_cta(hq, gemm_variant):
+    """Several output tiles per persistent CTA (both tensor-memory accumulators
+    reused, ring phases wrapping many times) with ragged rows, columns and K;
+    accumulators checked exactly on a seeded sample of rows from every
+    256-row tile, all columns."""
+    T, N, K = 4100, 4112, 320
+    g = np.random.default_rng(7)
+    A = g.integers(-8, 9, size=(T, K)).astype(np.int8)
+    B = g.integers(-8, 9, size=(N, K)).astype(np.int8)
+    sx = (g.random(T) * 0.1 + 1e-3).astype(np.float32)
+    sw = (g.random(N) * 0.01 + 1e-4).astype(np.float32)
+    desc = hq.LayerDesc(K, N, 64, a_bits=5, w_bits=5, act_gran=hq.HQ_PER_TOKEN)
+    Y = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    acc = torch.full((T, N), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    dev = lambda v: torch.from_numpy(v).cuda()
+    hq.hq_linear(desc, dev(A), dev(sx), None, dev(B), dev(sw), None, None, Y, acc)
+    assert hq.hq_check_device_error() == 0
+    rows = synth.sample_rows(T, 400, tile=256, seed=3)
+    acc_ref = oracle.gemm_acc(A[rows], B)
+    assert np.array_equal(acc.cpu().numpy()[rows].astype(np.int64), acc_ref)
+    _, y_ref = oracle.epilogue(acc_ref, sx[rows].astype(np.float64), sw.astype(np.float64))
+    assert rel_frob(bf16_bits(Y)[rows], y_ref) <= 1e-5
+
+
+def test_gemm_worst_case_int4_accumulation(hq, gemm_variant):
     T, N, K = 256, 256, 4608
     A = np.full((T, K), 7, dtype=np.int8)
     A[1::2] = -7
@@ -332,7 +365,7 @@ def test_layer_full_size_sampled(hq, idx):
     assert np.array_equal(acc_s[np.ix_(ra, ca)], ref["acc"][np.ix_(ra, ca)])
 
 
-def test_gemm_fed_oracle_codes_is_bit_exact(hq):
+def test_gemm_fed_oracle_codes_is_bit_exact(hq, gemm_variant):
     cfg = synth.CONFIGS[2].with_tokens(384)
     Xb, Wb, bb = synth.make_layer(cfg)
     ref = _oracle_layer(cfg, Xb, Wb[:512], bb[:512])
