@@ -10,9 +10,11 @@ reported separately.
 
 Prints one JSON line (rank 0).  `value` is device-timed throughput of the
 whole job in TOPS (2*T*K*N integer ops of the layer per step, summed over
-ranks, divided by the max over ranks of the summed per-step CUDA-event times).
-L2 is flushed (memset of a buffer twice the L2 size) before every timed step,
-outside the timed events.  Ranks are independent data-parallel shards: each
+ranks, divided by the max over ranks of the time of K steps).  The K steps
+run back to back from one CUDA graph between two CUDA events.  Every step
+reads a different copy of the token batch (copies totalling more than twice
+the L2 size), so activations come from HBM on every step without a flush
+inside the timed region.  Ranks are independent data-parallel shards: each
 rank owns its own batch of tokens and a replica of the prepared weights; there
 is no collective on the data path (weak scaling).
 """
@@ -244,8 +246,10 @@ def config_block(cfg, n_gpus):
     return {"workload": cfg.workload(), "tokens_per_gpu": cfg.T, "K": cfg.K, "N": cfg.N,
             "had_order": cfg.had_order, "bits": f"A{cfg.a_bits}W{cfg.w_bits}",
             "act_granularity": gran, "centering": bool(cfg.centering), "sigma": cfg.use_sigma,
-            "l2": "flushed before every timed step (memset of 2x L2, outside the timed events)",
-            "timing": "CUDA events around CUDA-graph replays (one graph per kernel)",
+            "l2": "inputs larger than L2: step i reads copy i % M of the token batch, "
+                  "M copies > 2x L2 (weights and intermediate codes stay L2-resident)",
+            "timing": "one CUDA graph of K back-to-back steps between two CUDA events; "
+                      "per-kernel times from graphs of K launches of that kernel",
             "parallelism": f"dp{n_gpus} (token shards, replicated weights, no collective)"}
 
 
@@ -295,11 +299,6 @@ def run_hq(args):
     sig_inv = layer.sigma_inv if layer.use_sigma else None
     mean_in = bufs["a_mean"] if cfg.centering else None
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
-
-    def quantize():
-        hq.hq_quantize_act(desc, X, sig_inv, bufs["a_codes"], bufs["a_scale"], bufs["a_mean"],
-                           layer.workspace)
 
     def linear():
         hq.hq_linear(desc, bufs["a_codes"], bufs["a_scale"], mean_in, layer.w_codes,
@@ -307,58 +306,71 @@ def run_hq(args):
 
     launches_per_step = (2 if cfg.act_gran == 1 else 1) + 1
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        quantize()
+    # Rotating inputs instead of an L2 flush inside the timed region: M copies
+    # of this rank's token batch, M * |X| > 2 x L2, and step i reads copy
+    # i % M, so every step's activations come from HBM.  The weights and the
+    # step's own intermediate codes stay L2-resident, as in a real layer.
+    x_bytes = X.numel() * X.element_size()
+    n_copies = int(min(512, max(2, -(-2 * l2 // x_bytes) + 1)))
+    Xs = [X] + [X.clone() for _ in range(n_copies - 1)]
+
+    def quantize_i(i):
+        hq.hq_quantize_act(desc, Xs[i % n_copies], sig_inv, bufs["a_codes"], bufs["a_scale"],
+                           bufs["a_mean"], layer.workspace)
+
+    for i in range(args.warmup):
+        quantize_i(i)
         linear()
     torch.cuda.synchronize()
     status = hq.hq_check_device_error()
     if status != 0:
         raise RuntimeError(f"device error during warm-up: {hq.STATUS_NAMES.get(status)}")
 
-    # One CUDA graph per kernel: replays carry no host launch overhead, and an
-    # event between the two replays times each kernel separately.
-    g_quant, g_linear = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_quant):
-        quantize()
-    with torch.cuda.graph(g_linear):
-        linear()
-    for _ in range(args.warmup):
-        flush.zero_()
-        g_quant.replay()
-        g_linear.replay()
+    # K steps captured back to back in one CUDA graph: no host launch cost and
+    # one pair of events around the whole timed region.  Two more graphs hold
+    # K launches of each kernel alone, for the per-kernel times.
+    def capture(do_q, do_l):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(args.steps):
+                if do_q:
+                    quantize_i(i)
+                if do_l:
+                    linear()
+        return g
+
+    g_step, g_quant, g_linear = capture(True, True), capture(True, False), capture(False, True)
+    for g in (g_step, g_quant, g_linear):
+        g.replay()
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    def timed(g):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.25)
-    for i in range(args.steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        g_quant.replay()
-        ev[i][1].record(stream)
-        g_linear.replay()
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
+    total_ms = timed(g_step)
     if world > 1:
         dist.barrier()
     clock_info = clocks.stop()
+    q_total = timed(g_quant)
+    g_total = timed(g_linear)
     status = hq.hq_check_device_error()
     if status != 0:
         raise RuntimeError(f"device error in the timed region: {hq.STATUS_NAMES.get(status)}")
-
-    q_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    g_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(step_ms)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([total_ms, q_total, g_total], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms, q_total, g_total = (float(v) for v in t.tolist())
     ms_per_step = total_ms / args.steps
     ops = layer_ops(cfg)
     value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
@@ -378,27 +390,18 @@ def run_hq(args):
             linear()
             Yh.copy_(Y, non_blocking=True)
 
-        e2e_body()
+        for _ in range(max(1, args.warmup)):
+            e2e_body()
         torch.cuda.synchronize()
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e):
-            e2e_body()
-
-        def e2e_step():
-            g_e2e.replay()
-
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+            for _ in range(args.steps):
+                e2e_body()
+        g_e2e.replay()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        s1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = s0.elapsed_time(s1)
+        e2e_ms = timed(g_e2e)
         if world > 1:
             t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -417,8 +420,8 @@ def run_hq(args):
         return 0
 
     peaks, peak_src = load_peaks()
-    q_med = statistics.median(q_ms)
-    g_med = statistics.median(g_ms)
+    q_med = q_total / args.steps
+    g_med = g_total / args.steps
     q_gbs = quantizer_bytes(cfg) / (q_med * 1e-3) / 1e9
     g_tops = ops / (g_med * 1e-3) / 1e12
     int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
@@ -442,9 +445,9 @@ def run_hq(args):
         "config": config_block(cfg, world),
         "roofline": roof,
         "kernels": {
-            "quantizer": {"ms_median": q_med, "GB/s": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
+            "quantizer": {"ms_per_launch": q_med, "GB/s": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
                           "bytes": quantizer_bytes(cfg)},
-            "gemm": {"ms_median": g_med, "TOPS": g_tops, "frac_int8": g_tops / int8_peak,
+            "gemm": {"ms_per_launch": g_med, "TOPS": g_tops, "frac_int8": g_tops / int8_peak,
                      "hbm_bytes": gemm_bytes(cfg)},
             "weight_prep_ms": prep_ms,
         },
