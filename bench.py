@@ -91,6 +91,83 @@ def gemm_bytes(cfg) -> float:
 
 
 # ---------------------------------------------------------------------------
+# DRAM traffic per launch from a committed ncu summary
+# ---------------------------------------------------------------------------
+
+PROFILES = {("gemm", 2): "gemm_i8_cfg2_pixart_qkv.md", ("quant", 2): "quant_rows_cfg2_pixart_qkv.md"}
+KERNEL_SOURCES = {"gemm": ("hq_gemm.cu", "hq_device.cuh", "hq_kernels.h"),
+                  "quant": ("hq_quant.cu", "hq_device.cuh", "hq_kernels.h")}
+
+
+def kernel_source_hash(kind, root=ROOT):
+    import hashlib
+    m = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(root, "hadamard_rotated_bit_token_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def profiled_traffic(kind, cfg_index, root=ROOT):
+    """dram__bytes_read + dram__bytes_write of one launch of the kernel, as
+    recorded in profiles/ for this workload, or None if there is no summary
+    or the kernel's sources changed since it was captured."""
+    name = PROFILES.get((kind, cfg_index))
+    if name is None:
+        return None
+    try:
+        with open(os.path.join(root, "profiles", name)) as fh:
+            text = fh.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        key, sep, val = line.strip().partition(":")
+        if sep and key in ("traffic_bytes_per_launch", "kernel_source_sha256"):
+            fields[key] = val.strip()
+    if fields.get("kernel_source_sha256") != kernel_source_hash(kind, root):
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# multi-rank aggregation (one process per GPU, independent token shards)
+# ---------------------------------------------------------------------------
+
+def rank_env():
+    """(world, rank, local_rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, world, dist=None, device=None):
+    """Element-wise max over ranks of a list of floats (identity for one rank).
+    Every rank must call it with the same number of values."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def shard_seed(cfg, rank):
+    """Seed of rank `rank`'s token batch: every rank quantizes and multiplies
+    its own tokens (data-parallel shards); the weights are the same on all."""
+    return cfg.index + 1000 * rank
+
+
+def job_throughput(ops_per_step, steps, world, total_ms):
+    """Whole-job throughput in units of 1e12 per second: every rank runs
+    `steps` steps of `ops_per_step` on its own shard (weak scaling); the
+    job's time is the slowest rank's `total_ms`."""
+    return world * ops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # clocks sampled while the timed region runs
 # ---------------------------------------------------------------------------
 
@@ -207,7 +284,7 @@ def cpu_baseline(cfg, Xb, Wb, bb, target_s):
 # ---------------------------------------------------------------------------
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
     cfg = synth.CONFIGS[args.config]
@@ -263,9 +340,7 @@ def run_hq(args):
 
     import hadamard_rotated_bit_token_b200 as hq
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -275,7 +350,7 @@ def run_hq(args):
     cfg = synth.CONFIGS[args.config]
     # replicated weights (same seed on every rank), rank-local token batch
     Wb, bb = synth.make_w(cfg)
-    Xb = synth.make_x(cfg, seed=cfg.index + 1000 * rank)
+    Xb = synth.make_x(cfg, seed=shard_seed(cfg, rank))
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
     X, W, b = to_dev(Xb), to_dev(Wb), to_dev(bb)
     T, K, N = cfg.T, cfg.K, cfg.N
@@ -367,13 +442,10 @@ def run_hq(args):
     status = hq.hq_check_device_error()
     if status != 0:
         raise RuntimeError(f"device error in the timed region: {hq.STATUS_NAMES.get(status)}")
-    if world > 1:
-        t = torch.tensor([total_ms, q_total, g_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, q_total, g_total = (float(v) for v in t.tolist())
+    total_ms, q_total, g_total = max_over_ranks([total_ms, q_total, g_total], world, dist, dev)
     ms_per_step = total_ms / args.steps
     ops = layer_ops(cfg)
-    value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(ops, args.steps, world, total_ms)
 
     # end to end through the public API with host buffers (pinned), per step:
     # H2D of X, quantize, GEMM, D2H of Y
@@ -401,12 +473,8 @@ def run_hq(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        e2e_ms = timed(g_e2e)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * ops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        e2e_ms = max_over_ranks([timed(g_e2e)], world, dist, dev)[0]
+        e2e = {"value": job_throughput(ops, args.steps, world, e2e_ms), "unit": "TOPS",
                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
                "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()),
                "ms_per_step": e2e_ms / args.steps}
@@ -428,13 +496,13 @@ def run_hq(args):
     if g_med >= q_med:
         roof = {"kernel": "hq_gemm_i8 (tcgen05 kind::i8 + epilogue)", "bound": "tensor",
                 "achieved": g_tops, "peak": int8_peak, "unit": "TFLOP/s",
-                "frac": g_tops / int8_peak, "traffic": None,
+                "frac": g_tops / int8_peak, "traffic": profiled_traffic("gemm", cfg.index),
                 "peak_source": f"{peak_src}: 2 x bf16_tflops (burst), dense int8:bf16 = 4.5:2.25",
                 "algorithmic": f"2*T*K*N = {ops:.4g} int ops per launch"}
     else:
         roof = {"kernel": "hq_quantize_act (fused FWHT quantizer)", "bound": "hbm",
                 "achieved": q_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": q_gbs / peaks["hbm_gbs"], "traffic": None,
+                "frac": q_gbs / peaks["hbm_gbs"], "traffic": profiled_traffic("quant", cfg.index),
                 "peak_source": f"{peak_src} hbm_gbs",
                 "algorithmic": f"{quantizer_bytes(cfg):.4g} bytes per launch"}
     line = {
