@@ -24,7 +24,7 @@ __all__ = [
     "HQError", "LayerDesc", "load_library", "library_path", "exported_symbols",
     "HQ_PER_TOKEN", "HQ_PER_TENSOR_DYNAMIC", "HQ_PER_TENSOR_STATIC",
     "HQ_CENTER_NONE", "HQ_CENTER_TOKEN_MEAN", "HQ_CODES_I8",
-    "HQ_FAULT_NONE", "HQ_FAULT_QUANT_WITHHOLD_LOAD", "STATUS_NAMES",
+    "HQ_FAULT_NONE", "HQ_FAULT_QUANT_WITHHOLD_ROW", "STATUS_NAMES",
     "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
@@ -38,7 +38,7 @@ _LIB_PATH = os.path.join(_PKG, "libhq.so")
 HQ_PER_TOKEN, HQ_PER_TENSOR_DYNAMIC, HQ_PER_TENSOR_STATIC = 0, 1, 2
 HQ_CENTER_NONE, HQ_CENTER_TOKEN_MEAN = 0, 1
 HQ_CODES_I8 = 0
-HQ_FAULT_NONE, HQ_FAULT_QUANT_WITHHOLD_LOAD = 0, 1
+HQ_FAULT_NONE, HQ_FAULT_QUANT_WITHHOLD_ROW = 0, 1
 HQ_GEMM_AUTO, HQ_GEMM_SINGLE_CTA, HQ_GEMM_CTA_PAIR = 0, 1, 2
 STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED",
                 3: "HQ_ERR_MISALIGNED", 4: "HQ_ERR_CUDA", 5: "HQ_ERR_TIMEOUT",

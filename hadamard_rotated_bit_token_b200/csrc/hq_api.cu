@@ -114,12 +114,15 @@ hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CU
 // Rows per tile R and threads per CTA for the row quantizer: one producer
 // warp plus worker warps in which every thread owns a 32-channel slice of one
 // row; prefer full warps and 8-9 worker warps.
+// Rows per tile R and threads per CTA (one thread per 32-channel slice of
+// each row, whole warps): the R that leaves the fewest idle lanes, preferring
+// larger CTAs.
 void quant_shape(int K, int* R_out, int* nt_out) {
   const int S = K / 32;
-  const int maxW = quant_max_threads() - 32;
+  const int maxT = quant_max_threads();
   int bestR = 1, bestNT = ((S + 31) / 32) * 32;
   double bestScore = -1.0;
-  for (int R = 1; R * S <= maxW && kQuantRowsPerThread * R <= 256; ++R) {  // a tile is one TMA box
+  for (int R = 1; R * S <= maxT; ++R) {
     const int nt = ((R * S + 31) / 32) * 32;
     const double util = double(R * S) / nt;
     const double size_pref = nt >= 256 ? 1.0 : double(nt) / 256.0;
@@ -131,31 +134,16 @@ void quant_shape(int K, int* R_out, int* nt_out) {
     }
   }
   *R_out = bestR;
-  *nt_out = bestNT + 32;  // + producer warp
+  *nt_out = bestNT;
 }
 
 struct QuantLaunch {
   QuantParams p;
-  CUtensorMap tmap;
   int threads;
   size_t smem;
   int grid;
   int logn;
 };
-
-hq_status encode_rows_bf16(CUtensorMap* m, const void* base, int64_t rows, int K, int R) {
-  // [rows, K] bf16 viewed as {64 elements, K/64 line groups, rows}; one box is
-  // a whole tile of R rows, written to shared memory with 128-byte swizzle
-  cuuint64_t dims[3] = {64u, cuuint64_t(K / 64), cuuint64_t(rows)};
-  cuuint64_t strides[2] = {128u, cuuint64_t(K) * 2u};
-  cuuint32_t box[3] = {64u, cuuint32_t(K / 64), cuuint32_t(R)};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
-}
 
 hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, const uint16_t* X,
                             QuantLaunch* out) {
@@ -164,34 +152,23 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
   int R, nt;
   quant_shape(K, &R, &nt);
   const int logn = ilog2_exact(n);
-  const bool xpose = logn >= 6;            // shared-memory transposes for n >= 64
-  const int per_sm = 2;                    // CTAs per SM (kernel launch bounds)
-  const int B = K / n;
-  const uint32_t raw = uint32_t(kQuantRowsPerThread * R) * uint32_t(K) * 2u;  // one tile
-  const uint32_t tile_bytes = (raw + 1023u) & ~1023u;
-  const uint32_t budget = per_sm == 1 ? 150u * 1024u : 100u * 1024u;
-  const size_t fixed = quant_smem_bytes(0, tile_bytes, R, K, B, (nt - 32) / 32, xpose);
-  int nstage = int((budget - uint32_t(fixed)) / tile_bytes);
-  if (nstage > 6) nstage = 6;
-  if (nstage < 2) nstage = 2;
+  const bool xpose = logn >= 6;  // shared-memory transposes for n >= 64
+  const int per_sm = 2;          // CTAs per SM (kernel launch bounds)
+  L.p.X = X;
   L.p.T = T;
   L.p.K = K;
   L.p.S = K / 32;
   L.p.R = R;
-  L.p.nstage = nstage;
-  L.p.tile_bytes = tile_bytes;
   L.p.inv_sqrt_n = float(1.0 / std::sqrt(double(n)));
   L.p.sqrt_n = float(std::sqrt(double(n)));
   L.p.err = dev->err;
   L.p.wait_ns = wait_ns();
   L.threads = nt;
   L.logn = logn;
-  L.smem = quant_smem_bytes(nstage, tile_bytes, R, K, B, (nt - 32) / 32, xpose);
-  const int64_t tile_rows = kQuantRowsPerThread * R;
-  const int64_t ntiles = (T + tile_rows - 1) / tile_rows;
+  L.smem = quant_smem_bytes(R, K, K / n, nt / 32, xpose);
+  const int64_t ntiles = (T + R - 1) / R;
   const int64_t slots = int64_t(dev->sm_count) * per_sm;
   L.grid = int(ntiles < slots ? ntiles : slots);
-  if (T > 0) return encode_rows_bf16(&L.tmap, X, T, K, kQuantRowsPerThread * R);
   return HQ_OK;
 }
 
@@ -204,13 +181,13 @@ hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, bool center, cud
     std::lock_guard<std::mutex> lock(g_mutex);
     bool& set = dev->quant_attr_set[logn - 4 < 0 ? 0 : logn - 4][mode][center ? 1 : 0];
     if (!set) {
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024) !=
           cudaSuccess)
         return HQ_ERR_CUDA;
       set = true;
     }
   }
-  void* args[] = {&L.tmap, &L.p};
+  void* args[] = {&L.p};
   return from_cuda(cudaLaunchKernel(fn, dim3(L.grid), dim3(L.threads), args, L.smem, st));
 }
 
@@ -396,7 +373,7 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   L.p.mean = a_mean;
   L.p.rowsum = nullptr;
   L.p.q = (1 << (desc->a_bits - 1)) - 1;
-  L.p.fault_skip_load = g_fault == HQ_FAULT_QUANT_WITHHOLD_LOAD ? 1 : 0;
+  L.p.fault_withhold_row = g_fault == HQ_FAULT_QUANT_WITHHOLD_ROW ? 1 : 0;
   const bool center = desc->centering == HQ_CENTER_TOKEN_MEAN;
   if (desc->act_gran == HQ_PER_TOKEN) return run_quant(dev, L, 0, center, st);
   if (desc->act_gran == HQ_PER_TENSOR_STATIC) {
@@ -410,7 +387,7 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   QuantLaunch L1 = L;
   L1.p.codes = nullptr;
   L1.p.mean = nullptr;
-  L1.p.fault_skip_load = 0;
+  L1.p.fault_withhold_row = 0;
   s = run_quant(dev, L1, 1, center, st);
   if (s != HQ_OK) return s;
   return run_quant(dev, L, 2, center, st);
@@ -532,7 +509,7 @@ hq_status hq_debug_set_gemm_variant(int variant) {
 }
 
 hq_status hq_debug_inject_fault(int kind) {
-  if (kind != HQ_FAULT_NONE && kind != HQ_FAULT_QUANT_WITHHOLD_LOAD) return HQ_ERR_INVALID_ARGUMENT;
+  if (kind != HQ_FAULT_NONE && kind != HQ_FAULT_QUANT_WITHHOLD_ROW) return HQ_ERR_INVALID_ARGUMENT;
   std::lock_guard<std::mutex> lock(g_mutex);
   g_fault = kind;
   return HQ_OK;

@@ -20,29 +20,23 @@ struct QuantParams {
   int64_t T;
   int K;
   int S;                      // 32-channel slices per row (K / 32)
-  int R;                      // rows per thread pass (a tile holds kQuantRowsPerThread*R rows)
+  int R;                      // rows per tile (one thread per slice of each row)
   int q;                      // 2^(bits-1) - 1
-  int nstage;                 // shared-memory stages
-  uint32_t tile_bytes;        // bytes per stage (tile rows * K * 2 rounded up to 1024)
   float inv_sqrt_n;           // 1 / sqrt(n), fp32
   float sqrt_n;               // sqrt(n), fp32
-  int fault_skip_load;        // test hook: withhold the first tile load
+  int fault_withhold_row;     // test hook: never release the first row of the first tile
   unsigned int* err;          // device error word
   unsigned long long wait_ns; // bounded-wait limit
 };
 
 // Returns the kernel entry for log2(n) in [4,10], mode in [0,3]; the kernel
-// takes (const CUtensorMap tmX, QuantParams p): tmX views the [T,K] bf16 rows
-// as a 3-D tensor {64, K/64, T} with box {64, K/64, R} and 128-byte swizzle.
+// takes (QuantParams p) and runs R * S active threads per CTA (rounded up to
+// whole warps, at most quant_max_threads()).
 const void* quant_kernel_ptr(int logn, int mode, bool center);
 int quant_max_threads();
-// Dynamic shared memory of one quantizer CTA (includes 1 KB of alignment slack).
-// Rows of a tile each quantizer worker thread handles (one 32-channel slice of
-// each); a tile holds kQuantRowsPerThread * R rows.
-constexpr int kQuantRowsPerThread = 1;
-// R = rows covered by one pass of the worker threads.
-size_t quant_smem_bytes(int nstage, uint32_t tile_bytes, int R, int K, int B, int nworker_warps,
-                        bool xpose);
+// Dynamic shared memory of one quantizer CTA: R rows per tile, K channels,
+// B blocks per row, `nwarps` warps, transposes for n >= 64.
+size_t quant_smem_bytes(int R, int K, int B, int nwarps, bool xpose);
 
 struct GemmParams {
   const float* a_scale;   // [T] or [1]

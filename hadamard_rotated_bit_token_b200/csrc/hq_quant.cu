@@ -23,21 +23,25 @@
 // Row mean: sum_k Z_hat[b,k] = n * Y[b,0] for each block b (every column of
 // H~ but the first sums to zero), so mu_hat = (n / K) * sum_b Y[b,0]; this
 // identity (HaTQ Eq. (23) read column-wise) gives the exact mean of the
-// rotated row from the first channel of each block, summed in a fixed order.
+// rotated row from the first channel of each block, summed in block order.
 //
-// Work decomposition (persistent CTAs over tiles of R rows):
-//   warp 0 (one thread) streams tiles into a ring of shared-memory stages with
-//     a 3-D TMA tensor load (128-byte swizzle, so the row slices below are
-//     read without bank conflicts);
-//   worker warps: each thread owns a 32-channel slice of one row.  bf16 ->
-//     fp32, times the channel multiplier (kept in registers) -> butterflies on
-//     the 5 in-register index bits -> the remaining bits across the n/32
-//     threads of a block: warp shuffles for n <= 128; for n >= 256 an 8-lane
-//     shared-memory transpose swaps index bits 2-4 with 5-7 and shuffles take
-//     bits 8 and up -> row max / min by shared-memory atomics on ordered
-//     integers -> a per-row mbarrier (one arrival per thread of the row) ->
-//     codes packed 4 per word and stored.  No CTA-wide barrier in the loop:
-//     warps only wait for the other warps of their own rows.
+// Work decomposition (persistent CTAs over tiles of R rows; every thread
+// owns one 32-channel slice of one row of each tile, the same slice of every
+// tile):
+//   load     four coalesced 16-byte loads straight into registers, issued one
+//            tile ahead of the tile being processed (no shared-memory stage);
+//   rotate   bf16 -> fp32, times the channel multiplier, butterflies on the 5
+//            in-register index bits, then the remaining bits across the n/32
+//            threads of a block: warp shuffles for n <= 128 beyond the
+//            transpose; for n >= 64 an 8-lane shared-memory transpose swaps
+//            index bits 2-4 with 5-7 and shuffles take bits 8 and up;
+//   stats    the row's max / min by a warp reduction over the lanes of the
+//            row (redux.sync) and one shared-memory atomic per warp segment;
+//            the segment that completes the row (a per-row arrival counter)
+//            computes the row's mean, scale and reciprocal once, publishes
+//            them and releases the row's barrier;
+//   quantize codes packed 4 per word and stored.
+// No CTA-wide barrier in the loop: warps wait only for the rows they hold.
 // Arithmetic on pairs of lanes uses Blackwell's packed fp32x2 instructions.
 #include <cuda.h>
 
@@ -48,10 +52,9 @@ namespace hq {
 
 namespace {
 
-constexpr int kQuantThreads = 320;  // 1 producer warp + up to 9 worker warps
+constexpr int kQuantThreads = 320;          // up to 10 warps, all workers
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
-constexpr int kStatBufs = 3;
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -67,7 +70,8 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
   return d;
 }
 
-// Order-preserving map of floats onto unsigned integers (for atomicMax/Min).
+// Order-preserving map of floats onto unsigned integers (for max / min of
+// floats by integer reductions and atomics).
 __device__ __forceinline__ uint32_t ord_f32(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -76,46 +80,47 @@ __device__ __forceinline__ float unord_f32(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-__device__ __forceinline__ uint32_t f2lo_bits(f2 x) { return __float_as_uint(x.x); }
-__device__ __forceinline__ uint32_t f2hi_bits(f2 x) { return __float_as_uint(x.y); }
-__device__ __forceinline__ f2 f2_from_bits(uint32_t lo, uint32_t hi) {
-  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+// Streaming 16-byte load of data read once (not kept in L1).
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
 }
 
-// Shared-memory layout of one CTA (offsets in bytes, from a 1024-byte aligned base).
+// Shared-memory layout of one CTA (byte offsets from a 16-byte aligned base).
 struct QuantSmem {
-  uint32_t stages, full, empty, rowbar, rowmax, rowmin, y0, mult, xbuf, flags, total;
+  uint32_t mult, xbuf, pmax, pmin, cnt, res, y0, rowbar, flags, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 __host__ __device__ inline int padded_blocks(int B) { return (B + 3) & ~3; }
 
-// RT = rows per tile (2 per thread), K channels, B blocks per row.
-__host__ __device__ inline QuantSmem quant_smem_layout(int nstage, uint32_t tile_bytes, int RT, int K,
-                                                       int B, int nworker_warps, bool xpose) {
+// R rows per tile, K channels, B blocks per row, `nwarps` warps.  The row
+// statistics are double-buffered by tile parity.
+__host__ __device__ inline QuantSmem quant_smem_layout(int R, int K, int B, int nwarps, bool xpose) {
   QuantSmem L;
   uint32_t off = 0;
-  L.stages = off;
-  off += uint32_t(nstage) * tile_bytes;
-  L.full = off;
-  off += 8u * nstage;
-  L.empty = off;
-  off += 8u * nstage;
-  L.rowbar = off;
-  off += 8u * RT;
-  L.rowmax = off;
-  off += 4u * kStatBufs * RT;
-  L.rowmin = off;
-  off += 4u * kStatBufs * RT;
-  off = align_up(off, 16);
-  L.y0 = off;  // [kStatBufs][RT][padded B] first channel of every block
-  off += 4u * kStatBufs * RT * padded_blocks(B);
-  off = align_up(off, 16);
   L.mult = off;  // channel multipliers, chunk-major [8][K/32] float4
   off += 4u * K;
-  L.xbuf = off;
-  off += xpose ? 4096u * nworker_warps : 0u;
-  L.flags = off;
+  L.xbuf = off;  // per-warp transpose buffers
+  off += xpose ? 4096u * nwarps : 0u;
+  L.pmax = off;
+  off += 4u * 2 * R;
+  L.pmin = off;
+  off += 4u * 2 * R;
+  L.cnt = off;
+  off += 4u * 2 * R;
+  off = align_up(off, 8);
+  L.res = off;  // [2][R] (mean, reciprocal scale)
+  off += 8u * 2 * R;
+  off = align_up(off, 16);
+  L.y0 = off;  // [2][R][padded B] first channel of every block
+  off += 4u * 2 * R * padded_blocks(B);
+  off = align_up(off, 8);
+  L.rowbar = off;
+  off += 8u * R;
+  L.flags = off;  // [0] abort, [1] CTA max (mode 1)
   off += 16;
   L.total = off;
   return L;
@@ -123,22 +128,16 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int nstage, uint32_t tile
 
 }  // namespace
 
-size_t quant_smem_bytes(int nstage, uint32_t tile_bytes, int R, int K, int B, int nworker_warps,
-                        bool xpose) {
-  return quant_smem_layout(nstage, tile_bytes, kQuantRowsPerThread * R, K, B, nworker_warps, xpose)
-             .total + 1024;
+size_t quant_smem_bytes(int R, int K, int B, int nwarps, bool xpose) {
+  return quant_smem_layout(R, K, B, nwarps, xpose).total;
 }
 
 // MODE 0: per-row dynamic scale (activations per token, or weights per row)
 // MODE 1: per-tensor pass 1: only the tensor-wide max |V| (into tensor_max)
 // MODE 2: per-tensor pass 2: scale from tensor_max
 // MODE 3: per-tensor static scale from static_scale[0] (real units)
-//
-// Each worker thread owns one 32-channel slice of RPT rows of a tile (rows r,
-// r + R, ...); the per-tile bookkeeping and multipliers are shared by them.
 template <int LOGN, int MODE, bool CENTER>
-__global__ void __launch_bounds__(kQuantThreads, 2)
-    quant_rows_kernel(const __grid_constant__ CUtensorMap tmX, const QuantParams p) {
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const QuantParams p) {
   constexpr int N = 1 << LOGN;
   constexpr int LREG = LOGN < 5 ? LOGN : 5;        // index bits inside a thread's slice
   constexpr int LOG_TT = LOGN > 5 ? LOGN - 5 : 0;  // index bits across threads
@@ -154,56 +153,66 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   constexpr bool XPOSE = LX > 0;
   constexpr int NSHFL = LOG_TT - LX;
   constexpr int BPT = N >= 32 ? 1 : 32 / N;        // blocks per thread slice (n < 32)
-  constexpr int RPT = kQuantRowsPerThread;         // rows per thread
   constexpr bool kClamp = (MODE >= 2);
   constexpr bool kQuantize = (MODE != 1);
 
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-
+  extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int nworkers = int(blockDim.x) - 32;
-  const int S = p.S;
-  const int R = p.R;            // rows per half tile (threads cover R x S slices)
-  const int RT = RPT * R;       // rows per tile
+  const int S = p.S;  // 32-channel slices per row
+  const int R = p.R;  // rows per tile
   const int K = p.K;
   const int B = K >> LOGN;
   const int BP = padded_blocks(B);
-  const int lines_per_row = K >> 6;  // 128-byte lines of bf16
   const int64_t T = p.T;
-  const int64_t ntiles = (T + RT - 1) / RT;
-  const QuantSmem L = quant_smem_layout(p.nstage, p.tile_bytes, RT, K, B, nworkers >> 5, XPOSE);
-  uint8_t* stages = smem + L.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.full);
-  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L.empty);
-  uint64_t* rowbar = reinterpret_cast<uint64_t*>(smem + L.rowbar);
-  uint32_t* rowmax = reinterpret_cast<uint32_t*>(smem + L.rowmax);
-  uint32_t* rowmin = reinterpret_cast<uint32_t*>(smem + L.rowmin);
-  float* y0buf = reinterpret_cast<float*>(smem + L.y0);
+  const int64_t ntiles = (T + R - 1) / R;
+  const QuantSmem L = quant_smem_layout(R, K, B, int(blockDim.x) >> 5, XPOSE);
   float4* msm = reinterpret_cast<float4*>(smem + L.mult);
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);  // [0] abort, [1] cta max
+  uint32_t* pmax = reinterpret_cast<uint32_t*>(smem + L.pmax);
+  uint32_t* pmin = reinterpret_cast<uint32_t*>(smem + L.pmin);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + L.cnt);
+  float2* res = reinterpret_cast<float2*>(smem + L.res);
+  float* y0buf = reinterpret_cast<float*>(smem + L.y0);
+  uint64_t* rowbar = reinterpret_cast<uint64_t*>(smem + L.rowbar);
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);
   const WaitCtl wc{p.err, p.wait_ns};
   const bool has_mult = p.mult != nullptr;
   const bool need_sum = CENTER || p.rowsum != nullptr;
 
-  if (tid == 0) {
-    for (int s = 0; s < p.nstage; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], uint32_t(nworkers));
+  const bool active = tid < R * S;
+  const int row0 = active ? tid / S : 0;  // this thread's row of every tile
+  const int slice = active ? tid - row0 * S : 0;
+  const int member = slice & (TT - 1);
+  const int blk = slice >> LOG_TT;        // block of the row (n >= 32)
+
+  // first tile's slice in flight while the CTA sets up
+  const uint16_t* xcol = p.X + slice * 32;
+  uint4 nxt[4] = {};
+  auto load_slice = [&](int64_t tile) {
+    const int64_t row = tile * R + row0;
+    if (active && row < T) {
+      const uint4* src = reinterpret_cast<const uint4*>(xcol + row * K);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) nxt[c] = ld_stream(src + c);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) nxt[c] = make_uint4(0, 0, 0, 0);
     }
-    for (int r = 0; r < RT; ++r) mbar_init(&rowbar[r], uint32_t(S));
+  };
+  if (int64_t(blockIdx.x) < ntiles) load_slice(blockIdx.x);
+
+  if (tid == 0) {
+    for (int r = 0; r < R; ++r) mbar_init(&rowbar[r], 1);
     flags[0] = 0;
     flags[1] = 0;
     fence_mbarrier_init();
   }
-  for (int i = tid; i < kStatBufs * RT; i += blockDim.x) {
-    rowmax[i] = 0u;
-    rowmin[i] = 0xFFFFFFFFu;
+  for (int i = tid; i < 2 * R; i += blockDim.x) {
+    pmax[i] = 0u;
+    pmin[i] = 0xFFFFFFFFu;
+    cnt[i] = 0u;
   }
-  for (int i = tid; i < kStatBufs * RT * BP; i += blockDim.x) y0buf[i] = 0.0f;
   if (has_mult) {
     // chunk-major copy: thread `slice` reads chunk c at msm[c * S + slice], so
     // consecutive slices hit consecutive 16-byte words
@@ -221,332 +230,235 @@ __global__ void __launch_bounds__(kQuantThreads, 2)
   }
   __syncthreads();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tmX);
-      const uint32_t box_bytes = uint32_t(RT) * uint32_t(K) * 2u;
-      int s = 0;
-      uint32_t ph = 0;
-      int issued = 0;
-      bool skipped = false;
-      for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        if (flags[0] || !mbar_wait(&empty[s], ph ^ 1u, wc)) {
-          flags[0] = 1;
-          break;
-        }
-        if (issued == 0 && p.fault_skip_load && !skipped) {
-          skipped = true;  // test hook: this stage's barrier never completes
-        } else {
-          mbar_arrive_expect_tx(&full[s], box_bytes);
-          tma_load_3d(stages + size_t(s) * p.tile_bytes, &tmX, 0, 0, int32_t(tile * RT), &full[s]);
-        }
-        ++issued;
-        if (++s == p.nstage) {
-          s = 0;
-          ph ^= 1u;
-        }
+  // lanes of this warp that hold slices of this thread's row
+  const int wbase = warp * 32;
+  const int seg_lo = max(row0 * S, wbase) - wbase;
+  const int seg_hi = min(min(row0 * S + S, R * S), wbase + 32) - wbase;
+  const int seg_len = seg_hi - seg_lo;
+  const unsigned segmask = seg_len >= 32 ? 0xFFFFFFFFu : (((1u << seg_len) - 1u) << seg_lo);
+  const bool seg_leader = active && lane == seg_lo;
+
+  const int tl = lane & (G - 1);        // lane within the transpose group
+  const int sub = lane >> LX;           // transpose group within the warp
+  uint8_t* xb = smem + L.xbuf + warp * 4096 + sub * (G * 128);
+  const int csw = sub & (CH - 1);       // chunk swizzle of this transpose group
+
+  float r_tensor = 0.0f;
+  if (MODE == 2) {
+    const float a = __uint_as_float(*p.tensor_max);
+    r_tensor = a > 0.0f ? __fdiv_rn(float(p.q), a) : 0.0f;
+    if (blockIdx.x == 0 && tid == 0 && p.scale) p.scale[0] = (a / float(p.q)) * p.inv_sqrt_n;
+  } else if (MODE == 3) {
+    const float s = p.static_scale[0];
+    r_tensor = s > 0.0f ? __fdiv_rn(1.0f, s * p.sqrt_n) : 0.0f;
+  }
+  const float n_over_k = float(N) / float(K);
+  const float qf = float(p.q);
+
+  int it = 0;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int pb = it & 1;  // statistics buffer of this tile
+    const int sr = pb * R + row0;
+    f2 w[16];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      w[4 * c + 0] = pk(bf16lo(nxt[c].x), bf16hi(nxt[c].x));
+      w[4 * c + 1] = pk(bf16lo(nxt[c].y), bf16hi(nxt[c].y));
+      w[4 * c + 2] = pk(bf16lo(nxt[c].z), bf16hi(nxt[c].z));
+      w[4 * c + 3] = pk(bf16lo(nxt[c].w), bf16hi(nxt[c].w));
+    }
+    if (tile + gridDim.x < ntiles) load_slice(tile + gridDim.x);  // one tile ahead
+
+    if (has_mult) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 m4 = msm[i * S + slice];
+        w[2 * i] = mul2(w[2 * i], pk(m4.x, m4.y));
+        w[2 * i + 1] = mul2(w[2 * i + 1], pk(m4.z, m4.w));
       }
-      if (flags[0]) {
-        // let copies still in flight land before the CTA exits
-        int s2 = s;
-        uint32_t ph2 = ph;
-        for (int i = 0; i < p.nstage && i < issued; ++i) {
-          if (--s2 < 0) {
-            s2 = p.nstage - 1;
-            ph2 ^= 1u;
-          }
-          if (!(skipped && i == issued - 1)) (void)mbar_wait(&full[s2], ph2, wc);
+    }
+    // first channel of each block (Y[b,0]) for the row mean / row sum
+    if (need_sum && active && member == 0) {
+      float* yrow = y0buf + sr * BP;
+#pragma unroll
+      for (int b = 0; b < BPT; ++b) yrow[blk * BPT + b] = w[(b * N) >> 1].x;
+    }
+    // index bit 0: the two halves of a pair
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float a = w[i].x, b = w[i].y;
+      w[i] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+    // index bits 1 .. LREG-1: between pairs
+#pragma unroll
+    for (int bit = 1; bit < LREG; ++bit) {
+      const int hh = 1 << (bit - 1);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if ((i & hh) == 0) {
+          const f2 x = w[i], y = w[i + hh];
+          w[i] = add2(x, y);
+          w[i + hh] = sub2(x, y);
         }
       }
     }
-  } else {
-    // -------------------------------------------------------------- workers
-    const int wid = tid - 32;
-    const bool active = wid < R * S;
-    const int row0 = active ? wid / S : 0;   // rows row0, row0 + R, ... of the tile
-    const int slice = active ? wid - row0 * S : 0;
-    const int member = slice & (TT - 1);
-    const int blk = slice >> LOG_TT;      // block of the row (n >= 32)
-    const int tl = lane & (G - 1);        // lane within the transpose group
-    const int sub = lane >> LX;           // transpose group within the warp
-    uint8_t* xb = smem + L.xbuf + (warp - 1) * 4096 + sub * (G * 128);
-    const int csw = sub & (CH - 1);       // chunk swizzle of this transpose group
-
-    float r_tensor = 0.0f;
-    if (MODE == 2) {
-      const float a = __uint_as_float(*p.tensor_max);
-      r_tensor = a > 0.0f ? __fdiv_rn(float(p.q), a) : 0.0f;
-      if (blockIdx.x == 0 && wid == 0 && p.scale) p.scale[0] = (a / float(p.q)) * p.inv_sqrt_n;
-    } else if (MODE == 3) {
-      const float s = p.static_scale[0];
-      r_tensor = s > 0.0f ? __fdiv_rn(1.0f, s * p.sqrt_n) : 0.0f;
-    }
-    const float n_over_k = float(N) / float(K);
-    const float qf = float(p.q);
-
-    // byte offsets of this thread's slices inside a stage (128-byte swizzle)
-    uint32_t chunk_off[RPT][4];
+    if (XPOSE) {
+      // swap index bits 5..4+LX (lanes of a G-lane group) with bits
+      // 5-LX..4 (register groups of GS elements); slots XOR-swizzled by
+      // lane, chunks by group, so 16-byte accesses do not conflict
 #pragma unroll
-    for (int h = 0; h < RPT; ++h) {
-      const int line = (row0 + h * R) * lines_per_row + (slice >> 1);
-      const int c0 = (slice & 1) * 4;
+      for (int g = 0; g < G; ++g) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) chunk_off[h][c] = uint32_t(line) * 128u + (uint32_t((c0 + c) ^ (line & 7)) << 4);
-    }
-
-    int s = 0;
-    uint32_t ph = 0;
-    int it = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-      const int sb = it % kStatBufs;
-      const bool got = mbar_wait(&full[s], ph, wc);
-      if (!__all_sync(0xffffffffu, got && !flags[0])) {  // warp-uniform exit
-        flags[0] = 1;
-        break;
-      }
-      const uint8_t* st = stages + size_t(s) * p.tile_bytes;
-
-      f2 w[RPT][16];
-#pragma unroll
-      for (int h = 0; h < RPT; ++h) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (active) v = *reinterpret_cast<const uint4*>(st + chunk_off[h][c]);
-          w[h][4 * c + 0] = pk(bf16lo(v.x), bf16hi(v.x));
-          w[h][4 * c + 1] = pk(bf16lo(v.y), bf16hi(v.y));
-          w[h][4 * c + 2] = pk(bf16lo(v.z), bf16hi(v.z));
-          w[h][4 * c + 3] = pk(bf16lo(v.w), bf16hi(v.w));
+        for (int c = 0; c < CH; ++c) {
+          const f2 a = w[g * GP + 2 * c], b = w[g * GP + 2 * c + 1];
+          *reinterpret_cast<float4*>(xb + (tl * G + (g ^ tl)) * (GS * 4) + ((c ^ csw) << 4)) =
+              make_float4(a.x, a.y, b.x, b.y);
         }
       }
-      mbar_arrive(&empty[s]);  // this thread is done with the stage
-      if (++s == p.nstage) {
-        s = 0;
-        ph ^= 1u;
-      }
-
-      if (has_mult) {
+      __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 m4 = msm[i * S + slice];
-          const f2 ma = pk(m4.x, m4.y), mb = pk(m4.z, m4.w);
+      for (int g = 0; g < G; ++g) {
 #pragma unroll
-          for (int h = 0; h < RPT; ++h) {
-            w[h][2 * i] = mul2(w[h][2 * i], ma);
-            w[h][2 * i + 1] = mul2(w[h][2 * i + 1], mb);
-          }
+        for (int c = 0; c < CH; ++c) {
+          const float4 v = *reinterpret_cast<const float4*>(xb + (g * G + (tl ^ g)) * (GS * 4) +
+                                                            ((c ^ csw) << 4));
+          w[g * GP + 2 * c] = pk(v.x, v.y);
+          w[g * GP + 2 * c + 1] = pk(v.z, v.w);
         }
       }
-      // first channel of each block (Y[b,0]) for the row mean / row sum
-      if (need_sum && active && member == 0) {
+      __syncwarp();
+      // index bits 5..4+LX are now the register-group bits
 #pragma unroll
-        for (int h = 0; h < RPT; ++h) {
-          float* yrow = y0buf + (sb * RT + row0 + h * R) * BP;
-#pragma unroll
-          for (int b = 0; b < BPT; ++b) yrow[blk * BPT + b] = w[h][(b * N) >> 1].x;
-        }
-      }
-      // index bit 0: the two halves of a pair
-#pragma unroll
-      for (int h = 0; h < RPT; ++h) {
+      for (int k = 0; k < LX; ++k) {
+        const int hh = GP << k;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float a = w[h][i].x, b = w[h][i].y;
-          w[h][i] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
-        }
-      }
-      // index bits 1 .. LREG-1: between pairs
-#pragma unroll
-      for (int bit = 1; bit < LREG; ++bit) {
-        const int hh = 1 << (bit - 1);
-#pragma unroll
-        for (int h = 0; h < RPT; ++h) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if ((i & hh) == 0) {
-              const f2 x = w[h][i], y = w[h][i + hh];
-              w[h][i] = add2(x, y);
-              w[h][i + hh] = sub2(x, y);
-            }
+          if ((i & hh) == 0) {
+            const f2 x = w[i], y = w[i + hh];
+            w[i] = add2(x, y);
+            w[i + hh] = sub2(x, y);
           }
         }
       }
-      if (XPOSE) {
-        // swap index bits 5..4+LX (lanes of a G-lane group) with bits
-        // 5-LX..4 (register groups of GS elements); slots XOR-swizzled by
-        // lane, chunks by group, so 16-byte accesses do not conflict
+    }
+    // remaining index bits (5+LX and up) across lanes
 #pragma unroll
-        for (int h = 0; h < RPT; ++h) {
+    for (int j = 0; j < NSHFL; ++j) {
+      const int mask = 1 << (LX + j);
+      const float sg = (lane & mask) ? -1.0f : 1.0f;
+      const f2 sg2 = pk(sg, sg);
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int c = 0; c < CH; ++c) {
-              const f2 a = w[h][g * GP + 2 * c], b = w[h][g * GP + 2 * c + 1];
-              *reinterpret_cast<float4*>(xb + (tl * G + (g ^ tl)) * (GS * 4) + ((c ^ csw) << 4)) =
-                  make_float4(a.x, a.y, b.x, b.y);
-            }
-          }
-          __syncwarp();
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int c = 0; c < CH; ++c) {
-              const float4 v = *reinterpret_cast<const float4*>(xb + (g * G + (tl ^ g)) * (GS * 4) +
-                                                                ((c ^ csw) << 4));
-              w[h][g * GP + 2 * c] = pk(v.x, v.y);
-              w[h][g * GP + 2 * c + 1] = pk(v.z, v.w);
-            }
-          }
-          __syncwarp();
-        }
-        // index bits 5..4+LX are now the register-group bits
-#pragma unroll
-        for (int k = 0; k < LX; ++k) {
-          const int hh = GP << k;
-#pragma unroll
-          for (int h = 0; h < RPT; ++h) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if ((i & hh) == 0) {
-                const f2 x = w[h][i], y = w[h][i + hh];
-                w[h][i] = add2(x, y);
-                w[h][i + hh] = sub2(x, y);
-              }
-            }
-          }
-        }
+      for (int i = 0; i < 16; ++i) {
+        const f2 o = pk(__shfl_xor_sync(0xffffffffu, w[i].x, mask),
+                        __shfl_xor_sync(0xffffffffu, w[i].y, mask));
+        w[i] = fma2(w[i], sg2, o);
       }
-      // remaining index bits (5+LX and up) across lanes
-#pragma unroll
-      for (int j = 0; j < NSHFL; ++j) {
-        const int mask = 1 << (LX + j);
-        const float sg = (lane & mask) ? -1.0f : 1.0f;
-        const f2 sg2 = pk(sg, sg);
-#pragma unroll
-        for (int h = 0; h < RPT; ++h) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const f2 o = pk(__shfl_xor_sync(0xffffffffu, w[h][i].x, mask),
-                            __shfl_xor_sync(0xffffffffu, w[h][i].y, mask));
-            w[h][i] = fma2(w[h][i], sg2, o);
-          }
-        }
-      }
+    }
 
-      // row max / min, one row barrier per row (S arrivals)
-      bool ok = true;
+    // row max / min: reduce over this warp's lanes of the row, one atomic per
+    // warp segment; the segment that completes the row finalizes it
+    float mx = max3(w[0].x, w[0].y, w[1].x);
+    float mn = min3(w[0].x, w[0].y, w[1].x);
+    mx = fmaxf(mx, w[1].y);
+    mn = fminf(mn, w[1].y);
 #pragma unroll
-      for (int h = 0; h < RPT; ++h) {
-        float mx = max3(w[h][0].x, w[h][0].y, w[h][1].x);
-        float mn = min3(w[h][0].x, w[h][0].y, w[h][1].x);
-        mx = fmaxf(mx, w[h][1].y);
-        mn = fminf(mn, w[h][1].y);
-#pragma unroll
-        for (int i = 2; i < 16; ++i) {
-          mx = max3(mx, w[h][i].x, w[h][i].y);
-          mn = min3(mn, w[h][i].x, w[h][i].y);
-        }
-        if (active) {
-          const int r = row0 + h * R;
-          atomicMax(&rowmax[sb * RT + r], ord_f32(mx));
-          atomicMin(&rowmin[sb * RT + r], ord_f32(mn));
-          mbar_arrive(&rowbar[r]);
-        }
-      }
-      if (active) {
-#pragma unroll
-        for (int h = 0; h < RPT; ++h) ok = ok && mbar_wait(&rowbar[row0 + h * R], uint32_t(it & 1), wc);
-      }
-      if (!__all_sync(0xffffffffu, ok)) {
-        flags[0] = 1;
-        break;
-      }
-      if (!active) continue;
-
-#pragma unroll
-      for (int h = 0; h < RPT; ++h) {
-        const int r = row0 + h * R;
-        float rsum = 0.0f;
-        if (need_sum) {
-          // sum of the row's first channels, in block order
-          const float4* y4 = reinterpret_cast<const float4*>(y0buf + (sb * RT + r) * BP);
-          for (int b4 = 0; b4 < (B + 3) / 4; ++b4) {
-            const float4 v = y4[b4];
-            rsum = __fadd_rn(rsum, v.x);
-            if (4 * b4 + 1 < B) rsum = __fadd_rn(rsum, v.y);
-            if (4 * b4 + 2 < B) rsum = __fadd_rn(rsum, v.z);
-            if (4 * b4 + 3 < B) rsum = __fadd_rn(rsum, v.w);
+    for (int i = 2; i < 16; ++i) {
+      mx = max3(mx, w[i].x, w[i].y);
+      mn = min3(mn, w[i].x, w[i].y);
+    }
+    __syncwarp();  // this warp's first-channel stores precede its leaders' arrivals
+    bool ok = true;
+    if (active) {
+      const uint32_t umx = __reduce_max_sync(segmask, ord_f32(mx));
+      const uint32_t umn = __reduce_min_sync(segmask, ord_f32(mn));
+      if (seg_leader) {
+        atomicMax(&pmax[sr], umx);
+        atomicMin(&pmin[sr], umn);
+        __threadfence_block();
+        const uint32_t before = atomicAdd(&cnt[sr], uint32_t(seg_len));
+        if (before + uint32_t(seg_len) == uint32_t(S)) {
+          // last segment of the row: every slice's max, min and first
+          // channels are in shared memory
+          __threadfence_block();
+          const int64_t row = tile * R + row0;
+          float rsum = 0.0f;
+          if (need_sum) {
+            const float* yrow = y0buf + sr * BP;
+            for (int b = 0; b < B; ++b) rsum = __fadd_rn(rsum, yrow[b]);  // block order
           }
-        }
-        const float m_hat = CENTER ? n_over_k * rsum : 0.0f;
-        const float rmx = unord_f32(rowmax[sb * RT + r]);
-        const float rmn = unord_f32(rowmin[sb * RT + r]);
-        const float a_hat = fmaxf(__fsub_rn(rmx, m_hat), __fsub_rn(m_hat, rmn));
-        float r_rec;
-        if (MODE == 0) {
-          r_rec = a_hat > 0.0f ? __fdiv_rn(qf, a_hat) : 0.0f;
-        } else {
-          r_rec = r_tensor;
-        }
-        const int64_t row = tile * RT + r;
-        const bool valid = row < T;
-        if (slice == 0) {
-          // stats buffer of the previous tile is free again (see the row barrier)
-          rowmax[((it + 2) % kStatBufs) * RT + r] = 0u;
-          rowmin[((it + 2) % kStatBufs) * RT + r] = 0xFFFFFFFFu;
-          if (valid) {
+          const float m_hat = CENTER ? n_over_k * rsum : 0.0f;
+          const float rmx = unord_f32(pmax[sr]);
+          const float rmn = unord_f32(pmin[sr]);
+          const float a_hat = fmaxf(__fsub_rn(rmx, m_hat), __fsub_rn(m_hat, rmn));
+          float r_rec = r_tensor;
+          if (MODE == 0) r_rec = a_hat > 0.0f ? __fdiv_rn(qf, a_hat) : 0.0f;
+          res[sr] = make_float2(m_hat, r_rec);
+          pmax[sr] = 0u;  // ready for tile it + 2
+          pmin[sr] = 0xFFFFFFFFu;
+          cnt[sr] = 0u;
+          if (row < T) {
             if (MODE == 0) p.scale[row] = (a_hat / qf) * p.inv_sqrt_n;
-            if (MODE == 1) atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])),
-                                     __float_as_uint(a_hat));
+            if (MODE == 1)
+              atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])),
+                        __float_as_uint(a_hat));
             if (kQuantize && p.mean) p.mean[row] = m_hat * p.inv_sqrt_n;
             if (p.rowsum) p.rowsum[row] = rsum * p.sqrt_n;  // sqrt(n) * sum_b Y[b,0]
           }
+          // test hook: the first row of this CTA's first tile is never released
+          if (!(p.fault_withhold_row && it == 0 && row0 == 0)) mbar_arrive(&rowbar[row0]);
         }
-        if (!kQuantize || !valid) continue;
+      }
+      ok = mbar_wait(&rowbar[row0], uint32_t(it & 1), wc);
+    }
+    if (!__all_sync(0xffffffffu, ok && !flags[0])) {  // warp-uniform exit
+      flags[0] = 1;
+      break;
+    }
+    if (!active) continue;
 
-        const f2 mh2 = pk(m_hat, m_hat), rr2 = pk(r_rec, r_rec), mg2 = pk(kRoundMagic, kRoundMagic);
-        uint32_t words[8];
+    const int64_t row = tile * R + row0;
+    if (!kQuantize || row >= T) continue;
+    const float2 st = res[sr];
+    const f2 mh2 = pk(st.x, st.x), rr2 = pk(st.y, st.y), mg2 = pk(kRoundMagic, kRoundMagic);
+    uint32_t words[8];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          uint32_t b[4];
+    for (int g = 0; g < 8; ++g) {
+      uint32_t b[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const f2 t = fma2(sub2(w[h][2 * g + u], mh2), rr2, mg2);
-            b[2 * u] = __float_as_uint(t.x);
-            b[2 * u + 1] = __float_as_uint(t.y);
-          }
-          if (kClamp) {
+      for (int u = 0; u < 2; ++u) {
+        const f2 t = fma2(sub2(w[2 * g + u], mh2), rr2, mg2);
+        b[2 * u] = __float_as_uint(t.x);
+        b[2 * u + 1] = __float_as_uint(t.y);
+      }
+      if (kClamp) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              int c = int(b[u] - kRoundMagicBits);
-              b[u] = uint32_t(max(-p.q, min(p.q, c)));
-            }
-          }
-          words[g] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
-                                 0x5410);
+        for (int u = 0; u < 4; ++u) {
+          int c = int(b[u] - kRoundMagicBits);
+          b[u] = uint32_t(max(-p.q, min(p.q, c)));
         }
-        int8_t* crow = p.codes + row * K;
-        if (!XPOSE) {
-          uint4* dst = reinterpret_cast<uint4*>(crow + slice * 32);
-          dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-          dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-        } else {
-          // register group g: index bits 5..4+LX = g, bits 5-LX..4 = tl, bits
-          // 5+LX.. = member >> LX; GS consecutive codes per group
-          int8_t* base = crow + blk * N + GS * tl + (32 * G) * (member >> LX);
-          constexpr int WPG = GS / 4;  // words per group
+      }
+      words[g] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                             0x5410);
+    }
+    int8_t* crow = p.codes + row * K;
+    if (!XPOSE) {
+      uint4* dst = reinterpret_cast<uint4*>(crow + slice * 32);
+      dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+      dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    } else {
+      // register group g: index bits 5..4+LX = g, bits 5-LX..4 = tl, bits
+      // 5+LX.. = member >> LX; GS consecutive codes per group
+      int8_t* base = crow + blk * N + GS * tl + (32 * G) * (member >> LX);
+      constexpr int WPG = GS / 4;  // words per group
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            if (WPG == 4) {
-              *reinterpret_cast<uint4*>(base + 32 * g) =
-                  make_uint4(words[4 * g], words[4 * g + 1], words[4 * g + 2], words[4 * g + 3]);
-            } else if (WPG == 2) {
-              *reinterpret_cast<uint2*>(base + 32 * g) = make_uint2(words[2 * g], words[2 * g + 1]);
-            } else {
-              *reinterpret_cast<uint32_t*>(base + 32 * g) = words[g];
-            }
-          }
+      for (int g = 0; g < G; ++g) {
+        if (WPG == 4) {
+          *reinterpret_cast<uint4*>(base + 32 * g) =
+              make_uint4(words[4 * g], words[4 * g + 1], words[4 * g + 2], words[4 * g + 3]);
+        } else if (WPG == 2) {
+          *reinterpret_cast<uint2*>(base + 32 * g) = make_uint2(words[2 * g], words[2 * g + 1]);
+        } else {
+          *reinterpret_cast<uint32_t*>(base + 32 * g) = words[g];
         }
       }
     }

@@ -210,12 +210,13 @@ hq_status hq_debug_set_gemm_variant(int variant);
 
 /* Test hook for the bounded-wait error path, without faulting the GPU:
  *   HQ_FAULT_NONE (0)                    normal operation;
- *   HQ_FAULT_QUANT_WITHHOLD_LOAD (1)     each CTA of the next activation
- *       quantize launches skips its first tile copy, so the barrier it waits
- *       on never completes; the bounded wait expires, the kernel records
- *       HQ_ERR_TIMEOUT, lets its other copies land and exits.
+ *   HQ_FAULT_QUANT_WITHHOLD_ROW (1)      in each CTA of the next activation
+ *       quantize launches, the statistics of the first row of the first
+ *       tile are never released, so the threads of that row wait on a
+ *       barrier that never completes; the bounded wait expires, the kernel
+ *       records HQ_ERR_TIMEOUT and exits (it has no copies in flight).
  * Host state, applies to launches issued after the call. */
-enum { HQ_FAULT_NONE = 0, HQ_FAULT_QUANT_WITHHOLD_LOAD = 1 };
+enum { HQ_FAULT_NONE = 0, HQ_FAULT_QUANT_WITHHOLD_ROW = 1 };
 hq_status hq_debug_inject_fault(int kind);
 
 #ifdef __cplusplus

@@ -405,7 +405,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(hq):
     desc = hq.LayerDesc(1152, 16, 128, a_bits=4)
     Xb = synth.make_x(synth.CONFIGS[2].with_tokens(64))
     hq.hq_debug_set_wait_limit(2_000_000)  # 2 ms
-    hq.hq_debug_inject_fault(hq.HQ_FAULT_QUANT_WITHHOLD_LOAD)
+    hq.hq_debug_inject_fault(hq.HQ_FAULT_QUANT_WITHHOLD_ROW)
     try:
         X = to_dev_u16(Xb, torch)
         codes = torch.empty((64, 1152), dtype=torch.int8, device="cuda")
