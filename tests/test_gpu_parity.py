@@ -420,3 +420,63 @@ def test_bounded_wait_reports_timeout_and_context_survives(hq):
     codes2, scale2, _ = _gpu_quantize(hq, desc, Xb)
     ref = oracle.quantize_act(Xb, 128, 4)
     check_codes(codes2, ref["codes"], ref["tie"], "after timeout")
+
+
+# ---------------------------------------------------------------------------
+# steps issued back to back on one stream
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("variant", ["auto", "cta_pair"])
+def test_back_to_back_steps_match_isolated_steps(hq, variant):
+    """quantize -> linear -> quantize -> ... with no synchronization between
+    launches (eagerly and from one CUDA graph), one codes buffer reused by
+    every step, must give bit-identical results to the same steps run one at
+    a time."""
+    cfg = synth.CONFIGS[2].with_tokens(1000)
+    Xb, Wb, bb = synth.make_layer(cfg)
+    T, K = Xb.shape
+    N = Wb.shape[0]
+    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering)
+    hq.hq_debug_set_gemm_variant(hq.HQ_GEMM_CTA_PAIR if variant == "cta_pair" else hq.HQ_GEMM_AUTO)
+    try:
+        X0 = to_dev_u16(Xb, torch)
+        absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
+        hq.hq_calib_act_absmax(desc, X0, absmax)
+        layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), absmax,
+                                       cfg.alpha)
+        # three different token batches: the rows of X rotated
+        Xs = [torch.roll(X0, shifts=s * 97, dims=0).contiguous() for s in range(3)]
+        iso = []
+        for X in Xs:
+            Y = layer(X)
+            assert hq.hq_check_device_error() == 0
+            iso.append(Y.clone())
+        # eager, no synchronization between steps (one codes buffer reused:
+        # each quantize overwrites what the previous GEMM reads)
+        outs = [torch.empty((T, N), dtype=torch.bfloat16, device="cuda") for _ in Xs]
+        bufs = layer.buffers(T)
+        mean = bufs["a_mean"] if cfg.centering else None
+
+        def steps():
+            for X, Y in zip(Xs, outs):
+                hq.hq_quantize_act(desc, X, layer.sigma_inv, bufs["a_codes"], bufs["a_scale"],
+                                   bufs["a_mean"], layer.workspace)
+                hq.hq_linear(desc, bufs["a_codes"], bufs["a_scale"], mean, layer.w_codes,
+                             layer.w_scale, layer.colsum, layer.bias_f32, Y)
+
+        steps()
+        assert hq.hq_check_device_error() == 0
+        for Y, R in zip(outs, iso):
+            assert torch.equal(Y.view(torch.int16), R.view(torch.int16))
+        for Y in outs:
+            Y.fill_(float("nan"))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            steps()
+        g.replay()
+        assert hq.hq_check_device_error() == 0
+        for Y, R in zip(outs, iso):
+            assert torch.equal(Y.view(torch.int16), R.view(torch.int16))
+    finally:
+        hq.hq_debug_set_gemm_variant(hq.HQ_GEMM_AUTO)
