@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     pmin[i] = 0xFFFFFFFFu;
     cnt[i] = 0u;
   }
+  for (int i = tid; i < 2 * R * BP; i += blockDim.x) y0buf[i] = 0.0f;  // padding stays zero
   if (has_mult) {
     // chunk-major copy: thread `slice` reads chunk c at msm[c * S + slice], so
     // consecutive slices hit consecutive 16-byte words
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   }
   const float n_over_k = float(N) / float(K);
   const float qf = float(p.q);
+  const float s_unit = p.inv_sqrt_n / qf;
 
   int it = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
@@ -383,21 +385,27 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
           const int64_t row = tile * R + row0;
           float rsum = 0.0f;
           if (need_sum) {
-            const float* yrow = y0buf + sr * BP;
-            for (int b = 0; b < B; ++b) rsum = __fadd_rn(rsum, yrow[b]);  // block order
+            // block order; the padding past B holds zeros, which leave the sum unchanged
+            const float4* y4 = reinterpret_cast<const float4*>(y0buf + sr * BP);
+            for (int b4 = 0; b4 < (B + 3) / 4; ++b4) {
+              const float4 v = y4[b4];
+              rsum = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(rsum, v.x), v.y), v.z), v.w);
+            }
           }
           const float m_hat = CENTER ? n_over_k * rsum : 0.0f;
           const float rmx = unord_f32(pmax[sr]);
           const float rmn = unord_f32(pmin[sr]);
           const float a_hat = fmaxf(__fsub_rn(rmx, m_hat), __fsub_rn(m_hat, rmn));
           float r_rec = r_tensor;
-          if (MODE == 0) r_rec = a_hat > 0.0f ? __fdiv_rn(qf, a_hat) : 0.0f;
+          // q / a_hat to within 2 ulp: moves a code only when V * q / a_hat
+          // lies within a few ulp of a rounding boundary
+          if (MODE == 0) r_rec = a_hat > 0.0f ? __fdividef(qf, a_hat) : 0.0f;
           res[sr] = make_float2(m_hat, r_rec);
           pmax[sr] = 0u;  // ready for tile it + 2
           pmin[sr] = 0xFFFFFFFFu;
           cnt[sr] = 0u;
           if (row < T) {
-            if (MODE == 0) p.scale[row] = (a_hat / qf) * p.inv_sqrt_n;
+            if (MODE == 0) p.scale[row] = a_hat * s_unit;  // a_hat / (q sqrt(n))
             if (MODE == 1)
               atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])),
                         __float_as_uint(a_hat));
