@@ -249,7 +249,8 @@ def oracle_step(cfg, Xb, sig, w, rows, nthreads):
                             centering=cfg.centering, sigma=sig, rows=rows, want_tie=False,
                             nthreads=nthreads)
     acc = oracle.gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
-    oracle.epilogue(acc, a["scale"], w["scale"], colsum=w["colsum"], bias=w["bias"],
+    oracle.epilogue(acc, a["scale"], w["scale"], colsum=oracle.correction(w, cfg.centering),
+                    bias=w["bias"],
                     mean=a["mean"] if cfg.centering else None)
 
 

@@ -23,7 +23,7 @@ import threading
 __all__ = [
     "HQError", "LayerDesc", "load_library", "library_path", "exported_symbols",
     "HQ_PER_TOKEN", "HQ_PER_TENSOR_DYNAMIC", "HQ_PER_TENSOR_STATIC",
-    "HQ_CENTER_NONE", "HQ_CENTER_TOKEN_MEAN", "HQ_CODES_I8",
+    "HQ_CENTER_NONE", "HQ_CENTER_TOKEN_MEAN", "HQ_CENTER_TOKEN_MEAN_PRE", "HQ_CODES_I8",
     "HQ_FAULT_NONE", "HQ_FAULT_QUANT_WITHHOLD_ROW", "STATUS_NAMES",
     "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
@@ -36,7 +36,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libhq.so")
 
 HQ_PER_TOKEN, HQ_PER_TENSOR_DYNAMIC, HQ_PER_TENSOR_STATIC = 0, 1, 2
-HQ_CENTER_NONE, HQ_CENTER_TOKEN_MEAN = 0, 1
+HQ_CENTER_NONE, HQ_CENTER_TOKEN_MEAN, HQ_CENTER_TOKEN_MEAN_PRE = 0, 1, 2
 HQ_CODES_I8 = 0
 HQ_FAULT_NONE, HQ_FAULT_QUANT_WITHHOLD_ROW = 0, 1
 HQ_GEMM_AUTO, HQ_GEMM_SINGLE_CTA, HQ_GEMM_CTA_PAIR = 0, 1, 2
@@ -279,7 +279,7 @@ class HadamardQuantLinear:
         if Y is None:
             Y = torch.empty((T, self.desc.N), dtype=torch.bfloat16, device=X.device)
         b = self.quantize(X)
-        mean = b["a_mean"] if self.desc.centering == HQ_CENTER_TOKEN_MEAN else None
+        mean = b["a_mean"] if self.desc.centering != HQ_CENTER_NONE else None
         hq_linear(self.desc, b["a_codes"], b["a_scale"], mean, self.w_codes, self.w_scale,
                   self.colsum, self.bias_f32, Y, acc_debug)
         return Y

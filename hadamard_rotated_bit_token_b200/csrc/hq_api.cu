@@ -31,7 +31,7 @@ struct DeviceState {
   int sm_count = 0;
   int cc_major = 0, cc_minor = 0;
   unsigned int* err = nullptr;
-  bool quant_attr_set[8][4][2] = {};
+  bool quant_attr_set[8][4][3] = {};
   int pair_clusters = -1;  // co-resident clusters of the CTA-pair GEMM (-1: not queried)
 };
 
@@ -99,7 +99,7 @@ hq_status check_desc(const hq_layer_desc* d) {
   if (d == nullptr) return HQ_ERR_INVALID_ARGUMENT;
   if (d->N <= 0) return HQ_ERR_INVALID_ARGUMENT;
   if (d->act_gran < HQ_PER_TOKEN || d->act_gran > HQ_PER_TENSOR_STATIC) return HQ_ERR_INVALID_ARGUMENT;
-  if (d->centering < HQ_CENTER_NONE || d->centering > HQ_CENTER_TOKEN_MEAN)
+  if (d->centering < HQ_CENTER_NONE || d->centering > HQ_CENTER_TOKEN_MEAN_PRE)
     return HQ_ERR_INVALID_ARGUMENT;
   hq_status s = check_k_side(d);
   if (s != HQ_OK) return s;
@@ -172,14 +172,14 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
   return HQ_OK;
 }
 
-hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, bool center, cudaStream_t st) {
+hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, int center, cudaStream_t st) {
   const int logn = L.logn;
   const void* fn = quant_kernel_ptr(logn, mode, center);
   if (fn == nullptr) return HQ_ERR_UNSUPPORTED;
   if (L.p.T <= 0) return HQ_OK;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    bool& set = dev->quant_attr_set[logn - 4 < 0 ? 0 : logn - 4][mode][center ? 1 : 0];
+    bool& set = dev->quant_attr_set[logn - 4 < 0 ? 0 : logn - 4][mode][center];
     if (!set) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024) !=
           cudaSuccess)
@@ -331,8 +331,9 @@ hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const
   L.p.scale = w_scale;
   L.p.mean = nullptr;
   L.p.rowsum = colsum;
+  L.p.rowsum_pre = desc->centering == HQ_CENTER_TOKEN_MEAN_PRE ? 1 : 0;
   L.p.q = (1 << (desc->w_bits - 1)) - 1;
-  s = run_quant(dev, L, 0, false, st);
+  s = run_quant(dev, L, 0, 0, st);
   if (s != HQ_OK) return s;
   if (bias) return from_cuda(launch_bf16_to_f32(bias, bias_f32, N, st));
   return from_cuda(launch_fill(bias_f32, N, 0.0f, st));
@@ -374,7 +375,7 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   L.p.rowsum = nullptr;
   L.p.q = (1 << (desc->a_bits - 1)) - 1;
   L.p.fault_withhold_row = g_fault == HQ_FAULT_QUANT_WITHHOLD_ROW ? 1 : 0;
-  const bool center = desc->centering == HQ_CENTER_TOKEN_MEAN;
+  const int center = desc->centering;  // HQ_CENTER_* = the kernel's centering mode
   if (desc->act_gran == HQ_PER_TOKEN) return run_quant(dev, L, 0, center, st);
   if (desc->act_gran == HQ_PER_TENSOR_STATIC) {
     L.p.static_scale = a_scale;

@@ -14,7 +14,8 @@ struct QuantParams {
   int8_t* codes;              // [T,K] int8 codes
   float* scale;               // [T] per-row scales, or [1] for per-tensor modes
   float* mean;                // [T] per-row mean of the rotated row (real units), or null
-  float* rowsum;              // [T] per-row sum of the rotated row (real units), or null
+  float* rowsum;              // [T] per-row correction sum (see rowsum_pre), or null
+  int rowsum_pre;             // rowsum = sum_k Y[t,k] (1) or the rotated row's sum (0)
   unsigned int* tensor_max;   // per-tensor: bits of max |V_hat| (unnormalized)
   const float* static_scale;  // per-tensor static scale (real units)
   int64_t T;
@@ -29,10 +30,11 @@ struct QuantParams {
   unsigned long long wait_ns; // bounded-wait limit
 };
 
-// Returns the kernel entry for log2(n) in [4,10], mode in [0,3]; the kernel
+// Returns the kernel entry for log2(n) in [4,10], mode in [0,3], centering
+// in [0,2] (the HQ_CENTER_* values); the kernel
 // takes (QuantParams p) and runs R * S active threads per CTA (rounded up to
 // whole warps, at most quant_max_threads()).
-const void* quant_kernel_ptr(int logn, int mode, bool center);
+const void* quant_kernel_ptr(int logn, int mode, int center);
 int quant_max_threads();
 // Dynamic shared memory of one quantizer CTA: R rows per tile, K channels,
 // B blocks per row, `nwarps` warps, transposes for n >= 64.

@@ -136,8 +136,12 @@ size_t quant_smem_bytes(int R, int K, int B, int nwarps, bool xpose) {
 // MODE 1: per-tensor pass 1: only the tensor-wide max |V| (into tensor_max)
 // MODE 2: per-tensor pass 2: scale from tensor_max
 // MODE 3: per-tensor static scale from static_scale[0] (real units)
-template <int LOGN, int MODE, bool CENTER>
+// CM: 0 no centering, 1 the row mean removed after the rotation, 2 removed
+// before it (the HQ_CENTER_* values).
+template <int LOGN, int MODE, int CM>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const QuantParams p) {
+  constexpr bool CENTER = (CM == 1);
+  constexpr bool PRE = (CM == 2);
   constexpr int N = 1 << LOGN;
   constexpr int LREG = LOGN < 5 ? LOGN : 5;        // index bits inside a thread's slice
   constexpr int LOG_TT = LOGN > 5 ? LOGN - 5 : 0;  // index bits across threads
@@ -178,7 +182,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);
   const WaitCtl wc{p.err, p.wait_ns};
   const bool has_mult = p.mult != nullptr;
-  const bool need_sum = CENTER || p.rowsum != nullptr;
+  const bool need_sum = CM != 0 || p.rowsum != nullptr;
+  // the rows' block sums (first rotated channel of each block) instead of
+  // their blocks' first input channels
+  const bool block_sums = PRE || (p.rowsum != nullptr && p.rowsum_pre);
 
   const bool active = tid < R * S;
   const int row0 = active ? tid / S : 0;  // this thread's row of every tile
@@ -254,6 +261,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     r_tensor = s > 0.0f ? __fdiv_rn(1.0f, s * p.sqrt_n) : 0.0f;
   }
   const float n_over_k = float(N) / float(K);
+  const float inv_k = 1.0f / float(K);
   const float qf = float(p.q);
   const float s_unit = p.inv_sqrt_n / qf;
 
@@ -280,7 +288,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
       }
     }
     // first channel of each block (Y[b,0]) for the row mean / row sum
-    if (need_sum && active && member == 0) {
+    if (need_sum && !block_sums && active && member == 0) {
       float* yrow = y0buf + sr * BP;
 #pragma unroll
       for (int b = 0; b < BPT; ++b) yrow[blk * BPT + b] = w[(b * N) >> 1].x;
@@ -357,6 +365,20 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
       }
     }
 
+    // each block's first rotated channel is its block sum sum_j Y[b,j]; the
+    // row needs them when centering before the rotation (they are the only
+    // channels it moves) and for the weights' pre-rotation correction
+    float first[BPT];
+    if (block_sums && member == 0) {
+#pragma unroll
+      for (int b = 0; b < BPT; ++b) {
+        first[b] = w[(b * N) >> 1].x;
+        if (active) y0buf[sr * BP + blk * BPT + b] = first[b];
+        // left out of this slice's max / min (channel 1 of block 0 stands in)
+        if (PRE) w[(b * N) >> 1].x = w[0].y;
+      }
+    }
+
     // row max / min: reduce over this warp's lanes of the row, one atomic per
     // warp segment; the segment that completes the row finalizes it
     float mx = max3(w[0].x, w[0].y, w[1].x);
@@ -367,6 +389,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     for (int i = 2; i < 16; ++i) {
       mx = max3(mx, w[i].x, w[i].y);
       mn = min3(mn, w[i].x, w[i].y);
+    }
+    if (PRE && member == 0) {
+#pragma unroll
+      for (int b = 0; b < BPT; ++b) w[(b * N) >> 1].x = first[b];
     }
     __syncwarp();  // this warp's first-channel stores precede its leaders' arrivals
     bool ok = true;
@@ -392,10 +418,24 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
               rsum = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(rsum, v.x), v.y), v.z), v.w);
             }
           }
-          const float m_hat = CENTER ? n_over_k * rsum : 0.0f;
-          const float rmx = unord_f32(pmax[sr]);
-          const float rmn = unord_f32(pmin[sr]);
-          const float a_hat = fmaxf(__fsub_rn(rmx, m_hat), __fsub_rn(m_hat, rmn));
+          // CM 1: m_hat = mean of the rotated row, subtracted everywhere.
+          // CM 2: mu = rsum / K (the blocks' sums add up to the row's sum);
+          // the rotated row changes only at each block's first channel, by
+          // -n mu (unnormalized transform), which m_hat then holds.
+          const float mu = PRE ? rsum * inv_k : 0.0f;
+          const float m_hat = CENTER ? n_over_k * rsum : (PRE ? float(N) * mu : 0.0f);
+          float rmx = unord_f32(pmax[sr]);
+          float rmn = unord_f32(pmin[sr]);
+          if (PRE) {
+            const float* yrow = y0buf + sr * BP;
+            for (int b = 0; b < B; ++b) {
+              const float v = __fsub_rn(yrow[b], m_hat);
+              rmx = fmaxf(rmx, v);
+              rmn = fminf(rmn, v);
+            }
+          }
+          const float a_hat = PRE ? fmaxf(rmx, -rmn)
+                                  : fmaxf(__fsub_rn(rmx, m_hat), __fsub_rn(m_hat, rmn));
           float r_rec = r_tensor;
           // q / a_hat to within 2 ulp: moves a code only when V * q / a_hat
           // lies within a few ulp of a rounding boundary
@@ -409,8 +449,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
             if (MODE == 1)
               atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])),
                         __float_as_uint(a_hat));
-            if (kQuantize && p.mean) p.mean[row] = m_hat * p.inv_sqrt_n;
-            if (p.rowsum) p.rowsum[row] = rsum * p.sqrt_n;  // sqrt(n) * sum_b Y[b,0]
+            if (kQuantize && p.mean) p.mean[row] = PRE ? mu : m_hat * p.inv_sqrt_n;
+            // sum_k sigma_k W[n,k] = the blocks' sums, or
+            // sum_k W~[n,k] = sqrt(n) * sum_b Y[b,0]
+            if (p.rowsum) p.rowsum[row] = p.rowsum_pre ? rsum : rsum * p.sqrt_n;
           }
           // test hook: the first row of this CTA's first tile is never released
           if (!(p.fault_withhold_row && it == 0 && row0 == 0)) mbar_arrive(&rowbar[row0]);
@@ -427,7 +469,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     const int64_t row = tile * R + row0;
     if (!kQuantize || row >= T) continue;
     const float2 st = res[sr];
-    const f2 mh2 = pk(st.x, st.x), rr2 = pk(st.y, st.y), mg2 = pk(kRoundMagic, kRoundMagic);
+    if (PRE && member == 0) {
+#pragma unroll
+      for (int b = 0; b < BPT; ++b) w[(b * N) >> 1].x = __fsub_rn(w[(b * N) >> 1].x, st.x);
+    }
+    const float mshift = PRE ? 0.0f : st.x;
+    const f2 mh2 = pk(mshift, mshift), rr2 = pk(st.y, st.y), mg2 = pk(kRoundMagic, kRoundMagic);
     uint32_t words[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
@@ -477,26 +524,36 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
 }
 
 // ---------------------------------------------------------------- dispatch
-template <int MODE, bool CENTER>
+template <int MODE, int CM>
 static const void* pick_by_logn(int logn) {
   switch (logn) {
-    case 4: return (const void*)quant_rows_kernel<4, MODE, CENTER>;
-    case 5: return (const void*)quant_rows_kernel<5, MODE, CENTER>;
-    case 6: return (const void*)quant_rows_kernel<6, MODE, CENTER>;
-    case 7: return (const void*)quant_rows_kernel<7, MODE, CENTER>;
-    case 8: return (const void*)quant_rows_kernel<8, MODE, CENTER>;
-    case 9: return (const void*)quant_rows_kernel<9, MODE, CENTER>;
-    case 10: return (const void*)quant_rows_kernel<10, MODE, CENTER>;
+    case 4: return (const void*)quant_rows_kernel<4, MODE, CM>;
+    case 5: return (const void*)quant_rows_kernel<5, MODE, CM>;
+    case 6: return (const void*)quant_rows_kernel<6, MODE, CM>;
+    case 7: return (const void*)quant_rows_kernel<7, MODE, CM>;
+    case 8: return (const void*)quant_rows_kernel<8, MODE, CM>;
+    case 9: return (const void*)quant_rows_kernel<9, MODE, CM>;
+    case 10: return (const void*)quant_rows_kernel<10, MODE, CM>;
     default: return nullptr;
   }
 }
 
-const void* quant_kernel_ptr(int logn, int mode, bool center) {
+template <int MODE>
+static const void* pick_by_center(int logn, int center) {
+  switch (center) {
+    case 0: return pick_by_logn<MODE, 0>(logn);
+    case 1: return pick_by_logn<MODE, 1>(logn);
+    case 2: return pick_by_logn<MODE, 2>(logn);
+    default: return nullptr;
+  }
+}
+
+const void* quant_kernel_ptr(int logn, int mode, int center) {
   switch (mode) {
-    case 0: return center ? pick_by_logn<0, true>(logn) : pick_by_logn<0, false>(logn);
-    case 1: return center ? pick_by_logn<1, true>(logn) : pick_by_logn<1, false>(logn);
-    case 2: return center ? pick_by_logn<2, true>(logn) : pick_by_logn<2, false>(logn);
-    case 3: return center ? pick_by_logn<3, true>(logn) : pick_by_logn<3, false>(logn);
+    case 0: return pick_by_center<0>(logn, center);
+    case 1: return pick_by_center<1>(logn, center);
+    case 2: return pick_by_center<2>(logn, center);
+    case 3: return pick_by_center<3>(logn, center);
     default: return nullptr;
   }
 }

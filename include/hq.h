@@ -62,7 +62,7 @@ typedef enum hq_status {
 } hq_status;
 
 enum { HQ_PER_TOKEN = 0, HQ_PER_TENSOR_DYNAMIC = 1, HQ_PER_TENSOR_STATIC = 2 };
-enum { HQ_CENTER_NONE = 0, HQ_CENTER_TOKEN_MEAN = 1 };
+enum { HQ_CENTER_NONE = 0, HQ_CENTER_TOKEN_MEAN = 1, HQ_CENTER_TOKEN_MEAN_PRE = 2 };
 enum { HQ_CODES_I8 = 0 };
 
 /* Layer description, host memory, passed by const pointer.
@@ -76,7 +76,14 @@ enum { HQ_CODES_I8 = 0 };
  *               max |X~| (two passes over X).
  *               HQ_PER_TENSOR_STATIC: one scale given by the caller.
  *   centering   HQ_CENTER_TOKEN_MEAN: mu_t = mean over all K channels of the
- *               scaled and rotated token (HadaNorm review Eq. (1)).
+ *               scaled and rotated token, removed after the rotation
+ *               (HadaNorm review, "What carries the argument", Eq. (1)).
+ *               HQ_CENTER_TOKEN_MEAN_PRE: mu_t = mean over all K channels of
+ *               the scaled token Y = X diag(sigma^-1), removed before the
+ *               rotation: V = (Y - mu_t) H, i.e. Eq. (1)'s mu read as the
+ *               vector mu_t 1^T H.  Only each block's first rotated channel
+ *               changes (by -sqrt(n) mu_t); the layer's correction becomes
+ *               mu_t * sum_k sigma_k W[n,k].
  *               HQ_CENTER_NONE: mu = 0.
  *   code_format HQ_CODES_I8 (one signed code per byte). */
 typedef struct hq_layer_desc {
@@ -108,7 +115,8 @@ hq_status hq_calib_act_absmax(const hq_layer_desc* desc, const uint16_t* X,
  *   sigma_inv = 1 / sigma  (fp32 [K]; feeds hq_quantize_act)
  *   W~[n,:]   = (W[n,:] * sigma) H    (W~ = H^T diag(sigma) W in the pages'
  *               orientation), computed with a fast Walsh-Hadamard transform
- *   colsum[n] = sum_k W~[n,k]          (the mu W~ term of b~)
+ *   colsum[n] = sum_k W~[n,k]          (the mu W~ term of b~), or, for
+ *               HQ_CENTER_TOKEN_MEAN_PRE, sum_k sigma_k W[n,k]
  *   w_scale[n]= max_k |W~[n,k]| / q_w,  w_codes = clamp(rne(W~ / w_scale), +-q_w)
  *   bias_f32  = float(bias), or 0 when bias == NULL.
  * Inputs:  W bf16 [N,K], bias bf16 [N] or NULL, act_absmax fp32 [K] or NULL.
@@ -128,13 +136,16 @@ size_t hq_quantize_act_workspace_bytes(const hq_layer_desc* desc, int64_t T);
 /* hq_quantize_act -- runtime activation side of Eq. (1), fused in one pass
  * over X (two for HQ_PER_TENSOR_DYNAMIC):
  *   Y = X diag(sigma^-1); Z = Y H (block fast Walsh-Hadamard transform);
- *   m_t = mean_k Z[t,k] (HQ_CENTER_TOKEN_MEAN) else 0;  V = Z - m;
+ *   HQ_CENTER_TOKEN_MEAN:     m_t = mean_k Z[t,k], V = Z - m;
+ *   HQ_CENTER_TOKEN_MEAN_PRE: m_t = mean_k Y[t,k], V = (Y - m_t) H;
+ *   HQ_CENTER_NONE:           m_t = 0, V = Z;
  *   s = max|V| / q_a per token (or per tensor);  codes = clamp(rne(V/s), +-q_a).
  * Inputs:  X bf16 [T,K]; sigma_inv fp32 [K] or NULL (sigma = 1).
  * Outputs: a_codes int8 [T,K];
  *          a_scale fp32 [T] (HQ_PER_TOKEN) or [1] (per tensor; for
  *            HQ_PER_TENSOR_STATIC it is an INPUT holding s);
- *          a_mean fp32 [T] or NULL (written with zeros when centering is off).
+ *          a_mean fp32 [T] or NULL: m_t, in the units hq_linear multiplies
+ *            by colsum (zeros when centering is off).
  * workspace: device, >= hq_quantize_act_workspace_bytes(), 16-byte aligned,
  *   contents need not be initialised (the call clears what it uses).
  * A token whose max|V| is 0 gets scale 0 and all-zero codes. */

@@ -71,7 +71,7 @@ def _load():
                 _i8p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
             lib.hqo_prepare_weights.argtypes = [
                 ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
-                _u16p, _u16p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+                _u16p, _u16p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
             lib.hqo_gemm_acc.argtypes = [_i8p, _i8p, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_int64, _i64p, ctypes.c_int64, _i64p,
                                          ctypes.c_int]
@@ -193,16 +193,26 @@ def prepare_weights(W_bits, n, bits, bias_bits=None, sigma=None, want_tie=True,
     codes = np.zeros((N, K), dtype=np.int8)
     scale = np.zeros(N, dtype=np.float64)
     colsum = np.zeros(N, dtype=np.float64)
+    corr_pre = np.zeros(N, dtype=np.float64)
     bias = np.zeros(N, dtype=np.float64)
     tie = np.zeros((N, K), dtype=np.float64) if want_tie else None
     Wt = np.zeros((N, K), dtype=np.float64) if want_Wt else None
     rc = _load().hqo_prepare_weights(
         K, N, n, bits, _ptr(W, ctypes.c_uint16), _ptr(b, ctypes.c_uint16),
         _ptr(sig, ctypes.c_double), _ptr(codes, ctypes.c_int8), _ptr(scale, ctypes.c_double),
-        _ptr(colsum, ctypes.c_double), _ptr(bias, ctypes.c_double), _ptr(tie, ctypes.c_double),
+        _ptr(colsum, ctypes.c_double), _ptr(corr_pre, ctypes.c_double),
+        _ptr(bias, ctypes.c_double), _ptr(tie, ctypes.c_double),
         _ptr(Wt, ctypes.c_double), nthreads or default_threads())
     _check(rc, "prepare_weights")
-    return {"codes": codes, "scale": scale, "colsum": colsum, "bias": bias, "tie": tie, "Wt": Wt}
+    return {"codes": codes, "scale": scale, "colsum": colsum, "corr_pre": corr_pre,
+            "bias": bias, "tie": tie, "Wt": Wt}
+
+
+def correction(w, centering):
+    """The correction vector c of the epilogue's m_t * c[n] term for a
+    centering mode: colsum(W~) after the rotation (1), sum_k sigma_k W[n,k]
+    before it (2)."""
+    return w["corr_pre"] if centering == 2 else w["colsum"]
 
 
 def gemm_acc(A, B, rows=None, nthreads=None) -> np.ndarray:
@@ -273,6 +283,6 @@ def layer(X_bits, W_bits, bias_bits, n, a_bits, w_bits, gran=0, centering=1, alp
     a = quantize_act(X_bits, n, a_bits, gran=gran, centering=centering, sigma=sig,
                      static_scale=static_scale, rows=rows, nthreads=nthreads)
     acc = gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
-    y, yb = epilogue(acc, a["scale"], w["scale"], colsum=w["colsum"], bias=w["bias"],
+    y, yb = epilogue(acc, a["scale"], w["scale"], colsum=correction(w, centering), bias=w["bias"],
                      mean=a["mean"] if centering else None)
     return {"sigma": sig, "w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb}

@@ -171,7 +171,7 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
                      int8_t* codes, double* scale, double* mean, double* tie,
                      double* Z, int nthreads) {
   if (K <= 0 || !is_pow2(n) || K % n != 0 || bits < 2 || bits > 8) return -1;
-  if (gran < 0 || gran > 2 || centering < 0 || centering > 1) return -1;
+  if (gran < 0 || gran > 2 || centering < 0 || centering > 2) return -1;
   if (X == nullptr || T < 0 || nrows < 0 || codes == nullptr ||
       scale == nullptr || mean == nullptr)
     return -1;
@@ -183,12 +183,24 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
   const double q = double(qmax_for_bits(bits));
   const std::vector<double> Hn = dense_block(n);
 
-  /* Step 1: Z = X diag(sigma^-1) H, then mean and V = Z - m for one row. */
-  auto transform_row = [&](int64_t t, std::vector<double>& V, double& m) {
+  /* Step 1 for one row: Y = X diag(sigma^-1); with centering 2 the row's
+   * mean mu is subtracted from Y here, before the rotation; Z = Y H; with
+   * centering 1 the mean m of Z is what is subtracted after it.  `shift`
+   * is the value removed from Z (m, or 0), `mean_out` the row's reported
+   * mean (m for centering 1, mu for centering 2, else 0). */
+  auto transform_row = [&](int64_t t, std::vector<double>& V, double& shift,
+                           double& mean_out) {
     std::vector<double> Y(K);
     for (int64_t j = 0; j < K; ++j) {
       double s = sigma ? sigma[j] : 1.0;
       Y[j] = hqo_bf16_to_f64(X[t * K + j]) / s;
+    }
+    mean_out = 0.0;
+    if (centering == 2) {
+      double sum = 0.0;
+      for (int64_t j = 0; j < K; ++j) sum += Y[j];
+      mean_out = sum / double(K);
+      for (int64_t j = 0; j < K; ++j) Y[j] -= mean_out;
     }
     V.assign(K, 0.0);
     for (int64_t k = 0; k < K; ++k) {
@@ -198,11 +210,12 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
         acc += Y[j] * Hn[size_t((j - b0) * n + (k - b0))];
       V[k] = acc;
     }
-    m = 0.0;
+    shift = 0.0;
     if (centering == 1) {
       double sum = 0.0;
       for (int64_t k = 0; k < K; ++k) sum += V[k];
-      m = sum / double(K);
+      shift = sum / double(K);
+      mean_out = shift;
     }
   };
 
@@ -212,8 +225,8 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
     std::vector<double> row_max(T, 0.0);
     parallel_rows(T, nthreads, [&](int64_t t) {
       std::vector<double> V;
-      double m;
-      transform_row(t, V, m);
+      double m, mu;
+      transform_row(t, V, m, mu);
       double a = 0.0;
       for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(V[k] - m));
       row_max[t] = a;
@@ -228,8 +241,8 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
   parallel_rows(nrows, nthreads, [&](int64_t i) {
     int64_t t = rows ? rows[i] : i;
     std::vector<double> V;
-    double m;
-    transform_row(t, V, m);
+    double m, mu;
+    transform_row(t, V, m, mu);
     if (Z) {
       for (int64_t k = 0; k < K; ++k) Z[i * K + k] = V[k];
     }
@@ -243,7 +256,7 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
       s = tensor_scale;
     }
     scale[i] = s;
-    mean[i] = m;
+    mean[i] = mu;
     for (int64_t k = 0; k < K; ++k) {
       double c = 0.0, d = 0.5;
       if (s > 0.0) {
@@ -262,8 +275,8 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
 int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
                         const uint16_t* W, const uint16_t* bias,
                         const double* sigma, int8_t* w_codes, double* w_scale,
-                        double* colsum, double* bias_out, double* tie,
-                        double* Wt, int nthreads) {
+                        double* colsum, double* corr_pre, double* bias_out,
+                        double* tie, double* Wt, int nthreads) {
   if (K <= 0 || N <= 0 || !is_pow2(n) || K % n != 0 || bits < 2 || bits > 8)
     return -1;
   if (W == nullptr || w_codes == nullptr || w_scale == nullptr ||
@@ -291,6 +304,12 @@ int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
       a = std::fmax(a, std::fabs(wt[k]));
     }
     colsum[c] = sum;
+    if (corr_pre) {
+      /* the correction of centering before the rotation: sum_k sigma_k W[c,k] */
+      double cp = 0.0;
+      for (int64_t k = 0; k < K; ++k) cp += (sigma ? sigma[k] : 1.0) * hqo_bf16_to_f64(W[c * K + k]);
+      corr_pre[c] = cp;
+    }
     double s = a / q;
     w_scale[c] = s;
     for (int64_t k = 0; k < K; ++k) {

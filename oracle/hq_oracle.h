@@ -56,9 +56,12 @@ int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
 
 /* Activation side of the layer for the rows listed in `rows` (all T rows when
  * rows == NULL, then nrows must equal T):
- *   Z = X diag(sigma^-1) H            (dense block-diagonal H of order n)
- *   m_t = mean_k Z[t,k]  (centering = 1) or 0 (centering = 0)
- *   V = Z - m
+ *   Y = X diag(sigma^-1)
+ *   centering 0: V = Y H                       (dense block-diagonal H of order n)
+ *   centering 1: Z = Y H, m_t = mean_k Z[t,k], V = Z - m      (HadaNorm's mu
+ *                after the rotation; reported mean m_t)
+ *   centering 2: mu_t = mean_k Y[t,k], V = (Y - mu_t) H       (the mean removed
+ *                before the rotation; reported mean mu_t)
  *   per token  (gran 0): s_t = max_k |V[t,k]| / q
  *   per tensor (gran 1): s   = max_{t,k} |V[t,k]| / q   over ALL T rows
  *   static     (gran 2): s   = static_scale
@@ -73,15 +76,17 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
                      double* Z, int nthreads);
 
 /* Weight side:  W~[n,k] = sum_j H[j,k] sigma_j W[n,j]  (W~ = H^T diag(sigma) W
- * in the pages' orientation), colsum[n] = sum_k W~[n,k],
+ * in the pages' orientation), colsum[n] = sum_k W~[n,k] (the correction of
+ * centering 1), corr_pre[n] = sum_k sigma_k W[n,k] (the correction of
+ * centering 2; optional output),
  * w_scale[n] = max_k |W~[n,k]| / q, w_codes = clamp(rne(W~ / w_scale), -q, q),
  * bias_out[n] = b[n] (0 when bias == NULL).  sigma == NULL means sigma = 1.
  * Optional outputs: tie[N*K] and Wt[N*K] (the unquantized W~). */
 int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
                         const uint16_t* W, const uint16_t* bias,
                         const double* sigma, int8_t* w_codes, double* w_scale,
-                        double* colsum, double* bias_out, double* tie,
-                        double* Wt, int nthreads);
+                        double* colsum, double* corr_pre, double* bias_out,
+                        double* tie, double* Wt, int nthreads);
 
 /* acc[i*N+c] = sum_k A[rows[i],k] * B[c,k] in 64-bit integers, for int8
  * matrices A[M,K] and B[N,K] (rows == NULL: all M rows, nrows == M). */

@@ -65,7 +65,7 @@ def test_quantize_validation(hq):
     assert _call_quant(hq, D(1024, 16, 1024, a_bits=5)) == 2
     assert _call_quant(hq, D(1024, 16, 1024, w_bits=3)) == 2
     assert _call_quant(hq, D(1024, 16, 1024, act_gran=7)) == 1
-    assert _call_quant(hq, D(1024, 16, 1024, centering=2)) == 1
+    assert _call_quant(hq, D(1024, 16, 1024, centering=3)) == 1
     assert _call_quant(hq, D(1024, 16, 1024, code_format=1)) == 2
     assert _call_quant(hq, D(1024, 16, 1024), X=FAKE + 2) == 3   # misaligned
     assert _call_quant(hq, D(1024, 16, 1024), codes=FAKE + 8) == 3

@@ -51,7 +51,7 @@ def _check_act(ref, codes, scale, mean, per_row=True, min_match=None, what="act"
     else:
         check_rel(scale[:1], ref["scale"][:1], SCALE_RTOL, what + " tensor scale")
     if ref["Z"] is not None:
-        tol = 1e-6 * np.mean(np.abs(ref["Z"]), axis=1) + 1e-30
+        tol = 1e-6 * (np.mean(np.abs(ref["Z"]), axis=1) + np.abs(ref["mean"])) + 1e-30
         assert np.all(np.abs(mean - ref["mean"]) <= tol), what + " mean"
 
 
@@ -67,7 +67,13 @@ for i, (n, B) in enumerate([(16, 4), (16, 12), (32, 2), (32, 6), (64, 1), (64, 5
         SMALL.append((n * B, n, T, bits, (i + T) % 2, (i % 3) != 0))
 
 
-@pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL)
+# the mean removed before the rotation (HQ_CENTER_TOKEN_MEAN_PRE), every order
+SMALL_PRE = [(n * B, n, T, (4, 3, 8)[i % 3], 2, i % 2 == 0)
+             for i, (n, B, T) in enumerate([(16, 4, 129), (32, 6, 7), (64, 5, 300), (128, 9, 129),
+                                            (256, 3, 300), (512, 2, 7), (1024, 3, 129)])]
+
+
+@pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL + SMALL_PRE)
 def test_quantize_small(hq, K, n, T, bits, center, use_sigma):
     g = np.random.default_rng(K * 1000 + T)
     x = g.standard_normal((T, K)).astype(np.float32)
@@ -86,7 +92,8 @@ def test_quantize_small(hq, K, n, T, bits, center, use_sigma):
 
 
 @pytest.mark.parametrize("gran", [1, 2])
-@pytest.mark.parametrize("K,n,T,center", [(320, 64, 300, 0), (256, 256, 129, 1), (1024, 1024, 77, 0)])
+@pytest.mark.parametrize("K,n,T,center", [(320, 64, 300, 0), (256, 256, 129, 1), (1024, 1024, 77, 0),
+                                            (1152, 128, 200, 2)])
 def test_quantize_per_tensor(hq, gran, K, n, T, center):
     cfg = synth.CONFIGS[4]
     g = np.random.default_rng(K + T)
@@ -140,11 +147,13 @@ def test_exact_ties_are_rounded_half_to_even(hq):
 # weight preparation
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("N,K,n,w_bits,use_sigma",
-                         [(48, 64, 16, 4, True), (160, 256, 64, 8, True), (64, 1152, 128, 4, True),
-                          (32, 3072, 1024, 4, True), (320, 320, 64, 8, False),
-                          (1024, 1024, 1024, 4, True)])
-def test_prepare_weights(hq, N, K, n, w_bits, use_sigma):
+@pytest.mark.parametrize("N,K,n,w_bits,use_sigma,center",
+                         [(48, 64, 16, 4, True, 1), (160, 256, 64, 8, True, 1),
+                          (64, 1152, 128, 4, True, 1), (32, 3072, 1024, 4, True, 1),
+                          (320, 320, 64, 8, False, 0), (1024, 1024, 1024, 4, True, 1),
+                          (64, 1152, 128, 4, True, 2), (48, 512, 16, 8, False, 2),
+                          (32, 3072, 1024, 4, True, 2)])
+def test_prepare_weights(hq, N, K, n, w_bits, use_sigma, center):
     g = np.random.default_rng(N + K)
     Xb = synth.f32_to_bf16_bits(g.standard_normal((64, K)).astype(np.float32) *
                                 (1 + 20 * (g.random(K) < 0.02)).astype(np.float32))
@@ -152,7 +161,7 @@ def test_prepare_weights(hq, N, K, n, w_bits, use_sigma):
     bb = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32) * 0.01)
     sig = oracle.sigma(oracle.col_absmax(Xb), oracle.col_absmax(Wb), 0.5) if use_sigma else None
     ref = oracle.prepare_weights(Wb, n, w_bits, bias_bits=bb, sigma=sig, want_Wt=True)
-    desc = hq.LayerDesc(K, N, n, a_bits=4, w_bits=w_bits)
+    desc = hq.LayerDesc(K, N, n, a_bits=4, w_bits=w_bits, centering=center)
     X = to_dev_u16(Xb, torch)
     W = to_dev_u16(Wb, torch)
     b = to_dev_u16(bb, torch)
@@ -174,8 +183,13 @@ def test_prepare_weights(hq, N, K, n, w_bits, use_sigma):
         assert np.all(sigma_inv.cpu().numpy() == 1.0)
     check_codes(w_codes.cpu().numpy(), ref["codes"], ref["tie"], "w_codes")
     check_rel(w_scale.cpu().numpy(), ref["scale"], SCALE_RTOL, "w_scale")
-    tol = 1e-6 * np.abs(ref["Wt"]).sum(axis=1)
-    assert np.all(np.abs(colsum.cpu().numpy() - ref["colsum"]) <= tol), "colsum"
+    if center == 2:   # sum_k sigma_k W[n,k]: bound by the sum of its terms' magnitudes
+        sw = synth.bf16_bits_to_f32(Wb).astype(np.float64) * (sig if sig is not None else 1.0)
+        tol = 1e-6 * np.abs(sw).sum(axis=1)
+    else:
+        tol = 1e-6 * np.abs(ref["Wt"]).sum(axis=1)
+    want = oracle.correction(ref, center)
+    assert np.all(np.abs(colsum.cpu().numpy() - want) <= tol), "colsum"
     assert np.array_equal(bias_f32.cpu().numpy().astype(np.float64), ref["bias"])
 
 
@@ -301,8 +315,8 @@ def _oracle_layer(cfg, Xb, Wb, bb, rows=None, cols=None):
     a = oracle.quantize_act(Xb, cfg.had_order, cfg.a_bits, gran=cfg.act_gran,
                             centering=cfg.centering, sigma=sig, rows=rows, want_Z=True)
     acc = oracle.gemm_acc(a["codes"], w["codes"])
-    y, yb = oracle.epilogue(acc, a["scale"], w["scale"], colsum=w["colsum"], bias=w["bias"],
-                            mean=a["mean"] if cfg.centering else None)
+    y, yb = oracle.epilogue(acc, a["scale"], w["scale"], colsum=oracle.correction(w, cfg.centering),
+                            bias=w["bias"], mean=a["mean"] if cfg.centering else None)
     return {"w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb, "sigma": sig}
 
 
@@ -323,6 +337,28 @@ def test_layer_reduced_tokens(hq, idx, T):
             np.all(layer.w_codes.cpu().numpy() == ref["w"]["codes"]))
     if same:
         assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+
+
+@pytest.mark.parametrize("idx,T", [(1, 300), (2, 257), (3, 130), (5, 129)])
+def test_layer_pre_rotation_centering(hq, idx, T):
+    """The mean removed before the rotation (HQ_CENTER_TOKEN_MEAN_PRE): codes,
+    the correction sum_k sigma_k W[n,k] and the layer output against the
+    oracle, and its output is closer to the exact product than the default."""
+    import dataclasses
+    cfg = dataclasses.replace(synth.CONFIGS[idx].with_tokens(T), centering=2)
+    Xb, Wb, bb = synth.make_layer(cfg)
+    if idx == 5:
+        Wb, bb = Wb[:768], bb[:768]
+    layer, bufs, Y, acc = _gpu_layer(hq, cfg, Xb, Wb, bb)
+    ref = _oracle_layer(cfg, Xb, Wb, bb)
+    check_codes(bufs["a_codes"].cpu().numpy(), ref["a"]["codes"], ref["a"]["tie"], "a_codes")
+    check_codes(layer.w_codes.cpu().numpy(), ref["w"]["codes"], ref["w"]["tie"], "w_codes")
+    err = rel_frob(bf16_bits(Y), ref["y_bf16"])
+    assert err <= Y_REL_FROB, err
+    y_exact = oracle.exact_linear(Xb, Wb, bb)
+    ref1 = _oracle_layer(dataclasses.replace(cfg, centering=1), Xb, Wb, bb)
+    gpu_err = np.linalg.norm(synth.bf16_bits_to_f32(bf16_bits(Y)).astype(np.float64) - y_exact)
+    assert gpu_err < np.linalg.norm(ref1["y"] - y_exact)
 
 
 def test_centering_off_variant_of_w4a3(hq):

@@ -117,7 +117,7 @@ def _bf16(x):
 
 @pytest.mark.parametrize("K,n,N,T", [(16, 4, 8, 5), (64, 16, 24, 9), (256, 64, 40, 7),
                                      (1152, 128, 32, 4), (3072, 1024, 16, 3)])
-@pytest.mark.parametrize("centering", [0, 1])
+@pytest.mark.parametrize("centering", [0, 1, 2])
 def test_eq1_identity_unquantized(K, n, N, T, centering):
     g = np.random.default_rng(K + n + centering)
     X = synth.f32_to_bf16_bits(g.standard_normal((T, K)) * 2 + g.standard_normal((T, 1)) * 3)
@@ -127,8 +127,12 @@ def test_eq1_identity_unquantized(K, n, N, T, centering):
     assert np.all(sig > 0) and not np.allclose(sig, 1.0)
     a = oracle.quantize_act(X, n, 8, centering=centering, sigma=sig, want_Z=True)
     w = oracle.prepare_weights(W, n, 8, bias_bits=b, sigma=sig, want_Wt=True)
-    V = a["Z"] - a["mean"][:, None]                       # X~ = X diag(s^-1) H - mu
-    y_tilde = V @ w["Wt"].T + w["bias"][None, :] + a["mean"][:, None] * w["colsum"][None, :]
+    # X~ = X diag(s^-1) H - mu: mu removed after the rotation (centering 1) or
+    # before it (centering 2, where Z is already (Y - mu_t) H)
+    shift = a["mean"] if centering == 1 else np.zeros(T)
+    V = a["Z"] - shift[:, None]
+    c = oracle.correction(w, centering)
+    y_tilde = V @ w["Wt"].T + w["bias"][None, :] + a["mean"][:, None] * c[None, :]
     y = _bf16(X) @ _bf16(W).T + _bf16(b)[None, :]          # XW + b
     rel = np.linalg.norm(y_tilde - y) / np.linalg.norm(y)
     assert rel <= 1e-10, rel
@@ -172,6 +176,54 @@ def test_invariants(K, n):
                            rtol=1e-12)
 
 
+@pytest.mark.parametrize("K,n", [(64, 16), (1152, 128), (320, 64), (2048, 1024)])
+def test_invariants_pre_rotation_centering(K, n):
+    """Centering 2 removes mean_k Y[t,k] before the rotation.  Because every
+    column of H~ but each block's first sums to zero, this changes only the
+    first channel of each block, by -sqrt(n) mu_t, and those channels then
+    sum to zero; the weight-side correction is sum_k sigma_k W[n,k]."""
+    T, N = 6, 10
+    g = np.random.default_rng(K + 1)
+    X = synth.f32_to_bf16_bits(g.standard_normal((T, K)) + 2.0)
+    W = synth.f32_to_bf16_bits(g.standard_normal((N, K)) * 0.02)
+    sig = oracle.sigma(oracle.col_absmax(X), oracle.col_absmax(W), 0.5)
+    a2 = oracle.quantize_act(X, n, 4, centering=2, sigma=sig, want_Z=True)
+    a0 = oracle.quantize_act(X, n, 4, centering=0, sigma=sig, want_Z=True)
+    w = oracle.prepare_weights(W, n, 4, sigma=sig)
+    Y = _bf16(X) / sig[None, :]
+    mu = Y.mean(axis=1)
+    assert np.allclose(a2["mean"], mu, rtol=1e-13, atol=1e-13)
+    diff = a2["Z"] - a0["Z"]
+    first = np.zeros(K, dtype=bool)
+    first[::n] = True
+    assert np.allclose(diff[:, ~first], 0.0, atol=1e-12)
+    assert np.allclose(diff[:, first], -math.sqrt(n) * mu[:, None], rtol=1e-12, atol=1e-12)
+    assert np.allclose(a2["Z"][:, first].sum(axis=1), 0.0, atol=1e-10 * np.abs(a0["Z"]).max())
+    assert np.allclose(w["corr_pre"], (_bf16(W) * sig[None, :]).sum(axis=1), rtol=1e-12,
+                       atol=1e-13)
+    # and in terms of the rotated weights: sqrt(n) times their blocks' first channels
+    w2 = oracle.prepare_weights(W, n, 4, sigma=sig, want_Wt=True)
+    assert np.allclose(w["corr_pre"], math.sqrt(n) * w2["Wt"][:, first].sum(axis=1),
+                       rtol=1e-11, atol=1e-12)
+
+
+def test_pre_rotation_centering_removes_the_token_offset():
+    """On the configurations' token-offset data, removing the mean before the
+    rotation leaves a much smaller max |V| than removing it after (which only
+    moves the mean of V), so its output is closer to the exact product."""
+    for idx in (1, 2):
+        cfg = synth.CONFIGS[idx].with_tokens(64)
+        Xb, Wb, bb = synth.make_layer(cfg)
+        y_ex = oracle.exact_linear(Xb, Wb, bb)
+
+        def sqnr(c):
+            r = oracle.layer(Xb, Wb, bb, cfg.had_order, cfg.a_bits, cfg.w_bits, centering=c,
+                             alpha=cfg.alpha, use_sigma=cfg.use_sigma)
+            return 10 * np.log10(np.linalg.norm(y_ex) ** 2 / np.linalg.norm(r["y"] - y_ex) ** 2)
+
+        assert sqnr(2) > sqnr(1) + 6.0, idx
+
+
 # --------------------------------------------------------------------------
 # brute force at K = 8: exact integer decision of every code
 # --------------------------------------------------------------------------
@@ -186,7 +238,13 @@ def _exact_codes_int(x_int, n, q, centering):
     H = kron_sylvester(n)
     zh = np.concatenate([x_int[:, b * n:(b + 1) * n] @ H for b in range(B)], axis=1)
     K = x_int.shape[1]
-    U = K * zh - (zh.sum(axis=1, keepdims=True) if centering else 0)
+    if centering == 2:
+        # K (x - mean(x)) H~ = K Z_hat - sum(x) (n at each block's first
+        # channel, 0 elsewhere); sum(x) = sum of the blocks' first channels
+        U = K * zh
+        U[:, ::n] -= n * zh[:, ::n].sum(axis=1, keepdims=True)
+    else:
+        U = K * zh - (zh.sum(axis=1, keepdims=True) if centering else 0)
     D = np.abs(U).max(axis=1, keepdims=True)
     num = q * U
     den = np.where(D == 0, 1, D)
@@ -197,11 +255,11 @@ def _exact_codes_int(x_int, n, q, centering):
     tie = two_r == den
     codes = f + up + (tie & (f % 2 != 0))
     codes = np.where(D == 0, 0, codes)
-    return codes, tie & (D != 0), zh
+    return codes, tie & (D != 0), (U / K if centering == 2 else zh)
 
 
 @pytest.mark.parametrize("n", [4, 8])
-@pytest.mark.parametrize("bits,centering", [(4, 1), (3, 1), (4, 0)])
+@pytest.mark.parametrize("bits,centering", [(4, 1), (3, 1), (4, 0), (4, 2), (3, 2)])
 def test_bruteforce_k8(n, bits, centering):
     vals = np.arange(-2, 3)
     x_int = np.array(list(itertools.product(vals, repeat=8)), dtype=np.int64)  # 5^8 rows
@@ -221,7 +279,7 @@ def test_bruteforce_k8(n, bits, centering):
     assert np.all(np.abs(codes) <= q)
     # exhaustive arg-min over the 2q+1 grid levels agrees with the code
     levels = np.arange(-q, q + 1)
-    V = r["Z"] - r["mean"][:, None]
+    V = r["Z"] - (r["mean"][:, None] if centering == 1 else 0.0)
     s = r["scale"][:, None]
     safe = np.where(s == 0, 1.0, s)
     dist = np.abs((V / safe)[..., None] - levels[None, None, :])
