@@ -50,6 +50,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--centering", type=int, default=None, choices=[0, 1, 2],
+                    help="override the configuration's centering mode (2: the mean removed "
+                         "before the rotation)")
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -288,7 +291,7 @@ def run_reference(args):
     _, rank, _ = rank_env()
     if rank != 0:
         return 0
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload_config(args)
     Xb, Wb, bb = synth.make_layer(cfg)
     nthreads = os.cpu_count() or 1
     sig, w = oracle_prepare(cfg, Xb, Wb, bb)
@@ -319,11 +322,24 @@ def run_reference(args):
     return 0
 
 
+def workload_config(args):
+    import dataclasses
+    cfg = synth.CONFIGS[args.config]
+    if args.centering is not None:
+        cfg = dataclasses.replace(cfg, centering=args.centering)
+    return cfg
+
+
 def config_block(cfg, n_gpus):
     gran = {0: "per_token", 1: "per_tensor_dynamic", 2: "per_tensor_static"}[cfg.act_gran]
-    return {"workload": cfg.workload(), "tokens_per_gpu": cfg.T, "K": cfg.K, "N": cfg.N,
+    workload = cfg.workload()
+    if cfg.centering != synth.CONFIGS[cfg.index].centering:
+        workload += f":centering{cfg.centering}"
+    return {"workload": workload, "tokens_per_gpu": cfg.T, "K": cfg.K, "N": cfg.N,
             "had_order": cfg.had_order, "bits": f"A{cfg.a_bits}W{cfg.w_bits}",
-            "act_granularity": gran, "centering": bool(cfg.centering), "sigma": cfg.use_sigma,
+            "act_granularity": gran,
+            "centering": {0: "none", 1: "token mean after H", 2: "token mean before H"}[cfg.centering],
+            "sigma": cfg.use_sigma,
             "l2": "inputs larger than L2: step i reads copy i % M of the token batch, "
                   "M copies > 2x L2 (weights and intermediate codes stay L2-resident)",
             "timing": "one CUDA graph of K back-to-back steps between two CUDA events; "
@@ -348,7 +364,7 @@ def run_hq(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
     hq.load_library()
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload_config(args)
     # replicated weights (same seed on every rank), rank-local token batch
     Wb, bb = synth.make_w(cfg)
     Xb = synth.make_x(cfg, seed=shard_seed(cfg, rank))
