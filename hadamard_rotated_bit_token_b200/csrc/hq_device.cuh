@@ -185,16 +185,6 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tma
       ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(y), "r"(bar_cl) : "memory");
 }
 
-// 3-D tiled tensor load (tensor map in param space), no multicast.
-__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int32_t x, int32_t y,
-                                            int32_t z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];"
-      ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // 2-D tiled tensor store shared -> global (bulk-group completion); the box
 // is clipped at the tensor's bounds.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int32_t x,
@@ -330,10 +320,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 typedef float2 f2;
 
 __device__ __forceinline__ f2 pk(float a, float b) { return make_float2(a, b); }
-__device__ __forceinline__ void upk(f2 x, float& a, float& b) {
-  a = x.x;
-  b = x.y;
-}
 __device__ __forceinline__ f2 add2(f2 a, f2 b) { return __fadd2_rn(a, b); }
 // a - b as one fused multiply-add: a + (-1) * b rounds exactly like a - b
 __device__ __forceinline__ f2 sub2(f2 a, f2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }

@@ -15,12 +15,15 @@
 //               commits each stage back to the producer and each finished
 //               accumulator to the epilogue;
 //   warps 2..9  the epilogue: two warps per 32-lane quarter of tensor memory,
-//               each taking half of the tile's columns.  Per 32-column chunk a
-//               warp reads the accumulator (tcgen05.ld), applies the epilogue
-//               in fp32 (row scale and mean from registers, prefetched one
-//               tile ahead; column parameters from the ring), writes bf16 to
-//               a 64-byte swizzled shared buffer and lets a TMA tensor store
-//               write the 32 x 32 box to Y (clipped at the tensor's edges).
+//               each taking half of the tile's columns.  A warp reads its
+//               columns of the accumulator (tcgen05.ld, up to three 32-column
+//               chunks per wait) and hands the accumulator back to the MMA
+//               issuer as soon as the last read has landed; then per chunk it
+//               applies the epilogue in fp32 (row scale and mean from
+//               registers, prefetched one tile ahead; column parameters from
+//               the ring), writes bf16 to a 64-byte swizzled shared buffer and
+//               lets a TMA tensor store write the 32 x 32 box to Y (clipped at
+//               the tensor's edges).
 //
 // gemm_i8_kernel<BN>: one CTA per 128 x BN output tile (BN 64..256).
 // gemm_i8_pair_kernel: a cluster of two CTAs per 256 x 256 output tile with
@@ -129,18 +132,13 @@ __device__ __forceinline__ void load_row_params(const GemmParams& p, int64_t row
 }
 
 // One 32-column chunk c of the warp's columns: accumulators r (this thread's
-// row) -> fp32 epilogue -> bf16 -> swizzled staging buffer -> TMA store.
-// prm points at the warp's first column in a parameter slot of width W.
-// NBUF staging buffers of kStageBox bytes rotate; `nstore` counts the stores
-// this warp issued (warp-uniform).
-template <int W, int NBUF>
-__device__ __forceinline__ void epi_chunk(const GemmParams& p, const CUtensorMap* tmY,
-                                          const uint32_t (&r)[32], int c, const EpiTile& e,
-                                          const float* prm, uint8_t* stg, int lane,
-                                          uint32_t& nstore) {
-  const int col0 = e.col_base + c * 32;
+// row) -> fp32 epilogue -> bf16 pairs in `packed`.  prm points at the warp's
+// first column in a parameter slot of width W.
+template <int W>
+__device__ __forceinline__ void epi_math(const GemmParams& p, const uint32_t (&r)[32], int c,
+                                         const EpiTile& e, const float* prm,
+                                         uint32_t (&packed)[16]) {
   const float* pw = prm + c * 32;
-  uint32_t packed[16];
   const f2 sx2 = pk(e.sx, e.sx), mt2 = pk(e.mt, e.mt);
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
@@ -166,27 +164,8 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const CUtensorMap
     packed[2 * g] = pack_bf16x2(y01.x, y01.y);
     packed[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
   }
-  const bool do_store = col0 < p.N && e.row0 < p.T;  // warp-uniform
-  if (do_store) {
-    uint8_t* buf = stg + (nstore % NBUF) * kStageBox;
-    // the store that last used this buffer must have finished reading it
-    if (lane == 0) bulk_wait_group_read<NBUF - 1>();
-    __syncwarp();
-    const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this thread's row
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ swz) << 4)) =
-          make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_2d(tmY, buf, col0, e.row0);
-      bulk_commit_group();
-    }
-    ++nstore;
-  }
   if (p.acc_debug && e.row_ok) {
+    const int col0 = e.col_base + c * 32;
     int32_t* arow = p.acc_debug + e.row * p.N;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
@@ -198,27 +177,63 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const CUtensorMap
   }
 }
 
-// The warp's HC columns of one accumulator starting at tensor-memory address
-// t_addr (lane quarter already encoded): two chunks per tensor-memory wait.
-template <int HC, int W, int NBUF>
+// Chunk c's bf16 values into staging box `buf` (64-byte swizzled rows), then
+// one thread stores the 32 x 32 box to Y (clipped at the tensor's edges) as
+// its own bulk group.
+__device__ __forceinline__ void epi_store_chunk(const GemmParams& p, const CUtensorMap* tmY,
+                                                const uint32_t (&packed)[16], int col0, int row0,
+                                                uint8_t* buf, int lane) {
+  const int swz = (lane >> 1) & 3;  // 64-byte swizzle of this thread's row
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ swz) << 4)) =
+        make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && col0 < p.N && row0 < p.T) {
+    tma_store_2d(tmY, buf, col0, row0);
+    bulk_commit_group();
+  }
+}
+
+// The warp's HC columns (HC / 32 chunks) of one accumulator at tensor-memory
+// address t_addr (lane quarter already encoded), through NBOX staging boxes
+// of kStageBox bytes:
+//   - the chunks are read from tensor memory in groups of up to three per
+//     wait (96 accumulator registers); right after the last group's wait
+//     `release_acc` hands the accumulator back to the MMA issuer, so the
+//     next main loop into it can start while this tile is still being stored;
+//   - per chunk: the epilogue arithmetic, then a wait until the store that
+//     last used the chunk's box has read it, then the box and its TMA store;
+//   - `release_params` frees the parameter slot after the last chunk's
+//     arithmetic.
+template <int HC, int W, int NBOX, class RelAcc, class RelPrm>
 __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap* tmY,
                                          uint32_t t_addr, const EpiTile& e, const float* prm,
-                                         uint8_t* stg, int lane, uint32_t& nstore) {
+                                         uint8_t* stg, int lane, RelAcc release_acc,
+                                         RelPrm release_params) {
   constexpr int NCH = HC / 32;
-#pragma unroll 1
-  for (int c = 0; c + 1 < NCH; c += 2) {
-    uint32_t r0[32], r1[32];
-    tmem_ld_32x32b_x32(t_addr + uint32_t(c * 32), r0);
-    tmem_ld_32x32b_x32(t_addr + uint32_t(c * 32 + 32), r1);
+  constexpr int G = NCH <= 3 ? NCH : 2;
+  static_assert(NCH % G == 0, "whole groups of chunks");
+#pragma unroll
+  for (int c0 = 0; c0 < NCH; c0 += G) {
+    uint32_t r[G][32];
+#pragma unroll
+    for (int c = 0; c < G; ++c) tmem_ld_32x32b_x32(t_addr + uint32_t((c0 + c) * 32), r[c]);
     tmem_wait_ld();
-    epi_chunk<W, NBUF>(p, tmY, r0, c, e, prm, stg, lane, nstore);
-    epi_chunk<W, NBUF>(p, tmY, r1, c + 1, e, prm, stg, lane, nstore);
-  }
-  if (NCH & 1) {
-    uint32_t r0[32];
-    tmem_ld_32x32b_x32(t_addr + uint32_t((NCH - 1) * 32), r0);
-    tmem_wait_ld();
-    epi_chunk<W, NBUF>(p, tmY, r0, NCH - 1, e, prm, stg, lane, nstore);
+    if (c0 + G == NCH) release_acc();
+#pragma unroll
+    for (int c = 0; c < G; ++c) {
+      const int ch = c0 + c;
+      uint32_t packed[16];
+      epi_math<W>(p, r[c], ch, e, prm, packed);
+      if (ch == NCH - 1) release_params();
+      if (lane == 0) bulk_wait_group_read<NBOX - 1>();
+      __syncwarp();
+      epi_store_chunk(p, tmY, packed, e.col_base + ch * 32, e.row0, stg + (ch % NBOX) * kStageBox,
+                      lane);
+    }
   }
 }
 
@@ -231,8 +246,8 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int HC = BN / 2;  // columns per epilogue warp
-  static constexpr int NBUF = 1;     // output staging buffers per epilogue warp
-  static constexpr int EPI_STAGE_BYTES = NBUF * kStageBox;
+  static constexpr int NBOX = 1;  // output staging boxes per epilogue warp
+  static constexpr int EPI_STAGE_BYTES = NBOX * kStageBox;
   static constexpr int RING_BYTES = 2 * 3 * BN * 4;
   static constexpr int CTL_BYTES = 256;
   static constexpr int FIXED = kEpiWarps * EPI_STAGE_BYTES + RING_BYTES + CTL_BYTES + 1024;
@@ -407,7 +422,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;    // TMEM lanes [32*quarter, 32*quarter + 32)
     const int half = ew >> 2;        // columns [half*HC, half*HC + HC) of the tile
     uint8_t* stg = epi_stage + ew * C::EPI_STAGE_BYTES;
-    uint32_t nstore = 0;
     int acc_iter = 0;
     float sx_next = 0.0f, mt_next = 0.0f;
     if (int(blockIdx.x) < num_tiles)
@@ -438,14 +452,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + uint32_t(acc * BN + half * C::HC) +
                               (uint32_t(quarter * 32) << 16);
-      epi_tile<C::HC, BN, C::NBUF>(p, &tmY, t_addr, e, ring + acc * 3 * BN + half * C::HC, stg,
-                                   lane, nstore);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tempty[acc]);
-        mbar_arrive(&pempty[acc]);
-      }
+      epi_tile<C::HC, BN, C::NBOX>(
+          p, &tmY, t_addr, e, ring + acc * 3 * BN + half * C::HC, stg, lane,
+          [&] {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+          },
+          [&] {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[acc]);
+          });
     }
     if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
     __syncwarp();
@@ -468,8 +485,8 @@ struct PairCfg {
   static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
   static constexpr int HC = BN / 2;  // columns per epilogue warp
-  static constexpr int NBUF = 2;     // output staging buffers per epilogue warp
-  static constexpr int EPI_STAGE_BYTES = NBUF * kStageBox;
+  static constexpr int NBOX = 2;  // output staging boxes per epilogue warp
+  static constexpr int EPI_STAGE_BYTES = NBOX * kStageBox;
   static constexpr int RING_BYTES = 2 * 3 * BN * 4;
   static constexpr int CTL_BYTES = 512;
   static constexpr int FIXED = kEpiWarps * EPI_STAGE_BYTES + RING_BYTES + CTL_BYTES + 1024;
@@ -665,7 +682,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint8_t* stg = epi_stage + ew * C::EPI_STAGE_BYTES;
     const uint32_t tempty0 = mapa_shared(tempty, 0);
     const int row_off = int(rank) * BM + quarter * 32 + lane;
-    uint32_t nstore = 0;
     int acc_iter = 0;
     float sx_next = 0.0f, mt_next = 0.0f;
     if (cluster_id < num_tiles)
@@ -696,14 +712,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + uint32_t(acc * C::BN + half * C::HC) +
                               (uint32_t(quarter * 32) << 16);
-      epi_tile<C::HC, C::BN, C::NBUF>(p, &tmY, t_addr, e, ring + acc * 3 * C::BN + half * C::HC,
-                                      stg, lane, nstore);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_remote(tempty0 + uint32_t(acc) * 8u);
-        mbar_arrive(&pempty[acc]);
-      }
+      epi_tile<C::HC, C::BN, C::NBOX>(
+          p, &tmY, t_addr, e, ring + acc * 3 * C::BN + half * C::HC, stg, lane,
+          [&] {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(tempty0 + uint32_t(acc) * 8u);
+          },
+          [&] {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[acc]);
+          });
     }
     if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
     __syncwarp();
