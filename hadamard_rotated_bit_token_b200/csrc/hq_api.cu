@@ -152,7 +152,7 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
   int R, nt;
   quant_shape(K, &R, &nt);
   const int logn = ilog2_exact(n);
-  const bool xpose = logn >= 6;  // shared-memory transposes for n >= 64
+  const bool xpose = logn >= 8;  // shared-memory transposes for n >= 256
   const int per_sm = 2;          // CTAs per SM (kernel launch bounds)
   L.p.X = X;
   L.p.T = T;

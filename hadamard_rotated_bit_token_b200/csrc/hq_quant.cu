@@ -32,9 +32,9 @@
 //            tile ahead of the tile being processed (no shared-memory stage);
 //   rotate   bf16 -> fp32, times the channel multiplier, butterflies on the 5
 //            in-register index bits, then the remaining bits across the n/32
-//            threads of a block: warp shuffles for n <= 128 beyond the
-//            transpose; for n >= 64 an 8-lane shared-memory transpose swaps
-//            index bits 2-4 with 5-7 and shuffles take bits 8 and up;
+//            threads of a block: warp shuffles for n <= 128; for n >= 256 a
+//            shared-memory transpose among up to 8 lanes swaps index bits
+//            with in-register ones and shuffles take bits 8 and up;
 //   stats    the row's max / min by a warp reduction over the lanes of the
 //            row (redux.sync) and one shared-memory atomic per warp segment;
 //            the segment that completes the row (a per-row arrival counter)
@@ -146,10 +146,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   constexpr int LREG = LOGN < 5 ? LOGN : 5;        // index bits inside a thread's slice
   constexpr int LOG_TT = LOGN > 5 ? LOGN - 5 : 0;  // index bits across threads
   constexpr int TT = 1 << LOG_TT;                  // threads per Hadamard block
-  // Cross-thread bits: the lowest LX of them by a shared-memory transpose
-  // among G = 2^LX lanes (swapping them with in-register bits 5-LX..4), the
-  // rest by warp shuffles.
-  constexpr int LX = LOG_TT < 3 ? LOG_TT : 3;
+  // Cross-thread bits: for n <= 128 (at most two) all by warp shuffles; for
+  // larger blocks the lowest LX of them by a shared-memory transpose among
+  // G = 2^LX lanes (swapping them with in-register bits 5-LX..4), the rest
+  // by warp shuffles (measured: shuffles win at two cross-thread bits, the
+  // transpose at three and more).
+  constexpr int LX = LOGN <= 7 ? 0 : (LOG_TT < 3 ? LOG_TT : 3);
   constexpr int G = 1 << LX;                       // lanes per transpose group = groups per thread
   constexpr int GS = 32 / G;                       // elements per group
   constexpr int GP = GS / 2;                       // f32x2 pairs per group
