@@ -80,9 +80,17 @@ def _load():
             lib.hqo_exact_linear.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int64,
                                              ctypes.c_int64, ctypes.c_int64, _i64p,
                                              ctypes.c_int64, _f64p, ctypes.c_int]
+            lib.hqo_prepare_weights_wh.argtypes = [
+                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                _u16p, _u16p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+            lib.hqo_epilogue_wh.argtypes = [_i64p, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.c_int64, _f64p, _f64p, _f64p, _f64p, _u16p]
+            lib.hqo_output_rotation.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64,
+                                                ctypes.c_int64, _f64p]
             for name in ("hqo_sylvester", "hqo_col_absmax", "hqo_sigma", "hqo_quantize_act",
                          "hqo_prepare_weights", "hqo_gemm_acc", "hqo_epilogue",
-                         "hqo_exact_linear"):
+                         "hqo_exact_linear", "hqo_prepare_weights_wh", "hqo_epilogue_wh",
+                         "hqo_output_rotation"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -250,6 +258,56 @@ def epilogue(acc, sx, sw, colsum=None, bias=None, mean=None):
     return y, yb
 
 
+def prepare_weights_wh(W_bits, n_out, bits, bias_bits=None, sigma=None, want_tie=True,
+                       want_Wbar=False, nthreads=None):
+    """Weight-only Hadamard form (HaTQ Eq. (15)-(17), supplement Eq. (40)):
+    Wbar = H_out W diag(sigma) rotated along the output channels (blocks of
+    n_out), quantized per row, and b_bar = b H_out.
+    Returns dict(codes int8 [N,K], scale [N], b_bar [N], tie, Wbar)."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    b = _c(bias_bits, np.uint16)
+    sig = _c(sigma, np.float64)
+    codes = np.zeros((N, K), dtype=np.int8)
+    scale = np.zeros(N, dtype=np.float64)
+    b_bar = np.zeros(N, dtype=np.float64)
+    tie = np.zeros((N, K), dtype=np.float64) if want_tie else None
+    Wbar = np.zeros((N, K), dtype=np.float64) if want_Wbar else None
+    rc = _load().hqo_prepare_weights_wh(
+        K, N, n_out, bits, _ptr(W, ctypes.c_uint16), _ptr(b, ctypes.c_uint16),
+        _ptr(sig, ctypes.c_double), _ptr(codes, ctypes.c_int8), _ptr(scale, ctypes.c_double),
+        _ptr(b_bar, ctypes.c_double), _ptr(tie, ctypes.c_double), _ptr(Wbar, ctypes.c_double),
+        nthreads or default_threads())
+    _check(rc, "prepare_weights_wh")
+    return {"codes": codes, "scale": scale, "b_bar": b_bar, "tie": tie, "Wbar": Wbar}
+
+
+def output_rotation(M, n_out) -> np.ndarray:
+    """M H_out for an fp64 matrix [rows, N] (blocks of n_out along N)."""
+    M = _c(np.atleast_2d(M), np.float64)
+    out = np.zeros_like(M)
+    _check(_load().hqo_output_rotation(_ptr(M, ctypes.c_double), M.shape[0], M.shape[1],
+                                       n_out, _ptr(out, ctypes.c_double)), "output_rotation")
+    return out
+
+
+def epilogue_wh(acc, n_out, sx, sw, b_bar=None):
+    """WH output side (supplement Eq. (41)): (s_x s_w acc + b_bar) H_out.
+    Returns (y f64 [r,N], y_bf16 uint16 [r,N])."""
+    acc = _c(acc, np.int64)
+    nr, N = acc.shape
+    sx = _c(np.broadcast_to(np.asarray(sx, dtype=np.float64), (nr,)), np.float64)
+    sw = _c(sw, np.float64)
+    bb = _c(b_bar, np.float64)
+    y = np.zeros((nr, N), dtype=np.float64)
+    yb = np.zeros((nr, N), dtype=np.uint16)
+    _check(_load().hqo_epilogue_wh(_ptr(acc, ctypes.c_int64), nr, N, n_out,
+                                   _ptr(sx, ctypes.c_double), _ptr(sw, ctypes.c_double),
+                                   _ptr(bb, ctypes.c_double), _ptr(y, ctypes.c_double),
+                                   _ptr(yb, ctypes.c_uint16)), "epilogue_wh")
+    return y, yb
+
+
 def exact_linear(X_bits, W_bits, bias_bits=None, rows=None, nthreads=None) -> np.ndarray:
     X = _c(X_bits, np.uint16)
     W = _c(W_bits, np.uint16)
@@ -285,4 +343,23 @@ def layer(X_bits, W_bits, bias_bits, n, a_bits, w_bits, gran=0, centering=1, alp
     acc = gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
     y, yb = epilogue(acc, a["scale"], w["scale"], colsum=correction(w, centering), bias=w["bias"],
                      mean=a["mean"] if centering else None)
+    return {"sigma": sig, "w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb}
+
+
+def layer_wh(X_bits, W_bits, bias_bits, n_out, a_bits, w_bits, gran=0, alpha=0.5,
+             use_sigma=False, rows=None, static_scale=0.0, nthreads=None):
+    """Weight-only Hadamard form of the layer (HaTQ Eq. (17) with the bias of
+    supplement Eq. (40)-(41)): X quantized in its original basis (no rotation,
+    no centering), Wbar = H_out W quantized per row, integer GEMM, then
+    (dequantized accumulator + b_bar) H_out.  sigma (Eq. 3 of the HadaNorm
+    review) is optional smoothing, off by default as on the HaTQ page."""
+    sig = None
+    if use_sigma:
+        sig = sigma(col_absmax(X_bits), col_absmax(W_bits), alpha)
+    w = prepare_weights_wh(W_bits, n_out, w_bits, bias_bits=bias_bits, sigma=sig,
+                           nthreads=nthreads)
+    a = quantize_act(X_bits, 1, a_bits, gran=gran, centering=0, sigma=sig,
+                     static_scale=static_scale, rows=rows, nthreads=nthreads)
+    acc = gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
+    y, yb = epilogue_wh(acc, n_out, a["scale"], w["scale"], b_bar=w["b_bar"])
     return {"sigma": sig, "w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb}

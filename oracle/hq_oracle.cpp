@@ -15,6 +15,9 @@
  *                              s_x * s_w.
  *   Data-free 4-bit blog, "Hadamard rotation", step 7: H block-diagonal,
  *                              one block per group.
+ *   HaTQ Sec. IV-B, Eq. (15)-(17), supplement Eq. (40)-(41): the weight-only
+ *                              form, W rotated along the output channels and
+ *                              the output basis restored after accumulation.
  * No fast transform is used: the block Hadamard product is a dense sum over
  * the popcount-sign entries, and the GEMM is a triple loop.
  */
@@ -392,6 +395,92 @@ int hqo_exact_linear(const uint16_t* X, const uint16_t* W, const uint16_t* bias,
       y[i * N + c] = s + (bias ? hqo_bf16_to_f64(bias[c]) : 0.0);
     }
   });
+  return 0;
+}
+
+int hqo_prepare_weights_wh(int64_t K, int64_t N, int64_t n_out, int bits,
+                           const uint16_t* W, const uint16_t* bias,
+                           const double* sigma, int8_t* w_codes, double* w_scale,
+                           double* b_bar, double* tie, double* Wbar, int nthreads) {
+  if (K <= 0 || N <= 0 || !is_pow2(n_out) || N % n_out != 0 || bits < 2 || bits > 8)
+    return -1;
+  if (W == nullptr || w_codes == nullptr || w_scale == nullptr || b_bar == nullptr) return -1;
+  const double q = double(qmax_for_bits(bits));
+  const std::vector<double> Hn = dense_block(n_out);
+  parallel_rows(N, nthreads, [&](int64_t c) {
+    /* Wbar[c,k] = sum_j H_out[c,j] sigma_k W[j,k], j over c's block of N */
+    const int64_t c0 = (c / n_out) * n_out;
+    std::vector<double> wb(K);
+    for (int64_t k = 0; k < K; ++k) {
+      const double s = sigma ? sigma[k] : 1.0;
+      double acc = 0.0;
+      for (int64_t j = c0; j < c0 + n_out; ++j)
+        acc += Hn[size_t((c - c0) * n_out + (j - c0))] * s * hqo_bf16_to_f64(W[j * K + k]);
+      wb[k] = acc;
+    }
+    double a = 0.0;
+    for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(wb[k]));
+    const double sc = a / q;
+    w_scale[c] = sc;
+    for (int64_t k = 0; k < K; ++k) {
+      double code = 0.0, d = 0.5;
+      if (sc > 0.0) {
+        const double x = wb[k] / sc;
+        code = clampd(hqo_rne(x), -q, q);
+        const double ax = std::fabs(x);
+        d = std::fabs(ax - std::floor(ax) - 0.5);
+      }
+      w_codes[c * K + k] = int8_t(code);
+      if (tie) tie[c * K + k] = d;
+      if (Wbar) Wbar[c * K + k] = wb[k];
+    }
+    /* b_bar[c] = sum_j b[j] H_out[j,c] */
+    double bb = 0.0;
+    if (bias) {
+      for (int64_t j = c0; j < c0 + n_out; ++j)
+        bb += hqo_bf16_to_f64(bias[j]) * Hn[size_t((j - c0) * n_out + (c - c0))];
+    }
+    b_bar[c] = bb;
+  });
+  return 0;
+}
+
+int hqo_output_rotation(const double* M, int64_t rows, int64_t N, int64_t n_out,
+                        double* out) {
+  if (M == nullptr || out == nullptr || rows < 0 || N <= 0 || !is_pow2(n_out) ||
+      N % n_out != 0)
+    return -1;
+  const std::vector<double> Hn = dense_block(n_out);
+  for (int64_t i = 0; i < rows; ++i) {
+    for (int64_t c = 0; c < N; ++c) {
+      const int64_t c0 = (c / n_out) * n_out;
+      double acc = 0.0;
+      for (int64_t j = c0; j < c0 + n_out; ++j)
+        acc += M[i * N + j] * Hn[size_t((j - c0) * n_out + (c - c0))];
+      out[i * N + c] = acc;
+    }
+  }
+  return 0;
+}
+
+int hqo_epilogue_wh(const int64_t* acc, int64_t nrows, int64_t N, int64_t n_out,
+                    const double* sx, const double* sw, const double* b_bar,
+                    double* y, uint16_t* y_bf16) {
+  if (acc == nullptr || sx == nullptr || sw == nullptr || nrows < 0 || N <= 0 ||
+      !is_pow2(n_out) || N % n_out != 0)
+    return -1;
+  std::vector<double> A(static_cast<size_t>(N)), Y(static_cast<size_t>(N));
+  for (int64_t i = 0; i < nrows; ++i) {
+    /* the bracket of Eq. (41): dequantized Q(X) Q(Wbar)^T plus b_bar */
+    for (int64_t j = 0; j < N; ++j)
+      A[size_t(j)] = sx[i] * sw[j] * double(acc[i * N + j]) + (b_bar ? b_bar[j] : 0.0);
+    /* back to the original output basis: times (T_out)^T = H_out */
+    if (hqo_output_rotation(A.data(), 1, N, n_out, Y.data()) != 0) return -1;
+    for (int64_t c = 0; c < N; ++c) {
+      if (y) y[i * N + c] = Y[size_t(c)];
+      if (y_bf16) y_bf16[i * N + c] = hqo_f64_to_bf16(Y[size_t(c)]);
+    }
+  }
   return 0;
 }
 

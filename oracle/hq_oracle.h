@@ -107,6 +107,32 @@ int hqo_exact_linear(const uint16_t* X, const uint16_t* W, const uint16_t* bias,
                      int64_t T, int64_t K, int64_t N, const int64_t* rows,
                      int64_t nrows, double* y, int nthreads);
 
+/* Weight-only Hadamard (WH) form, HaTQ Sec. IV-B Eq. (15)-(17) and
+ * supplement Eq. (40)-(41): the weights are rotated along the output
+ * channels instead of the input channels.  H_out is block diagonal with
+ * normalized Sylvester blocks of order n_out along N.
+ *   Wbar[c,k] = sum_j H_out[c,j] sigma_k W[j,k]   (Wbar = H_out W diag(sigma))
+ *   b_bar     = b H_out
+ *   w_scale[c] = max_k |Wbar[c,k]| / q,  w_codes = clamp(rne(Wbar / w_scale), +-q)
+ * sigma == NULL means sigma = 1; bias == NULL means b = 0.  tie (distance of
+ * each |Wbar / w_scale| from a rounding tie) and Wbar may be NULL. */
+int hqo_prepare_weights_wh(int64_t K, int64_t N, int64_t n_out, int bits,
+                           const uint16_t* W, const uint16_t* bias,
+                           const double* sigma, int8_t* w_codes, double* w_scale,
+                           double* b_bar, double* tie, double* Wbar, int nthreads);
+
+/* The WH output side (Eq. (41)): A[i,j] = sx[i] * sw[j] * acc[i*N+j] + b_bar[j],
+ * then y[i,c] = sum_j A[i,j] H_out[j,c] (back to the original output basis),
+ * and y_bf16 its bf16 rounding (either output may be NULL; b_bar may be NULL). */
+int hqo_epilogue_wh(const int64_t* acc, int64_t nrows, int64_t N, int64_t n_out,
+                    const double* sx, const double* sw, const double* b_bar,
+                    double* y, uint16_t* y_bf16);
+
+/* out[i,c] = sum_j M[i,j] H_out[j,c] for an fp64 matrix M [rows, N]: the WH
+ * output-basis restoration alone. */
+int hqo_output_rotation(const double* M, int64_t rows, int64_t N, int64_t n_out,
+                        double* out);
+
 #ifdef __cplusplus
 }
 #endif

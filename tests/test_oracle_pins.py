@@ -399,3 +399,103 @@ def test_quantization_noise_is_within_grid_bound():
     V = r["Z"] - r["mean"][:, None]
     err = np.abs(V - r["scale"][:, None] * r["codes"])
     assert np.all(err <= r["scale"][:, None] / 2 * (1 + 1e-12))
+
+
+# --------------------------------------------------------------------------
+# weight-only Hadamard form: HaTQ Eq. (15)-(17), supplement Eq. (40)-(41)
+# --------------------------------------------------------------------------
+
+def _block_h(N, n_out):
+    """Normalized block-diagonal Sylvester matrix built from the Kronecker
+    power (independent of the oracle's popcount construction)."""
+    return np.kron(np.eye(N // n_out), kron_sylvester(n_out) / math.sqrt(n_out))
+
+
+@pytest.mark.parametrize("N,n_out", [(4, 2), (32, 16), (64, 64), (96, 32)])
+def test_wh_weights_are_the_output_side_rotation(N, n_out):
+    """Wbar = H_out W diag(sigma) and b_bar = b H_out against explicit
+    matrices; the codes quantize Wbar row by row."""
+    K = 24
+    g = np.random.default_rng(N + n_out)
+    W = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32))
+    b = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32))
+    sig = 10.0 ** g.uniform(-0.5, 0.5, size=K)
+    w = oracle.prepare_weights_wh(W, n_out, 8, bias_bits=b, sigma=sig, want_Wbar=True)
+    Hout = _block_h(N, n_out)
+    Wf = synth.bf16_bits_to_f32(W).astype(np.float64)
+    bf = synth.bf16_bits_to_f32(b).astype(np.float64)
+    assert np.allclose(w["Wbar"], Hout @ (Wf * sig[None, :]), rtol=0, atol=1e-12)
+    assert np.allclose(w["b_bar"], bf @ Hout, rtol=0, atol=1e-12)
+    s = np.abs(w["Wbar"]).max(axis=1) / 127.0
+    assert np.allclose(w["scale"], s, rtol=1e-15)
+    assert np.all(np.abs(w["codes"]).max(axis=1) == 127)
+    assert np.array_equal(w["codes"], np.clip(oracle.rne(w["Wbar"] / s[:, None]), -127, 127))
+
+
+@pytest.mark.parametrize("n_out", [1, 2, 16, 64])
+def test_wh_identity_unquantized(n_out):
+    """Eq. (16) / (41) with quantization off: (X Wbar^T + b_bar) H_out = X W^T + b."""
+    T, K, N = 7, 40, 128
+    g = np.random.default_rng(n_out)
+    X = synth.f32_to_bf16_bits(g.standard_normal((T, K)).astype(np.float32))
+    W = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32))
+    b = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32))
+    w = oracle.prepare_weights_wh(W, n_out, 8, bias_bits=b, want_Wbar=True)
+    Xf = synth.bf16_bits_to_f32(X).astype(np.float64)
+    y = oracle.output_rotation(Xf @ w["Wbar"].T + w["b_bar"][None, :], n_out)
+    ex = oracle.exact_linear(X, W, b)
+    assert np.allclose(y, ex, rtol=0, atol=1e-11 * np.abs(ex).max())
+
+
+def test_wh_hand_worked_example():
+    """N = 2, n_out = 2, K = 1, W = [3, 1]^T, b = [1, -1], 4-bit codes:
+    Wbar = H_2 W = [4, 2] / sqrt(2), b_bar = b H_2 = [0, 2] / sqrt(2);
+    row scales Wbar / 7 put both codes at 7.  With X = [[2]] quantized per
+    token (code 7, scale 2/7), acc = [49, 49] and the bracket of Eq. (41) is
+    [2 * 4/sqrt(2), 2 * 2/sqrt(2) + 2/sqrt(2)] = [8, 6] / sqrt(2); times H_2
+    gives [14, 2] / 2 = [7, 1] = X W^T + b exactly (2*3 + 1, 2*1 - 1)."""
+    W = synth.f32_to_bf16_bits(np.array([[3.0], [1.0]], dtype=np.float32))
+    b = synth.f32_to_bf16_bits(np.array([1.0, -1.0], dtype=np.float32))
+    X = synth.f32_to_bf16_bits(np.array([[2.0]], dtype=np.float32))
+    r = oracle.layer_wh(X, W, b, 2, 4, 4)
+    r2 = math.sqrt(2.0)
+    assert np.allclose(r["w"]["scale"], [4 / r2 / 7, 2 / r2 / 7], rtol=1e-15)
+    assert np.array_equal(r["w"]["codes"], [[7], [7]])
+    assert np.allclose(r["w"]["b_bar"], [0.0, 2 / r2], atol=1e-15)
+    assert np.array_equal(r["a"]["codes"], [[7]])
+    assert np.array_equal(r["acc"], [[49, 49]])
+    assert np.allclose(r["y"], [[7.0, 1.0]], atol=1e-14)
+
+
+def test_wh_order_one_is_the_plain_quantized_product():
+    """n_out = 1: no rotation on either side; the WH layer is then the
+    per-token quantized product dequantized column by column, recomputed here
+    with integer numpy arithmetic."""
+    T, K, N = 9, 48, 20
+    g = np.random.default_rng(3)
+    X = synth.f32_to_bf16_bits(g.standard_normal((T, K)).astype(np.float32))
+    W = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32))
+    b = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32))
+    r = oracle.layer_wh(X, W, b, 1, 4, 4)
+    Xf = synth.bf16_bits_to_f32(X).astype(np.float64)
+    Wf = synth.bf16_bits_to_f32(W).astype(np.float64)
+    sx = np.abs(Xf).max(axis=1) / 7.0
+    sw = np.abs(Wf).max(axis=1) / 7.0
+    ax = np.clip(oracle.rne(Xf / sx[:, None]), -7, 7).astype(np.int64)
+    aw = np.clip(oracle.rne(Wf / sw[:, None]), -7, 7).astype(np.int64)
+    y = (ax @ aw.T) * sx[:, None] * sw[None, :] + synth.bf16_bits_to_f32(b)[None, :]
+    assert np.array_equal(r["a"]["codes"], ax) and np.array_equal(r["w"]["codes"], aw)
+    assert np.allclose(r["y"], y, rtol=0, atol=1e-12 * np.abs(y).max())
+
+
+@pytest.mark.parametrize("n_out", [16, 64])
+def test_wh_epilogue_against_explicit_matrices(n_out):
+    """The WH epilogue on random integer accumulators equals
+    (diag(sx) acc diag(sw) + b_bar) H_out built from the Kronecker power."""
+    nr, N = 5, 128
+    g = np.random.default_rng(n_out + 1)
+    acc = g.integers(-5000, 5000, size=(nr, N)).astype(np.int64)
+    sx, sw, bb = g.random(nr) + 0.1, g.random(N) * 0.01, g.standard_normal(N)
+    y, _ = oracle.epilogue_wh(acc, n_out, sx, sw, bb)
+    ref = (sx[:, None] * acc * sw[None, :] + bb[None, :]) @ _block_h(N, n_out)
+    assert np.allclose(y, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
