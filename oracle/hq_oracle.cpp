@@ -223,7 +223,7 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
   };
 
   /* Per-tensor dynamic scale: max |Z - m| over every row of the tensor. */
-  double tensor_scale = 0.0;
+  double tensor_scale = 0.0, tensor_max = 0.0;
   if (gran == 1) {
     std::vector<double> row_max(T, 0.0);
     parallel_rows(T, nthreads, [&](int64_t t) {
@@ -236,6 +236,7 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
     });
     double a = 0.0;
     for (int64_t t = 0; t < T; ++t) a = std::fmax(a, row_max[t]);
+    tensor_max = a;
     tensor_scale = a / q;
   } else if (gran == 2) {
     tensor_scale = static_scale;
@@ -250,20 +251,24 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
       for (int64_t k = 0; k < K; ++k) Z[i * K + k] = V[k];
     }
     for (int64_t k = 0; k < K; ++k) V[k] -= m; /* V = Z - mu */
-    double s;
+    /* s = a / q with a = max |V| (dynamic), or the given s (static).  The
+     * scaled value V / s is formed as V * q / a for a dynamic scale: the same
+     * number, one rounding instead of two, so a value that lies exactly on a
+     * rounding tie stays on it (unrotated bf16 inputs do). */
+    double s, a = 0.0;
     if (gran == 0) {
-      double a = 0.0;
       for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(V[k]));
       s = a / q;
     } else {
       s = tensor_scale;
+      a = tensor_max;
     }
     scale[i] = s;
     mean[i] = mu;
     for (int64_t k = 0; k < K; ++k) {
       double c = 0.0, d = 0.5;
       if (s > 0.0) {
-        double x = V[k] / s;
+        double x = gran == 2 ? V[k] / s : (V[k] * q) / a;
         c = clampd(hqo_rne(x), -q, q);
         double ax = std::fabs(x);
         d = std::fabs(ax - std::floor(ax) - 0.5);
@@ -318,7 +323,7 @@ int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
     for (int64_t k = 0; k < K; ++k) {
       double code = 0.0, d = 0.5;
       if (s > 0.0) {
-        double x = wt[k] / s;
+        double x = (wt[k] * q) / a; /* = wt / s, one rounding (see hqo_quantize_act) */
         code = clampd(hqo_rne(x), -q, q);
         double ax = std::fabs(x);
         d = std::fabs(ax - std::floor(ax) - 0.5);
@@ -407,32 +412,36 @@ int hqo_prepare_weights_wh(int64_t K, int64_t N, int64_t n_out, int bits,
   if (W == nullptr || w_codes == nullptr || w_scale == nullptr || b_bar == nullptr) return -1;
   const double q = double(qmax_for_bits(bits));
   const std::vector<double> Hn = dense_block(n_out);
+  const double inv_sqrt_m = 1.0 / std::sqrt(double(n_out));
   parallel_rows(N, nthreads, [&](int64_t c) {
-    /* Wbar[c,k] = sum_j H_out[c,j] sigma_k W[j,k], j over c's block of N */
+    /* S[c,k] = sum_j H~_out[c,j] sigma_k W[j,k] with the +-1 entries, j over
+     * c's block of N; Wbar = S / sqrt(n_out).  The codes depend only on
+     * Wbar / max|Wbar| = S / max|S|, formed from S so that the normalization
+     * does not move a value that lies exactly on a rounding tie. */
     const int64_t c0 = (c / n_out) * n_out;
-    std::vector<double> wb(K);
+    std::vector<double> su(K);
     for (int64_t k = 0; k < K; ++k) {
       const double s = sigma ? sigma[k] : 1.0;
       double acc = 0.0;
       for (int64_t j = c0; j < c0 + n_out; ++j)
-        acc += Hn[size_t((c - c0) * n_out + (j - c0))] * s * hqo_bf16_to_f64(W[j * K + k]);
-      wb[k] = acc;
+        acc += double(hqo_hadamard_entry(c - c0, j - c0)) * s * hqo_bf16_to_f64(W[j * K + k]);
+      su[k] = acc;
     }
-    double a = 0.0;
-    for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(wb[k]));
-    const double sc = a / q;
+    double au = 0.0;
+    for (int64_t k = 0; k < K; ++k) au = std::fmax(au, std::fabs(su[k]));
+    const double sc = (au * inv_sqrt_m) / q; /* max|Wbar| / q */
     w_scale[c] = sc;
     for (int64_t k = 0; k < K; ++k) {
       double code = 0.0, d = 0.5;
-      if (sc > 0.0) {
-        const double x = wb[k] / sc;
+      if (au > 0.0) {
+        const double x = (su[k] * q) / au; /* = Wbar / w_scale */
         code = clampd(hqo_rne(x), -q, q);
         const double ax = std::fabs(x);
         d = std::fabs(ax - std::floor(ax) - 0.5);
       }
       w_codes[c * K + k] = int8_t(code);
       if (tie) tie[c * K + k] = d;
-      if (Wbar) Wbar[c * K + k] = wb[k];
+      if (Wbar) Wbar[c * K + k] = su[k] * inv_sqrt_m;
     }
     /* b_bar[c] = sum_j b[j] H_out[j,c] */
     double bb = 0.0;

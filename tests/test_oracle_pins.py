@@ -5,6 +5,7 @@ import itertools
 import json
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -429,7 +430,10 @@ def test_wh_weights_are_the_output_side_rotation(N, n_out):
     s = np.abs(w["Wbar"]).max(axis=1) / 127.0
     assert np.allclose(w["scale"], s, rtol=1e-15)
     assert np.all(np.abs(w["codes"]).max(axis=1) == 127)
-    assert np.array_equal(w["codes"], np.clip(oracle.rne(w["Wbar"] / s[:, None]), -127, 127))
+    # codes from the unnormalized +-1 sums (the normalization cancels in Wbar / max|Wbar|)
+    S = np.kron(np.eye(N // n_out), kron_sylvester(n_out)) @ (Wf * sig[None, :])
+    x = S * 127.0 / np.abs(S).max(axis=1)[:, None]
+    assert np.array_equal(w["codes"], np.clip(oracle.rne(x), -127, 127))
 
 
 @pytest.mark.parametrize("n_out", [1, 2, 16, 64])
@@ -481,8 +485,21 @@ def test_wh_order_one_is_the_plain_quantized_product():
     Wf = synth.bf16_bits_to_f32(W).astype(np.float64)
     sx = np.abs(Xf).max(axis=1) / 7.0
     sw = np.abs(Wf).max(axis=1) / 7.0
-    ax = np.clip(oracle.rne(Xf / sx[:, None]), -7, 7).astype(np.int64)
-    aw = np.clip(oracle.rne(Wf / sw[:, None]), -7, 7).astype(np.int64)
+
+    def exact_codes(M):
+        # rne(7 m / max|row|) in exact rational arithmetic (bf16 values are dyadic)
+        out = np.zeros(M.shape, dtype=np.int64)
+        for i, row in enumerate(M):
+            a = max(abs(Fraction(float(v))) for v in row)
+            for j, v in enumerate(row):
+                x = Fraction(float(v)) * 7 / a
+                f = math.floor(x)
+                c = f + 1 if x - f > Fraction(1, 2) else (f if x - f < Fraction(1, 2) else
+                                                         (f if f % 2 == 0 else f + 1))
+                out[i, j] = max(-7, min(7, c))
+        return out
+
+    ax, aw = exact_codes(Xf), exact_codes(Wf)
     y = (ax @ aw.T) * sx[:, None] * sw[None, :] + synth.bf16_bits_to_f32(b)[None, :]
     assert np.array_equal(r["a"]["codes"], ax) and np.array_equal(r["w"]["codes"], aw)
     assert np.allclose(r["y"], y, rtol=0, atol=1e-12 * np.abs(y).max())
