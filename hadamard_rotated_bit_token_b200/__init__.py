@@ -60,11 +60,14 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("had_order", ctypes.c_int32),
                 ("a_bits", ctypes.c_int32), ("w_bits", ctypes.c_int32),
                 ("act_gran", ctypes.c_int32), ("centering", ctypes.c_int32),
-                ("code_format", ctypes.c_int32)]
+                ("code_format", ctypes.c_int32), ("out_order", ctypes.c_int32)]
 
     def __init__(self, K, N, had_order, a_bits=4, w_bits=4, act_gran=HQ_PER_TOKEN,
-                 centering=HQ_CENTER_TOKEN_MEAN, code_format=HQ_CODES_I8):
-        super().__init__(K, N, had_order, a_bits, w_bits, act_gran, centering, code_format)
+                 centering=HQ_CENTER_TOKEN_MEAN, code_format=HQ_CODES_I8, out_order=0):
+        """out_order > 1 selects the weight-only Hadamard form (had_order 1,
+        centering HQ_CENTER_NONE): W rotated along N in blocks of out_order."""
+        super().__init__(K, N, had_order, a_bits, w_bits, act_gran, centering, code_format,
+                         out_order)
 
 
 _lib = None

@@ -19,7 +19,7 @@ __device__ unsigned int g_error_word = 0;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kVersion = 10100;  // 1.1.0: out_order (weight-only Hadamard form)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -31,7 +31,7 @@ struct DeviceState {
   int sm_count = 0;
   int cc_major = 0, cc_minor = 0;
   unsigned int* err = nullptr;
-  bool quant_attr_set[8][4][3] = {};
+  bool quant_attr_set[11][4][3] = {};  // [log2 n][mode][centering]
   int pair_clusters = -1;  // co-resident clusters of the CTA-pair GEMM (-1: not queried)
 };
 
@@ -89,9 +89,21 @@ int ilog2_exact(int n) {
 hq_status check_k_side(const hq_layer_desc* d) {
   const int logn = ilog2_exact(d->had_order);
   if (d->K <= 0 || d->had_order <= 0) return HQ_ERR_INVALID_ARGUMENT;
-  if (logn < 4 || logn > 10) return HQ_ERR_UNSUPPORTED;
+  if (logn != 0 && (logn < 4 || logn > 10)) return HQ_ERR_UNSUPPORTED;
   if (d->K % d->had_order != 0 || d->K % 64 != 0 || d->K > 9216) return HQ_ERR_UNSUPPORTED;
   if (d->code_format != HQ_CODES_I8) return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+
+// The output side: out_order 0 or 1 is the double-Hadamard form; 16, 32 or
+// 64 the weight-only Hadamard form, which leaves K unrotated and has no
+// centering.
+hq_status check_out_side(const hq_layer_desc* d) {
+  if (d->out_order < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (d->out_order <= 1) return HQ_OK;
+  if (d->out_order != 16 && d->out_order != 32 && d->out_order != 64) return HQ_ERR_UNSUPPORTED;
+  if (d->had_order != 1 || d->centering != HQ_CENTER_NONE) return HQ_ERR_UNSUPPORTED;
+  if (d->N % d->out_order != 0) return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
 
@@ -104,6 +116,9 @@ hq_status check_desc(const hq_layer_desc* d) {
   hq_status s = check_k_side(d);
   if (s != HQ_OK) return s;
   if (d->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  s = check_out_side(d);
+  if (s != HQ_OK) return s;
+  if (d->had_order == 1 && d->centering != HQ_CENTER_NONE) return HQ_ERR_UNSUPPORTED;
   if (d->a_bits != 3 && d->a_bits != 4 && d->a_bits != 8) return HQ_ERR_UNSUPPORTED;
   if (d->w_bits != 4 && d->w_bits != 8) return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
@@ -165,7 +180,7 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
   L.p.wait_ns = wait_ns();
   L.threads = nt;
   L.logn = logn;
-  L.smem = quant_smem_bytes(R, K, K / n, nt / 32, xpose);
+  L.smem = quant_smem_bytes(R, K, n == 1 ? 0 : K / n, nt / 32, xpose);
   const int64_t ntiles = (T + R - 1) / R;
   const int64_t slots = int64_t(dev->sm_count) * per_sm;
   L.grid = int(ntiles < slots ? ntiles : slots);
@@ -179,7 +194,7 @@ hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, int center, cuda
   if (L.p.T <= 0) return HQ_OK;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    bool& set = dev->quant_attr_set[logn - 4 < 0 ? 0 : logn - 4][mode][center];
+    bool& set = dev->quant_attr_set[logn][mode][center];
     if (!set) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024) !=
           cudaSuccess)
@@ -228,13 +243,16 @@ struct GemmChoice {
   int bn;  // single-CTA tile width
 };
 
-GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int variant) {
+GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int variant,
+                       int logo) {
   static const int cands[] = {256, 192, 128, 64};
   const int64_t mt = (T + 127) / 128;
   const int64_t kb = (K + 127) / 128;
-  int best_bn = 64;
+  int best_bn = 128;
   double best_cost = 1e300;
   for (int bn : cands) {
+    // 64-column output blocks of the weight-only form need 64 columns per epilogue warp
+    if (logo == 6 && bn % 128 != 0) continue;
     const int64_t tiles = mt * ((N + bn - 1) / bn);
     const int64_t rounds = (tiles + sms - 1) / sms;
     const double tile = double(kb) * 4.0 * (126.0 + bn / 16.0) * 1.15 + 2000.0 * (bn / 64);
@@ -244,7 +262,8 @@ GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int 
       best_bn = bn;
     }
   }
-  if (variant == HQ_GEMM_SINGLE_CTA || pair_clusters <= 0) return {false, best_bn};
+  // the weight-only Hadamard epilogue runs in the single-CTA kernel only
+  if (variant == HQ_GEMM_SINGLE_CTA || pair_clusters <= 0 || logo > 0) return {false, best_bn};
   if (variant == HQ_GEMM_CTA_PAIR) return {true, 256};
   // automatic: the pair for long main loops (>= 20 K blocks) over N in whole
   // 256-column tiles, when it needs no more tile rounds than the best single
@@ -319,8 +338,20 @@ hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const
     s = from_cuda(launch_fill(sigma_inv, K, 1.0f, st));
   }
   if (s != HQ_OK) return s;
+  const int qw = (1 << (desc->w_bits - 1)) - 1;
+  if (desc->out_order > 1) {
+    // weight-only Hadamard form: Wbar = H_out W diag(sigma) quantized per row;
+    // no centering, so no correction vector
+    s = from_cuda(launch_wh_weights(W, act_absmax ? sigma_inv : nullptr, K, N, desc->out_order,
+                                    qw, w_codes, w_scale, st));
+    if (s == HQ_OK) s = from_cuda(launch_fill(colsum, N, 0.0f, st));
+    if (s != HQ_OK) return s;
+    if (bias) return from_cuda(launch_bf16_to_f32(bias, bias_f32, N, st));
+    return from_cuda(launch_fill(bias_f32, N, 0.0f, st));
+  }
   // W~ rows: multiply by sigma (= 1 / sigma_inv), rotate, quantize per row,
-  // and record each row's sum (colsum of W~ in the pages' orientation)
+  // and record each row's sum (colsum of W~ in the pages' orientation); with
+  // had_order 1 (no rotation, no centering) no sum is needed
   QuantLaunch L;
   s = make_quant_launch(dev, K, desc->had_order, N, W, &L);
   if (s != HQ_OK) return s;
@@ -330,10 +361,11 @@ hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const
   L.p.codes = w_codes;
   L.p.scale = w_scale;
   L.p.mean = nullptr;
-  L.p.rowsum = colsum;
+  L.p.rowsum = desc->had_order > 1 ? colsum : nullptr;
   L.p.rowsum_pre = desc->centering == HQ_CENTER_TOKEN_MEAN_PRE ? 1 : 0;
-  L.p.q = (1 << (desc->w_bits - 1)) - 1;
+  L.p.q = qw;
   s = run_quant(dev, L, 0, 0, st);
+  if (s == HQ_OK && desc->had_order == 1) s = from_cuda(launch_fill(colsum, N, 0.0f, st));
   if (s != HQ_OK) return s;
   if (bias) return from_cuda(launch_bf16_to_f32(bias, bias_f32, N, st));
   return from_cuda(launch_fill(bias_f32, N, 0.0f, st));
@@ -405,6 +437,13 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
   if (desc->a_bits < 2 || desc->a_bits > 8 || desc->w_bits < 2 || desc->w_bits > 8)
     return HQ_ERR_UNSUPPORTED;
+  if (desc->out_order < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->out_order > 1) {
+    if (desc->out_order != 16 && desc->out_order != 32 && desc->out_order != 64)
+      return HQ_ERR_UNSUPPORTED;
+    if (desc->N % desc->out_order != 0) return HQ_ERR_UNSUPPORTED;
+    if (a_mean != nullptr) return HQ_ERR_INVALID_ARGUMENT;  // the form has no centering
+  }
   if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
   if (a_codes == nullptr || a_scale == nullptr || w_codes == nullptr || w_scale == nullptr ||
       Y == nullptr)
@@ -432,8 +471,11 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
     std::lock_guard<std::mutex> lock(g_mutex);
     variant = g_gemm_variant;
   }
-  if (variant == HQ_GEMM_CTA_PAIR && dev->pair_clusters <= 0) return HQ_ERR_UNSUPPORTED;
-  const GemmChoice gc = choose_gemm(T, N, K, dev->sm_count, dev->pair_clusters, variant);
+  // weight-only Hadamard form: output blocks of m = out_order columns
+  const int m = desc->out_order > 1 ? desc->out_order : 1;
+  const int logo = ilog2_exact(m);
+  if (variant == HQ_GEMM_CTA_PAIR && dev->pair_clusters <= 0 && logo == 0) return HQ_ERR_UNSUPPORTED;
+  const GemmChoice gc = choose_gemm(T, N, K, dev->sm_count, dev->pair_clusters, variant, logo);
   const int bn = gc.pair ? 256 : gc.bn;
   CUtensorMap ta, tb, ty;
   s = encode_kmajor_i8(&ta, a_codes, T, K, 128);
@@ -460,6 +502,7 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.T = T;
   p.N = N;
   p.K = K;
+  p.inv_sqrt_out = float(1.0 / std::sqrt(double(m)));
   p.err = dev->err;
   p.wait_ns = wait_ns();
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -474,7 +517,7 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.num_n_tiles = (N + bn - 1) / bn;
   const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
   const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
-  return from_cuda(launch_gemm(bn, &ta, &tb, &ty, p, grid, st));
+  return from_cuda(launch_gemm(bn, logo, &ta, &tb, &ty, p, grid, st));
 }
 
 hq_status hq_check_device_error(hq_stream_t stream) {

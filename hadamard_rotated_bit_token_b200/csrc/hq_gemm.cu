@@ -131,6 +131,22 @@ __device__ __forceinline__ void load_row_params(const GemmParams& p, int64_t row
   }
 }
 
+// Raw accumulators of chunk c to acc_debug (bit-exact checks), when asked for.
+__device__ __forceinline__ void epi_acc_debug(const GemmParams& p, const uint32_t (&r)[32], int c,
+                                              const EpiTile& e) {
+  if (p.acc_debug && e.row_ok) {
+    const int col0 = e.col_base + c * 32;
+    int32_t* arow = p.acc_debug + e.row * p.N;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (col0 + 4 * g < p.N) {
+        *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
+            make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+      }
+    }
+  }
+}
+
 // One 32-column chunk c of the warp's columns: accumulators r (this thread's
 // row) -> fp32 epilogue -> bf16 pairs in `packed`.  prm points at the warp's
 // first column in a parameter slot of width W.
@@ -164,16 +180,74 @@ __device__ __forceinline__ void epi_math(const GemmParams& p, const uint32_t (&r
     packed[2 * g] = pack_bf16x2(y01.x, y01.y);
     packed[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
   }
-  if (p.acc_debug && e.row_ok) {
-    const int col0 = e.col_base + c * 32;
-    int32_t* arow = p.acc_debug + e.row * p.N;
+  epi_acc_debug(p, r, c, e);
+}
+
+// Weight-only Hadamard form, step 1 for chunk c: z = acc * (s_x * s_w) in the
+// output Hadamard basis (no mean term: the form has no centering).
+template <int W>
+__device__ __forceinline__ void epi_dequant(const GemmParams& p, const uint32_t (&r)[32], int c,
+                                            const EpiTile& e, const float* prm, f2 (&z)[16]) {
+  const float* pw = prm + c * 32;
+  const f2 sx2 = pk(e.sx, e.sx);
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      if (col0 + 4 * g < p.N) {
-        *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
-            make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+  for (int g = 0; g < 8; ++g) {
+    const float4 sw = *reinterpret_cast<const float4*>(pw + 4 * g);
+    f2 a01, a23;
+    if (p.small_acc) {
+      const f2 mg = pk(kAccMagic, kAccMagic);
+      a01 = sub2(pk(__int_as_float(int(r[4 * g + 0]) + kAccMagicBits),
+                    __int_as_float(int(r[4 * g + 1]) + kAccMagicBits)), mg);
+      a23 = sub2(pk(__int_as_float(int(r[4 * g + 2]) + kAccMagicBits),
+                    __int_as_float(int(r[4 * g + 3]) + kAccMagicBits)), mg);
+    } else {
+      a01 = pk(__int2float_rn(int(r[4 * g + 0])), __int2float_rn(int(r[4 * g + 1])));
+      a23 = pk(__int2float_rn(int(r[4 * g + 2])), __int2float_rn(int(r[4 * g + 3])));
+    }
+    z[2 * g] = mul2(a01, mul2(sx2, pk(sw.x, sw.y)));
+    z[2 * g + 1] = mul2(a23, mul2(sx2, pk(sw.z, sw.w)));
+  }
+  epi_acc_debug(p, r, c, e);
+}
+
+// Unnormalized fast Walsh-Hadamard transform over blocks of 2^LOGB (<= 32)
+// consecutive columns of a chunk held as 16 column pairs: index bit 0 inside
+// each pair, bits 1 .. LOGB-1 between pairs.
+template <int LOGB>
+__device__ __forceinline__ void fwht_chunk(f2 (&z)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = z[i].x, b = z[i].y;
+    z[i] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+#pragma unroll
+  for (int bit = 1; bit < LOGB; ++bit) {
+    const int hh = 1 << (bit - 1);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & hh) == 0) {
+        const f2 x = z[i], y = z[i + hh];
+        z[i] = add2(x, y);
+        z[i + hh] = sub2(x, y);
       }
     }
+  }
+}
+
+// Weight-only Hadamard form, last step for chunk c: y = z / sqrt(m) + b in
+// the original output basis -> bf16 pairs.
+template <int W>
+__device__ __forceinline__ void epi_finish(const GemmParams& p, const f2 (&z)[16], int c,
+                                           const float* prm, uint32_t (&packed)[16]) {
+  const float* pw = prm + c * 32;
+  const f2 inv2 = pk(p.inv_sqrt_out, p.inv_sqrt_out);
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const float4 bb = *reinterpret_cast<const float4*>(pw + 2 * W + 4 * g);
+    const f2 y01 = fma2(z[2 * g], inv2, pk(bb.x, bb.y));
+    const f2 y23 = fma2(z[2 * g + 1], inv2, pk(bb.z, bb.w));
+    packed[2 * g] = pack_bf16x2(y01.x, y01.y);
+    packed[2 * g + 1] = pack_bf16x2(y23.x, y23.y);
   }
 }
 
@@ -208,7 +282,11 @@ __device__ __forceinline__ void epi_store_chunk(const GemmParams& p, const CUten
 //     last used the chunk's box has read it, then the box and its TMA store;
 //   - `release_params` frees the parameter slot after the last chunk's
 //     arithmetic.
-template <int HC, int W, int NBOX, class RelAcc, class RelPrm>
+// LOGO > 0 selects the weight-only Hadamard epilogue with output blocks of
+// 2^LOGO columns (4, 5 or 6): dequantize, a fast Walsh-Hadamard transform
+// over each block (inside a chunk, and for 64-column blocks one more stage
+// between the two chunks of a group), then 1/sqrt(m) and the bias.
+template <int HC, int W, int NBOX, int LOGO, class RelAcc, class RelPrm>
 __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap* tmY,
                                          uint32_t t_addr, const EpiTile& e, const float* prm,
                                          uint8_t* stg, int lane, RelAcc release_acc,
@@ -216,6 +294,8 @@ __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap*
   constexpr int NCH = HC / 32;
   constexpr int G = NCH <= 3 ? NCH : 2;
   static_assert(NCH % G == 0, "whole groups of chunks");
+  static_assert(LOGO == 0 || (LOGO >= 4 && LOGO <= 5) || (LOGO == 6 && G % 2 == 0),
+                "output blocks of 16 or 32 columns, or 64 over chunk pairs");
 #pragma unroll
   for (int c0 = 0; c0 < NCH; c0 += G) {
     uint32_t r[G][32];
@@ -223,16 +303,48 @@ __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap*
     for (int c = 0; c < G; ++c) tmem_ld_32x32b_x32(t_addr + uint32_t((c0 + c) * 32), r[c]);
     tmem_wait_ld();
     if (c0 + G == NCH) release_acc();
+    if constexpr (LOGO == 0) {
 #pragma unroll
-    for (int c = 0; c < G; ++c) {
-      const int ch = c0 + c;
-      uint32_t packed[16];
-      epi_math<W>(p, r[c], ch, e, prm, packed);
-      if (ch == NCH - 1) release_params();
-      if (lane == 0) bulk_wait_group_read<NBOX - 1>();
-      __syncwarp();
-      epi_store_chunk(p, tmY, packed, e.col_base + ch * 32, e.row0, stg + (ch % NBOX) * kStageBox,
-                      lane);
+      for (int c = 0; c < G; ++c) {
+        const int ch = c0 + c;
+        uint32_t packed[16];
+        epi_math<W>(p, r[c], ch, e, prm, packed);
+        if (ch == NCH - 1) release_params();
+        if (lane == 0) bulk_wait_group_read<NBOX - 1>();
+        __syncwarp();
+        epi_store_chunk(p, tmY, packed, e.col_base + ch * 32, e.row0,
+                        stg + (ch % NBOX) * kStageBox, lane);
+      }
+    } else {
+      f2 z[G][16];
+#pragma unroll
+      for (int c = 0; c < G; ++c) {
+        epi_dequant<W>(p, r[c], c0 + c, e, prm, z[c]);
+        fwht_chunk<(LOGO < 5 ? LOGO : 5)>(z[c]);
+      }
+      if constexpr (LOGO == 6) {
+        // index bit 5: between the two 32-column chunks of each pair
+#pragma unroll
+        for (int c = 0; c < G; c += 2) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const f2 x = z[c][i], y = z[c + 1][i];
+            z[c][i] = add2(x, y);
+            z[c + 1][i] = sub2(x, y);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < G; ++c) {
+        const int ch = c0 + c;
+        uint32_t packed[16];
+        epi_finish<W>(p, z[c], ch, prm, packed);
+        if (ch == NCH - 1) release_params();
+        if (lane == 0) bulk_wait_group_read<NBOX - 1>();
+        __syncwarp();
+        epi_store_chunk(p, tmY, packed, e.col_base + ch * 32, e.row0,
+                        stg + (ch % NBOX) * kStageBox, lane);
+      }
     }
   }
 }
@@ -263,7 +375,7 @@ struct GemmCfg {
   static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
 };
 
-template <int BN>
+template <int BN, int LOGO>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -452,7 +564,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + uint32_t(acc * BN + half * C::HC) +
                               (uint32_t(quarter * 32) << 16);
-      epi_tile<C::HC, BN, C::NBOX>(
+      epi_tile<C::HC, BN, C::NBOX, LOGO>(
           p, &tmY, t_addr, e, ring + acc * 3 * BN + half * C::HC, stg, lane,
           [&] {
             tc_fence_before();
@@ -712,7 +824,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + uint32_t(acc * C::BN + half * C::HC) +
                               (uint32_t(quarter * 32) << 16);
-      epi_tile<C::HC, C::BN, C::NBOX>(
+      epi_tile<C::HC, C::BN, C::NBOX, 0>(
           p, &tmY, t_addr, e, ring + acc * 3 * C::BN + half * C::HC, stg, lane,
           [&] {
             tc_fence_before();
@@ -752,30 +864,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 }
 
 // ------------------------------------------------------------------ launch
-template <int BN>
+template <int BN, int LOGO>
 static cudaError_t launch_bn(const void* tmap_a, const void* tmap_b, const void* tmap_y,
                              const GemmParams& p, int grid, cudaStream_t st) {
   using C = GemmCfg<BN>;
   static bool configured = false;  // attribute is per function, device-agnostic
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<BN>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<BN, LOGO>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  gemm_i8_kernel<BN><<<grid, kGemmThreads, C::SMEM, st>>>(
+  gemm_i8_kernel<BN, LOGO><<<grid, kGemmThreads, C::SMEM, st>>>(
       *reinterpret_cast<const CUtensorMap*>(tmap_a), *reinterpret_cast<const CUtensorMap*>(tmap_b),
       *reinterpret_cast<const CUtensorMap*>(tmap_y), p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const void* tmap_y,
-                        const GemmParams& p, int grid, cudaStream_t st) {
+template <int LOGO>
+static cudaError_t launch_logo(int bn, const void* tmap_a, const void* tmap_b,
+                               const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
   switch (bn) {
-    case 64: return launch_bn<64>(tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 128: return launch_bn<128>(tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 192: return launch_bn<192>(tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 256: return launch_bn<256>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 128: return launch_bn<128, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 256: return launch_bn<256, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    default:
+      if constexpr (LOGO <= 5) {
+        if (bn == 64) return launch_bn<64, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
+        if (bn == 192) return launch_bn<192, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
+      }
+      return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gemm(int bn, int logo, const void* tmap_a, const void* tmap_b,
+                        const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
+  switch (logo) {
+    case 0: return launch_logo<0>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 4: return launch_logo<4>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 5: return launch_logo<5>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 6: return launch_logo<6>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -30,8 +30,9 @@ struct QuantParams {
   unsigned long long wait_ns; // bounded-wait limit
 };
 
-// Returns the kernel entry for log2(n) in [4,10], mode in [0,3], centering
-// in [0,2] (the HQ_CENTER_* values); the kernel
+// Returns the kernel entry for log2(n) in [4,10] (or 0: n = 1, no rotation,
+// centering 0 only), mode in [0,3], centering in [0,2] (the HQ_CENTER_*
+// values), or NULL; the kernel
 // takes (QuantParams p) and runs R * S active threads per CTA (rounded up to
 // whole warps, at most quant_max_threads()).
 const void* quant_kernel_ptr(int logn, int mode, int center);
@@ -55,16 +56,19 @@ struct GemmParams {
   int K;
   int num_m_tiles;
   int num_n_tiles;
+  float inv_sqrt_out;         // 1/sqrt(m) of the output-side transform (weight-only form)
   unsigned int* err;          // device error word
   unsigned long long wait_ns; // bounded-wait limit
 };
 
-// Launches the tcgen05 GEMM for N tile width bn (64, 128, 192 or 256).
-// tmap_a / tmap_b / tmap_y point to host CUtensorMap objects (copied into the
-// launch): A [T,K] and B [N,K] int8 with box {128, 128 | bn} and 128-byte
-// swizzle; Y [T,N] bf16 with box {32, 32} and 64-byte swizzle.
-cudaError_t launch_gemm(int bn, const void* tmap_a, const void* tmap_b, const void* tmap_y,
-                        const GemmParams& p, int grid, cudaStream_t st);
+// Launches the tcgen05 GEMM for N tile width bn (64, 128, 192 or 256) and
+// output-side transform log2(m) = logo (0: none; 4 or 5 with any bn; 6 with
+// bn 128 or 256).  tmap_a / tmap_b / tmap_y point to host CUtensorMap
+// objects (copied into the launch): A [T,K] and B [N,K] int8 with box
+// {128, 128 | bn} and 128-byte swizzle; Y [T,N] bf16 with box {32, 32} and
+// 64-byte swizzle.
+cudaError_t launch_gemm(int bn, int logo, const void* tmap_a, const void* tmap_b,
+                        const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st);
 size_t gemm_smem_bytes(int bn);
 int gemm_threads();
 
@@ -84,5 +88,10 @@ cudaError_t launch_sigma_inv(const float* act_absmax, float* sigma_inv, int K, f
                              cudaStream_t st);
 cudaError_t launch_fill(float* p, int n, float v, cudaStream_t st);
 cudaError_t launch_bf16_to_f32(const uint16_t* in, float* out, int n, cudaStream_t st);
+// Weight-only Hadamard form, weight side: codes [N,K] and w_scale [N] of
+// Wbar = H_out W diag(sigma) (blocks of m in {16, 32, 64} rows; N % m == 0);
+// sigma_inv NULL means sigma = 1.
+cudaError_t launch_wh_weights(const uint16_t* W, const float* sigma_inv, int K, int N, int m,
+                              int q, int8_t* codes, float* w_scale, cudaStream_t st);
 
 }  // namespace hq

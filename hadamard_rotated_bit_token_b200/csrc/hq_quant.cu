@@ -45,6 +45,8 @@
 // Arithmetic on pairs of lanes uses Blackwell's packed fp32x2 instructions.
 #include <cuda.h>
 
+#include <cmath>
+
 #include "hq_device.cuh"
 #include "hq_kernels.h"
 
@@ -169,7 +171,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   const int S = p.S;  // 32-channel slices per row
   const int R = p.R;  // rows per tile
   const int K = p.K;
-  const int B = K >> LOGN;
+  // blocks whose first channels are kept (none for n = 1: no rotation, no
+  // centering, no row sums)
+  const int B = LOGN == 0 ? 0 : K >> LOGN;
   const int BP = padded_blocks(B);
   const int64_t T = p.T;
   const int64_t ntiles = (T + R - 1) / R;
@@ -184,10 +188,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);
   const WaitCtl wc{p.err, p.wait_ns};
   const bool has_mult = p.mult != nullptr;
-  const bool need_sum = CM != 0 || p.rowsum != nullptr;
+  const bool need_sum = LOGN > 0 && (CM != 0 || p.rowsum != nullptr);
   // the rows' block sums (first rotated channel of each block) instead of
   // their blocks' first input channels
-  const bool block_sums = PRE || (p.rowsum != nullptr && p.rowsum_pre);
+  const bool block_sums = LOGN > 0 && (PRE || (p.rowsum != nullptr && p.rowsum_pre));
 
   const bool active = tid < R * S;
   const int row0 = active ? tid / S : 0;  // this thread's row of every tile
@@ -254,12 +258,20 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   const int csw = sub & (CH - 1);       // chunk swizzle of this transpose group
 
   float r_tensor = 0.0f;
+  // n = 1 (no rotation): the code is rne(V * num / den) with a correctly
+  // rounded division -- num = q and den = max |V| for dynamic scales, num = 1
+  // and den = s for a static one -- so a bf16 value lying exactly on a
+  // rounding tie (common without a rotation) is rounded half to even, as the
+  // quantizer's definition asks; den_tensor is the per-tensor den
+  float den_tensor = 0.0f;
   if (MODE == 2) {
     const float a = __uint_as_float(*p.tensor_max);
+    den_tensor = a;
     r_tensor = a > 0.0f ? __fdiv_rn(float(p.q), a) : 0.0f;
     if (blockIdx.x == 0 && tid == 0 && p.scale) p.scale[0] = (a / float(p.q)) * p.inv_sqrt_n;
   } else if (MODE == 3) {
     const float s = p.static_scale[0];
+    den_tensor = s * p.sqrt_n;
     r_tensor = s > 0.0f ? __fdiv_rn(1.0f, s * p.sqrt_n) : 0.0f;
   }
   const float n_over_k = float(N) / float(K);
@@ -295,11 +307,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
 #pragma unroll
       for (int b = 0; b < BPT; ++b) yrow[blk * BPT + b] = w[(b * N) >> 1].x;
     }
-    // index bit 0: the two halves of a pair
+    // index bit 0: the two halves of a pair (n = 1: no rotation)
+    if (LOGN >= 1) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float a = w[i].x, b = w[i].y;
-      w[i] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
+      for (int i = 0; i < 16; ++i) {
+        const float a = w[i].x, b = w[i].y;
+        w[i] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
+      }
     }
     // index bits 1 .. LREG-1: between pairs
 #pragma unroll
@@ -442,7 +456,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
           // q / a_hat to within 2 ulp: moves a code only when V * q / a_hat
           // lies within a few ulp of a rounding boundary
           if (MODE == 0) r_rec = a_hat > 0.0f ? __fdividef(qf, a_hat) : 0.0f;
-          res[sr] = make_float2(m_hat, r_rec);
+          // n = 1 keeps the row's max itself, the divisor of its exact path
+          res[sr] = make_float2(m_hat, LOGN == 0 ? a_hat : r_rec);
           pmax[sr] = 0u;  // ready for tile it + 2
           pmin[sr] = 0xFFFFFFFFu;
           cnt[sr] = 0u;
@@ -477,15 +492,28 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     }
     const float mshift = PRE ? 0.0f : st.x;
     const f2 mh2 = pk(mshift, mshift), rr2 = pk(st.y, st.y), mg2 = pk(kRoundMagic, kRoundMagic);
+    // n = 1: numerator factor and divisor of the exact path
+    const float num = MODE == 3 ? 1.0f : qf;
+    const float den = MODE == 0 ? st.y : den_tensor;
     uint32_t words[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       uint32_t b[4];
+      if (LOGN == 0) {
+        // codes as int32 + the magic's bit pattern, like the fused path
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const f2 t = fma2(sub2(w[2 * g + u], mh2), rr2, mg2);
-        b[2 * u] = __float_as_uint(t.x);
-        b[2 * u + 1] = __float_as_uint(t.y);
+        for (int u = 0; u < 4; ++u) {
+          const float v = (u & 1) ? w[2 * g + (u >> 1)].y : w[2 * g + (u >> 1)].x;
+          const int c = den > 0.0f ? __float2int_rn(__fdiv_rn(__fmul_rn(v, num), den)) : 0;
+          b[u] = uint32_t(c) + kRoundMagicBits;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const f2 t = fma2(sub2(w[2 * g + u], mh2), rr2, mg2);
+          b[2 * u] = __float_as_uint(t.x);
+          b[2 * u + 1] = __float_as_uint(t.y);
+        }
       }
       if (kClamp) {
 #pragma unroll
@@ -529,6 +557,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
 template <int MODE, int CM>
 static const void* pick_by_logn(int logn) {
   switch (logn) {
+    case 0:  // n = 1, no rotation: only without centering
+      if constexpr (CM == 0) return (const void*)quant_rows_kernel<0, MODE, 0>;
+      return nullptr;
     case 4: return (const void*)quant_rows_kernel<4, MODE, CM>;
     case 5: return (const void*)quant_rows_kernel<5, MODE, CM>;
     case 6: return (const void*)quant_rows_kernel<6, MODE, CM>;
@@ -631,6 +662,94 @@ __global__ void fill_kernel(float* __restrict__ p, int n, float v) {
 __global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ in, float* __restrict__ out, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = __uint_as_float(uint32_t(in[i]) << 16);
+}
+
+// ------------------------------------------- weight-only Hadamard weights
+// Weight side of the weight-only Hadamard form (HaTQ Sec. IV-B, Eq. (15)-
+// (17)): Wbar = H_out W diag(sigma), the rows of W rotated along the output
+// channels in blocks of M = 2^LOGO (unnormalized fast Walsh-Hadamard
+// transform over the M rows of a block, then times 1/sqrt(M)), quantized per
+// row.  The codes depend only on Wbar / max|Wbar| = S / max|S| with S the
+// unnormalized sums, so they are formed from S: offline (once per layer),
+// in fp64, where sums of bf16 values are exact, so rne(S q / max|S|) with a
+// correctly rounded division decides a value lying exactly on a rounding tie
+// half to even (such ties are common: S is a sum of bf16 values).  Without a
+// rotation along K the activations keep their outlier channels, which
+// multiply any weight code flip into whole output columns.  One CTA per block of M rows; thread j takes columns j,
+// j + blockDim, ...; pass 1 collects each row's max |Wbar| (shared-memory
+// atomics on the bits of non-negative doubles), pass 2 recomputes the same
+// values and writes the codes.
+template <int LOGO>
+__global__ void __launch_bounds__(256) wh_weights_kernel(const uint16_t* __restrict__ W,
+                                                         const float* __restrict__ sigma_inv,
+                                                         int K, int q, double inv_sqrt_m,
+                                                         int8_t* __restrict__ codes,
+                                                         float* __restrict__ w_scale) {
+  constexpr int M = 1 << LOGO;
+  __shared__ unsigned long long rmax[M];  // bits of each row's max |S| (non-negative)
+  const int64_t r0 = int64_t(blockIdx.x) * M;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) rmax[i] = 0ull;
+  __syncthreads();
+  // column k of the block: sigma_k W[r0 + j, k] rotated over j, unnormalized (fp64)
+  auto column = [&](int k, double (&v)[M]) {
+    // sigma = 1 / sigma_inv in fp32, as the activation side divides by it
+    const double sg = sigma_inv ? double(1.0f / sigma_inv[k]) : 1.0;
+#pragma unroll
+    for (int j = 0; j < M; ++j) v[j] = double(bf16lo(uint32_t(W[(r0 + j) * K + k]))) * sg;
+#pragma unroll
+    for (int h = 1; h < M; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < M; ++i) {
+        if ((i & h) == 0) {
+          const double a = v[i], b = v[i + h];
+          v[i] = a + b;
+          v[i + h] = a - b;
+        }
+      }
+    }
+  };
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    double v[M];
+    column(k, v);
+#pragma unroll
+    for (int j = 0; j < M; ++j)
+      if (v[j] != 0.0) atomicMax(&rmax[j], (unsigned long long)__double_as_longlong(fabs(v[j])));
+  }
+  __syncthreads();
+  const double qd = double(q);
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    double v[M];
+    column(k, v);
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      const double a = __longlong_as_double((long long)rmax[j]);
+      const int c = a > 0.0 ? __double2int_rn((v[j] * qd) / a) : 0;  // round half to even
+      codes[(r0 + j) * K + k] = int8_t(max(-q, min(q, c)));
+    }
+  }
+  for (int j = threadIdx.x; j < M; j += blockDim.x)
+    w_scale[r0 + j] = float((__longlong_as_double((long long)rmax[j]) * inv_sqrt_m) / qd);
+}
+
+cudaError_t launch_wh_weights(const uint16_t* W, const float* sigma_inv, int K, int N, int m,
+                              int q, int8_t* codes, float* w_scale, cudaStream_t st) {
+  const double inv = 1.0 / std::sqrt(double(m));
+  const dim3 grid(unsigned(N / m));
+  const int threads = K < 256 ? ((K + 31) / 32) * 32 : 256;
+  switch (m) {
+    case 16:
+      wh_weights_kernel<4><<<grid, threads, 0, st>>>(W, sigma_inv, K, q, inv, codes, w_scale);
+      break;
+    case 32:
+      wh_weights_kernel<5><<<grid, threads, 0, st>>>(W, sigma_inv, K, q, inv, codes, w_scale);
+      break;
+    case 64:
+      wh_weights_kernel<6><<<grid, threads, 0, st>>>(W, sigma_inv, K, q, inv, codes, w_scale);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_col_absmax(const uint16_t* M, int64_t rows, int K, float* out, cudaStream_t st) {

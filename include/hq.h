@@ -67,7 +67,9 @@ enum { HQ_CODES_I8 = 0 };
 
 /* Layer description, host memory, passed by const pointer.
  *   K, N        input / output channels.
- *   had_order   Hadamard block order n (H = diag(H_n, ..., H_n), K/n blocks).
+ *   had_order   Hadamard block order n along K (H = diag(H_n, ..., H_n), K/n
+ *               blocks): 16 .. 1024, or 1 for no input-side rotation (then
+ *               centering must be HQ_CENTER_NONE).
  *   a_bits      activation code width: 4 (int4, [-7,7]), 3 (int3, [-3,3]) or
  *               8 (int8, [-127,127]); q_a = 2^(a_bits-1) - 1.
  *   w_bits      weight code width: 4 or 8; q_w = 2^(w_bits-1) - 1.
@@ -85,13 +87,21 @@ enum { HQ_CODES_I8 = 0 };
  *               changes (by -sqrt(n) mu_t); the layer's correction becomes
  *               mu_t * sum_k sigma_k W[n,k].
  *               HQ_CENTER_NONE: mu = 0.
- *   code_format HQ_CODES_I8 (one signed code per byte). */
+ *   code_format HQ_CODES_I8 (one signed code per byte).
+ *   out_order   0 or 1: the double-Hadamard form above (no output-side
+ *               transform).  16, 32 or 64: the weight-only Hadamard form
+ *               (HaTQ Sec. IV-B, Eq. (15)-(17)): the weights are rotated
+ *               along the output channels by H_out = diag(H_m, ..., H_m),
+ *               m = out_order, and the output basis is restored after the
+ *               integer GEMM; requires had_order == 1, centering
+ *               HQ_CENTER_NONE and N % out_order == 0. */
 typedef struct hq_layer_desc {
   int32_t K, N, had_order;
   int32_t a_bits, w_bits;
   int32_t act_gran;
   int32_t centering;
   int32_t code_format;
+  int32_t out_order;
 } hq_layer_desc;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -120,6 +130,14 @@ hq_status hq_calib_act_absmax(const hq_layer_desc* desc, const uint16_t* X,
  *   w_scale[n]= max_k |W~[n,k]| / q_w,  w_codes = clamp(rne(W~ / w_scale), +-q_w)
  *   bias_f32  = float(bias), or 0 when bias == NULL.
  * Inputs:  W bf16 [N,K], bias bf16 [N] or NULL, act_absmax fp32 [K] or NULL.
+ * Weight-only Hadamard form (desc->out_order > 1; had_order is 1, so no
+ * rotation along K):
+ *   Wbar[n,:] = sum_j H_out[n,j] sigma W[j,:]   (Wbar = H_out W diag(sigma),
+ *               HaTQ Eq. (15)-(17); j over n's block of out_order rows)
+ *   w_scale[n]= max_k |Wbar[n,k]| / q_w,  w_codes = clamp(rne(Wbar / w_scale), +-q_w)
+ *   colsum    = 0;  bias_f32 = float(bias) (added after the output basis is
+ *               restored, which equals supplement Eq. (41)'s b_bar = b H_out
+ *               added before it).
  * Outputs: w_codes int8 [N,K], w_scale fp32 [N], colsum fp32 [N],
  *          sigma_inv fp32 [K], bias_f32 fp32 [N] (all device, caller-owned).
  * sigma_inv is also used as scratch during the call.  alpha in [0, 1]. */
@@ -148,6 +166,8 @@ size_t hq_quantize_act_workspace_bytes(const hq_layer_desc* desc, int64_t T);
  *            by colsum (zeros when centering is off).
  * workspace: device, >= hq_quantize_act_workspace_bytes(), 16-byte aligned,
  *   contents need not be initialised (the call clears what it uses).
+ * With had_order == 1 (no input-side rotation, as in the weight-only
+ * Hadamard form) H is the identity and Z = Y.
  * A token whose max|V| is 0 gets scale 0 and all-zero codes. */
 hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X,
                           int64_t T, const float* sigma_inv, int8_t* a_codes,
@@ -165,6 +185,14 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X,
  *          when a_mean is NULL), bias_f32 fp32 [N] or NULL (b = 0).
  * Outputs: Y bf16 [T,N]; acc_debug int32 [T,N] or NULL (raw accumulators, for
  *          bit-exact checks; costs an extra 4 bytes per output).
+ * Weight-only Hadamard form (desc->out_order = m > 1; a_mean and colsum
+ * must be NULL): the accumulator is in the output Hadamard basis and the
+ * epilogue restores the original basis (HaTQ Eq. (17), supplement Eq. (41)):
+ *   Z[t,n]   = s_x[t] * w_scale[n] * acc[t,n]
+ *   Y[t,:]   = bf16_rne( Z[t,:] H_out + bias_f32 ),  H_out = diag(H_m, ...)
+ * with H_m the normalized Sylvester block, applied as an fp32 fast
+ * Walsh-Hadamard transform over each group of m output columns.
+ * acc_debug then holds the accumulators in the Hadamard basis.
  * Codes must lie within the declared widths: |a_codes| <= 2^(a_bits-1) and
  * |w_codes| <= 2^(w_bits-1) (a_bits, w_bits in [2, 8]; 8 admits every int8
  * value).  The epilogue converts accumulators exactly either way. */

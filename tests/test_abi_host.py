@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(hq):
 
 
 def test_version_and_status_strings(hq):
-    assert hq.hq_version() == 10000
+    assert hq.hq_version() == 10100
     for code, name in hq.STATUS_NAMES.items():
         assert hq.hq_status_string(code) == name
     assert hq.hq_status_string(99) == "HQ_ERR_UNKNOWN"
@@ -74,6 +74,19 @@ def test_quantize_validation(hq):
     assert _call_quant(hq, D(1024, 16, 1024, act_gran=1), ws=FAKE + 4, ws_bytes=16) == 3
     # T = 0 with valid arguments is a no-op that never touches the device
     assert _call_quant(hq, D(1024, 16, 1024), T=0) == 0
+    # had_order 1: no rotation along K, only without centering
+    assert _call_quant(hq, D(1024, 16, 1, centering=0), T=0) == 0
+    assert _call_quant(hq, D(1024, 16, 1, centering=1)) == 2
+    assert _call_quant(hq, D(1024, 16, 1, centering=2)) == 2
+    # weight-only Hadamard form (out_order > 1): had_order 1, no centering, N % out_order == 0
+    assert _call_quant(hq, D(1024, 64, 1, centering=0, out_order=64), T=0) == 0
+    assert _call_quant(hq, D(1024, 64, 1, centering=0, out_order=1), T=0) == 0
+    assert _call_quant(hq, D(1024, 64, 1024, centering=0, out_order=64)) == 2
+    assert _call_quant(hq, D(1024, 64, 1, centering=1, out_order=64)) == 2
+    assert _call_quant(hq, D(1024, 48, 1, centering=0, out_order=32)) == 2
+    assert _call_quant(hq, D(1024, 64, 1, centering=0, out_order=8)) == 2
+    assert _call_quant(hq, D(1024, 64, 1, centering=0, out_order=128)) == 2
+    assert _call_quant(hq, D(1024, 64, 1, centering=0, out_order=-1)) == 1
 
 
 def test_workspace_bytes(hq):
@@ -100,6 +113,26 @@ def test_linear_validation(hq):
     assert call(D(1024, 16, 1024), y=FAKE + 2) == 3
     assert call(D(1024, 16, 1024), sw=FAKE + 4) == 3
     assert call(D(1024, 16, 1024), T=0) == 0
+    wh = dict(centering=0, out_order=64)
+    assert call(D(1024, 128, 1, **wh), T=0) == 0
+    assert call(D(1024, 128, 1, **wh), m=FAKE, cs=FAKE) == 1   # the form has no centering
+    assert call(D(1024, 80, 1, **wh)) == 2                     # N not a multiple of out_order
+    assert call(D(1024, 128, 1, centering=0, out_order=48)) == 2
+    assert call(D(1024, 128, 1, centering=0, out_order=-2)) == 1
+
+
+def test_layer_desc_layout_matches_the_header(hq):
+    """The binding's struct has the header's fields, in order, all int32."""
+    text = open(os.path.join(ROOT, "include", "hq.h")).read()
+    body = re.search(r"typedef struct hq_layer_desc \{(.*?)\} hq_layer_desc;", text, re.S).group(1)
+    names = []
+    for line in body.strip().splitlines():
+        decl = line.strip().rstrip(";")
+        assert decl.startswith("int32_t ")
+        names += [n.strip() for n in decl[len("int32_t "):].split(",")]
+    assert [f[0] for f in hq.LayerDesc._fields_] == names
+    assert all(f[1] is ctypes.c_int32 for f in hq.LayerDesc._fields_)
+    assert ctypes.sizeof(hq.LayerDesc) == 4 * len(names)
 
 
 def test_prepare_and_calib_validation(hq):

@@ -516,3 +516,137 @@ def test_back_to_back_steps_match_isolated_steps(hq, variant):
             assert torch.equal(Y.view(torch.int16), R.view(torch.int16))
     finally:
         hq.hq_debug_set_gemm_variant(hq.HQ_GEMM_AUTO)
+
+
+# ---------------------------------------------------------------------------
+# no input-side rotation and the weight-only Hadamard form (HaTQ Eq. (15)-(17))
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K,T,bits,gran", [(320, 300, 8, 1), (1024, 129, 4, 0), (1152, 77, 3, 0),
+                                           (320, 513, 8, 0)])
+def test_quantize_without_rotation(hq, K, T, bits, gran):
+    """had_order 1: the activations are quantized in their own basis."""
+    g = np.random.default_rng(K + T)
+    x = (g.laplace(0, 1, size=(T, K)) * 10.0 ** g.uniform(-1, 1, size=K)).astype(np.float32)
+    X = synth.f32_to_bf16_bits(x)
+    ref = oracle.quantize_act(X, 1, bits, gran=gran, centering=0, want_Z=True)
+    desc = hq.LayerDesc(K, 16, 1, a_bits=bits, w_bits=8, act_gran=gran, centering=0)
+    codes, scale, mean = _gpu_quantize(hq, desc, X)
+    _check_act(ref, codes, scale, mean, per_row=(gran == 0))
+    assert np.all(mean == 0.0)
+
+
+WH_CASES = [(320, 320, 64, 8, False), (1152, 3456, 32, 4, True), (256, 128, 16, 8, True),
+            (3072, 1024, 64, 4, False)]
+
+
+@pytest.mark.parametrize("K,N,m,w_bits,use_sigma", WH_CASES)
+def test_wh_prepare_weights(hq, K, N, m, w_bits, use_sigma):
+    """Wbar = H_out W diag(sigma) quantized per row, against the oracle."""
+    g = np.random.default_rng(K + N + m)
+    Wb = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32) *
+                                (1 + 10 * (g.random(N) < 0.05)).astype(np.float32)[:, None])
+    bb = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32))
+    absmax_np = None
+    sig = None
+    if use_sigma:
+        absmax_np = (np.abs(g.standard_normal(K)) * 3 + 0.1).astype(np.float32)
+        sig = oracle.sigma(absmax_np.astype(np.float64), oracle.col_absmax(Wb), 0.5)
+    ref = oracle.prepare_weights_wh(Wb, m, w_bits, bias_bits=bb, sigma=sig)
+    desc = hq.LayerDesc(K, N, 1, a_bits=8, w_bits=w_bits, centering=0, out_order=m)
+    absmax = None if absmax_np is None else torch.from_numpy(absmax_np).cuda()
+    layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), absmax)
+    assert hq.hq_check_device_error() == 0
+    check_codes(layer.w_codes.cpu().numpy(), ref["codes"], ref["tie"], "wh w_codes",
+                min_match=0.999)
+    check_rel(layer.w_scale.cpu().numpy(), ref["scale"], SCALE_RTOL, "wh w_scale")
+    assert np.all(layer.colsum.cpu().numpy() == 0.0)
+    assert np.array_equal(layer.bias_f32.cpu().numpy(),
+                          synth.bf16_bits_to_f32(bb).astype(np.float32))
+
+
+@pytest.mark.parametrize("T,K,N,m", [(300, 320, 320, 64), (129, 1152, 640, 32), (513, 256, 128, 16),
+                                     (200, 512, 1024, 64)])
+def test_wh_gemm_fed_oracle_codes(hq, gemm_variant, T, K, N, m):
+    """The oracle's codes through hq_linear in the weight-only form: int32
+    accumulators bit-exact (in the Hadamard basis), output against the
+    oracle's (dequantized accumulator + b_bar) H_out.  The form always runs
+    the single-CTA kernel, whichever variant is asked for."""
+    g = np.random.default_rng(T + K + N)
+    Xb = synth.f32_to_bf16_bits(g.standard_normal((T, K)).astype(np.float32))
+    Wb = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32) * 0.05)
+    bb = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32))
+    r = oracle.layer_wh(Xb, Wb, bb, m, 8, 8)
+    desc = hq.LayerDesc(K, N, 1, a_bits=8, w_bits=8, centering=0, out_order=m)
+    d = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in dict(
+        A=r["a"]["codes"], B=r["w"]["codes"], sx=r["a"]["scale"].astype(np.float32),
+        sw=r["w"]["scale"].astype(np.float32),
+        b=synth.bf16_bits_to_f32(bb).astype(np.float32)).items()}
+    Y = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    acc = torch.full((T, N), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    hq.hq_linear(desc, d["A"], d["sx"], None, d["B"], d["sw"], None, d["b"], Y, acc)
+    assert hq.hq_check_device_error() == 0
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), r["acc"])
+    # the same accumulators and fp32-rounded scales through the oracle's output side
+    _, y_ref = oracle.epilogue_wh(r["acc"], m, r["a"]["scale"].astype(np.float32).astype(np.float64),
+                                  r["w"]["scale"].astype(np.float32).astype(np.float64),
+                                  b_bar=r["w"]["b_bar"])
+    # fp32 against fp64 on both sides of the bf16 rounding: the fp32 transform
+    # over m columns is off by about log2(m) sqrt(m) 2^-24 of an output
+    # (~3e-6 for m = 64), which moves an output across a bf16 rounding
+    # boundary for ~2 * 3e-6 / 2^-8 ~ 0.15% of outputs, each by one bf16 ulp
+    # (2^-8 relative): a Frobenius error of about sqrt(1.5e-3) * 2^-8 ~ 1e-4
+    err = rel_frob(bf16_bits(Y), y_ref)
+    assert err <= 1e-4, err
+
+
+@pytest.mark.parametrize("T,K,N,m,a_bits,w_bits,gran,use_sigma",
+                         [(1000, 320, 320, 64, 8, 8, 1, False), (257, 1152, 3456, 32, 4, 4, 0, False),
+                          (300, 256, 512, 16, 8, 8, 0, True), (129, 3072, 1024, 64, 4, 4, 0, False)])
+def test_wh_layer(hq, T, K, N, m, a_bits, w_bits, gran, use_sigma):
+    """The whole weight-only Hadamard layer on the GPU against oracle.layer_wh."""
+    g = np.random.default_rng(T + N)
+    x = (g.laplace(0, 1, size=(T, K)) * (1 + 8 * (g.random(K) < 0.02))).astype(np.float32)
+    x += np.abs(g.standard_normal((T, 1))).astype(np.float32)  # a nonzero channel mean
+    Xb = synth.f32_to_bf16_bits(x)
+    Wb = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32) * 0.03)
+    bb = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32) * 0.1)
+    ref = oracle.layer_wh(Xb, Wb, bb, m, a_bits, w_bits, gran=gran, use_sigma=use_sigma)
+    desc = hq.LayerDesc(K, N, 1, a_bits=a_bits, w_bits=w_bits, act_gran=gran, centering=0,
+                        out_order=m)
+    X = to_dev_u16(Xb, torch)
+    absmax = None
+    if use_sigma:
+        absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
+        hq.hq_calib_act_absmax(desc, X, absmax)
+    layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), absmax)
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    Y = layer(X, acc_debug=acc)
+    assert hq.hq_check_device_error() == 0
+    bufs = layer.buffers(T)
+    check_codes(bufs["a_codes"].cpu().numpy(), ref["a"]["codes"], ref["a"]["tie"], "wh a_codes")
+    check_codes(layer.w_codes.cpu().numpy(), ref["w"]["codes"], ref["w"]["tie"], "wh w_codes")
+    err = rel_frob(bf16_bits(Y), ref["y_bf16"])
+    assert err <= Y_REL_FROB, err
+    same = (np.all(bufs["a_codes"].cpu().numpy() == ref["a"]["codes"]) and
+            np.all(layer.w_codes.cpu().numpy() == ref["w"]["codes"]))
+    if same:
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+
+
+def test_no_rotation_double_form_layer(hq):
+    """had_order 1 with no output transform: the plain per-token quantized
+    product, through the same library calls."""
+    T, K, N = 300, 1024, 512
+    g = np.random.default_rng(11)
+    Xb = synth.f32_to_bf16_bits(g.standard_normal((T, K)).astype(np.float32))
+    Wb = synth.f32_to_bf16_bits(g.standard_normal((N, K)).astype(np.float32) * 0.05)
+    bb = synth.f32_to_bf16_bits(g.standard_normal(N).astype(np.float32))
+    ref = oracle.layer(Xb, Wb, bb, 1, 8, 8, centering=0, use_sigma=False)
+    desc = hq.LayerDesc(K, N, 1, a_bits=8, w_bits=8, centering=0)
+    layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), None)
+    Y = layer(to_dev_u16(Xb, torch))
+    assert hq.hq_check_device_error() == 0
+    check_codes(layer.w_codes.cpu().numpy(), ref["w"]["codes"], ref["w"]["tie"], "w_codes")
+    assert np.all(layer.colsum.cpu().numpy() == 0.0)
+    assert rel_frob(bf16_bits(Y), ref["y_bf16"]) <= Y_REL_FROB
