@@ -46,13 +46,22 @@ class LayerConfig:
     outlier_count: int
     outlier_mult: float
     offset_std: float
+    out_order: int = 0     # > 1: the weight-only Hadamard form (had_order 1, W rotated along N)
 
     def with_tokens(self, T: int) -> "LayerConfig":
         return dataclasses.replace(self, T=T)
 
     def workload(self) -> str:
+        rot = f"WH{self.out_order}" if self.out_order > 1 else f"H{self.had_order}"
         return (f"cfg{self.index}:{self.name}:T{self.T}xK{self.K}xN{self.N}"
-                f":H{self.had_order}:A{self.a_bits}W{self.w_bits}")
+                f":{rot}:A{self.a_bits}W{self.w_bits}")
+
+    def weight_only(self, out_order: int) -> "LayerConfig":
+        """The same layer shape and inputs in the weight-only Hadamard form:
+        no rotation along K, no centering, no smoothing, W rotated along N in
+        blocks of out_order."""
+        return dataclasses.replace(self, had_order=1, centering=0, use_sigma=False,
+                                   out_order=out_order)
 
 
 CONFIGS = {
