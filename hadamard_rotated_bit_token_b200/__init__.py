@@ -288,3 +288,81 @@ class HadamardQuantLinear:
         return Y
 
     __call__ = forward
+
+    # ------------------------------------------------------------------
+    # prepared-weights blob (deployment: skip hq_prepare_weights at load)
+    # ------------------------------------------------------------------
+    # Little-endian layout:
+    #   b"HQPW", u32 version (1), 9 x i32 hq_layer_desc fields in header order,
+    #   u32 use_sigma, then five sections, each u64 byte count + payload:
+    #   w_codes int8 [N*K], w_scale f32 [N], colsum f32 [N], sigma_inv f32 [K],
+    #   bias_f32 f32 [N]; then u32 CRC-32 of everything before it.
+    _BLOB_MAGIC = b"HQPW"
+    _BLOB_VERSION = 1
+
+    def export_prepared(self) -> bytes:
+        """The prepared weights and the layer description as one blob."""
+        import struct
+        import zlib
+        import numpy as np
+        d = self.desc
+        head = self._BLOB_MAGIC + struct.pack("<I", self._BLOB_VERSION)
+        head += struct.pack("<9i", d.K, d.N, d.had_order, d.a_bits, d.w_bits, d.act_gran,
+                            d.centering, d.code_format, d.out_order)
+        head += struct.pack("<I", 1 if self.use_sigma else 0)
+        parts = [head]
+        for t, dt in ((self.w_codes, np.int8), (self.w_scale, np.float32),
+                      (self.colsum, np.float32), (self.sigma_inv, np.float32),
+                      (self.bias_f32, np.float32)):
+            raw = t.detach().contiguous().cpu().numpy().astype(dt, copy=False).tobytes()
+            parts.append(struct.pack("<Q", len(raw)) + raw)
+        body = b"".join(parts)
+        return body + struct.pack("<I", zlib.crc32(body) & 0xFFFFFFFF)
+
+    @classmethod
+    def from_prepared(cls, blob: bytes, device=None) -> "HadamardQuantLinear":
+        """A layer from export_prepared()'s blob, without running the weight
+        preparation.  Raises ValueError on a malformed or corrupted blob."""
+        import struct
+        import zlib
+        import numpy as np
+        import torch
+        blob = bytes(blob)
+        if len(blob) < 4 + 4 + 36 + 4 + 4 or blob[:4] != cls._BLOB_MAGIC:
+            raise ValueError("not a prepared-weights blob")
+        body, crc = blob[:-4], struct.unpack("<I", blob[-4:])[0]
+        if zlib.crc32(body) & 0xFFFFFFFF != crc:
+            raise ValueError("prepared-weights blob: checksum mismatch")
+        version = struct.unpack_from("<I", body, 4)[0]
+        if version != cls._BLOB_VERSION:
+            raise ValueError(f"prepared-weights blob: unsupported version {version}")
+        f = struct.unpack_from("<9i", body, 8)
+        desc = LayerDesc(f[0], f[1], f[2], a_bits=f[3], w_bits=f[4], act_gran=f[5],
+                         centering=f[6], code_format=f[7], out_order=f[8])
+        use_sigma = bool(struct.unpack_from("<I", body, 44)[0])
+        K, N = desc.K, desc.N
+        off = 48
+        arrays = []
+        for dt, count in ((np.int8, N * K), (np.float32, N), (np.float32, N), (np.float32, K),
+                          (np.float32, N)):
+            if off + 8 > len(body):
+                raise ValueError("prepared-weights blob: truncated")
+            nbytes = struct.unpack_from("<Q", body, off)[0]
+            off += 8
+            if nbytes != count * np.dtype(dt).itemsize or off + nbytes > len(body):
+                raise ValueError("prepared-weights blob: section size does not match the description")
+            arrays.append(np.frombuffer(body, dtype=dt, count=count, offset=off).copy())
+            off += nbytes
+        if off != len(body):
+            raise ValueError("prepared-weights blob: trailing bytes")
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        self = cls.__new__(cls)
+        self.desc = desc
+        self.w_codes = torch.from_numpy(arrays[0].reshape(N, K)).to(dev)
+        self.w_scale, self.colsum, self.sigma_inv, self.bias_f32 = (
+            torch.from_numpy(a).to(dev) for a in arrays[1:])
+        self.use_sigma = use_sigma
+        ws = hq_quantize_act_workspace_bytes(desc, 0) if dev.type == "cuda" else 0
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev) if ws else None
+        self._bufs = {}
+        return self
