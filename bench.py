@@ -100,6 +100,7 @@ def gemm_bytes(cfg) -> float:
 # DRAM traffic per launch from a committed ncu summary
 # ---------------------------------------------------------------------------
 
+E2E_CHUNKS = 8  # row chunks of the end-to-end pipeline (hq_forward_host)
 PROFILES = {("gemm", 2): "gemm_i8_cfg2_pixart_qkv.md", ("quant", 2): "quant_rows_cfg2_pixart_qkv.md"}
 KERNEL_SOURCES = {"gemm": ("hq_gemm.cu", "hq_device.cuh", "hq_kernels.h"),
                   "quant": ("hq_quant.cu", "hq_device.cuh", "hq_kernels.h")}
@@ -487,11 +488,11 @@ def run_hq(args):
         Xd = torch.empty_like(X)
 
         def e2e_body():
-            Xd.copy_(Xh, non_blocking=True)
-            hq.hq_quantize_act(desc, Xd, sig_inv, bufs["a_codes"], bufs["a_scale"],
-                               bufs["a_mean"], layer.workspace)
-            linear()
-            Yh.copy_(Y, non_blocking=True)
+            # one public call: uploads, the layer's kernels and downloads of
+            # row chunks overlapped on the library's copy streams
+            hq.hq_forward_host(desc, Xh, Xd, sig_inv, bufs["a_codes"], bufs["a_scale"],
+                               bufs["a_mean"], layer.workspace, layer.w_codes, layer.w_scale,
+                               layer.colsum, layer.bias_f32, Y, Yh, chunks=E2E_CHUNKS)
 
         for _ in range(max(1, args.warmup)):
             e2e_body()

@@ -26,7 +26,7 @@ __all__ = [
     "HQ_CENTER_NONE", "HQ_CENTER_TOKEN_MEAN", "HQ_CENTER_TOKEN_MEAN_PRE", "HQ_CODES_I8",
     "HQ_FAULT_NONE", "HQ_FAULT_QUANT_WITHHOLD_ROW", "STATUS_NAMES",
     "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
-    "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
+    "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
     "hq_debug_set_gemm_variant", "HQ_GEMM_AUTO", "HQ_GEMM_SINGLE_CTA", "HQ_GEMM_CTA_PAIR",
     "hq_quantize_act_noalloc", "HadamardQuantLinear",
@@ -44,7 +44,7 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED
                 3: "HQ_ERR_MISALIGNED", 4: "HQ_ERR_CUDA", 5: "HQ_ERR_TIMEOUT",
                 6: "HQ_ERR_DEVICE"}
 EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare_weights",
-            "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear",
+            "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
             "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
             "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc")
 
@@ -103,6 +103,9 @@ def load_library():
                                         ctypes.c_size_t, _vp]
         lib.hq_linear.argtypes = [desc_p, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                   _vp, _vp]
+        lib.hq_forward_host.argtypes = [desc_p, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        ctypes.c_int, _vp]
         lib.hq_quantize_act_noalloc.argtypes = [desc_p, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp,
                                                 _vp]
         lib.hq_check_device_error.argtypes = [_vp]
@@ -110,6 +113,7 @@ def load_library():
         lib.hq_debug_inject_fault.argtypes = [ctypes.c_int]
         lib.hq_debug_set_gemm_variant.argtypes = [ctypes.c_int]
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
+                     "hq_forward_host",
                      "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
                      "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc"):
             getattr(lib, name).restype = ctypes.c_int
@@ -133,6 +137,18 @@ def _ptr(t):
         return t
     if not t.is_cuda:
         raise ValueError("tensor must live in CUDA device memory")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _host_ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if t.is_cuda:
+        raise ValueError("tensor must live in host memory")
     if not t.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return t.data_ptr()
@@ -198,6 +214,21 @@ def hq_linear(desc: LayerDesc, a_codes, a_scale, a_mean, w_codes, w_scale, colsu
         ctypes.byref(desc), T, _ptr(a_codes), _ptr(a_scale), _ptr(a_mean), _ptr(w_codes),
         _ptr(w_scale), _ptr(colsum), _ptr(bias_f32), _ptr(Y), _ptr(acc_debug), _stream(stream)),
         "hq_linear")
+
+
+def hq_forward_host(desc: LayerDesc, X_host, X_dev, sigma_inv, a_codes, a_scale, a_mean,
+                    workspace, w_codes, w_scale, colsum, bias_f32, Y_dev, Y_host, chunks=8,
+                    T=None, stream=None):
+    """The layer end to end on (pinned) host tensors: uploads, kernels and
+    downloads of `chunks` row chunks overlapped (see include/hq.h).  X_host
+    and Y_host are CPU tensors; X_dev, Y_dev device staging tensors."""
+    T = X_host.shape[0] if T is None else T
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().hq_forward_host(
+        ctypes.byref(desc), _host_ptr(X_host), T, _ptr(X_dev), _ptr(sigma_inv), _ptr(a_codes),
+        _ptr(a_scale), _ptr(a_mean), _ptr(workspace), ws_bytes, _ptr(w_codes), _ptr(w_scale),
+        _ptr(colsum), _ptr(bias_f32), _ptr(Y_dev), _host_ptr(Y_host), int(chunks),
+        _stream(stream)), "hq_forward_host")
 
 
 def hq_quantize_act_noalloc(desc: LayerDesc, X, sigma_inv, a_codes, a_scale, a_mean=None,
@@ -288,6 +319,24 @@ class HadamardQuantLinear:
         return Y
 
     __call__ = forward
+
+    def forward_host(self, X_host, Y_host=None, chunks=8):
+        """Y_host = the layer on X_host (pinned CPU bf16 tensors), with the
+        uploads, kernels and downloads of `chunks` row chunks overlapped
+        (hq_forward_host).  Device staging buffers are kept per token count."""
+        import torch
+        T = X_host.shape[0]
+        b = self.buffers(T)
+        dev = self.w_codes.device
+        if "X_dev" not in b:
+            b["X_dev"] = torch.empty((T, self.desc.K), dtype=torch.bfloat16, device=dev)
+            b["Y_dev"] = torch.empty((T, self.desc.N), dtype=torch.bfloat16, device=dev)
+        if Y_host is None:
+            Y_host = torch.empty((T, self.desc.N), dtype=torch.bfloat16).pin_memory()
+        hq_forward_host(self.desc, X_host, b["X_dev"], self.sigma_inv if self.use_sigma else None,
+                        b["a_codes"], b["a_scale"], b["a_mean"], self.workspace, self.w_codes,
+                        self.w_scale, self.colsum, self.bias_f32, b["Y_dev"], Y_host, chunks)
+        return Y_host
 
     # ------------------------------------------------------------------
     # prepared-weights blob (deployment: skip hq_prepare_weights at load)

@@ -19,7 +19,8 @@ __device__ unsigned int g_error_word = 0;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kVersion = 10100;  // 1.1.0: out_order (weight-only Hadamard form)
+constexpr int kVersion = 10200;  // 1.2.0: hq_forward_host
+constexpr int kMaxHostChunks = 64;  // row chunks of hq_forward_host
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -33,6 +34,8 @@ struct DeviceState {
   unsigned int* err = nullptr;
   bool quant_attr_set[11][4][3] = {};  // [log2 n][mode][centering]
   int pair_clusters = -1;  // co-resident clusters of the CTA-pair GEMM (-1: not queried)
+  // hq_forward_host's upload and download streams (created on first use)
+  cudaStream_t up = nullptr, down = nullptr;
 };
 
 std::mutex g_mutex;
@@ -274,6 +277,56 @@ GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int 
   return {pair, best_bn};
 }
 
+// Argument checks of hq_quantize_act (description, pointers, alignment);
+// T == 0 passes without looking at the pointers.
+hq_status check_quant_args(const hq_layer_desc* desc, const uint16_t* X, int64_t T,
+                           const float* sigma_inv, const int8_t* a_codes, const float* a_scale,
+                           const float* a_mean, const void* workspace, size_t workspace_bytes) {
+  hq_status s = check_desc(desc);
+  if (s != HQ_OK) return s;
+  if (T < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
+  if (X == nullptr || a_codes == nullptr || a_scale == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  const bool dyn = desc->act_gran == HQ_PER_TENSOR_DYNAMIC;
+  if (dyn && (workspace == nullptr || workspace_bytes < 16)) return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(X) || !aligned16(a_codes) || !aligned4(a_scale) || (a_mean && !aligned4(a_mean)) ||
+      (sigma_inv && !aligned16(sigma_inv)) || (dyn && !aligned16(workspace)))
+    return HQ_ERR_MISALIGNED;
+  return HQ_OK;
+}
+
+// Argument checks of hq_linear (shape, pointers, alignment); T == 0 passes
+// without looking at the pointers.
+hq_status check_linear_args(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
+                            const float* a_scale, const float* a_mean, const int8_t* w_codes,
+                            const float* w_scale, const float* colsum, const float* bias_f32,
+                            const uint16_t* Y, const int32_t* acc_debug) {
+  if (desc == nullptr || T < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->K <= 0 || desc->N <= 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->act_gran < HQ_PER_TOKEN || desc->act_gran > HQ_PER_TENSOR_STATIC)
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (desc->a_bits < 2 || desc->a_bits > 8 || desc->w_bits < 2 || desc->w_bits > 8)
+    return HQ_ERR_UNSUPPORTED;
+  if (desc->out_order < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (desc->out_order > 1) {
+    if (desc->out_order != 16 && desc->out_order != 32 && desc->out_order != 64)
+      return HQ_ERR_UNSUPPORTED;
+    if (desc->N % desc->out_order != 0) return HQ_ERR_UNSUPPORTED;
+    if (a_mean != nullptr) return HQ_ERR_INVALID_ARGUMENT;  // the form has no centering
+  }
+  if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
+  if (a_codes == nullptr || a_scale == nullptr || w_codes == nullptr || w_scale == nullptr ||
+      Y == nullptr)
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (a_mean != nullptr && colsum == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(Y) || !aligned16(w_scale) ||
+      (colsum && !aligned16(colsum)) || (bias_f32 && !aligned16(bias_f32)) || !aligned4(a_scale) ||
+      (a_mean && !aligned4(a_mean)) || (acc_debug && !aligned16(acc_debug)))
+    return HQ_ERR_MISALIGNED;
+  return HQ_OK;
+}
+
 }  // namespace
 }  // namespace hq
 
@@ -380,17 +433,10 @@ size_t hq_quantize_act_workspace_bytes(const hq_layer_desc* desc, int64_t T) {
 hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t T,
                           const float* sigma_inv, int8_t* a_codes, float* a_scale, float* a_mean,
                           void* workspace, size_t workspace_bytes, hq_stream_t stream) {
-  hq_status s = check_desc(desc);
-  if (s != HQ_OK) return s;
-  if (T < 0) return HQ_ERR_INVALID_ARGUMENT;
-  if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
-  if (X == nullptr || a_codes == nullptr || a_scale == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  hq_status s = check_quant_args(desc, X, T, sigma_inv, a_codes, a_scale, a_mean, workspace,
+                                 workspace_bytes);
+  if (s != HQ_OK || T == 0) return s;
   const bool dyn = desc->act_gran == HQ_PER_TENSOR_DYNAMIC;
-  if (dyn && (workspace == nullptr || workspace_bytes < 16)) return HQ_ERR_INVALID_ARGUMENT;
-  if (!aligned16(X) || !aligned16(a_codes) || !aligned4(a_scale) || (a_mean && !aligned4(a_mean)) ||
-      (sigma_inv && !aligned16(sigma_inv)) || (dyn && !aligned16(workspace)))
-    return HQ_ERR_MISALIGNED;
-  if (T == 0) return HQ_OK;
   DeviceState* dev;
   s = device_state(&dev);
   if (s != HQ_OK) return s;
@@ -430,32 +476,11 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
                     const float* a_scale, const float* a_mean, const int8_t* w_codes,
                     const float* w_scale, const float* colsum, const float* bias_f32, uint16_t* Y,
                     int32_t* acc_debug, hq_stream_t stream) {
-  if (desc == nullptr || T < 0) return HQ_ERR_INVALID_ARGUMENT;
-  if (desc->K <= 0 || desc->N <= 0) return HQ_ERR_INVALID_ARGUMENT;
-  if (desc->act_gran < HQ_PER_TOKEN || desc->act_gran > HQ_PER_TENSOR_STATIC)
-    return HQ_ERR_INVALID_ARGUMENT;
-  if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
-  if (desc->a_bits < 2 || desc->a_bits > 8 || desc->w_bits < 2 || desc->w_bits > 8)
-    return HQ_ERR_UNSUPPORTED;
-  if (desc->out_order < 0) return HQ_ERR_INVALID_ARGUMENT;
-  if (desc->out_order > 1) {
-    if (desc->out_order != 16 && desc->out_order != 32 && desc->out_order != 64)
-      return HQ_ERR_UNSUPPORTED;
-    if (desc->N % desc->out_order != 0) return HQ_ERR_UNSUPPORTED;
-    if (a_mean != nullptr) return HQ_ERR_INVALID_ARGUMENT;  // the form has no centering
-  }
-  if (T == 0) return HQ_OK;  // nothing to read or write: pointers may be null
-  if (a_codes == nullptr || a_scale == nullptr || w_codes == nullptr || w_scale == nullptr ||
-      Y == nullptr)
-    return HQ_ERR_INVALID_ARGUMENT;
-  if (a_mean != nullptr && colsum == nullptr) return HQ_ERR_INVALID_ARGUMENT;
-  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(Y) || !aligned16(w_scale) ||
-      (colsum && !aligned16(colsum)) || (bias_f32 && !aligned16(bias_f32)) || !aligned4(a_scale) ||
-      (a_mean && !aligned4(a_mean)) || (acc_debug && !aligned16(acc_debug)))
-    return HQ_ERR_MISALIGNED;
-  if (T == 0) return HQ_OK;
+  hq_status s = check_linear_args(desc, T, a_codes, a_scale, a_mean, w_codes, w_scale, colsum,
+                                  bias_f32, Y, acc_debug);
+  if (s != HQ_OK || T == 0) return s;
   DeviceState* dev;
-  hq_status s = device_state(&dev);
+  s = device_state(&dev);
   if (s != HQ_OK) return s;
   const int K = desc->K, N = desc->N;
   if (dev->pair_clusters < 0) {
@@ -518,6 +543,111 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
   const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
   return from_cuda(launch_gemm(bn, logo, &ta, &tb, &ty, p, grid, st));
+}
+
+hq_status hq_forward_host(const hq_layer_desc* desc, const uint16_t* X_host, int64_t T,
+                          uint16_t* X_dev, const float* sigma_inv, int8_t* a_codes,
+                          float* a_scale, float* a_mean, void* workspace, size_t workspace_bytes,
+                          const int8_t* w_codes, const float* w_scale, const float* colsum,
+                          const float* bias_f32, uint16_t* Y_dev, uint16_t* Y_host, int chunks,
+                          hq_stream_t stream) {
+  hq_status s = check_quant_args(desc, X_dev, T, sigma_inv, a_codes, a_scale, a_mean, workspace,
+                                 workspace_bytes);
+  if (s != HQ_OK) return s;
+  const float* mean_in = desc->centering != HQ_CENTER_NONE ? a_mean : nullptr;
+  s = check_linear_args(desc, T, a_codes, a_scale, mean_in, w_codes, w_scale, colsum, bias_f32,
+                        Y_dev, nullptr);
+  if (s != HQ_OK) return s;
+  if (chunks < 1 || chunks > kMaxHostChunks) return HQ_ERR_INVALID_ARGUMENT;
+  if (T == 0) return HQ_OK;
+  if (X_host == nullptr || Y_host == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  DeviceState* dev;
+  s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (dev->up == nullptr) {
+      cudaStream_t up = nullptr, down = nullptr;
+      if (cudaStreamCreateWithFlags(&up, cudaStreamNonBlocking) != cudaSuccess) return HQ_ERR_CUDA;
+      if (cudaStreamCreateWithFlags(&down, cudaStreamNonBlocking) != cudaSuccess) {
+        (void)cudaStreamDestroy(up);
+        return HQ_ERR_CUDA;
+      }
+      dev->up = up;
+      dev->down = down;
+    }
+  }
+  const int K = desc->K, N = desc->N;
+  const bool per_row = desc->act_gran == HQ_PER_TOKEN;
+  // a tensor-wide dynamic scale needs every row before any code: one chunk
+  if (desc->act_gran == HQ_PER_TENSOR_DYNAMIC) chunks = 1;
+  // chunk boundaries: multiples of 128 rows (the GEMM's tile), at most `chunks` of them
+  int64_t step = ((T + chunks - 1) / chunks + 127) / 128 * 128;
+  const int nc = int((T + step - 1) / step);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // this call's events, destroyed once their waits are enqueued (CUDA
+  // releases them when the work completes)
+  cudaEvent_t ev[2 * kMaxHostChunks + 2] = {};
+  const int nev = 2 * nc + 2;
+  auto release = [&]() {
+    for (int e = 0; e < nev; ++e)
+      if (ev[e]) (void)cudaEventDestroy(ev[e]);
+  };
+  for (int e = 0; e < nev; ++e) {
+    if (cudaEventCreateWithFlags(&ev[e], cudaEventDisableTiming) != cudaSuccess) {
+      release();
+      return HQ_ERR_CUDA;
+    }
+  }
+  cudaEvent_t ev_fork = ev[0], ev_join = ev[1], *ev_in = ev + 2, *ev_done = ev + 2 + nc;
+  auto fail = [&](hq_status code) {
+    // join what was started, so that nothing outlives the call's ordering on `stream`
+    (void)cudaEventRecord(ev_join, dev->down);
+    (void)cudaStreamWaitEvent(st, ev_join, 0);
+    (void)cudaEventRecord(ev_join, dev->up);
+    (void)cudaStreamWaitEvent(st, ev_join, 0);
+    release();
+    return code;
+  };
+  // fork: both copy streams start after the work already on `stream`
+  if (cudaEventRecord(ev_fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(dev->up, ev_fork, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(dev->down, ev_fork, 0) != cudaSuccess)
+    return fail(HQ_ERR_CUDA);
+  // uploads of every chunk, back to back on the upload stream
+  for (int c = 0; c < nc; ++c) {
+    const int64_t lo = c * step, rows = (T - lo) < step ? (T - lo) : step;
+    if (cudaMemcpyAsync(X_dev + lo * K, X_host + lo * K, size_t(rows) * K * 2,
+                        cudaMemcpyHostToDevice, dev->up) != cudaSuccess ||
+        cudaEventRecord(ev_in[c], dev->up) != cudaSuccess)
+      return fail(HQ_ERR_CUDA);
+  }
+  // each chunk's layer on `stream` once its upload has landed, and its
+  // download on the download stream once its output is ready
+  for (int c = 0; c < nc; ++c) {
+    const int64_t lo = c * step, rows = (T - lo) < step ? (T - lo) : step;
+    if (cudaStreamWaitEvent(st, ev_in[c], 0) != cudaSuccess) return fail(HQ_ERR_CUDA);
+    const bool whole = nc == 1;
+    s = hq_quantize_act(desc, X_dev + lo * K, rows, sigma_inv, a_codes + lo * K,
+                        (per_row && !whole) ? a_scale + lo : a_scale,
+                        a_mean ? a_mean + lo : nullptr, workspace, workspace_bytes, stream);
+    if (s == HQ_OK)
+      s = hq_linear(desc, rows, a_codes + lo * K, (per_row && !whole) ? a_scale + lo : a_scale,
+                    mean_in ? mean_in + lo : nullptr, w_codes, w_scale, colsum, bias_f32,
+                    Y_dev + lo * N, nullptr, stream);
+    if (s != HQ_OK) return fail(s);
+    if (cudaEventRecord(ev_done[c], st) != cudaSuccess ||
+        cudaStreamWaitEvent(dev->down, ev_done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(Y_host + lo * N, Y_dev + lo * N, size_t(rows) * N * 2,
+                        cudaMemcpyDeviceToHost, dev->down) != cudaSuccess)
+      return fail(HQ_ERR_CUDA);
+  }
+  // join: `stream` continues after the last download
+  if (cudaEventRecord(ev_join, dev->down) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev_join, 0) != cudaSuccess)
+    return fail(HQ_ERR_CUDA);
+  release();
+  return HQ_OK;
 }
 
 hq_status hq_check_device_error(hq_stream_t stream) {

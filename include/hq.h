@@ -202,6 +202,32 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
                     const float* colsum, const float* bias_f32, uint16_t* Y,
                     int32_t* acc_debug, hq_stream_t stream);
 
+/* hq_forward_host -- the layer end to end on host buffers:
+ *   upload X_host -> X_dev, hq_quantize_act, hq_linear -> Y_dev, download
+ *   Y_dev -> Y_host,
+ * split into up to `chunks` row chunks (multiples of 128 rows) whose uploads,
+ * kernels and downloads overlap: the uploads run back to back on a
+ * library-owned upload stream, each chunk's two kernels run on `stream` as
+ * soon as its upload has landed, and its download runs on a library-owned
+ * download stream once its output is ready, so that both directions of the
+ * host link are busy at once.  Results equal the four steps made one after
+ * the other.  HQ_PER_TENSOR_DYNAMIC uses one chunk (its scale needs every
+ * row).  Fork and join use events, so the call is ordered on `stream` and
+ * may be captured in a CUDA graph; the first call on a device creates the two
+ * streams, which live until the process exits (make it before any stream
+ * capture).  X_host and Y_host should be page-locked (cudaHostAlloc or
+ * pinned) for the copies to be asynchronous.
+ * Arguments: X_host bf16 [T,K] and Y_host bf16 [T,N] (host); X_dev bf16 [T,K]
+ * and Y_dev bf16 [T,N] (device staging, caller-owned); chunks in [1, 64];
+ * the others as in hq_quantize_act and hq_linear (a_mean is passed on to the
+ * GEMM only when desc->centering is not HQ_CENTER_NONE). */
+hq_status hq_forward_host(const hq_layer_desc* desc, const uint16_t* X_host, int64_t T,
+                          uint16_t* X_dev, const float* sigma_inv, int8_t* a_codes,
+                          float* a_scale, float* a_mean, void* workspace,
+                          size_t workspace_bytes, const int8_t* w_codes,
+                          const float* w_scale, const float* colsum, const float* bias_f32,
+                          uint16_t* Y_dev, uint16_t* Y_host, int chunks, hq_stream_t stream);
+
 /* hq_quantize_act_noalloc -- hq_quantize_act without a caller workspace.
  * (The paper has no counterpart: this is a deployment convenience.)
  * For callers that cannot allocate device memory when they quantize -- a

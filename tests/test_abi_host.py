@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(hq):
 
 
 def test_version_and_status_strings(hq):
-    assert hq.hq_version() == 10100
+    assert hq.hq_version() == 10200
     for code, name in hq.STATUS_NAMES.items():
         assert hq.hq_status_string(code) == name
     assert hq.hq_status_string(99) == "HQ_ERR_UNKNOWN"
@@ -119,6 +119,31 @@ def test_linear_validation(hq):
     assert call(D(1024, 80, 1, **wh)) == 2                     # N not a multiple of out_order
     assert call(D(1024, 128, 1, centering=0, out_order=48)) == 2
     assert call(D(1024, 128, 1, centering=0, out_order=-2)) == 1
+
+
+def test_forward_host_validation(hq):
+    """hq_forward_host checks both calls' arguments and its own before it
+    enqueues anything."""
+    lib = hq.load_library()
+    D = hq.LayerDesc
+
+    def call(desc, T=4096, Xh=FAKE, Xd=FAKE, a=FAKE, sx=FAKE, m=None, ws=None, wsb=0, w=FAKE,
+             sw=FAKE, cs=FAKE, b=None, yd=FAKE, yh=FAKE, chunks=4):
+        d = None if desc is None else ctypes.byref(desc)
+        return lib.hq_forward_host(d, Xh, T, Xd, None, a, sx, m, ws, wsb, w, sw, cs, b, yd, yh,
+                                   chunks, None)
+
+    assert call(None) == 1
+    assert call(D(1024, 16, 1024), T=-1) == 1
+    assert call(D(1024, 16, 1024), Xh=None) == 1
+    assert call(D(1024, 16, 1024), yh=None) == 1
+    assert call(D(1024, 16, 1024), w=None) == 1
+    assert call(D(1024, 16, 1024), chunks=0) == 1
+    assert call(D(1024, 16, 1024), chunks=65) == 1
+    assert call(D(1024, 16, 1000)) == 2
+    assert call(D(1024, 16, 1024), Xd=FAKE + 2) == 3
+    assert call(D(1024, 16, 1024), yd=FAKE + 8) == 3
+    assert call(D(1024, 16, 1024), T=0) == 0
 
 
 def test_layer_desc_layout_matches_the_header(hq):

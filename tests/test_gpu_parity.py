@@ -650,3 +650,61 @@ def test_no_rotation_double_form_layer(hq):
     check_codes(layer.w_codes.cpu().numpy(), ref["w"]["codes"], ref["w"]["tie"], "w_codes")
     assert np.all(layer.colsum.cpu().numpy() == 0.0)
     assert rel_frob(bf16_bits(Y), ref["y_bf16"]) <= Y_REL_FROB
+
+
+# ---------------------------------------------------------------------------
+# hq_forward_host: uploads, kernels and downloads overlapped by row chunks
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("idx,T,over,chunks", [(2, 8192, {}, 8), (2, 1000, {}, 8),
+                                               (2, 4099, {"centering": 2}, 3),
+                                               (4, 65536, {}, 8), (4, 6000, {"act_gran": 2}, 4),
+                                               (4, 8192, {"out_order": 64}, 8), (3, 300, {}, 1)])
+def test_forward_host_equals_the_device_path(hq, idx, T, over, chunks):
+    """Y_host from hq_forward_host equals upload + quantize + GEMM + download
+    done one after the other, bit for bit, eagerly and from a CUDA graph
+    replayed on fresh input data each time (a stale upload or an early
+    download would show as another replay's output)."""
+    import dataclasses
+    cfg = synth.CONFIGS[idx].with_tokens(T)
+    cfg = (cfg.weight_only(over["out_order"]) if "out_order" in over
+           else dataclasses.replace(cfg, **over))
+    Xb, Wb, bb = synth.make_layer(cfg)
+    K, N = Xb.shape[1], Wb.shape[0]
+    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering, out_order=cfg.out_order)
+    X0 = to_dev_u16(Xb, torch)
+    absmax = None
+    if cfg.use_sigma:
+        absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
+        hq.hq_calib_act_absmax(desc, X0, absmax)
+    layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), absmax,
+                                   cfg.alpha)
+    if cfg.act_gran == hq.HQ_PER_TENSOR_STATIC:
+        layer.buffers(T)["a_scale"].fill_(0.02)
+    inputs = [X0, torch.roll(X0, 131, dims=0).contiguous(), (X0 * 0.5).contiguous()]
+
+    def reference(X):
+        Y = layer.forward(X)     # device path: hq_quantize_act then hq_linear
+        torch.cuda.synchronize()
+        return Y.cpu()
+
+    refs = [reference(X) for X in inputs]
+    X_host = torch.empty((T, K), dtype=torch.bfloat16).pin_memory()
+    Y_host = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
+    for X, R in zip(inputs, refs):                              # eager
+        X_host.copy_(X.cpu())
+        Y_host.fill_(float("nan"))
+        layer.forward_host(X_host, Y_host, chunks=chunks)
+        torch.cuda.synchronize()
+        assert hq.hq_check_device_error() == 0
+        assert torch.equal(Y_host.view(torch.int16), R.view(torch.int16))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward_host(X_host, Y_host, chunks=chunks)
+    for X, R in zip(inputs[::-1], refs[::-1]):                  # graph, fresh data each replay
+        X_host.copy_(X.cpu())
+        Y_host.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(Y_host.view(torch.int16), R.view(torch.int16))
