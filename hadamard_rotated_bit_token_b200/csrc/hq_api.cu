@@ -129,9 +129,6 @@ hq_status check_desc(const hq_layer_desc* d) {
 
 hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
-// Rows per tile R and threads per CTA for the row quantizer: one producer
-// warp plus worker warps in which every thread owns a 32-channel slice of one
-// row; prefer full warps and 8-9 worker warps.
 // Rows per tile R and threads per CTA (one thread per 32-channel slice of
 // each row, whole warps): the R that leaves the fewest idle lanes, preferring
 // larger CTAs.

@@ -25,7 +25,11 @@
 //               lets a TMA tensor store write the 32 x 32 box to Y (clipped at
 //               the tensor's edges).
 //
-// gemm_i8_kernel<BN>: one CTA per 128 x BN output tile (BN 64..256).
+// gemm_i8_kernel<BN, LOGO>: one CTA per 128 x BN output tile (BN 64..256).
+//   LOGO > 0 selects the weight-only Hadamard epilogue (HaTQ Sec. IV-B
+//   Eq. (17)): Y = (s_x s_w acc) H_out + b, the fast Walsh-Hadamard transform
+//   over each block of 2^LOGO output columns done in registers after the
+//   dequantization (no mean term: that form has no centering).
 // gemm_i8_pair_kernel: a cluster of two CTAs per 256 x 256 output tile with
 //   the CTA-pair MMA (cta_group::2, M = 256): each CTA loads 128 rows of A and
 //   128 rows of B into its own shared memory, so one SM moves half the B

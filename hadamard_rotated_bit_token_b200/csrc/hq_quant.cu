@@ -42,6 +42,12 @@
 //            them and releases the row's barrier;
 //   quantize codes packed 4 per word and stored.
 // No CTA-wide barrier in the loop: warps wait only for the rows they hold.
+// With n = 1 (no rotation) the transform is skipped and the codes are formed
+// by a correctly rounded division (see the quantize step).
+//
+// Also here: the offline column reductions for sigma, and the weight side of
+// the weight-only Hadamard form (wh_weights_kernel: W rotated along the
+// output channels, quantized per row, in fp64).
 // Arithmetic on pairs of lanes uses Blackwell's packed fp32x2 instructions.
 #include <cuda.h>
 

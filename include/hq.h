@@ -15,12 +15,16 @@
  * (or per tensor) and W~ per output channel with the symmetric quantizer of
  * HaTQ Sec. III-A Eq. (3), round half to even, and the product runs as an
  * int8 x int8 -> int32 tensor-core GEMM whose accumulator has scale
- * s_x * s_w (HaTQ Sec. IV-B Eq. (18)).
+ * s_x * s_w (HaTQ Sec. IV-B Eq. (18)).  HaTQ's weight-only Hadamard form
+ * (Sec. IV-B Eq. (15)-(17)) is the same pipeline with X unrotated and W
+ * rotated along the output channels (hq_layer_desc.out_order).
  *
  * Memory conventions (all entry points):
- *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
- *     library never allocates, frees or retains device memory; it keeps one
- *     4-byte device error word per device (see hq_check_device_error).
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller, except
+ *     the host buffers of hq_forward_host.  The library never allocates,
+ *     frees or retains device memory; it keeps one 4-byte device error word
+ *     per device (see hq_check_device_error), and hq_forward_host creates two
+ *     copy streams per device on its first call.
  *   - Matrices are row-major.  X is [T,K] (tokens x input channels; NHWC
  *     pixels for a 1x1 convolution), W is [N,K] (output x input channels, the
  *     nn.Linear orientation, i.e. the transpose of the pages' W), Y is [T,N].
@@ -28,15 +32,17 @@
  *   - Pointers to tensors read or written by the tensor-memory engine or by
  *     16-byte vector accesses must be 16-byte aligned (HQ_ERR_MISALIGNED).
  *   - All calls are asynchronous on `stream` (NULL = legacy default stream)
- *     and never synchronize, except hq_check_device_error.
+ *     and never synchronize, except hq_check_device_error; hq_forward_host
+ *     forks onto its copy streams and joins back into `stream`.
  *   - Errors are returned, never raised: the library does not abort, exit or
  *     trap.  Argument checks happen before any launch; a rejected call
  *     launches nothing.
  *
- * Shapes supported:  had_order a power of two in [16, 1024]; K a multiple of
- * had_order and of 64, K <= 9216; N a multiple of 16; T >= 0 (T = 0 is a
- * no-op); a_bits in {3, 4, 8}, w_bits in {4, 8} (codes in an int8 container,
- * one code per byte).
+ * Shapes supported:  had_order a power of two in [16, 1024], or 1 (no
+ * rotation along K); K a multiple of had_order and of 64, K <= 9216; N a
+ * multiple of 16 (and of out_order in the weight-only form, out_order in
+ * {16, 32, 64}); T >= 0 (T = 0 is a no-op); a_bits in {3, 4, 8}, w_bits in
+ * {4, 8} (codes in an int8 container, one code per byte).
  */
 #ifndef HQ_H
 #define HQ_H
