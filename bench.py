@@ -474,7 +474,25 @@ def run_hq(args):
     status = hq.hq_check_device_error()
     if status != 0:
         raise RuntimeError(f"device error in the timed region: {hq.STATUS_NAMES.get(status)}")
-    total_ms, q_total, g_total = max_over_ranks([total_ms, q_total, g_total], world, dist, dev)
+    # context only, outside the timed step: the same layer unquantized, as one
+    # cuBLAS bf16 GEMM (torch.matmul) over the same rotating inputs
+    Yc = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+
+    def cublas_i(i):
+        torch.matmul(Xs[i % n_copies], W.t(), out=Yc)
+
+    cublas_i(0)
+    torch.cuda.synchronize()
+    g_cublas = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_cublas):
+        for i in range(args.steps):
+            cublas_i(i)
+    g_cublas.replay()
+    torch.cuda.synchronize()
+    c_total = timed(g_cublas)
+    del g_cublas, Yc
+    total_ms, q_total, g_total, c_total = max_over_ranks([total_ms, q_total, g_total, c_total],
+                                                         world, dist, dev)
     ms_per_step = total_ms / args.steps
     ops = layer_ops(cfg)
     value = job_throughput(ops, args.steps, world, total_ms)
@@ -555,6 +573,11 @@ def run_hq(args):
                      "hbm_bytes": gemm_bytes(cfg)},
             "weight_prep_ms": prep_ms,
         },
+        "context": {"cublas_bf16_gemm": {
+            "ms_per_launch": c_total / args.steps,
+            "TFLOP/s": ops / (c_total / args.steps * 1e-3) / 1e12,
+            "what": "torch.matmul(X, W^T) in bf16 (cuBLAS) on the same shape and inputs, "
+                    "unquantized; context only, not on the path"}},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock_info,
         "e2e": e2e,
