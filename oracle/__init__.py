@@ -33,6 +33,7 @@ _i64p = ctypes.POINTER(ctypes.c_int64)
 _f64p = ctypes.POINTER(ctypes.c_double)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
 _i8p = ctypes.POINTER(ctypes.c_int8)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 
 
 def build(force: bool = False) -> str:
@@ -87,7 +88,9 @@ def _load():
                                             ctypes.c_int64, _f64p, _f64p, _f64p, _f64p, _u16p]
             lib.hqo_output_rotation.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64,
                                                 ctypes.c_int64, _f64p]
-            for name in ("hqo_sylvester", "hqo_col_absmax", "hqo_sigma", "hqo_quantize_act",
+            lib.hqo_pack_i4.argtypes = [_i8p, ctypes.c_int64, _u8p]
+            lib.hqo_unpack_i4.argtypes = [_u8p, ctypes.c_int64, _i8p]
+            for name in ("hqo_pack_i4", "hqo_unpack_i4", "hqo_sylvester", "hqo_col_absmax", "hqo_sigma", "hqo_quantize_act",
                          "hqo_prepare_weights", "hqo_gemm_acc", "hqo_epilogue",
                          "hqo_exact_linear", "hqo_prepare_weights_wh", "hqo_epilogue_wh",
                          "hqo_output_rotation"):
@@ -221,6 +224,29 @@ def correction(w, centering):
     centering mode: colsum(W~) after the rotation (1), sum_k sigma_k W[n,k]
     before it (2)."""
     return w["corr_pre"] if centering == 2 else w["colsum"]
+
+
+def pack_i4(codes) -> np.ndarray:
+    """Codes [..., K] (K even, each in [-8, 7]) -> packed bytes [..., K/2]:
+    element 2j in the low nibble of byte j, 2j+1 in the high one, as 4-bit
+    two's complement (the packed-code reading of the W4A4 GEMM's 4-bit
+    operands, "Data-free 4-bit quantization for diffusion transformers")."""
+    c = _c(codes, np.int8)
+    if c.shape[-1] % 2:
+        raise ValueError("pack_i4 needs an even number of codes per row")
+    out = np.empty(c.shape[:-1] + (c.shape[-1] // 2,), dtype=np.uint8)
+    _check(_load().hqo_pack_i4(_ptr(c, ctypes.c_int8), c.size, _ptr(out, ctypes.c_uint8)),
+           "pack_i4")
+    return out
+
+
+def unpack_i4(packed) -> np.ndarray:
+    """Packed bytes [..., K/2] -> codes [..., K] (the inverse of pack_i4)."""
+    b = _c(packed, np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int8)
+    _check(_load().hqo_unpack_i4(_ptr(b, ctypes.c_uint8), out.size, _ptr(out, ctypes.c_int8)),
+           "unpack_i4")
+    return out
 
 
 def gemm_acc(A, B, rows=None, nthreads=None) -> np.ndarray:

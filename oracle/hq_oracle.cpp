@@ -493,4 +493,29 @@ int hqo_epilogue_wh(const int64_t* acc, int64_t nrows, int64_t N, int64_t n_out,
   return 0;
 }
 
+int hqo_pack_i4(const int8_t* codes, int64_t count, uint8_t* out) {
+  if (count < 0 || count % 2 != 0 || (count > 0 && (codes == nullptr || out == nullptr)))
+    return -1;
+  for (int64_t j = 0; j < count / 2; ++j) {
+    const int lo = codes[2 * j], hi = codes[2 * j + 1];
+    if (lo < -8 || lo > 7 || hi < -8 || hi > 7) return -1;
+    /* a 4-bit two's-complement value v is stored as v mod 16 */
+    const int lo4 = lo < 0 ? lo + 16 : lo;
+    const int hi4 = hi < 0 ? hi + 16 : hi;
+    out[j] = uint8_t(lo4 + 16 * hi4);
+  }
+  return 0;
+}
+
+int hqo_unpack_i4(const uint8_t* packed, int64_t count, int8_t* codes) {
+  if (count < 0 || count % 2 != 0 || (count > 0 && (codes == nullptr || packed == nullptr)))
+    return -1;
+  for (int64_t j = 0; j < count / 2; ++j) {
+    const int lo4 = packed[j] % 16, hi4 = packed[j] / 16;
+    codes[2 * j] = int8_t(lo4 >= 8 ? lo4 - 16 : lo4);
+    codes[2 * j + 1] = int8_t(hi4 >= 8 ? hi4 - 16 : hi4);
+  }
+  return 0;
+}
+
 }  /* extern "C" */

@@ -133,6 +133,18 @@ int hqo_epilogue_wh(const int64_t* acc, int64_t nrows, int64_t N, int64_t n_out,
 int hqo_output_rotation(const double* M, int64_t rows, int64_t N, int64_t n_out,
                         double* out);
 
+/* Packed storage of 3- and 4-bit codes, two per byte.  The blog "Data-free
+ * 4-bit quantization for diffusion transformers" ("Hadamard rotation: the int4
+ * improvement") runs a W4A4 GEMM on 4-bit operands but fixes no storage
+ * layout; the reading taken here: element 2j of a row in the
+ * low nibble of byte j, element 2j+1 in the high nibble, each as a 4-bit
+ * two's-complement value.  count is the number of codes (even); every code
+ * must lie in [-8, 7] (hqo_pack_i4 returns -1 otherwise). */
+int hqo_pack_i4(const int8_t* codes, int64_t count, uint8_t* out);
+/* The inverse: count codes from count / 2 bytes, nibble v read as v - 16 when
+ * v >= 8. */
+int hqo_unpack_i4(const uint8_t* packed, int64_t count, int8_t* codes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -516,3 +516,47 @@ def test_wh_epilogue_against_explicit_matrices(n_out):
     y, _ = oracle.epilogue_wh(acc, n_out, sx, sw, bb)
     ref = (sx[:, None] * acc * sw[None, :] + bb[None, :]) @ _block_h(N, n_out)
     assert np.allclose(y, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+# ---------------------------------------------------------------- packed codes
+# Two 3- or 4-bit codes per byte, element 2j in the low nibble of byte j and
+# element 2j+1 in the high nibble, each a 4-bit two's-complement value (the
+# storage reading for the 4-bit operands of the W4A4 GEMM in "Data-free 4-bit
+# quantization for diffusion transformers", which fixes no layout).
+
+def test_packed_codes_hand_worked_bytes():
+    # the int4 and int3 hand-worked quantizer examples above, packed by hand:
+    #   [7, -2 | -4, -1]: 0x7 + 16 * 0xE = 0xE7, 0xC + 16 * 0xF = 0xFC
+    #   [3, -1 | -2,  0]: 0x3 + 16 * 0xF = 0xF3, 0xE + 16 * 0x0 = 0x0E
+    assert oracle.pack_i4(np.array([[7, -2, -4, -1]])).tolist() == [[0xE7, 0xFC]]
+    assert oracle.pack_i4(np.array([[3, -1, -2, 0]])).tolist() == [[0xF3, 0x0E]]
+    assert oracle.unpack_i4(np.array([[0xE7, 0xFC]], np.uint8)).tolist() == [[7, -2, -4, -1]]
+
+
+def test_packed_codes_are_a_bijection_on_all_bytes():
+    every_byte = np.arange(256, dtype=np.uint8)
+    codes = oracle.unpack_i4(every_byte)
+    assert codes.min() == -8 and codes.max() == 7
+    assert np.array_equal(oracle.pack_i4(codes), every_byte)
+    pairs = np.array(list(itertools.product(range(-8, 8), repeat=2)), dtype=np.int8).reshape(-1)
+    assert np.array_equal(oracle.unpack_i4(oracle.pack_i4(pairs)), pairs)
+
+
+def test_packed_nibbles_are_arithmetic_shifts_of_the_signed_byte():
+    # independent reading of the layout: the byte as int8, shifted right
+    # arithmetically by 4, is the high code; shifted left by 4 first (a wrap
+    # in int8), the low code
+    every_byte = np.arange(256, dtype=np.uint8)
+    codes = oracle.unpack_i4(every_byte)
+    signed = every_byte.view(np.int8)
+    assert np.array_equal(codes[1::2], signed >> 4)
+    assert np.array_equal(codes[0::2], (every_byte << 4).astype(np.uint8).view(np.int8) >> 4)
+
+
+def test_packed_codes_reject_out_of_range_values():
+    with pytest.raises(ValueError):
+        oracle.pack_i4(np.array([8, 0], dtype=np.int8))
+    with pytest.raises(ValueError):
+        oracle.pack_i4(np.array([0, -9], dtype=np.int8))
+    with pytest.raises(ValueError):
+        oracle.pack_i4(np.array([1, 2, 3], dtype=np.int8))
