@@ -24,6 +24,7 @@ __all__ = [
     "HQError", "LayerDesc", "load_library", "library_path", "exported_symbols",
     "HQ_PER_TOKEN", "HQ_PER_TENSOR_DYNAMIC", "HQ_PER_TENSOR_STATIC",
     "HQ_CENTER_NONE", "HQ_CENTER_TOKEN_MEAN", "HQ_CENTER_TOKEN_MEAN_PRE", "HQ_CODES_I8",
+    "HQ_CODES_I4_PACKED",
     "HQ_FAULT_NONE", "HQ_FAULT_QUANT_WITHHOLD_ROW", "STATUS_NAMES",
     "hq_version", "hq_status_string", "hq_calib_act_absmax", "hq_prepare_weights",
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
@@ -37,7 +38,7 @@ _LIB_PATH = os.path.join(_PKG, "libhq.so")
 
 HQ_PER_TOKEN, HQ_PER_TENSOR_DYNAMIC, HQ_PER_TENSOR_STATIC = 0, 1, 2
 HQ_CENTER_NONE, HQ_CENTER_TOKEN_MEAN, HQ_CENTER_TOKEN_MEAN_PRE = 0, 1, 2
-HQ_CODES_I8 = 0
+HQ_CODES_I8, HQ_CODES_I4_PACKED = 0, 1
 HQ_FAULT_NONE, HQ_FAULT_QUANT_WITHHOLD_ROW = 0, 1
 HQ_GEMM_AUTO, HQ_GEMM_SINGLE_CTA, HQ_GEMM_CTA_PAIR = 0, 1, 2
 STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED",
@@ -295,7 +296,11 @@ class HadamardQuantLinear:
         if b is None:
             dev = self.w_codes.device
             per_row = self.desc.act_gran == HQ_PER_TOKEN
-            b = {"a_codes": torch.empty((T, self.desc.K), dtype=torch.int8, device=dev),
+            if self.desc.code_format == HQ_CODES_I4_PACKED:  # two codes per byte
+                codes = torch.empty((T, self.desc.K // 2), dtype=torch.uint8, device=dev)
+            else:
+                codes = torch.empty((T, self.desc.K), dtype=torch.int8, device=dev)
+            b = {"a_codes": codes,
                  "a_scale": torch.empty(T if per_row else 1, dtype=torch.float32, device=dev),
                  "a_mean": torch.empty(T, dtype=torch.float32, device=dev)}
             self._bufs[T] = b

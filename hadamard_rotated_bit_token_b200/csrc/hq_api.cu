@@ -19,7 +19,7 @@ __device__ unsigned int g_error_word = 0;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kVersion = 10200;  // 1.2.0: hq_forward_host
+constexpr int kVersion = 10300;  // 1.3.0: packed 3/4-bit activation codes
 constexpr int kMaxHostChunks = 64;  // row chunks of hq_forward_host
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -94,8 +94,17 @@ hq_status check_k_side(const hq_layer_desc* d) {
   if (d->K <= 0 || d->had_order <= 0) return HQ_ERR_INVALID_ARGUMENT;
   if (logn != 0 && (logn < 4 || logn > 10)) return HQ_ERR_UNSUPPORTED;
   if (d->K % d->had_order != 0 || d->K % 64 != 0 || d->K > 9216) return HQ_ERR_UNSUPPORTED;
-  if (d->code_format != HQ_CODES_I8) return HQ_ERR_UNSUPPORTED;
+  if (d->code_format != HQ_CODES_I8 && d->code_format != HQ_CODES_I4_PACKED)
+    return HQ_ERR_UNSUPPORTED;
+  // two codes per byte hold 3- and 4-bit activation codes only
+  if (d->code_format == HQ_CODES_I4_PACKED && d->a_bits != 3 && d->a_bits != 4)
+    return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
+}
+
+// Bytes per row of activation codes: K, or K / 2 when packed.
+int64_t code_row_bytes(const hq_layer_desc* d) {
+  return d->code_format == HQ_CODES_I4_PACKED ? d->K / 2 : d->K;
 }
 
 // The output side: out_order 0 or 1 is the double-Hadamard form; 16, 32 or
@@ -217,6 +226,19 @@ hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K
   return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
 }
 
+// Packed activation codes [T, K/2] bytes: box {64 bytes (one K block of 128
+// codes), 128 rows}, no swizzle (the GEMM widens the tile itself).
+hq_status encode_packed_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(K / 2)};
+  cuuint32_t box[2] = {64u, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
 hq_status encode_out_bf16(CUtensorMap* m, const void* base, int64_t rows, int N) {
   cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(N) * 2u};
@@ -244,7 +266,7 @@ struct GemmChoice {
 };
 
 GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int variant,
-                       int logo) {
+                       int logo, bool packed) {
   static const int cands[] = {256, 192, 128, 64};
   const int64_t mt = (T + 127) / 128;
   const int64_t kb = (K + 127) / 128;
@@ -262,8 +284,10 @@ GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int 
       best_bn = bn;
     }
   }
-  // the weight-only Hadamard epilogue runs in the single-CTA kernel only
-  if (variant == HQ_GEMM_SINGLE_CTA || pair_clusters <= 0 || logo > 0) return {false, best_bn};
+  // the weight-only Hadamard epilogue and packed codes run in the
+  // single-CTA kernel only
+  if (variant == HQ_GEMM_SINGLE_CTA || pair_clusters <= 0 || logo > 0 || packed)
+    return {false, best_bn};
   if (variant == HQ_GEMM_CTA_PAIR) return {true, 256};
   // automatic: the pair for long main loops (>= 20 K blocks) over N in whole
   // 256-column tiles, when it needs no more tile rounds than the best single
@@ -304,6 +328,11 @@ hq_status check_linear_args(const hq_layer_desc* desc, int64_t T, const int8_t* 
     return HQ_ERR_INVALID_ARGUMENT;
   if (desc->K % 16 != 0 || desc->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
   if (desc->a_bits < 2 || desc->a_bits > 8 || desc->w_bits < 2 || desc->w_bits > 8)
+    return HQ_ERR_UNSUPPORTED;
+  if (desc->code_format != HQ_CODES_I8 && desc->code_format != HQ_CODES_I4_PACKED)
+    return HQ_ERR_UNSUPPORTED;
+  // packed: codes of at most 4 bits, and rows of K / 2 bytes in whole 16-byte units
+  if (desc->code_format == HQ_CODES_I4_PACKED && (desc->a_bits > 4 || desc->K % 32 != 0))
     return HQ_ERR_UNSUPPORTED;
   if (desc->out_order < 0) return HQ_ERR_INVALID_ARGUMENT;
   if (desc->out_order > 1) {
@@ -449,6 +478,7 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   L.p.mean = a_mean;
   L.p.rowsum = nullptr;
   L.p.q = (1 << (desc->a_bits - 1)) - 1;
+  L.p.packed = desc->code_format == HQ_CODES_I4_PACKED ? 1 : 0;
   L.p.fault_withhold_row = g_fault == HQ_FAULT_QUANT_WITHHOLD_ROW ? 1 : 0;
   const int center = desc->centering;  // HQ_CENTER_* = the kernel's centering mode
   if (desc->act_gran == HQ_PER_TOKEN) return run_quant(dev, L, 0, center, st);
@@ -496,11 +526,13 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   // weight-only Hadamard form: output blocks of m = out_order columns
   const int m = desc->out_order > 1 ? desc->out_order : 1;
   const int logo = ilog2_exact(m);
+  const bool packed = desc->code_format == HQ_CODES_I4_PACKED;
   if (variant == HQ_GEMM_CTA_PAIR && dev->pair_clusters <= 0 && logo == 0) return HQ_ERR_UNSUPPORTED;
-  const GemmChoice gc = choose_gemm(T, N, K, dev->sm_count, dev->pair_clusters, variant, logo);
+  const GemmChoice gc =
+      choose_gemm(T, N, K, dev->sm_count, dev->pair_clusters, variant, logo, packed);
   const int bn = gc.pair ? 256 : gc.bn;
   CUtensorMap ta, tb, ty;
-  s = encode_kmajor_i8(&ta, a_codes, T, K, 128);
+  s = packed ? encode_packed_a(&ta, a_codes, T, K) : encode_kmajor_i8(&ta, a_codes, T, K, 128);
   if (s != HQ_OK) return s;
   s = encode_kmajor_i8(&tb, w_codes, N, K, gc.pair ? 128 : bn);
   if (s != HQ_OK) return s;
@@ -511,10 +543,15 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.a_scale = a_scale;
   p.a_scale_per_row = desc->act_gran == HQ_PER_TOKEN ? 1 : 0;
   {
-    // |acc| <= 2^(a_bits-1) * 2^(w_bits-1) * K for codes within their declared widths
-    const double bound = std::ldexp(1.0, desc->a_bits - 1) * std::ldexp(1.0, desc->w_bits - 1) * K;
+    // |acc| <= 2^(a_bits-1) * 2^(w_bits-1) * K for codes within their declared
+    // widths, 16 times that for packed codes (widened to 16 * code)
+    const double bound = std::ldexp(1.0, desc->a_bits - 1) * std::ldexp(1.0, desc->w_bits - 1) *
+                         K * (packed ? 16.0 : 1.0);
     p.small_acc = bound < 4194304.0 ? 1 : 0;
   }
+  p.acc_unit = packed ? 0.0625f : 1.0f;
+  p.acc_shift = packed ? 4 : 0;
+  p.a_packed = packed ? reinterpret_cast<const uint8_t*>(a_codes) : nullptr;
   p.a_mean = a_mean;
   p.w_scale = w_scale;
   p.colsum = colsum;
@@ -539,7 +576,7 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.num_n_tiles = (N + bn - 1) / bn;
   const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
   const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
-  return from_cuda(launch_gemm(bn, logo, &ta, &tb, &ty, p, grid, st));
+  return from_cuda(launch_gemm(bn, logo, packed, &ta, &tb, &ty, p, grid, st));
 }
 
 hq_status hq_forward_host(const hq_layer_desc* desc, const uint16_t* X_host, int64_t T,
@@ -575,6 +612,7 @@ hq_status hq_forward_host(const hq_layer_desc* desc, const uint16_t* X_host, int
     }
   }
   const int K = desc->K, N = desc->N;
+  const int64_t cb = code_row_bytes(desc);  // bytes per row of a_codes
   const bool per_row = desc->act_gran == HQ_PER_TOKEN;
   // a tensor-wide dynamic scale needs every row before any code: one chunk
   if (desc->act_gran == HQ_PER_TENSOR_DYNAMIC) chunks = 1;
@@ -625,11 +663,11 @@ hq_status hq_forward_host(const hq_layer_desc* desc, const uint16_t* X_host, int
     const int64_t lo = c * step, rows = (T - lo) < step ? (T - lo) : step;
     if (cudaStreamWaitEvent(st, ev_in[c], 0) != cudaSuccess) return fail(HQ_ERR_CUDA);
     const bool whole = nc == 1;
-    s = hq_quantize_act(desc, X_dev + lo * K, rows, sigma_inv, a_codes + lo * K,
+    s = hq_quantize_act(desc, X_dev + lo * K, rows, sigma_inv, a_codes + lo * cb,
                         (per_row && !whole) ? a_scale + lo : a_scale,
                         a_mean ? a_mean + lo : nullptr, workspace, workspace_bytes, stream);
     if (s == HQ_OK)
-      s = hq_linear(desc, rows, a_codes + lo * K, (per_row && !whole) ? a_scale + lo : a_scale,
+      s = hq_linear(desc, rows, a_codes + lo * cb, (per_row && !whole) ? a_scale + lo : a_scale,
                     mean_in ? mean_in + lo : nullptr, w_codes, w_scale, colsum, bias_f32,
                     Y_dev + lo * N, nullptr, stream);
     if (s != HQ_OK) return fail(s);

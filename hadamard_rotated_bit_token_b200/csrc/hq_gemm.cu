@@ -25,11 +25,24 @@
 //               lets a TMA tensor store write the 32 x 32 box to Y (clipped at
 //               the tensor's edges).
 //
-// gemm_i8_kernel<BN, LOGO>: one CTA per 128 x BN output tile (BN 64..256).
+// gemm_i8_kernel<BN, LOGO, PK>: one CTA per 128 x BN output tile (BN 64..256).
 //   LOGO > 0 selects the weight-only Hadamard epilogue (HaTQ Sec. IV-B
 //   Eq. (17)): Y = (s_x s_w acc) H_out + b, the fast Walsh-Hadamard transform
 //   over each block of 2^LOGO output columns done in registers after the
 //   dequantization (no mean term: that form has no centering).
+//   PK: A holds two 4-bit codes per byte.  Two more warps (warps 10 and
+//   11) take the place of A's tensor loads: they read each stage's 128 x
+//   64-byte packed tile from global memory straight into registers, three K
+//   blocks ahead, widen it into the 128-byte-swizzled int8 tile the MMA reads
+//   (each nibble moved to the high half of its byte: 16 * code, sign
+//   included) and release the stage to the MMA issuer on a third barrier.
+//   The accumulator is then 16 times the code products' sum, exactly; the
+//   epilogue's row scale carries the factor 1/16.  No tensor-core kind
+//   multiplies 4-bit integers on sm_100a, so the widening is the price of
+//   reading half the activation bytes.  The packed tile does not pass
+//   through shared memory: the main loop is bound by shared-memory traffic
+//   (tensor loads in, MMA operand reads out), and a staged packed tile would
+//   add its own write and read to every stage.
 // gemm_i8_pair_kernel: a cluster of two CTAs per 256 x 256 output tile with
 //   the CTA-pair MMA (cta_group::2, M = 256): each CTA loads 128 rows of A and
 //   128 rows of B into its own shared memory, so one SM moves half the B
@@ -55,6 +68,7 @@ constexpr int BM = 128;
 constexpr int BK = 128;  // K bytes per stage: one 128-byte swizzle row
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kConvWarps = 2;  // packed-A converters of the single-CTA kernel
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kStageBox = 2048;           // one 32 x 32 bf16 output box
 constexpr float kAccMagic = 12582912.0f;  // 1.5 * 2^23
@@ -114,6 +128,18 @@ __device__ __forceinline__ void param_ring_load(const GemmParams& p, float* slot
   if (bi) bulk_load(slot + 2 * W, p.bias + n0, nb, bar);
 }
 
+// ------------------------------------------------------- packed A operand
+// One word of eight 4-bit two's-complement codes (element 2j in the low
+// nibble of byte j) -> two words of eight int8 values 16 * code, in element
+// order: each nibble moved to the high half of its own byte is already the
+// sign-extended code times 16, so no sign extension is needed.
+__device__ __forceinline__ void widen_i4x8(uint32_t v, uint32_t& lo, uint32_t& hi) {
+  const uint32_t ev = (v << 4) & 0xF0F0F0F0u;  // elements 0, 2, 4, 6
+  const uint32_t od = v & 0xF0F0F0F0u;         // elements 1, 3, 5, 7
+  lo = __byte_perm(ev, od, 0x5140);
+  hi = __byte_perm(ev, od, 0x7362);
+}
+
 // ------------------------------------------------------------- epilogue
 // Per-warp state of the epilogue for one output tile.
 struct EpiTile {
@@ -130,7 +156,9 @@ __device__ __forceinline__ void load_row_params(const GemmParams& p, int64_t row
   sx = 0.0f;
   mt = 0.0f;
   if (row < p.T) {
-    sx = p.a_scale_per_row ? p.a_scale[row] : p.a_scale[0];
+    // packed A enters the MMA as 16 * code, so the accumulator is 16 times
+    // the code products' sum; times acc_unit = 1/16 (exact) undoes it
+    sx = (p.a_scale_per_row ? p.a_scale[row] : p.a_scale[0]) * p.acc_unit;
     mt = p.a_mean ? p.a_mean[row] : 0.0f;
   }
 }
@@ -144,8 +172,10 @@ __device__ __forceinline__ void epi_acc_debug(const GemmParams& p, const uint32_
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       if (col0 + 4 * g < p.N) {
-        *reinterpret_cast<uint4*>(arow + col0 + 4 * g) =
-            make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+        const int sh = p.acc_shift;  // exact: a packed A's accumulator is a multiple of 16
+        *reinterpret_cast<int4*>(arow + col0 + 4 * g) =
+            make_int4(int(r[4 * g]) >> sh, int(r[4 * g + 1]) >> sh, int(r[4 * g + 2]) >> sh,
+                      int(r[4 * g + 3]) >> sh);
       }
     }
   }
@@ -356,11 +386,15 @@ __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap*
 }  // namespace
 
 // ------------------------------------------------------- single-CTA kernel
-template <int BN>
+template <int BN, bool PK>
 struct GemmCfg {
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  // bytes the tensor loads bring per stage (packed A arrives through the converters)
+  static constexpr uint32_t STAGE_TX = uint32_t((PK ? 0 : A_BYTES) + B_BYTES);
+  static constexpr int THREADS = kGemmThreads + (PK ? 32 * kConvWarps : 0);
+  static constexpr int NBAR_STAGE = PK ? 3 : 2;  // full, empty (, converted)
   static constexpr int HC = BN / 2;  // columns per epilogue warp
   static constexpr int NBOX = 1;  // output staging boxes per epilogue warp
   static constexpr int EPI_STAGE_BYTES = NBOX * kStageBox;
@@ -368,22 +402,23 @@ struct GemmCfg {
   static constexpr int CTL_BYTES = 256;
   static constexpr int FIXED = kEpiWarps * EPI_STAGE_BYTES + RING_BYTES + CTL_BYTES + 1024;
   static constexpr int STAGES_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int STAGE_CAP = PK ? 7 : 8;  // barrier block size
+  static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
   static constexpr int TMEM_COLS = tmem_cols_for(2 * BN);
   static constexpr uint32_t IDESC = i8_idesc(BM, BN);
   static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + FIXED;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "two 32-column-aligned halves");
   static_assert(B_BYTES % 1024 == 0, "stage bases must stay 1024-byte aligned");
   static_assert(STAGES >= 2, "shared memory budget");
-  static_assert(16 * STAGES + 80 <= CTL_BYTES, "barrier block");
+  static_assert(8 * NBAR_STAGE * STAGES + 80 <= CTL_BYTES, "barrier block");
   static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
 };
 
-template <int BN, int LOGO>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int BN, int LOGO, bool PK>
+__global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, PK>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -393,7 +428,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float* ring = reinterpret_cast<float*>(epi_stage + kEpiWarps * C::EPI_STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ring) + C::RING_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* tfull = empty + C::STAGES;   // [2] accumulator complete
+  uint64_t* conv = empty + C::STAGES;    // (PK) stage s's A widened to int8
+  uint64_t* tfull = conv + (PK ? C::STAGES : 0);  // [2] accumulator complete
   uint64_t* tempty = tfull + 2;          // [2] accumulator drained by the epilogue
   uint64_t* pfull = tempty + 2;          // [2] parameter slot loaded
   uint64_t* pempty = pfull + 2;          // [2] parameter slot read by the epilogue
@@ -405,12 +441,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   const WaitCtl wc{p.err, p.wait_ns};
 
-  param_ring_zero<BN>(ring, threadIdx.x, kGemmThreads);
+  param_ring_zero<BN>(ring, threadIdx.x, C::THREADS);
   fence_proxy_async_smem();  // the zeros precede the ring's bulk copies
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      if (PK) mbar_init(&conv[s], kConvWarps);  // one arrival per converter warp
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -421,7 +458,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
-    prefetch_tmap(&tmA);
+    if (!PK) prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmY);
   }
@@ -461,8 +498,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + size_t(stage) * C::A_BYTES, &tmA, kb * BK, m_idx * BM, &full[stage]);
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
+          if constexpr (!PK)
+            tma_load_2d(sA + size_t(stage) * C::A_BYTES, &tmA, kb * BK, m_idx * BM, &full[stage]);
           tma_load_2d(sB + size_t(stage) * C::B_BYTES, &tmB, kb * BK, n_idx * BN, &full[stage]);
           ++issued;
           if (++stage == C::STAGES) {
@@ -505,7 +543,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
-          if (*abort_flag || !mbar_wait(&full[stage], phase, wc)) {
+          // B landed (full) and, for packed A, the converters wrote A (conv)
+          if (*abort_flag || !mbar_wait(&full[stage], phase, wc) ||
+              (PK && !mbar_wait(&conv[stage], phase, wc))) {
             *abort_flag = 1;
             ok = false;
             break;
@@ -532,7 +572,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mma_commit(drain);
       (void)mbar_wait(drain, 0, wc);
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ----------------------------------------------------------- epilogue
     const int ew = warp - 2;         // 0 .. 7
     const int quarter = warp & 3;    // TMEM lanes [32*quarter, 32*quarter + 32)
@@ -582,6 +622,85 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
     __syncwarp();
+  } else if constexpr (PK) {
+    // ------------------------------------------------- packed-A converters
+    // Stage s's A tile: packed rows [128 m, 128 m + 128) x bytes [64 kb,
+    // 64 kb + 64) of a_packed -> the int8 tile the MMA reads (128 rows x 128
+    // bytes, 128-byte swizzle: 16-byte chunk j of row r at chunk j ^ (r & 7)
+    // of its row, 8-row atoms of 1024 bytes).  Thread ct (0..63) owns packed
+    // chunk ct & 3 of rows ct / 4 + 16 i, i = 0..7: a warp's load covers 8
+    // whole 64-byte row segments, and its stores hit 8 rows' distinct
+    // swizzled chunks (no bank conflicts).  Rows past T and bytes past K / 2
+    // read as zero codes.  The loads of the next D stages are in flight
+    // (registers) while a stage is widened.
+    constexpr int D = 3;
+    const int ct = (warp - 2 - kEpiWarps) * 32 + lane;
+    const int rsub = ct >> 2;          // row within each group of 16
+    const int cc = ct & 3;             // 16-byte chunk of the 64-byte row segment
+    const int swz = rsub & 7;          // r & 7 for every r = rsub + 16 i
+    const int64_t prow = p.K / 2;      // packed bytes per row
+    const int my_tiles =
+        int(blockIdx.x) < num_tiles ? (num_tiles - int(blockIdx.x) + int(gridDim.x) - 1) /
+                                          int(gridDim.x)
+                                    : 0;
+    const int total = my_tiles * KB;   // stages this CTA's main loops consume
+    uint4 pre[D][8];
+    auto fetch = [&](int j, uint4 (&dst)[8]) {
+      const int t = j / KB;
+      const int kb = j - t * KB;
+      const int tile = int(blockIdx.x) + t * int(gridDim.x);
+      const int64_t row0 = int64_t(tile % p.num_m_tiles) * BM + rsub;
+      const int64_t col = int64_t(kb) * (BK / 2) + cc * 16;
+      const bool col_ok = col < prow;  // K / 2 is a multiple of 16: whole chunks
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t row = row0 + 16 * i;
+        dst[i] = (col_ok && row < p.T)
+                     ? __ldg(reinterpret_cast<const uint4*>(p.a_packed + row * prow + col))
+                     : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+      if (d < total) fetch(d, pre[d]);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int j0 = 0; j0 < total && ok; j0 += D) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        const int j = j0 + d;
+        if (j >= total) break;
+        // the MMAs that read stage s's previous A have completed
+        const bool got = !(*abort_flag) && mbar_wait(&empty[stage], phase ^ 1u, wc);
+        if (!__all_sync(0xffffffffu, got)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* dst = sA + size_t(stage) * C::A_BYTES + (rsub >> 3) * 1024 + swz * 128;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint4 o0, o1;
+          widen_i4x8(pre[d][i].x, o0.x, o0.y);
+          widen_i4x8(pre[d][i].y, o0.z, o0.w);
+          widen_i4x8(pre[d][i].z, o1.x, o1.y);
+          widen_i4x8(pre[d][i].w, o1.z, o1.w);
+          // row rsub + 16 i: two 8-row atoms further per i
+          uint8_t* row = dst + i * 2048;
+          *reinterpret_cast<uint4*>(row + (((2 * cc) ^ swz) << 4)) = o0;
+          *reinterpret_cast<uint4*>(row + (((2 * cc + 1) ^ swz) << 4)) = o1;
+        }
+        fence_proxy_async_smem();  // the tile is read by the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[stage]);
+        if (j + D < total) fetch(j + D, pre[d]);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
   }
 
   tc_fence_before();
@@ -868,47 +987,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 }
 
 // ------------------------------------------------------------------ launch
-template <int BN, int LOGO>
+template <int BN, int LOGO, bool PK>
 static cudaError_t launch_bn(const void* tmap_a, const void* tmap_b, const void* tmap_y,
                              const GemmParams& p, int grid, cudaStream_t st) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, PK>;
   static bool configured = false;  // attribute is per function, device-agnostic
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<BN, LOGO>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<BN, LOGO, PK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  gemm_i8_kernel<BN, LOGO><<<grid, kGemmThreads, C::SMEM, st>>>(
+  gemm_i8_kernel<BN, LOGO, PK><<<grid, C::THREADS, C::SMEM, st>>>(
       *reinterpret_cast<const CUtensorMap*>(tmap_a), *reinterpret_cast<const CUtensorMap*>(tmap_b),
       *reinterpret_cast<const CUtensorMap*>(tmap_y), p);
   return cudaGetLastError();
 }
 
-template <int LOGO>
+template <int LOGO, bool PK>
 static cudaError_t launch_logo(int bn, const void* tmap_a, const void* tmap_b,
                                const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
   switch (bn) {
-    case 128: return launch_bn<128, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 256: return launch_bn<256, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 128: return launch_bn<128, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 256: return launch_bn<256, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
     default:
       if constexpr (LOGO <= 5) {
-        if (bn == 64) return launch_bn<64, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
-        if (bn == 192) return launch_bn<192, LOGO>(tmap_a, tmap_b, tmap_y, p, grid, st);
+        if (bn == 64) return launch_bn<64, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
+        if (bn == 192) return launch_bn<192, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
       }
       return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_gemm(int bn, int logo, const void* tmap_a, const void* tmap_b,
-                        const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
+template <bool PK>
+static cudaError_t launch_pk(int bn, int logo, const void* tmap_a, const void* tmap_b,
+                             const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
   switch (logo) {
-    case 0: return launch_logo<0>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 4: return launch_logo<4>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 5: return launch_logo<5>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 6: return launch_logo<6>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 0: return launch_logo<0, PK>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 4: return launch_logo<4, PK>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 5: return launch_logo<5, PK>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 6: return launch_logo<6, PK>(bn, tmap_a, tmap_b, tmap_y, p, grid, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_gemm(int bn, int logo, bool packed_a, const void* tmap_a, const void* tmap_b,
+                        const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
+  return packed_a ? launch_pk<true>(bn, logo, tmap_a, tmap_b, tmap_y, p, grid, st)
+                  : launch_pk<false>(bn, logo, tmap_a, tmap_b, tmap_y, p, grid, st);
 }
 
 static cudaError_t configure_pair() {
@@ -948,19 +1074,24 @@ cudaError_t launch_gemm_pair(const void* tmap_a, const void* tmap_b, const void*
   return cudaGetLastError();
 }
 
-size_t gemm_smem_bytes(int bn) {
+template <bool PK>
+static size_t smem_of(int bn) {
   switch (bn) {
-    case 64: return GemmCfg<64>::SMEM;
-    case 128: return GemmCfg<128>::SMEM;
-    case 192: return GemmCfg<192>::SMEM;
-    case 256: return GemmCfg<256>::SMEM;
+    case 64: return GemmCfg<64, PK>::SMEM;
+    case 128: return GemmCfg<128, PK>::SMEM;
+    case 192: return GemmCfg<192, PK>::SMEM;
+    case 256: return GemmCfg<256, PK>::SMEM;
     default: return 0;
   }
+}
+
+size_t gemm_smem_bytes(int bn, bool packed_a) {
+  return packed_a ? smem_of<true>(bn) : smem_of<false>(bn);
 }
 
 size_t gemm_pair_smem_bytes() { return PairCfg::SMEM; }
 int gemm_pair_stages() { return PairCfg::STAGES; }
 
-int gemm_threads() { return kGemmThreads; }
+int gemm_threads(bool packed_a) { return kGemmThreads + (packed_a ? 32 * kConvWarps : 0); }
 
 }  // namespace hq

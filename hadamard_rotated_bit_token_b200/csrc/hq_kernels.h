@@ -11,7 +11,8 @@ struct QuantParams {
   const uint16_t* X;          // [T,K] bf16 rows to transform
   const float* mult;          // [K] channel multiplier (sigma^-1 or sigma), or null
   int invert_mult;            // 1: use 1/mult[k] as the multiplier
-  int8_t* codes;              // [T,K] int8 codes
+  int8_t* codes;              // [T,K] int8 codes, or [T,K/2] bytes when packed
+  int packed;                 // 1: two codes per byte (element 2j in the low nibble)
   float* scale;               // [T] per-row scales, or [1] for per-tensor modes
   float* mean;                // [T] per-row mean of the rotated row (real units), or null
   float* rowsum;              // [T] per-row correction sum (see rowsum_pre), or null
@@ -57,6 +58,9 @@ struct GemmParams {
   int num_m_tiles;
   int num_n_tiles;
   float inv_sqrt_out;         // 1/sqrt(m) of the output-side transform (weight-only form)
+  float acc_unit;             // accumulator units per code product: 1, or 1/16 when A is packed
+  int acc_shift;              // acc_debug = raw accumulator >> acc_shift (0, or 4 when packed)
+  const uint8_t* a_packed;    // packed A [T, K/2] bytes (packed kernels read it directly)
   unsigned int* err;          // device error word
   unsigned long long wait_ns; // bounded-wait limit
 };
@@ -66,11 +70,14 @@ struct GemmParams {
 // bn 128 or 256).  tmap_a / tmap_b / tmap_y point to host CUtensorMap
 // objects (copied into the launch): A [T,K] and B [N,K] int8 with box
 // {128, 128 | bn} and 128-byte swizzle; Y [T,N] bf16 with box {32, 32} and
-// 64-byte swizzle.
-cudaError_t launch_gemm(int bn, int logo, const void* tmap_a, const void* tmap_b,
+// 64-byte swizzle.  packed_a: A holds two 4-bit codes per byte, [T,K/2]
+// bytes at GemmParams.a_packed (read directly; tmap_a is not used); the
+// kernel widens each tile to int8 (16 * code) in shared memory, so the
+// caller passes acc_unit = 1/16 and acc_shift = 4.
+cudaError_t launch_gemm(int bn, int logo, bool packed_a, const void* tmap_a, const void* tmap_b,
                         const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st);
-size_t gemm_smem_bytes(int bn);
-int gemm_threads();
+size_t gemm_smem_bytes(int bn, bool packed_a);
+int gemm_threads(bool packed_a);
 
 // The CTA-pair GEMM: clusters of two CTAs, each cluster computing 256 x 256
 // output tiles (GemmParams.num_m_tiles / num_n_tiles count pair tiles).

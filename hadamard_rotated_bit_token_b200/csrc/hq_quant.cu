@@ -40,7 +40,9 @@
 //            the segment that completes the row (a per-row arrival counter)
 //            computes the row's mean, scale and reciprocal once, publishes
 //            them and releases the row's barrier;
-//   quantize codes packed 4 per word and stored.
+//   quantize codes packed 4 per word and stored, one per byte, or two per
+//            byte (4-bit two's-complement nibbles, element 2j in the low
+//            nibble) when the caller asks for packed codes.
 // No CTA-wide barrier in the loop: warps wait only for the rows they hold.
 // With n = 1 (no rotation) the transform is skipped and the codes are formed
 // by a correctly rounded division (see the quantize step).
@@ -530,6 +532,27 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
       }
       words[g] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
                              0x5410);
+    }
+    if (p.packed) {
+      // two codes per byte, element 2j of the row in the low nibble of byte
+      // j: t keeps (c0 | c1 << 4) in byte 0 and (c2 | c3 << 4) in byte 2 of
+      // each word of four codes
+      uint32_t t[8];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) t[g] = (words[g] & 0x0F0F0F0Fu) | ((words[g] >> 4) & 0xF0F0F0F0u);
+      uint8_t* prow = reinterpret_cast<uint8_t*>(p.codes) + row * (K / 2);
+      if constexpr (!XPOSE) {
+        *reinterpret_cast<uint4*>(prow + slice * 16) =
+            make_uint4(__byte_perm(t[0], t[1], 0x6420), __byte_perm(t[2], t[3], 0x6420),
+                       __byte_perm(t[4], t[5], 0x6420), __byte_perm(t[6], t[7], 0x6420));
+      } else {
+        static_assert(GS == 4, "four codes (two bytes) per register group");
+        uint8_t* base = prow + (blk * N + GS * tl + (32 * G) * (member >> LX)) / 2;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          *reinterpret_cast<uint16_t*>(base + 16 * g) = uint16_t(__byte_perm(t[g], 0u, 0x0020));
+      }
+      continue;
     }
     int8_t* crow = p.codes + row * K;
     if (!XPOSE) {

@@ -42,7 +42,8 @@
  * rotation along K); K a multiple of had_order and of 64, K <= 9216; N a
  * multiple of 16 (and of out_order in the weight-only form, out_order in
  * {16, 32, 64}); T >= 0 (T = 0 is a no-op); a_bits in {3, 4, 8}, w_bits in
- * {4, 8} (codes in an int8 container, one code per byte).
+ * {4, 8} (codes in an int8 container, one code per byte; 3- and 4-bit
+ * activation codes optionally two per byte, hq_layer_desc.code_format).
  */
 #ifndef HQ_H
 #define HQ_H
@@ -69,7 +70,7 @@ typedef enum hq_status {
 
 enum { HQ_PER_TOKEN = 0, HQ_PER_TENSOR_DYNAMIC = 1, HQ_PER_TENSOR_STATIC = 2 };
 enum { HQ_CENTER_NONE = 0, HQ_CENTER_TOKEN_MEAN = 1, HQ_CENTER_TOKEN_MEAN_PRE = 2 };
-enum { HQ_CODES_I8 = 0 };
+enum { HQ_CODES_I8 = 0, HQ_CODES_I4_PACKED = 1 };
 
 /* Layer description, host memory, passed by const pointer.
  *   K, N        input / output channels.
@@ -93,7 +94,14 @@ enum { HQ_CODES_I8 = 0 };
  *               changes (by -sqrt(n) mu_t); the layer's correction becomes
  *               mu_t * sum_k sigma_k W[n,k].
  *               HQ_CENTER_NONE: mu = 0.
- *   code_format HQ_CODES_I8 (one signed code per byte).
+ *   code_format HQ_CODES_I8: one signed activation code per byte, a_codes
+ *               [T,K] int8.
+ *               HQ_CODES_I4_PACKED (a_bits 3 or 4): two activation codes per
+ *               byte, a_codes [T,K/2] bytes: element 2j of a row in the low
+ *               nibble of byte j, element 2j+1 in the high nibble, each a
+ *               4-bit two's-complement value.  hq_quantize_act writes this
+ *               form and hq_linear reads it (the GEMM widens each tile to
+ *               int8 in shared memory).  Weight codes stay one per byte.
  *   out_order   0 or 1: the double-Hadamard form above (no output-side
  *               transform).  16, 32 or 64: the weight-only Hadamard form
  *               (HaTQ Sec. IV-B, Eq. (15)-(17)): the weights are rotated
@@ -165,7 +173,8 @@ size_t hq_quantize_act_workspace_bytes(const hq_layer_desc* desc, int64_t T);
  *   HQ_CENTER_NONE:           m_t = 0, V = Z;
  *   s = max|V| / q_a per token (or per tensor);  codes = clamp(rne(V/s), +-q_a).
  * Inputs:  X bf16 [T,K]; sigma_inv fp32 [K] or NULL (sigma = 1).
- * Outputs: a_codes int8 [T,K];
+ * Outputs: a_codes int8 [T,K], or [T,K/2] bytes of two codes each for
+ *            HQ_CODES_I4_PACKED;
  *          a_scale fp32 [T] (HQ_PER_TOKEN) or [1] (per tensor; for
  *            HQ_PER_TENSOR_STATIC it is an INPUT holding s);
  *          a_mean fp32 [T] or NULL: m_t, in the units hq_linear multiplies
@@ -185,12 +194,16 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X,
  *   Y[t,n]   = bf16_rne( s_x[t] * w_scale[n] * acc[t,n]
  *                        + bias_f32[n] + a_mean[t] * colsum[n] )
  * on 5th-generation tensor cores (tcgen05 kind::i8, accumulator in TMEM).
- * Inputs:  a_codes int8 [T,K], a_scale fp32 [T] or [1] (per tensor, selected
+ * Inputs:  a_codes int8 [T,K] (or [T,K/2] packed bytes, HQ_CODES_I4_PACKED:
+ *          K a multiple of 32, a_bits <= 4; such A tiles enter the tensor
+ *          cores as 16 * code and the accumulator is scaled back by 1/16,
+ *          exactly), a_scale fp32 [T] or [1] (per tensor, selected
  *          by desc->act_gran), a_mean fp32 [T] or NULL (then mu = 0),
  *          w_codes int8 [N,K], w_scale fp32 [N], colsum fp32 [N] (may be NULL
  *          when a_mean is NULL), bias_f32 fp32 [N] or NULL (b = 0).
- * Outputs: Y bf16 [T,N]; acc_debug int32 [T,N] or NULL (raw accumulators, for
- *          bit-exact checks; costs an extra 4 bytes per output).
+ * Outputs: Y bf16 [T,N]; acc_debug int32 [T,N] or NULL (the accumulators
+ *          sum_k a_codes * w_codes, for bit-exact checks; costs an extra 4
+ *          bytes per output).
  * Weight-only Hadamard form (desc->out_order = m > 1; a_mean and colsum
  * must be NULL): the accumulator is in the output Hadamard basis and the
  * epilogue restores the original basis (HaTQ Eq. (17), supplement Eq. (41)):

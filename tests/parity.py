@@ -63,3 +63,24 @@ def rel_frob(gpu_bits, ref_bits):
     g = synth.bf16_bits_to_f32(gpu_bits).astype(np.float64)
     r = synth.bf16_bits_to_f32(ref_bits).astype(np.float64)
     return float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300))
+
+
+def check_bf16_outputs(gpu_bits, y64, mag, what="Y"):
+    """GPU bf16 outputs against the exact fp64 values y64 of the same epilogue
+    inputs.  The epilogue forms fma(acc, fl(s_x s_w), fma(m, c, b)) in fp32:
+    three roundings of relative size 2^-24 on terms no larger than
+    mag = |acc s_x s_w| + |m c| + |b|, so its fp32 value v lies within
+    tol = 4 * 2^-24 * mag of y64, and since rounding to bf16 is monotone the
+    output bf16_rne(v) lies between bf16_rne(y64 - tol) and bf16_rne(y64 + tol).
+    Outside a tol-wide neighbourhood of a bf16 rounding midpoint that interval
+    holds one value, bf16_rne(y64), so the check is exact there."""
+    import oracle
+    import synth
+    gpu = synth.bf16_bits_to_f32(np.asarray(gpu_bits, dtype=np.uint16)).astype(np.float64)
+    tol = 4.0 * 2.0 ** -24 * np.asarray(mag, dtype=np.float64)
+    lo = synth.bf16_bits_to_f32(oracle.f64_to_bf16(y64 - tol)).astype(np.float64)
+    hi = synth.bf16_bits_to_f32(oracle.f64_to_bf16(y64 + tol)).astype(np.float64)
+    ok = (gpu >= lo) & (gpu <= hi)
+    assert np.all(ok), (f"{what}: {int((~ok).sum())} outputs outside the fp32 epilogue's "
+                        f"rounding interval")
+    return int((gpu != synth.bf16_bits_to_f32(oracle.f64_to_bf16(y64))).sum())

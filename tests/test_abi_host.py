@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(hq):
 
 
 def test_version_and_status_strings(hq):
-    assert hq.hq_version() == 10200
+    assert hq.hq_version() == 10300
     for code, name in hq.STATUS_NAMES.items():
         assert hq.hq_status_string(code) == name
     assert hq.hq_status_string(99) == "HQ_ERR_UNKNOWN"
@@ -66,7 +66,12 @@ def test_quantize_validation(hq):
     assert _call_quant(hq, D(1024, 16, 1024, w_bits=3)) == 2
     assert _call_quant(hq, D(1024, 16, 1024, act_gran=7)) == 1
     assert _call_quant(hq, D(1024, 16, 1024, centering=3)) == 1
-    assert _call_quant(hq, D(1024, 16, 1024, code_format=1)) == 2
+    # packed codes: 3- and 4-bit activations only; other formats unknown
+    assert _call_quant(hq, D(1024, 16, 1024, code_format=1), T=0) == 0
+    assert _call_quant(hq, D(1024, 16, 1024, a_bits=3, code_format=1), T=0) == 0
+    assert _call_quant(hq, D(1024, 16, 1024, a_bits=8, code_format=1)) == 2
+    assert _call_quant(hq, D(1024, 16, 1024, code_format=2)) == 2
+    assert _call_quant(hq, D(1024, 16, 1024, code_format=-1)) == 2
     assert _call_quant(hq, D(1024, 16, 1024), X=FAKE + 2) == 3   # misaligned
     assert _call_quant(hq, D(1024, 16, 1024), codes=FAKE + 8) == 3
     # per-tensor dynamic needs its workspace
@@ -119,6 +124,11 @@ def test_linear_validation(hq):
     assert call(D(1024, 80, 1, **wh)) == 2                     # N not a multiple of out_order
     assert call(D(1024, 128, 1, centering=0, out_order=48)) == 2
     assert call(D(1024, 128, 1, centering=0, out_order=-2)) == 1
+    # packed activation codes: at most 4 bits, K / 2 bytes a multiple of 16
+    assert call(D(1024, 16, 1024, code_format=1), T=0) == 0
+    assert call(D(1024, 16, 1024, a_bits=8, code_format=1)) == 2
+    assert call(D(1040, 16, 16, code_format=1)) == 2
+    assert call(D(1024, 16, 1024, code_format=5)) == 2
 
 
 def test_forward_host_validation(hq):
