@@ -227,14 +227,15 @@ hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K
 }
 
 // Packed activation codes [T, K/2] bytes: box {64 bytes (one K block of 128
-// codes), 128 rows}, no swizzle (the GEMM widens the tile itself).
+// codes), 128 rows}, 64-byte swizzle (the GEMM's converters read one row per
+// lane without bank conflicts and widen it themselves).
 hq_status encode_packed_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
   cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(K / 2)};
   cuuint32_t box[2] = {64u, 128u};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
 }
@@ -275,6 +276,8 @@ GemmChoice choose_gemm(int64_t T, int N, int K, int sms, int pair_clusters, int 
   for (int bn : cands) {
     // 64-column output blocks of the weight-only form need 64 columns per epilogue warp
     if (logo == 6 && bn % 128 != 0) continue;
+    // packed codes keep A's stages in tensor memory beside the accumulators
+    if (packed && bn > 192) continue;
     const int64_t tiles = mt * ((N + bn - 1) / bn);
     const int64_t rounds = (tiles + sms - 1) / sms;
     const double tile = double(kb) * 4.0 * (126.0 + bn / 16.0) * 1.15 + 2000.0 * (bn / 64);
@@ -551,7 +554,6 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   }
   p.acc_unit = packed ? 0.0625f : 1.0f;
   p.acc_shift = packed ? 4 : 0;
-  p.a_packed = packed ? reinterpret_cast<const uint8_t*>(a_codes) : nullptr;
   p.a_mean = a_mean;
   p.w_scale = w_scale;
   p.colsum = colsum;

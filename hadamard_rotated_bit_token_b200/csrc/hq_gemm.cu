@@ -30,19 +30,20 @@
 //   Eq. (17)): Y = (s_x s_w acc) H_out + b, the fast Walsh-Hadamard transform
 //   over each block of 2^LOGO output columns done in registers after the
 //   dequantization (no mean term: that form has no centering).
-//   PK: A holds two 4-bit codes per byte.  Two more warps (warps 10 and
-//   11) take the place of A's tensor loads: they read each stage's 128 x
-//   64-byte packed tile from global memory straight into registers, three K
-//   blocks ahead, widen it into the 128-byte-swizzled int8 tile the MMA reads
-//   (each nibble moved to the high half of its byte: 16 * code, sign
-//   included) and release the stage to the MMA issuer on a third barrier.
-//   The accumulator is then 16 times the code products' sum, exactly; the
-//   epilogue's row scale carries the factor 1/16.  No tensor-core kind
-//   multiplies 4-bit integers on sm_100a, so the widening is the price of
-//   reading half the activation bytes.  The packed tile does not pass
-//   through shared memory: the main loop is bound by shared-memory traffic
-//   (tensor loads in, MMA operand reads out), and a staged packed tile would
-//   add its own write and read to every stage.
+//   PK: A holds two 4-bit codes per byte.  TMA loads each stage's 128 x
+//   64-byte packed tile (64-byte swizzle) next to B; four more warps (warps
+//   10..13, one per 32-lane quarter of tensor memory) each read their rows'
+//   packed bytes, widen them to int8 (each nibble moved to the high half of
+//   its byte: 16 * code, sign included) and store them with tcgen05.st into
+//   tensor memory, where the MMA takes its A operand; a third barrier hands
+//   the stage to the MMA issuer.  The accumulator is then 16 times the code
+//   products' sum, exactly; the epilogue's row scale carries the factor
+//   1/16.  No tensor-core kind multiplies 4-bit integers on sm_100a; with A
+//   in tensor memory the widened tile never passes through shared memory,
+//   whose traffic (tensor loads in, MMA operand reads out) bounds the main
+//   loop, so the packed stage costs less shared-memory traffic than an int8
+//   one.  A's stages sit in tensor memory after the two accumulators, so
+//   packed tiles are at most 192 columns wide.
 // gemm_i8_pair_kernel: a cluster of two CTAs per 256 x 256 output tile with
 //   the CTA-pair MMA (cta_group::2, M = 256): each CTA loads 128 rows of A and
 //   128 rows of B into its own shared memory, so one SM moves half the B
@@ -68,7 +69,7 @@ constexpr int BM = 128;
 constexpr int BK = 128;  // K bytes per stage: one 128-byte swizzle row
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
-constexpr int kConvWarps = 2;  // packed-A converters of the single-CTA kernel
+constexpr int kConvWarps = 4;  // packed-A converters of the single-CTA kernel (one per lane quarter)
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kStageBox = 2048;           // one 32 x 32 bf16 output box
 constexpr float kAccMagic = 12582912.0f;  // 1.5 * 2^23
@@ -320,13 +321,14 @@ __device__ __forceinline__ void epi_store_chunk(const GemmParams& p, const CUten
 // 2^LOGO columns (4, 5 or 6): dequantize, a fast Walsh-Hadamard transform
 // over each block (inside a chunk, and for 64-column blocks one more stage
 // between the two chunks of a group), then 1/sqrt(m) and the bias.
-template <int HC, int W, int NBOX, int LOGO, class RelAcc, class RelPrm>
+template <int HC, int W, int NBOX, int LOGO, int GMAX, class RelAcc, class RelPrm>
 __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap* tmY,
                                          uint32_t t_addr, const EpiTile& e, const float* prm,
                                          uint8_t* stg, int lane, RelAcc release_acc,
                                          RelPrm release_params) {
   constexpr int NCH = HC / 32;
-  constexpr int G = NCH <= 3 ? NCH : 2;
+  constexpr int G0 = NCH <= 3 ? NCH : 2;
+  constexpr int G = G0 <= GMAX ? G0 : (NCH % 2 == 0 && GMAX >= 2 ? 2 : 1);
   static_assert(NCH % G == 0, "whole groups of chunks");
   static_assert(LOGO == 0 || (LOGO >= 4 && LOGO <= 5) || (LOGO == 6 && G % 2 == 0),
                 "output blocks of 16 or 32 columns, or 64 over chunk pairs");
@@ -388,28 +390,36 @@ __device__ __forceinline__ void epi_tile(const GemmParams& p, const CUtensorMap*
 // ------------------------------------------------------- single-CTA kernel
 template <int BN, bool PK>
 struct GemmCfg {
-  static constexpr int A_BYTES = BM * BK;
+  static constexpr int A_BYTES = PK ? 0 : BM * BK;      // A's shared stage (PK: in tensor memory)
   static constexpr int B_BYTES = BN * BK;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  // bytes the tensor loads bring per stage (packed A arrives through the converters)
-  static constexpr uint32_t STAGE_TX = uint32_t((PK ? 0 : A_BYTES) + B_BYTES);
+  static constexpr int P_BYTES = PK ? BM * BK / 2 : 0;  // packed A as loaded (64-byte swizzle)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr uint32_t STAGE_TX = uint32_t(STAGE_BYTES);  // bytes the tensor loads bring
   static constexpr int THREADS = kGemmThreads + (PK ? 32 * kConvWarps : 0);
   static constexpr int NBAR_STAGE = PK ? 3 : 2;  // full, empty (, converted)
   static constexpr int HC = BN / 2;  // columns per epilogue warp
+  // accumulator chunks read per tensor-memory wait: at most 3; one for packed
+  // 192-column tiles, whose 448 threads leave 128 registers a thread
+  static constexpr int EPI_GMAX = (PK && BN == 192) ? 1 : 3;
   static constexpr int NBOX = 1;  // output staging boxes per epilogue warp
   static constexpr int EPI_STAGE_BYTES = NBOX * kStageBox;
   static constexpr int RING_BYTES = 2 * 3 * BN * 4;
   static constexpr int CTL_BYTES = 256;
   static constexpr int FIXED = kEpiWarps * EPI_STAGE_BYTES + RING_BYTES + CTL_BYTES + 1024;
   static constexpr int STAGES_RAW = (kSmemLimit - FIXED) / STAGE_BYTES;
-  static constexpr int STAGE_CAP = PK ? 7 : 8;  // barrier block size
+  // PK: A's stages (32 columns each) follow the two accumulators in the 512
+  // columns of tensor memory; the barrier block holds 7 stages of 3 barriers
+  static constexpr int TMEM_STAGE_CAP = PK ? (512 - 2 * BN) / 32 : 8;
+  static constexpr int STAGE_CAP = PK ? (TMEM_STAGE_CAP < 7 ? TMEM_STAGE_CAP : 7) : 8;
   static constexpr int STAGES = STAGES_RAW > STAGE_CAP ? STAGE_CAP : STAGES_RAW;
-  static constexpr int TMEM_COLS = tmem_cols_for(2 * BN);
+  static constexpr int A_COL0 = 2 * BN;  // first tensor-memory column of A's stages (PK)
+  static constexpr int TMEM_COLS = tmem_cols_for(2 * BN + (PK ? 32 * STAGES : 0));
   static constexpr uint32_t IDESC = i8_idesc(BM, BN);
   static constexpr size_t SMEM = size_t(STAGES) * STAGE_BYTES + FIXED;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "two 32-column-aligned halves");
   static_assert(B_BYTES % 1024 == 0, "stage bases must stay 1024-byte aligned");
-  static_assert(STAGES >= 2, "shared memory budget");
+  static_assert(STAGES >= 2, "shared / tensor memory budget");
+  static_assert(!PK || 2 * BN + 32 * STAGES <= 512, "tensor memory budget");
   static_assert(8 * NBAR_STAGE * STAGES + 80 <= CTL_BYTES, "barrier block");
   static_assert(SMEM <= size_t(kSmemLimit), "shared memory budget");
 };
@@ -424,11 +434,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sA = smem;
   uint8_t* sB = smem + size_t(C::STAGES) * C::A_BYTES;
-  uint8_t* epi_stage = sB + size_t(C::STAGES) * C::B_BYTES;  // 1024-aligned
+  uint8_t* sP = sB + size_t(C::STAGES) * C::B_BYTES;  // packed A (PK only)
+  uint8_t* epi_stage = sP + size_t(C::STAGES) * C::P_BYTES;  // 1024-aligned
   float* ring = reinterpret_cast<float*>(epi_stage + kEpiWarps * C::EPI_STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ring) + C::RING_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* conv = empty + C::STAGES;    // (PK) stage s's A widened to int8
+  uint64_t* conv = empty + C::STAGES;    // (PK) stage s's A widened into tensor memory
   uint64_t* tfull = conv + (PK ? C::STAGES : 0);  // [2] accumulator complete
   uint64_t* tempty = tfull + 2;          // [2] accumulator drained by the epilogue
   uint64_t* pfull = tempty + 2;          // [2] parameter slot loaded
@@ -458,7 +469,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
-    if (!PK) prefetch_tmap(&tmA);
+    prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmY);
   }
@@ -499,7 +510,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_TX);
-          if constexpr (!PK)
+          if constexpr (PK)  // K bytes of packed A per stage: BK / 2 (a multiple of 16)
+            tma_load_2d(sP + size_t(stage) * C::P_BYTES, &tmA, kb * (BK / 2), m_idx * BM,
+                        &full[stage]);
+          else
             tma_load_2d(sA + size_t(stage) * C::A_BYTES, &tmA, kb * BK, m_idx * BM, &full[stage]);
           tma_load_2d(sB + size_t(stage) * C::B_BYTES, &tmB, kb * BK, n_idx * BN, &full[stage]);
           ++issued;
@@ -543,7 +557,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
-          // B landed (full) and, for packed A, the converters wrote A (conv)
+          // B landed (full) and, for packed A, the converters stored A (conv)
           if (*abort_flag || !mbar_wait(&full[stage], phase, wc) ||
               (PK && !mbar_wait(&conv[stage], phase, wc))) {
             *abort_flag = 1;
@@ -556,8 +570,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k) {
             // advance 32 bytes along K inside the swizzle row (encoded >> 4)
-            mma_i8(d_tmem, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), C::IDESC,
-                   (kb > 0 || k > 0) ? 1u : 0u);
+            if constexpr (PK)  // A in tensor memory: 8 columns of four codes per 32 bytes
+              mma_i8_tmem_a(d_tmem, tmem_base + uint32_t(C::A_COL0 + 32 * stage + 8 * k),
+                            bdesc + uint64_t(2 * k), C::IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+            else
+              mma_i8(d_tmem, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), C::IDESC,
+                     (kb > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -608,7 +626,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + uint32_t(acc * BN + half * C::HC) +
                               (uint32_t(quarter * 32) << 16);
-      epi_tile<C::HC, BN, C::NBOX, LOGO>(
+      epi_tile<C::HC, BN, C::NBOX, LOGO, C::EPI_GMAX>(
           p, &tmY, t_addr, e, ring + acc * 3 * BN + half * C::HC, stg, lane,
           [&] {
             tc_fence_before();
@@ -624,77 +642,46 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
     __syncwarp();
   } else if constexpr (PK) {
     // ------------------------------------------------- packed-A converters
-    // Stage s's A tile: packed rows [128 m, 128 m + 128) x bytes [64 kb,
-    // 64 kb + 64) of a_packed -> the int8 tile the MMA reads (128 rows x 128
-    // bytes, 128-byte swizzle: 16-byte chunk j of row r at chunk j ^ (r & 7)
-    // of its row, 8-row atoms of 1024 bytes).  Thread ct (0..63) owns packed
-    // chunk ct & 3 of rows ct / 4 + 16 i, i = 0..7: a warp's load covers 8
-    // whole 64-byte row segments, and its stores hit 8 rows' distinct
-    // swizzled chunks (no bank conflicts).  Rows past T and bytes past K / 2
-    // read as zero codes.  The loads of the next D stages are in flight
-    // (registers) while a stage is widened.
-    constexpr int D = 3;
-    const int ct = (warp - 2 - kEpiWarps) * 32 + lane;
-    const int rsub = ct >> 2;          // row within each group of 16
-    const int cc = ct & 3;             // 16-byte chunk of the 64-byte row segment
-    const int swz = rsub & 7;          // r & 7 for every r = rsub + 16 i
-    const int64_t prow = p.K / 2;      // packed bytes per row
-    const int my_tiles =
-        int(blockIdx.x) < num_tiles ? (num_tiles - int(blockIdx.x) + int(gridDim.x) - 1) /
-                                          int(gridDim.x)
-                                    : 0;
-    const int total = my_tiles * KB;   // stages this CTA's main loops consume
-    uint4 pre[D][8];
-    auto fetch = [&](int j, uint4 (&dst)[8]) {
-      const int t = j / KB;
-      const int kb = j - t * KB;
-      const int tile = int(blockIdx.x) + t * int(gridDim.x);
-      const int64_t row0 = int64_t(tile % p.num_m_tiles) * BM + rsub;
-      const int64_t col = int64_t(kb) * (BK / 2) + cc * 16;
-      const bool col_ok = col < prow;  // K / 2 is a multiple of 16: whole chunks
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t row = row0 + 16 * i;
-        dst[i] = (col_ok && row < p.T)
-                     ? __ldg(reinterpret_cast<const uint4*>(p.a_packed + row * prow + col))
-                     : make_uint4(0u, 0u, 0u, 0u);
-      }
-    };
-#pragma unroll
-    for (int d = 0; d < D; ++d)
-      if (d < total) fetch(d, pre[d]);
+    // Lane i of converter warp w owns row r = 32 (w % 4) + i of every A tile,
+    // which is tensor-memory lane r.  Per stage it reads the row's 64 packed
+    // bytes (four 16-byte chunks; with the 64-byte swizzle chunk c of row r
+    // sits at chunk c ^ ((r >> 1) & 3), so the 8 rows of a quarter-warp read
+    // 8 distinct bank groups), widens them to 128 int8 values and stores
+    // them as 32 columns of four values each at A's stage in tensor memory.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int swz = (r >> 1) & 3;
+    const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(C::A_COL0);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int j0 = 0; j0 < total && ok; j0 += D) {
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        const int j = j0 + d;
-        if (j >= total) break;
-        // the MMAs that read stage s's previous A have completed
-        const bool got = !(*abort_flag) && mbar_wait(&empty[stage], phase ^ 1u, wc);
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        // the stage's packed tile has landed, and the MMAs that read its
+        // previous A from tensor memory have completed
+        const bool got = !(*abort_flag) && mbar_wait(&full[stage], phase, wc) &&
+                         mbar_wait(&empty[stage], phase ^ 1u, wc);
         if (!__all_sync(0xffffffffu, got)) {
           *abort_flag = 1;
           ok = false;
           break;
         }
-        uint8_t* dst = sA + size_t(stage) * C::A_BYTES + (rsub >> 3) * 1024 + swz * 128;
+        tc_fence_after();
+        const uint8_t* src = sP + size_t(stage) * C::P_BYTES + r * 64;
+        uint32_t a[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint4 o0, o1;
-          widen_i4x8(pre[d][i].x, o0.x, o0.y);
-          widen_i4x8(pre[d][i].y, o0.z, o0.w);
-          widen_i4x8(pre[d][i].z, o1.x, o1.y);
-          widen_i4x8(pre[d][i].w, o1.z, o1.w);
-          // row rsub + 16 i: two 8-row atoms further per i
-          uint8_t* row = dst + i * 2048;
-          *reinterpret_cast<uint4*>(row + (((2 * cc) ^ swz) << 4)) = o0;
-          *reinterpret_cast<uint4*>(row + (((2 * cc + 1) ^ swz) << 4)) = o1;
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + ((c ^ swz) << 4));
+          widen_i4x8(v.x, a[8 * c + 0], a[8 * c + 1]);
+          widen_i4x8(v.y, a[8 * c + 2], a[8 * c + 3]);
+          widen_i4x8(v.z, a[8 * c + 4], a[8 * c + 5]);
+          widen_i4x8(v.w, a[8 * c + 6], a[8 * c + 7]);
         }
-        fence_proxy_async_smem();  // the tile is read by the tensor cores
+        tmem_st_32x32b_x32(t_row + uint32_t(32 * stage), a);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&conv[stage]);
-        if (j + D < total) fetch(j + D, pre[d]);
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -947,7 +934,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_addr = tmem_base + uint32_t(acc * C::BN + half * C::HC) +
                               (uint32_t(quarter * 32) << 16);
-      epi_tile<C::HC, C::BN, C::NBOX, 0>(
+      epi_tile<C::HC, C::BN, C::NBOX, 0, 3>(
           p, &tmY, t_addr, e, ring + acc * 3 * C::BN + half * C::HC, stg, lane,
           [&] {
             tc_fence_before();
@@ -1009,7 +996,9 @@ static cudaError_t launch_logo(int bn, const void* tmap_a, const void* tmap_b,
                                const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st) {
   switch (bn) {
     case 128: return launch_bn<128, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
-    case 256: return launch_bn<256, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
+    case 256:  // packed A's stages leave no tensor memory for 256-column tiles
+      if constexpr (!PK) return launch_bn<256, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
+      return cudaErrorInvalidValue;
     default:
       if constexpr (LOGO <= 5) {
         if (bn == 64) return launch_bn<64, LOGO, PK>(tmap_a, tmap_b, tmap_y, p, grid, st);
@@ -1080,7 +1069,9 @@ static size_t smem_of(int bn) {
     case 64: return GemmCfg<64, PK>::SMEM;
     case 128: return GemmCfg<128, PK>::SMEM;
     case 192: return GemmCfg<192, PK>::SMEM;
-    case 256: return GemmCfg<256, PK>::SMEM;
+    case 256:
+      if constexpr (!PK) return GemmCfg<256, PK>::SMEM;
+      return 0;
     default: return 0;
   }
 }

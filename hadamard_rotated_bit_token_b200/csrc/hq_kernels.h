@@ -60,7 +60,6 @@ struct GemmParams {
   float inv_sqrt_out;         // 1/sqrt(m) of the output-side transform (weight-only form)
   float acc_unit;             // accumulator units per code product: 1, or 1/16 when A is packed
   int acc_shift;              // acc_debug = raw accumulator >> acc_shift (0, or 4 when packed)
-  const uint8_t* a_packed;    // packed A [T, K/2] bytes (packed kernels read it directly)
   unsigned int* err;          // device error word
   unsigned long long wait_ns; // bounded-wait limit
 };
@@ -71,9 +70,9 @@ struct GemmParams {
 // objects (copied into the launch): A [T,K] and B [N,K] int8 with box
 // {128, 128 | bn} and 128-byte swizzle; Y [T,N] bf16 with box {32, 32} and
 // 64-byte swizzle.  packed_a: A holds two 4-bit codes per byte, [T,K/2]
-// bytes at GemmParams.a_packed (read directly; tmap_a is not used); the
-// kernel widens each tile to int8 (16 * code) in shared memory, so the
-// caller passes acc_unit = 1/16 and acc_shift = 4.
+// bytes with box {64, 128} and 64-byte swizzle; the kernel widens each tile
+// to int8 (16 * code) in tensor memory, so the caller passes acc_unit =
+// 1/16 and acc_shift = 4; bn 64, 128 or 192 (128 with logo 6).
 cudaError_t launch_gemm(int bn, int logo, bool packed_a, const void* tmap_a, const void* tmap_b,
                         const void* tmap_y, const GemmParams& p, int grid, cudaStream_t st);
 size_t gemm_smem_bytes(int bn, bool packed_a);
