@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--out-order", type=int, default=0, choices=[0, 16, 32, 64],
                     help="run the configuration's shape in the weight-only Hadamard form "
                          "(W rotated along N in blocks of this order; no rotation along K)")
+    ap.add_argument("--packed", action="store_true",
+                    help="store the activation codes two per byte (3- and 4-bit codes)")
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -83,17 +85,18 @@ def layer_ops(cfg) -> float:
 
 
 def quantizer_bytes(cfg) -> float:
-    """Algorithmic bytes of hq_quantize_act: read X (2 B/elt), write int8 codes
-    (1 B/elt in the int8 container), write scale + mean (8 B/token); the
-    per-tensor dynamic mode reads X twice."""
+    """Algorithmic bytes of hq_quantize_act: read X (2 B/elt), write the codes
+    (1 B/elt in the int8 container, 1/2 B packed), write scale + mean
+    (8 B/token); the per-tensor dynamic mode reads X twice."""
     passes = 2 if cfg.act_gran == 1 else 1
-    return cfg.T * cfg.K * (2.0 * passes + 1.0) + 8.0 * cfg.T
+    return cfg.T * cfg.K * (2.0 * passes + cfg.code_bytes()) + 8.0 * cfg.T
 
 
 def gemm_bytes(cfg) -> float:
     """Algorithmic HBM bytes of hq_linear: A codes + B codes + bf16 Y + per-row
     and per-column fp32 vectors."""
-    return cfg.T * cfg.K + cfg.N * cfg.K + 2.0 * cfg.T * cfg.N + 8.0 * cfg.T + 12.0 * cfg.N
+    return (cfg.T * cfg.K * cfg.code_bytes() + cfg.N * cfg.K + 2.0 * cfg.T * cfg.N +
+            8.0 * cfg.T + 12.0 * cfg.N)
 
 
 # ---------------------------------------------------------------------------
@@ -340,6 +343,8 @@ def workload_config(args):
         cfg = dataclasses.replace(cfg, centering=args.centering)
     if args.out_order:
         cfg = cfg.weight_only(args.out_order)
+    if getattr(args, "packed", False):
+        cfg = cfg.packed()
     return cfg
 
 
@@ -353,6 +358,7 @@ def config_block(cfg, n_gpus):
             "form": (f"weight-only Hadamard (W rotated along N, blocks of {cfg.out_order})"
                      if cfg.out_order > 1 else "double Hadamard (X and W rotated along K)"),
             "act_granularity": gran,
+            "activation_codes": "two per byte" if cfg.code_format else "one per byte",
             "centering": {0: "none", 1: "token mean after H", 2: "token mean before H"}[cfg.centering],
             "sigma": cfg.use_sigma,
             "l2": "inputs larger than L2: step i reads copy i % M of the token batch, "
@@ -387,7 +393,8 @@ def run_hq(args):
     X, W, b = to_dev(Xb), to_dev(Wb), to_dev(bb)
     T, K, N = cfg.T, cfg.K, cfg.N
     desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
-                        act_gran=cfg.act_gran, centering=cfg.centering, out_order=cfg.out_order)
+                        act_gran=cfg.act_gran, centering=cfg.centering,
+                        code_format=cfg.code_format, out_order=cfg.out_order)
     stream = torch.cuda.current_stream()
 
     # offline: calibration + weight preparation (timed once, not part of the step)

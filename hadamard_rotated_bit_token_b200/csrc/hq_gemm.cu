@@ -5,8 +5,10 @@
 //   Y[t,n]   = bf16( s_x[t] * s_w[n] * acc[t,n]      (accumulator scale, HaTQ Eq. (18))
 //                    + b[n] + mu_t * colsum[n] )      (b~ = b + mu W~, HadaNorm Eq. (1))
 //
-// A = activation codes [T,K] int8, B = weight codes [N,K] int8, both K-major.
-// Two kernels share one warp layout (320 threads, one CTA per SM):
+// A = activation codes [T,K] int8 (or two 4-bit codes per byte, see PK
+// below), B = weight codes [N,K] int8, both K-major.
+// Two kernels share one warp layout (320 threads, one CTA per SM; the packed
+// form adds warps 10..13):
 //   warp 0      one thread issues TMA tensor loads (128-byte swizzle) of the
 //               A and B K-slices into a ring of shared-memory stages, and per
 //               output tile bulk copies of the tile's columns of s_w, colsum

@@ -47,6 +47,7 @@ class LayerConfig:
     outlier_mult: float
     offset_std: float
     out_order: int = 0     # > 1: the weight-only Hadamard form (had_order 1, W rotated along N)
+    code_format: int = 0   # 1: activation codes two per byte (3- and 4-bit codes only)
 
     def with_tokens(self, T: int) -> "LayerConfig":
         return dataclasses.replace(self, T=T)
@@ -54,7 +55,17 @@ class LayerConfig:
     def workload(self) -> str:
         rot = f"WH{self.out_order}" if self.out_order > 1 else f"H{self.had_order}"
         return (f"cfg{self.index}:{self.name}:T{self.T}xK{self.K}xN{self.N}"
-                f":{rot}:A{self.a_bits}W{self.w_bits}")
+                f":{rot}:A{self.a_bits}W{self.w_bits}" + (":packed" if self.code_format else ""))
+
+    def code_bytes(self) -> float:
+        """Bytes per activation code as stored: 1, or 1/2 when packed."""
+        return 0.5 if self.code_format else 1.0
+
+    def packed(self) -> "LayerConfig":
+        """The same layer with its 3- or 4-bit activation codes two per byte."""
+        if self.a_bits > 4:
+            raise ValueError("packed codes hold 3- and 4-bit activations only")
+        return dataclasses.replace(self, code_format=1)
 
     def weight_only(self, out_order: int) -> "LayerConfig":
         """The same layer shape and inputs in the weight-only Hadamard form:
