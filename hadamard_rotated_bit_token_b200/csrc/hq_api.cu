@@ -482,7 +482,6 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   hq_status s = check_quant_args(desc, X, T, sigma_inv, a_codes, a_scale, a_mean, workspace,
                                  workspace_bytes);
   if (s != HQ_OK || T == 0) return s;
-  const bool dyn = desc->act_gran == HQ_PER_TENSOR_DYNAMIC;
   DeviceState* dev;
   s = device_state(&dev);
   if (s != HQ_OK) return s;
