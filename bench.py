@@ -58,6 +58,8 @@ def parse_args(argv=None):
                          "(W rotated along N in blocks of this order; no rotation along K)")
     ap.add_argument("--packed", action="store_true",
                     help="store the activation codes two per byte (3- and 4-bit codes)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the packed-code variant measured beside the headline")
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -498,8 +500,53 @@ def run_hq(args):
     torch.cuda.synchronize()
     c_total = timed(g_cublas)
     del g_cublas, Yc
-    total_ms, q_total, g_total, c_total = max_over_ranks([total_ms, q_total, g_total, c_total],
-                                                         world, dist, dev)
+
+    # variant beside the headline (same inputs and weights, timed the same
+    # way): 3- and 4-bit activation codes stored two per byte, widened to
+    # int8 inside the GEMM
+    pk_times = [0.0, 0.0, 0.0]
+    with_packed = cfg.code_format == 0 and cfg.a_bits <= 4 and not args.no_variants
+    if with_packed:
+        pdesc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                             act_gran=cfg.act_gran, centering=cfg.centering,
+                             code_format=hq.HQ_CODES_I4_PACKED, out_order=cfg.out_order)
+        player = hq.HadamardQuantLinear(pdesc, W, b, absmax, cfg.alpha)
+        pbufs = player.buffers(T)
+        pmean = pbufs["a_mean"] if cfg.centering else None
+
+        def pk_quant(i):
+            hq.hq_quantize_act(pdesc, Xs[i % n_copies], sig_inv, pbufs["a_codes"],
+                               pbufs["a_scale"], pbufs["a_mean"], player.workspace)
+
+        def pk_linear():
+            hq.hq_linear(pdesc, pbufs["a_codes"], pbufs["a_scale"], pmean, player.w_codes,
+                         player.w_scale, player.colsum, player.bias_f32, Y)
+
+        for i in range(args.warmup):
+            pk_quant(i)
+            pk_linear()
+        torch.cuda.synchronize()
+        pgs = []
+        for do_q, do_l in ((True, True), (True, False), (False, True)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(args.steps):
+                    if do_q:
+                        pk_quant(i)
+                    if do_l:
+                        pk_linear()
+            g.replay()
+            pgs.append(g)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        pk_times = [timed(g) for g in pgs]
+        status = hq.hq_check_device_error()
+        if status != 0:
+            raise RuntimeError(f"device error in the packed variant: {hq.STATUS_NAMES.get(status)}")
+        del pgs, player, pbufs
+    (total_ms, q_total, g_total, c_total, pk_step, pk_q, pk_g) = max_over_ranks(
+        [total_ms, q_total, g_total, c_total] + pk_times, world, dist, dev)
     ms_per_step = total_ms / args.steps
     ops = layer_ops(cfg)
     value = job_throughput(ops, args.steps, world, total_ms)
@@ -589,6 +636,23 @@ def run_hq(args):
         "clocks": clock_info,
         "e2e": e2e,
     }
+    if with_packed:
+        pcfg = cfg.packed()
+        line["variants"] = {"packed_codes": {
+            "what": "the same layer, inputs and weights with the activation codes stored two "
+                    "per byte (HQ_CODES_I4_PACKED) and widened to int8 inside the GEMM; "
+                    "outputs bit-identical to the headline's",
+            "value": job_throughput(ops, args.steps, world, pk_step), "unit": "TOPS",
+            "ms_per_step": pk_step / args.steps,
+            "quantizer": {"ms_per_launch": pk_q / args.steps,
+                          "GB/s": quantizer_bytes(pcfg) / (pk_q / args.steps * 1e-3) / 1e9,
+                          "frac_hbm": quantizer_bytes(pcfg) / (pk_q / args.steps * 1e-3) / 1e9 /
+                                      peaks["hbm_gbs"],
+                          "bytes": quantizer_bytes(pcfg)},
+            "gemm": {"ms_per_launch": pk_g / args.steps,
+                     "TOPS": ops / (pk_g / args.steps * 1e-3) / 1e12,
+                     "frac_int8": ops / (pk_g / args.steps * 1e-3) / 1e12 / int8_peak,
+                     "hbm_bytes": gemm_bytes(pcfg)}}}
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(cfg, Xb, Wb, bb, args.cpu_seconds)
     print(json.dumps(line), flush=True)
