@@ -170,6 +170,19 @@ def test_layer_desc_layout_matches_the_header(hq):
     assert ctypes.sizeof(hq.LayerDesc) == 4 * len(names)
 
 
+def test_enum_constants_match_the_header(hq):
+    """Every HQ_* enumerator and status code in the header has the same value
+    in the binding."""
+    text = open(os.path.join(ROOT, "include", "hq.h")).read()
+    pairs = re.findall(r"\b(HQ_[A-Z0-9_]+)\s*=\s*(\d+)", text)
+    assert len(pairs) >= 20
+    for name, value in pairs:
+        if name.startswith("HQ_ERR_") or name == "HQ_OK":
+            assert hq.STATUS_NAMES[int(value)] == name
+        else:
+            assert getattr(hq, name) == int(value), name
+
+
 def test_prepare_and_calib_validation(hq):
     lib = hq.load_library()
     D = hq.LayerDesc
