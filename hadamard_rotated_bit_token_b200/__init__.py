@@ -30,7 +30,7 @@ __all__ = [
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
     "hq_debug_set_gemm_variant", "HQ_GEMM_AUTO", "HQ_GEMM_SINGLE_CTA", "HQ_GEMM_CTA_PAIR",
-    "hq_quantize_act_noalloc", "HadamardQuantLinear",
+    "hq_quantize_act_noalloc", "hq_debug_plan", "HadamardQuantLinear",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -47,7 +47,7 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED
 EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare_weights",
             "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
             "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-            "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc")
+            "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan")
 
 
 class HQError(RuntimeError):
@@ -113,10 +113,13 @@ def load_library():
         lib.hq_debug_set_wait_limit.argtypes = [ctypes.c_uint64]
         lib.hq_debug_inject_fault.argtypes = [ctypes.c_int]
         lib.hq_debug_set_gemm_variant.argtypes = [ctypes.c_int]
+        _i32p = ctypes.POINTER(ctypes.c_int32)
+        lib.hq_debug_plan.argtypes = [desc_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                      _i32p, _i32p, _i32p, _i32p]
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
                      "hq_forward_host",
                      "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-                     "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc"):
+                     "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -256,6 +259,16 @@ def hq_debug_set_wait_limit(nanoseconds: int):
 
 def hq_debug_inject_fault(kind: int):
     _check(load_library().hq_debug_inject_fault(int(kind)), "hq_debug_inject_fault")
+
+
+def hq_debug_plan(desc: LayerDesc, T: int, sms: int, pair_clusters: int) -> dict:
+    """The launch shapes the library chooses for desc and T tokens on a device
+    with `sms` SMs and `pair_clusters` CTA-pair clusters (host only)."""
+    out = [ctypes.c_int32(0) for _ in range(4)]
+    _check(load_library().hq_debug_plan(ctypes.byref(desc), int(T), int(sms), int(pair_clusters),
+                                        *(ctypes.byref(o) for o in out)), "hq_debug_plan")
+    return {"quant_rows": out[0].value, "quant_threads": out[1].value,
+            "gemm_pair": bool(out[2].value), "gemm_bn": out[3].value}
 
 
 def hq_debug_set_gemm_variant(variant: int):

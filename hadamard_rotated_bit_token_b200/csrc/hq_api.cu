@@ -138,6 +138,8 @@ hq_status check_desc(const hq_layer_desc* d) {
 
 hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
+constexpr int kQuantCtasPerSm = 2;  // quantizer CTAs per SM (its launch bounds)
+
 // Rows per tile R and threads per CTA (one thread per 32-channel slice of
 // each row, whole warps).  The kernel is issue-bound, so an SM's time is
 // about (tiles it runs) x (threads of its CTAs): the cost of R is the tile
@@ -190,7 +192,7 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
                             QuantLaunch* out) {
   QuantLaunch& L = *out;
   std::memset(&L.p, 0, sizeof(L.p));
-  const int per_sm = 2;          // CTAs per SM (kernel launch bounds)
+  const int per_sm = kQuantCtasPerSm;
   int R, nt;
   quant_shape(K, T > 0 ? T : 1, dev->sm_count, per_sm, &R, &nt);
   const int logn = ilog2_exact(n);
@@ -732,6 +734,24 @@ hq_status hq_debug_set_gemm_variant(int variant) {
     return HQ_ERR_INVALID_ARGUMENT;
   std::lock_guard<std::mutex> lock(g_mutex);
   g_gemm_variant = variant;
+  return HQ_OK;
+}
+
+hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_clusters,
+                        int32_t* quant_rows, int32_t* quant_threads, int32_t* gemm_pair,
+                        int32_t* gemm_bn) {
+  hq_status s = check_desc(desc);
+  if (s != HQ_OK) return s;
+  if (T < 1 || sms < 1 || pair_clusters < 0) return HQ_ERR_INVALID_ARGUMENT;
+  int R, nt;
+  quant_shape(desc->K, T, sms, kQuantCtasPerSm, &R, &nt);
+  const int logo = ilog2_exact(desc->out_order > 1 ? desc->out_order : 1);
+  const GemmChoice gc = choose_gemm(T, desc->N, desc->K, sms, pair_clusters, HQ_GEMM_AUTO, logo,
+                                    desc->code_format == HQ_CODES_I4_PACKED);
+  if (quant_rows) *quant_rows = R;
+  if (quant_threads) *quant_threads = nt;
+  if (gemm_pair) *gemm_pair = gc.pair ? 1 : 0;
+  if (gemm_bn) *gemm_bn = gc.pair ? 256 : gc.bn;
   return HQ_OK;
 }
 

@@ -303,6 +303,20 @@ hq_status hq_debug_set_gemm_variant(int variant);
 enum { HQ_FAULT_NONE = 0, HQ_FAULT_QUANT_WITHHOLD_ROW = 1 };
 hq_status hq_debug_inject_fault(int kind);
 
+/* Test hook, host only (no device call, usable without a GPU): the launch
+ * shapes hq_quantize_act and hq_linear choose for `desc` and T tokens on a
+ * device with `sms` SMs that holds `pair_clusters` co-resident CTA-pair
+ * clusters (0: none), under the automatic GEMM choice.
+ *   quant_rows, quant_threads  rows per quantizer tile, threads per CTA;
+ *   gemm_pair                  1: the CTA-pair kernel, 0: one CTA per tile;
+ *   gemm_bn                    the tile width (256 for the pair).
+ * Output pointers are host pointers and may be NULL.  Returns the
+ * description's validation status, or HQ_ERR_INVALID_ARGUMENT for T < 1,
+ * sms < 1 or pair_clusters < 0. */
+hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_clusters,
+                        int32_t* quant_rows, int32_t* quant_threads, int32_t* gemm_pair,
+                        int32_t* gemm_bn);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,85 @@
+"""The library's launch-shape choices (hq_debug_plan: host logic, no GPU):
+the quantizer's rows per tile and threads per CTA, and the GEMM kernel and
+tile width, for a 148-SM B200 holding 74 CTA-pair clusters."""
+import itertools
+
+import pytest
+
+SMS, PAIRS = 148, 74
+
+
+@pytest.fixture(scope="module")
+def hq():
+    import hadamard_rotated_bit_token_b200 as hq_mod
+    from hadamard_rotated_bit_token_b200 import build as hq_build
+    hq_build.build()
+    hq_mod.load_library()
+    return hq_mod
+
+
+def _plan(hq, K, N, n, T, **kw):
+    return hq.hq_debug_plan(hq.LayerDesc(K, N, n, **kw), T, SMS, PAIRS)
+
+
+def test_measured_choices_for_the_configurations(hq):
+    # config 2: 7-row tiles (1171 tiles fill the last round of 296 CTAs),
+    # 192-column GEMM tiles
+    assert _plan(hq, 1152, 3456, 128, 8192) == {"quant_rows": 7, "quant_threads": 256,
+                                                 "gemm_pair": False, "gemm_bn": 192}
+    # config 3: 2 rows of 144 slices; N = 1152 is not a whole number of pair tiles
+    p = _plan(hq, 4608, 1152, 256, 8192, a_bits=3)
+    assert (p["quant_rows"], p["quant_threads"], p["gemm_pair"], p["gemm_bn"]) == (2, 288, False, 192)
+    # config 4: per-tensor W8A8 1x1 convolution
+    p = _plan(hq, 320, 320, 64, 65536, a_bits=8, w_bits=8, act_gran=1, centering=0)
+    assert (p["quant_rows"], p["quant_threads"], p["gemm_bn"]) == (32, 320, 192)
+    # config 5: long K over N in whole 256-column tiles takes the CTA pair,
+    # and R = 3 (not the 2 % cheaper R = 2, measured slower)
+    assert _plan(hq, 3072, 12288, 1024, 16384) == {"quant_rows": 3, "quant_threads": 288,
+                                                    "gemm_pair": True, "gemm_bn": 256}
+    # config 1: one small wave
+    assert _plan(hq, 1024, 1024, 1024, 256)["gemm_bn"] == 64
+
+
+def test_forms_that_exclude_the_pair_or_wide_tiles(hq):
+    # packed codes keep A in tensor memory beside two accumulators: <= 192 columns, no pair
+    p = _plan(hq, 3072, 12288, 1024, 16384, code_format=1)
+    assert not p["gemm_pair"] and p["gemm_bn"] <= 192
+    # the weight-only form runs in the single-CTA kernel; 64-column output
+    # blocks need whole 64-column halves
+    p = _plan(hq, 3072, 12288, 1, 16384, centering=0, out_order=64)
+    assert not p["gemm_pair"] and p["gemm_bn"] in (128, 256)
+    # no pair clusters on the device: single CTA
+    d = hq.LayerDesc(3072, 12288, 1024)
+    assert not hq.hq_debug_plan(d, 16384, SMS, 0)["gemm_pair"]
+
+
+def test_plan_invariants_over_shapes(hq):
+    Ks = [64, 320, 1024, 1152, 3072, 4608, 9216]
+    Ts = [1, 7, 127, 128, 1000, 8192, 65536]
+    Ns = [16, 320, 3456, 12288]
+    for K, T, N, packed in itertools.product(Ks, Ts, Ns, (0, 1)):
+        n = 64 if K % 64 == 0 else 16
+        p = _plan(hq, K, N, n, T, code_format=packed)
+        S = K // 32
+        R, nt = p["quant_rows"], p["quant_threads"]
+        assert R >= 1 and R * S <= 320 and nt % 32 == 0 and R * S <= nt < R * S + 32
+        assert p["gemm_bn"] in (64, 128, 192, 256)
+        if packed:
+            assert not p["gemm_pair"] and p["gemm_bn"] <= 192
+        if p["gemm_pair"]:
+            assert N % 256 == 0 and p["gemm_bn"] == 256
+
+
+def test_plan_validation(hq):
+    import ctypes
+    lib = hq.load_library()
+    D = hq.LayerDesc
+    assert lib.hq_debug_plan(None, 8, SMS, PAIRS, None, None, None, None) == 1
+    assert lib.hq_debug_plan(ctypes.byref(D(1024, 16, 1024)), 0, SMS, PAIRS, None, None, None,
+                             None) == 1
+    assert lib.hq_debug_plan(ctypes.byref(D(1024, 16, 1024)), 8, 0, PAIRS, None, None, None,
+                             None) == 1
+    assert lib.hq_debug_plan(ctypes.byref(D(1000, 16, 8)), 8, SMS, PAIRS, None, None, None,
+                             None) == 2
+    assert lib.hq_debug_plan(ctypes.byref(D(1024, 16, 1024)), 8, SMS, PAIRS, None, None, None,
+                             None) == 0
