@@ -154,6 +154,10 @@ def test_forward_host_validation(hq):
     assert call(D(1024, 16, 1024), Xd=FAKE + 2) == 3
     assert call(D(1024, 16, 1024), yd=FAKE + 8) == 3
     assert call(D(1024, 16, 1024), T=0) == 0
+    # packed codes: only 3- and 4-bit activations; unknown formats refused
+    assert call(D(1024, 16, 1024, a_bits=8, code_format=1)) == 2
+    assert call(D(1024, 16, 1024, code_format=7)) == 2
+    assert call(D(1024, 16, 1024, code_format=1), T=0) == 0
 
 
 def test_layer_desc_layout_matches_the_header(hq):
