@@ -101,7 +101,8 @@ enum { HQ_CODES_I8 = 0, HQ_CODES_I4_PACKED = 1 };
  *               nibble of byte j, element 2j+1 in the high nibble, each a
  *               4-bit two's-complement value.  hq_quantize_act writes this
  *               form and hq_linear reads it (the GEMM widens each tile to
- *               int8 in shared memory).  Weight codes stay one per byte.
+ *               int8 in tensor memory, where the MMA takes its A operand).
+ *               Weight codes stay one per byte.
  *   out_order   0 or 1: the double-Hadamard form above (no output-side
  *               transform).  16, 32 or 64: the weight-only Hadamard form
  *               (HaTQ Sec. IV-B, Eq. (15)-(17)): the weights are rotated

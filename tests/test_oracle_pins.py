@@ -560,3 +560,96 @@ def test_packed_codes_reject_out_of_range_values():
         oracle.pack_i4(np.array([0, -9], dtype=np.int8))
     with pytest.raises(ValueError):
         oracle.pack_i4(np.array([1, 2, 3], dtype=np.int8))
+
+
+# --------------------------------------------------------------------------
+# Calibration: HadaNorm review, "What carries the argument", Eq. (3)
+# sigma_i = max|X_i|^alpha / max|W_i|^(1-alpha), with max over the tokens of
+# input channel i for X and over the output channels of input channel i for W
+# --------------------------------------------------------------------------
+
+def _bf16_bits(values):
+    """bf16 bit patterns of values that bf16 holds exactly (hand-checked)."""
+    table = {1.0: 0x3F80, -1.0: 0xBF80, 2.0: 0x4000, -2.0: 0xC000, 0.5: 0x3F00,
+             0.25: 0x3E80, -3.5: 0xC060, -4.0: 0xC080, 3.0: 0x4040, 0.0: 0x0000}
+    out = []
+    for v in values:
+        if isinstance(v, str):  # "-0": the negative zero bit pattern
+            out.append(0x8000)
+        else:
+            out.append(table[v])
+    return out
+
+
+def test_col_absmax_hand_built_matrix():
+    """max over rows of |M[r, c]| for a 3 x 4 bf16 matrix written out by
+    hand: negative entries, a column of +0 and -0 only, the largest magnitude
+    in the first, middle and last row.  A signed max (no absolute value)
+    would give [1, 0, 0.5, 3]; a max along rows instead of columns has
+    three entries, not four."""
+    rows = [[1.0, "-0", -3.5, 3.0],
+            [-2.0, 0.0, 0.5, -1.0],
+            [0.25, "-0", -4.0, 2.0]]
+    M = np.array([_bf16_bits(r) for r in rows], dtype=np.uint16)
+    got = oracle.col_absmax(M)
+    assert got.shape == (4,)
+    assert got.tolist() == [2.0, 0.0, 4.0, 3.0]
+    assert not np.signbit(got[1])  # |-0| is +0
+    # a single row is its own absolute value; no rows leaves the zero start
+    assert oracle.col_absmax(M[1:2]).tolist() == [2.0, 0.0, 0.5, 1.0]
+    assert oracle.col_absmax(M[:0]).tolist() == [0.0, 0.0, 0.0, 0.0]
+
+
+def test_sigma_hand_worked_values_of_eq3():
+    """sigma = amax_x^alpha / amax_w^(1-alpha), worked by hand:
+      amax_x = 4,  amax_w = 1/4, alpha = 1/2:  2 / (1/2)        = 4
+      amax_x = 16, amax_w = 81,  alpha = 1/4:  16^(1/4) / 81^(3/4) = 2 / 27
+    The second case separates the plausible slips: swapping alpha and
+    1 - alpha gives 16^(3/4) / 81^(1/4) = 8/3, the inverted ratio 27/2."""
+    ax = np.array([4.0, 16.0])
+    aw = np.array([0.25, 81.0])
+    s = oracle.sigma(ax, aw, 0.5)
+    assert s[0] == pytest.approx(4.0, rel=1e-15)
+    s = oracle.sigma(ax, aw, 0.25)
+    assert s[1] == pytest.approx(2.0 / 27.0, rel=1e-14)
+    assert s[1] != pytest.approx(8.0 / 3.0) and s[1] != pytest.approx(27.0 / 2.0)
+
+
+def test_sigma_end_points_of_alpha():
+    """alpha = 0 leaves only the weight term, sigma = 1 / amax_w; alpha = 1
+    only the activation term, sigma = amax_x (HadaNorm review Eq. (3) at the
+    ends of its range)."""
+    ax = np.array([3.0, 0.5, 12.0, 1.0])
+    aw = np.array([0.02, 4.0, 0.125, 1.0])
+    assert np.allclose(oracle.sigma(ax, aw, 0.0), 1.0 / aw, rtol=1e-15, atol=0)
+    assert np.allclose(oracle.sigma(ax, aw, 1.0), ax, rtol=1e-15, atol=0)
+
+
+def test_sigma_is_one_when_a_maximum_is_zero():
+    """A channel that is identically zero on either side has no scale to
+    balance: sigma = 1 there (the oracle's guard; the pages are silent), and
+    the neighbouring channels keep their Eq. (3) values."""
+    ax = np.array([0.0, 4.0, 0.0, 4.0])
+    aw = np.array([0.25, 0.0, 0.0, 0.25])
+    s = oracle.sigma(ax, aw, 0.5)
+    assert s.tolist() == [1.0, 1.0, 1.0, pytest.approx(4.0, rel=1e-15)]
+    assert np.all(np.isfinite(oracle.sigma(ax, aw, 0.3)))
+
+
+def test_sigma_balances_the_channel_maxima():
+    """The point of Eq. (3): after X diag(sigma^-1) and diag(sigma) W the
+    channel maxima satisfy max|X_i / sigma_i| = amax_x^(1-alpha) amax_w^(1-alpha)
+    and max|sigma_i W_i| = amax_x^alpha amax_w^alpha, so at alpha = 1/2 both
+    sides share the maximum sqrt(amax_x amax_w) (SmoothQuant-style balance)."""
+    g = np.random.default_rng(5)
+    X = synth.f32_to_bf16_bits((g.standard_normal((64, 48)) * np.exp(g.standard_normal(48))).astype(np.float32))
+    W = synth.f32_to_bf16_bits((g.standard_normal((32, 48)) * 0.02).astype(np.float32))
+    ax, aw = oracle.col_absmax(X), oracle.col_absmax(W)
+    for alpha in (0.5, 0.3):
+        s = oracle.sigma(ax, aw, alpha)
+        xs = np.max(np.abs(oracle.bf16_to_f64(X)) / s, axis=0)
+        ws = np.max(np.abs(oracle.bf16_to_f64(W)) * s, axis=0)
+        assert np.allclose(xs, ax ** (1 - alpha) * aw ** (1 - alpha), rtol=1e-12)
+        assert np.allclose(ws, ax ** alpha * aw ** alpha, rtol=1e-12)
+        if alpha == 0.5:
+            assert np.allclose(xs, ws, rtol=1e-12)
