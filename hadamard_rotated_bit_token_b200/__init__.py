@@ -286,8 +286,13 @@ class HadamardQuantLinear:
     Allocation is the caller's (PyTorch); the library only reads and writes the
     tensors it is given.  `forward(X)` = hq_quantize_act + hq_linear."""
 
-    def __init__(self, desc: LayerDesc, W, bias=None, act_absmax=None, alpha=0.5, device=None):
+    def __init__(self, desc: LayerDesc, W, bias=None, act_absmax=None, alpha=0.5, device=None,
+                 static_scale=None):
+        """static_scale: the activation scale s (real units, code = rne(V / s))
+        of HQ_PER_TENSOR_STATIC, required in that mode and refused in the
+        others; it is written into a_scale[0] of every buffer set."""
         import torch
+        self.static_scale = self._check_static_scale(desc, static_scale)
         self.desc = desc
         dev = W.device if device is None else device
         K, N = desc.K, desc.N
@@ -316,8 +321,24 @@ class HadamardQuantLinear:
             b = {"a_codes": codes,
                  "a_scale": torch.empty(T if per_row else 1, dtype=torch.float32, device=dev),
                  "a_mean": torch.empty(T, dtype=torch.float32, device=dev)}
+            if self.desc.act_gran == HQ_PER_TENSOR_STATIC:
+                # an input of the quantizer and of the GEMM in this mode
+                b["a_scale"].fill_(self.static_scale)
             self._bufs[T] = b
         return b
+
+    @staticmethod
+    def _check_static_scale(desc, static_scale):
+        if desc.act_gran == HQ_PER_TENSOR_STATIC:
+            if static_scale is None:
+                raise ValueError("HQ_PER_TENSOR_STATIC needs static_scale (the activation scale)")
+            v = float(static_scale)
+            if not (v > 0.0 and v < float("inf")):
+                raise ValueError(f"static_scale must be positive and finite, got {v}")
+            return v
+        if static_scale is not None:
+            raise ValueError("static_scale is only used with HQ_PER_TENSOR_STATIC")
+        return None
 
     def quantize(self, X):
         b = self.buffers(X.shape[0])
@@ -360,12 +381,14 @@ class HadamardQuantLinear:
     # prepared-weights blob (deployment: skip hq_prepare_weights at load)
     # ------------------------------------------------------------------
     # Little-endian layout:
-    #   b"HQPW", u32 version (1), 9 x i32 hq_layer_desc fields in header order,
-    #   u32 use_sigma, then five sections, each u64 byte count + payload:
+    #   b"HQPW", u32 version (2), 9 x i32 hq_layer_desc fields in header order,
+    #   u32 use_sigma, f64 static_scale (0 when the mode has none; version 2
+    #   only -- version 1 blobs, without it, still load), then five sections,
+    #   each u64 byte count + payload:
     #   w_codes int8 [N*K], w_scale f32 [N], colsum f32 [N], sigma_inv f32 [K],
     #   bias_f32 f32 [N]; then u32 CRC-32 of everything before it.
     _BLOB_MAGIC = b"HQPW"
-    _BLOB_VERSION = 1
+    _BLOB_VERSION = 2
 
     def export_prepared(self) -> bytes:
         """The prepared weights and the layer description as one blob."""
@@ -377,6 +400,7 @@ class HadamardQuantLinear:
         head += struct.pack("<9i", d.K, d.N, d.had_order, d.a_bits, d.w_bits, d.act_gran,
                             d.centering, d.code_format, d.out_order)
         head += struct.pack("<I", 1 if self.use_sigma else 0)
+        head += struct.pack("<d", self.static_scale if self.static_scale is not None else 0.0)
         parts = [head]
         for t, dt in ((self.w_codes, np.int8), (self.w_scale, np.float32),
                       (self.colsum, np.float32), (self.sigma_inv, np.float32),
@@ -401,7 +425,7 @@ class HadamardQuantLinear:
         if zlib.crc32(body) & 0xFFFFFFFF != crc:
             raise ValueError("prepared-weights blob: checksum mismatch")
         version = struct.unpack_from("<I", body, 4)[0]
-        if version != cls._BLOB_VERSION:
+        if version not in (1, cls._BLOB_VERSION):
             raise ValueError(f"prepared-weights blob: unsupported version {version}")
         f = struct.unpack_from("<9i", body, 8)
         desc = LayerDesc(f[0], f[1], f[2], a_bits=f[3], w_bits=f[4], act_gran=f[5],
@@ -409,6 +433,18 @@ class HadamardQuantLinear:
         use_sigma = bool(struct.unpack_from("<I", body, 44)[0])
         K, N = desc.K, desc.N
         off = 48
+        static_scale = None
+        if version >= 2:
+            if len(body) < off + 8:
+                raise ValueError("prepared-weights blob: truncated")
+            s_val = struct.unpack_from("<d", body, off)[0]
+            off += 8
+            if desc.act_gran == HQ_PER_TENSOR_STATIC:
+                static_scale = s_val
+        try:
+            static_scale = cls._check_static_scale(desc, static_scale)
+        except ValueError as e:
+            raise ValueError(f"prepared-weights blob: {e}") from None
         arrays = []
         for dt, count in ((np.int8, N * K), (np.float32, N), (np.float32, N), (np.float32, K),
                           (np.float32, N)):
@@ -429,6 +465,7 @@ class HadamardQuantLinear:
         self.w_scale, self.colsum, self.sigma_inv, self.bias_f32 = (
             torch.from_numpy(a).to(dev) for a in arrays[1:])
         self.use_sigma = use_sigma
+        self.static_scale = static_scale
         ws = hq_quantize_act_workspace_bytes(desc, 0) if dev.type == "cuda" else 0
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev) if ws else None
         self._bufs = {}
