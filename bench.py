@@ -39,7 +39,10 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 METRIC = "HadaNorm W4A4 linear TOPS & quantizer HBM GB/s (fraction of roofline), 1×B200"
-DEFAULT_CONFIG = 2          # the PixArt-Sigma-shaped qkv projection (the metric's workload)
+DEFAULT_CONFIG = 5          # the large DiT linear: the largest single-GPU W4A4 workload
+# the other workloads, measured in the same run (configuration, centering override)
+PER_CONFIG = ((1, None), (2, None), (3, None), (3, 0), (4, None), (5, None))
+CEILING_K_BLOCKS = 4096     # MMA-only loop: k blocks (4 MMAs each) per CTA
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 2.0        # nominal dense int8 : bf16 tensor ratio (4.5 : 2.25 PFLOP/s)
 
@@ -60,6 +63,8 @@ def parse_args(argv=None):
                     help="store the activation codes two per byte (3- and 4-bit codes)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the packed-code variant measured beside the headline")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the records of the other workloads (configs 1-5)")
     ap.add_argument("--impl", default="hq", choices=["hq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -374,6 +379,157 @@ def config_block(cfg, n_gpus):
 # the CUDA path
 # ---------------------------------------------------------------------------
 
+def setup_layer(hq, torch, cfg, dev, rank, l2):
+    """One workload on the device: replicated weights (same seed on every
+    rank), the rank's own token batch, the prepared layer and its buffers,
+    and M copies of the token batch (M * |X| > 2 x L2) so that step i can
+    read copy i % M from HBM."""
+    Wb, bb = synth.make_w(cfg)
+    Xb = synth.make_x(cfg, seed=shard_seed(cfg, rank))
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    X, W, b = to_dev(Xb), to_dev(Wb), to_dev(bb)
+    T, K, N = cfg.T, cfg.K, cfg.N
+    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering,
+                        code_format=cfg.code_format, out_order=cfg.out_order)
+    stream = torch.cuda.current_stream()
+    # offline: calibration + weight preparation (timed once, not part of the step)
+    absmax = torch.zeros(K, dtype=torch.float32, device=dev) if cfg.use_sigma else None
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    if absmax is not None:
+        hq.hq_calib_act_absmax(desc, X, absmax)
+    layer = hq.HadamardQuantLinear(desc, W, b, absmax, cfg.alpha)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    x_bytes = X.numel() * X.element_size()
+    n_copies = int(min(512, max(2, -(-2 * l2 // x_bytes) + 1)))
+    return {"cfg": cfg, "desc": desc, "layer": layer, "bufs": layer.buffers(T),
+            "Y": torch.empty((T, N), dtype=torch.bfloat16, device=dev),
+            "Xs": [X] + [X.clone() for _ in range(n_copies - 1)], "W": W, "b": b,
+            "absmax": absmax, "Xb": Xb, "Wb": Wb, "bb": bb,
+            "sig_inv": layer.sigma_inv if layer.use_sigma else None,
+            "prep_ms": p0.elapsed_time(p1),
+            "launches_per_step": (2 if cfg.act_gran == 1 else 1) + 1}
+
+
+def capture_layer_graphs(torch, ctx, steps, warmup):
+    """Warm-up, then three CUDA graphs of `steps` launches each: whole steps
+    (quantize + GEMM), the quantizer alone, the GEMM alone.  Step i reads
+    copy i % M of the token batch, so the activations come from HBM."""
+    import hadamard_rotated_bit_token_b200 as hq
+    desc, layer, bufs, Xs, Y = (ctx[k] for k in ("desc", "layer", "bufs", "Xs", "Y"))
+    mean_in = bufs["a_mean"] if desc.centering else None
+    n = len(Xs)
+
+    def quantize_i(i):
+        hq.hq_quantize_act(desc, Xs[i % n], ctx["sig_inv"], bufs["a_codes"], bufs["a_scale"],
+                           bufs["a_mean"], layer.workspace)
+
+    def linear():
+        hq.hq_linear(desc, bufs["a_codes"], bufs["a_scale"], mean_in, layer.w_codes,
+                     layer.w_scale, layer.colsum, layer.bias_f32, Y)
+
+    for i in range(warmup):
+        quantize_i(i)
+        linear()
+    torch.cuda.synchronize()
+    graphs = []
+    for do_q, do_l in ((True, True), (True, False), (False, True)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                if do_q:
+                    quantize_i(i)
+                if do_l:
+                    linear()
+        g.replay()
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
+def measure_mma_ceiling(hq, torch):
+    """The measured int8 tensor-core ceiling: the GEMMs' main loops with
+    nothing but the MMAs (hq_debug_mma_ceiling), one CTA per SM, timed with
+    CUDA events around each launch (about a millisecond each); best of three
+    launches after one warm-up launch."""
+    out = {"k_blocks_per_cta": CEILING_K_BLOCKS,
+           "what": "MMA-only loop (tcgen05.mma kind::i8 128x256x32 per CTA; pair: cta_group::2 "
+                   "256x256x32 per cluster), no loads, no epilogue; operands in shared memory"}
+    for name, pair in (("single_cta_TOPS", False), ("cta_pair_TOPS", True)):
+        try:
+            best = 0.0
+            stream = torch.cuda.current_stream()
+            for rep in range(4):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                ctas = hq.hq_debug_mma_ceiling(pair, CEILING_K_BLOCKS)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ops = ctas * CEILING_K_BLOCKS * 4 * 2.0 * 128 * 256 * 32
+                if rep > 0:  # the first launch configures the kernel
+                    best = max(best, ops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+            out[name] = best
+        except Exception as e:  # pair clusters unavailable on this device
+            out[name] = None
+            out[name + "_error"] = str(e)
+    return out
+
+
+def kernel_record(hq, cfg, q_ms, g_ms, step_ms, peaks, ceiling):
+    """Per-kernel figures of one workload: achieved bytes/s (quantizer) and
+    int ops/s (GEMM) against the measured peaks."""
+    ops = layer_ops(cfg)
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    q_gbs = quantizer_bytes(cfg) / (q_ms * 1e-3) / 1e9
+    g_tops = ops / (g_ms * 1e-3) / 1e12
+    desc = hq.LayerDesc(cfg.K, cfg.N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering,
+                        code_format=cfg.code_format, out_order=cfg.out_order)
+    import torch
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    pair_ok = ceiling.get("cta_pair_TOPS") is not None
+    plan = hq.hq_debug_plan(desc, cfg.T, props.multi_processor_count,
+                            props.multi_processor_count // 2 if pair_ok else 0)
+    ceil = ceiling.get("cta_pair_TOPS" if plan["gemm_pair"] else "single_cta_TOPS")
+    return {
+        "step_ms": step_ms, "step_TOPS": ops / (step_ms * 1e-3) / 1e12,
+        "quantizer": {"ms_per_launch": q_ms, "GB/s": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
+                      "bytes": quantizer_bytes(cfg), "tile_rows": plan["quant_rows"],
+                      "threads": plan["quant_threads"]},
+        "gemm": {"ms_per_launch": g_ms, "TOPS": g_tops, "frac_int8": g_tops / int8_peak,
+                 "mma_ceiling_TOPS": ceil,
+                 "frac_mma_ceiling": (g_tops / ceil) if ceil else None,
+                 "kernel": "CTA pair 256x256" if plan["gemm_pair"] else
+                           f"single CTA 128x{plan['gemm_bn']}",
+                 "hbm_bytes": gemm_bytes(cfg)},
+    }
+
+
+def per_config_records(hq, torch, args, head_cfg, dev, l2, peaks, ceiling, timed, check):
+    """The other workloads measured in the same run, the same way as the
+    headline (graphs of K launches, rotating inputs), one at a time."""
+    import dataclasses
+    out = {}
+    for index, centering in PER_CONFIG:
+        cfg = synth.CONFIGS[index]
+        if centering is not None:
+            cfg = dataclasses.replace(cfg, centering=centering)
+        if cfg == head_cfg:
+            continue
+        name = cfg.workload() + (f":centering{cfg.centering}" if centering is not None else "")
+        ctx = setup_layer(hq, torch, cfg, dev, 0, l2)
+        graphs = capture_layer_graphs(torch, ctx, args.steps, args.warmup)
+        step_ms, q_ms, g_ms = (timed(g) / args.steps for g in graphs)
+        check(f"in {name}")
+        out[name] = kernel_record(hq, cfg, q_ms, g_ms, step_ms, peaks, ceiling)
+        del graphs, ctx
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_hq(args):
     import torch
     import torch.distributed as dist
@@ -388,77 +544,8 @@ def run_hq(args):
                                 device_id=dev)
     hq.load_library()
     cfg = workload_config(args)
-    # replicated weights (same seed on every rank), rank-local token batch
-    Wb, bb = synth.make_w(cfg)
-    Xb = synth.make_x(cfg, seed=shard_seed(cfg, rank))
-    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
-    X, W, b = to_dev(Xb), to_dev(Wb), to_dev(bb)
-    T, K, N = cfg.T, cfg.K, cfg.N
-    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
-                        act_gran=cfg.act_gran, centering=cfg.centering,
-                        code_format=cfg.code_format, out_order=cfg.out_order)
     stream = torch.cuda.current_stream()
-
-    # offline: calibration + weight preparation (timed once, not part of the step)
-    absmax = torch.zeros(K, dtype=torch.float32, device=dev) if cfg.use_sigma else None
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record(stream)
-    if absmax is not None:
-        hq.hq_calib_act_absmax(desc, X, absmax)
-    layer = hq.HadamardQuantLinear(desc, W, b, absmax, cfg.alpha)
-    p1.record(stream)
-    torch.cuda.synchronize()
-    prep_ms = p0.elapsed_time(p1)
-
-    bufs = layer.buffers(T)
-    Y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
-    sig_inv = layer.sigma_inv if layer.use_sigma else None
-    mean_in = bufs["a_mean"] if cfg.centering else None
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-
-    def linear():
-        hq.hq_linear(desc, bufs["a_codes"], bufs["a_scale"], mean_in, layer.w_codes,
-                     layer.w_scale, layer.colsum, layer.bias_f32, Y)
-
-    launches_per_step = (2 if cfg.act_gran == 1 else 1) + 1
-
-    # Rotating inputs instead of an L2 flush inside the timed region: M copies
-    # of this rank's token batch, M * |X| > 2 x L2, and step i reads copy
-    # i % M, so every step's activations come from HBM.  The weights and the
-    # step's own intermediate codes stay L2-resident, as in a real layer.
-    x_bytes = X.numel() * X.element_size()
-    n_copies = int(min(512, max(2, -(-2 * l2 // x_bytes) + 1)))
-    Xs = [X] + [X.clone() for _ in range(n_copies - 1)]
-
-    def quantize_i(i):
-        hq.hq_quantize_act(desc, Xs[i % n_copies], sig_inv, bufs["a_codes"], bufs["a_scale"],
-                           bufs["a_mean"], layer.workspace)
-
-    for i in range(args.warmup):
-        quantize_i(i)
-        linear()
-    torch.cuda.synchronize()
-    status = hq.hq_check_device_error()
-    if status != 0:
-        raise RuntimeError(f"device error during warm-up: {hq.STATUS_NAMES.get(status)}")
-
-    # K steps captured back to back in one CUDA graph: no host launch cost and
-    # one pair of events around the whole timed region.  Two more graphs hold
-    # K launches of each kernel alone, for the per-kernel times.
-    def capture(do_q, do_l):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(args.steps):
-                if do_q:
-                    quantize_i(i)
-                if do_l:
-                    linear()
-        return g
-
-    g_step, g_quant, g_linear = capture(True, True), capture(True, False), capture(False, True)
-    for g in (g_step, g_quant, g_linear):
-        g.replay()
-    torch.cuda.synchronize()
 
     def timed(g):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -467,6 +554,16 @@ def run_hq(args):
         e1.record(stream)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1)
+
+    def check(where):
+        status = hq.hq_check_device_error()
+        if status != 0:
+            raise RuntimeError(f"device error {where}: {hq.STATUS_NAMES.get(status)}")
+
+    ctx = setup_layer(hq, torch, cfg, dev, rank, l2)
+    graphs = capture_layer_graphs(torch, ctx, args.steps, args.warmup)
+    check("during warm-up")
+    g_step, g_quant, g_linear = graphs
 
     clocks = ClockSampler(local)
     if world > 1:
@@ -480,9 +577,12 @@ def run_hq(args):
     clock_info = clocks.stop()
     q_total = timed(g_quant)
     g_total = timed(g_linear)
-    status = hq.hq_check_device_error()
-    if status != 0:
-        raise RuntimeError(f"device error in the timed region: {hq.STATUS_NAMES.get(status)}")
+    check("in the timed region")
+    del graphs, g_step, g_quant, g_linear
+    T, K, N = cfg.T, cfg.K, cfg.N
+    desc, layer, bufs, Xs, Y, W = (ctx[k] for k in ("desc", "layer", "bufs", "Xs", "Y", "W"))
+    n_copies = len(Xs)
+
     # context only, outside the timed step: the same layer unquantized, as one
     # cuBLAS bf16 GEMM (torch.matmul) over the same rotating inputs
     Yc = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
@@ -507,44 +607,18 @@ def run_hq(args):
     pk_times = [0.0, 0.0, 0.0]
     with_packed = cfg.code_format == 0 and cfg.a_bits <= 4 and not args.no_variants
     if with_packed:
+        pctx = dict(ctx)
         pdesc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
                              act_gran=cfg.act_gran, centering=cfg.centering,
                              code_format=hq.HQ_CODES_I4_PACKED, out_order=cfg.out_order)
-        player = hq.HadamardQuantLinear(pdesc, W, b, absmax, cfg.alpha)
-        pbufs = player.buffers(T)
-        pmean = pbufs["a_mean"] if cfg.centering else None
-
-        def pk_quant(i):
-            hq.hq_quantize_act(pdesc, Xs[i % n_copies], sig_inv, pbufs["a_codes"],
-                               pbufs["a_scale"], pbufs["a_mean"], player.workspace)
-
-        def pk_linear():
-            hq.hq_linear(pdesc, pbufs["a_codes"], pbufs["a_scale"], pmean, player.w_codes,
-                         player.w_scale, player.colsum, player.bias_f32, Y)
-
-        for i in range(args.warmup):
-            pk_quant(i)
-            pk_linear()
-        torch.cuda.synchronize()
-        pgs = []
-        for do_q, do_l in ((True, True), (True, False), (False, True)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for i in range(args.steps):
-                    if do_q:
-                        pk_quant(i)
-                    if do_l:
-                        pk_linear()
-            g.replay()
-            pgs.append(g)
-        torch.cuda.synchronize()
+        player = hq.HadamardQuantLinear(pdesc, W, ctx["b"], ctx["absmax"], cfg.alpha)
+        pctx.update(desc=pdesc, layer=player, bufs=player.buffers(T))
+        pgs = capture_layer_graphs(torch, pctx, args.steps, args.warmup)
         if world > 1:
             dist.barrier()
         pk_times = [timed(g) for g in pgs]
-        status = hq.hq_check_device_error()
-        if status != 0:
-            raise RuntimeError(f"device error in the packed variant: {hq.STATUS_NAMES.get(status)}")
-        del pgs, player, pbufs
+        check("in the packed variant")
+        del pgs, player, pctx
     (total_ms, q_total, g_total, c_total, pk_step, pk_q, pk_g) = max_over_ranks(
         [total_ms, q_total, g_total, c_total] + pk_times, world, dist, dev)
     ms_per_step = total_ms / args.steps
@@ -555,14 +629,14 @@ def run_hq(args):
     # H2D of X, quantize, GEMM, D2H of Y
     e2e = None
     if not args.no_e2e:
-        Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Xh = torch.from_numpy(ctx["Xb"].view(np.int16)).view(torch.bfloat16).pin_memory()
         Yh = torch.empty((T, N), dtype=torch.bfloat16).pin_memory()
-        Xd = torch.empty_like(X)
+        Xd = torch.empty_like(Xs[0])
 
         def e2e_body():
             # one public call: uploads, the layer's kernels and downloads of
             # row chunks overlapped on the library's copy streams
-            hq.hq_forward_host(desc, Xh, Xd, sig_inv, bufs["a_codes"], bufs["a_scale"],
+            hq.hq_forward_host(desc, Xh, Xd, ctx["sig_inv"], bufs["a_codes"], bufs["a_scale"],
                                bufs["a_mean"], layer.workspace, layer.w_codes, layer.w_scale,
                                layer.colsum, layer.bias_f32, Y, Yh, chunks=E2E_CHUNKS)
 
@@ -582,9 +656,8 @@ def run_hq(args):
                "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
                "d2h_bytes_per_step": int(Yh.numel() * Yh.element_size()),
                "ms_per_step": e2e_ms / args.steps}
-        status = hq.hq_check_device_error()
-        if status != 0:
-            raise RuntimeError(f"device error in the e2e region: {hq.STATUS_NAMES.get(status)}")
+        check("in the e2e region")
+        del g_e2e, Xh, Yh, Xd
 
     if world > 1:
         dist.destroy_process_group()
@@ -592,19 +665,26 @@ def run_hq(args):
         return 0
 
     peaks, peak_src = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    ceiling = measure_mma_ceiling(hq, torch)
+    check("in the MMA-only loop")
+    headline = kernel_record(hq, cfg, q_total / args.steps, g_total / args.steps,
+                             ms_per_step, peaks, ceiling)
     q_med = q_total / args.steps
     g_med = g_total / args.steps
-    q_gbs = quantizer_bytes(cfg) / (q_med * 1e-3) / 1e9
-    g_tops = ops / (g_med * 1e-3) / 1e12
-    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    q_gbs = headline["quantizer"]["GB/s"]
+    g_tops = headline["gemm"]["TOPS"]
     # the committed ncu summaries cover the configurations as defined, not overrides
     profiled = cfg == synth.CONFIGS[cfg.index]
     if g_med >= q_med:
-        roof = {"kernel": "hq_gemm_i8 (tcgen05 kind::i8 + epilogue)", "bound": "tensor",
+        roof = {"kernel": "hq_gemm_i8 (tcgen05 kind::i8 + epilogue, "
+                          f"{headline['gemm']['kernel']})", "bound": "tensor",
                 "achieved": g_tops, "peak": int8_peak, "unit": "TFLOP/s",
                 "frac": g_tops / int8_peak,
                 "traffic": profiled_traffic("gemm", cfg.index) if profiled else None,
                 "peak_source": f"{peak_src}: 2 x bf16_tflops (burst), dense int8:bf16 = 4.5:2.25",
+                "frac_of_mma_ceiling": headline["gemm"]["frac_mma_ceiling"],
+                "mma_ceiling_TOPS": headline["gemm"]["mma_ceiling_TOPS"],
                 "algorithmic": f"2*T*K*N = {ops:.4g} int ops per launch"}
     else:
         roof = {"kernel": "hq_quantize_act (fused FWHT quantizer)", "bound": "hbm",
@@ -613,6 +693,10 @@ def run_hq(args):
                 "traffic": profiled_traffic("quant", cfg.index) if profiled else None,
                 "peak_source": f"{peak_src} hbm_gbs",
                 "algorithmic": f"{quantizer_bytes(cfg):.4g} bytes per launch"}
+    kernels = {"quantizer": headline["quantizer"], "gemm": headline["gemm"],
+               "weight_prep_ms": ctx["prep_ms"]}
+    kernels["quantizer"]["traffic"] = profiled_traffic("quant", cfg.index) if profiled else None
+    kernels["gemm"]["traffic"] = profiled_traffic("gemm", cfg.index) if profiled else None
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -620,19 +704,14 @@ def run_hq(args):
         "dtype": "int8 (s8 x s8 -> s32; fp32 transform)", "data": "synthetic",
         "config": config_block(cfg, world),
         "roofline": roof,
-        "kernels": {
-            "quantizer": {"ms_per_launch": q_med, "GB/s": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
-                          "bytes": quantizer_bytes(cfg)},
-            "gemm": {"ms_per_launch": g_med, "TOPS": g_tops, "frac_int8": g_tops / int8_peak,
-                     "hbm_bytes": gemm_bytes(cfg)},
-            "weight_prep_ms": prep_ms,
-        },
+        "kernels": kernels,
+        "int8_ceiling": ceiling,
         "context": {"cublas_bf16_gemm": {
             "ms_per_launch": c_total / args.steps,
             "TFLOP/s": ops / (c_total / args.steps * 1e-3) / 1e12,
             "what": "torch.matmul(X, W^T) in bf16 (cuBLAS) on the same shape and inputs, "
                     "unquantized; context only, not on the path"}},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": ctx["launches_per_step"] * args.steps,
         "clocks": clock_info,
         "e2e": e2e,
     }
@@ -644,17 +723,16 @@ def run_hq(args):
                     "outputs bit-identical to the headline's",
             "value": job_throughput(ops, args.steps, world, pk_step), "unit": "TOPS",
             "ms_per_step": pk_step / args.steps,
-            "quantizer": {"ms_per_launch": pk_q / args.steps,
-                          "GB/s": quantizer_bytes(pcfg) / (pk_q / args.steps * 1e-3) / 1e9,
-                          "frac_hbm": quantizer_bytes(pcfg) / (pk_q / args.steps * 1e-3) / 1e9 /
-                                      peaks["hbm_gbs"],
-                          "bytes": quantizer_bytes(pcfg)},
-            "gemm": {"ms_per_launch": pk_g / args.steps,
-                     "TOPS": ops / (pk_g / args.steps * 1e-3) / 1e12,
-                     "frac_int8": ops / (pk_g / args.steps * 1e-3) / 1e12 / int8_peak,
-                     "hbm_bytes": gemm_bytes(pcfg)}}}
+            **kernel_record(hq, pcfg, pk_q / args.steps, pk_g / args.steps,
+                            pk_step / args.steps, peaks, ceiling)}}
+    host = (ctx["Xb"], ctx["Wb"], ctx["bb"])
+    del ctx, layer, bufs, Xs, Y, W
+    torch.cuda.empty_cache()
+    if not args.no_per_config and world == 1:
+        line["per_config"] = per_config_records(hq, torch, args, cfg, dev, l2, peaks, ceiling,
+                                                timed, check)
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(cfg, Xb, Wb, bb, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(cfg, *host, args.cpu_seconds)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -30,7 +30,7 @@ __all__ = [
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
     "hq_debug_set_gemm_variant", "HQ_GEMM_AUTO", "HQ_GEMM_SINGLE_CTA", "HQ_GEMM_CTA_PAIR",
-    "hq_quantize_act_noalloc", "hq_debug_plan", "HadamardQuantLinear",
+    "hq_quantize_act_noalloc", "hq_debug_plan", "hq_debug_mma_ceiling", "HadamardQuantLinear",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -47,7 +47,8 @@ STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARGUMENT", 2: "HQ_ERR_UNSUPPORTED
 EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare_weights",
             "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
             "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-            "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan")
+            "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan",
+            "hq_debug_mma_ceiling")
 
 
 class HQError(RuntimeError):
@@ -116,10 +117,12 @@ def load_library():
         _i32p = ctypes.POINTER(ctypes.c_int32)
         lib.hq_debug_plan.argtypes = [desc_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                       _i32p, _i32p, _i32p, _i32p]
+        lib.hq_debug_mma_ceiling.argtypes = [ctypes.c_int, ctypes.c_int64, _i32p, _vp]
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
                      "hq_forward_host",
                      "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
-                     "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan"):
+                     "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan",
+            "hq_debug_mma_ceiling"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -269,6 +272,17 @@ def hq_debug_plan(desc: LayerDesc, T: int, sms: int, pair_clusters: int) -> dict
                                         *(ctypes.byref(o) for o in out)), "hq_debug_plan")
     return {"quant_rows": out[0].value, "quant_threads": out[1].value,
             "gemm_pair": bool(out[2].value), "gemm_bn": out[3].value}
+
+
+def hq_debug_mma_ceiling(pair: bool, k_blocks: int, stream=None) -> int:
+    """Launches the MMA-only loop (int8 tensor-core ceiling) on the stream;
+    returns the number of CTAs launched (ops = ctas * k_blocks * 4 * 2 *
+    128 * 256 * 32)."""
+    lib = load_library()
+    n = ctypes.c_int32(0)
+    _check(lib.hq_debug_mma_ceiling(1 if pair else 0, int(k_blocks), ctypes.byref(n),
+                                    _stream(stream)), "hq_debug_mma_ceiling")
+    return int(n.value)
 
 
 def hq_debug_set_gemm_variant(variant: int):

@@ -755,6 +755,30 @@ hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_
   return HQ_OK;
 }
 
+hq_status hq_debug_mma_ceiling(int pair, int64_t k_blocks, int32_t* ctas, hq_stream_t stream) {
+  if ((pair != 0 && pair != 1) || k_blocks < 1 || k_blocks > (int64_t(1) << 24) || ctas == nullptr)
+    return HQ_ERR_INVALID_ARGUMENT;
+  DeviceState* dev;
+  hq_status s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  int n = dev->sm_count;
+  if (pair) {
+    if (dev->pair_clusters < 0) {
+      int c = 0;
+      if (gemm_pair_max_clusters(&c) != cudaSuccess) {
+        (void)cudaGetLastError();
+        c = 0;
+      }
+      dev->pair_clusters = c;
+    }
+    if (dev->pair_clusters <= 0) return HQ_ERR_UNSUPPORTED;
+    n = 2 * dev->pair_clusters;
+  }
+  *ctas = n;
+  return from_cuda(launch_mma_ceiling(pair != 0, k_blocks, n, dev->err, wait_ns(),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 hq_status hq_debug_inject_fault(int kind) {
   if (kind != HQ_FAULT_NONE && kind != HQ_FAULT_QUANT_WITHHOLD_ROW) return HQ_ERR_INVALID_ARGUMENT;
   std::lock_guard<std::mutex> lock(g_mutex);

@@ -975,6 +975,122 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------- tensor-core ceiling
+// The dense int8 rate of this device, measured: the GEMMs' main loop with
+// nothing but the MMAs.  Each CTA zeroes STAGES operand stages laid out
+// exactly as the GEMMs' (A 128 x 128 bytes, B 256 x 128 bytes per stage,
+// 128-byte swizzle), then one thread issues k_blocks x 4 MMAs of 128 x 256 x
+// 32 (kind::i8) into one tensor-memory accumulator, cycling through the
+// stages, commits and waits.  No loads, no epilogue: an upper bound for the
+// single-CTA GEMM.  The CTA-pair form (clusters of two, cta_group::2, M =
+// 256, N = 256, each CTA holding half of A and half of B) bounds the pair
+// GEMM.  The operands are zeros, so the accumulator ends at zero.
+struct CeilCfg {
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = 256 * BK;  // single CTA: 256 rows; pair: 128 of them used
+  static constexpr size_t SMEM = size_t(STAGES) * (A_BYTES + B_BYTES) + 1024 + 64;
+};
+
+template <bool PAIR>
+__global__ void __launch_bounds__(128, 1) mma_ceiling_kernel(int64_t k_blocks, unsigned int* err,
+                                                             unsigned long long wait_ns) {
+  using C = CeilCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + size_t(C::STAGES) * C::A_BYTES;
+  uint64_t* drain = reinterpret_cast<uint64_t*>(sB + size_t(C::STAGES) * C::B_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  const int warp = threadIdx.x >> 5;
+  const WaitCtl wc{err, wait_ns};
+  uint4* z = reinterpret_cast<uint4*>(smem);
+  const int n16 = C::STAGES * (C::A_BYTES + C::B_BYTES) / 16;
+  for (int i = threadIdx.x; i < n16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();  // the zeros precede the tensor cores' operand reads
+  if (threadIdx.x == 0) {
+    mbar_init(drain, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 0) {
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, 256);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 256);
+      tmem_relinquish();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) cluster_sync();
+  tc_fence_after();
+  const uint32_t d_tmem = *tmem_slot;
+  const bool issuer = threadIdx.x == 0 && (!PAIR || cluster_ctarank() == 0);
+  if (issuer) {
+    const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+    constexpr uint32_t idesc = PAIR ? i8_idesc(2 * BM, 256) : i8_idesc(BM, 256);
+    for (int64_t kb = 0; kb < k_blocks; ++kb) {
+      const int s = int(kb % C::STAGES);
+      const uint64_t adesc = sw128_kmajor_desc(a_base + uint32_t(s) * C::A_BYTES);
+      const uint64_t bdesc = sw128_kmajor_desc(b_base + uint32_t(s) * C::B_BYTES);
+#pragma unroll
+      for (int k = 0; k < BK / 32; ++k) {
+        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+        if constexpr (PAIR)
+          mma_i8_pair(d_tmem, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), idesc, accum);
+        else
+          mma_i8(d_tmem, adesc + uint64_t(2 * k), bdesc + uint64_t(2 * k), idesc, accum);
+      }
+    }
+    if constexpr (PAIR)
+      mma_commit_pair(drain, 0x3);
+    else
+      mma_commit(drain);
+  }
+  if (threadIdx.x == 0) (void)mbar_wait<PAIR>(drain, 0, wc);  // every MMA has completed
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    if constexpr (PAIR)
+      tmem_dealloc_pair(d_tmem, 256);
+    else
+      tmem_dealloc(d_tmem, 256);
+  }
+}
+
+cudaError_t launch_mma_ceiling(bool pair, int64_t k_blocks, int ctas, unsigned int* err,
+                               unsigned long long wait_ns, cudaStream_t st) {
+  static bool configured[2] = {false, false};
+  const void* fn = pair ? (const void*)mma_ceiling_kernel<true> : (const void*)mma_ceiling_kernel<false>;
+  if (!configured[pair ? 1 : 0]) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(CeilCfg::SMEM));
+    if (e != cudaSuccess) return e;
+    configured[pair ? 1 : 0] = true;
+  }
+  if (pair) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(ctas));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = CeilCfg::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, mma_ceiling_kernel<true>, k_blocks, err, wait_ns);
+  }
+  mma_ceiling_kernel<false><<<ctas, 128, CeilCfg::SMEM, st>>>(k_blocks, err, wait_ns);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ launch
 template <int BN, int LOGO, bool PK>
 static cudaError_t launch_bn(const void* tmap_a, const void* tmap_b, const void* tmap_y,

@@ -89,6 +89,12 @@ cudaError_t gemm_pair_max_clusters(int* clusters);
 size_t gemm_pair_smem_bytes();
 int gemm_pair_stages();
 
+// MMA-only loop (the int8 tensor-core ceiling): `ctas` CTAs (an even number
+// of them in clusters of two when pair), each issuing k_blocks x 4 MMAs of
+// 128 x 256 x 32 (pair: 256 x 256 x 32 per cluster, half per CTA).
+cudaError_t launch_mma_ceiling(bool pair, int64_t k_blocks, int ctas, unsigned int* err,
+                               unsigned long long wait_ns, cudaStream_t st);
+
 cudaError_t launch_col_absmax(const uint16_t* M, int64_t rows, int K, float* out, cudaStream_t st);
 cudaError_t launch_sigma_inv(const float* act_absmax, float* sigma_inv, int K, float alpha,
                              cudaStream_t st);

@@ -318,6 +318,21 @@ hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_
                         int32_t* quant_rows, int32_t* quant_threads, int32_t* gemm_pair,
                         int32_t* gemm_bn);
 
+/* Measurement hook (no counterpart on the pages): the int8 tensor-core
+ * ceiling of this device, the denominator the GEMM's throughput is reported
+ * against beside the nominal figure.  Launches the GEMM's main loop with
+ * nothing but the MMAs: every CTA (one per SM, resident at once) zeroes four
+ * operand stages laid out like the GEMM's and one thread issues k_blocks x 4
+ * tcgen05.mma kind::i8 of 128 x 256 x 32 into tensor memory (pair = 1:
+ * clusters of two CTAs issuing cta_group::2 MMAs of 256 x 256 x 32, the
+ * CTA-pair GEMM's shape), then waits for them.  No loads, no epilogue.
+ *   pair      0 or 1;  k_blocks  1 .. 2^24 (four MMAs each);
+ *   ctas      (host) receives the number of CTAs launched, so that one launch
+ *             performs ctas * k_blocks * 4 * 2 * 128 * 256 * 32 integer ops.
+ * Time the launch on `stream` with events.  Returns HQ_ERR_UNSUPPORTED for
+ * pair = 1 on a device that cannot hold a cluster of two such CTAs. */
+hq_status hq_debug_mma_ceiling(int pair, int64_t k_blocks, int32_t* ctas, hq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
