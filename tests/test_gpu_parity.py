@@ -678,10 +678,9 @@ def test_forward_host_equals_the_device_path(hq, idx, T, over, chunks):
     if cfg.use_sigma:
         absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
         hq.hq_calib_act_absmax(desc, X0, absmax)
+    static = 0.02 if cfg.act_gran == hq.HQ_PER_TENSOR_STATIC else None
     layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), absmax,
-                                   cfg.alpha)
-    if cfg.act_gran == hq.HQ_PER_TENSOR_STATIC:
-        layer.buffers(T)["a_scale"].fill_(0.02)
+                                   cfg.alpha, static_scale=static)
     inputs = [X0, torch.roll(X0, 131, dims=0).contiguous(), (X0 * 0.5).contiguous()]
 
     def reference(X):
