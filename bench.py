@@ -113,7 +113,8 @@ def gemm_bytes(cfg) -> float:
 E2E_CHUNKS = 8  # row chunks of the end-to-end pipeline (hq_forward_host)
 PROFILES = {("gemm", 2): "gemm_i8_cfg2_pixart_qkv.md", ("quant", 2): "quant_rows_cfg2_pixart_qkv.md"}
 KERNEL_SOURCES = {"gemm": ("hq_gemm.cu", "hq_device.cuh", "hq_kernels.h"),
-                  "quant": ("hq_quant.cu", "hq_device.cuh", "hq_kernels.h")}
+                  "quant": ("hq_quant_act.cu", "hq_quant_common.cuh", "hq_device.cuh",
+                            "hq_kernels.h")}
 
 
 def kernel_source_hash(kind, root=ROOT):

@@ -33,6 +33,7 @@ struct DeviceState {
   int cc_major = 0, cc_minor = 0;
   unsigned int* err = nullptr;
   bool quant_attr_set[11][4][3] = {};  // [log2 n][mode][centering]
+  bool qact_attr_set[6][11][4][3] = {};  // [kernel][log2 n][mode][centering] attributes set
   int pair_clusters = -1;  // co-resident clusters of the CTA-pair GEMM (-1: not queried)
   // hq_forward_host's upload and download streams (created on first use)
   cudaStream_t up = nullptr, down = nullptr;
@@ -232,6 +233,229 @@ hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, int center, cuda
   }
   void* args[] = {&L.p};
   return from_cuda(cudaLaunchKernel(fn, dim3(L.grid), dim3(L.threads), args, L.smem, st));
+}
+
+// ---------------------------------------------------------------------------
+// The TMA-fed activation quantizers (had_order >= 16).
+
+constexpr int kQActCtasPerSm = 2;
+constexpr size_t kQActSmemPerCta = size_t(228 / kQActCtasPerSm - 1) * 1024;
+
+// Rows of the [T*S, 32] view per tensor copy for a stage of RS rows: the
+// whole stage when it fits one box (at most 256 rows), else the largest
+// multiple of 8 rows that divides RS (so every copy starts on a 512-byte
+// boundary, where the 64-byte swizzle pattern starts over); 0 if none.
+int qact_box_rows(int RS) {
+  if (RS <= 256) return RS;
+  for (int br = 256; br >= 8; br -= 8)
+    if (RS % br == 0) return br;
+  return 0;
+}
+
+// Warp segments the longest row of a segment-kernel tile spans.
+int qact_max_seg(int R, int S) {
+  int m = 1;
+  for (int r = 0; r < R; ++r) {
+    const int n = (r * S + S - 1) / 32 - (r * S) / 32 + 1;
+    if (n > m) m = n;
+  }
+  return m;
+}
+
+// How hq_quantize_act runs for K channels, blocks of n and T tokens.
+struct ActPlan {
+  bool wrow;     // the warp-row kernel (else the segment kernel)
+  int spl;       // warp-row: slices a lane (0: several rows per warp)
+  int rpw;       // warp-row: rows per warp
+  int rows;      // rows per tile
+  int threads;   // per CTA (producer warp included)
+  int stages;    // ring stages
+  int max_seg;   // segment kernel: segments a row spans
+  size_t smem;   // dynamic shared memory per CTA
+};
+
+// Ring stages that fit beside `fixed` bytes (at most 6, at least 2; 0 if not).
+int qact_stages(size_t fixed, int rows, int S) {
+  const size_t stage = (size_t(rows) * S * 64 + 1023) / 1024 * 1024;
+  if (fixed + 2 * stage > kQActSmemPerCta) return 0;
+  const size_t st = (kQActSmemPerCta - fixed) / stage;
+  return int(st > 6 ? 6 : st);
+}
+
+// Warp-row kernel when every row fits a warp (K = 1024 spl, spl <= 4, or
+// K < 1024); otherwise the segment kernel with the tile shape of the
+// issue-bound cost model (tile rounds x CTAs on the busiest SM x threads per
+// CTA, the most threads within 3 % of the lowest cost).
+bool qact_plan(int K, int n, int centering, int64_t T, int sms, ActPlan* out) {
+  ActPlan& P = *out;
+  const int S = K / 32;
+  const bool pre = centering == HQ_CENTER_TOKEN_MEAN_PRE;
+  if ((S % 32 == 0 && S / 32 <= 4) || S < 32) {
+    P.wrow = true;
+    P.spl = S < 32 ? 0 : S / 32;
+    P.rpw = S < 32 ? 32 / S : 1;
+    const int nw = quant_wrow_warps(P.spl);
+    P.rows = nw * P.rpw;
+    P.threads = 32 * (nw + 1);
+    P.max_seg = 1;
+    if (qact_box_rows(P.rows * S) == 0) return false;
+    P.stages = qact_stages(quant_wrow_smem_bytes(P.rows, S, K, n, 0, nw, P.rpw), P.rows, S);
+    if (P.stages < 2) return false;
+    P.smem = quant_wrow_smem_bytes(P.rows, S, K, n, P.stages, nw, P.rpw);
+    return true;
+  }
+  P.wrow = false;
+  P.spl = 0;
+  P.rpw = 0;
+  const int maxC = quant_seg_max_consumers();
+  const int64_t slots = int64_t(sms) * kQActCtasPerSm;
+  auto stages_for = [&](int R) {
+    if (qact_box_rows(R * S) == 0) return 0;
+    return qact_stages(quant_seg_smem_bytes(R, S, K, n, 0, qact_max_seg(R, S), pre), R, S);
+  };
+  auto cost_of = [&](int R, int nt) {
+    const int64_t tiles = (T + R - 1) / R;
+    const int64_t grid = tiles < slots ? tiles : slots;
+    const int64_t rounds = (tiles + grid - 1) / grid;
+    const int64_t ctas_per_sm = (grid + sms - 1) / sms;
+    return double(rounds) * double(ctas_per_sm) * nt;
+  };
+  double lowest = 1e300;
+  for (int R = 1; R * S <= maxC; ++R) {
+    if (stages_for(R) < 2) continue;
+    const double c = cost_of(R, ((R * S + 31) / 32) * 32);
+    if (c < lowest) lowest = c;
+  }
+  int bestR = 0, bestNT = 0;
+  for (int R = 1; R * S <= maxC; ++R) {
+    if (stages_for(R) < 2) continue;
+    const int nt = ((R * S + 31) / 32) * 32;
+    if (cost_of(R, nt) <= lowest * 1.03 && nt > bestNT) {
+      bestR = R;
+      bestNT = nt;
+    }
+  }
+  if (bestR == 0) return false;
+  P.rows = bestR;
+  P.threads = bestNT + 32;
+  P.max_seg = qact_max_seg(bestR, S);
+  P.stages = stages_for(bestR);
+  P.smem = quant_seg_smem_bytes(bestR, S, K, n, P.stages, P.max_seg, pre);
+  return true;
+}
+
+hq_status encode_act_view(CUtensorMap* m, const void* X, int64_t T, int K, int box_rows) {
+  const int S = K / 32;
+  cuuint64_t dims[2] = {32u, cuuint64_t(T) * cuuint64_t(S)};
+  cuuint64_t strides[1] = {64u};
+  cuuint32_t box[2] = {32u, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
+struct QActLaunch {
+  QuantParams p;
+  CUtensorMap tmap;
+  ActPlan plan;
+  int grid;
+  int logn;
+};
+
+hq_status make_quant_act_launch(const DeviceState* dev, const hq_layer_desc* d, int64_t T,
+                                const uint16_t* X, QActLaunch* out) {
+  QActLaunch& L = *out;
+  std::memset(&L.p, 0, sizeof(L.p));
+  const int K = d->K, n = d->had_order;
+  if (!qact_plan(K, n, d->centering, T > 0 ? T : 1, dev->sm_count, &L.plan))
+    return HQ_ERR_UNSUPPORTED;
+  const ActPlan& P = L.plan;
+  const int S = K / 32;
+  if (T * int64_t(S) + int64_t(P.rows) * S >= (int64_t(1) << 31)) return HQ_ERR_UNSUPPORTED;
+  L.logn = ilog2_exact(n);
+  L.p.X = X;
+  L.p.T = T;
+  L.p.K = K;
+  L.p.S = S;
+  L.p.R = P.rows;
+  L.p.rpw = P.rpw;
+  L.p.inv_sqrt_n = float(1.0 / std::sqrt(double(n)));
+  L.p.sqrt_n = float(std::sqrt(double(n)));
+  L.p.err = dev->err;
+  L.p.wait_ns = wait_ns();
+  L.p.stages = P.stages;
+  L.p.box_rows = qact_box_rows(P.rows * S);
+  L.p.boxes = P.rows * S / L.p.box_rows;
+  L.p.max_seg = P.max_seg;
+  L.p.n_over_k = float(n) / float(K);
+  L.p.inv_k = 1.0f / float(K);
+  const int64_t ntiles = (T + P.rows - 1) / P.rows;
+  const int64_t slots = int64_t(dev->sm_count) * kQActCtasPerSm;
+  L.grid = int(ntiles < slots ? ntiles : slots);
+  return encode_act_view(&L.tmap, X, T, K, L.p.box_rows);
+}
+
+hq_status run_quant_act(DeviceState* dev, QActLaunch& L, int mode, int center, cudaStream_t st) {
+  const int logn = L.logn;
+  const ActPlan& P = L.plan;
+  const void* fn = P.wrow ? quant_wrow_kernel_ptr(logn, mode, center, P.spl)
+                          : quant_seg_kernel_ptr(logn, mode, center);
+  if (fn == nullptr) return HQ_ERR_UNSUPPORTED;
+  if (L.p.T <= 0) return HQ_OK;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    const int slot = P.wrow ? 1 + P.spl : 0;
+    bool& set = dev->qact_attr_set[slot][logn][mode][center];
+    if (!set) {
+      // kQActCtasPerSm CTAs of up to kQActSmemPerCta each: the largest
+      // shared-memory carveout
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(kQActSmemPerCta)) != cudaSuccess ||
+          cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+        return HQ_ERR_CUDA;
+      set = true;
+    }
+  }
+  void* args[] = {&L.tmap, &L.p};
+  return from_cuda(cudaLaunchKernel(fn, dim3(L.grid), dim3(P.threads), args, P.smem, st));
+}
+
+// hq_quantize_act with a Hadamard rotation along K: the TMA-fed kernel.
+hq_status quantize_act_tma(DeviceState* dev, const hq_layer_desc* desc, const uint16_t* X,
+                           int64_t T, const float* sigma_inv, int8_t* a_codes, float* a_scale,
+                           float* a_mean, void* workspace, cudaStream_t st) {
+  QActLaunch L;
+  hq_status s = make_quant_act_launch(dev, desc, T, X, &L);
+  if (s != HQ_OK) return s;
+  L.p.mult = sigma_inv;
+  L.p.invert_mult = 0;
+  L.p.codes = a_codes;
+  L.p.scale = a_scale;
+  L.p.mean = a_mean;
+  L.p.q = (1 << (desc->a_bits - 1)) - 1;
+  L.p.s_unit = L.p.inv_sqrt_n / float(L.p.q);
+  L.p.packed = desc->code_format == HQ_CODES_I4_PACKED ? 1 : 0;
+  L.p.fault_withhold_row = g_fault == HQ_FAULT_QUANT_WITHHOLD_ROW ? 1 : 0;
+  const int center = desc->centering;
+  if (desc->act_gran == HQ_PER_TOKEN) return run_quant_act(dev, L, 0, center, st);
+  if (desc->act_gran == HQ_PER_TENSOR_STATIC) {
+    L.p.static_scale = a_scale;
+    L.p.scale = nullptr;
+    return run_quant_act(dev, L, 3, center, st);
+  }
+  // dynamic per tensor: pass 1 finds max |V| over the tensor, pass 2 quantizes
+  L.p.tensor_max = static_cast<unsigned int*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, 16, st) != cudaSuccess) return HQ_ERR_CUDA;
+  QActLaunch L1 = L;
+  L1.p.codes = nullptr;
+  L1.p.mean = nullptr;
+  L1.p.fault_withhold_row = 0;
+  s = run_quant_act(dev, L1, 1, center, st);
+  if (s != HQ_OK) return s;
+  return run_quant_act(dev, L, 2, center, st);
 }
 
 hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
@@ -488,6 +712,8 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   s = device_state(&dev);
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (desc->had_order >= 16) return quantize_act_tma(dev, desc, X, T, sigma_inv, a_codes, a_scale,
+                                                     a_mean, workspace, st);
   QuantLaunch L;
   s = make_quant_launch(dev, desc->K, desc->had_order, T, X, &L);
   if (s != HQ_OK) return s;

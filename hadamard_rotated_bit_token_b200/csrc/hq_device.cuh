@@ -117,6 +117,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// As mbar_wait, for waits that are usually short and on the critical path:
+// spins on try_wait (which itself parks the thread in hardware until the
+// phase completes or a short system time limit passes) and reads the clock
+// only every 32 unsuccessful tries, so no software sleep is inserted.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > w.limit_ns) {
+      report_error(w.err, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Hardware named barrier `id` among `nthreads` threads (whole warps, each
+// converged at the call).  No timeout: callers make sure every participant
+// arrives, on every path.
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Counts `bytes` as transferred on the mbarrier without a copy (cancels an
 // expectation whose copy was never issued).
 __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {

@@ -29,6 +29,15 @@ struct QuantParams {
   int fault_withhold_row;     // test hook: never release the first row of the first tile
   unsigned int* err;          // device error word
   unsigned long long wait_ns; // bounded-wait limit
+  // TMA-fed activation kernels only (hq_quant_act.cu)
+  int stages;                 // shared-memory ring stages of R rows each
+  int box_rows;               // rows of the [T*K/32, 32] view per tensor copy (S or S/2)
+  int boxes;                  // tensor copies per stage (R * S / box_rows)
+  int max_seg;                // warp segments a row can span (slots per row)
+  int rpw;                    // warp-row kernel with S < 32: rows per warp
+  float n_over_k;             // n / K (the rotated row's mean from its blocks' first channels)
+  float inv_k;                // 1 / K
+  float s_unit;               // 1 / (q sqrt(n)): reported scale per unit of max |V_hat|
 };
 
 // Returns the kernel entry for log2(n) in [4,10] (or 0: n = 1, no rotation,
@@ -38,9 +47,28 @@ struct QuantParams {
 // whole warps, at most quant_max_threads()).
 const void* quant_kernel_ptr(int logn, int mode, int center);
 int quant_max_threads();
+
 // Dynamic shared memory of one quantizer CTA: R rows per tile, K channels,
-// B blocks per row, `nwarps` warps, transposes for n >= 64.
+// B blocks per row, `nwarps` warps, transposes for n >= 256.
 size_t quant_smem_bytes(int R, int K, int B, int nwarps, bool xpose);
+
+// The TMA-fed activation quantizers (hq_quant_act.cu): one producer warp
+// streams tiles of rows into a ring of shared-memory stages through a tensor
+// map over X viewed as [T*K/32, 32] bf16 (64-byte rows, 64-byte swizzle, box
+// {32, box_rows}); each kernel takes (const CUtensorMap tmX, QuantParams p).
+// log2(n) in [4, 10], mode in [0, 3], centering in [0, 2].
+//   segment kernel: any K (a multiple of 32); R * S consumer threads, one per
+//     32-channel slice of each of the tile's R rows, 32 more for the producer.
+//   warp-row kernel: warps own whole rows; spl = K / 1024 in [1, 4] slices a
+//     lane and one row per warp, or spl = 0 for S = K/32 < 32: p.rpw rows
+//     of S lanes each per warp; quant_wrow_warps(spl) consumer warps.
+const void* quant_seg_kernel_ptr(int logn, int mode, int center);
+const void* quant_wrow_kernel_ptr(int logn, int mode, int center, int spl);
+int quant_seg_max_consumers();
+int quant_wrow_warps(int spl);
+// Dynamic shared memory of one CTA (n = Hadamard order; rows per tile).
+size_t quant_seg_smem_bytes(int R, int S, int K, int n, int stages, int max_seg, bool pre);
+size_t quant_wrow_smem_bytes(int rows, int S, int K, int n, int stages, int ncw, int rpw);
 
 struct GemmParams {
   const float* a_scale;   // [T] or [1]

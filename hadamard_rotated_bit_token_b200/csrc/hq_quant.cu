@@ -128,8 +128,6 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int R, int K, int B, int 
   L.y0 = off;  // [2][R][padded B] first channel of every block
   off += 4u * 2 * R * padded_blocks(B);
   off = align_up(off, 8);
-  L.rowbar = off;
-  off += 8u * R;
   L.flags = off;  // [0] abort, [1] CTA max (mode 1)
   off += 16;
   L.total = off;

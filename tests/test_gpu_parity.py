@@ -60,8 +60,13 @@ def _check_act(ref, codes, scale, mean, per_row=True, min_match=None, what="act"
 # ---------------------------------------------------------------------------
 
 SMALL = []
+# K below 1024 (several rows per warp), K = 1024 .. 4096 in whole warps of
+# slices (one row per warp, one to four slices a lane), and other K (rows
+# spanning warps)
 for i, (n, B) in enumerate([(16, 4), (16, 12), (32, 2), (32, 6), (64, 1), (64, 5), (128, 1),
-                            (128, 9), (256, 1), (256, 3), (512, 2), (1024, 1), (1024, 3)]):
+                            (128, 9), (256, 1), (256, 3), (512, 2), (1024, 1), (1024, 3),
+                            (16, 128), (128, 16), (1024, 2), (64, 64), (256, 16), (512, 8),
+                            (1024, 5)]):
     for T in (1, 7, 129, 300):
         bits = (4, 3, 8)[(i + T) % 3]
         SMALL.append((n * B, n, T, bits, (i + T) % 2, (i % 3) != 0))
@@ -70,7 +75,8 @@ for i, (n, B) in enumerate([(16, 4), (16, 12), (32, 2), (32, 6), (64, 1), (64, 5
 # the mean removed before the rotation (HQ_CENTER_TOKEN_MEAN_PRE), every order
 SMALL_PRE = [(n * B, n, T, (4, 3, 8)[i % 3], 2, i % 2 == 0)
              for i, (n, B, T) in enumerate([(16, 4, 129), (32, 6, 7), (64, 5, 300), (128, 9, 129),
-                                            (256, 3, 300), (512, 2, 7), (1024, 3, 129)])]
+                                            (256, 3, 300), (512, 2, 7), (1024, 3, 129),
+                                            (128, 16, 129), (1024, 4, 7), (1024, 5, 129)])]
 
 
 @pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL + SMALL_PRE)
