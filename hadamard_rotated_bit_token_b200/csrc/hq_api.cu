@@ -238,8 +238,10 @@ hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, int center, cuda
 // ---------------------------------------------------------------------------
 // The TMA-fed activation quantizers (had_order >= 16).
 
+// CTAs of the warp-row kernel per SM, and the shared memory each may use
 constexpr int kQActCtasPerSm = 2;
 constexpr size_t kQActSmemPerCta = size_t(228 / kQActCtasPerSm - 1) * 1024;
+size_t seg_smem_per_cta() { return size_t(228 / quant_seg_ctas_per_sm() - 1) * 1024; }
 
 // Rows of the [T*S, 32] view per tensor copy for a stage of RS rows: the
 // whole stage when it fits one box (at most 256 rows), else the largest
@@ -274,11 +276,12 @@ struct ActPlan {
   size_t smem;   // dynamic shared memory per CTA
 };
 
-// Ring stages that fit beside `fixed` bytes (at most 6, at least 2; 0 if not).
-int qact_stages(size_t fixed, int rows, int S) {
+// Ring stages that fit beside `fixed` bytes in `budget` (at most 6, at least
+// 2; 0 if not).
+int qact_stages(size_t fixed, int rows, int S, size_t budget = kQActSmemPerCta) {
   const size_t stage = (size_t(rows) * S * 64 + 1023) / 1024 * 1024;
-  if (fixed + 2 * stage > kQActSmemPerCta) return 0;
-  const size_t st = (kQActSmemPerCta - fixed) / stage;
+  if (fixed + 2 * stage > budget) return 0;
+  const size_t st = (budget - fixed) / stage;
   return int(st > 6 ? 6 : st);
 }
 
@@ -308,10 +311,11 @@ bool qact_plan(int K, int n, int centering, int64_t T, int sms, ActPlan* out) {
   P.spl = 0;
   P.rpw = 0;
   const int maxC = quant_seg_max_consumers();
-  const int64_t slots = int64_t(sms) * kQActCtasPerSm;
+  const int64_t slots = int64_t(sms) * quant_seg_ctas_per_sm();
   auto stages_for = [&](int R) {
     if (qact_box_rows(R * S) == 0) return 0;
-    return qact_stages(quant_seg_smem_bytes(R, S, K, n, 0, qact_max_seg(R, S), pre), R, S);
+    return qact_stages(quant_seg_smem_bytes(R, S, K, n, 0, qact_max_seg(R, S), pre), R, S,
+                       seg_smem_per_cta());
   };
   auto cost_of = [&](int R, int nt) {
     const int64_t tiles = (T + R - 1) / R;
@@ -392,7 +396,8 @@ hq_status make_quant_act_launch(const DeviceState* dev, const hq_layer_desc* d, 
   L.p.n_over_k = float(n) / float(K);
   L.p.inv_k = 1.0f / float(K);
   const int64_t ntiles = (T + P.rows - 1) / P.rows;
-  const int64_t slots = int64_t(dev->sm_count) * kQActCtasPerSm;
+  const int64_t slots =
+      int64_t(dev->sm_count) * (P.wrow ? kQActCtasPerSm : quant_seg_ctas_per_sm());
   L.grid = int(ntiles < slots ? ntiles : slots);
   return encode_act_view(&L.tmap, X, T, K, L.p.box_rows);
 }
@@ -412,7 +417,7 @@ hq_status run_quant_act(DeviceState* dev, QActLaunch& L, int mode, int center, c
       // kQActCtasPerSm CTAs of up to kQActSmemPerCta each: the largest
       // shared-memory carveout
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(kQActSmemPerCta)) != cudaSuccess ||
+                               int(P.wrow ? kQActSmemPerCta : seg_smem_per_cta())) != cudaSuccess ||
           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
         return HQ_ERR_CUDA;
@@ -712,8 +717,12 @@ hq_status hq_quantize_act(const hq_layer_desc* desc, const uint16_t* X, int64_t 
   s = device_state(&dev);
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (desc->had_order >= 16) return quantize_act_tma(dev, desc, X, T, sigma_inv, a_codes, a_scale,
-                                                     a_mean, workspace, st);
+  // rotated activations: the TMA-fed kernels, whenever a tile of them fits
+  // (every K up to 8192); otherwise, and without a rotation, the row kernel
+  ActPlan ap;
+  if (desc->had_order >= 16 &&
+      qact_plan(desc->K, desc->had_order, desc->centering, T, dev->sm_count, &ap))
+    return quantize_act_tma(dev, desc, X, T, sigma_inv, a_codes, a_scale, a_mean, workspace, st);
   QuantLaunch L;
   s = make_quant_launch(dev, desc->K, desc->had_order, T, X, &L);
   if (s != HQ_OK) return s;
@@ -970,7 +979,13 @@ hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_
   if (s != HQ_OK) return s;
   if (T < 1 || sms < 1 || pair_clusters < 0) return HQ_ERR_INVALID_ARGUMENT;
   int R, nt;
-  quant_shape(desc->K, T, sms, kQuantCtasPerSm, &R, &nt);
+  ActPlan ap;
+  if (desc->had_order >= 16 && qact_plan(desc->K, desc->had_order, desc->centering, T, sms, &ap)) {
+    R = ap.rows;  // the TMA-fed kernels
+    nt = ap.threads;
+  } else {
+    quant_shape(desc->K, T, sms, kQuantCtasPerSm, &R, &nt);
+  }
   const int logo = ilog2_exact(desc->out_order > 1 ? desc->out_order : 1);
   const GemmChoice gc = choose_gemm(T, desc->N, desc->K, sms, pair_clusters, HQ_GEMM_AUTO, logo,
                                     desc->code_format == HQ_CODES_I4_PACKED);

@@ -65,6 +65,7 @@ size_t quant_smem_bytes(int R, int K, int B, int nwarps, bool xpose);
 const void* quant_seg_kernel_ptr(int logn, int mode, int center);
 const void* quant_wrow_kernel_ptr(int logn, int mode, int center, int spl);
 int quant_seg_max_consumers();
+int quant_seg_ctas_per_sm();
 int quant_wrow_warps(int spl);
 // Dynamic shared memory of one CTA (n = Hadamard order; rows per tile).
 size_t quant_seg_smem_bytes(int R, int S, int K, int n, int stages, int max_seg, bool pre);

@@ -43,24 +43,35 @@ using namespace qc;
 namespace {
 
 // ------------------------------------------------------------ shared parts
-constexpr int kSegConsumers = 256;  // segment kernel: 8 consumer warps, 2 CTAs per SM
+#ifndef HQ_SEG_CTAS
+#define HQ_SEG_CTAS 2
+#endif
+#ifndef HQ_SEG_CONSUMERS
+#define HQ_SEG_CONSUMERS 256
+#endif
+constexpr int kSegConsumers = HQ_SEG_CONSUMERS;  // segment kernel: 8 consumer warps, 2 CTAs per SM
 constexpr int kSegThreads = kSegConsumers + 32;
+constexpr int kSegCtas = HQ_SEG_CTAS;
 
 // Shared-memory layout (byte offsets from a 1024-aligned base): the ring of
 // stages first, then the channel multipliers, the per-warp transpose
 // buffers, the row statistics, the barriers and flags.
 struct ActSmem {
-  uint32_t stage_bytes, mult, xbuf, slots, y0, full, empty, flags, total;
+  uint32_t stage_bytes, park, mult, xbuf, slots, y0, full, empty, stat, flags, total;
 };
 
 // rows: rows per tile; ncw: consumer warps; slot_f4: float4 slots (segment
-// kernel); y0_floats: floats of mean terms.
+// kernel); y0_floats: floats of mean terms; park_bytes: parked transformed
+// slices (segment kernel); stat_bars: tile-statistics barriers.
 __host__ __device__ inline ActSmem act_smem_layout(int rows, int S, int K, int stages, int ncw,
                                                    uint32_t xbuf_per_warp, int slot_f4,
-                                                   int y0_floats) {
+                                                   int y0_floats, uint32_t park_bytes = 0,
+                                                   int stat_bars = 0) {
   ActSmem L;
   L.stage_bytes = align_up(uint32_t(rows * S * 64), 1024u);
   uint32_t off = uint32_t(stages) * L.stage_bytes;
+  L.park = off;  // 1024-aligned
+  off += park_bytes;
   L.mult = off;  // chunk-major [8][S] float4
   off += 4u * K;
   L.xbuf = off;
@@ -75,6 +86,8 @@ __host__ __device__ inline ActSmem act_smem_layout(int rows, int S, int K, int s
   off += 8u * stages;
   L.empty = off;
   off += 8u * stages;
+  L.stat = off;
+  off += 8u * stat_bars;
   L.flags = off;  // [1] CTA max (mode 1), [2 + tile parity] consumers stop
   off += 16;
   L.total = off + 1024;  // room to align the dynamic base
@@ -360,7 +373,7 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
 // ------------------------------------------------------------ segment kernel
 // Any K: consumer c owns slice c % S of row c / S of every tile (p.R rows).
 template <int LOGN, int MODE, int CM>
-__global__ void __launch_bounds__(kSegThreads, 2)
+__global__ void __launch_bounds__(kSegThreads, kSegCtas)
     quant_seg_kernel(const __grid_constant__ CUtensorMap tmX, const QuantParams p) {
   using F = Fwht<LOGN>;
   constexpr bool CENTER = (CM == 1);
@@ -650,15 +663,17 @@ int quant_wrow_warps(int spl) {
   }
 }
 
+int quant_seg_ctas_per_sm() { return kSegCtas; }
+
 size_t quant_seg_smem_bytes(int R, int S, int K, int n, int stages, int max_seg, bool pre) {
   const int ncw = (R * S + 31) / 32;
-  const uint32_t xb = n >= 64 ? 4096u : 0u;
+  const uint32_t xb = n >= (1 << HQ_XPOSE_MIN_LOGN) && n >= 64 ? 4096u : 0u;
   return act_smem_layout(R, S, K, stages, ncw, xb, 2 * R * max_seg * (pre ? 2 : 1),
                          2 * R * padded_blocks(K / n)).total;
 }
 
 size_t quant_wrow_smem_bytes(int rows, int S, int K, int n, int stages, int ncw, int rpw) {
-  const uint32_t xb = n >= 64 ? 4096u : 0u;
+  const uint32_t xb = n >= (1 << HQ_XPOSE_MIN_LOGN) && n >= 64 ? 4096u : 0u;
   return act_smem_layout(rows, S, K, stages, ncw, xb, 0, ncw * rpw * padded_blocks(K / n)).total;
 }
 #endif

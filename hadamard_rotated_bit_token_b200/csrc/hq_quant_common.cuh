@@ -18,14 +18,18 @@
 // place in the thread's slice (register bits); bits 5 .. LOGN-1 select the
 // slice among the TT = n/32 slices of the block and equal the low bits of the
 // thread's lane (a block's slices sit in TT consecutive, aligned lanes).
-// The cross-thread bits go through one shared-memory transpose among G = 2^LX
-// lanes (up to three bits, n >= 64) and warp shuffles for the rest
-// (n = 512, 1024).
+// The cross-thread bits go through warp shuffles for n <= 128 (at most two
+// bits); for n >= 256 the first three through one shared-memory transpose
+// among G = 2^LX lanes and the rest (n = 512, 1024) through shuffles.
 #pragma once
 
 #include <cstdint>
 
 #include "hq_device.cuh"
+
+#ifndef HQ_XPOSE_MIN_LOGN
+#define HQ_XPOSE_MIN_LOGN 8
+#endif
 
 namespace hq {
 namespace qc {
@@ -74,7 +78,8 @@ struct Fwht {
   static constexpr int LREG = LOGN < 5 ? LOGN : 5;        // index bits inside the slice
   static constexpr int LOG_TT = LOGN > 5 ? LOGN - 5 : 0;  // index bits across lanes
   static constexpr int TT = 1 << LOG_TT;                  // slices (lanes) per block
-  static constexpr int LX = LOGN <= 5 ? 0 : (LOG_TT < 3 ? LOG_TT : 3);  // transposed bits
+  // transposed bits: from n = 2^HQ_XPOSE_MIN_LOGN on (shuffles below)
+  static constexpr int LX = LOGN < HQ_XPOSE_MIN_LOGN ? 0 : (LOG_TT < 3 ? LOG_TT : 3);
   static constexpr int G = 1 << LX;       // lanes per transpose group
   static constexpr int GS = 32 / G;       // elements per register group
   static constexpr int GP = GS / 2;       // fp32 pairs per register group

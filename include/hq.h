@@ -296,10 +296,12 @@ hq_status hq_debug_set_gemm_variant(int variant);
 /* Test hook for the bounded-wait error path, without faulting the GPU:
  *   HQ_FAULT_NONE (0)                    normal operation;
  *   HQ_FAULT_QUANT_WITHHOLD_ROW (1)      in each CTA of the next activation
- *       quantize launches, the statistics of the first row of the first
- *       tile are never released, so the threads of that row wait on a
- *       barrier that never completes; the bounded wait expires, the kernel
- *       records HQ_ERR_TIMEOUT and exits (it has no copies in flight).
+ *       quantize launches, one wait never completes: with a rotation along K
+ *       (had_order >= 16, K <= 8192) the copy of the CTA's first tile of
+ *       rows into shared memory is never issued, so its consumers' bounded
+ *       wait for it expires; otherwise the statistics of the first row of
+ *       the first tile are never released.  The kernel records
+ *       HQ_ERR_TIMEOUT, waits for the copies it did issue and exits.
  * Host state, applies to launches issued after the call. */
 enum { HQ_FAULT_NONE = 0, HQ_FAULT_QUANT_WITHHOLD_ROW = 1 };
 hq_status hq_debug_inject_fault(int kind);

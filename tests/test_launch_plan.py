@@ -22,22 +22,25 @@ def _plan(hq, K, N, n, T, **kw):
 
 
 def test_measured_choices_for_the_configurations(hq):
-    # config 2: 7-row tiles (1171 tiles fill the last round of 296 CTAs),
-    # 192-column GEMM tiles
-    assert _plan(hq, 1152, 3456, 128, 8192) == {"quant_rows": 7, "quant_threads": 256,
+    # config 2: rows of 36 slices span warps (segment kernel): 7-row tiles,
+    # 252 consumers in 8 warps plus the producer warp; 192-column GEMM tiles
+    assert _plan(hq, 1152, 3456, 128, 8192) == {"quant_rows": 7, "quant_threads": 288,
                                                  "gemm_pair": False, "gemm_bn": 192}
-    # config 3: 2 rows of 144 slices; N = 1152 is not a whole number of pair tiles
+    # config 3: one row of 144 slices per tile (5 consumer warps);
+    # N = 1152 is not a whole number of pair tiles
     p = _plan(hq, 4608, 1152, 256, 8192, a_bits=3)
-    assert (p["quant_rows"], p["quant_threads"], p["gemm_pair"], p["gemm_bn"]) == (2, 288, False, 192)
-    # config 4: per-tensor W8A8 1x1 convolution
+    assert (p["quant_rows"], p["quant_threads"], p["gemm_pair"], p["gemm_bn"]) == (1, 192, False, 192)
+    # config 4: rows of 10 slices, three to a warp (warp-row kernel): 24 rows
+    # per tile over 8 consumer warps
     p = _plan(hq, 320, 320, 64, 65536, a_bits=8, w_bits=8, act_gran=1, centering=0)
-    assert (p["quant_rows"], p["quant_threads"], p["gemm_bn"]) == (32, 320, 192)
-    # config 5: long K over N in whole 256-column tiles takes the CTA pair,
-    # and R = 3 (not the 2 % cheaper R = 2, measured slower)
-    assert _plan(hq, 3072, 12288, 1024, 16384) == {"quant_rows": 3, "quant_threads": 288,
+    assert (p["quant_rows"], p["quant_threads"], p["gemm_bn"]) == (24, 288, 192)
+    # config 5: three slices a lane, one row per warp, 4 consumer warps;
+    # long K over N in whole 256-column tiles takes the CTA pair
+    assert _plan(hq, 3072, 12288, 1024, 16384) == {"quant_rows": 4, "quant_threads": 160,
                                                     "gemm_pair": True, "gemm_bn": 256}
-    # config 1: one small wave
-    assert _plan(hq, 1024, 1024, 1024, 256)["gemm_bn"] == 64
+    # config 1: one row per warp, 8 consumer warps; one small GEMM wave
+    p = _plan(hq, 1024, 1024, 1024, 256)
+    assert (p["quant_rows"], p["quant_threads"], p["gemm_bn"]) == (8, 288, 64)
 
 
 def test_forms_that_exclude_the_pair_or_wide_tiles(hq):
@@ -62,7 +65,15 @@ def test_plan_invariants_over_shapes(hq):
         p = _plan(hq, K, N, n, T, code_format=packed)
         S = K // 32
         R, nt = p["quant_rows"], p["quant_threads"]
-        assert R >= 1 and R * S <= 320 and nt % 32 == 0 and R * S <= nt < R * S + 32
+        assert R >= 1 and nt % 32 == 0
+        if S < 32:  # warp-row kernel, several rows per warp, plus the producer warp
+            assert R == (nt // 32 - 1) * (32 // S)
+        elif S % 32 == 0 and S <= 128:  # warp-row kernel, one row per warp
+            assert R == nt // 32 - 1
+        elif R * S <= 256:  # segment kernel: one thread per slice, plus the producer warp
+            assert R * S + 32 <= nt < R * S + 64
+        else:  # the row kernel (K above 8192): one thread per slice
+            assert R * S <= nt < R * S + 32 and R * S <= 320
         assert p["gemm_bn"] in (64, 128, 192, 256)
         if packed:
             assert not p["gemm_pair"] and p["gemm_bn"] <= 192
