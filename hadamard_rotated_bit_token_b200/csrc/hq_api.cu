@@ -140,6 +140,10 @@ hq_status check_desc(const hq_layer_desc* d) {
 hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
 
 constexpr int kQuantCtasPerSm = 2;  // quantizer CTAs per SM (its launch bounds)
+#ifndef HQ_GROUP_M
+#define HQ_GROUP_M 8
+#endif
+constexpr int kGroupM = HQ_GROUP_M;  // M tiles per group of the GEMM's tile order
 
 // Rows per tile R and threads per CTA (one thread per 32-channel slice of
 // each row, whole warps).  The kernel is issue-bound, so an SM's time is
@@ -820,6 +824,8 @@ hq_status hq_linear(const hq_layer_desc* desc, int64_t T, const int8_t* a_codes,
   p.err = dev->err;
   p.wait_ns = wait_ns();
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // tile order: groups of kGroupM M tiles (shared A and B tiles stay in L2)
+  p.group_m = kGroupM;
   if (gc.pair) {
     p.num_m_tiles = int((T + 255) / 256);
     p.num_n_tiles = (N + 255) / 256;

@@ -106,6 +106,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Output tile `tile` -> (M tile, N tile) in groups of p.group_m M tiles: the
+// tiles of a group run N tile by N tile over the group's M tiles, so the CTAs
+// working at one time share a few M tiles of A and a few N tiles of B, which
+// stay in L2 while the output streams past (plain M-fastest order sweeps all
+// of A every round of tiles, and the output evicts it).
+__device__ __forceinline__ int tile_m(const GemmParams& p, int tile) {
+  const int gsize = p.group_m * p.num_n_tiles;
+  const int first = (tile / gsize) * p.group_m;
+  const int gm = min(p.num_m_tiles - first, p.group_m);
+  return first + (tile % gsize) % gm;
+}
+__device__ __forceinline__ int tile_n(const GemmParams& p, int tile) {
+  const int gsize = p.group_m * p.num_n_tiles;
+  const int first = (tile / gsize) * p.group_m;
+  const int gm = min(p.num_m_tiles - first, p.group_m);
+  return (tile % gsize) / gm;
+}
+
 // ------------------------------------------------------- parameter ring
 // Slot a holds the columns [n0, n0 + W) of one output tile: s_w at [0, W),
 // colsum at [W, 2W), bias at [2W, 3W) (fp32).  An absent vector, and every
@@ -495,8 +513,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
       int issued = 0, tiles_issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_idx = tile % p.num_m_tiles;
-        const int n_idx = tile / p.num_m_tiles;
+        const int m_idx = tile_m(p, tile);
+        const int n_idx = tile_n(p, tile);
         const int a = tiles_issued & 1;
         if (*abort_flag || !mbar_wait(&pempty[a], ((tiles_issued >> 1) & 1) ^ 1u, wc)) {
           *abort_flag = 1;
@@ -601,13 +619,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
     int acc_iter = 0;
     float sx_next = 0.0f, mt_next = 0.0f;
     if (int(blockIdx.x) < num_tiles)
-      load_row_params(p, int64_t(int(blockIdx.x) % p.num_m_tiles) * BM + quarter * 32 + lane,
+      load_row_params(p, int64_t(tile_m(p, int(blockIdx.x))) * BM + quarter * 32 + lane,
                       sx_next, mt_next);
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++acc_iter) {
       const int acc = acc_iter & 1;
       const uint32_t acc_phase = (acc_iter >> 1) & 1;
-      const int m_idx = tile % p.num_m_tiles;
-      const int n_idx = tile / p.num_m_tiles;
+      const int m_idx = tile_m(p, tile);
+      const int n_idx = tile_n(p, tile);
       EpiTile e;
       e.row0 = m_idx * BM + quarter * 32;
       e.col_base = n_idx * BN + half * C::HC;
@@ -617,7 +635,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
       e.mt = mt_next;
       const int next = tile + int(gridDim.x);
       if (next < num_tiles)  // next tile's row parameters, in flight during this one
-        load_row_params(p, int64_t(next % p.num_m_tiles) * BM + quarter * 32 + lane, sx_next,
+        load_row_params(p, int64_t(tile_m(p, next)) * BM + quarter * 32 + lane, sx_next,
                         mt_next);
       const bool got = !(*abort_flag) && mbar_wait(&tfull[acc], acc_phase, wc) &&
                        mbar_wait(&pfull[acc], acc_phase, wc);
@@ -814,8 +832,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int issued = 0, tiles_issued = 0;
       bool ok = true;
       for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-        const int m_idx = tile % p.num_m_tiles;
-        const int n_idx = tile / p.num_m_tiles;
+        const int m_idx = tile_m(p, tile);
+        const int n_idx = tile_n(p, tile);
         const int a_row = m_idx * C::BM_PAIR + int(rank) * BM;
         const int b_row = n_idx * C::BN + int(rank) * C::B_ROWS;
         const int a = tiles_issued & 1;
@@ -909,13 +927,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int acc_iter = 0;
     float sx_next = 0.0f, mt_next = 0.0f;
     if (cluster_id < num_tiles)
-      load_row_params(p, int64_t(cluster_id % p.num_m_tiles) * C::BM_PAIR + row_off, sx_next,
+      load_row_params(p, int64_t(tile_m(p, cluster_id)) * C::BM_PAIR + row_off, sx_next,
                       mt_next);
     for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++acc_iter) {
       const int acc = acc_iter & 1;
       const uint32_t acc_phase = (acc_iter >> 1) & 1;
-      const int m_idx = tile % p.num_m_tiles;
-      const int n_idx = tile / p.num_m_tiles;
+      const int m_idx = tile_m(p, tile);
+      const int n_idx = tile_n(p, tile);
       EpiTile e;
       e.row0 = m_idx * C::BM_PAIR + int(rank) * BM + quarter * 32;
       e.col_base = n_idx * C::BN + half * C::HC;
@@ -925,7 +943,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       e.mt = mt_next;
       const int next = tile + num_clusters;
       if (next < num_tiles)  // next tile's row parameters, in flight during this one
-        load_row_params(p, int64_t(next % p.num_m_tiles) * C::BM_PAIR + row_off, sx_next,
+        load_row_params(p, int64_t(tile_m(p, next)) * C::BM_PAIR + row_off, sx_next,
                         mt_next);
       const bool got = !(*abort_flag) && mbar_wait<true>(&tfull[acc], acc_phase, wc) &&
                        mbar_wait(&pfull[acc], acc_phase, wc);

@@ -86,6 +86,7 @@ struct GemmParams {
   int K;
   int num_m_tiles;
   int num_n_tiles;
+  int group_m;                // M tiles per group of the tile order (>= 1)
   float inv_sqrt_out;         // 1/sqrt(m) of the output-side transform (weight-only form)
   float acc_unit;             // accumulator units per code product: 1, or 1/16 when A is packed
   int acc_shift;              // acc_debug = raw accumulator >> acc_shift (0, or 4 when packed)
