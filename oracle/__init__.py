@@ -68,11 +68,13 @@ def _load():
             lib.hqo_sigma.argtypes = [ctypes.c_int64, _f64p, _f64p, ctypes.c_double, _f64p]
             lib.hqo_quantize_act.argtypes = [
                 ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                _u16p, ctypes.c_int64, _f64p, ctypes.c_double, _i64p, ctypes.c_int64,
+                _u16p, ctypes.c_int64, _f64p, _f64p, ctypes.c_double, _i64p, ctypes.c_int64,
                 _i8p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
             lib.hqo_prepare_weights.argtypes = [
                 ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
-                _u16p, _u16p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+                _u16p, _u16p, _f64p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
+                ctypes.c_int]
+            lib.hqo_channel_mean.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, _f64p]
             lib.hqo_gemm_acc.argtypes = [_i8p, _i8p, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_int64, _i64p, ctypes.c_int64, _i64p,
                                          ctypes.c_int]
@@ -90,7 +92,8 @@ def _load():
                                                 ctypes.c_int64, _f64p]
             lib.hqo_pack_i4.argtypes = [_i8p, ctypes.c_int64, _u8p]
             lib.hqo_unpack_i4.argtypes = [_u8p, ctypes.c_int64, _i8p]
-            for name in ("hqo_pack_i4", "hqo_unpack_i4", "hqo_sylvester", "hqo_col_absmax", "hqo_sigma", "hqo_quantize_act",
+            for name in ("hqo_pack_i4", "hqo_unpack_i4", "hqo_sylvester", "hqo_col_absmax",
+                         "hqo_channel_mean", "hqo_sigma", "hqo_quantize_act",
                          "hqo_prepare_weights", "hqo_gemm_acc", "hqo_epilogue",
                          "hqo_exact_linear", "hqo_prepare_weights_wh", "hqo_epilogue_wh",
                          "hqo_output_rotation"):
@@ -163,6 +166,16 @@ def col_absmax(M_bits: np.ndarray) -> np.ndarray:
     return out
 
 
+def channel_mean(M_bits: np.ndarray) -> np.ndarray:
+    """Per-channel mean over the rows of a bf16 matrix (fp64)."""
+    M = _c(M_bits, np.uint16)
+    R, C = M.shape
+    out = np.zeros(C, dtype=np.float64)
+    _check(_load().hqo_channel_mean(_ptr(M, ctypes.c_uint16), R, C, _ptr(out, ctypes.c_double)),
+           "channel_mean")
+    return out
+
+
 def sigma(amax_x: np.ndarray, amax_w: np.ndarray, alpha: float) -> np.ndarray:
     ax = _c(amax_x, np.float64)
     aw = _c(amax_w, np.float64)
@@ -173,11 +186,14 @@ def sigma(amax_x: np.ndarray, amax_w: np.ndarray, alpha: float) -> np.ndarray:
 
 
 def quantize_act(X_bits, n, bits, gran=0, centering=1, sigma=None, static_scale=0.0,
-                 rows=None, want_tie=True, want_Z=False, nthreads=None):
-    """Returns dict(codes int8 [r,K], scale f64 [r], mean f64 [r], tie, Z)."""
+                 rows=None, want_tie=True, want_Z=False, nthreads=None, shift=None):
+    """Returns dict(codes int8 [r,K], scale f64 [r], mean f64 [r], tie, Z).
+    shift: per-channel vector removed from Y = X diag(sigma^-1) before the
+    rotation (the appended-token centring), or None."""
     X = _c(X_bits, np.uint16)
     T, K = X.shape
     sig = _c(sigma, np.float64)
+    sh = _c(shift, np.float64)
     r = None if rows is None else _c(rows, np.int64)
     nr = T if r is None else r.size
     codes = np.zeros((nr, K), dtype=np.int8)
@@ -187,7 +203,7 @@ def quantize_act(X_bits, n, bits, gran=0, centering=1, sigma=None, static_scale=
     Z = np.zeros((nr, K), dtype=np.float64) if want_Z else None
     rc = _load().hqo_quantize_act(
         K, n, bits, gran, centering, _ptr(X, ctypes.c_uint16), T, _ptr(sig, ctypes.c_double),
-        float(static_scale), _ptr(r, ctypes.c_int64), nr, _ptr(codes, ctypes.c_int8),
+        _ptr(sh, ctypes.c_double), float(static_scale), _ptr(r, ctypes.c_int64), nr, _ptr(codes, ctypes.c_int8),
         _ptr(scale, ctypes.c_double), _ptr(mean, ctypes.c_double), _ptr(tie, ctypes.c_double),
         _ptr(Z, ctypes.c_double), nthreads or default_threads())
     _check(rc, "quantize_act")
@@ -195,12 +211,15 @@ def quantize_act(X_bits, n, bits, gran=0, centering=1, sigma=None, static_scale=
 
 
 def prepare_weights(W_bits, n, bits, bias_bits=None, sigma=None, want_tie=True,
-                    want_Wt=False, nthreads=None):
-    """Returns dict(codes int8 [N,K], scale [N], colsum [N], bias [N], tie, Wt)."""
+                    want_Wt=False, nthreads=None, shift=None):
+    """Returns dict(codes int8 [N,K], scale [N], colsum [N], bias [N], tie, Wt).
+    shift: the activations' per-channel shift (appended-token centring); its
+    product with diag(sigma) W is added to the bias."""
     W = _c(W_bits, np.uint16)
     N, K = W.shape
     b = _c(bias_bits, np.uint16)
     sig = _c(sigma, np.float64)
+    sh = _c(shift, np.float64)
     codes = np.zeros((N, K), dtype=np.int8)
     scale = np.zeros(N, dtype=np.float64)
     colsum = np.zeros(N, dtype=np.float64)
@@ -210,7 +229,8 @@ def prepare_weights(W_bits, n, bits, bias_bits=None, sigma=None, want_tie=True,
     Wt = np.zeros((N, K), dtype=np.float64) if want_Wt else None
     rc = _load().hqo_prepare_weights(
         K, N, n, bits, _ptr(W, ctypes.c_uint16), _ptr(b, ctypes.c_uint16),
-        _ptr(sig, ctypes.c_double), _ptr(codes, ctypes.c_int8), _ptr(scale, ctypes.c_double),
+        _ptr(sig, ctypes.c_double), _ptr(sh, ctypes.c_double), _ptr(codes, ctypes.c_int8),
+        _ptr(scale, ctypes.c_double),
         _ptr(colsum, ctypes.c_double), _ptr(corr_pre, ctypes.c_double),
         _ptr(bias, ctypes.c_double), _ptr(tie, ctypes.c_double),
         _ptr(Wt, ctypes.c_double), nthreads or default_threads())

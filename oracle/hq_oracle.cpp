@@ -154,6 +154,16 @@ int hqo_col_absmax(const uint16_t* M, int64_t R, int64_t C, double* out) {
   return 0;
 }
 
+int hqo_channel_mean(const uint16_t* M, int64_t R, int64_t C, double* out) {
+  if (M == nullptr || out == nullptr || R <= 0 || C <= 0) return -1;
+  for (int64_t c = 0; c < C; ++c) {
+    double sum = 0.0;
+    for (int64_t r = 0; r < R; ++r) sum += hqo_bf16_to_f64(M[r * C + c]);
+    out[c] = sum / double(R);
+  }
+  return 0;
+}
+
 int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
               double alpha, double* sigma) {
   if (K <= 0 || amax_x == nullptr || amax_w == nullptr || sigma == nullptr)
@@ -170,7 +180,7 @@ int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
 
 int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
                      const uint16_t* X, int64_t T, const double* sigma,
-                     double static_scale, const int64_t* rows, int64_t nrows,
+                     const double* shift, double static_scale, const int64_t* rows, int64_t nrows,
                      int8_t* codes, double* scale, double* mean, double* tie,
                      double* Z, int nthreads) {
   if (K <= 0 || !is_pow2(n) || K % n != 0 || bits < 2 || bits > 8) return -1;
@@ -188,15 +198,16 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
 
   /* Step 1 for one row: Y = X diag(sigma^-1); with centering 2 the row's
    * mean mu is subtracted from Y here, before the rotation; Z = Y H; with
-   * centering 1 the mean m of Z is what is subtracted after it.  `shift`
+   * centering 1 the mean m of Z is what is subtracted after it.  `zshift`
    * is the value removed from Z (m, or 0), `mean_out` the row's reported
    * mean (m for centering 1, mu for centering 2, else 0). */
-  auto transform_row = [&](int64_t t, std::vector<double>& V, double& shift,
+  auto transform_row = [&](int64_t t, std::vector<double>& V, double& zshift,
                            double& mean_out) {
     std::vector<double> Y(K);
     for (int64_t j = 0; j < K; ++j) {
       double s = sigma ? sigma[j] : 1.0;
       Y[j] = hqo_bf16_to_f64(X[t * K + j]) / s;
+      if (shift) Y[j] -= shift[j]; /* the per-channel mean over tokens */
     }
     mean_out = 0.0;
     if (centering == 2) {
@@ -213,12 +224,12 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
         acc += Y[j] * Hn[size_t((j - b0) * n + (k - b0))];
       V[k] = acc;
     }
-    shift = 0.0;
+    zshift = 0.0;
     if (centering == 1) {
       double sum = 0.0;
       for (int64_t k = 0; k < K; ++k) sum += V[k];
-      shift = sum / double(K);
-      mean_out = shift;
+      zshift = sum / double(K);
+      mean_out = zshift;
     }
   };
 
@@ -282,7 +293,7 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
 
 int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
                         const uint16_t* W, const uint16_t* bias,
-                        const double* sigma, int8_t* w_codes, double* w_scale,
+                        const double* sigma, const double* shift, int8_t* w_codes, double* w_scale,
                         double* colsum, double* corr_pre, double* bias_out,
                         double* tie, double* Wt, int nthreads) {
   if (K <= 0 || N <= 0 || !is_pow2(n) || K % n != 0 || bits < 2 || bits > 8)
@@ -333,6 +344,14 @@ int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
       if (Wt) Wt[c * K + k] = wt[k];
     }
     bias_out[c] = bias ? hqo_bf16_to_f64(bias[c]) : 0.0;
+    if (shift) {
+      /* the removed per-channel mean, mu diag(sigma) W in the pages'
+       * orientation, is the same for every token: a bias term */
+      double cs = 0.0;
+      for (int64_t k = 0; k < K; ++k)
+        cs += shift[k] * (sigma ? sigma[k] : 1.0) * hqo_bf16_to_f64(W[c * K + k]);
+      bias_out[c] += cs;
+    }
   });
   return 0;
 }

@@ -49,6 +49,10 @@ double hqo_rne(double x);
 /* out[c] = max_r |M[r,c]| for a bf16 matrix M[R,C]. */
 int hqo_col_absmax(const uint16_t* M, int64_t R, int64_t C, double* out);
 
+/* out[c] = (1/R) sum_r M[r,c] for a bf16 matrix M[R,C] (R > 0): the
+ * per-channel mean over tokens of the appended-token centring. */
+int hqo_channel_mean(const uint16_t* M, int64_t R, int64_t C, double* out);
+
 /* sigma_k = amax_x[k]^alpha / amax_w[k]^(1-alpha); sigma_k = 1 when either
  * maximum is zero. */
 int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
@@ -62,6 +66,11 @@ int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
  *                after the rotation; reported mean m_t)
  *   centering 2: mu_t = mean_k Y[t,k], V = (Y - mu_t) H       (the mean removed
  *                before the rotation; reported mean mu_t)
+ *   shift (any centering; NULL = none): a per-channel vector removed from Y
+ *                before everything above, Y[t,k] -= shift[k] (the per-channel
+ *                mean over tokens, in Y's units: the appended-token reading
+ *                of the HadaNorm review's mu in R^d; its product with the
+ *                weights goes into the bias, see hqo_prepare_weights)
  *   per token  (gran 0): s_t = max_k |V[t,k]| / q
  *   per tensor (gran 1): s   = max_{t,k} |V[t,k]| / q   over ALL T rows
  *   static     (gran 2): s   = static_scale
@@ -71,7 +80,7 @@ int hqo_sigma(int64_t K, const double* amax_x, const double* amax_w,
  * from a rounding tie, in code units; 0.5 when s = 0) and Z[i*K+k]. */
 int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
                      const uint16_t* X, int64_t T, const double* sigma,
-                     double static_scale, const int64_t* rows, int64_t nrows,
+                     const double* shift, double static_scale, const int64_t* rows, int64_t nrows,
                      int8_t* codes, double* scale, double* mean, double* tie,
                      double* Z, int nthreads);
 
@@ -80,11 +89,13 @@ int hqo_quantize_act(int64_t K, int64_t n, int bits, int gran, int centering,
  * centering 1), corr_pre[n] = sum_k sigma_k W[n,k] (the correction of
  * centering 2; optional output),
  * w_scale[n] = max_k |W~[n,k]| / q, w_codes = clamp(rne(W~ / w_scale), -q, q),
- * bias_out[n] = b[n] (0 when bias == NULL).  sigma == NULL means sigma = 1.
+ * bias_out[n] = b[n] (0 when bias == NULL) + sum_k shift_k sigma_k W[n,k]
+ * (the appended token's contribution, shift == NULL: none).  sigma == NULL
+ * means sigma = 1.
  * Optional outputs: tie[N*K] and Wt[N*K] (the unquantized W~). */
 int hqo_prepare_weights(int64_t K, int64_t N, int64_t n, int bits,
                         const uint16_t* W, const uint16_t* bias,
-                        const double* sigma, int8_t* w_codes, double* w_scale,
+                        const double* sigma, const double* shift, int8_t* w_codes, double* w_scale,
                         double* colsum, double* corr_pre, double* bias_out,
                         double* tie, double* Wt, int nthreads);
 

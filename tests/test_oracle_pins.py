@@ -571,7 +571,8 @@ def test_packed_codes_reject_out_of_range_values():
 def _bf16_bits(values):
     """bf16 bit patterns of values that bf16 holds exactly (hand-checked)."""
     table = {1.0: 0x3F80, -1.0: 0xBF80, 2.0: 0x4000, -2.0: 0xC000, 0.5: 0x3F00,
-             0.25: 0x3E80, -3.5: 0xC060, -4.0: 0xC080, 3.0: 0x4040, 0.0: 0x0000}
+             0.25: 0x3E80, -3.5: 0xC060, -4.0: 0xC080, 3.0: 0x4040, 0.0: 0x0000,
+             4.0: 0x4080}
     out = []
     for v in values:
         if isinstance(v, str):  # "-0": the negative zero bit pattern
@@ -653,3 +654,102 @@ def test_sigma_balances_the_channel_maxima():
         assert np.allclose(ws, ax ** alpha * aw ** alpha, rtol=1e-12)
         if alpha == 0.5:
             assert np.allclose(xs, ws, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Per-channel centring over tokens: HadaNorm review, Figure 2 caption (mu, sigma
+# in R^d) and Desk Editor's Note (the bias absorbed into an appended token).
+# mu_k = mean_t Y[t,k] is removed before the rotation, V = (Y - mu) H, and its
+# product with the weights, mu diag(sigma) W, is the same for every token: a
+# bias term.
+# --------------------------------------------------------------------------
+
+def test_channel_mean_hand_built_matrix():
+    """Mean over the rows of each column of a 4 x 4 bf16 matrix written out
+    by hand (dyadic values, so the means are exact); a mean along rows would
+    give (1 + -2 + 0.5 + 3) / 4 = 0.625 first."""
+    vals = [[1.0, -2.0, 0.5, 3.0],
+            [3.0, 2.0, "-0", 1.0],
+            [0.0, 0.25, 0.5, -4.0],
+            [-2.0, -1.0, 3.0, 0.0]]
+    M = np.array([_bf16_bits(r) for r in vals], dtype=np.uint16)
+    assert oracle.channel_mean(M).tolist() == [0.5, -0.1875, 1.0, 0.0]
+
+
+def _two_token_layer():
+    # X = [[1,2,3,4],[3,2,1,0]] in bf16, sigma = 1, n = K = 4
+    X = np.array([_bf16_bits([1.0, 2.0, 3.0, 4.0]), _bf16_bits([3.0, 2.0, 1.0, 0.0])],
+                 dtype=np.uint16)
+    return X
+
+
+def test_channel_centring_hand_worked_example():
+    """Worked by hand: the channel mean is mu = [2, 2, 2, 2]; Y - mu =
+    [-1, 0, 1, 2] and its negation; with H = H~_4 / 2 the rotated rows are
+    V = [1, -1, -2, 0] and [-1, 1, 2, 0], max |V| = 2.
+      int4 (q = 7): V * 7 / 2 = [3.5, -3.5, -7, 0] -> half to even [4, -4, -7, 0]
+      int3 (q = 3): V * 3 / 2 = [1.5, -1.5, -3, 0] -> [2, -2, -3, 0]
+    With the token mean also removed before H (centring 2): row 0 becomes
+    [-1.5, -0.5, 0.5, 1.5], V = [0, -1, -2, 0], int4 codes [0, -4, -7, 0],
+    reported mean 0.5.  The weight side adds mu diag(sigma) W to the bias:
+    W = [1, 0, -1, 0.5], b = 0.25 -> 0.25 + 2 * 0.5 = 1.25."""
+    X = _two_token_layer()
+    mu = oracle.channel_mean(X)
+    assert mu.tolist() == [2.0, 2.0, 2.0, 2.0]
+    a4 = oracle.quantize_act(X, 4, 4, centering=0, shift=mu, want_Z=True)
+    assert a4["Z"].tolist() == [[1.0, -1.0, -2.0, 0.0], [-1.0, 1.0, 2.0, 0.0]]
+    assert a4["codes"].tolist() == [[4, -4, -7, 0], [-4, 4, 7, 0]]
+    assert a4["scale"].tolist() == pytest.approx([2.0 / 7.0, 2.0 / 7.0], rel=1e-15)
+    assert a4["mean"].tolist() == [0.0, 0.0]
+    assert np.all(a4["tie"][:, :2] == 0.0)  # 3.5 and -3.5 lie exactly on ties
+    a3 = oracle.quantize_act(X, 4, 3, centering=0, shift=mu)
+    assert a3["codes"].tolist() == [[2, -2, -3, 0], [-2, 2, 3, 0]]
+    a42 = oracle.quantize_act(X[:1], 4, 4, centering=2, shift=mu, want_Z=True)
+    assert a42["Z"].tolist() == [[0.0, -1.0, -2.0, 0.0]]
+    assert a42["codes"].tolist() == [[0, -4, -7, 0]]
+    assert a42["mean"].tolist() == [0.5]
+    W = np.array([_bf16_bits([1.0, 0.0, -1.0, 0.5])], dtype=np.uint16)
+    b = np.array(_bf16_bits([0.25]), dtype=np.uint16)
+    w = oracle.prepare_weights(W, 4, 4, bias_bits=b, shift=mu)
+    assert w["bias"].tolist() == [1.25]
+    assert oracle.prepare_weights(W, 4, 4, bias_bits=b)["bias"].tolist() == [0.25]
+
+
+@pytest.mark.parametrize("K,n,N,T", [(64, 16, 24, 9), (256, 64, 40, 7), (1152, 128, 16, 5)])
+@pytest.mark.parametrize("centering", [0, 1, 2])
+def test_eq1_identity_with_channel_centring(K, n, N, T, centering):
+    """With quantization off the layer is exact: the rotated, centred
+    activations times W~ plus the bias (which now carries mu diag(sigma) W)
+    plus the per-token mean's correction reproduce X W + b (HadaNorm review
+    Eq. (1)), to 1e-10 relative, with any per-token centring on top."""
+    g = np.random.default_rng(K + T + centering)
+    X = synth.f32_to_bf16_bits((g.standard_normal((T, K)) + g.standard_normal(K) * 3.0)
+                               .astype(np.float32))
+    W = synth.f32_to_bf16_bits((g.standard_normal((N, K)) * 0.05).astype(np.float32))
+    b = synth.f32_to_bf16_bits((g.standard_normal(N) * 0.1).astype(np.float32))
+    sig = oracle.sigma(oracle.col_absmax(X), oracle.col_absmax(W), 0.5)
+    mu = oracle.channel_mean(X) / sig  # the mean of Y = X diag(sigma^-1)
+    a = oracle.quantize_act(X, n, 8, centering=centering, sigma=sig, shift=mu, want_Z=True)
+    w = oracle.prepare_weights(W, n, 8, bias_bits=b, sigma=sig, shift=mu, want_Wt=True)
+    Z = a["Z"]
+    m = a["mean"] if centering else np.zeros(T)
+    y = (Z - (m[:, None] if centering == 1 else 0.0)) @ w["Wt"].T + w["bias"][None, :]
+    if centering:
+        y += m[:, None] * oracle.correction(w, centering)[None, :]
+    exact = oracle.exact_linear(X, W, b)
+    assert np.linalg.norm(y - exact) <= 1e-10 * np.linalg.norm(exact)
+
+
+def test_channel_centring_zeroes_every_channel_sum():
+    """When mu is the channel mean of the same tokens, every channel of
+    Y - mu sums to zero over the tokens, and so does every rotated channel
+    of V = (Y - mu) H (H is linear)."""
+    g = np.random.default_rng(11)
+    X = synth.f32_to_bf16_bits((g.standard_normal((33, 256)) + 2.0).astype(np.float32))
+    mu = oracle.channel_mean(X)
+    a = oracle.quantize_act(X, 64, 8, centering=0, shift=mu, want_Z=True)
+    col = a["Z"].sum(axis=0)
+    assert np.max(np.abs(col)) <= 1e-11 * np.max(np.abs(a["Z"])) * 33
+    # without the shift the channel sums are far from zero
+    a0 = oracle.quantize_act(X, 64, 8, centering=0, want_Z=True)
+    assert np.max(np.abs(a0["Z"].sum(axis=0))) > 10.0
