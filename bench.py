@@ -450,6 +450,32 @@ def capture_layer_graphs(torch, ctx, steps, warmup):
     return graphs
 
 
+def host_call_cost(hq, torch, ctx, calls=200):
+    """Host microseconds per eager call of hq_quantize_act and hq_linear
+    (launch included, the device not waited for): the per-call host cost a
+    caller pays outside a CUDA graph."""
+    desc, layer, bufs, Xs, Y = (ctx[k] for k in ("desc", "layer", "bufs", "Xs", "Y"))
+    mean_in = bufs["a_mean"] if desc.centering else None
+    q = lambda: hq.hq_quantize_act(desc, Xs[0], ctx["sig_inv"], bufs["a_codes"],
+                                   bufs["a_scale"], bufs["a_mean"], layer.workspace)
+    g = lambda: hq.hq_linear(desc, bufs["a_codes"], bufs["a_scale"], mean_in, layer.w_codes,
+                             layer.w_scale, layer.colsum, layer.bias_f32, Y)
+    out = {}
+    for name, fn in (("hq_quantize_act", q), ("hq_linear", g)):
+        fn()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            fn()
+        dt = time.perf_counter() - t0
+        torch.cuda.synchronize()
+        out[name] = dt / calls * 1e6
+    out["what"] = ("host time per eager call through the Python binding, device not waited "
+                   "for; tensor maps come from the library's cache after the first call")
+    out["tmap_cache"] = hq.hq_debug_tmap_cache()
+    return out
+
+
 def measure_mma_ceiling(hq, torch):
     """The measured int8 tensor-core ceiling: the GEMMs' main loops with
     nothing but the MMAs (hq_debug_mma_ceiling), one CTA per SM, timed with
@@ -660,6 +686,8 @@ def run_hq(args):
         check("in the e2e region")
         del g_e2e, Xh, Yh, Xd
 
+    ctx_host = host_call_cost(hq, torch, ctx) if rank == 0 else None
+
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -716,6 +744,9 @@ def run_hq(args):
         "clocks": clock_info,
         "e2e": e2e,
     }
+    # host time of one eager call of each entry point (tensor maps from the
+    # library's cache after the first call); outside any timed region
+    line["host_us_per_call"] = ctx_host
     if with_packed:
         pcfg = cfg.packed()
         line["variants"] = {"packed_codes": {

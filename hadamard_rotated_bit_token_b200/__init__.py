@@ -30,7 +30,8 @@ __all__ = [
     "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
     "hq_debug_set_gemm_variant", "HQ_GEMM_AUTO", "HQ_GEMM_SINGLE_CTA", "HQ_GEMM_CTA_PAIR",
-    "hq_quantize_act_noalloc", "hq_debug_plan", "hq_debug_mma_ceiling", "HadamardQuantLinear",
+    "hq_quantize_act_noalloc", "hq_debug_plan", "hq_debug_mma_ceiling", "hq_debug_tmap_cache",
+    "HadamardQuantLinear",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -48,7 +49,7 @@ EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare
             "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
             "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
             "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan",
-            "hq_debug_mma_ceiling")
+            "hq_debug_mma_ceiling", "hq_debug_tmap_cache")
 
 
 class HQError(RuntimeError):
@@ -118,11 +119,13 @@ def load_library():
         lib.hq_debug_plan.argtypes = [desc_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                       _i32p, _i32p, _i32p, _i32p]
         lib.hq_debug_mma_ceiling.argtypes = [ctypes.c_int, ctypes.c_int64, _i32p, _vp]
+        _u64p = ctypes.POINTER(ctypes.c_uint64)
+        lib.hq_debug_tmap_cache.argtypes = [_u64p, _u64p]
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
                      "hq_forward_host",
                      "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
                      "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan",
-            "hq_debug_mma_ceiling"):
+            "hq_debug_mma_ceiling", "hq_debug_tmap_cache"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -283,6 +286,14 @@ def hq_debug_mma_ceiling(pair: bool, k_blocks: int, stream=None) -> int:
     _check(lib.hq_debug_mma_ceiling(1 if pair else 0, int(k_blocks), ctypes.byref(n),
                                     _stream(stream)), "hq_debug_mma_ceiling")
     return int(n.value)
+
+
+def hq_debug_tmap_cache() -> dict:
+    """Cumulative tensor-map cache hits and misses of the library."""
+    h, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check(load_library().hq_debug_tmap_cache(ctypes.byref(h), ctypes.byref(m)),
+           "hq_debug_tmap_cache")
+    return {"hits": int(h.value), "misses": int(m.value)}
 
 
 def hq_debug_set_gemm_variant(variant: int):

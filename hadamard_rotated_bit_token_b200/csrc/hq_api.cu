@@ -33,7 +33,7 @@ struct DeviceState {
   int cc_major = 0, cc_minor = 0;
   unsigned int* err = nullptr;
   bool quant_attr_set[11][4][3] = {};  // [log2 n][mode][centering]
-  bool qact_attr_set[6][11][4][3] = {};  // [kernel][log2 n][mode][centering] attributes set
+  bool qact_attr_set[7][11][4][3] = {};  // [kernel][log2 n][mode][centering] attributes set
   int pair_clusters = -1;  // co-resident clusters of the CTA-pair GEMM (-1: not queried)
   // hq_forward_host's upload and download streams (created on first use)
   cudaStream_t up = nullptr, down = nullptr;
@@ -94,11 +94,17 @@ hq_status check_k_side(const hq_layer_desc* d) {
   const int logn = ilog2_exact(d->had_order);
   if (d->K <= 0 || d->had_order <= 0) return HQ_ERR_INVALID_ARGUMENT;
   if (logn != 0 && (logn < 4 || logn > 10)) return HQ_ERR_UNSUPPORTED;
-  if (d->K % d->had_order != 0 || d->K % 64 != 0 || d->K > 9216) return HQ_ERR_UNSUPPORTED;
+  // K: whole blocks, whole 16-channel groups; at most 15360 with a rotation
+  // (the segment kernel's 480 slices a row), 10240 without one (the row
+  // kernel's 320 slices)
+  if (d->K % d->had_order != 0 || d->K % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (d->K > (logn == 0 ? 10240 : 15360)) return HQ_ERR_UNSUPPORTED;
   if (d->code_format != HQ_CODES_I8 && d->code_format != HQ_CODES_I4_PACKED)
     return HQ_ERR_UNSUPPORTED;
-  // two codes per byte hold 3- and 4-bit activation codes only
-  if (d->code_format == HQ_CODES_I4_PACKED && d->a_bits != 3 && d->a_bits != 4)
+  // two codes per byte hold 3- and 4-bit activation codes only, in rows of
+  // whole 16-byte units
+  if (d->code_format == HQ_CODES_I4_PACKED &&
+      ((d->a_bits != 3 && d->a_bits != 4) || d->K % 32 != 0))
     return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
@@ -156,7 +162,7 @@ constexpr int kGroupM = HQ_GROUP_M;  // M tiles per group of the GEMM's tile ord
 // full last round) over R = 8 (1024 tiles), 15.2 -> 14.4 us; for K = 3072,
 // T = 16384 the 2 % cheaper R = 2 made the step slower than R = 3.
 void quant_shape(int K, int64_t T, int sms, int per_sm, int* R_out, int* nt_out) {
-  const int S = K / 32;
+  const int S = (K + 31) / 32;  // the last slice may hold 16 channels
   const int maxT = quant_max_threads();
   const int64_t slots = int64_t(sms) * per_sm;
   auto cost_of = [&](int R, int nt) {
@@ -180,7 +186,7 @@ void quant_shape(int K, int64_t T, int sms, int per_sm, int* R_out, int* nt_out)
       bestNT = nt;
     }
   }
-  if (bestNT == 0) bestNT = ((S + 31) / 32) * 32;  // S > maxT cannot occur (K <= 9216)
+  if (bestNT == 0) bestNT = ((S + 31) / 32) * 32;  // S > maxT cannot occur (K <= 10240)
   *R_out = bestR;
   *nt_out = bestNT;
 }
@@ -205,7 +211,7 @@ hq_status make_quant_launch(const DeviceState* dev, int K, int n, int64_t T, con
   L.p.X = X;
   L.p.T = T;
   L.p.K = K;
-  L.p.S = K / 32;
+  L.p.S = (K + 31) / 32;
   L.p.R = R;
   L.p.inv_sqrt_n = float(1.0 / std::sqrt(double(n)));
   L.p.sqrt_n = float(std::sqrt(double(n)));
@@ -245,7 +251,7 @@ hq_status run_quant(DeviceState* dev, QuantLaunch& L, int mode, int center, cuda
 // CTAs of the warp-row kernel per SM, and the shared memory each may use
 constexpr int kQActCtasPerSm = 2;
 constexpr size_t kQActSmemPerCta = size_t(228 / kQActCtasPerSm - 1) * 1024;
-size_t seg_smem_per_cta() { return size_t(228 / quant_seg_ctas_per_sm() - 1) * 1024; }
+size_t seg_smem_per_cta(bool big) { return size_t(228 / quant_seg_ctas_per_sm(big) - 1) * 1024; }
 
 // Rows of the [T*S, 32] view per tensor copy for a stage of RS rows: the
 // whole stage when it fits one box (at most 256 rows), else the largest
@@ -271,6 +277,7 @@ int qact_max_seg(int R, int S) {
 // How hq_quantize_act runs for K channels, blocks of n and T tokens.
 struct ActPlan {
   bool wrow;     // the warp-row kernel (else the segment kernel)
+  bool big;      // segment kernel: the large-row variant
   int spl;       // warp-row: slices a lane (0: several rows per warp)
   int rpw;       // warp-row: rows per warp
   int rows;      // rows per tile
@@ -295,10 +302,12 @@ int qact_stages(size_t fixed, int rows, int S, size_t budget = kQActSmemPerCta) 
 // CTA, the most threads within 3 % of the lowest cost).
 bool qact_plan(int K, int n, int centering, int64_t T, int sms, ActPlan* out) {
   ActPlan& P = *out;
+  if (K % 32 != 0 || n < 16) return false;  // whole 32-channel slices, a rotation
   const int S = K / 32;
   const bool pre = centering == HQ_CENTER_TOKEN_MEAN_PRE;
   if ((S % 32 == 0 && S / 32 <= 4) || S < 32) {
     P.wrow = true;
+    P.big = false;
     P.spl = S < 32 ? 0 : S / 32;
     P.rpw = S < 32 ? 32 / S : 1;
     const int nw = quant_wrow_warps(P.spl);
@@ -314,12 +323,14 @@ bool qact_plan(int K, int n, int centering, int64_t T, int sms, ActPlan* out) {
   P.wrow = false;
   P.spl = 0;
   P.rpw = 0;
-  const int maxC = quant_seg_max_consumers();
-  const int64_t slots = int64_t(sms) * quant_seg_ctas_per_sm();
+  P.big = S > quant_seg_max_consumers(false);  // rows longer than the normal CTA
+  const bool big = P.big;
+  const int maxC = quant_seg_max_consumers(big);
+  const int64_t slots = int64_t(sms) * quant_seg_ctas_per_sm(big);
   auto stages_for = [&](int R) {
     if (qact_box_rows(R * S) == 0) return 0;
     return qact_stages(quant_seg_smem_bytes(R, S, K, n, 0, qact_max_seg(R, S), pre), R, S,
-                       seg_smem_per_cta());
+                       seg_smem_per_cta(big));
   };
   auto cost_of = [&](int R, int nt) {
     const int64_t tiles = (T + R - 1) / R;
@@ -352,7 +363,57 @@ bool qact_plan(int K, int n, int centering, int64_t T, int sms, ActPlan* out) {
   return true;
 }
 
-hq_status encode_act_view(CUtensorMap* m, const void* X, int64_t T, int K, int box_rows) {
+// ---------------------------------------------------------------------------
+// Tensor-map cache.  A tensor map is a pure function of its parameters (base
+// address, extents, box, layout), so maps are kept in a small table keyed by
+// them and reused by later calls on the same buffers and shapes, instead of
+// being encoded on the host on every call.  Round-robin replacement; guarded
+// by g_mutex.
+struct TmapKey {
+  int kind;  // which encoder
+  const void* base;
+  int64_t rows;
+  int64_t cols;
+  int box;
+  bool operator==(const TmapKey& o) const {
+    return kind == o.kind && base == o.base && rows == o.rows && cols == o.cols && box == o.box;
+  }
+};
+constexpr int kTmapCacheSize = 64;
+struct TmapCache {
+  TmapKey key[kTmapCacheSize];
+  CUtensorMap map[kTmapCacheSize];
+  bool used[kTmapCacheSize] = {};
+  int next = 0;
+};
+TmapCache g_tmaps;
+unsigned long long g_tmap_hits = 0, g_tmap_misses = 0;
+
+template <class Encode>
+hq_status cached_tmap(const TmapKey& k, CUtensorMap* out, Encode encode) {
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    for (int i = 0; i < kTmapCacheSize; ++i) {
+      if (g_tmaps.used[i] && g_tmaps.key[i] == k) {
+        *out = g_tmaps.map[i];
+        ++g_tmap_hits;
+        return HQ_OK;
+      }
+    }
+  }
+  hq_status s = encode(out);
+  if (s != HQ_OK) return s;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  const int i = g_tmaps.next;
+  g_tmaps.next = (i + 1) % kTmapCacheSize;
+  g_tmaps.key[i] = k;
+  g_tmaps.map[i] = *out;
+  g_tmaps.used[i] = true;
+  ++g_tmap_misses;
+  return HQ_OK;
+}
+
+hq_status encode_act_view_raw(CUtensorMap* m, const void* X, int64_t T, int K, int box_rows) {
   const int S = K / 32;
   cuuint64_t dims[2] = {32u, cuuint64_t(T) * cuuint64_t(S)};
   cuuint64_t strides[1] = {64u};
@@ -373,11 +434,11 @@ struct QActLaunch {
 };
 
 hq_status make_quant_act_launch(const DeviceState* dev, const hq_layer_desc* d, int64_t T,
-                                const uint16_t* X, QActLaunch* out) {
+                                const uint16_t* X, QActLaunch* out, int centering) {
   QActLaunch& L = *out;
   std::memset(&L.p, 0, sizeof(L.p));
   const int K = d->K, n = d->had_order;
-  if (!qact_plan(K, n, d->centering, T > 0 ? T : 1, dev->sm_count, &L.plan))
+  if (!qact_plan(K, n, centering, T > 0 ? T : 1, dev->sm_count, &L.plan))
     return HQ_ERR_UNSUPPORTED;
   const ActPlan& P = L.plan;
   const int S = K / 32;
@@ -401,27 +462,31 @@ hq_status make_quant_act_launch(const DeviceState* dev, const hq_layer_desc* d, 
   L.p.inv_k = 1.0f / float(K);
   const int64_t ntiles = (T + P.rows - 1) / P.rows;
   const int64_t slots =
-      int64_t(dev->sm_count) * (P.wrow ? kQActCtasPerSm : quant_seg_ctas_per_sm());
+      int64_t(dev->sm_count) * (P.wrow ? kQActCtasPerSm : quant_seg_ctas_per_sm(P.big));
   L.grid = int(ntiles < slots ? ntiles : slots);
-  return encode_act_view(&L.tmap, X, T, K, L.p.box_rows);
+  const int box_rows = L.p.box_rows;
+  return cached_tmap(TmapKey{4, X, T, K, box_rows}, &L.tmap, [&](CUtensorMap* o) {
+    return encode_act_view_raw(o, X, T, K, box_rows);
+  });
 }
 
 hq_status run_quant_act(DeviceState* dev, QActLaunch& L, int mode, int center, cudaStream_t st) {
   const int logn = L.logn;
   const ActPlan& P = L.plan;
   const void* fn = P.wrow ? quant_wrow_kernel_ptr(logn, mode, center, P.spl)
-                          : quant_seg_kernel_ptr(logn, mode, center);
+                          : quant_seg_kernel_ptr(logn, mode, center, P.big);
   if (fn == nullptr) return HQ_ERR_UNSUPPORTED;
   if (L.p.T <= 0) return HQ_OK;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    const int slot = P.wrow ? 1 + P.spl : 0;
+    const int slot = P.wrow ? 1 + P.spl : (P.big ? 6 : 0);
     bool& set = dev->qact_attr_set[slot][logn][mode][center];
     if (!set) {
       // kQActCtasPerSm CTAs of up to kQActSmemPerCta each: the largest
       // shared-memory carveout
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(P.wrow ? kQActSmemPerCta : seg_smem_per_cta())) != cudaSuccess ||
+                               int(P.wrow ? kQActSmemPerCta : seg_smem_per_cta(P.big))) !=
+              cudaSuccess ||
           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
         return HQ_ERR_CUDA;
@@ -437,7 +502,7 @@ hq_status quantize_act_tma(DeviceState* dev, const hq_layer_desc* desc, const ui
                            int64_t T, const float* sigma_inv, int8_t* a_codes, float* a_scale,
                            float* a_mean, void* workspace, cudaStream_t st) {
   QActLaunch L;
-  hq_status s = make_quant_act_launch(dev, desc, T, X, &L);
+  hq_status s = make_quant_act_launch(dev, desc, T, X, &L, desc->centering);
   if (s != HQ_OK) return s;
   L.p.mult = sigma_inv;
   L.p.invert_mult = 0;
@@ -467,7 +532,8 @@ hq_status quantize_act_tma(DeviceState* dev, const hq_layer_desc* desc, const ui
   return run_quant_act(dev, L, 2, center, st);
 }
 
-hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+hq_status encode_kmajor_i8_raw(CUtensorMap* m, const void* base, int64_t rows, int K,
+                               int box_rows) {
   cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(K)};
   cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
@@ -481,7 +547,7 @@ hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K
 // Packed activation codes [T, K/2] bytes: box {64 bytes (one K block of 128
 // codes), 128 rows}, 64-byte swizzle (the GEMM's converters read one row per
 // lane without bank conflicts and widen it themselves).
-hq_status encode_packed_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
+hq_status encode_packed_a_raw(CUtensorMap* m, const void* base, int64_t rows, int K) {
   cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(K / 2)};
   cuuint32_t box[2] = {64u, 128u};
@@ -492,7 +558,7 @@ hq_status encode_packed_a(CUtensorMap* m, const void* base, int64_t rows, int K)
   return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
 }
 
-hq_status encode_out_bf16(CUtensorMap* m, const void* base, int64_t rows, int N) {
+hq_status encode_out_bf16_raw(CUtensorMap* m, const void* base, int64_t rows, int N) {
   cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(N) * 2u};
   cuuint32_t box[2] = {32u, 32u};
@@ -502,6 +568,20 @@ hq_status encode_out_bf16(CUtensorMap* m, const void* base, int64_t rows, int N)
                         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+}
+
+hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+  return cached_tmap(TmapKey{1, base, rows, K, box_rows}, m, [&](CUtensorMap* o) {
+    return encode_kmajor_i8_raw(o, base, rows, K, box_rows);
+  });
+}
+hq_status encode_packed_a(CUtensorMap* m, const void* base, int64_t rows, int K) {
+  return cached_tmap(TmapKey{2, base, rows, K, 0}, m,
+                     [&](CUtensorMap* o) { return encode_packed_a_raw(o, base, rows, K); });
+}
+hq_status encode_out_bf16(CUtensorMap* m, const void* base, int64_t rows, int N) {
+  return cached_tmap(TmapKey{3, base, rows, N, 0}, m,
+                     [&](CUtensorMap* o) { return encode_out_bf16_raw(o, base, rows, N); });
 }
 
 // GEMM kernel choice.  Both kernels are persistent with one CTA per SM, so a
@@ -685,7 +765,27 @@ hq_status hq_prepare_weights(const hq_layer_desc* desc, const uint16_t* W, const
   }
   // W~ rows: multiply by sigma (= 1 / sigma_inv), rotate, quantize per row,
   // and record each row's sum (colsum of W~ in the pages' orientation); with
-  // had_order 1 (no rotation, no centering) no sum is needed
+  // had_order 1 (no rotation, no centering) no sum is needed.  Rows of whole
+  // 32-channel slices take the TMA-fed kernels, the others the row kernel.
+  ActPlan wap;
+  if (desc->had_order >= 16 && qact_plan(K, desc->had_order, HQ_CENTER_NONE, N, dev->sm_count, &wap)) {
+    QActLaunch AL;
+    s = make_quant_act_launch(dev, desc, N, W, &AL, HQ_CENTER_NONE);
+    if (s != HQ_OK) return s;
+    AL.p.mult = act_absmax ? sigma_inv : nullptr;
+    AL.p.invert_mult = 1;
+    AL.p.codes = w_codes;
+    AL.p.scale = w_scale;
+    AL.p.mean = nullptr;
+    AL.p.rowsum = colsum;
+    AL.p.rowsum_pre = desc->centering == HQ_CENTER_TOKEN_MEAN_PRE ? 1 : 0;
+    AL.p.q = qw;
+    AL.p.s_unit = AL.p.inv_sqrt_n / float(qw);
+    s = run_quant_act(dev, AL, 0, HQ_CENTER_NONE, st);
+    if (s != HQ_OK) return s;
+    if (bias) return from_cuda(launch_bf16_to_f32(bias, bias_f32, N, st));
+    return from_cuda(launch_fill(bias_f32, N, 0.0f, st));
+  }
   QuantLaunch L;
   s = make_quant_launch(dev, K, desc->had_order, N, W, &L);
   if (s != HQ_OK) return s;
@@ -1024,6 +1124,13 @@ hq_status hq_debug_mma_ceiling(int pair, int64_t k_blocks, int32_t* ctas, hq_str
   *ctas = n;
   return from_cuda(launch_mma_ceiling(pair != 0, k_blocks, n, dev->err, wait_ns(),
                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hq_status hq_debug_tmap_cache(uint64_t* hits, uint64_t* misses) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (hits) *hits = g_tmap_hits;
+  if (misses) *misses = g_tmap_misses;
+  return HQ_OK;
 }
 
 hq_status hq_debug_inject_fault(int kind) {

@@ -62,10 +62,14 @@ size_t quant_smem_bytes(int R, int K, int B, int nwarps, bool xpose);
 //   warp-row kernel: warps own whole rows; spl = K / 1024 in [1, 4] slices a
 //     lane and one row per warp, or spl = 0 for S = K/32 < 32: p.rpw rows
 //     of S lanes each per warp; quant_wrow_warps(spl) consumer warps.
-const void* quant_seg_kernel_ptr(int logn, int mode, int center);
+//   big: the segment kernel for rows of more than 256 slices (up to 480
+//     consumers, one CTA per SM).
+// Both kernels also serve the weight side (p.invert_mult: multiply by
+// 1 / p.mult; p.rowsum: the row's correction sum).
+const void* quant_seg_kernel_ptr(int logn, int mode, int center, bool big);
 const void* quant_wrow_kernel_ptr(int logn, int mode, int center, int spl);
-int quant_seg_max_consumers();
-int quant_seg_ctas_per_sm();
+int quant_seg_max_consumers(bool big);
+int quant_seg_ctas_per_sm(bool big);
 int quant_wrow_warps(int spl);
 // Dynamic shared memory of one CTA (n = Hadamard order; rows per tile).
 size_t quant_seg_smem_bytes(int R, int S, int K, int n, int stages, int max_seg, bool pre);

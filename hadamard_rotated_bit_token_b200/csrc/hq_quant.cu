@@ -111,8 +111,8 @@ __host__ __device__ inline int padded_blocks(int B) { return (B + 3) & ~3; }
 __host__ __device__ inline QuantSmem quant_smem_layout(int R, int K, int B, int nwarps, bool xpose) {
   QuantSmem L;
   uint32_t off = 0;
-  L.mult = off;  // channel multipliers, chunk-major [8][K/32] float4
-  off += 4u * K;
+  L.mult = off;  // channel multipliers, chunk-major [8][S] float4 (S = ceil(K / 32))
+  off += 128u * uint32_t((K + 31) / 32);
   L.xbuf = off;  // per-warp transpose buffers
   off += xpose ? 4096u * nwarps : 0u;
   L.pmax = off;
@@ -204,6 +204,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
   const int slice = active ? tid - row0 * S : 0;
   const int member = slice & (TT - 1);
   const int blk = slice >> LOG_TT;        // block of the row (n >= 32)
+  // K a multiple of 16 but not of 32 (n = 16 or 1): the row's last slice
+  // holds 16 channels; its upper half is padding, kept out of every
+  // statistic and never stored
+  const bool half = (K & 31) != 0 && slice == S - 1;
 
   // first tile's slice in flight while the CTA sets up
   const uint16_t* xcol = p.X + slice * 32;
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     if (active && row < T) {
       const uint4* src = reinterpret_cast<const uint4*>(xcol + row * K);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) nxt[c] = ld_stream(src + c);
+      for (int c = 0; c < 4; ++c) nxt[c] = (half && c >= 2) ? make_uint4(0, 0, 0, 0) : ld_stream(src + c);
     } else {
 #pragma unroll
       for (int c = 0; c < 4; ++c) nxt[c] = make_uint4(0, 0, 0, 0);
@@ -238,6 +242,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     // consecutive slices hit consecutive 16-byte words
     for (int i = tid; i < 8 * S; i += blockDim.x) {
       const int c = i / S, sl = i - c * S;
+      if (sl * 32 + 4 * c >= K) {  // past the row's end (a half slice): unused
+        msm[i] = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        continue;
+      }
       float4 m4 = *reinterpret_cast<const float4*>(p.mult + sl * 32 + 4 * c);
       if (p.invert_mult) {
         m4.x = 1.0f / m4.x;
@@ -311,7 +319,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     if (need_sum && !block_sums && active && member == 0) {
       float* yrow = y0buf + sr * BP;
 #pragma unroll
-      for (int b = 0; b < BPT; ++b) yrow[blk * BPT + b] = w[(b * N) >> 1].x;
+      for (int b = 0; b < BPT; ++b)
+        if (blk * BPT + b < B) yrow[blk * BPT + b] = w[(b * N) >> 1].x;
     }
     // index bit 0: the two halves of a pair (n = 1: no rotation)
     if (LOGN >= 1) {
@@ -395,12 +404,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
 #pragma unroll
       for (int b = 0; b < BPT; ++b) {
         first[b] = w[(b * N) >> 1].x;
-        if (active) y0buf[sr * BP + blk * BPT + b] = first[b];
+        if (active && blk * BPT + b < B) y0buf[sr * BP + blk * BPT + b] = first[b];
         // left out of this slice's max / min (channel 1 of block 0 stands in)
         if (PRE) w[(b * N) >> 1].x = w[0].y;
       }
     }
 
+    // a half slice's padding repeats a real value (channels 2 and 3, never a
+    // block's first channel), so it leaves the max and min unchanged
+    if (half) {
+#pragma unroll
+      for (int i = 8; i < 16; ++i) w[i] = w[1];
+    }
     // row max / min: reduce over this warp's lanes of the row, one atomic per
     // warp segment; the segment that completes the row finalizes it
     float mx = max3(w[0].x, w[0].y, w[1].x);
@@ -540,9 +555,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
       for (int g = 0; g < 8; ++g) t[g] = (words[g] & 0x0F0F0F0Fu) | ((words[g] >> 4) & 0xF0F0F0F0u);
       uint8_t* prow = reinterpret_cast<uint8_t*>(p.codes) + row * (K / 2);
       if constexpr (!XPOSE) {
-        *reinterpret_cast<uint4*>(prow + slice * 16) =
-            make_uint4(__byte_perm(t[0], t[1], 0x6420), __byte_perm(t[2], t[3], 0x6420),
-                       __byte_perm(t[4], t[5], 0x6420), __byte_perm(t[6], t[7], 0x6420));
+        if (half)
+          *reinterpret_cast<uint2*>(prow + slice * 16) =
+              make_uint2(__byte_perm(t[0], t[1], 0x6420), __byte_perm(t[2], t[3], 0x6420));
+        else
+          *reinterpret_cast<uint4*>(prow + slice * 16) =
+              make_uint4(__byte_perm(t[0], t[1], 0x6420), __byte_perm(t[2], t[3], 0x6420),
+                         __byte_perm(t[4], t[5], 0x6420), __byte_perm(t[6], t[7], 0x6420));
       } else {
         static_assert(GS == 4, "four codes (two bytes) per register group");
         uint8_t* base = prow + (blk * N + GS * tl + (32 * G) * (member >> LX)) / 2;
@@ -556,7 +575,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_rows_kernel(const Quan
     if (!XPOSE) {
       uint4* dst = reinterpret_cast<uint4*>(crow + slice * 32);
       dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-      dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+      if (!half) dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
     } else {
       // register group g: index bits 5..4+LX = g, bits 5-LX..4 = tl, bits
       // 5+LX.. = member >> LX; GS consecutive codes per group

@@ -51,6 +51,10 @@ namespace {
 #endif
 constexpr int kSegConsumers = HQ_SEG_CONSUMERS;  // segment kernel: 8 consumer warps, 2 CTAs per SM
 constexpr int kSegThreads = kSegConsumers + 32;
+// rows of more than 256 slices (K above 8192): up to 480 consumers, one CTA
+// per SM
+constexpr int kSegConsumersBig = 480;
+constexpr int kSegThreadsBig = kSegConsumersBig + 32;
 constexpr int kSegCtas = HQ_SEG_CTAS;
 
 // Shared-memory layout (byte offsets from a 1024-aligned base): the ring of
@@ -118,7 +122,14 @@ __device__ __forceinline__ void act_setup(const QuantParams& p, uint8_t* smem, c
     float4* msm = reinterpret_cast<float4*>(smem + L.mult);
     for (int i = tid; i < 8 * p.S; i += blockDim.x) {
       const int c = i / p.S, sl = i - c * p.S;
-      msm[i] = *reinterpret_cast<const float4*>(p.mult + sl * 32 + 4 * c);
+      float4 m4 = *reinterpret_cast<const float4*>(p.mult + sl * 32 + 4 * c);
+      if (p.invert_mult) {  // the weight side multiplies by sigma = 1 / sigma_inv
+        m4.x = 1.0f / m4.x;
+        m4.y = 1.0f / m4.y;
+        m4.z = 1.0f / m4.z;
+        m4.w = 1.0f / m4.w;
+      }
+      msm[i] = m4;
     }
   }
 }
@@ -228,6 +239,11 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);
   const WaitCtl wc{p.err, p.wait_ns};
 
+  // which per-block terms the row needs: the mean after H and the weights'
+  // rotated row sum take the blocks' first input channels, the mean before H
+  // and the weights' pre-rotation sum the blocks' sums
+  const bool y0_terms = CENTER || (p.rowsum != nullptr && !p.rowsum_pre);
+  const bool sum_terms = PRE || (p.rowsum != nullptr && p.rowsum_pre);
   act_setup(p, smem, L, ncw, &tmX);
   for (int i = threadIdx.x; i < ncw * RPW * BP; i += blockDim.x) y0buf[i] = 0.0f;  // padding
   __syncthreads();
@@ -277,23 +293,26 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
           unpack32(x, w[j]);
         }
         if (p.mult) scale32(w[j], msm, S, slice);
-        // the mean's terms after H: the blocks' first input channels
-        if (CENTER && active && member == 0) {
+        // the mean's (or the row sum's) terms, one per block: the blocks'
+        // first input channels (their rotated row sums are n times these)
+        if (y0_terms && active && member == 0) {
 #pragma unroll
           for (int b = 0; b < F::BPT; ++b) y0row[blk * F::BPT + b] = w[j][first_pair<LOGN>(b)].x;
         }
         fwht32<LOGN>(w[j], xb, lane);
-        // centring before H: the blocks' rotated first channels (block sums)
-        // are the mean's terms and the only channels the centring moves;
-        // they stay out of the max / min here and enter them after the shift
-        if (PRE && member == 0) {
+        // or the blocks' rotated first channels, the block sums; centring
+        // before H moves only these channels, so they stay out of the max /
+        // min here and enter them after the shift
+        if (sum_terms && member == 0) {
 #pragma unroll
           for (int b = 0; b < F::BPT; ++b) {
             first[j][b] = w[j][first_pair<LOGN>(b)].x;
             if (active) y0row[blk * F::BPT + b] = first[j][b];
-            fmx = fmaxf(fmx, first[j][b]);
-            fmn = fminf(fmn, first[j][b]);
-            w[j][first_pair<LOGN>(b)].x = w[j][0].y;  // channel 1 of block 0 stands in
+            if (PRE) {
+              fmx = fmaxf(fmx, first[j][b]);
+              fmn = fminf(fmn, first[j][b]);
+              w[j][first_pair<LOGN>(b)].x = w[j][0].y;  // channel 1 of block 0 stands in
+            }
           }
         }
         float a, c;
@@ -322,7 +341,7 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
           rfx = unord_f32(__reduce_max_sync(segmask, ord_f32(fmx)));
           rfn = unord_f32(__reduce_min_sync(segmask, ord_f32(fmn)));
         }
-        if (CENTER || PRE) {  // in block order: independent of the tiling
+        if (y0_terms || sum_terms) {  // in block order: independent of the tiling
           const float4* y4 = reinterpret_cast<const float4*>(y0row);
           for (int b4 = 0; b4 < BP / 4; ++b4) {
             const float4 v = y4[b4];
@@ -346,6 +365,9 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
         if (MODE == 1)
           atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])), __float_as_uint(a_hat));
         if (kQuantize && p.mean) p.mean[row] = PRE ? mu : m_hat * p.inv_sqrt_n;
+        // weights: sum_k sigma_k W[n,k] (the blocks' sums) or sum_k W~[n,k] =
+        // sqrt(n) sum_b Y[b,0]
+        if (p.rowsum) p.rowsum[row] = p.rowsum_pre ? rsum : rsum * p.sqrt_n;
       }
       if (!kQuantize || !row_ok) continue;
       // q / a_hat to within 2 ulp: moves a code only when V q / a_hat lies
@@ -372,8 +394,8 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
 
 // ------------------------------------------------------------ segment kernel
 // Any K: consumer c owns slice c % S of row c / S of every tile (p.R rows).
-template <int LOGN, int MODE, int CM>
-__global__ void __launch_bounds__(kSegThreads, kSegCtas)
+template <int LOGN, int MODE, int CM, bool BIG>
+__global__ void __launch_bounds__(BIG ? kSegThreadsBig : kSegThreads, BIG ? 1 : kSegCtas)
     quant_seg_kernel(const __grid_constant__ CUtensorMap tmX, const QuantParams p) {
   using F = Fwht<LOGN>;
   constexpr bool CENTER = (CM == 1);
@@ -405,6 +427,8 @@ __global__ void __launch_bounds__(kSegThreads, kSegCtas)
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flags);
   const WaitCtl wc{p.err, p.wait_ns};
 
+  const bool y0_terms = CENTER || (p.rowsum != nullptr && !p.rowsum_pre);
+  const bool sum_terms = PRE || (p.rowsum != nullptr && p.rowsum_pre);
   act_setup(p, smem, L, ncw, &tmX);
   // neutral statistics in every slot: the slots past a row's last segment
   // are never written and combine as no-ops; the mean terms' padding is zero
@@ -460,21 +484,23 @@ __global__ void __launch_bounds__(kSegThreads, kSegCtas)
       }
       if (p.mult) scale32(w, msm, S, slice);
       float* y0row = y0buf + (pb * R + row0) * BP + blk * F::BPT;
-      if (CENTER && active && member == 0) {
+      if (y0_terms && active && member == 0) {
 #pragma unroll
         for (int b = 0; b < F::BPT; ++b) y0row[b] = w[first_pair<LOGN>(b)].x;
       }
       fwht32<LOGN>(w, xb, lane);
       float first[F::BPT];
       float fmx = -INFINITY, fmn = INFINITY;
-      if (PRE && member == 0) {
+      if (sum_terms && member == 0) {
 #pragma unroll
         for (int b = 0; b < F::BPT; ++b) {
           first[b] = w[first_pair<LOGN>(b)].x;
           if (active) y0row[b] = first[b];
-          fmx = fmaxf(fmx, first[b]);
-          fmn = fminf(fmn, first[b]);
-          w[first_pair<LOGN>(b)].x = w[0].y;  // channel 1 of block 0 stands in
+          if (PRE) {
+            fmx = fmaxf(fmx, first[b]);
+            fmn = fminf(fmn, first[b]);
+            w[first_pair<LOGN>(b)].x = w[0].y;  // channel 1 of block 0 stands in
+          }
         }
       }
       float mx, mn;
@@ -515,7 +541,7 @@ __global__ void __launch_bounds__(kSegThreads, kSegCtas)
         }
       }
       // the mean's terms in block order (independent of the tiling)
-      if (CENTER || PRE) {
+      if (y0_terms || sum_terms) {
         const float4* y4 = reinterpret_cast<const float4*>(y0buf + (pb * R + row0) * BP);
         for (int b4 = 0; b4 < BP / 4; ++b4) {
           const float4 v = y4[b4];
@@ -537,6 +563,7 @@ __global__ void __launch_bounds__(kSegThreads, kSegCtas)
         if (MODE == 1)
           atomicMax(reinterpret_cast<unsigned*>(const_cast<int*>(&flags[1])), __float_as_uint(a_hat));
         if (kQuantize && p.mean) p.mean[row] = PRE ? mu : m_hat * p.inv_sqrt_n;
+        if (p.rowsum) p.rowsum[row] = p.rowsum_pre ? rsum : rsum * p.sqrt_n;
       }
       if (!kQuantize || !row_ok) continue;
       const float rr = MODE == 0 ? (a_hat > 0.0f ? __fdividef(float(p.q), a_hat) : 0.0f) : r_tensor;
@@ -596,7 +623,42 @@ static const void* wrow_ptr(int logn, int mode, int center) {
   }
 }
 
-#if HQ_ACT_PART == 2
+template <int MODE, int CM, bool BIG>
+static const void* seg_by_logn(int logn) {
+  switch (logn) {
+    case 4: return (const void*)quant_seg_kernel<4, MODE, CM, BIG>;
+    case 5: return (const void*)quant_seg_kernel<5, MODE, CM, BIG>;
+    case 6: return (const void*)quant_seg_kernel<6, MODE, CM, BIG>;
+    case 7: return (const void*)quant_seg_kernel<7, MODE, CM, BIG>;
+    case 8: return (const void*)quant_seg_kernel<8, MODE, CM, BIG>;
+    case 9: return (const void*)quant_seg_kernel<9, MODE, CM, BIG>;
+    case 10: return (const void*)quant_seg_kernel<10, MODE, CM, BIG>;
+    default: return nullptr;
+  }
+}
+
+template <bool BIG>
+static const void* seg_ptr(int logn, int mode, int center) {
+  switch (mode * 3 + center) {
+    case 0: return seg_by_logn<0, 0, BIG>(logn);
+    case 1: return seg_by_logn<0, 1, BIG>(logn);
+    case 2: return seg_by_logn<0, 2, BIG>(logn);
+    case 3: return seg_by_logn<1, 0, BIG>(logn);
+    case 4: return seg_by_logn<1, 1, BIG>(logn);
+    case 5: return seg_by_logn<1, 2, BIG>(logn);
+    case 6: return seg_by_logn<2, 0, BIG>(logn);
+    case 7: return seg_by_logn<2, 1, BIG>(logn);
+    case 8: return seg_by_logn<2, 2, BIG>(logn);
+    case 9: return seg_by_logn<3, 0, BIG>(logn);
+    case 10: return seg_by_logn<3, 1, BIG>(logn);
+    case 11: return seg_by_logn<3, 2, BIG>(logn);
+    default: return nullptr;
+  }
+}
+
+#if HQ_ACT_PART == 5
+const void* quant_seg_big_ptr(int logn, int mode, int center) { return seg_ptr<true>(logn, mode, center); }
+#elif HQ_ACT_PART == 2
 const void* quant_wrow_ptr_spl2(int logn, int mode, int center) { return wrow_ptr<2>(logn, mode, center); }
 #elif HQ_ACT_PART == 3
 const void* quant_wrow_ptr_spl3(int logn, int mode, int center) { return wrow_ptr<3>(logn, mode, center); }
@@ -606,38 +668,12 @@ const void* quant_wrow_ptr_spl4(int logn, int mode, int center) { return wrow_pt
 const void* quant_wrow_ptr_spl2(int logn, int mode, int center);
 const void* quant_wrow_ptr_spl3(int logn, int mode, int center);
 const void* quant_wrow_ptr_spl4(int logn, int mode, int center);
+const void* quant_seg_big_ptr(int logn, int mode, int center);
 
-template <int MODE, int CM>
-static const void* seg_by_logn(int logn) {
-  switch (logn) {
-    case 4: return (const void*)quant_seg_kernel<4, MODE, CM>;
-    case 5: return (const void*)quant_seg_kernel<5, MODE, CM>;
-    case 6: return (const void*)quant_seg_kernel<6, MODE, CM>;
-    case 7: return (const void*)quant_seg_kernel<7, MODE, CM>;
-    case 8: return (const void*)quant_seg_kernel<8, MODE, CM>;
-    case 9: return (const void*)quant_seg_kernel<9, MODE, CM>;
-    case 10: return (const void*)quant_seg_kernel<10, MODE, CM>;
-    default: return nullptr;
-  }
+const void* quant_seg_kernel_ptr(int logn, int mode, int center, bool big) {
+  return big ? quant_seg_big_ptr(logn, mode, center) : seg_ptr<false>(logn, mode, center);
 }
 
-const void* quant_seg_kernel_ptr(int logn, int mode, int center) {
-  switch (mode * 3 + center) {
-    case 0: return seg_by_logn<0, 0>(logn);
-    case 1: return seg_by_logn<0, 1>(logn);
-    case 2: return seg_by_logn<0, 2>(logn);
-    case 3: return seg_by_logn<1, 0>(logn);
-    case 4: return seg_by_logn<1, 1>(logn);
-    case 5: return seg_by_logn<1, 2>(logn);
-    case 6: return seg_by_logn<2, 0>(logn);
-    case 7: return seg_by_logn<2, 1>(logn);
-    case 8: return seg_by_logn<2, 2>(logn);
-    case 9: return seg_by_logn<3, 0>(logn);
-    case 10: return seg_by_logn<3, 1>(logn);
-    case 11: return seg_by_logn<3, 2>(logn);
-    default: return nullptr;
-  }
-}
 
 const void* quant_wrow_kernel_ptr(int logn, int mode, int center, int spl) {
   switch (spl) {
@@ -650,7 +686,7 @@ const void* quant_wrow_kernel_ptr(int logn, int mode, int center, int spl) {
   }
 }
 
-int quant_seg_max_consumers() { return kSegConsumers; }
+int quant_seg_max_consumers(bool big) { return big ? kSegConsumersBig : kSegConsumers; }
 
 int quant_wrow_warps(int spl) {
   switch (spl) {
@@ -663,7 +699,7 @@ int quant_wrow_warps(int spl) {
   }
 }
 
-int quant_seg_ctas_per_sm() { return kSegCtas; }
+int quant_seg_ctas_per_sm(bool big) { return big ? 1 : kSegCtas; }
 
 size_t quant_seg_smem_bytes(int R, int S, int K, int n, int stages, int max_seg, bool pre) {
   const int ncw = (R * S + 31) / 32;

@@ -320,6 +320,14 @@ hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_
                         int32_t* quant_rows, int32_t* quant_threads, int32_t* gemm_pair,
                         int32_t* gemm_bn);
 
+/* Test hook, host only: how many tensor maps hq_linear and hq_quantize_act
+ * took from the library's cache and how many they encoded.  A tensor map
+ * depends only on its buffer's address, extents and box, so the library keeps
+ * the last 64 it encoded and reuses them for later calls on the same buffers
+ * and shapes (no per-call encoding on the host).  Outputs are host pointers
+ * and may be NULL; counts are cumulative for the process. */
+hq_status hq_debug_tmap_cache(uint64_t* hits, uint64_t* misses);
+
 /* Measurement hook (no counterpart on the pages): the int8 tensor-core
  * ceiling of this device, the denominator the GEMM's throughput is reported
  * against beside the nominal figure.  Launches the GEMM's main loop with

@@ -60,7 +60,19 @@ def test_quantize_validation(hq):
     assert _call_quant(hq, D(1024, 16, 8)) == 2             # order below 16
     assert _call_quant(hq, D(1000, 16, 8)) == 2
     assert _call_quant(hq, D(96, 16, 64)) == 2              # K not a multiple of the order
-    assert _call_quant(hq, D(16384, 16, 1024)) == 2         # K above the limit
+    assert _call_quant(hq, D(16384, 16, 1024)) == 2         # K above the limit (15360)
+    # K: a multiple of 16 and of the order; up to 15360 with a rotation, 10240
+    # without one
+    assert _call_quant(hq, D(80, 16, 16), T=0) == 0
+    assert _call_quant(hq, D(80, 16, 1, centering=0), T=0) == 0
+    assert _call_quant(hq, D(88, 16, 8)) == 2                  # K not a multiple of 16
+    assert _call_quant(hq, D(12288, 16, 1024), T=0) == 0
+    assert _call_quant(hq, D(15360, 16, 1024), T=0) == 0
+    assert _call_quant(hq, D(15872, 16, 512)) == 2
+    assert _call_quant(hq, D(10240, 16, 1, centering=0), T=0) == 0
+    assert _call_quant(hq, D(10496, 16, 1, centering=0)) == 2
+    # two codes per byte need rows of whole 16-byte units (K a multiple of 32)
+    assert _call_quant(hq, D(80, 16, 16, code_format=1)) == 2
     assert _call_quant(hq, D(1024, 15, 1024)) == 2          # N not a multiple of 16
     assert _call_quant(hq, D(1024, 16, 1024, a_bits=5)) == 2
     assert _call_quant(hq, D(1024, 16, 1024, w_bits=3)) == 2

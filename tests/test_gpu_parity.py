@@ -79,7 +79,15 @@ SMALL_PRE = [(n * B, n, T, (4, 3, 8)[i % 3], 2, i % 2 == 0)
                                             (128, 16, 129), (1024, 4, 7), (1024, 5, 129)])]
 
 
-@pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL + SMALL_PRE)
+# K a multiple of 16 but not of 32 (n = 16: the row's last slice holds 16
+# channels), and rows longer than 8192 channels
+SMALL_ENVELOPE = [(80, 16, T, 4, c, True) for T, c in ((1, 0), (7, 1), (300, 2))] + \
+                 [(144, 16, 129, 3, 1, False), (16 * 27, 16, 65, 8, 0, True)] + \
+                 [(12288, n, T, 4, c, True) for n, T, c in ((1024, 7, 1), (256, 33, 2),
+                                                           (128, 3, 0))]
+
+
+@pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL + SMALL_PRE + SMALL_ENVELOPE)
 def test_quantize_small(hq, K, n, T, bits, center, use_sigma):
     g = np.random.default_rng(K * 1000 + T)
     x = g.standard_normal((T, K)).astype(np.float32)
@@ -158,7 +166,11 @@ def test_exact_ties_are_rounded_half_to_even(hq):
                           (64, 1152, 128, 4, True, 1), (32, 3072, 1024, 4, True, 1),
                           (320, 320, 64, 8, False, 0), (1024, 1024, 1024, 4, True, 1),
                           (64, 1152, 128, 4, True, 2), (48, 512, 16, 8, False, 2),
-                          (32, 3072, 1024, 4, True, 2)])
+                          (32, 3072, 1024, 4, True, 2),
+                          # K a multiple of 16 only (n = 16), and K above 8192
+                          (48, 80, 16, 4, True, 1), (32, 144, 16, 8, True, 2),
+                          (16, 12288, 1024, 4, True, 1), (16, 12288, 256, 4, True, 2),
+                          (32, 4096, 512, 4, True, 1), (32, 2048, 64, 8, False, 0)])
 def test_prepare_weights(hq, N, K, n, w_bits, use_sigma, center):
     g = np.random.default_rng(N + K)
     Xb = synth.f32_to_bf16_bits(g.standard_normal((64, K)).astype(np.float32) *
@@ -713,3 +725,65 @@ def test_forward_host_equals_the_device_path(hq, idx, T, over, chunks):
         g.replay()
         torch.cuda.synchronize()
         assert torch.equal(Y_host.view(torch.int16), R.view(torch.int16))
+
+
+def test_tensor_maps_are_reused_across_calls(hq):
+    """Repeated calls on the same buffers and shapes take their tensor maps
+    from the library's cache (no host encoding per call) and still compute
+    the same output; a new output buffer costs one new map."""
+    cfg = synth.CONFIGS[2].with_tokens(300)
+    Xb, Wb, bb = synth.make_layer(cfg)
+    T, K = Xb.shape
+    N = Wb.shape[0]
+    desc = hq.LayerDesc(K, N, cfg.had_order, a_bits=cfg.a_bits, w_bits=cfg.w_bits,
+                        act_gran=cfg.act_gran, centering=cfg.centering)
+    X = to_dev_u16(Xb, torch)
+    layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), None)
+    Y1 = torch.empty((T, N), dtype=torch.bfloat16, device="cuda")
+    layer(X, Y1)
+    torch.cuda.synchronize()
+    c0 = hq.hq_debug_tmap_cache()
+    for _ in range(3):
+        layer(X, Y1)
+    torch.cuda.synchronize()
+    c1 = hq.hq_debug_tmap_cache()
+    # three GEMM maps and one quantizer map per step, all from the cache
+    assert c1["misses"] == c0["misses"] and c1["hits"] - c0["hits"] == 3 * 4
+    Y2 = torch.empty_like(Y1)
+    layer(X, Y2)
+    torch.cuda.synchronize()
+    c2 = hq.hq_debug_tmap_cache()
+    assert c2["misses"] == c1["misses"] + 1
+    assert hq.hq_check_device_error() == 0
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("K,n,N,T,gran", [(80, 16, 48, 130, 0), (144, 16, 64, 33, 1),
+                                         (12288, 1024, 256, 129, 0), (12288, 256, 128, 40, 1)])
+def test_layer_at_the_shape_envelope(hq, K, n, N, T, gran):
+    """The whole layer where K is a multiple of 16 only, and where K exceeds
+    8192: codes, exact accumulators and output against the oracle."""
+    g = np.random.default_rng(K + N + T)
+    x = g.standard_normal((T, K)).astype(np.float32)
+    x[:, g.choice(K, size=max(1, K // 100), replace=False)] *= 25.0
+    x += g.standard_normal((T, 1)).astype(np.float32)
+    Xb = synth.f32_to_bf16_bits(x)
+    Wb = synth.f32_to_bf16_bits((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    bb = synth.f32_to_bf16_bits((g.standard_normal(N) * 0.01).astype(np.float32))
+    ref = oracle.layer(Xb, Wb, bb, n, 4, 4, gran=gran, centering=1)
+    desc = hq.LayerDesc(K, N, n, a_bits=4, w_bits=4, act_gran=gran, centering=1)
+    X = to_dev_u16(Xb, torch)
+    absmax = torch.zeros(K, dtype=torch.float32, device="cuda")
+    hq.hq_calib_act_absmax(desc, X, absmax)
+    layer = hq.HadamardQuantLinear(desc, to_dev_u16(Wb, torch), to_dev_u16(bb, torch), absmax, 0.5)
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    Y = layer(X, acc_debug=acc)
+    assert hq.hq_check_device_error() == 0
+    check_codes(layer.w_codes.cpu().numpy(), ref["w"]["codes"], ref["w"]["tie"], "w_codes")
+    codes = layer.buffers(T)["a_codes"].cpu().numpy()
+    check_codes(codes, ref["a"]["codes"], ref["a"]["tie"], "a_codes")
+    same = np.all(codes == ref["a"]["codes"], axis=1)
+    wsame = np.all(layer.w_codes.cpu().numpy() == ref["w"]["codes"], axis=1)
+    a = acc.cpu().numpy()
+    assert np.array_equal(a[np.ix_(same, wsame)], ref["acc"][np.ix_(same, wsame)])
+    assert rel_frob(bf16_bits(Y), ref["y_bf16"]) <= Y_REL_FROB

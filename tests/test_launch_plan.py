@@ -57,7 +57,7 @@ def test_forms_that_exclude_the_pair_or_wide_tiles(hq):
 
 
 def test_plan_invariants_over_shapes(hq):
-    Ks = [64, 320, 1024, 1152, 3072, 4608, 9216]
+    Ks = [64, 320, 1024, 1152, 3072, 4608, 9216, 12288, 15360]
     Ts = [1, 7, 127, 128, 1000, 8192, 65536]
     Ns = [16, 320, 3456, 12288]
     for K, T, N, packed in itertools.product(Ks, Ts, Ns, (0, 1)):
@@ -70,10 +70,9 @@ def test_plan_invariants_over_shapes(hq):
             assert R == (nt // 32 - 1) * (32 // S)
         elif S % 32 == 0 and S <= 128:  # warp-row kernel, one row per warp
             assert R == nt // 32 - 1
-        elif R * S <= 256:  # segment kernel: one thread per slice, plus the producer warp
-            assert R * S + 32 <= nt < R * S + 64
-        else:  # the row kernel (K above 8192): one thread per slice
-            assert R * S <= nt < R * S + 32 and R * S <= 320
+        else:  # segment kernel: one thread per slice, plus the producer warp
+            # (up to 256 slices a tile, or 480 in the large-row variant)
+            assert R * S + 32 <= nt < R * S + 64 and R * S <= (256 if S <= 256 else 480)
         assert p["gemm_bn"] in (64, 128, 192, 256)
         if packed:
             assert not p["gemm_pair"] and p["gemm_bn"] <= 192
