@@ -12,7 +12,10 @@ g++ and marshals numpy arrays through ctypes.
 Parity pins: see ``tests/test_oracle_pins.py`` (Hadamard orthogonality and the
 Sylvester recursion, the Eq. (1) identity with quantization off, hand-worked
 quantizer examples, brute force at K = 4 / 8, closed-form invariants, integer
-accumulation).  Every function here is pinned there; none is "parity unpinned".
+accumulation; for the group-wise int4 form with its low-rank branch a
+hand-worked two-group example, the unquantized identity and brute force of the
+group quantizer against the per-token one).  Every function here is pinned
+there; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -75,6 +78,16 @@ def _load():
                 _u16p, _u16p, _f64p, _f64p, _i8p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
                 ctypes.c_int]
             lib.hqo_channel_mean.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int64, _f64p]
+            _i64 = ctypes.c_int64
+            lib.hqo_gw_prepare_weights.argtypes = [
+                _i64, _i64, _i64, ctypes.c_int, _i64, _u16p, _u16p, _f64p, _f64p, _f64p,
+                _u16p, _u16p, _i8p, _f64p, _f64p, _f64p, _f64p, ctypes.c_int]
+            lib.hqo_gw_quantize_act.argtypes = [
+                _i64, _i64, ctypes.c_int, _i64, _u16p, _i64, _f64p, _u16p, _i64p, _i64,
+                _i8p, _f64p, _u16p, _f64p, _f64p, ctypes.c_int]
+            lib.hqo_gw_epilogue.argtypes = [
+                _i8p, _i8p, _i64, _i64, _i64, _i64, _f64p, _f64p, _u16p, _u16p, _i64, _f64p,
+                _f64p, _u16p, ctypes.c_int]
             lib.hqo_gemm_acc.argtypes = [_i8p, _i8p, ctypes.c_int64, ctypes.c_int64,
                                          ctypes.c_int64, _i64p, ctypes.c_int64, _i64p,
                                          ctypes.c_int]
@@ -94,6 +107,7 @@ def _load():
             lib.hqo_unpack_i4.argtypes = [_u8p, ctypes.c_int64, _i8p]
             for name in ("hqo_pack_i4", "hqo_unpack_i4", "hqo_sylvester", "hqo_col_absmax",
                          "hqo_channel_mean", "hqo_sigma", "hqo_quantize_act",
+                         "hqo_gw_prepare_weights", "hqo_gw_quantize_act", "hqo_gw_epilogue",
                          "hqo_prepare_weights", "hqo_gemm_acc", "hqo_epilogue",
                          "hqo_exact_linear", "hqo_prepare_weights_wh", "hqo_epilogue_wh",
                          "hqo_output_rotation"):
@@ -409,3 +423,110 @@ def layer_wh(X_bits, W_bits, bias_bits, n_out, a_bits, w_bits, gran=0, alpha=0.5
     acc = gemm_acc(a["codes"], w["codes"], nthreads=nthreads)
     y, yb = epilogue_wh(acc, n_out, a["scale"], w["scale"], b_bar=w["b_bar"])
     return {"sigma": sig, "w": w, "a": a, "acc": acc, "y": y, "y_bf16": yb}
+
+
+# ---------------------------------------------------------------------------
+# group-wise form with a low-rank branch ("Data-free 4-bit quantization for
+# diffusion transformers", "Hadamard rotation: the int4 improvement")
+# ---------------------------------------------------------------------------
+
+def low_rank_factors(W_bits, sigma, rank):
+    """Rank-r factors of W^ = W diag(sigma) ([N,K]) from its singular value
+    decomposition: L2 = U_r diag(S_r) [N,r], L1 = V_r^T [r,K] (fp64).  A
+    library routine serves as this step (the method fixes only L2 L1, the
+    best rank-r approximation)."""
+    W = bf16_to_f64(_c(W_bits, np.uint16))
+    if sigma is not None:
+        W = W * np.asarray(sigma, dtype=np.float64)[None, :]
+    if rank == 0:
+        return np.zeros((0, W.shape[1])), np.zeros((W.shape[0], 0))
+    U, S, Vt = np.linalg.svd(W, full_matrices=False)
+    return np.ascontiguousarray(Vt[:rank]), np.ascontiguousarray(U[:, :rank] * S[:rank])
+
+
+def gw_prepare_weights(W_bits, g, bits, rank, L1, L2, bias_bits=None, sigma=None,
+                       want_tie=True, want_Rh=False, nthreads=None):
+    """Returns dict(codes [N,K], gscale [N,K/g], l1 bf16 bits [r,K], l2 bf16
+    bits [N,r], bias [N], tie, Rh)."""
+    W = _c(W_bits, np.uint16)
+    N, K = W.shape
+    b = _c(bias_bits, np.uint16)
+    sig = _c(sigma, np.float64)
+    l1 = np.zeros((rank, K), dtype=np.uint16)
+    l2 = np.zeros((N, rank), dtype=np.uint16)
+    codes = np.zeros((N, K), dtype=np.int8)
+    gscale = np.zeros((N, K // g), dtype=np.float64)
+    bias = np.zeros(N, dtype=np.float64)
+    tie = np.zeros((N, K), dtype=np.float64) if want_tie else None
+    Rh = np.zeros((N, K), dtype=np.float64) if want_Rh else None
+    L1c = _c(L1, np.float64) if rank else None
+    L2c = _c(L2, np.float64) if rank else None
+    rc = _load().hqo_gw_prepare_weights(
+        K, N, g, bits, rank, _ptr(W, ctypes.c_uint16), _ptr(b, ctypes.c_uint16),
+        _ptr(sig, ctypes.c_double), _ptr(L1c, ctypes.c_double), _ptr(L2c, ctypes.c_double),
+        _ptr(l1, ctypes.c_uint16), _ptr(l2, ctypes.c_uint16), _ptr(codes, ctypes.c_int8),
+        _ptr(gscale, ctypes.c_double), _ptr(bias, ctypes.c_double), _ptr(tie, ctypes.c_double),
+        _ptr(Rh, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "gw_prepare_weights")
+    return {"codes": codes, "gscale": gscale, "l1": l1, "l2": l2, "bias": bias, "tie": tie,
+            "Rh": Rh}
+
+
+def gw_quantize_act(X_bits, g, bits, rank, l1_bits, sigma=None, rows=None, want_tie=True,
+                    want_Z=False, nthreads=None):
+    """Returns dict(codes [r,K], gscale [r,K/g], u bf16 bits [r,rank], tie, Z)."""
+    X = _c(X_bits, np.uint16)
+    T, K = X.shape
+    sig = _c(sigma, np.float64)
+    l1 = _c(l1_bits, np.uint16) if rank else None
+    r = None if rows is None else _c(rows, np.int64)
+    nr = T if r is None else r.size
+    codes = np.zeros((nr, K), dtype=np.int8)
+    gscale = np.zeros((nr, K // g), dtype=np.float64)
+    u = np.zeros((nr, rank), dtype=np.uint16)
+    tie = np.zeros((nr, K), dtype=np.float64) if want_tie else None
+    Z = np.zeros((nr, K), dtype=np.float64) if want_Z else None
+    rc = _load().hqo_gw_quantize_act(
+        K, g, bits, rank, _ptr(X, ctypes.c_uint16), T, _ptr(sig, ctypes.c_double),
+        _ptr(l1, ctypes.c_uint16), _ptr(r, ctypes.c_int64), nr, _ptr(codes, ctypes.c_int8),
+        _ptr(gscale, ctypes.c_double), _ptr(u, ctypes.c_uint16), _ptr(tie, ctypes.c_double),
+        _ptr(Z, ctypes.c_double), nthreads or default_threads())
+    _check(rc, "gw_quantize_act")
+    return {"codes": codes, "gscale": gscale, "u": u, "tie": tie, "Z": Z}
+
+
+def gw_epilogue(A, B, g, ascale, wscale, u_bits, l2_bits, bias=None, nthreads=None):
+    """(y fp64, y bf16 bits) of the group-wise form's output."""
+    A = _c(A, np.int8)
+    B = _c(B, np.int8)
+    nr, K = A.shape
+    N = B.shape[0]
+    rank = 0 if u_bits is None else np.asarray(u_bits).shape[1]
+    a = _c(ascale, np.float64)
+    w = _c(wscale, np.float64)
+    u = _c(u_bits, np.uint16) if rank else None
+    l2 = _c(l2_bits, np.uint16) if rank else None
+    b = _c(bias, np.float64)
+    y = np.zeros((nr, N), dtype=np.float64)
+    yb = np.zeros((nr, N), dtype=np.uint16)
+    rc = _load().hqo_gw_epilogue(
+        _ptr(A, ctypes.c_int8), _ptr(B, ctypes.c_int8), nr, N, K, g, _ptr(a, ctypes.c_double),
+        _ptr(w, ctypes.c_double), _ptr(u, ctypes.c_uint16), _ptr(l2, ctypes.c_uint16), rank,
+        _ptr(b, ctypes.c_double), _ptr(y, ctypes.c_double), _ptr(yb, ctypes.c_uint16),
+        nthreads or default_threads())
+    _check(rc, "gw_epilogue")
+    return y, yb
+
+
+def layer_gw(X_bits, W_bits, bias_bits, g=64, bits=4, rank=32, sigma=None, rows=None,
+             factors=None, nthreads=None):
+    """The group-wise form end to end for the listed rows; factors = (L1, L2)
+    or None for the rank-r SVD of W diag(sigma)."""
+    L1, L2 = factors if factors is not None else low_rank_factors(W_bits, sigma, rank)
+    w = gw_prepare_weights(W_bits, g, bits, rank, L1, L2, bias_bits=bias_bits, sigma=sigma,
+                           nthreads=nthreads)
+    a = gw_quantize_act(X_bits, g, bits, rank, w["l1"], sigma=sigma, rows=rows,
+                        nthreads=nthreads)
+    y, yb = gw_epilogue(a["codes"], w["codes"], g, a["gscale"], w["gscale"], a["u"], w["l2"],
+                        bias=w["bias"], nthreads=nthreads)
+    return {"w": w, "a": a, "y": y, "y_bf16": yb, "L1": L1, "L2": L2}

@@ -538,3 +538,147 @@ int hqo_unpack_i4(const uint8_t* packed, int64_t count, int8_t* codes) {
 }
 
 }  /* extern "C" */
+
+/* ---------------------------------------------------------------------------
+ * Group-wise form with a low-rank branch (see hq_oracle.h). */
+
+namespace {
+/* The symmetric quantizer of one group of values: s = max |v| / q, codes
+ * rne(v q / max) (one rounding), clamp; s = 0 gives zero codes. */
+void quantize_group(const double* v, int64_t g, double q, int8_t* codes, double* scale,
+                    double* tie) {
+  double a = 0.0;
+  for (int64_t i = 0; i < g; ++i) a = std::fmax(a, std::fabs(v[i]));
+  *scale = a / q;
+  for (int64_t i = 0; i < g; ++i) {
+    double c = 0.0, d = 0.5;
+    if (a > 0.0) {
+      const double x = (v[i] * q) / a;
+      c = clampd(hqo_rne(x), -q, q);
+      const double ax = std::fabs(x);
+      d = std::fabs(ax - std::floor(ax) - 0.5);
+    }
+    codes[i] = int8_t(c);
+    if (tie) tie[i] = d;
+  }
+}
+}  // namespace
+
+extern "C" {
+
+int hqo_gw_prepare_weights(int64_t K, int64_t N, int64_t g, int bits, int64_t rank,
+                           const uint16_t* W, const uint16_t* bias, const double* sigma,
+                           const double* L1, const double* L2, uint16_t* l1s, uint16_t* l2b,
+                           int8_t* w_codes, double* w_gscale, double* bias_out, double* tie,
+                           double* Rh, int nthreads) {
+  if (K <= 0 || N <= 0 || !is_pow2(g) || K % g != 0 || bits < 2 || bits > 8 || rank < 0)
+    return -1;
+  if (W == nullptr || w_codes == nullptr || w_gscale == nullptr || bias_out == nullptr)
+    return -1;
+  if (rank > 0 && (L1 == nullptr || L2 == nullptr || l1s == nullptr || l2b == nullptr)) return -1;
+  const double q = double(qmax_for_bits(bits));
+  const std::vector<double> Hg = dense_block(g);
+  const int64_t G = K / g;
+  /* the 16-bit factors: l2 = bf16(L2), l1 = bf16(L1 diag(sigma^-1)) */
+  for (int64_t r = 0; r < rank; ++r)
+    for (int64_t k = 0; k < K; ++k)
+      l1s[r * K + k] = hqo_f64_to_bf16(L1[r * K + k] / (sigma ? sigma[k] : 1.0));
+  for (int64_t i = 0; i < N * rank; ++i) l2b[i] = hqo_f64_to_bf16(L2[i]);
+  parallel_rows(N, nthreads, [&](int64_t c) {
+    /* R[c,k] = W[c,k] sigma_k - sum_r l2[c,r] l1[r,k] sigma_k */
+    std::vector<double> R(K);
+    for (int64_t k = 0; k < K; ++k) {
+      const double s = sigma ? sigma[k] : 1.0;
+      double lr = 0.0;
+      for (int64_t r = 0; r < rank; ++r)
+        lr += hqo_bf16_to_f64(l2b[c * rank + r]) * hqo_bf16_to_f64(l1s[r * K + k]);
+      R[k] = hqo_bf16_to_f64(W[c * K + k]) * s - lr * s;
+    }
+    /* R H, one g x g block per group, then the group quantizer */
+    std::vector<double> v(g);
+    for (int64_t j = 0; j < G; ++j) {
+      for (int64_t i = 0; i < g; ++i) {
+        double acc = 0.0;
+        for (int64_t m = 0; m < g; ++m) acc += R[j * g + m] * Hg[size_t(m * g + i)];
+        v[i] = acc;
+        if (Rh) Rh[c * K + j * g + i] = acc;
+      }
+      quantize_group(v.data(), g, q, w_codes + c * K + j * g, w_gscale + c * G + j,
+                     tie ? tie + c * K + j * g : nullptr);
+    }
+    bias_out[c] = bias ? hqo_bf16_to_f64(bias[c]) : 0.0;
+  });
+  return 0;
+}
+
+int hqo_gw_quantize_act(int64_t K, int64_t g, int bits, int64_t rank, const uint16_t* X,
+                        int64_t T, const double* sigma, const uint16_t* l1s, const int64_t* rows,
+                        int64_t nrows, int8_t* codes, double* gscale, uint16_t* u, double* tie,
+                        double* Z, int nthreads) {
+  if (K <= 0 || !is_pow2(g) || K % g != 0 || bits < 2 || bits > 8 || rank < 0) return -1;
+  if (X == nullptr || T < 0 || nrows < 0 || codes == nullptr || gscale == nullptr) return -1;
+  if (rank > 0 && (l1s == nullptr || u == nullptr)) return -1;
+  if (rows == nullptr && nrows != T) return -1;
+  if (rows != nullptr) {
+    for (int64_t i = 0; i < nrows; ++i)
+      if (rows[i] < 0 || rows[i] >= T) return -1;
+  }
+  const double q = double(qmax_for_bits(bits));
+  const std::vector<double> Hg = dense_block(g);
+  const int64_t G = K / g;
+  parallel_rows(nrows, nthreads, [&](int64_t i) {
+    const int64_t t = rows ? rows[i] : i;
+    /* the 16-bit branch's down projection of the original input */
+    for (int64_t r = 0; r < rank; ++r) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k)
+        acc += hqo_bf16_to_f64(X[t * K + k]) * hqo_bf16_to_f64(l1s[r * K + k]);
+      u[i * rank + r] = hqo_f64_to_bf16(acc);
+    }
+    /* x^ H per group, then the group quantizer */
+    std::vector<double> xh(K), v(g);
+    for (int64_t k = 0; k < K; ++k)
+      xh[k] = hqo_bf16_to_f64(X[t * K + k]) / (sigma ? sigma[k] : 1.0);
+    for (int64_t j = 0; j < G; ++j) {
+      for (int64_t c = 0; c < g; ++c) {
+        double acc = 0.0;
+        for (int64_t m = 0; m < g; ++m) acc += xh[j * g + m] * Hg[size_t(m * g + c)];
+        v[c] = acc;
+        if (Z) Z[i * K + j * g + c] = acc;
+      }
+      quantize_group(v.data(), g, q, codes + i * K + j * g, gscale + i * G + j,
+                     tie ? tie + i * K + j * g : nullptr);
+    }
+  });
+  return 0;
+}
+
+int hqo_gw_epilogue(const int8_t* A, const int8_t* B, int64_t nrows, int64_t N, int64_t K,
+                    int64_t g, const double* ascale, const double* wscale, const uint16_t* u,
+                    const uint16_t* l2b, int64_t rank, const double* b, double* y,
+                    uint16_t* y_bf16, int nthreads) {
+  if (A == nullptr || B == nullptr || ascale == nullptr || wscale == nullptr || nrows < 0 ||
+      N <= 0 || K <= 0 || !is_pow2(g) || K % g != 0 || rank < 0)
+    return -1;
+  if (rank > 0 && (u == nullptr || l2b == nullptr)) return -1;
+  const int64_t G = K / g;
+  parallel_rows(nrows, nthreads, [&](int64_t i) {
+    for (int64_t c = 0; c < N; ++c) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < G; ++j) {
+        int64_t s = 0; /* the group's integer sum, exact */
+        for (int64_t k = j * g; k < (j + 1) * g; ++k) s += int64_t(A[i * K + k]) * int64_t(B[c * K + k]);
+        acc += ascale[i * G + j] * wscale[c * G + j] * double(s);
+      }
+      for (int64_t r = 0; r < rank; ++r)
+        acc += hqo_bf16_to_f64(u[i * rank + r]) * hqo_bf16_to_f64(l2b[c * rank + r]);
+      if (b) acc += b[c];
+      if (y) y[i * N + c] = acc;
+      if (y_bf16) y_bf16[i * N + c] = hqo_f64_to_bf16(acc);
+    }
+  });
+  return 0;
+}
+
+}  /* extern "C" */
+

@@ -144,6 +144,44 @@ int hqo_epilogue_wh(const int64_t* acc, int64_t nrows, int64_t N, int64_t n_out,
 int hqo_output_rotation(const double* M, int64_t rows, int64_t N, int64_t n_out,
                         double* out);
 
+/* Group-wise form with a low-rank branch ("Data-free 4-bit quantization for
+ * diffusion transformers", "Hadamard rotation: the int4 improvement", steps
+ * 1-7), in the [N,K] orientation (y[t,n] = sum_k W[n,k] X[t,k] + b[n]):
+ *   smoothing   x^ = X diag(sigma^-1),  W^ = W diag(sigma)          (step 2)
+ *   low rank    W^ = L2 L1 + R; the factors are kept in 16 bits: l2 =
+ *               bf16(L2), and the down factor with the smoothing folded in,
+ *               l1 = bf16(L1 diag(sigma^-1)), so that L1 x^ is computed as
+ *               l1 X; R is what the 16-bit branch leaves,
+ *               R = W^ - l2 l1 diag(sigma)                           (step 3)
+ *   rotation    H = diag(H_g, ..., H_g) (normalized Sylvester, one block per
+ *               quantization group of g channels): R H and x^ H       (5-7)
+ *   quantizers  per output channel and group of R H, per token and group of
+ *               x^ H: s = max |.| / q over the group's g values, codes =
+ *               clamp(rne(. / s), +-q)                                (4, 6)
+ *   output      y = sum_groups s_x s_w (codes . codes) + l2 bf16(l1 X) + b
+ * The caller supplies the rank-r factors L1 [rank,K] and L2 [N,rank] (fp64),
+ * e.g. from a singular value decomposition of W^; the method fixes only
+ * their product. */
+int hqo_gw_prepare_weights(int64_t K, int64_t N, int64_t g, int bits, int64_t rank,
+                           const uint16_t* W, const uint16_t* bias, const double* sigma,
+                           const double* L1, const double* L2, uint16_t* l1s, uint16_t* l2b,
+                           int8_t* w_codes, double* w_gscale, double* bias_out, double* tie,
+                           double* Rh, int nthreads);
+/* Activations for the listed rows: codes [nrows,K], gscale [nrows,K/g]
+ * (per token and group), u [nrows,rank] = bf16(l1 X) (the 16-bit branch's
+ * down projection, fp64 sums); optional tie and Z (x^ H) [nrows,K]. */
+int hqo_gw_quantize_act(int64_t K, int64_t g, int bits, int64_t rank, const uint16_t* X,
+                        int64_t T, const double* sigma, const uint16_t* l1s, const int64_t* rows,
+                        int64_t nrows, int8_t* codes, double* gscale, uint16_t* u, double* tie,
+                        double* Z, int nthreads);
+/* y[i,n] = sum_j ascale[i,j] wscale[n,j] sum_{k in group j} A[i,k] B[n,k]
+ *          + sum_r u[i,r] l2b[n,r] + b[n]   (fp64; the integer sums exact),
+ * and its bf16 rounding (either output may be NULL; b may be NULL). */
+int hqo_gw_epilogue(const int8_t* A, const int8_t* B, int64_t nrows, int64_t N, int64_t K,
+                    int64_t g, const double* ascale, const double* wscale, const uint16_t* u,
+                    const uint16_t* l2b, int64_t rank, const double* b, double* y,
+                    uint16_t* y_bf16, int nthreads);
+
 /* Packed storage of 3- and 4-bit codes, two per byte.  The blog "Data-free
  * 4-bit quantization for diffusion transformers" ("Hadamard rotation: the int4
  * improvement") runs a W4A4 GEMM on 4-bit operands but fixes no storage

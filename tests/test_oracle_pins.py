@@ -753,3 +753,88 @@ def test_channel_centring_zeroes_every_channel_sum():
     # without the shift the channel sums are far from zero
     a0 = oracle.quantize_act(X, 64, 8, centering=0, want_Z=True)
     assert np.max(np.abs(a0["Z"].sum(axis=0))) > 10.0
+
+
+# --------------------------------------------------------------------------
+# Group-wise int4 with a 16-bit low-rank branch: "Data-free 4-bit quantization
+# for diffusion transformers", "Hadamard rotation: the int4 improvement",
+# steps 1-7 (W^ = L2 L1 + R; y ~ L2 (L1 x^) + Q(R H) Q(H x^); one H_g block and
+# one scale per group of g input channels)
+# --------------------------------------------------------------------------
+
+def test_group_wise_hand_worked_example():
+    """Worked by hand with g = 4, K = 8, rank 1, sigma = 1, H_4 = H~_4 / 2:
+      L1 = [0.5 0.5 0.5 0.5 0 0 0 0], L2 = [2, 0]^T; W row 0 = [1 1 1 1 2 0 0 2],
+      row 1 = [0 0 0 0 1 1 1 1]; so R row 0 = [0 0 0 0 2 0 0 2], row 1 = W row 1.
+      R H per group: row 0 -> [0 0 0 0 | 2 0 0 2] (group 0 all zero: scale 0),
+      row 1 -> [0 0 0 0 | 2 0 0 0]; int4 codes [. | 7 0 0 7] and [. | 7 0 0 0],
+      scales 2/7.
+      x = [1 2 3 4 1 0 0 1]: x H per group = [5 -1 -2 0 | 1 0 0 1], codes
+      rne([7, -1.4, -2.8, 0]) = [7 -1 -3 0] and [7 0 0 7], scales 5/7, 1/7;
+      u = L1 x = 0.5 * 10 = 5.
+      y0 = (1/7)(2/7)(49 + 49) + 5 * 2 + 0.5 = 14.5 = W0 x + b0 exactly;
+      y1 = (1/7)(2/7) 49 - 0.25 = 1.75 = W1 x + b1 exactly."""
+    W = np.array([_bf16_bits([1.0, 1.0, 1.0, 1.0, 2.0, 0.0, 0.0, 2.0]),
+                  _bf16_bits([0.0, 0.0, 0.0, 0.0, 1.0, 1.0, 1.0, 1.0])], dtype=np.uint16)
+    b = np.array(_bf16_bits([0.5]) + [0xBE80], dtype=np.uint16)  # 0.5, -0.25
+    X = np.array([_bf16_bits([1.0, 2.0, 3.0, 4.0, 1.0, 0.0, 0.0, 1.0])], dtype=np.uint16)
+    L1 = np.array([[0.5, 0.5, 0.5, 0.5, 0.0, 0.0, 0.0, 0.0]])
+    L2 = np.array([[2.0], [0.0]])
+    out = oracle.layer_gw(X, W, b, g=4, bits=4, rank=1, factors=(L1, L2))
+    w, a = out["w"], out["a"]
+    assert w["codes"].tolist() == [[0, 0, 0, 0, 7, 0, 0, 7], [0, 0, 0, 0, 7, 0, 0, 0]]
+    assert w["gscale"].tolist() == [[0.0, pytest.approx(2 / 7)], [0.0, pytest.approx(2 / 7)]]
+    assert a["codes"].tolist() == [[7, -1, -3, 0, 7, 0, 0, 7]]
+    assert a["gscale"].tolist() == [[pytest.approx(5 / 7), pytest.approx(1 / 7)]]
+    assert oracle.bf16_to_f64(a["u"]).tolist() == [[5.0]]
+    assert out["y"].tolist() == [[pytest.approx(14.5, abs=1e-12), pytest.approx(1.75, abs=1e-12)]]
+
+
+@pytest.mark.parametrize("K,g,N,T,rank", [(128, 64, 16, 5, 4), (256, 16, 24, 3, 0),
+                                          (512, 64, 32, 4, 32)])
+def test_group_wise_identity_unquantized(K, g, N, T, rank):
+    """With the codes replaced by the values they quantize, the form is
+    exact: R H times x^ H (H H = I) plus the 16-bit branch's l2 (l1 X) (its
+    sum unrounded) plus b reproduces X W^T + b to 1e-10 relative -- whatever
+    the factors and sigma, because R is what the rounded factors leave."""
+    gen = np.random.default_rng(K + g + rank)
+    X = synth.f32_to_bf16_bits((gen.standard_normal((T, K)) * 2).astype(np.float32))
+    W = synth.f32_to_bf16_bits((gen.standard_normal((N, K)) * 0.05).astype(np.float32))
+    b = synth.f32_to_bf16_bits((gen.standard_normal(N) * 0.1).astype(np.float32))
+    sig = oracle.sigma(oracle.col_absmax(X), oracle.col_absmax(W), 0.5)
+    L1, L2 = oracle.low_rank_factors(W, sig, rank)
+    w = oracle.gw_prepare_weights(W, g, 4, rank, L1, L2, bias_bits=b, sigma=sig, want_Rh=True)
+    a = oracle.gw_quantize_act(X, g, 4, rank, w["l1"], sigma=sig, want_Z=True)
+    Xf = oracle.bf16_to_f64(X)
+    lr = (Xf @ oracle.bf16_to_f64(w["l1"]).T) @ oracle.bf16_to_f64(w["l2"]).T if rank else 0.0
+    y = a["Z"] @ w["Rh"].T + lr + w["bias"][None, :]
+    exact = oracle.exact_linear(X, W, b)
+    assert np.linalg.norm(y - exact) <= 1e-10 * np.linalg.norm(exact)
+
+
+def test_group_quantizer_is_the_token_quantizer_per_group():
+    """Brute force over every x in {-2..2}^8 with g = 4: each group's codes
+    and scale equal the (independently pinned) per-token quantizer applied to
+    that group's 4 values alone (n = K = 4, no centring)."""
+    vals = np.array(list(itertools.product([-2, -1, 0, 1, 2], repeat=8)), dtype=np.float32)
+    X = synth.f32_to_bf16_bits(vals)
+    a = oracle.gw_quantize_act(X, 4, 4, 0, None, want_tie=False)
+    for j in range(2):
+        ref = oracle.quantize_act(np.ascontiguousarray(X[:, 4 * j:4 * j + 4]), 4, 4, gran=0,
+                                  centering=0, want_tie=False)
+        assert np.array_equal(a["codes"][:, 4 * j:4 * j + 4], ref["codes"])
+        assert np.allclose(a["gscale"][:, j], ref["scale"], rtol=1e-15, atol=0)
+
+
+def test_low_rank_factors_are_the_best_rank_r_approximation():
+    """L2 L1 from the decomposition equals the truncated SVD of W diag(sigma)
+    (Eckart-Young: the residual's Frobenius norm is the root of the sum of
+    the dropped squared singular values)."""
+    gen = np.random.default_rng(3)
+    W = synth.f32_to_bf16_bits(gen.standard_normal((48, 96)).astype(np.float32))
+    sig = np.exp(gen.standard_normal(96) * 0.3)
+    L1, L2 = oracle.low_rank_factors(W, sig, 8)
+    What = oracle.bf16_to_f64(W) * sig[None, :]
+    s = np.linalg.svd(What, compute_uv=False)
+    assert np.isclose(np.linalg.norm(What - L2 @ L1), np.sqrt(np.sum(s[8:] ** 2)), rtol=1e-10)
+    assert np.allclose(L1 @ L1.T, np.eye(8), atol=1e-12)  # orthonormal rows
