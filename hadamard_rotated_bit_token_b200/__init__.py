@@ -12,7 +12,15 @@ missing or the device is not sm_100, the calls raise.
     hq_linear(desc, a_codes, a_scale, a_mean, w_codes, w_scale, colsum, bias_f32, Y, acc_debug)
     hq_check_device_error()
 
-`HadamardQuantLinear` bundles the caller-side buffers of one layer.
+The group-wise 4-bit form with a 16-bit low-rank branch (include/hq_gw.h):
+
+    hq_gw_sigma_inv(desc, W, act_absmax, alpha, sigma_inv)
+    hq_gw_prepare_weights(desc, W, bias, sigma_inv, L1, L2, w_codes, w_scale, l1s, l2b, bias_f32)
+    hq_gw_quantize_act(desc, X, sigma_inv, l1s, a_codes, a_scale, u)
+    hq_gw_linear(desc, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32, Y)
+
+`HadamardQuantLinear` and `GroupWiseQuantLinear` bundle the caller-side
+buffers of one layer of each form.
 """
 from __future__ import annotations
 
@@ -31,7 +39,9 @@ __all__ = [
     "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
     "hq_debug_set_gemm_variant", "HQ_GEMM_AUTO", "HQ_GEMM_SINGLE_CTA", "HQ_GEMM_CTA_PAIR",
     "hq_quantize_act_noalloc", "hq_debug_plan", "hq_debug_mma_ceiling", "hq_debug_tmap_cache",
-    "HadamardQuantLinear",
+    "HadamardQuantLinear", "GwDesc", "hq_gw_scale_ld", "hq_gw_sigma_inv", "hq_gw_prepare_weights",
+    "hq_gw_quantize_act", "hq_gw_linear", "hq_gw_debug_linear_f32", "GroupWiseQuantLinear",
+    "hq_debug_last_cuda_error",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -49,7 +59,9 @@ EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare
             "hq_quantize_act_workspace_bytes", "hq_quantize_act", "hq_linear", "hq_forward_host",
             "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
             "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan",
-            "hq_debug_mma_ceiling", "hq_debug_tmap_cache")
+            "hq_debug_mma_ceiling", "hq_debug_tmap_cache", "hq_gw_scale_ld", "hq_gw_sigma_inv",
+            "hq_gw_prepare_weights", "hq_gw_quantize_act", "hq_gw_linear",
+            "hq_gw_debug_linear_f32", "hq_debug_last_cuda_error")
 
 
 class HQError(RuntimeError):
@@ -71,6 +83,15 @@ class LayerDesc(ctypes.Structure):
         centering HQ_CENTER_NONE): W rotated along N in blocks of out_order."""
         super().__init__(K, N, had_order, a_bits, w_bits, act_gran, centering, code_format,
                          out_order)
+
+
+class GwDesc(ctypes.Structure):
+    """hq_gw_desc (host memory): the group-wise form's layer description."""
+    _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("rank", ctypes.c_int32), ("a_bits", ctypes.c_int32), ("w_bits", ctypes.c_int32)]
+
+    def __init__(self, K, N, group=64, rank=32, a_bits=4, w_bits=4):
+        super().__init__(K, N, group, rank, a_bits, w_bits)
 
 
 _lib = None
@@ -121,6 +142,22 @@ def load_library():
         lib.hq_debug_mma_ceiling.argtypes = [ctypes.c_int, ctypes.c_int64, _i32p, _vp]
         _u64p = ctypes.POINTER(ctypes.c_uint64)
         lib.hq_debug_tmap_cache.argtypes = [_u64p, _u64p]
+        lib.hq_debug_last_cuda_error.argtypes = []
+        lib.hq_debug_last_cuda_error.restype = ctypes.c_int
+        gw_p = ctypes.POINTER(GwDesc)
+        lib.hq_gw_scale_ld.argtypes = [ctypes.c_int64]
+        lib.hq_gw_scale_ld.restype = ctypes.c_int64
+        lib.hq_gw_sigma_inv.argtypes = [gw_p, _vp, _vp, ctypes.c_float, _vp, _vp]
+        lib.hq_gw_prepare_weights.argtypes = [gw_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                              _vp, _vp]
+        lib.hq_gw_quantize_act.argtypes = [gw_p, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
+                                           _vp]
+        lib.hq_gw_linear.argtypes = [gw_p, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp]
+        lib.hq_gw_debug_linear_f32.argtypes = list(lib.hq_gw_linear.argtypes)
+        for name in ("hq_gw_sigma_inv", "hq_gw_prepare_weights", "hq_gw_quantize_act",
+                     "hq_gw_linear", "hq_gw_debug_linear_f32"):
+            getattr(lib, name).restype = ctypes.c_int
         for name in ("hq_calib_act_absmax", "hq_prepare_weights", "hq_quantize_act", "hq_linear",
                      "hq_forward_host",
                      "hq_check_device_error", "hq_debug_set_wait_limit", "hq_debug_inject_fault",
@@ -175,6 +212,9 @@ def _stream(stream):
 
 def _check(status: int, where: str):
     if status != 0:
+        if status == 4:  # HQ_ERR_CUDA: name the code behind it
+            code = load_library().hq_debug_last_cuda_error()
+            raise HQError(status, f"{where} (CUDA code {code})")
         raise HQError(status, where)
 
 
@@ -299,6 +339,59 @@ def hq_debug_tmap_cache() -> dict:
 def hq_debug_set_gemm_variant(variant: int):
     """Selects the GEMM kernel of later hq_linear calls (HQ_GEMM_*)."""
     _check(load_library().hq_debug_set_gemm_variant(int(variant)), "hq_debug_set_gemm_variant")
+
+
+# ---------------------------------------------------------------------------
+# group-wise form (include/hq_gw.h), same names
+# ---------------------------------------------------------------------------
+
+def hq_debug_last_cuda_error() -> int:
+    """The code behind the last HQ_ERR_CUDA (cleared by reading)."""
+    return int(load_library().hq_debug_last_cuda_error())
+
+
+def hq_gw_scale_ld(T: int) -> int:
+    """Leading dimension of the [K/64][ld] activation scale array for T tokens."""
+    return int(load_library().hq_gw_scale_ld(int(T)))
+
+
+def hq_gw_sigma_inv(desc: GwDesc, W, act_absmax, alpha, sigma_inv, stream=None):
+    _check(load_library().hq_gw_sigma_inv(ctypes.byref(desc), _ptr(W), _ptr(act_absmax),
+                                          float(alpha), _ptr(sigma_inv), _stream(stream)),
+           "hq_gw_sigma_inv")
+
+
+def hq_gw_prepare_weights(desc: GwDesc, W, bias, sigma_inv, L1, L2, w_codes, w_scale, l1s, l2b,
+                          bias_f32, stream=None):
+    _check(load_library().hq_gw_prepare_weights(
+        ctypes.byref(desc), _ptr(W), _ptr(bias), _ptr(sigma_inv), _ptr(L1), _ptr(L2),
+        _ptr(w_codes), _ptr(w_scale), _ptr(l1s), _ptr(l2b), _ptr(bias_f32), _stream(stream)),
+        "hq_gw_prepare_weights")
+
+
+def hq_gw_quantize_act(desc: GwDesc, X, sigma_inv, l1s, a_codes, a_scale, u, T=None,
+                       stream=None):
+    T = X.shape[0] if T is None else T
+    _check(load_library().hq_gw_quantize_act(
+        ctypes.byref(desc), _ptr(X), T, _ptr(sigma_inv), _ptr(l1s), _ptr(a_codes), _ptr(a_scale),
+        _ptr(u), _stream(stream)), "hq_gw_quantize_act")
+
+
+def hq_gw_linear(desc: GwDesc, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32, Y, T=None,
+                 stream=None):
+    T = a_codes.shape[0] if T is None else T
+    _check(load_library().hq_gw_linear(
+        ctypes.byref(desc), T, _ptr(a_codes), _ptr(a_scale), _ptr(u), _ptr(w_codes),
+        _ptr(w_scale), _ptr(l2b), _ptr(bias_f32), _ptr(Y), _stream(stream)), "hq_gw_linear")
+
+
+def hq_gw_debug_linear_f32(desc: GwDesc, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32,
+                           Y32, T=None, stream=None):
+    T = a_codes.shape[0] if T is None else T
+    _check(load_library().hq_gw_debug_linear_f32(
+        ctypes.byref(desc), T, _ptr(a_codes), _ptr(a_scale), _ptr(u), _ptr(w_codes),
+        _ptr(w_scale), _ptr(l2b), _ptr(bias_f32), _ptr(Y32), _stream(stream)),
+        "hq_gw_debug_linear_f32")
 
 
 # ---------------------------------------------------------------------------
@@ -495,3 +588,82 @@ class HadamardQuantLinear:
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev) if ws else None
         self._bufs = {}
         return self
+
+
+class GroupWiseQuantLinear:
+    """Prepared weights and activation buffers of one group-wise layer
+    (include/hq_gw.h): 64-channel groups, each with its own H_64 block and
+    scale, and a rank-`rank` 16-bit branch.  `forward(X)` =
+    hq_gw_quantize_act + hq_gw_linear.
+
+    The low-rank factors are an input of the weight preparation: `factors` =
+    (L1 [rank,K], L2 [N,rank]) of W diag(sigma), or None to take them here
+    from a singular value decomposition of W diag(sigma) (torch.linalg.svd in
+    fp32 on the device, an offline step; the method fixes only L2 L1)."""
+
+    def __init__(self, desc: GwDesc, W, bias=None, act_absmax=None, alpha=0.5, factors=None):
+        import torch
+        self.desc = desc
+        dev = W.device
+        K, N, r = desc.K, desc.N, desc.rank
+        self.sigma_inv = torch.empty(K, dtype=torch.float32, device=dev)
+        hq_gw_sigma_inv(desc, W, act_absmax, alpha, self.sigma_inv)
+        self.use_sigma = act_absmax is not None
+        if r > 0:
+            if factors is None:
+                What = W.float() / self.sigma_inv[None, :]
+                U, S, Vh = torch.linalg.svd(What, full_matrices=False)
+                k = min(r, S.numel())  # beyond min(N, K) the factors are zero
+                L1 = torch.zeros((r, K), dtype=torch.float32, device=dev)
+                L2 = torch.zeros((N, r), dtype=torch.float32, device=dev)
+                L1[:k] = Vh[:k]
+                L2[:, :k] = U[:, :k] * S[:k]
+                factors = (L1, L2)
+            L1, L2 = (f.to(device=dev, dtype=torch.float32).contiguous() for f in factors)
+            if tuple(L1.shape) != (r, K) or tuple(L2.shape) != (N, r):
+                raise ValueError(f"factors must be L1 [{r},{K}] and L2 [{N},{r}], got "
+                                 f"{tuple(L1.shape)} and {tuple(L2.shape)}")
+            self.factors = (L1, L2)  # fp32, as given to the weight preparation
+            self.l1s = torch.empty((r, K), dtype=torch.bfloat16, device=dev)
+            self.l2b = torch.empty((N, r), dtype=torch.bfloat16, device=dev)
+        else:
+            L1 = L2 = None
+            self.factors = None
+            self.l1s = self.l2b = None
+        self.w_codes = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=dev)
+        self.w_scale = torch.empty((K // 64, N), dtype=torch.float32, device=dev)
+        self.bias_f32 = torch.empty(N, dtype=torch.float32, device=dev)
+        hq_gw_prepare_weights(desc, W, bias, self.sigma_inv if self.use_sigma else None, L1, L2,
+                              self.w_codes, self.w_scale, self.l1s, self.l2b, self.bias_f32)
+        self._bufs = {}
+
+    def buffers(self, T: int):
+        import torch
+        b = self._bufs.get(T)
+        if b is None:
+            dev = self.w_codes.device
+            K, r = self.desc.K, self.desc.rank
+            b = {"a_codes": torch.empty((T, K), dtype=torch.float8_e4m3fn, device=dev),
+                 "a_scale": torch.empty((K // 64, hq_gw_scale_ld(T)), dtype=torch.float32,
+                                        device=dev),
+                 "u": torch.empty((T, r), dtype=torch.bfloat16, device=dev) if r else None}
+            self._bufs[T] = b
+        return b
+
+    def quantize(self, X):
+        b = self.buffers(X.shape[0])
+        hq_gw_quantize_act(self.desc, X, self.sigma_inv if self.use_sigma else None, self.l1s,
+                           b["a_codes"], b["a_scale"], b["u"])
+        return b
+
+    def forward(self, X, Y=None):
+        import torch
+        if Y is None:
+            Y = torch.empty((X.shape[0], self.desc.N), dtype=torch.bfloat16, device=X.device)
+        b = self.quantize(X)
+        hq_gw_linear(self.desc, b["a_codes"], b["a_scale"], b["u"], self.w_codes, self.w_scale,
+                     self.l2b, self.bias_f32, Y, T=X.shape[0])
+        return Y
+
+    __call__ = forward
+

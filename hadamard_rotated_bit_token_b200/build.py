@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libhq.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 SOURCES = ["hq_api.cu", "hq_quant.cu", "hq_quant_act.cu", "hq_quant_act_spl2.cu",
-           "hq_quant_act_spl3.cu", "hq_quant_act_spl4.cu", "hq_quant_act_big.cu", "hq_gemm.cu"]
+           "hq_quant_act_spl3.cu", "hq_quant_act_spl4.cu", "hq_quant_act_big.cu", "hq_gemm.cu",
+           "hq_gw.cu"]
 HEADERS = ["hq_device.cuh", "hq_kernels.h", "hq_quant_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -34,6 +35,7 @@ def nvcc() -> str:
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
     files.append(os.path.join(ROOT, "include", "hq.h"))
+    files.append(os.path.join(ROOT, "include", "hq_gw.h"))
     return files
 
 

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/hq.h"
+#include "../../include/hq_gw.h"
 #include "hq_kernels.h"
 
 namespace hq {
@@ -19,7 +20,7 @@ __device__ unsigned int g_error_word = 0;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kVersion = 10300;  // 1.3.0: packed 3/4-bit activation codes
+constexpr int kVersion = 10400;  // 1.4.0: the group-wise form (include/hq_gw.h)
 constexpr int kMaxHostChunks = 64;  // row chunks of hq_forward_host
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -143,7 +144,22 @@ hq_status check_desc(const hq_layer_desc* d) {
   return HQ_OK;
 }
 
-hq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA; }
+// The last failure behind an HQ_ERR_CUDA (hq_debug_last_cuda_error): a
+// runtime error code, or 100000 + a driver result code from tensor-map
+// encoding.
+int g_last_cuda_error = 0;
+
+hq_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return HQ_OK;
+  g_last_cuda_error = int(e);
+  return HQ_ERR_CUDA;
+}
+
+hq_status from_cu(CUresult r) {
+  if (r == CUDA_SUCCESS) return HQ_OK;
+  g_last_cuda_error = 100000 + int(r);
+  return HQ_ERR_CUDA;
+}
 
 constexpr int kQuantCtasPerSm = 2;  // quantizer CTAs per SM (its launch bounds)
 #ifndef HQ_GROUP_M
@@ -422,7 +438,7 @@ hq_status encode_act_view_raw(CUtensorMap* m, const void* X, int64_t T, int K, i
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+  return from_cu(r);
 }
 
 struct QActLaunch {
@@ -541,7 +557,7 @@ hq_status encode_kmajor_i8_raw(CUtensorMap* m, const void* base, int64_t rows, i
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+  return from_cu(r);
 }
 
 // Packed activation codes [T, K/2] bytes: box {64 bytes (one K block of 128
@@ -555,7 +571,7 @@ hq_status encode_packed_a_raw(CUtensorMap* m, const void* base, int64_t rows, in
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+  return from_cu(r);
 }
 
 hq_status encode_out_bf16_raw(CUtensorMap* m, const void* base, int64_t rows, int N) {
@@ -567,7 +583,7 @@ hq_status encode_out_bf16_raw(CUtensorMap* m, const void* base, int64_t rows, in
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? HQ_OK : HQ_ERR_CUDA;
+  return from_cu(r);
 }
 
 hq_status encode_kmajor_i8(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
@@ -688,6 +704,135 @@ hq_status check_linear_args(const hq_layer_desc* desc, int64_t T, const int8_t* 
   return HQ_OK;
 }
 
+
+// ---------------------------------------------------------------------------
+// Group-wise form: tensor maps and shape rules.
+hq_status check_gw_desc(const hq_gw_desc* d) {
+  if (d == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  if (d->K <= 0 || d->N <= 0 || d->group <= 0 || d->rank < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if (d->group != 64 || d->K % 64 != 0 || d->K > 16384 || d->N % 16 != 0) return HQ_ERR_UNSUPPORTED;
+  if (d->rank != 0 && d->rank != 32) return HQ_ERR_UNSUPPORTED;
+  if (d->a_bits < 2 || d->a_bits > 4 || d->w_bits < 2 || d->w_bits > 4) return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+
+int64_t gw_ld(int64_t cols) { return (cols + 3) / 4 * 4; }
+
+// codes [rows, K] bytes, box {64, box_rows}, 64-byte swizzle
+hq_status encode_gw_codes(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+  return cached_tmap(TmapKey{10, base, rows, K, box_rows}, m, [&](CUtensorMap* o) {
+    cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(K)};
+    cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(o, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return from_cu(r);
+  });
+}
+
+// bf16 [rows, K], box {64, box_rows}, 128-byte swizzle (X tiles, l1 tiles)
+hq_status encode_gw_bf16_k64(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+  return cached_tmap(TmapKey{11, base, rows, K, box_rows}, m, [&](CUtensorMap* o) {
+    cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(K) * 2u};
+    cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return from_cu(r);
+  });
+}
+
+// fp32 [G][gw_ld(cols)] (cols valid per row), box {box, 1}, no swizzle
+hq_status encode_gw_scales(CUtensorMap* m, const void* base, int G, int64_t cols, int box) {
+  return cached_tmap(TmapKey{12, base, G, cols, box}, m, [&](CUtensorMap* o) {
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(G)};
+    cuuint64_t strides[1] = {cuuint64_t(gw_ld(cols)) * 4u};
+    cuuint32_t box2[2] = {cuuint32_t(box), 1u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims,
+                          strides, box2, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return from_cu(r);
+  });
+}
+
+// bf16 [rows, rank] (rank 32: 64-byte rows), box {rank, box_rows}, 64-byte swizzle
+hq_status encode_gw_rank(CUtensorMap* m, const void* base, int64_t rows, int rank, int box_rows) {
+  return cached_tmap(TmapKey{13, base, rows, rank, box_rows}, m, [&](CUtensorMap* o) {
+    cuuint64_t dims[2] = {cuuint64_t(rank), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(rank) * 2u};
+    cuuint32_t box[2] = {cuuint32_t(rank), cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return from_cu(r);
+  });
+}
+
+hq_status gw_linear_impl(const hq_gw_desc* d, int64_t T, const uint8_t* a_codes,
+                         const float* a_scale, const uint16_t* u, const uint8_t* w_codes,
+                         const float* w_scale, const uint16_t* l2b, const float* bias_f32,
+                         uint16_t* Y, float* Y32, hq_stream_t stream) {
+  hq_status s = check_gw_desc(d);
+  if (s != HQ_OK) return s;
+  if (T < 0) return HQ_ERR_INVALID_ARGUMENT;
+  if ((Y == nullptr && Y32 == nullptr) || a_codes == nullptr || a_scale == nullptr ||
+      w_codes == nullptr || w_scale == nullptr || (d->rank > 0 && (u == nullptr || l2b == nullptr)))
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(a_codes) || !aligned16(a_scale) || !aligned16(w_codes) || !aligned16(w_scale) ||
+      (bias_f32 && !aligned16(bias_f32)) || (Y && !aligned16(Y)) || (Y32 && !aligned16(Y32)) ||
+      (d->rank > 0 && (!aligned16(u) || !aligned16(l2b))))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceState* dev;
+  s = device_state(&dev);
+  if (s != HQ_OK) return s;
+  const int K = d->K, N = d->N, G = K / 64;
+  CUtensorMap maps[7];
+  if ((s = encode_gw_codes(&maps[0], a_codes, T, K, 128)) != HQ_OK) return s;
+  if ((s = encode_gw_codes(&maps[1], w_codes, N, K, 256)) != HQ_OK) return s;
+  if ((s = encode_gw_scales(&maps[2], a_scale, G, T, 128)) != HQ_OK) return s;
+  if ((s = encode_gw_scales(&maps[3], w_scale, G, N, 256)) != HQ_OK) return s;
+  if (d->rank > 0) {
+    if ((s = encode_gw_rank(&maps[4], u, T, d->rank, 128)) != HQ_OK) return s;
+    if ((s = encode_gw_rank(&maps[5], l2b, N, d->rank, 256)) != HQ_OK) return s;
+  } else {
+    maps[4] = maps[0];  // not read without the branch
+    maps[5] = maps[0];
+  }
+  if (Y) {
+    if ((s = encode_out_bf16(&maps[6], Y, T, N)) != HQ_OK) return s;
+  } else {
+    maps[6] = maps[0];  // not written: the fp32 sums go to Y32
+  }
+  GwGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.bias = bias_f32;
+  p.out_f32 = Y32;
+  p.T = T;
+  p.N = N;
+  p.K = K;
+  p.G = G;
+  p.rank = d->rank;
+  p.num_m_tiles = int((T + 127) / 128);
+  p.num_n_tiles = (N + 255) / 256;
+  p.group_m = 8;
+  p.err = dev->err;
+  p.wait_ns = wait_ns();
+  const int64_t tiles = int64_t(p.num_m_tiles) * p.num_n_tiles;
+  if (tiles >= (int64_t(1) << 31)) return HQ_ERR_UNSUPPORTED;
+  const int grid = int(tiles < dev->sm_count ? tiles : dev->sm_count);
+  return from_cuda(launch_gw_gemm(maps, p, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
 }  // namespace
 }  // namespace hq
 
@@ -1191,3 +1336,145 @@ extern "C" hq_status hq_quantize_act_noalloc(const hq_layer_desc* desc, const ui
   return hq_quantize_act(desc, X, T, sigma_inv, a_codes, a_scale, a_mean, ws,
                          ws ? kNoAllocScratchBytes : 0, stream);
 }
+
+// ---------------------------------------------------------------------------
+// Group-wise form (include/hq_gw.h).
+using namespace hq;
+
+extern "C" {
+
+int64_t hq_gw_scale_ld(int64_t T) { return T < 0 ? 0 : gw_ld(T); }
+
+int hq_debug_last_cuda_error(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  const int e = g_last_cuda_error;
+  g_last_cuda_error = 0;
+  return e;
+}
+
+hq_status hq_gw_sigma_inv(const hq_gw_desc* desc, const uint16_t* W, const float* act_absmax,
+                          float alpha, float* sigma_inv, hq_stream_t stream) {
+  hq_status s = check_gw_desc(desc);
+  if (s != HQ_OK) return s;
+  if (W == nullptr || sigma_inv == nullptr || !(alpha >= 0.0f && alpha <= 1.0f))
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(W) || !aligned16(sigma_inv) || (act_absmax && !aligned16(act_absmax)))
+    return HQ_ERR_MISALIGNED;
+  DeviceState* dev;
+  if ((s = device_state(&dev)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (act_absmax == nullptr) return from_cuda(launch_fill(sigma_inv, desc->K, 1.0f, st));
+  // sigma_inv first holds max_n |W[n,k]| (the column maxima accumulate into it)
+  s = from_cuda(cudaMemsetAsync(sigma_inv, 0, sizeof(float) * size_t(desc->K), st));
+  if (s != HQ_OK) return s;
+  s = from_cuda(launch_col_absmax(W, desc->N, desc->K, sigma_inv, st));
+  if (s != HQ_OK) return s;
+  return from_cuda(launch_sigma_inv(act_absmax, sigma_inv, desc->K, alpha, st));
+}
+
+hq_status hq_gw_prepare_weights(const hq_gw_desc* desc, const uint16_t* W, const uint16_t* bias,
+                                const float* sigma_inv, const float* L1, const float* L2,
+                                uint8_t* w_codes, float* w_scale, uint16_t* l1s, uint16_t* l2b,
+                                float* bias_f32, hq_stream_t stream) {
+  hq_status s = check_gw_desc(desc);
+  if (s != HQ_OK) return s;
+  const int rank = desc->rank;
+  if (W == nullptr || w_codes == nullptr || w_scale == nullptr || bias_f32 == nullptr ||
+      (rank > 0 && (L1 == nullptr || L2 == nullptr || l1s == nullptr || l2b == nullptr)))
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(W) || !aligned16(w_codes) || !aligned16(w_scale) || !aligned16(bias_f32) ||
+      (sigma_inv && !aligned16(sigma_inv)) || (bias && !aligned4(bias)) ||
+      (rank > 0 && (!aligned16(L1) || !aligned16(L2) || !aligned16(l1s) || !aligned16(l2b))))
+    return HQ_ERR_MISALIGNED;
+  DeviceState* dev;
+  if ((s = device_state(&dev)) != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (rank > 0) {
+    s = from_cuda(launch_gw_factors(L1, L2, sigma_inv, rank, desc->K, desc->N, l1s, l2b,
+                                    dev->sm_count, st));
+    if (s != HQ_OK) return s;
+  }
+  GwWeightParams p;
+  p.W = W;
+  p.bias = bias;
+  p.sigma_inv = sigma_inv;
+  p.l1s = rank > 0 ? l1s : nullptr;
+  p.l2b = rank > 0 ? l2b : nullptr;
+  p.w_codes = w_codes;
+  p.w_scale = w_scale;
+  p.bias_f32 = bias_f32;
+  p.K = desc->K;
+  p.N = desc->N;
+  p.rank = rank;
+  p.q = (1 << (desc->w_bits - 1)) - 1;
+  return from_cuda(launch_gw_weights(p, st));
+}
+
+hq_status hq_gw_quantize_act(const hq_gw_desc* desc, const uint16_t* X, int64_t T,
+                             const float* sigma_inv, const uint16_t* l1s, uint8_t* a_codes,
+                             float* a_scale, uint16_t* u, hq_stream_t stream) {
+  hq_status s = check_gw_desc(desc);
+  if (s != HQ_OK) return s;
+  const int rank = desc->rank;
+  if (T < 0 || X == nullptr || a_codes == nullptr || a_scale == nullptr ||
+      (rank > 0 && (l1s == nullptr || u == nullptr)))
+    return HQ_ERR_INVALID_ARGUMENT;
+  if (!aligned16(X) || !aligned16(a_codes) || !aligned16(a_scale) ||
+      (sigma_inv && !aligned16(sigma_inv)) || (rank > 0 && (!aligned16(l1s) || !aligned16(u))))
+    return HQ_ERR_MISALIGNED;
+  if (T == 0) return HQ_OK;
+  DeviceState* dev;
+  if ((s = device_state(&dev)) != HQ_OK) return s;
+  const int K = desc->K;
+  CUtensorMap tx, tl;
+  if ((s = encode_gw_bf16_k64(&tx, X, T, K, 128)) != HQ_OK) return s;
+  if (rank > 0) {
+    if ((s = encode_gw_bf16_k64(&tl, l1s, rank, K, rank)) != HQ_OK) return s;
+  } else {
+    tl = tx;  // not read without the branch
+  }
+  GwActParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.sigma_inv = sigma_inv;
+  p.codes = a_codes;
+  p.scale = a_scale;
+  p.u = rank > 0 ? u : nullptr;
+  p.T = T;
+  p.K = K;
+  p.ld = int(gw_ld(T));
+  p.rank = rank;
+  p.q = (1 << (desc->a_bits - 1)) - 1;
+  p.fault = g_fault == HQ_FAULT_QUANT_WITHHOLD_ROW ? 1 : 0;
+  p.err = dev->err;
+  p.wait_ns = wait_ns();
+  if (gw_ld(T) >= (int64_t(1) << 31)) return HQ_ERR_UNSUPPORTED;
+  // as many stages (up to 8) as fit beside sigma^-1
+  int stages = 8;
+  while (stages > 2 && gw_act_smem_bytes(K, rank, stages, sigma_inv != nullptr) > 227u * 1024u)
+    --stages;
+  p.stages = stages;
+  const int64_t grid = (T + 127) / 128;
+  if (grid >= (int64_t(1) << 31)) return HQ_ERR_UNSUPPORTED;
+  return from_cuda(
+      launch_gw_act(&tx, &tl, p, int(grid), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hq_status hq_gw_linear(const hq_gw_desc* desc, int64_t T, const uint8_t* a_codes,
+                       const float* a_scale, const uint16_t* u, const uint8_t* w_codes,
+                       const float* w_scale, const uint16_t* l2b, const float* bias_f32,
+                       uint16_t* Y, hq_stream_t stream) {
+  if (Y == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  return gw_linear_impl(desc, T, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32, Y, nullptr,
+                        stream);
+}
+
+hq_status hq_gw_debug_linear_f32(const hq_gw_desc* desc, int64_t T, const uint8_t* a_codes,
+                                 const float* a_scale, const uint16_t* u, const uint8_t* w_codes,
+                                 const float* w_scale, const uint16_t* l2b, const float* bias_f32,
+                                 float* Y32, hq_stream_t stream) {
+  if (Y32 == nullptr) return HQ_ERR_INVALID_ARGUMENT;
+  return gw_linear_impl(desc, T, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32, nullptr,
+                        Y32, stream);
+}
+
+}  // extern "C"

@@ -140,4 +140,60 @@ cudaError_t launch_bf16_to_f32(const uint16_t* in, float* out, int n, cudaStream
 cudaError_t launch_wh_weights(const uint16_t* W, const float* sigma_inv, int K, int N, int m,
                               int q, int8_t* codes, float* w_scale, cudaStream_t st);
 
+// ---------------------------------------------------------------------------
+// Group-wise form (64-channel groups, fp8 e4m3 bytes holding integer codes,
+// rank-32 16-bit low-rank branch): hq_gw.cu.
+struct GwWeightParams {
+  const uint16_t* W;        // [N,K] bf16
+  const uint16_t* bias;     // [N] bf16 or null
+  const float* sigma_inv;   // [K] or null
+  const uint16_t* l1s;      // [rank,K] bf16 (already rounded)
+  const uint16_t* l2b;      // [N,rank] bf16
+  uint8_t* w_codes;         // [N,K] e4m3
+  float* w_scale;           // [K/64][N]
+  float* bias_f32;          // [N]
+  int K, N, rank, q;
+};
+
+struct GwActParams {
+  const float* sigma_inv;   // [K] or null
+  uint8_t* codes;           // [T,K] e4m3
+  float* scale;             // [K/64][ld]
+  uint16_t* u;              // [T,rank] bf16 (rank > 0)
+  int64_t T;
+  int K, ld, rank, q, stages;
+  int fault;                // withhold the first tile's copy (timeout path)
+  unsigned int* err;
+  unsigned long long wait_ns;
+};
+
+struct GwGemmParams {
+  const float* bias;        // [N] or null
+  float* out_f32;           // [T,N] fp32 instead of the bf16 store, or null
+  int64_t T;
+  int N, K, G, rank;
+  int num_m_tiles, num_n_tiles, group_m;
+  unsigned int* err;
+  unsigned long long wait_ns;
+};
+
+// l1s = bf16(L1 diag(sigma_inv)) [rank,K], l2b = bf16(L2) [N,rank].
+cudaError_t launch_gw_factors(const float* L1, const float* L2, const float* sigma_inv, int rank,
+                              int K, int N, uint16_t* l1s, uint16_t* l2b, int sms, cudaStream_t st);
+// R = (W - l2 l1) sigma, R H_64 per group, codes and scales; one CTA per row.
+cudaError_t launch_gw_weights(const GwWeightParams& p, cudaStream_t st);
+// One CTA per 128 tokens.  tmap_x: X [T,K] bf16, box {64, 128}, 128-byte
+// swizzle; tmap_l1: l1s [rank,K] bf16, box {64, rank}, 128-byte swizzle.
+cudaError_t launch_gw_act(const void* tmap_x, const void* tmap_l1, const GwActParams& p, int grid,
+                          cudaStream_t st);
+size_t gw_act_smem_bytes(int K, int rank, int stages, bool sigma);
+int gw_act_threads();
+// tmaps: 7 CUtensorMap in order A codes [T,K] u8 box {64,128} and B codes
+// [N,K] u8 box {64,256} (64-byte swizzle); s_x [G][ld] f32 box {128,1}; s_w
+// [G][N] f32 box {256,1}; u [T,32] bf16 box {32,128} and l2 [N,32] bf16
+// box {32,256} (64-byte swizzle); Y [T,N] bf16 box {32,32} (64-byte swizzle).
+cudaError_t launch_gw_gemm(const void* tmaps, const GwGemmParams& p, int grid, cudaStream_t st);
+size_t gw_gemm_smem_bytes();
+int gw_gemm_threads();
+
 }  // namespace hq

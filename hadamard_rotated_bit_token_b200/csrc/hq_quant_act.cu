@@ -109,7 +109,7 @@ __device__ __forceinline__ void act_setup(const QuantParams& p, uint8_t* smem, c
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], uint32_t(ncw));
+      mbar_init(&empty[s], uint32_t(ncw) * 32u);  // every consumer thread
     }
     flags[0] = 0;
     flags[1] = 0;
@@ -326,9 +326,12 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
         if (NSL > 1) pin32(w[j]);
       }
       // every lane has the tile's slices in registers before the stage goes
-      // back; the mean's terms are in shared memory
+      // back; each thread releases its own loads, which went through the
+      // generic proxy, so a proxy fence orders them before the producer's
+      // next tensor copy into the stage; the mean's terms are in shared memory
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      fence_proxy_async_smem();
+      mbar_arrive(&empty[s]);
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
@@ -476,8 +479,10 @@ __global__ void __launch_bounds__(BIG ? kSegThreadsBig : kSegThreads, BIG ? 1 : 
       if (active) load_slice(smem_u32(smem) + uint32_t(s) * L.stage_bytes, c, x);
       f2 w[16];
       unpack32(x, w);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      // each thread releases its own loads (generic proxy), ordered before
+      // the producer's next tensor copy into the stage by a proxy fence
+      fence_proxy_async_smem();
+      mbar_arrive(&empty[s]);
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;

@@ -39,9 +39,10 @@
  *     launches nothing.
  *
  * Shapes supported:  had_order a power of two in [16, 1024], or 1 (no
- * rotation along K); K a multiple of had_order and of 64, K <= 9216; N a
- * multiple of 16 (and of out_order in the weight-only form, out_order in
- * {16, 32, 64}); T >= 0 (T = 0 is a no-op); a_bits in {3, 4, 8}, w_bits in
+ * rotation along K); K a multiple of had_order and of 16, K <= 15360 with a
+ * rotation and K <= 10240 without one (K a multiple of 32 for packed
+ * codes); N a multiple of 16 (and of out_order in the weight-only form,
+ * out_order in {16, 32, 64}); T >= 0 (T = 0 is a no-op); a_bits in {3, 4, 8}, w_bits in
  * {4, 8} (codes in an int8 container, one code per byte; 3- and 4-bit
  * activation codes optionally two per byte, hq_layer_desc.code_format).
  */
@@ -327,6 +328,11 @@ hq_status hq_debug_plan(const hq_layer_desc* desc, int64_t T, int sms, int pair_
  * and shapes (no per-call encoding on the host).  Outputs are host pointers
  * and may be NULL; counts are cumulative for the process. */
 hq_status hq_debug_tmap_cache(uint64_t* hits, uint64_t* misses);
+
+/* Diagnostic hook, host only: the code behind the last HQ_ERR_CUDA any call
+ * returned (a cudaError_t value, or 100000 + a CUresult from encoding a
+ * tensor map), 0 if none; reading it clears it. */
+int hq_debug_last_cuda_error(void);
 
 /* Measurement hook (no counterpart on the pages): the int8 tensor-core
  * ceiling of this device, the denominator the GEMM's throughput is reported

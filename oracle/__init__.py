@@ -430,18 +430,30 @@ def layer_wh(X_bits, W_bits, bias_bits, n_out, a_bits, w_bits, gran=0, alpha=0.5
 # diffusion transformers", "Hadamard rotation: the int4 improvement")
 # ---------------------------------------------------------------------------
 
+def _shape(name, a, shape):
+    """The C side reads exactly `shape`; anything else is refused here."""
+    if a is not None and tuple(np.shape(a)) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(np.shape(a))}")
+
+
 def low_rank_factors(W_bits, sigma, rank):
     """Rank-r factors of W^ = W diag(sigma) ([N,K]) from its singular value
-    decomposition: L2 = U_r diag(S_r) [N,r], L1 = V_r^T [r,K] (fp64).  A
-    library routine serves as this step (the method fixes only L2 L1, the
-    best rank-r approximation)."""
+    decomposition: L2 = U_r diag(S_r) [N,r], L1 = V_r^T [r,K] (fp64), zero
+    past min(N, K) components.  A library routine serves as this step (the
+    method fixes only L2 L1, the best rank-r approximation)."""
     W = bf16_to_f64(_c(W_bits, np.uint16))
     if sigma is not None:
         W = W * np.asarray(sigma, dtype=np.float64)[None, :]
+    N, K = W.shape
+    L1 = np.zeros((rank, K))
+    L2 = np.zeros((N, rank))
     if rank == 0:
-        return np.zeros((0, W.shape[1])), np.zeros((W.shape[0], 0))
+        return L1, L2
     U, S, Vt = np.linalg.svd(W, full_matrices=False)
-    return np.ascontiguousarray(Vt[:rank]), np.ascontiguousarray(U[:, :rank] * S[:rank])
+    k = min(rank, S.size)  # past min(N, K) the factors are zero
+    L1[:k] = Vt[:k]
+    L2[:, :k] = U[:, :k] * S[:k]
+    return L1, L2
 
 
 def gw_prepare_weights(W_bits, g, bits, rank, L1, L2, bias_bits=None, sigma=None,
@@ -452,6 +464,11 @@ def gw_prepare_weights(W_bits, g, bits, rank, L1, L2, bias_bits=None, sigma=None
     N, K = W.shape
     b = _c(bias_bits, np.uint16)
     sig = _c(sigma, np.float64)
+    _shape("sigma", sig, (K,))
+    _shape("bias", b, (N,))
+    if rank:
+        _shape("L1", L1, (rank, K))
+        _shape("L2", L2, (N, rank))
     l1 = np.zeros((rank, K), dtype=np.uint16)
     l2 = np.zeros((N, rank), dtype=np.uint16)
     codes = np.zeros((N, K), dtype=np.int8)
@@ -479,6 +496,9 @@ def gw_quantize_act(X_bits, g, bits, rank, l1_bits, sigma=None, rows=None, want_
     T, K = X.shape
     sig = _c(sigma, np.float64)
     l1 = _c(l1_bits, np.uint16) if rank else None
+    _shape("sigma", sig, (K,))
+    if rank:
+        _shape("l1", l1, (rank, K))
     r = None if rows is None else _c(rows, np.int64)
     nr = T if r is None else r.size
     codes = np.zeros((nr, K), dtype=np.int8)

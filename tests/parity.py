@@ -37,7 +37,12 @@ def check_codes(gpu, ref, tie, what="codes", min_match=None):
     bad = diff != 0
     nbad = int(bad.sum())
     if nbad:
-        assert np.all(np.abs(diff[bad]) == 1), f"{what}: a code differs by more than 1"
+        far = np.argwhere(np.abs(diff) > 1)
+        if far.size:
+            show = [(tuple(int(v) for v in ix), int(gpu[tuple(ix)]), int(ref[tuple(ix)]),
+                     float(tie[tuple(ix)])) for ix in far[:8]]
+            raise AssertionError(f"{what}: {len(far)} codes differ by more than 1 "
+                                 f"(index, gpu, oracle, tie): {show}")
         worst = float(np.max(tie[bad]))
         assert worst < TIE_TOL, f"{what}: mismatch {worst:.3g} code units away from a tie"
     match = 1.0 - nbad / max(1, gpu.size)

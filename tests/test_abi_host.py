@@ -2,6 +2,7 @@
 exports every entry point include/hq.h declares, and rejects bad arguments
 with the documented status codes before touching the device."""
 import ctypes
+import glob
 import os
 import re
 
@@ -20,14 +21,17 @@ def hq():
 
 
 def declared_functions():
-    text = open(os.path.join(ROOT, "include", "hq.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(hq_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for hdr in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))):
+        text = re.sub(r"/\*.*?\*/", "", open(hdr).read(), flags=re.S)
+        names |= set(re.findall(r"\b(hq_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_every_declared_symbol_is_exported(hq):
     names = declared_functions()
     assert "hq_quantize_act" in names and "hq_linear" in names and "hq_prepare_weights" in names
+    assert "hq_gw_quantize_act" in names and "hq_gw_linear" in names
     lib = hq.load_library()
     for name in names:
         assert hasattr(lib, name), name
@@ -35,7 +39,7 @@ def test_every_declared_symbol_is_exported(hq):
 
 
 def test_version_and_status_strings(hq):
-    assert hq.hq_version() == 10300
+    assert hq.hq_version() == 10400
     for code, name in hq.STATUS_NAMES.items():
         assert hq.hq_status_string(code) == name
     assert hq.hq_status_string(99) == "HQ_ERR_UNKNOWN"
@@ -239,3 +243,51 @@ def test_library_has_no_cpu_fallback():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "hq_oracle" not in text and "liboracle" not in text, f
+
+
+def test_gw_desc_layout_matches_the_header(hq):
+    """The binding's GwDesc has hq_gw_desc's fields, in order, all int32."""
+    text = open(os.path.join(ROOT, "include", "hq_gw.h")).read()
+    body = re.search(r"typedef struct hq_gw_desc \{(.*?)\} hq_gw_desc;", text, re.S).group(1)
+    names = [re.match(r"\s*int32_t (\w+);", line).group(1)
+             for line in body.strip().splitlines()]
+    assert [f[0] for f in hq.GwDesc._fields_] == names
+    assert all(f[1] is ctypes.c_int32 for f in hq.GwDesc._fields_)
+
+
+def _gw_quant(hq, desc, X=FAKE, T=4, codes=FAKE, scale=FAKE, l1s=FAKE, u=FAKE):
+    lib = hq.load_library()
+    d = None if desc is None else ctypes.byref(desc)
+    return lib.hq_gw_quantize_act(d, X, T, None, l1s, codes, scale, u, None)
+
+
+def _gw_linear(hq, desc, T=4, a=FAKE, sa=FAKE, u=FAKE, w=FAKE, sw=FAKE, l2=FAKE, Y=FAKE):
+    lib = hq.load_library()
+    return lib.hq_gw_linear(ctypes.byref(desc), T, a, sa, u, w, sw, l2, None, Y, None)
+
+
+def test_gw_validation(hq):
+    """Every group-wise entry rejects bad descriptions, pointers and sizes
+    before touching the device (so these run without a GPU)."""
+    G = hq.GwDesc
+    assert _gw_quant(hq, None) == 1
+    assert _gw_quant(hq, G(1024, 16), X=None) == 1
+    assert _gw_quant(hq, G(1024, 16), T=-1) == 1
+    assert _gw_quant(hq, G(1024, 16), X=FAKE + 8) == 3          # misaligned
+    assert _gw_quant(hq, G(1024, 16, rank=32), u=None) == 1     # branch without u
+    assert _gw_quant(hq, G(1000, 16)) == 2                      # K not whole groups
+    assert _gw_quant(hq, G(16384 + 64, 16)) == 2                # K above 16384
+    assert _gw_quant(hq, G(1024, 16, group=128)) == 2           # group other than 64
+    assert _gw_quant(hq, G(1024, 16, rank=16)) == 2             # rank other than 0 / 32
+    assert _gw_quant(hq, G(1024, 16, a_bits=8)) == 2            # codes beyond e4m3's integers
+    assert _gw_quant(hq, G(1024, 16, a_bits=1)) == 2
+    assert _gw_quant(hq, G(1024, 16), T=0) == 0                 # no-op
+    assert _gw_linear(hq, G(1024, 24)) == 2                     # N not a multiple of 16
+    assert _gw_linear(hq, G(1024, 16), Y=None) == 1
+    assert _gw_linear(hq, G(1024, 16), sw=FAKE + 4) == 3
+    assert _gw_linear(hq, G(1024, 16, rank=0), u=None, l2=None, T=0) == 0
+    lib = hq.load_library()
+    assert lib.hq_gw_prepare_weights(ctypes.byref(G(1024, 16)), FAKE, None, None, None, None,
+                                     FAKE, FAKE, None, None, FAKE, None) == 1  # rank 32, no factors
+    assert lib.hq_gw_sigma_inv(ctypes.byref(G(1024, 16)), FAKE, None, 1.5, FAKE, None) == 1
+    assert hq.hq_gw_scale_ld(0) == 0 and hq.hq_gw_scale_ld(5) == 8 and hq.hq_gw_scale_ld(8) == 8
