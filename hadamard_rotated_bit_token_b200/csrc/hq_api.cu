@@ -799,12 +799,13 @@ hq_status gw_linear_impl(const hq_gw_desc* d, int64_t T, const uint8_t* a_codes,
   const int K = d->K, N = d->N, G = K / 64;
   CUtensorMap maps[7];
   if ((s = encode_gw_codes(&maps[0], a_codes, T, K, 128)) != HQ_OK) return s;
-  if ((s = encode_gw_codes(&maps[1], w_codes, N, K, 256)) != HQ_OK) return s;
+  const int bn = gw_gemm_bn();
+  if ((s = encode_gw_codes(&maps[1], w_codes, N, K, bn)) != HQ_OK) return s;
   if ((s = encode_gw_scales(&maps[2], a_scale, G, T, 128)) != HQ_OK) return s;
-  if ((s = encode_gw_scales(&maps[3], w_scale, G, N, 256)) != HQ_OK) return s;
+  if ((s = encode_gw_scales(&maps[3], w_scale, G, N, bn)) != HQ_OK) return s;
   if (d->rank > 0) {
     if ((s = encode_gw_rank(&maps[4], u, T, d->rank, 128)) != HQ_OK) return s;
-    if ((s = encode_gw_rank(&maps[5], l2b, N, d->rank, 256)) != HQ_OK) return s;
+    if ((s = encode_gw_rank(&maps[5], l2b, N, d->rank, bn)) != HQ_OK) return s;
   } else {
     maps[4] = maps[0];  // not read without the branch
     maps[5] = maps[0];
@@ -823,8 +824,9 @@ hq_status gw_linear_impl(const hq_gw_desc* d, int64_t T, const uint8_t* a_codes,
   p.K = K;
   p.G = G;
   p.rank = d->rank;
+  if (gw_ld(T) >= (int64_t(1) << 31)) return HQ_ERR_UNSUPPORTED;
   p.num_m_tiles = int((T + 127) / 128);
-  p.num_n_tiles = (N + 255) / 256;
+  p.num_n_tiles = (N + bn - 1) / bn;
   p.group_m = 8;
   p.err = dev->err;
   p.wait_ns = wait_ns();

@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kEpiWarps);  // one arrival per epilogue warp
       mbar_init(&pfull[a], 1);
-      mbar_init(&pempty[a], kEpiWarps * 32);  // every epilogue thread
+      mbar_init(&pempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -654,10 +654,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, PK>::THREADS, 1)
             if (lane == 0) mbar_arrive(&tempty[acc]);
           },
           [&] {
-            // each thread's parameter reads (generic proxy), ordered before the
-            // next bulk copy into the slot by a proxy fence
+            // the parameter reads (generic proxy), each thread's ordered
+            // before the next bulk copy into the slot by its proxy fence
             fence_proxy_async_smem();
-            mbar_arrive(&pempty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[acc]);
           });
     }
     if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
@@ -800,7 +801,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 2 * kEpiWarps);
       mbar_init(&pfull[a], 1);
-      mbar_init(&pempty[a], kEpiWarps * 32);  // every epilogue thread
+      mbar_init(&pempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -964,10 +965,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (lane == 0) mbar_arrive_remote(tempty0 + uint32_t(acc) * 8u);
           },
           [&] {
-            // each thread's parameter reads (generic proxy), ordered before the
-            // next bulk copy into the slot by a proxy fence
+            // the parameter reads (generic proxy), each thread's ordered
+            // before the next bulk copy into the slot by its proxy fence
             fence_proxy_async_smem();
-            mbar_arrive(&pempty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[acc]);
           });
     }
     if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete

@@ -58,18 +58,43 @@ constexpr int kTokRows = 128;      // tokens per activation tile (MMA M)
 constexpr int kXTileBytes = kTokRows * kGroup * 2;  // bf16, one 128-byte row per token
 constexpr int kGwQuantWarps = 8;   // two teams of four (one warp per 32-token quarter)
 constexpr int kGwActThreads = 64 + 32 * kGwQuantWarps;
-constexpr int kGwBN = 256;         // output tile width of the GEMM
-constexpr int kGwEpiWarps = 16;    // four per 32-lane quarter of tensor memory
+// GEMM shape: output tile width, epilogue warps (a multiple of 4: each
+// 32-lane quarter of tensor memory gets kGwEpiWarps / 4 of them), columns
+// per tensor-memory load, and the register cap that lets the CTA launch
+// (the busiest sub-partition runs ceil(warps / 4) warps out of 16384
+// registers).
+#ifndef HQ_GW_BN
+#define HQ_GW_BN 256
+#endif
+#ifndef HQ_GW_EPI_WARPS
+#define HQ_GW_EPI_WARPS 16
+#endif
+#ifndef HQ_GW_LD_COLS
+#define HQ_GW_LD_COLS 8
+#endif
+#ifndef HQ_GW_MAXNREG
+#define HQ_GW_MAXNREG 96
+#endif
+constexpr int kGwBN = HQ_GW_BN;
+constexpr int kGwEpiWarps = HQ_GW_EPI_WARPS;
 constexpr int kGwEpiCols = kGwBN * 4 / kGwEpiWarps;  // output columns per epilogue warp
 constexpr int kGwEpiChunks = kGwEpiCols / 32;
+constexpr int kGwLdCols = HQ_GW_LD_COLS;
+static_assert(kGwEpiWarps % 4 == 0 && kGwEpiCols % 32 == 0 && kGwEpiCols % kGwLdCols == 0,
+              "whole 32-column chunks per epilogue warp");
+// accumulators in tensor memory (each kGwBN fp32 columns of 512): the MMA
+// issuer runs up to kGwNB - 1 groups ahead of the slowest epilogue warp
+constexpr int kGwNB = 512 / kGwBN > 4 ? 4 : 512 / kGwBN;
+static_assert(kGwNB >= 2, "at least two accumulators in tensor memory");
 constexpr int kGwGemmThreads = 64 + 32 * kGwEpiWarps;
 constexpr int kGwSmemLimit = 227 * 1024;
 constexpr int kGwStageBox = 2048;  // one 32 x 32 bf16 output box
 
-// GEMM stage: A codes 128 x 64 bytes, B codes 256 x 64 bytes (both 64-byte
-// swizzle), then the group's 128 activation scales and 256 weight scales;
-// a low-rank step puts u (128 x 32 bf16) and l2 (256 x 32 bf16) in the same
-// A and B slots.
+// GEMM stage: A codes 128 x 64 bytes and B codes kGwBN x 64 bytes (both
+// 64-byte swizzle), then the group's 128 activation scales and kGwBN weight
+// scales (the epilogue reads them here: shared-memory broadcast reads cost
+// far less than the same reads from L1); a low-rank step puts u (128 x 32
+// bf16) and l2 (kGwBN x 32 bf16) in the A and B slots.
 constexpr int kGwA = kTokRows * 64;
 constexpr int kGwB = kGwBN * 64;
 constexpr int kGwSA = kTokRows * 4;
@@ -139,20 +164,37 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 
-// 32 lanes x 8 consecutive 32-bit columns: thread i of the warp receives
-// columns [col, col+8) of tensor-memory lane (warp quarter * 32 + i).
-__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                 "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
-
 // Tensor-memory columns holding u (rank 32 or 64; allocations are powers of
 // two from 32).
 __device__ __forceinline__ uint32_t gw_u_cols(int rank) { return rank <= 32 ? 32u : 64u; }
 
 }  // namespace
+
+// 32 lanes x 8, 16, 32 or 64 consecutive 32-bit columns: thread i of the warp
+// receives that many columns from col on of tensor-memory lane
+// (warp quarter * 32 + i).
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld_32x32b_x32(taddr, r);
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld_32x32b_x32(taddr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 
 // ------------------------------------------------------------ weight side
 // l1[r,k] = bf16(L1[r,k] * sigma_inv[k]) and l2 = bf16(L2): the product is
@@ -289,9 +331,8 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
-      // every thread of the team (each releases its own loads), and the MMAs
-      // that read the stage's X tile
-      mbar_init(&empty[s], team_warps * 32 + (lowrank ? 1 : 0));
+      // the team's four warps, and the MMAs that read the stage's X tile
+      mbar_init(&empty[s], team_warps + (lowrank ? 1 : 0));
     }
     mbar_init(ufull, 1);
     *abort_flag = 0;
@@ -401,13 +442,14 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
       f2 w0[16], w1[16];
       qc::unpack32(*reinterpret_cast<const uint4(*)[4]>(&x[0]), w0);
       qc::unpack32(*reinterpret_cast<const uint4(*)[4]>(&x[4]), w1);
-      // the stage's X tile is in registers: each thread hands back its own
-      // reads.  They went through the generic proxy and the next write into
-      // the stage is a tensor copy (async proxy), so a proxy fence orders them
-      // before the arrive; without it, copies were seen overwriting a stage
-      // that some lanes were still reading.
+      // the stage's X tile is in registers: hand it back.  The reads went
+      // through the generic proxy and the next write into the stage is a
+      // tensor copy (async proxy), so every thread fences its own reads
+      // before the warp's arrive; without the fence, copies were seen
+      // overwriting a stage that some lanes were still reading.
       fence_proxy_async_smem();
-      mbar_arrive(&empty[stage]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
       if (p.sigma_inv) {
         const float4* s4 = reinterpret_cast<const float4*>(sig + j * kGroup);
 #pragma unroll
@@ -530,6 +572,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
 }  // namespace
 
 size_t gw_gemm_smem_bytes() { return kGwGemmSmem; }
+int gw_gemm_bn() { return kGwBN; }
 int gw_gemm_threads() { return kGwGemmThreads; }
 
 // Persistent: CTA b takes output tiles b, b + grid, ... in grouped order.
@@ -537,10 +580,11 @@ int gw_gemm_threads() { return kGwGemmThreads; }
 // the two accumulators in order: the low-rank step first (u x l2^T), then
 // group j = 0 .. G-1 (codes x codes^T over channels 64 j .. 64 j + 63).
 // Warp 0: producer (one thread); warp 1: tensor memory and (one thread) the
-// MMAs; warps 2..17: epilogue, four warps per 32-lane quarter of tensor
-// memory, each taking 64 of the tile's 256 columns, with the running sums in
-// registers (32 fp32 pairs a thread).
-__global__ void __maxnreg__(96)
+// MMAs; warps 2.. 2 + kGwEpiWarps - 1: epilogue, kGwEpiWarps / 4 warps per
+// 32-lane quarter of tensor memory, each taking kGwEpiCols of the tile's
+// columns, with the running sums in registers (kGwEpiCols / 2 fp32 pairs a
+// thread).
+__global__ void __maxnreg__(HQ_GW_MAXNREG)
     gw_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSW,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL2,
@@ -551,9 +595,9 @@ __global__ void __maxnreg__(96)
   uint8_t* epi_stage = smem + size_t(kGwStages) * kGwStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_stage + kGwEpiWarps * kGwStageBox);
   uint64_t* empty = full + kGwStages;
-  uint64_t* tfull = empty + kGwStages;  // [2] accumulator complete
-  uint64_t* tempty = tfull + 2;         // [2] accumulator read by the epilogue
-  uint64_t* drain = tempty + 2;
+  uint64_t* tfull = empty + kGwStages;  // [kGwNB] accumulator complete
+  uint64_t* tempty = tfull + kGwNB;     // [kGwNB] accumulator read by the epilogue
+  uint64_t* drain = tempty + kGwNB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -566,9 +610,9 @@ __global__ void __maxnreg__(96)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGwStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kGwEpiWarps * 32);  // the MMAs' commit and every epilogue thread
+      mbar_init(&empty[s], 1 + kGwEpiWarps);  // the MMAs' commit and every epilogue warp
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kGwNB; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kGwEpiWarps);
     }
@@ -651,8 +695,8 @@ __global__ void __maxnreg__(96)
       constexpr uint32_t kIdBf = bf16_idesc(kTokRows, kGwBN);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         for (int st = 0; st < steps; ++st, ++gstep) {
-          const int b = gstep & 1;
-          const uint32_t bph = uint32_t(gstep >> 1) & 1u;
+          const int b = gstep % kGwNB;
+          const uint32_t bph = uint32_t(gstep / kGwNB) & 1u;
           if (*abort_flag || !mbar_wait_spin(&tempty[b], bph ^ 1u, wc) ||
               !mbar_wait_spin(&full[stage], phase, wc)) {
             *abort_flag = 1;
@@ -703,9 +747,10 @@ __global__ void __maxnreg__(96)
       f2 acc[kGwEpiCols / 2];
 #pragma unroll
       for (int i = 0; i < kGwEpiCols / 2; ++i) acc[i] = pk(0.0f, 0.0f);
+
       for (int st = 0; st < steps; ++st, ++gstep) {
-        const int b = gstep & 1;
-        const uint32_t bph = uint32_t(gstep >> 1) & 1u;
+        const int b = gstep % kGwNB;
+        const uint32_t bph = uint32_t(gstep / kGwNB) & 1u;
         const bool got = !(*abort_flag) && mbar_wait_spin(&tfull[b], bph, wc) &&
                          mbar_wait_spin(&full[stage], phase, wc);
         if (!__all_sync(0xffffffffu, got)) {
@@ -714,57 +759,65 @@ __global__ void __maxnreg__(96)
           break;
         }
         tc_fence_after();
-        const uint32_t t_addr = t_warp + (b ? uint32_t(kGwBN) : 0u);
+        const uint32_t t_addr = t_warp + uint32_t(b * kGwBN);
         const uint32_t sb = smem_base + uint32_t(stage) * uint32_t(kGwStageBytes);
-        // eight columns per tensor-memory load keep the running sums (64 fp32
-        // a thread) and the loaded values within the 96 registers a thread
-        // has at 18 warps (five on the busiest sub-partition)
+        // kGwLdCols columns per tensor-memory load; a chunk's weight scales are
+        // read from shared memory before its load, so the two latencies
+        // overlap (tcgen05.wait::ld waits for every load in flight, which
+        // makes the load round trips the step's critical path).  The
+        // accumulator goes back to the MMA issuer once its last chunk landed.
+        constexpr int LDC = kGwLdCols;
         if (lowrank && st == 0) {
 #pragma unroll
-          for (int c = 0; c < kGwEpiCols / 8; ++c) {
-            uint32_t v[8];
-            tmem_ld_32x32b_x8(t_addr + uint32_t(8 * c), v);
+          for (int c = 0; c < kGwEpiCols / LDC; ++c) {
+            uint32_t v[LDC];
+            tmem_ld_cols(t_addr + uint32_t(LDC * c), v);
             tmem_wait_ld();
-            if (c == kGwEpiCols / 8 - 1) {
+            if (c == kGwEpiCols / LDC - 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&tempty[b]);
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              acc[4 * c + i] = add2(acc[4 * c + i],
-                                    pk(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])));
+            for (int i = 0; i < LDC / 2; ++i)
+              acc[(LDC / 2) * c + i] =
+                  add2(acc[(LDC / 2) * c + i],
+                       pk(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])));
           }
         } else {
           const float sa = ld_shared_f32(sb + uint32_t(kGwA + kGwB) + uint32_t(r) * 4u);
           const f2 sa2 = pk(sa, sa);
           const uint32_t sw = sb + uint32_t(kGwA + kGwB + kGwSA + part * kGwEpiCols * 4);
 #pragma unroll
-          for (int c = 0; c < kGwEpiCols / 8; ++c) {
-            uint32_t v[8];
-            tmem_ld_32x32b_x8(t_addr + uint32_t(8 * c), v);
+          for (int c = 0; c < kGwEpiCols / LDC; ++c) {
+            float4 w4[LDC / 4];
+#pragma unroll
+            for (int g = 0; g < LDC / 4; ++g) w4[g] = ld_shared_f4(sw + uint32_t(4 * (LDC * c + 4 * g)));
+            uint32_t v[LDC];
+            tmem_ld_cols(t_addr + uint32_t(LDC * c), v);
             tmem_wait_ld();
-            if (c == kGwEpiCols / 8 - 1) {
+            if (c == kGwEpiCols / LDC - 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&tempty[b]);
             }
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const float4 w4 = ld_shared_f4(sw + uint32_t(32 * c + 16 * g));
-              acc[4 * c + 2 * g] =
-                  fma2(pk(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1])),
-                       mul2(sa2, pk(w4.x, w4.y)), acc[4 * c + 2 * g]);
-              acc[4 * c + 2 * g + 1] =
-                  fma2(pk(__uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3])),
-                       mul2(sa2, pk(w4.z, w4.w)), acc[4 * c + 2 * g + 1]);
+            for (int g = 0; g < LDC / 4; ++g) {
+              f2& a0 = acc[(LDC / 2) * c + 2 * g];
+              f2& a1 = acc[(LDC / 2) * c + 2 * g + 1];
+              a0 = fma2(pk(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1])),
+                        mul2(sa2, pk(w4[g].x, w4[g].y)), a0);
+              a1 = fma2(pk(__uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3])),
+                        mul2(sa2, pk(w4[g].z, w4[g].w)), a1);
             }
           }
         }
-        // this thread's reads of the stage's scales, ordered before the next
-        // tensor copy into the stage (async proxy) by a proxy fence
+        // the warp's reads of the stage's scales, each thread's ordered
+        // before the next tensor copy into the stage (async proxy) by its
+        // proxy fence; one arrive per warp
         fence_proxy_async_smem();
-        mbar_arrive(&empty[stage]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
         if (++stage == kGwStages) {
           stage = 0;
           phase ^= 1u;

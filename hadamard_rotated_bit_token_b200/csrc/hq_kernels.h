@@ -189,11 +189,13 @@ cudaError_t launch_gw_act(const void* tmap_x, const void* tmap_l1, const GwActPa
 size_t gw_act_smem_bytes(int K, int rank, int stages, bool sigma);
 int gw_act_threads();
 // tmaps: 7 CUtensorMap in order A codes [T,K] u8 box {64,128} and B codes
-// [N,K] u8 box {64,256} (64-byte swizzle); s_x [G][ld] f32 box {128,1}; s_w
-// [G][N] f32 box {256,1}; u [T,32] bf16 box {32,128} and l2 [N,32] bf16
-// box {32,256} (64-byte swizzle); Y [T,N] bf16 box {32,32} (64-byte swizzle).
+// [N,K] u8 box {64,bn} (64-byte swizzle); s_x [G][ld] f32 box {128,1}; s_w
+// [G][N] f32 box {bn,1}; u [T,32] bf16 box {32,128} and l2 [N,32] bf16
+// box {32,bn} (64-byte swizzle); Y [T,N] bf16 box {32,32} (64-byte swizzle);
+// bn = gw_gemm_bn().
 cudaError_t launch_gw_gemm(const void* tmaps, const GwGemmParams& p, int grid, cudaStream_t st);
 size_t gw_gemm_smem_bytes();
 int gw_gemm_threads();
+int gw_gemm_bn();  // output tile width (the B, s_w and l2 boxes have this many rows)
 
 }  // namespace hq

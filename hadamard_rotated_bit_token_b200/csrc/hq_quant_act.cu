@@ -109,7 +109,7 @@ __device__ __forceinline__ void act_setup(const QuantParams& p, uint8_t* smem, c
   if (tid == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], uint32_t(ncw) * 32u);  // every consumer thread
+      mbar_init(&empty[s], uint32_t(ncw));  // one arrive per consumer warp
     }
     flags[0] = 0;
     flags[1] = 0;
@@ -326,12 +326,12 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
         if (NSL > 1) pin32(w[j]);
       }
       // every lane has the tile's slices in registers before the stage goes
-      // back; each thread releases its own loads, which went through the
-      // generic proxy, so a proxy fence orders them before the producer's
-      // next tensor copy into the stage; the mean's terms are in shared memory
-      __syncwarp();
+      // back; the loads went through the generic proxy, so each thread's proxy
+      // fence orders them before the producer's next tensor copy into the
+      // stage; the mean's terms are in shared memory
       fence_proxy_async_smem();
-      mbar_arrive(&empty[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
@@ -479,10 +479,11 @@ __global__ void __launch_bounds__(BIG ? kSegThreadsBig : kSegThreads, BIG ? 1 : 
       if (active) load_slice(smem_u32(smem) + uint32_t(s) * L.stage_bytes, c, x);
       f2 w[16];
       unpack32(x, w);
-      // each thread releases its own loads (generic proxy), ordered before
-      // the producer's next tensor copy into the stage by a proxy fence
+      // the loads went through the generic proxy: each thread's proxy fence
+      // orders them before the producer's next tensor copy into the stage
       fence_proxy_async_smem();
-      mbar_arrive(&empty[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
       if (++s == p.stages) {
         s = 0;
         ph ^= 1u;
