@@ -557,6 +557,101 @@ def per_config_records(hq, torch, args, head_cfg, dev, l2, peaks, ceiling, timed
     return out
 
 
+GW_GROUP, GW_RANK = 64, 32
+FP32_LANES_PER_SM = 128  # fp32 FMA lanes per SM (4 sub-partitions x 32)
+
+
+def group_wise_record(hq, torch, args, cfg, dev, l2, ceiling, clock_info, timed, check):
+    """The group-wise 4-bit form with its rank-32 16-bit branch (include/hq_gw.h)
+    on the same layer shape and inputs as the headline: graphs of K steps
+    (quantize + GEMM) over rotating inputs, and the two kernels alone.  The
+    GEMM's bound is the per-group rescale in its epilogue (two fp32 lane
+    operations per output element and group: the product of the two scales
+    and the fused multiply-add), so it reports against the fp32 lane rate
+    at the sampled SM clock as well as the tensor-core ceiling."""
+    Wb, bb = synth.make_w(cfg)
+    Xb = synth.make_x(cfg)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    X, W, b = to_dev(Xb), to_dev(Wb), to_dev(bb)
+    T, K, N = cfg.T, cfg.K, cfg.N
+    G = K // GW_GROUP
+    desc = hq.GwDesc(K, N, GW_GROUP, GW_RANK, 4, 4)
+    absmax = torch.zeros(K, dtype=torch.float32, device=dev)
+    hq.hq_calib_act_absmax(hq.LayerDesc(K, N, 1), X, absmax)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record()
+    layer = hq.GroupWiseQuantLinear(desc, W, b, absmax, cfg.alpha)
+    p1.record()
+    torch.cuda.synchronize()
+    bufs = layer.buffers(T)
+    Y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    n = int(min(512, max(2, -(-2 * l2 // (X.numel() * 2)) + 1)))
+    Xs = [X] + [X.clone() for _ in range(n - 1)]
+    si = layer.sigma_inv
+
+    def quantize_i(i):
+        hq.hq_gw_quantize_act(desc, Xs[i % n], si, layer.l1s, bufs["a_codes"], bufs["a_scale"],
+                              bufs["u"])
+
+    def linear():
+        hq.hq_gw_linear(desc, bufs["a_codes"], bufs["a_scale"], bufs["u"], layer.w_codes,
+                        layer.w_scale, layer.l2b, layer.bias_f32, Y, T=T)
+
+    for i in range(args.warmup):
+        quantize_i(i)
+        linear()
+    torch.cuda.synchronize()
+    graphs = []
+    for do_q, do_l in ((True, True), (True, False), (False, True)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(args.steps):
+                if do_q:
+                    quantize_i(i)
+                if do_l:
+                    linear()
+        g.replay()
+        graphs.append(g)
+    torch.cuda.synchronize()
+    step_ms, q_ms, g_ms = (timed(g) / args.steps for g in graphs)
+    check("in the group-wise form")
+    # the output against the unquantized layer (context: the error of the form)
+    ref = torch.matmul(X.float(), W.float().t()) + b.float()
+    quantize_i(0)
+    linear()
+    rel = float(((Y.float() - ref).norm() / ref.norm()).item())
+    ops = 2.0 * T * K * N + 2.0 * T * GW_RANK * (K + N)
+    q_bytes = T * K * 2 + T * K + T * G * 4 + T * GW_RANK * 2 + GW_RANK * K * 2
+    sm_mhz = (clock_info or {}).get("sm_mhz") or 1965.0
+    props = torch.cuda.get_device_properties(dev)
+    lane_ops = 2.0 * T * N * G + T * N  # scale product + multiply-add per group; branch add
+    lane_rate = props.multi_processor_count * FP32_LANES_PER_SM * sm_mhz * 1e6
+    g_tops = 2.0 * T * K * N / (g_ms * 1e-3) / 1e12
+    del graphs, Xs, layer, bufs
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"{cfg.workload()} in the group-wise form: groups of {GW_GROUP} channels "
+                    f"(H_{GW_GROUP} and one scale per group), W4A4, rank-{GW_RANK} bf16 branch",
+        "step_ms": step_ms, "step_TOPS": ops / (step_ms * 1e-3) / 1e12,
+        "weight_prep_ms": p0.elapsed_time(p1),
+        "rel_err_vs_unquantized": rel,
+        "quantizer": {"ms_per_launch": q_ms, "bytes": q_bytes,
+                      "GB/s": q_bytes / (q_ms * 1e-3) / 1e9,
+                      "what": "X read once: the group transform and codes on CUDA cores, "
+                              "u = X l1^T on the tensor cores from the same tiles"},
+        "gemm": {"ms_per_launch": g_ms, "TOPS": g_tops,
+                 "frac_mma_ceiling": g_tops / ceiling["single_cta_TOPS"]
+                 if ceiling.get("single_cta_TOPS") else None,
+                 "bound": "alu", "alu_lane_ops": lane_ops,
+                 "alu_floor_ms": lane_ops / lane_rate * 1e3,
+                 "frac_alu": lane_ops / lane_rate / (g_ms * 1e-3),
+                 "alu_peak": f"{props.multi_processor_count} SMs x {FP32_LANES_PER_SM} fp32 "
+                             f"lanes x {sm_mhz:.0f} MHz (sampled SM clock)",
+                 "what": "kind::f8f6f4 MMAs (e4m3 bytes holding the integer codes) into one "
+                         "fp32 accumulator per group, rescaled by s_x s_w in registers"},
+    }
+
+
 def run_hq(args):
     import torch
     import torch.distributed as dist
@@ -763,6 +858,9 @@ def run_hq(args):
     if not args.no_per_config and world == 1:
         line["per_config"] = per_config_records(hq, torch, args, cfg, dev, l2, peaks, ceiling,
                                                 timed, check)
+    if not args.no_variants and world == 1 and cfg.K % GW_GROUP == 0 and cfg.N % 16 == 0:
+        line["group_wise"] = group_wise_record(hq, torch, args, cfg, dev, l2, ceiling,
+                                               clock_info, timed, check)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(cfg, *host, args.cpu_seconds)
     print(json.dumps(line), flush=True)

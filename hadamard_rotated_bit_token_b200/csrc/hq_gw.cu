@@ -430,8 +430,11 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
     for (int j = team; j < G; j += 2) {
       const int stage = j % p.stages;
       const uint32_t phase = uint32_t(j / p.stages) & 1u;
-      const bool got = !(*abort_flag) && mbar_wait_spin(&full[stage], phase, wc);
-      if (!__all_sync(0xffffffffu, got)) {
+      // one lane waits; the warp barrier orders the others behind its acquire
+      bool got = true;
+      if (lane == 0) got = !(*abort_flag) && mbar_wait_spin(&full[stage], phase, wc);
+      __syncwarp();
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
         *abort_flag = 1;
         break;
       }
@@ -751,9 +754,14 @@ __global__ void __maxnreg__(HQ_GW_MAXNREG)
       for (int st = 0; st < steps; ++st, ++gstep) {
         const int b = gstep % kGwNB;
         const uint32_t bph = uint32_t(gstep / kGwNB) & 1u;
-        const bool got = !(*abort_flag) && mbar_wait_spin(&tfull[b], bph, wc) &&
-                         mbar_wait_spin(&full[stage], phase, wc);
-        if (!__all_sync(0xffffffffu, got)) {
+        // one lane waits (32 lanes spinning on one barrier word serialize in
+        // shared memory); the warp barrier orders the others behind its acquire
+        bool got = true;
+        if (lane == 0)
+          got = !(*abort_flag) && mbar_wait_spin(&tfull[b], bph, wc) &&
+                mbar_wait_spin(&full[stage], phase, wc);
+        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
           *abort_flag = 1;
           ok = false;
           break;

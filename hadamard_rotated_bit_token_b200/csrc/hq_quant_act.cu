@@ -275,7 +275,12 @@ __global__ void __maxnreg__(WRowCfg<SPL>::REGS)
     int s = 0;
     uint32_t ph = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-      if (!__all_sync(0xffffffffu, mbar_wait_spin(&full[s], ph, wc))) break;
+      // one lane waits (32 lanes spinning on one barrier word serialize in
+      // shared memory); the warp barrier orders the others behind its acquire
+      bool got = true;
+      if (lane == 0) got = mbar_wait_spin(&full[s], ph, wc);
+      __syncwarp();
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
       const uint32_t st_addr = smem_u32(smem) + uint32_t(s) * L.stage_bytes;
       f2 w[NSL][16];
       float mx = -INFINITY, mn = INFINITY, fmx = -INFINITY, fmn = INFINITY;
@@ -474,7 +479,9 @@ __global__ void __launch_bounds__(BIG ? kSegThreadsBig : kSegThreads, BIG ? 1 : 
       // together after the tile barrier below, so no warp is ever left
       // waiting there (the flag of a tile parity is read only after that
       // tile's barrier and written only before it)
-      if (!mbar_wait_spin(&full[s], ph, wc)) flags[2 + pb] = 1;
+      // one lane waits; the warp barrier orders the others behind its acquire
+      if (lane == 0 && !mbar_wait_spin(&full[s], ph, wc)) flags[2 + pb] = 1;
+      __syncwarp();
       uint4 x[4] = {};
       if (active) load_slice(smem_u32(smem) + uint32_t(s) * L.stage_bytes, c, x);
       f2 w[16];
