@@ -111,10 +111,15 @@ def gemm_bytes(cfg) -> float:
 # ---------------------------------------------------------------------------
 
 E2E_CHUNKS = 8  # row chunks of the end-to-end pipeline (hq_forward_host)
-PROFILES = {("gemm", 2): "gemm_i8_cfg2_pixart_qkv.md", ("quant", 2): "quant_rows_cfg2_pixart_qkv.md"}
+PROFILES = {("gemm", 2): "gemm_i8_cfg2_pixart_qkv.md", ("quant", 2): "quant_seg_cfg2_pixart_qkv.md",
+            ("gemm", 5): "gemm_i8_pair_cfg5_large_dit.md",
+            ("quant", 5): "quant_wrow_cfg5_large_dit.md",
+            ("gw_gemm", 5): "gw_gemm_cfg5_large_dit.md", ("gw_act", 5): "gw_act_cfg5_large_dit.md"}
 KERNEL_SOURCES = {"gemm": ("hq_gemm.cu", "hq_device.cuh", "hq_kernels.h"),
                   "quant": ("hq_quant_act.cu", "hq_quant_common.cuh", "hq_device.cuh",
-                            "hq_kernels.h")}
+                            "hq_kernels.h"),
+                  "gw_gemm": ("hq_gw.cu", "hq_quant_common.cuh", "hq_device.cuh", "hq_kernels.h"),
+                  "gw_act": ("hq_gw.cu", "hq_quant_common.cuh", "hq_device.cuh", "hq_kernels.h")}
 
 
 def kernel_source_hash(kind, root=ROOT):
@@ -629,6 +634,7 @@ def group_wise_record(hq, torch, args, cfg, dev, l2, ceiling, clock_info, timed,
     g_tops = 2.0 * T * K * N / (g_ms * 1e-3) / 1e12
     del graphs, Xs, layer, bufs
     torch.cuda.empty_cache()
+    profiled = cfg == synth.CONFIGS[cfg.index]
     return {
         "workload": f"{cfg.workload()} in the group-wise form: groups of {GW_GROUP} channels "
                     f"(H_{GW_GROUP} and one scale per group), W4A4, rank-{GW_RANK} bf16 branch",
@@ -637,9 +643,11 @@ def group_wise_record(hq, torch, args, cfg, dev, l2, ceiling, clock_info, timed,
         "rel_err_vs_unquantized": rel,
         "quantizer": {"ms_per_launch": q_ms, "bytes": q_bytes,
                       "GB/s": q_bytes / (q_ms * 1e-3) / 1e9,
+                      "traffic": profiled_traffic("gw_act", cfg.index) if profiled else None,
                       "what": "X read once: the group transform and codes on CUDA cores, "
                               "u = X l1^T on the tensor cores from the same tiles"},
         "gemm": {"ms_per_launch": g_ms, "TOPS": g_tops,
+                 "traffic": profiled_traffic("gw_gemm", cfg.index) if profiled else None,
                  "frac_mma_ceiling": g_tops / ceiling["single_cta_TOPS"]
                  if ceiling.get("single_cta_TOPS") else None,
                  "bound": "alu", "alu_lane_ops": lane_ops,
