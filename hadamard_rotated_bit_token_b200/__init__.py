@@ -601,14 +601,23 @@ class GroupWiseQuantLinear:
     from a singular value decomposition of W diag(sigma) (torch.linalg.svd in
     fp32 on the device, an offline step; the method fixes only L2 L1)."""
 
-    def __init__(self, desc: GwDesc, W, bias=None, act_absmax=None, alpha=0.5, factors=None):
+    def __init__(self, desc: GwDesc, W, bias=None, act_absmax=None, alpha=0.5, factors=None,
+                 sigma_inv=None):
+        """sigma_inv: a given smoothing vector (fp32 [K]) instead of the one
+        hq_gw_sigma_inv derives from act_absmax and alpha."""
         import torch
         self.desc = desc
         dev = W.device
         K, N, r = desc.K, desc.N, desc.rank
-        self.sigma_inv = torch.empty(K, dtype=torch.float32, device=dev)
-        hq_gw_sigma_inv(desc, W, act_absmax, alpha, self.sigma_inv)
-        self.use_sigma = act_absmax is not None
+        if sigma_inv is not None:
+            self.sigma_inv = sigma_inv.to(device=dev, dtype=torch.float32).contiguous()
+            if tuple(self.sigma_inv.shape) != (K,):
+                raise ValueError(f"sigma_inv must have shape ({K},)")
+            self.use_sigma = True
+        else:
+            self.sigma_inv = torch.empty(K, dtype=torch.float32, device=dev)
+            hq_gw_sigma_inv(desc, W, act_absmax, alpha, self.sigma_inv)
+            self.use_sigma = act_absmax is not None
         if r > 0:
             if factors is None:
                 What = W.float() / self.sigma_inv[None, :]
