@@ -144,6 +144,7 @@ CASES = [
     (130, 1024, 528, 32, 3, 4, False),
     (257, 2048, 784, 32, 4, 3, True),
     (64, 64 * 65, 32, 32, 4, 4, True),
+    (130, 16384, 48, 32, 4, 4, True),  # the largest K (sigma^-1 takes 64 KB of shared memory)
 ]
 
 
@@ -278,11 +279,14 @@ def test_gw_layer_module(hq):
     assert np.linalg.norm(y_ref - exact) <= 0.25 * np.linalg.norm(exact)
 
 
-def test_gw_large_dit_linear_sampled_rows(hq):
-    """T = 16384, K = 3072, N = 12288 (the large DiT linear) with rank 32: the
-    GPU computes every row; the oracle computes the weights in full and the
-    activations and outputs of sampled rows (first and last tiles included)."""
-    cfg = synth.CONFIGS[5]
+@pytest.mark.parametrize("cfg_index", [2, 5])
+def test_gw_full_layer_sampled_rows(hq, cfg_index):
+    """The PixArt-Sigma qkv layer (T = 8192, K = 1152, N = 3456) and the large
+    DiT linear (T = 16384, K = 3072, N = 12288) in the group-wise form with
+    rank 32: the GPU computes every row; the oracle computes the weights in
+    full and the activations and outputs of sampled rows (first and last
+    tiles included)."""
+    cfg = synth.CONFIGS[cfg_index]
     X, W, b = synth.make_layer(cfg)
     T, K, N = X.shape[0], X.shape[1], W.shape[0]
     si, sig = _sigma(X, W, True)
