@@ -838,3 +838,22 @@ def test_low_rank_factors_are_the_best_rank_r_approximation():
     s = np.linalg.svd(What, compute_uv=False)
     assert np.isclose(np.linalg.norm(What - L2 @ L1), np.sqrt(np.sum(s[8:] ** 2)), rtol=1e-10)
     assert np.allclose(L1 @ L1.T, np.eye(8), atol=1e-12)  # orthonormal rows
+
+
+def test_group_wise_inputs_of_the_wrong_shape_are_refused():
+    """The C side reads exactly the shapes the description implies: the
+    wrappers refuse factors, sigma or l1 of any other shape (a rank above
+    min(N, K) is zero-padded by low_rank_factors, not truncated)."""
+    W = synth.f32_to_bf16_bits(np.ones((4, 8), dtype=np.float32))
+    L1, L2 = oracle.low_rank_factors(W, None, 6)  # rank 6 > min(N, K) = 4
+    assert L1.shape == (6, 8) and L2.shape == (4, 6)
+    assert np.all(L1[4:] == 0) and np.all(L2[:, 4:] == 0)
+    with pytest.raises(ValueError):
+        oracle.gw_prepare_weights(W, 4, 4, 6, L1[:4], L2)
+    with pytest.raises(ValueError):
+        oracle.gw_prepare_weights(W, 4, 4, 6, L1, L2[:, :4])
+    with pytest.raises(ValueError):
+        oracle.gw_prepare_weights(W, 4, 4, 6, L1, L2, sigma=np.ones(7))
+    X = synth.f32_to_bf16_bits(np.ones((2, 8), dtype=np.float32))
+    with pytest.raises(ValueError):
+        oracle.gw_quantize_act(X, 4, 4, 2, np.zeros((3, 8), dtype=np.uint16))
