@@ -596,7 +596,7 @@ def group_wise_record(hq, torch, args, cfg, dev, l2, ceiling, clock_info, timed,
 
     def quantize_i(i):
         hq.hq_gw_quantize_act(desc, Xs[i % n], si, layer.l1s, bufs["a_codes"], bufs["a_scale"],
-                              bufs["u"])
+                              bufs["u"], bufs["workspace"])
 
     def linear():
         hq.hq_gw_linear(desc, bufs["a_codes"], bufs["a_scale"], bufs["u"], layer.w_codes,

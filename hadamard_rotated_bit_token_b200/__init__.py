@@ -16,7 +16,7 @@ The group-wise 4-bit form with a 16-bit low-rank branch (include/hq_gw.h):
 
     hq_gw_sigma_inv(desc, W, act_absmax, alpha, sigma_inv)
     hq_gw_prepare_weights(desc, W, bias, sigma_inv, L1, L2, w_codes, w_scale, l1s, l2b, bias_f32)
-    hq_gw_quantize_act(desc, X, sigma_inv, l1s, a_codes, a_scale, u)
+    hq_gw_quantize_act(desc, X, sigma_inv, l1s, a_codes, a_scale, u, workspace)
     hq_gw_linear(desc, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32, Y)
 
 `HadamardQuantLinear` and `GroupWiseQuantLinear` bundle the caller-side
@@ -41,7 +41,7 @@ __all__ = [
     "hq_quantize_act_noalloc", "hq_debug_plan", "hq_debug_mma_ceiling", "hq_debug_tmap_cache",
     "HadamardQuantLinear", "GwDesc", "hq_gw_scale_ld", "hq_gw_sigma_inv", "hq_gw_prepare_weights",
     "hq_gw_quantize_act", "hq_gw_linear", "hq_gw_debug_linear_f32", "GroupWiseQuantLinear",
-    "hq_debug_last_cuda_error",
+    "hq_debug_last_cuda_error", "hq_gw_quantize_act_workspace_bytes",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -61,7 +61,8 @@ EXPORTED = ("hq_status_string", "hq_version", "hq_calib_act_absmax", "hq_prepare
             "hq_debug_set_gemm_variant", "hq_quantize_act_noalloc", "hq_debug_plan",
             "hq_debug_mma_ceiling", "hq_debug_tmap_cache", "hq_gw_scale_ld", "hq_gw_sigma_inv",
             "hq_gw_prepare_weights", "hq_gw_quantize_act", "hq_gw_linear",
-            "hq_gw_debug_linear_f32", "hq_debug_last_cuda_error")
+            "hq_gw_debug_linear_f32", "hq_debug_last_cuda_error",
+            "hq_gw_quantize_act_workspace_bytes")
 
 
 class HQError(RuntimeError):
@@ -150,8 +151,10 @@ def load_library():
         lib.hq_gw_sigma_inv.argtypes = [gw_p, _vp, _vp, ctypes.c_float, _vp, _vp]
         lib.hq_gw_prepare_weights.argtypes = [gw_p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                               _vp, _vp]
+        lib.hq_gw_quantize_act_workspace_bytes.argtypes = [gw_p, ctypes.c_int64]
+        lib.hq_gw_quantize_act_workspace_bytes.restype = ctypes.c_size_t
         lib.hq_gw_quantize_act.argtypes = [gw_p, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
-                                           _vp]
+                                           _vp, ctypes.c_size_t, _vp]
         lib.hq_gw_linear.argtypes = [gw_p, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp]
         lib.hq_gw_debug_linear_f32.argtypes = list(lib.hq_gw_linear.argtypes)
@@ -369,12 +372,17 @@ def hq_gw_prepare_weights(desc: GwDesc, W, bias, sigma_inv, L1, L2, w_codes, w_s
         "hq_gw_prepare_weights")
 
 
-def hq_gw_quantize_act(desc: GwDesc, X, sigma_inv, l1s, a_codes, a_scale, u, T=None,
-                       stream=None):
+def hq_gw_quantize_act_workspace_bytes(desc: GwDesc, T: int) -> int:
+    return int(load_library().hq_gw_quantize_act_workspace_bytes(ctypes.byref(desc), int(T)))
+
+
+def hq_gw_quantize_act(desc: GwDesc, X, sigma_inv, l1s, a_codes, a_scale, u, workspace=None,
+                       T=None, stream=None):
     T = X.shape[0] if T is None else T
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().hq_gw_quantize_act(
         ctypes.byref(desc), _ptr(X), T, _ptr(sigma_inv), _ptr(l1s), _ptr(a_codes), _ptr(a_scale),
-        _ptr(u), _stream(stream)), "hq_gw_quantize_act")
+        _ptr(u), _ptr(workspace), ws_bytes, _stream(stream)), "hq_gw_quantize_act")
 
 
 def hq_gw_linear(desc: GwDesc, a_codes, a_scale, u, w_codes, w_scale, l2b, bias_f32, Y, T=None,
@@ -652,17 +660,19 @@ class GroupWiseQuantLinear:
         if b is None:
             dev = self.w_codes.device
             K, r = self.desc.K, self.desc.rank
+            ws = hq_gw_quantize_act_workspace_bytes(self.desc, T)
             b = {"a_codes": torch.empty((T, K), dtype=torch.float8_e4m3fn, device=dev),
                  "a_scale": torch.empty((K // 64, hq_gw_scale_ld(T)), dtype=torch.float32,
                                         device=dev),
-                 "u": torch.empty((T, r), dtype=torch.bfloat16, device=dev) if r else None}
+                 "u": torch.empty((T, r), dtype=torch.bfloat16, device=dev) if r else None,
+                 "workspace": torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None}
             self._bufs[T] = b
         return b
 
     def quantize(self, X):
         b = self.buffers(X.shape[0])
         hq_gw_quantize_act(self.desc, X, self.sigma_inv if self.use_sigma else None, self.l1s,
-                           b["a_codes"], b["a_scale"], b["u"])
+                           b["a_codes"], b["a_scale"], b["u"], b["workspace"])
         return b
 
     def forward(self, X, Y=None):

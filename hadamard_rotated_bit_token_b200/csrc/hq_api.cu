@@ -1412,9 +1412,17 @@ hq_status hq_gw_prepare_weights(const hq_gw_desc* desc, const uint16_t* W, const
   return from_cuda(launch_gw_weights(p, st));
 }
 
+size_t hq_gw_quantize_act_workspace_bytes(const hq_gw_desc* desc, int64_t T) {
+  if (check_gw_desc(desc) != HQ_OK || T <= 0 || desc->rank == 0) return 0;
+  const int64_t blocks = (T + 127) / 128;
+  // two fp32 parts of u per token, then one ticket per 128-token block
+  return size_t(2 * T * desc->rank * 4 + (blocks * 4 + 15) / 16 * 16);
+}
+
 hq_status hq_gw_quantize_act(const hq_gw_desc* desc, const uint16_t* X, int64_t T,
                              const float* sigma_inv, const uint16_t* l1s, uint8_t* a_codes,
-                             float* a_scale, uint16_t* u, hq_stream_t stream) {
+                             float* a_scale, uint16_t* u, void* workspace, size_t workspace_bytes,
+                             hq_stream_t stream) {
   hq_status s = check_gw_desc(desc);
   if (s != HQ_OK) return s;
   const int rank = desc->rank;
@@ -1422,7 +1430,8 @@ hq_status hq_gw_quantize_act(const hq_gw_desc* desc, const uint16_t* X, int64_t 
       (rank > 0 && (l1s == nullptr || u == nullptr)))
     return HQ_ERR_INVALID_ARGUMENT;
   if (!aligned16(X) || !aligned16(a_codes) || !aligned16(a_scale) ||
-      (sigma_inv && !aligned16(sigma_inv)) || (rank > 0 && (!aligned16(l1s) || !aligned16(u))))
+      (sigma_inv && !aligned16(sigma_inv)) || (rank > 0 && (!aligned16(l1s) || !aligned16(u))) ||
+      (workspace && !aligned16(workspace)))
     return HQ_ERR_MISALIGNED;
   if (T == 0) return HQ_OK;
   DeviceState* dev;
@@ -1455,10 +1464,26 @@ hq_status hq_gw_quantize_act(const hq_gw_desc* desc, const uint16_t* X, int64_t 
   while (stages > 2 && gw_act_smem_bytes(K, rank, stages, sigma_inv != nullptr) > 227u * 1024u)
     --stages;
   p.stages = stages;
-  const int64_t grid = (T + 127) / 128;
-  if (grid >= (int64_t(1) << 31)) return HQ_ERR_UNSUPPORTED;
-  return from_cuda(
-      launch_gw_act(&tx, &tl, p, int(grid), reinterpret_cast<cudaStream_t>(stream)));
+  const int64_t blocks = (T + 127) / 128;
+  if (blocks >= (int64_t(1) << 30)) return HQ_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Blocks that fill less than half the GPU are split: two CTAs per block,
+  // each taking half of the groups (the branch's parts of u go through the
+  // workspace, so without one a block stays whole).
+  p.split = 1;
+  const size_t need = hq_gw_quantize_act_workspace_bytes(desc, T);
+  if (2 * blocks <= dev->sm_count && K / 64 >= 2 &&
+      (rank == 0 || (workspace != nullptr && workspace_bytes >= need))) {
+    p.split = 2;
+    if (rank > 0) {
+      p.upart = static_cast<float*>(workspace);
+      p.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
+                                                   size_t(2 * T * rank * 4));
+      s = from_cuda(cudaMemsetAsync(p.counters, 0, size_t(blocks) * 4, st));
+      if (s != HQ_OK) return s;
+    }
+  }
+  return from_cuda(launch_gw_act(&tx, &tl, p, int(blocks * p.split), st));
 }
 
 hq_status hq_gw_linear(const hq_gw_desc* desc, int64_t T, const uint8_t* a_codes,

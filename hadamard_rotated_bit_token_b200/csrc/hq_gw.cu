@@ -164,6 +164,23 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
 
+// 32 fp32 values (bit patterns) -> 32 bf16 (round to nearest even) at dst
+// (64 bytes, 16-byte aligned).
+__device__ __forceinline__ void store_u32(uint16_t* dst16, const uint32_t (&v)[32]) {
+  uint4* dst = reinterpret_cast<uint4*>(dst16);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * c + 2 * e]),
+                                                __uint_as_float(v[8 * c + 2 * e + 1]));
+      h[e] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    dst[c] = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+}
+
 // Tensor-memory columns holding u (rank 32 or 64; allocations are powers of
 // two from 32).
 __device__ __forceinline__ uint32_t gw_u_cols(int rank) { return rank <= 32 ? 32u : 64u; }
@@ -317,11 +334,18 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
   uint64_t* ufull = empty + p.stages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ufull + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;  // this CTA adds the parts of u
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl wc{p.err, p.wait_ns};
   const int G = p.K / kGroup;
-  const int64_t row0 = int64_t(blockIdx.x) * kTokRows;
+  // p.split CTAs share a block of 128 tokens, each taking the groups
+  // [j0, j1); with a branch each accumulates its part of u, and the one to
+  // finish last adds the parts in part order
+  const int blk = int(blockIdx.x) / p.split, part = int(blockIdx.x) % p.split;
+  const int j0 = G * part / p.split, j1 = G * (part + 1) / p.split;
+  const int GL = j1 - j0;
+  const int64_t row0 = int64_t(blk) * kTokRows;
   const bool lowrank = p.rank > 0;
   const int team_warps = 4;
 
@@ -356,7 +380,7 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       const uint32_t tx = L.stage_bytes;
-      for (int j = 0; j < G; ++j) {
+      for (int j = j0; j < j1; ++j) {
         if (*abort_flag || !mbar_wait_spin(&empty[stage], phase ^ 1u, wc)) {
           *abort_flag = 1;
           ok = false;
@@ -365,7 +389,7 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
         mbar_arrive_expect_tx(&full[stage], tx);
         uint8_t* st = smem + size_t(stage) * L.stage_bytes;
         // the fault hook withholds the first tile's copy (its wait times out)
-        if (!(p.fault && j == 0))
+        if (!(p.fault && j == j0))
           tma_load_2d(st + L.x_off, &tmX, j * kGroup, int32_t(row0), &full[stage]);
         if (lowrank) tma_load_2d(st + L.l1_off, &tmL1, j * kGroup, 0, &full[stage]);
         ++issued;
@@ -393,7 +417,7 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
       const uint32_t idesc = bf16_idesc(kTokRows, p.rank);
       int stage = 0;
       uint32_t phase = 0;
-      for (int j = 0; j < G; ++j) {
+      for (int j = 0; j < GL; ++j) {
         if (*abort_flag || !mbar_wait_spin(&full[stage], phase, wc)) {
           *abort_flag = 1;
           break;
@@ -427,9 +451,10 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
     const int swz = r & 7;  // 128-byte swizzle: chunk c of row r at c ^ (r % 8)
     const float q = float(p.q);
     const f2 mg2 = pk(qc::kRoundMagic, qc::kRoundMagic);
-    for (int j = team; j < G; j += 2) {
-      const int stage = j % p.stages;
-      const uint32_t phase = uint32_t(j / p.stages) & 1u;
+    for (int jl = team; jl < GL; jl += 2) {
+      const int j = j0 + jl;  // the group; jl its place in this CTA's sequence
+      const int stage = jl % p.stages;
+      const uint32_t phase = uint32_t(jl / p.stages) & 1u;
       // one lane waits; the warp barrier orders the others behind its acquire
       bool got = true;
       if (lane == 0) got = !(*abort_flag) && mbar_wait_spin(&full[stage], phase, wc);
@@ -500,29 +525,67 @@ __global__ void __launch_bounds__(kGwActThreads, 1)
       // u = bf16(X l1^T) from tensor memory: lane quarter `quarter`, one
       // token per lane, rank fp32 columns
       const bool got = !(*abort_flag) && mbar_wait(ufull, 0, wc);
-      if (__all_sync(0xffffffffu, got)) {
-        tc_fence_after();
-        for (int c0 = 0; c0 < p.rank; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(c0), v);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.u + t * p.rank + c0);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t h[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * c + 2 * e]),
-                                                          __uint_as_float(v[8 * c + 2 * e + 1]));
-                h[e] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              dst[c] = make_uint4(h[0], h[1], h[2], h[3]);
-            }
+      const bool ok = __all_sync(0xffffffffu, got);
+      if (!ok) *abort_flag = 1;
+      if (p.split == 1) {
+        if (ok) {
+          tc_fence_after();
+          for (int c0 = 0; c0 < p.rank; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(c0), v);
+            tmem_wait_ld();
+            if (row_ok) store_u32(p.u + t * p.rank + c0, v);
           }
         }
       } else {
-        *abort_flag = 1;
+        // this CTA's part of u to its slot of the workspace; the CTA that
+        // finishes last (an atomic ticket per block) adds the parts in part
+        // order, so the sum does not depend on which CTA that is
+        if (ok) {
+          tc_fence_after();
+          for (int c0 = 0; c0 < p.rank; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(c0), v);
+            tmem_wait_ld();
+            if (row_ok) {
+              float4* dst = reinterpret_cast<float4*>(p.upart + (int64_t(part) * p.T + t) * p.rank + c0);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                dst[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                     __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+            }
+          }
+        }
+        __threadfence();
+        named_barrier_sync(1, 32 * team_warps);
+        if (warp == 2 && lane == 0)
+          *last_flag = atomicAdd(&p.counters[blk], 1u) == unsigned(p.split - 1) ? 1 : 0;
+        named_barrier_sync(1, 32 * team_warps);
+        if (*last_flag && !*abort_flag) {
+          __threadfence();
+          for (int c0 = 0; c0 < p.rank; c0 += 32) {
+            if (!row_ok) break;
+            float s[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) s[c] = 0.0f;
+            for (int q = 0; q < p.split; ++q) {
+              const float4* src =
+                  reinterpret_cast<const float4*>(p.upart + (int64_t(q) * p.T + t) * p.rank + c0);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const float4 w = __ldcg(src + c);
+                s[4 * c] += w.x;
+                s[4 * c + 1] += w.y;
+                s[4 * c + 2] += w.z;
+                s[4 * c + 3] += w.w;
+              }
+            }
+            uint32_t v[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(s[c]);
+            store_u32(p.u + t * p.rank + c0, v);
+          }
+        }
       }
     }
   }

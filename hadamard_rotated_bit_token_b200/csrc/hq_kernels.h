@@ -160,8 +160,11 @@ struct GwActParams {
   uint8_t* codes;           // [T,K] e4m3
   float* scale;             // [K/64][ld]
   uint16_t* u;              // [T,rank] bf16 (rank > 0)
+  float* upart;             // [split][T][rank] fp32 partial u (split > 1, rank > 0)
+  unsigned int* counters;   // [blocks] zeroed before the launch (split > 1, rank > 0)
   int64_t T;
   int K, ld, rank, q, stages;
+  int split;                // CTAs per 128-token block (1 or 2), each taking a range of groups
   int fault;                // withhold the first tile's copy (timeout path)
   unsigned int* err;
   unsigned long long wait_ns;
@@ -182,8 +185,9 @@ cudaError_t launch_gw_factors(const float* L1, const float* L2, const float* sig
                               int K, int N, uint16_t* l1s, uint16_t* l2b, int sms, cudaStream_t st);
 // R = (W - l2 l1) sigma, R H_64 per group, codes and scales; one CTA per row.
 cudaError_t launch_gw_weights(const GwWeightParams& p, cudaStream_t st);
-// One CTA per 128 tokens.  tmap_x: X [T,K] bf16, box {64, 128}, 128-byte
-// swizzle; tmap_l1: l1s [rank,K] bf16, box {64, rank}, 128-byte swizzle.
+// split CTAs per 128 tokens (grid = blocks * split).  tmap_x: X [T,K] bf16,
+// box {64, 128}, 128-byte swizzle; tmap_l1: l1s [rank,K] bf16, box
+// {64, rank}, 128-byte swizzle.
 cudaError_t launch_gw_act(const void* tmap_x, const void* tmap_l1, const GwActParams& p, int grid,
                           cudaStream_t st);
 size_t gw_act_smem_bytes(int K, int rank, int stages, bool sigma);

@@ -91,6 +91,11 @@ hq_status hq_gw_prepare_weights(const hq_gw_desc* desc, const uint16_t* W, const
                                 uint8_t* w_codes, float* w_scale, uint16_t* l1s, uint16_t* l2b,
                                 float* bias_f32, hq_stream_t stream);
 
+/* Bytes of device workspace that let hq_gw_quantize_act split a block of
+ * 128 tokens over two CTAs when the blocks fill less than half the GPU
+ * (0 when rank = 0, which needs none). */
+size_t hq_gw_quantize_act_workspace_bytes(const hq_gw_desc* desc, int64_t T);
+
 /* hq_gw_quantize_act -- runtime activation side, one pass over X (steps 2, 3,
  * 6, 7): per token t and group j, V = (X[t, group j] * sigma_inv) H~_64 and
  * a_scale[j * ld + t] = max|V| / (8 q), codes = rne(V q / max|V|); and, from
@@ -100,10 +105,18 @@ hq_status hq_gw_prepare_weights(const hq_gw_desc* desc, const uint16_t* W, const
  *          (from hq_gw_prepare_weights; NULL when rank = 0).
  * Outputs: a_codes e4m3 bytes [T,K]; a_scale fp32 [K/64][ld]; u bf16
  *          [T,rank] (NULL when rank = 0).  A group whose max is 0 gets scale
- *          0 and zero codes. */
+ *          0 and zero codes.
+ * workspace: device, 16-byte aligned, >= hq_gw_quantize_act_workspace_bytes
+ *   bytes, or NULL; contents need not be initialised.  When the blocks of 128
+ *   tokens fill less than half the GPU, a workspace lets each block's groups
+ *   be split over two CTAs, whose fp32 parts of u the one finishing last adds
+ *   in a fixed order (deterministic; codes and scales are the same either
+ *   way, u's fp32 sum is taken in two parts).  Without one, blocks stay
+ *   whole. */
 hq_status hq_gw_quantize_act(const hq_gw_desc* desc, const uint16_t* X, int64_t T,
                              const float* sigma_inv, const uint16_t* l1s, uint8_t* a_codes,
-                             float* a_scale, uint16_t* u, hq_stream_t stream);
+                             float* a_scale, uint16_t* u, void* workspace,
+                             size_t workspace_bytes, hq_stream_t stream);
 
 /* hq_gw_linear -- the output (step 4): the group-wise GEMM with the 16-bit
  * branch and the bias fused into its epilogue (the formula at the top).

@@ -258,7 +258,7 @@ def test_gw_desc_layout_matches_the_header(hq):
 def _gw_quant(hq, desc, X=FAKE, T=4, codes=FAKE, scale=FAKE, l1s=FAKE, u=FAKE):
     lib = hq.load_library()
     d = None if desc is None else ctypes.byref(desc)
-    return lib.hq_gw_quantize_act(d, X, T, None, l1s, codes, scale, u, None)
+    return lib.hq_gw_quantize_act(d, X, T, None, l1s, codes, scale, u, None, 0, None)
 
 
 def _gw_linear(hq, desc, T=4, a=FAKE, sa=FAKE, u=FAKE, w=FAKE, sw=FAKE, l2=FAKE, Y=FAKE):
@@ -291,3 +291,8 @@ def test_gw_validation(hq):
                                      FAKE, FAKE, None, None, FAKE, None) == 1  # rank 32, no factors
     assert lib.hq_gw_sigma_inv(ctypes.byref(G(1024, 16)), FAKE, None, 1.5, FAKE, None) == 1
     assert hq.hq_gw_scale_ld(0) == 0 and hq.hq_gw_scale_ld(5) == 8 and hq.hq_gw_scale_ld(8) == 8
+    # workspace: two fp32 parts of u per token and a ticket per 128-token block
+    assert hq.hq_gw_quantize_act_workspace_bytes(G(1024, 16), 300) == 2 * 300 * 32 * 4 + 16
+    assert hq.hq_gw_quantize_act_workspace_bytes(G(1024, 16, rank=0), 300) == 0
+    assert lib.hq_gw_quantize_act(ctypes.byref(G(1024, 16)), FAKE, 4, None, FAKE, FAKE, FAKE,
+                                  FAKE, FAKE + 4, 1 << 20, None) == 3  # misaligned workspace

@@ -94,15 +94,23 @@ def _gpu_prepare(hq, desc, W, b, si, L1, L2):
     return {"codes": w_codes, "scale": w_scale, "l1s": l1s, "l2b": l2b, "bias": bias_f32}
 
 
-def _gpu_quantize(hq, desc, X, si, l1s):
+def _gpu_quantize(hq, desc, X, si, l1s, workspace=True):
+    """workspace: give the call the workspace that lets small batches split
+    each token block over two CTAs (poisoned, since the call must not rely
+    on its contents)."""
     T, K = X.shape
     r = desc.rank
     ld = hq.hq_gw_scale_ld(T)
     a_codes = torch.full((T, K), 100.0, device="cuda").to(torch.float8_e4m3fn)
     a_scale = torch.full((K // 64, ld), float("nan"), device="cuda")
     u = torch.full((T, r), float("nan"), dtype=torch.bfloat16, device="cuda") if r else None
+    ws = None
+    nbytes = hq.hq_gw_quantize_act_workspace_bytes(desc, T)
+    if workspace and nbytes:
+        ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")
     Xd = to_dev_u16(X, torch)
-    hq.hq_gw_quantize_act(desc, Xd, None if si is None else _dev(si), l1s, a_codes, a_scale, u)
+    hq.hq_gw_quantize_act(desc, Xd, None if si is None else _dev(si), l1s, a_codes, a_scale, u,
+                          ws)
     assert hq.hq_check_device_error() == 0
     return {"codes": a_codes, "scale": a_scale, "u": u, "X": Xd}
 
@@ -233,6 +241,8 @@ def test_gw_zero_tokens_and_zero_groups(hq):
     wp = _gpu_prepare(hq, desc, W, b, None, L1, L2)
     spare = torch.full((64,), 7.0, dtype=torch.float32, device="cuda")  # never written for T = 0
     hq.hq_gw_quantize_act(desc, spare, None, wp["l1s"], spare, spare, spare, T=0)
+    assert hq.hq_gw_quantize_act_workspace_bytes(desc, 0) == 0
+    assert hq.hq_gw_quantize_act_workspace_bytes(hq.GwDesc(K, N, 64, 0, 4, 4), 1000) == 0
     hq.hq_gw_linear(desc, spare, spare, spare, wp["codes"], wp["scale"], wp["l2b"], wp["bias"],
                     spare, T=0)
     torch.cuda.synchronize()
@@ -328,6 +338,12 @@ def test_gw_wait_timeout_is_reported(hq):
         u = torch.empty((T, 32), dtype=torch.bfloat16, device="cuda")
         hq.hq_gw_quantize_act(desc, to_dev_u16(X, torch), None, wp["l1s"], a_codes, a_scale, u)
         torch.cuda.synchronize()
+        assert hq.hq_check_device_error() == 5  # HQ_ERR_TIMEOUT, blocks whole
+        ws = torch.empty(hq.hq_gw_quantize_act_workspace_bytes(desc, T), dtype=torch.uint8,
+                         device="cuda")
+        hq.hq_gw_quantize_act(desc, to_dev_u16(X, torch), None, wp["l1s"], a_codes, a_scale, u,
+                              ws)
+        torch.cuda.synchronize()
         assert hq.hq_check_device_error() == 5  # HQ_ERR_TIMEOUT
     finally:
         hq.hq_debug_inject_fault(hq.HQ_FAULT_NONE)
@@ -335,3 +351,25 @@ def test_gw_wait_timeout_is_reported(hq):
     assert hq.hq_check_device_error() == 0
     ap = _gpu_quantize(hq, desc, X, None, wp["l1s"])
     assert _codes_int(ap["codes"]).shape == (T, K)
+
+
+@pytest.mark.parametrize("T,K,rank", [(300, 1152, 32), (8192, 1152, 32), (129, 256, 0)])
+def test_gw_split_blocks_match_whole_blocks(hq, T, K, rank):
+    """With a workspace, small batches split each 128-token block's groups
+    over two CTAs: codes and scales are identical to the unsplit call, and u
+    (its fp32 sum taken in two parts) meets the same bound as the unsplit u."""
+    N = 64
+    X, W, b = _inputs(T, K, N, seed=T + K)
+    si, sig = _sigma(X, W, True)
+    L1, L2 = _factors(W, sig, rank)
+    desc = hq.GwDesc(K, N, 64, rank, 4, 4)
+    wp = _gpu_prepare(hq, desc, W, b, si, L1, L2)
+    whole = _gpu_quantize(hq, desc, X, si, wp["l1s"], workspace=False)
+    split = _gpu_quantize(hq, desc, X, si, wp["l1s"], workspace=True)
+    assert torch.equal(whole["codes"].view(torch.uint8), split["codes"].view(torch.uint8))
+    assert torch.equal(whole["scale"][:, :T], split["scale"][:, :T])
+    if rank:
+        # both within the fp32 accumulation bound of the exact sum (a value
+        # near zero may change sign between the two summation orders)
+        _check_u(bf16_bits(whole["u"]), X, bf16_bits(wp["l1s"]), "u, whole blocks")
+        _check_u(bf16_bits(split["u"]), X, bf16_bits(wp["l1s"]), "u, split blocks")
