@@ -30,10 +30,12 @@
 //                      quantizer warps, one token per lane and one group per
 //                      stage, apply sigma^-1, the 64-point fast Walsh-Hadamard
 //                      transform in registers, the group max and the codes;
-//                      at the end u leaves tensor memory as bf16;
+//                      at the end u leaves tensor memory as bf16 (a small
+//                      batch may split each block's groups over two CTAs,
+//                      whose parts of u the last to finish adds);
 //   gw_gemm_kernel     the output: per output tile (128 x 256) and group j,
 //                      two kind::f8f6f4 MMAs (K = 64) into one of two fp32
-//                      accumulators in tensor memory, and eight epilogue
+//                      accumulators in tensor memory, and sixteen epilogue
 //                      warps that add s_x[t,j] s_w[n,j] times each finished
 //                      accumulator into registers while the tensor cores fill
 //                      the other; the low-rank term is one more step of two
