@@ -26,10 +26,14 @@ def test_measured_choices_for_the_configurations(hq):
     # 252 consumers in 8 warps plus the producer warp; 192-column GEMM tiles
     assert _plan(hq, 1152, 3456, 128, 8192) == {"quant_rows": 7, "quant_threads": 288,
                                                  "gemm_pair": False, "gemm_bn": 192}
-    # config 3: one row of 144 slices per tile (5 consumer warps);
-    # N = 1152 is not a whole number of pair tiles
+    # config 3: rows of 144 slices; three-row tiles of the one-CTA variant
+    # (432 consumers in 14 warps) take 19 tile rounds where one-row tiles of
+    # the two-CTA variant take 28; N = 1152 is not a whole number of pair tiles
     p = _plan(hq, 4608, 1152, 256, 8192, a_bits=3)
-    assert (p["quant_rows"], p["quant_threads"], p["gemm_pair"], p["gemm_bn"]) == (1, 192, False, 192)
+    assert (p["quant_rows"], p["quant_threads"], p["gemm_pair"], p["gemm_bn"]) == (3, 480, False, 192)
+    # ... and with few tokens, where both take one round, the two-CTA variant
+    p = _plan(hq, 4608, 1152, 256, 130, a_bits=3)
+    assert (p["quant_rows"], p["quant_threads"]) == (1, 192)
     # config 4: rows of 10 slices, three to a warp (warp-row kernel): 24 rows
     # per tile over 8 consumer warps
     p = _plan(hq, 320, 320, 64, 65536, a_bits=8, w_bits=8, act_gran=1, centering=0)
@@ -71,8 +75,9 @@ def test_plan_invariants_over_shapes(hq):
         elif S % 32 == 0 and S <= 128:  # warp-row kernel, one row per warp
             assert R == nt // 32 - 1
         else:  # segment kernel: one thread per slice, plus the producer warp
-            # (up to 256 slices a tile, or 480 in the large-row variant)
-            assert R * S + 32 <= nt < R * S + 64 and R * S <= (256 if S <= 256 else 480)
+            # (up to 256 slices a tile in the two-CTA variant, 480 in the
+            # one-CTA variant, the only one for rows of more than 256 slices)
+            assert R * S + 32 <= nt < R * S + 64 and R * S <= 480
         assert p["gemm_bn"] in (64, 128, 192, 256)
         if packed:
             assert not p["gemm_pair"] and p["gemm_bn"] <= 192
