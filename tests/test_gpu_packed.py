@@ -50,7 +50,8 @@ def _quantize(hq, desc, X, sigma_inv=None, static_scale=None):
 # per-tensor passes
 QUANT_CASES = [(1152, 128, 257, 4, 1, 0), (4608, 256, 130, 3, 1, 0), (3072, 1024, 129, 4, 2, 0),
                (320, 64, 300, 4, 0, 1), (320, 64, 300, 3, 1, 2), (1024, 1, 129, 4, 0, 0),
-               (512, 16, 65, 3, 1, 0), (1024, 32, 100, 4, 1, 0), (2048, 512, 33, 4, 0, 1)]
+               (512, 16, 65, 3, 1, 0), (1024, 32, 100, 4, 1, 0), (2048, 512, 33, 4, 0, 1),
+               (4608, 256, 1000, 3, 1, 0)]
 
 
 @pytest.mark.parametrize("K,n,T,bits,center,gran", QUANT_CASES)

@@ -86,8 +86,14 @@ SMALL_ENVELOPE = [(80, 16, T, 4, c, True) for T, c in ((1, 0), (7, 1), (300, 2))
                  [(12288, n, T, 4, c, True) for n, T, c in ((1024, 7, 1), (256, 33, 2),
                                                            (128, 3, 0))]
 
+# rows of 75-160 slices over enough tokens that the launch plan takes the
+# one-CTA segment variant (three rows a tile) or wider two-CTA tiles
+SMALL_PLAN = [(4608, 256, 1000, 3, 1, True), (4608, 256, 1000, 4, 2, False),
+              (2400, 32, 4000, 4, 1, True), (2816, 256, 700, 8, 0, True)]
 
-@pytest.mark.parametrize("K,n,T,bits,center,use_sigma", SMALL + SMALL_PRE + SMALL_ENVELOPE)
+
+@pytest.mark.parametrize("K,n,T,bits,center,use_sigma",
+                         SMALL + SMALL_PRE + SMALL_ENVELOPE + SMALL_PLAN)
 def test_quantize_small(hq, K, n, T, bits, center, use_sigma):
     g = np.random.default_rng(K * 1000 + T)
     x = g.standard_normal((T, K)).astype(np.float32)
