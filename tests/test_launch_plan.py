@@ -85,6 +85,38 @@ def test_plan_invariants_over_shapes(hq):
             assert N % 256 == 0 and p["gemm_bn"] == 256
 
 
+def _box_ok(RS):
+    # one tensor copy of the whole stage, or equal copies of a multiple of 8 rows
+    return RS <= 256 or any(RS % b == 0 for b in range(8, 257, 8))
+
+
+def _rounds(T, R, slots):
+    tiles = -(-T // R)
+    grid = min(tiles, slots)
+    return -(-tiles // grid)
+
+
+def test_segment_plan_takes_the_fewest_tile_rounds(hq):
+    """The segment quantizer is latency-bound, so its plan takes the tile
+    shape with the fewest rounds of tiles over the resident CTAs (two CTAs of
+    up to 256 consumers an SM, or one of up to 480), the two-CTA variant on a
+    tie; never more rounds than another shape that fits."""
+    for K in range(1056, 8193, 32 * 7):
+        S = K // 32
+        if S % 32 == 0 and S <= 128:
+            continue  # warp-row kernel
+        for T in (1, 100, 1000, 8192, 65536):
+            p = _plan(hq, K, 64, 32, T)
+            R, nt = p["quant_rows"], p["quant_threads"]
+            one_cta = nt > 288
+            got = _rounds(T, R, SMS * (1 if one_cta else 2))
+            two = [_rounds(T, r, 2 * SMS) for r in range(1, 256 // S + 1) if _box_ok(r * S)]
+            one = [_rounds(T, r, SMS) for r in range(1, 480 // S + 1) if _box_ok(r * S)]
+            assert got == min(two + one), (K, T, R, nt)
+            if one_cta:
+                assert not two or min(one) < min(two), (K, T)
+
+
 def test_plan_validation(hq):
     import ctypes
     lib = hq.load_library()
