@@ -826,6 +826,22 @@ def test_group_quantizer_is_the_token_quantizer_per_group():
         assert np.allclose(a["gscale"][:, j], ref["scale"], rtol=1e-15, atol=0)
 
 
+def test_group_weight_quantizer_is_the_token_quantizer_per_group():
+    """The weight side, brute force over every row in {-2..2}^8 with g = 4 and
+    no branch (R = W, sigma = 1): each (row, group) scale and its codes equal
+    the per-token quantizer applied to that group's 4 weights alone, at 4 and
+    at 3 bits."""
+    vals = np.array(list(itertools.product([-2, -1, 0, 1, 2], repeat=8)), dtype=np.float32)
+    W = synth.f32_to_bf16_bits(vals)
+    for bits in (4, 3):
+        w = oracle.gw_prepare_weights(W, 4, bits, 0, None, None, want_tie=False)
+        for j in range(2):
+            ref = oracle.quantize_act(np.ascontiguousarray(W[:, 4 * j:4 * j + 4]), 4, bits,
+                                      gran=0, centering=0, want_tie=False)
+            assert np.array_equal(w["codes"][:, 4 * j:4 * j + 4], ref["codes"])
+            assert np.allclose(w["gscale"][:, j], ref["scale"], rtol=1e-15, atol=0)
+
+
 def test_low_rank_factors_are_the_best_rank_r_approximation():
     """L2 L1 from the decomposition equals the truncated SVD of W diag(sigma)
     (Eckart-Young: the residual's Frobenius norm is the root of the sum of
