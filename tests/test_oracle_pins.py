@@ -260,7 +260,7 @@ def _exact_codes_int(x_int, n, q, centering):
 
 
 @pytest.mark.parametrize("n", [4, 8])
-@pytest.mark.parametrize("bits,centering", [(4, 1), (3, 1), (4, 0), (4, 2), (3, 2)])
+@pytest.mark.parametrize("bits,centering", [(4, 1), (3, 1), (4, 0), (4, 2), (3, 2), (2, 0), (2, 1)])
 def test_bruteforce_k8(n, bits, centering):
     vals = np.arange(-2, 3)
     x_int = np.array(list(itertools.product(vals, repeat=8)), dtype=np.int64)  # 5^8 rows
@@ -812,18 +812,21 @@ def test_group_wise_identity_unquantized(K, g, N, T, rank):
     assert np.linalg.norm(y - exact) <= 1e-10 * np.linalg.norm(exact)
 
 
-def test_group_quantizer_is_the_token_quantizer_per_group():
+@pytest.mark.parametrize("bits", [4, 3, 2])
+def test_group_quantizer_is_the_token_quantizer_per_group(bits):
     """Brute force over every x in {-2..2}^8 with g = 4: each group's codes
     and scale equal the (independently pinned) per-token quantizer applied to
-    that group's 4 values alone (n = K = 4, no centring)."""
+    that group's 4 values alone (n = K = 4, no centring), at every code width
+    the group-wise form takes."""
     vals = np.array(list(itertools.product([-2, -1, 0, 1, 2], repeat=8)), dtype=np.float32)
     X = synth.f32_to_bf16_bits(vals)
-    a = oracle.gw_quantize_act(X, 4, 4, 0, None, want_tie=False)
+    a = oracle.gw_quantize_act(X, 4, bits, 0, None, want_tie=False)
     for j in range(2):
-        ref = oracle.quantize_act(np.ascontiguousarray(X[:, 4 * j:4 * j + 4]), 4, 4, gran=0,
+        ref = oracle.quantize_act(np.ascontiguousarray(X[:, 4 * j:4 * j + 4]), 4, bits, gran=0,
                                   centering=0, want_tie=False)
         assert np.array_equal(a["codes"][:, 4 * j:4 * j + 4], ref["codes"])
         assert np.allclose(a["gscale"][:, j], ref["scale"], rtol=1e-15, atol=0)
+    assert np.abs(a["codes"]).max() == 2 ** (bits - 1) - 1
 
 
 def test_group_weight_quantizer_is_the_token_quantizer_per_group():
