@@ -151,6 +151,7 @@ CASES = [
     (200, 576, 256, 0, 3, 4, True),
     (130, 1024, 528, 32, 3, 4, False),
     (257, 2048, 784, 32, 4, 3, True),
+    (96, 512, 80, 32, 2, 2, True),  # 2-bit codes on both sides
     (64, 64 * 65, 32, 32, 4, 4, True),
     (130, 16384, 48, 32, 4, 4, True),  # the largest K (sigma^-1 takes 64 KB of shared memory)
 ]
